@@ -1,0 +1,538 @@
+"""Benchmark of the element-routed MoE layer (forward + input VJP) on B200.
+
+One step = one pass of the MoE layer over one synthetic batch:
+    route -> dispatch -> expert MLP fwd -> combine            (forward)
+    weighted dispatch of dY -> expert MLP VJP -> combine      (input VJP)
+with the interaction-block slice workload also running the edge aggregation
+and the per-element-type FP16 packing (quant -> dequant) in front.
+
+Metric: routed atom-expert tokens/s (tokens = N*K routed rows) per layer pass.
+Default workload: MatRIS-MoE(S)-shaped layer (N=8192, T=89 Zipf(1.1), E=72,
+K=4, d=h=2560), model table of the paper review 'Breaking the Training
+Barrier of Billion-Parameter Universal Machine Learning Interatomic
+Potentials', section 3.1 Table II.
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload S|M|L|slice|tiny]
+                  [--mode simt|3xtf32] [--impl janus|reference] [--no-cpu-baseline]
+Multi-GPU (weak scaling, one independent layer per rank, no collective on the
+data path): python -m torch.distributed.run --nproc-per-node N bench.py --gpus N
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from element_routed_moe_b200 import synth  # noqa: E402
+
+METRIC = "routed atom-expert tokens/sec per MoE layer (fwd+VJP)"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 2 ** 20
+SM_COUNT = 148
+FP32_LANES_PER_SM = 128
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="S", choices=list(synth.CONFIGS))
+    ap.add_argument("--mode", default="simt", choices=["simt", "3xtf32"])
+    ap.add_argument("--impl", default="janus", choices=["janus", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing
+# --------------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64,
+                     device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def describe(cfg) -> dict:
+    w = {"tiny": "tiny layer", "S": "MatRIS-MoE(S)-shaped layer", "M": "MatRIS-MoE(M)-shaped layer",
+         "L": "MatRIS-MoE(L)-shaped layer", "slice": "interaction-block slice at M shape"}[cfg.name]
+    return {
+        "workload": f"{w}: N={cfg.n_atoms} atoms, T={cfg.n_types} element types "
+                    f"({'Zipf(1.1)' if cfg.type_dist == 'zipf' else 'uniform'}), E={cfg.n_experts}, "
+                    f"K={cfg.top_k}, d=h={cfg.d}, FP32, fwd+input-VJP"
+                    + (", edge aggregation + FP16 per-type packing" if cfg.name == "slice" else ""),
+        "n_atoms": cfg.n_atoms, "n_types": cfg.n_types, "n_experts": cfg.n_experts,
+        "top_k": cfg.top_k, "d": cfg.d, "h": cfg.h, "routed_tokens": cfg.n_rows,
+    }
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self, wall0: float, wall1: float) -> dict | None:
+        """Summary of the samples taken between wall0 and wall1 (time.time());
+        all samples if fewer than three fall inside the window."""
+        import datetime
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9 or not f[1].replace(".", "").isdigit():
+                continue
+            try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                ts = None
+            rows.append((ts, f))
+        os.unlink(self.path)
+        inside = [f for ts, f in rows if ts is not None and wall0 <= ts <= wall1]
+        used = inside if len(inside) >= 3 else [f for _, f in rows]
+        if not used:
+            return None
+        sm = [float(r[1]) for r in used]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for r in used for j in range(4) if r[5 + j].lower() == "active"})
+        pw = [float(r[3]) for r in used if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(used[0][2]),
+                "samples": len(used), "samples_in_timed_region": len(inside),
+                "power_w_max": max(pw) if pw else None, "reasons": reasons}
+
+
+def measured_peaks() -> tuple[dict, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0}, "fallback"
+
+
+# --------------------------------------------------------------------------
+# the layer pass through the C ABI (device-resident inputs)
+# --------------------------------------------------------------------------
+class Layer:
+    """Preallocated buffers and the ordered ABI calls of one layer pass."""
+
+    OPS_FWD = ("route", "dispatch", "ffn_fwd", "combine")
+    OPS_VJP = ("dispatch_w", "ffn_vjp", "combine_vjp")
+
+    def __init__(self, cfg, mode: int, seed: int, dev):
+        from element_routed_moe_b200 import janus as J
+        self.J = J
+        self.cfg = cfg
+        self.mode = mode
+        N, T, E, K, d, h = cfg.n_atoms, cfg.n_types, cfg.n_experts, cfg.top_k, cfg.d, cfg.h
+        R = N * K
+        self.slice = cfg.name == "slice"
+        inp = synth.layer_inputs(cfg, seed=seed, device=dev, with_edges=self.slice)
+        self.inp = inp
+        self.types = torch.as_tensor(inp["types"], device=dev)
+        self.gate = torch.as_tensor(inp["gate"], device=dev)
+        self.w1, self.w2 = inp["w1"], inp["w2"]
+        self.x, self.g = inp["x"], inp["g"]
+        if self.slice:
+            self.msg = inp["msg"]
+            self.row_ptr = torch.as_tensor(inp["row_ptr"], device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.route_out = dict(topk_expert=torch.empty((N, K), **i32),
+                              topk_weight=torch.empty((N, K), **f32),
+                              counts=torch.empty((E,), **i32), offsets=torch.empty((E + 1,), **i32),
+                              perm=torch.empty((R,), **i32), slot_of=torch.empty((R,), **i32))
+        self.route_ws = torch.empty(J.janus_route_workspace_size(N, T, E, K), dtype=torch.uint8, device=dev)
+        self.xd = torch.empty((R, d), **f32)
+        self.yd = torch.empty((R, d), **f32)
+        self.act = torch.empty((R, h), **f32)
+        self.y = torch.empty((N, d), **f32)
+        self.gd = torch.empty((R, d), **f32)
+        self.dxd = torch.empty((R, d), **f32)
+        self.dx = torch.empty((N, d), **f32)
+        nb = max(J.janus_expert_ffn_workspace_size(R, d, h, E, False, True, mode),
+                 J.janus_expert_ffn_workspace_size(R, d, h, E, True, True, mode))
+        self.ffn_ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        if self.slice:
+            self.xagg = torch.empty((N, d), **f32)
+            self.payload = torch.empty((R, d), dtype=torch.float16, device=dev)
+            self.scale = torch.empty((T,), **f32)
+            self.quant_ws = torch.empty(J.janus_quant_by_type_workspace_size(T), dtype=torch.uint8,
+                                        device=dev)
+        if self.slice:
+            self.ops = ("edge_aggregate", "route", "quant", "dequant", "ffn_fwd", "combine") + self.OPS_VJP
+        else:
+            self.ops = self.OPS_FWD + self.OPS_VJP
+        # our kernels per step (see each call's launches in csrc/)
+        per = {"edge_aggregate": 1, "quant": 2, "dequant": 1, "route": 4, "dispatch": 1,
+               "ffn_fwd": 2, "combine": 1, "dispatch_w": 1, "ffn_vjp": 2, "combine_vjp": 1}
+        self.launches_per_step = sum(per[o] for o in self.ops)
+
+    def step(self, x=None, g=None, types=None, events=None):
+        """One layer pass.  events: dict op -> (start, end) CUDA events, or None."""
+        J = self.J
+        cfg = self.cfg
+        T, K = cfg.n_types, cfg.top_k
+        x = self.x if x is None else x
+        g = self.g if g is None else g
+        types = self.types if types is None else types
+        r = self.route_out
+
+        def mark(op, i):
+            if events is not None:
+                events[op][i].record()
+
+        if self.slice:
+            mark("edge_aggregate", 0)
+            J.janus_edge_aggregate(self.msg, self.row_ptr, out=self.xagg)
+            mark("edge_aggregate", 1)
+            x = self.xagg
+        mark("route", 0)
+        J.janus_route(types, self.gate, K, out=r, workspace=self.route_ws)
+        mark("route", 1)
+        if self.slice:
+            mark("quant", 0)
+            J.janus_quant_by_type(x, types, T, r["slot_of"], K, payload=self.payload,
+                                  scale=self.scale, workspace=self.quant_ws)
+            mark("quant", 1)
+            mark("dequant", 0)
+            J.janus_dequant_by_type(self.payload, types, T, r["perm"], K, self.scale, out=self.xd)
+            mark("dequant", 1)
+        else:
+            mark("dispatch", 0)
+            J.janus_dispatch(x, r["slot_of"], K, out=self.xd)
+            mark("dispatch", 1)
+        mark("ffn_fwd", 0)
+        J.janus_expert_ffn_fwd(self.xd, r["offsets"], self.w1, self.w2, mode=self.mode, out=self.yd,
+                               act=self.act, workspace=self.ffn_ws)
+        mark("ffn_fwd", 1)
+        mark("combine", 0)
+        J.janus_combine(self.yd, r["slot_of"], K, r["topk_weight"], out=self.y)
+        mark("combine", 1)
+        mark("dispatch_w", 0)
+        J.janus_dispatch(g, r["slot_of"], K, r["topk_weight"], out=self.gd)
+        mark("dispatch_w", 1)
+        mark("ffn_vjp", 0)
+        J.janus_expert_ffn_vjp(self.xd, self.gd, r["offsets"], self.w1, self.w2, act=self.act,
+                               mode=self.mode, out=self.dxd, workspace=self.ffn_ws)
+        mark("ffn_vjp", 1)
+        mark("combine_vjp", 0)
+        J.janus_combine(self.dxd, r["slot_of"], K, out=self.dx)
+        mark("combine_vjp", 1)
+        return self.y, self.dx
+
+    # algorithmic bytes (memory-bound ops) and FLOPs (expert MLP) per call
+    def work(self):
+        c = self.cfg
+        N, R, d, h = c.n_atoms, c.n_rows, c.d, c.h
+        w = {
+            "dispatch": ("bytes", 4 * d * (N + R) + 4 * R),
+            "dispatch_w": ("bytes", 4 * d * (N + R) + 8 * R),
+            "combine": ("bytes", 4 * d * (R + N) + 8 * R),
+            "combine_vjp": ("bytes", 4 * d * (R + N) + 4 * R),
+            "ffn_fwd": ("flops", 4 * R * d * h),
+            "ffn_vjp": ("flops", 4 * R * d * h),
+            "route": ("bytes", 4 * N + 8 * R * 2 + 8 * R),
+        }
+        if self.slice:
+            Ed = int(self.inp["row_ptr"][-1])
+            w["edge_aggregate"] = ("bytes", 4 * Ed * d + 4 * N * d + 8 * (N + 1))
+            w["quant"] = ("bytes", 4 * N * d * 2 + 2 * R * d + 4 * R)
+            w["dequant"] = ("bytes", 2 * R * d + 4 * R * d + 8 * R)
+        return w
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (the reported CPU baseline; never the product path)
+# --------------------------------------------------------------------------
+def oracle_pass(cfg, host_inp, n: int) -> float:
+    """Wall time of the oracle's layer pass (route, dispatch, FFN fwd,
+    combine, weighted dispatch, FFN VJP, combine) on the first n atoms of the
+    workload, with the full expert weights."""
+    import oracle
+    types = host_inp["types"][:n]
+    x, g = host_inp["x"][:n], host_inp["g"][:n]
+    w1, w2 = host_inp["w1"], host_inp["w2"]
+    K = cfg.top_k
+    t0 = time.perf_counter()
+    r = oracle.route(types, host_inp["gate"], K)
+    xd = oracle.dispatch(x, r["perm"], K)
+    yd = oracle.expert_ffn_fwd(xd, r["offsets"], w1, w2)
+    oracle.combine(yd, r["slot_of"], K, r["topk_weight"])
+    gd = oracle.dispatch(g, r["perm"], K, r["topk_weight"])
+    dxd = oracle.expert_ffn_vjp(xd, gd, r["offsets"], w1, w2)
+    oracle.combine(dxd, r["slot_of"], K)
+    return time.perf_counter() - t0
+
+
+def oracle_calibrate(cfg, host_inp, target_s: float) -> int:
+    """Number of atoms whose oracle pass takes about target_s seconds."""
+    n = 4
+    dt = oracle_pass(cfg, host_inp, n)
+    while dt < 0.1 * target_s and n < cfg.n_atoms:
+        n = min(cfg.n_atoms, n * 4)
+        dt = oracle_pass(cfg, host_inp, n)
+    return int(min(cfg.n_atoms, max(1, n * target_s / max(dt, 1e-6))))
+
+
+def host_inputs(cfg, layer):
+    return dict(types=np.asarray(layer.inp["types"]), gate=np.asarray(layer.inp["gate"]),
+                x=layer.x.cpu().numpy(), g=layer.g.cpu().numpy(),
+                w1=layer.w1.cpu().numpy(), w2=layer.w2.cpu().numpy())
+
+
+def cpu_descr():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# --------------------------------------------------------------------------
+# reference arm: the oracle on the host cores
+# --------------------------------------------------------------------------
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import oracle
+    cfg = synth.CONFIGS[args.workload]
+    inp = synth.layer_inputs(cfg, seed=args.seed, device="cpu", with_edges=False)
+    host = dict(types=inp["types"], gate=inp["gate"], x=inp["x"].numpy(), g=inp["g"].numpy(),
+                w1=inp["w1"].numpy(), w2=inp["w2"].numpy())
+    per_step = max(2.0, min(15.0, 150.0 / max(1, args.steps + args.warmup)))
+    n_s = oracle_calibrate(cfg, host, per_step)
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt = oracle_pass(cfg, host, n_s)
+        if i >= args.warmup:
+            times.append(dt)
+    t = float(np.mean(times))
+    value = n_s * cfg.top_k / t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": describe(cfg),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"first {n_s} of {cfg.n_atoms} atoms ({n_s * cfg.top_k} routed tokens) "
+                                   f"per step, full expert weights; host {cpu_descr()}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------
+# janus arm
+# --------------------------------------------------------------------------
+def run_janus(args, world, rank, local):
+    from element_routed_moe_b200 import janus as J
+    J.lib()   # fails loudly if the CUDA library is missing
+    dev = torch.device("cuda", local)
+    cfg = synth.CONFIGS[args.workload]
+    mode = J.JANUS_FFN_3XTF32 if args.mode == "3xtf32" else J.JANUS_FFN_FP32_SIMT
+    layer = Layer(cfg, mode, seed=args.seed + 1000 * rank, dev=dev)
+    work = layer.work()
+    peaks, peak_src = measured_peaks()
+
+    for _ in range(args.warmup):
+        layer.step()
+    torch.cuda.synchronize()
+    J.janus_check(layer.route_ws)
+
+    ev = [{op: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for op in layer.ops} for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local))
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    t_start.record()
+    for k in range(args.steps):
+        layer.step(events=ev[k])
+    t_end.record()
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    clocks = sampler.stop(wall0, wall1)
+    barrier(world)
+    elapsed = t_start.elapsed_time(t_end) / 1e3
+    t_max = max_over_ranks(elapsed, world)
+    tokens = cfg.n_rows * args.steps * world
+    value = tokens / t_max
+
+    op_ms = {op: float(np.mean([e[op][0].elapsed_time(e[op][1]) for e in ev])) for op in layer.ops}
+    kernels = {}
+    for op, (kind, amount) in work.items():
+        if op not in op_ms or kind != "bytes" or op == "route":
+            continue
+        gbs = amount / (op_ms[op] * 1e-3) / 1e9
+        kernels[op] = {"ms": op_ms[op], "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                       "algorithmic_bytes": amount}
+    kernels["route"] = {"ms": op_ms["route"]}
+
+    # roofline of the dominant kernel: the grouped expert-MLP GEMM (4 launches
+    # per step: two forward, two VJP, each 2*R*d*h FLOPs)
+    ffn_ms = op_ms["ffn_fwd"] + op_ms["ffn_vjp"]
+    ffn_flops = work["ffn_fwd"][1] + work["ffn_vjp"][1]
+    achieved = ffn_flops / (ffn_ms * 1e-3) / 1e12
+    if mode == J.JANUS_FFN_FP32_SIMT:
+        peak = SM_COUNT * FP32_LANES_PER_SM * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+        roof = {"bound": "alu", "peak_source": "148 SMs x 128 FP32 lanes x 2 FLOP x max SM clock"}
+    else:
+        peak = peaks["bf16_tflops_sustained"] * (1.125 / 2.25) / 3.0
+        roof = {"bound": "tensor", "peak_source": f"{peak_src} sustained bf16 x (TF32/BF16 nominal 1.125/2.25) / 3 products"}
+    roof.update({"kernel": "grouped expert-MLP GEMM", "achieved": achieved, "peak": peak,
+                 "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                 "algorithmic_flops_per_launch": ffn_flops / 4, "launches_per_step": 4})
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_max / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {**describe(cfg), "ffn_mode": args.mode, "parallelism": f"replicas x{world}",
+                   "l2": "no flush: per-step working set "
+                         f"{(layer.w1.numel() + layer.w2.numel()) * 4 / 2**30:.1f} GiB weights + "
+                         f"{cfg.n_rows * cfg.d * 4 * 4 / 2**30:.2f} GiB activations >> 126 MB L2"},
+        "roofline": roof,
+        "kernels": kernels,
+        "breakdown_ms": op_ms,
+        "gpu_launches": layer.launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+
+    if not args.no_e2e and not layer.slice:
+        line["e2e"] = run_e2e(layer, args)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = host_inputs(cfg, layer)
+        n_s = oracle_calibrate(cfg, host, 15.0)
+        dt = oracle_pass(cfg, host, n_s)
+        import oracle
+        line["cpu_baseline"] = {
+            "value": n_s * cfg.top_k / dt, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"first {n_s} of {cfg.n_atoms} atoms ({n_s * cfg.top_k} routed tokens), "
+                      f"full expert weights, {dt:.1f} s; host {cpu_descr()}"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(layer, args):
+    """Same metric through the public API with the step's inputs in pinned
+    host memory: H2D of (x, dY, types) and D2H of (y, dX) inside the timing."""
+    dev = layer.x.device
+    x_h = layer.x.cpu().pin_memory()
+    g_h = layer.g.cpu().pin_memory()
+    t_h = layer.types.cpu().pin_memory()
+    y_h = torch.empty(layer.y.shape, dtype=torch.float32).pin_memory()
+    dx_h = torch.empty(layer.dx.shape, dtype=torch.float32).pin_memory()
+    x_d, g_d, t_d = torch.empty_like(layer.x), torch.empty_like(layer.g), torch.empty_like(layer.types)
+
+    def step():
+        x_d.copy_(x_h, non_blocking=True)
+        g_d.copy_(g_h, non_blocking=True)
+        t_d.copy_(t_h, non_blocking=True)
+        y, dx = layer.step(x_d, g_d, t_d)
+        y_h.copy_(y, non_blocking=True)
+        dx_h.copy_(dx, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    t = a.elapsed_time(b) / 1e3
+    h2d = x_h.numel() * 4 + g_h.numel() * 4 + t_h.numel() * 4
+    d2h = y_h.numel() * 4 + dx_h.numel() * 4
+    return {"value": layer.cfg.n_rows * args.steps / t, "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_janus(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,139 @@
+// janus_expert_ffn_fwd / janus_expert_ffn_vjp: the grouped expert MLP of the
+// element-routed MoE layer and its input VJP.
+//
+// Sources: paper review "Breaking the Training Barrier of Billion-Parameter
+// Universal Machine Learning Interatomic Potentials" section 3.1 Table II
+// (MLP hidden size = feature size) and section 3.3 (forces and stress by
+// autodiff of the energy, so training needs the input gradient).  The expert
+// is read as bias-free Linear(d,h) -> SiLU -> Linear(h,d).
+//
+// Forward (two grouped GEMMs, SiLU fused into the first one's epilogue):
+//   G1: a = xd W1[e]          -> act (optional), H = silu(a) (workspace)
+//   G2: yd = H W2[e]
+// Input VJP (SiLU' fused into the first GEMM's epilogue):
+//   G0: a = xd W1[e]          (only when the forward's act is not supplied)
+//   G3: dA = (gd W2[e]^T) * silu'(a)   (workspace)
+//   G4: dxd = dA W1[e]^T
+#include "common.cuh"
+#include "ffn_simt.cuh"
+#include "ffn_tc.cuh"
+
+namespace janus {
+namespace {
+
+struct FfnLayout {
+  size_t off_h, total;
+};
+
+FfnLayout ffn_layout(int64_t R, int32_t h, bool vjp, bool have_act) {
+  FfnLayout L;
+  const size_t rh = align_up(sizeof(float) * (size_t)R * (size_t)h, 256);
+  L.off_h = sizeof(WsHeader);
+  size_t n_bufs = vjp ? (have_act ? 1 : 2) : 1;
+  L.total = L.off_h + n_bufs * rh + tc::workspace_extra();
+  return L;
+}
+
+janus_status check_ffn(const float* xd, const int32_t* offsets, int32_t E, int64_t R, int32_t d,
+                       int32_t h, const float* w1, const float* w2, const float* out,
+                       janus_ffn_mode mode) {
+  JANUS_CHECK_ARG(E >= 1 && E <= kMaxExperts);
+  JANUS_CHECK_ARG(R >= 0 && R < (int64_t)INT32_MAX);
+  JANUS_CHECK_ARG(d >= 1 && d <= kMaxDim && h >= 1 && h <= kMaxDim);
+  JANUS_CHECK_ARG(mode == JANUS_FFN_FP32_SIMT || mode == JANUS_FFN_3XTF32);
+  JANUS_CHECK_ALIGN(d % 4 == 0 && h % 4 == 0);
+  JANUS_CHECK_ARG(offsets && w1 && w2);
+  JANUS_CHECK_ARG(R == 0 || (xd && out));
+  JANUS_CHECK_ALIGN(aligned(w1, 16) && aligned(w2, 16));
+  JANUS_CHECK_ALIGN(R == 0 || (aligned(xd, 16) && aligned(out, 16)));
+  return JANUS_OK;
+}
+
+template <bool kNT, int kEpi>
+void launch_simt(const simt::Args& a, cudaStream_t s) {
+  simt::grouped_gemm_kernel<kNT, kEpi><<<num_sms() * 2, simt::kThreads, 0, s>>>(a);
+}
+
+simt::Args make_args(const float* A, const float* B, int64_t bstride, float* C, float* C2,
+                     const float* aux, const int32_t* offsets, int E, int Kd, int N) {
+  simt::Args a;
+  a.A = A; a.B = B; a.b_expert_stride = bstride; a.C = C; a.C2 = C2; a.aux = aux;
+  a.offsets = offsets; a.E = E; a.Kd = Kd; a.N = N;
+  return a;
+}
+
+}  // namespace
+}  // namespace janus
+
+using namespace janus;
+
+extern "C" janus_status janus_expert_ffn_workspace_size(int64_t n_rows, int32_t d, int32_t h,
+                                                        int32_t n_experts, int32_t vjp,
+                                                        int32_t have_act, janus_ffn_mode mode,
+                                                        size_t* bytes) {
+  JANUS_CHECK_ARG(bytes && n_rows >= 0 && d >= 1 && h >= 1 && n_experts >= 1);
+  JANUS_CHECK_ARG(mode == JANUS_FFN_FP32_SIMT || mode == JANUS_FFN_3XTF32);
+  *bytes = ffn_layout(n_rows, h, vjp != 0, have_act != 0).total;
+  return JANUS_OK;
+}
+
+extern "C" janus_status janus_expert_ffn_fwd(const float* xd, const int32_t* offsets,
+                                             int32_t n_experts, int64_t n_rows, int32_t d,
+                                             int32_t h, const float* w1, const float* w2,
+                                             float* yd, float* act, janus_ffn_mode mode,
+                                             void* workspace, size_t workspace_bytes,
+                                             janus_stream_t stream_) {
+  cudaStream_t stream = (cudaStream_t)stream_;
+  janus_status st = check_ffn(xd, offsets, n_experts, n_rows, d, h, w1, w2, yd, mode);
+  if (st != JANUS_OK) return st;
+  const FfnLayout L = ffn_layout(n_rows, h, false, act != nullptr);
+  JANUS_CHECK_ARG(workspace && workspace_bytes >= L.total);
+  JANUS_CHECK_ALIGN(aligned(workspace, 256) && (act == nullptr || aligned(act, 16)));
+  if (n_rows == 0) return JANUS_OK;
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  float* H = (float*)((char*)workspace + L.off_h);
+  const int64_t sw = (int64_t)d * h;
+  if (mode == JANUS_FFN_3XTF32) {
+    st = tc::expert_ffn_fwd(xd, offsets, n_experts, n_rows, d, h, w1, w2, yd, act, H,
+                            (char*)workspace + L.total - tc::workspace_extra(), stream);
+    if (st != JANUS_OK) return st;
+    return launch_status();
+  }
+  launch_simt<false, simt::kEpiSilu>(make_args(xd, w1, sw, H, act, nullptr, offsets, n_experts, d, h), stream);
+  launch_simt<false, simt::kEpiStore>(make_args(H, w2, sw, yd, nullptr, nullptr, offsets, n_experts, h, d), stream);
+  return launch_status();
+}
+
+extern "C" janus_status janus_expert_ffn_vjp(const float* xd, const float* gd, const float* act,
+                                             const int32_t* offsets, int32_t n_experts,
+                                             int64_t n_rows, int32_t d, int32_t h,
+                                             const float* w1, const float* w2, float* dxd,
+                                             janus_ffn_mode mode, void* workspace,
+                                             size_t workspace_bytes, janus_stream_t stream_) {
+  cudaStream_t stream = (cudaStream_t)stream_;
+  janus_status st = check_ffn(xd, offsets, n_experts, n_rows, d, h, w1, w2, dxd, mode);
+  if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(n_rows == 0 || gd);
+  JANUS_CHECK_ALIGN(n_rows == 0 || aligned(gd, 16));
+  JANUS_CHECK_ALIGN(act == nullptr || aligned(act, 16));
+  const FfnLayout L = ffn_layout(n_rows, h, true, act != nullptr);
+  JANUS_CHECK_ARG(workspace && workspace_bytes >= L.total);
+  JANUS_CHECK_ALIGN(aligned(workspace, 256));
+  if (n_rows == 0) return JANUS_OK;
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  const size_t rh = align_up(sizeof(float) * (size_t)n_rows * (size_t)h, 256);
+  float* dA = (float*)((char*)workspace + L.off_h);
+  float* A = act ? const_cast<float*>(act) : (float*)((char*)workspace + L.off_h + rh);
+  const int64_t sw = (int64_t)d * h;
+  if (mode == JANUS_FFN_3XTF32) {
+    st = tc::expert_ffn_vjp(xd, gd, act, A, offsets, n_experts, n_rows, d, h, w1, w2, dxd, dA,
+                            (char*)workspace + L.total - tc::workspace_extra(), stream);
+    if (st != JANUS_OK) return st;
+    return launch_status();
+  }
+  if (!act)
+    launch_simt<false, simt::kEpiStore>(make_args(xd, w1, sw, A, nullptr, nullptr, offsets, n_experts, d, h), stream);
+  launch_simt<true, simt::kEpiDSilu>(make_args(gd, w2, sw, dA, nullptr, A, offsets, n_experts, d, h), stream);
+  launch_simt<true, simt::kEpiStore>(make_args(dA, w1, sw, dxd, nullptr, nullptr, offsets, n_experts, h, d), stream);
+  return launch_status();
+}

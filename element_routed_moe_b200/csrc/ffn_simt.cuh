@@ -1,0 +1,214 @@
+// Grouped FP32 GEMM on the CUDA cores (FFMA), used by the expert MLP in
+// JANUS_FFN_FP32_SIMT mode.  Internal header, included by expert_ffn.cu.
+//
+//   C[p, :] = epilogue( A[p, :] * B_e )   for rows p in [offsets[e], offsets[e+1])
+//
+// A is row-major [R, Kd]; B_e is expert e's weight, either stored [Kd][N]
+// (kNT = false, "x W") or [N][Kd] (kNT = true, "x W^T").
+//
+// Tiling: 128x128 output tile, k-step 16, 256 threads, 8x8 outputs per
+// thread as two 4x4 quadrants in each direction (conflict-free 128-bit shared
+// loads), global->register->shared double buffering with one barrier per
+// k-step.  A persistent grid walks a device-side tile list built from
+// `offsets` (expert-major, then m-tile, then n-tile), so concurrently running
+// CTAs share the same expert's weights and A rows in L2 and the host never
+// reads the routing result.
+#pragma once
+
+#include "common.cuh"
+
+namespace janus {
+namespace simt {
+
+constexpr int BM = 128, BN = 128, BK = 16, kThreads = 256;
+
+enum Epilogue : int {
+  kEpiStore = 0,   // C = acc
+  kEpiSilu = 1,    // C2 = acc (if C2), C = silu(acc)
+  kEpiDSilu = 2    // C = acc * silu'(aux)
+};
+
+struct Args {
+  const float* A;
+  const float* B;
+  int64_t b_expert_stride;   // elements between experts' weights
+  float* C;
+  float* C2;                 // optional second output (pre-activation)
+  const float* aux;          // pre-activation for kEpiDSilu, [R, N]
+  const int32_t* offsets;
+  int E;
+  int Kd;                    // reduction length
+  int N;                     // output columns
+};
+
+__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + expf(-a)); }
+__device__ __forceinline__ float dsilu_f(float a) {
+  const float s = 1.0f / (1.0f + expf(-a));
+  return s * (1.0f + a * (1.0f - s));
+}
+
+// Expert-major tile list: tile_start[e] = sum_{e'<e} ceil(count_e'/BM).
+struct TileMap {
+  int off[kMaxExperts + 1];
+  int start[kMaxExperts + 1];
+};
+
+__device__ __forceinline__ void build_tile_map(TileMap& tm, const int32_t* offsets, int E) {
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) tm.off[e] = offsets[e];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int e = 0; e < E; ++e) {
+      tm.start[e] = acc;
+      acc += (tm.off[e + 1] - tm.off[e] + BM - 1) / BM;
+    }
+    tm.start[E] = acc;
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ int find_expert(const TileMap& tm, int E, int mt) {
+  int lo = 0, hi = E;          // invariant: start[lo] <= mt < start[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (tm.start[mid] <= mt) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+template <bool kNT, int kEpi>
+__global__ void __launch_bounds__(kThreads, 2) grouped_gemm_kernel(Args args) {
+  __shared__ __align__(16) float As[2][BK][BM];
+  __shared__ __align__(16) float Bs[2][BK][BN];
+  __shared__ TileMap tm;
+  build_tile_map(tm, args.offsets, args.E);
+
+  const int tid = threadIdx.x;
+  const int tx = tid % 16, ty = tid / 16;
+  const int Kd = args.Kd, N = args.N;
+  const int n_tiles_n = (N + BN - 1) / BN;
+  const int total = tm.start[args.E] * n_tiles_n;
+  const int nk = (Kd + BK - 1) / BK;
+
+  for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    const int mt = tile / n_tiles_n, nt = tile % n_tiles_n;
+    const int e = find_expert(tm, args.E, mt);
+    const int m0 = tm.off[e] + (mt - tm.start[e]) * BM;
+    const int m_end = tm.off[e + 1];
+    const int n0 = nt * BN;
+    const float* A = args.A;
+    const float* B = args.B + (int64_t)e * args.b_expert_stride;
+
+    float4 ra[2], rb[2];
+    // A (and B when kNT): element (row r, k-quad q) at idx = tid + j*256,
+    // r = idx % 128, q = idx / 128; consecutive lanes -> consecutive rows, so
+    // the transposed shared stores are conflict-free.
+    auto load_tile = [&](int kt) {
+      const int k0 = kt * BK;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int idx = tid + j * kThreads;
+        const int r = idx % BM, q = idx / BM;
+        const int kk = k0 + q * 4;
+        const bool ok = (m0 + r < m_end) && (kk < Kd);
+        ra[j] = ok ? __ldg(reinterpret_cast<const float4*>(A + (int64_t)(m0 + r) * Kd + kk))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int idx = tid + j * kThreads;
+        if (kNT) {
+          const int n = idx % BN, q = idx / BN;
+          const int kk = k0 + q * 4;
+          const bool ok = (n0 + n < N) && (kk < Kd);
+          rb[j] = ok ? __ldg(reinterpret_cast<const float4*>(B + (int64_t)(n0 + n) * Kd + kk))
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+          const int kr = idx / (BN / 4), nq = idx % (BN / 4);
+          const bool ok = (k0 + kr < Kd) && (n0 + nq * 4 < N);
+          rb[j] = ok ? __ldg(reinterpret_cast<const float4*>(B + (int64_t)(k0 + kr) * N + n0 + nq * 4))
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+    };
+    auto store_tile = [&](int buf) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int idx = tid + j * kThreads;
+        const int r = idx % BM, q = idx / BM;
+        As[buf][q * 4 + 0][r] = ra[j].x;
+        As[buf][q * 4 + 1][r] = ra[j].y;
+        As[buf][q * 4 + 2][r] = ra[j].z;
+        As[buf][q * 4 + 3][r] = ra[j].w;
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int idx = tid + j * kThreads;
+        if (kNT) {
+          const int n = idx % BN, q = idx / BN;
+          Bs[buf][q * 4 + 0][n] = rb[j].x;
+          Bs[buf][q * 4 + 1][n] = rb[j].y;
+          Bs[buf][q * 4 + 2][n] = rb[j].z;
+          Bs[buf][q * 4 + 3][n] = rb[j].w;
+        } else {
+          const int kr = idx / (BN / 4), nq = idx % (BN / 4);
+          *reinterpret_cast<float4*>(&Bs[buf][kr][nq * 4]) = rb[j];
+        }
+      }
+    };
+
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+    load_tile(0);
+    store_tile(0);
+    __syncthreads();
+    for (int kt = 0; kt < nk; ++kt) {
+      const int cur = kt & 1;
+      if (kt + 1 < nk) load_tile(kt + 1);
+#pragma unroll
+      for (int k = 0; k < BK; ++k) {
+        const float4 a0 = *reinterpret_cast<const float4*>(&As[cur][k][ty * 4]);
+        const float4 a1 = *reinterpret_cast<const float4*>(&As[cur][k][64 + ty * 4]);
+        const float4 b0 = *reinterpret_cast<const float4*>(&Bs[cur][k][tx * 4]);
+        const float4 b1 = *reinterpret_cast<const float4*>(&Bs[cur][k][64 + tx * 4]);
+        const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+      }
+      if (kt + 1 < nk) store_tile(cur ^ 1);
+      __syncthreads();
+    }
+
+    // epilogue
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+      if (r >= m_end) continue;
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        const int c = n0 + g * 64 + tx * 4;
+        if (c >= N) continue;
+        float4 v = make_float4(acc[i][g * 4 + 0], acc[i][g * 4 + 1], acc[i][g * 4 + 2], acc[i][g * 4 + 3]);
+        const int64_t o = (int64_t)r * N + c;
+        if (kEpi == kEpiSilu) {
+          if (args.C2) *reinterpret_cast<float4*>(args.C2 + o) = v;
+          v = make_float4(silu_f(v.x), silu_f(v.y), silu_f(v.z), silu_f(v.w));
+        } else if (kEpi == kEpiDSilu) {
+          const float4 a = __ldg(reinterpret_cast<const float4*>(args.aux + o));
+          v = make_float4(v.x * dsilu_f(a.x), v.y * dsilu_f(a.y), v.z * dsilu_f(a.z), v.w * dsilu_f(a.w));
+        }
+        *reinterpret_cast<float4*>(args.C + o) = v;
+      }
+    }
+  }
+}
+
+}  // namespace simt
+}  // namespace janus

@@ -1,0 +1,23 @@
+// Grouped expert MLP on the tcgen05 tensor cores with the 3xTF32 split
+// (JANUS_FFN_3XTF32).  Internal header, included by expert_ffn.cu.
+#pragma once
+
+#include "common.cuh"
+
+namespace janus {
+namespace tc {
+
+// extra workspace bytes the tensor-core path needs beyond the activations
+size_t workspace_extra();
+
+janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, int64_t R,
+                            int32_t d, int32_t h, const float* w1, const float* w2, float* yd,
+                            float* act, float* H, void* extra, cudaStream_t stream);
+
+janus_status expert_ffn_vjp(const float* xd, const float* gd, const float* act_in, float* A,
+                            const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
+                            const float* w1, const float* w2, float* dxd, float* dA, void* extra,
+                            cudaStream_t stream);
+
+}  // namespace tc
+}  // namespace janus

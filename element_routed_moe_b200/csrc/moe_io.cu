@@ -1,0 +1,375 @@
+// Token movement of the MoE layer: dispatch, combine, and the atom-type-aware
+// FP16 packing of the dispatch buffer.
+//
+// Sources: paper review "Breaking the Training Barrier of Billion-Parameter
+// Universal Machine Learning Interatomic Potentials" section 3.5 (CNIS:
+// MoE dispatch/combine kernels; atom-type-aware FP16 compression), and
+// "MatRIS-MoE与Janus框架" section 3.2 (gate-weighted sum of expert outputs).
+//
+// All four are HBM-bound streams.  Layout choices for B200:
+//   * one warp per atom row, 128-bit accesses, U = 4 independent 16-byte
+//     loads per lane in flight (2 KB per warp) before any store;
+//   * dispatch and pack run in scatter form: the atom row is read once and
+//     written to its K dispatch rows (slot_of gives each destination; every
+//     destination is distinct, so no atomics and a deterministic result);
+//   * combine runs in gather form: the K expert rows of an atom are read and
+//     summed in k order, one output row written;
+//   * grids are a multiple of the SM count with grid-stride loops over rows.
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+
+namespace janus {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarpsPerBlock = kThreads / 32;
+constexpr int kU = 4;
+
+inline unsigned rows_grid(int64_t rows, int blocks_per_sm) {
+  int64_t need = (rows + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  int64_t cap = (int64_t)num_sms() * blocks_per_sm;
+  return (unsigned)(need < cap ? (need > 0 ? need : 1) : cap);
+}
+
+__device__ __forceinline__ int64_t global_warp() {
+  return ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+}
+__device__ __forceinline__ int64_t total_warps() {
+  return (int64_t)gridDim.x * blockDim.x / 32;
+}
+
+// slot_of / weight of the atom's k-th slot: lanes < K hold them when K <= 32
+template <bool kWeighted>
+__device__ __forceinline__ void slot_k(int k, int K, int64_t i, int my_slot, float my_w,
+                                       const int32_t* __restrict__ slot_of,
+                                       const float* __restrict__ w, int64_t* p, float* wk) {
+  if (K <= 32) {
+    *p = __shfl_sync(0xffffffffu, my_slot, k);
+    *wk = kWeighted ? __shfl_sync(0xffffffffu, my_w, k) : 1.0f;
+  } else {
+    *p = slot_of[i * K + k];
+    *wk = kWeighted ? w[i * K + k] : 1.0f;
+  }
+}
+
+template <bool kWeighted>
+__global__ void __launch_bounds__(kThreads)
+dispatch_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K,
+                const int32_t* __restrict__ slot_of, const float* __restrict__ w,
+                float4* __restrict__ xd) {
+  const int lane = threadIdx.x % 32;
+  for (int64_t i = global_warp(); i < n_atoms; i += total_warps()) {
+    const int my_slot = lane < K ? slot_of[i * K + lane] : 0;
+    const float my_w = (kWeighted && lane < K) ? w[i * K + lane] : 1.0f;
+    const float4* src = x + i * d4;
+    for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
+      float4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < d4) v[u] = __ldcs(src + c);
+      }
+      for (int k = 0; k < K; ++k) {
+        int64_t p;
+        float wk;
+        slot_k<kWeighted>(k, K, i, my_slot, my_w, slot_of, w, &p, &wk);
+        float4* dst = xd + p * d4;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int c = c0 + u * 32 + lane;
+          if (c < d4) {
+            float4 o = v[u];
+            if (kWeighted) { o.x *= wk; o.y *= wk; o.z *= wk; o.w *= wk; }
+            dst[c] = o;
+          }
+        }
+      }
+    }
+  }
+}
+
+template <bool kWeighted>
+__global__ void __launch_bounds__(kThreads)
+combine_kernel(const float4* __restrict__ yd, const int32_t* __restrict__ slot_of,
+               const float* __restrict__ w, int64_t n_atoms, int K, int d4,
+               float4* __restrict__ y) {
+  const int lane = threadIdx.x % 32;
+  for (int64_t i = global_warp(); i < n_atoms; i += total_warps()) {
+    const int my_slot = lane < K ? slot_of[i * K + lane] : 0;
+    const float my_w = (kWeighted && lane < K) ? w[i * K + lane] : 1.0f;
+    for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
+      float4 acc[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int k = 0; k < K; ++k) {
+        int64_t p;
+        float wk;
+        slot_k<kWeighted>(k, K, i, my_slot, my_w, slot_of, w, &p, &wk);
+        const float4* src = yd + p * d4;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int c = c0 + u * 32 + lane;
+          if (c < d4) {
+            const float4 v = __ldcs(src + c);
+            if (kWeighted) {
+              acc[u].x = fmaf(wk, v.x, acc[u].x);
+              acc[u].y = fmaf(wk, v.y, acc[u].y);
+              acc[u].z = fmaf(wk, v.z, acc[u].z);
+              acc[u].w = fmaf(wk, v.w, acc[u].w);
+            } else {
+              acc[u].x += v.x; acc[u].y += v.y; acc[u].z += v.z; acc[u].w += v.w;
+            }
+          }
+        }
+      }
+      float4* dst = y + i * d4;
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < d4) dst[c] = acc[u];
+      }
+    }
+  }
+}
+
+// ---- atom-type-aware FP16 packing ------------------------------------------
+
+// |x| as ordered bits: for non-negative floats the integer order is the
+// float order, and any NaN compares above +inf.
+__device__ __forceinline__ uint32_t abs_bits(float v) { return __float_as_uint(v) & 0x7fffffffu; }
+
+__global__ void __launch_bounds__(kThreads)
+quant_amax_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4,
+                  const int32_t* __restrict__ types, int T, uint32_t* __restrict__ amax_bits,
+                  WsHeader* ws) {
+  extern __shared__ uint32_t s_amax[];
+  for (int t = threadIdx.x; t < T; t += kThreads) s_amax[t] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x % 32;
+  for (int64_t i = global_warp(); i < n_atoms; i += total_warps()) {
+    int t = types[i];
+    if (t < 0 || t >= T) {
+      if (lane == 0) record_fault(ws, kFaultBadType);
+      t = 0;
+    }
+    const float4* src = x + i * d4;
+    uint32_t m = 0;
+    for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
+      float4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + u * 32 + lane;
+        v[u] = c < d4 ? __ldg(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        m = max(m, max(max(abs_bits(v[u].x), abs_bits(v[u].y)), max(abs_bits(v[u].z), abs_bits(v[u].w))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0 && m) atomicMax(&s_amax[t], m);
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < T; t += kThreads)
+    if (s_amax[t]) atomicMax(&amax_bits[t], s_amax[t]);
+}
+
+// Exponent e of the type scale 2^e: the smallest e with amax <= 65504 * 2^e,
+// clamped to [-126, 127].  With amax = 1.M * 2^(Eb-127) (Eb = biased
+// exponent field), 65504 = (2 - 2^-10) * 2^15, so e = Eb - 142, plus one when
+// the mantissa exceeds that of 65504 (M > 0x7FE000).
+__device__ __forceinline__ int scale_exponent_from_bits(uint32_t amax) {
+  if (amax == 0) return 0;
+  const int eb = (int)(amax >> 23);
+  const uint32_t mant = amax & 0x7fffffu;
+  int e = (eb == 0) ? -126 : eb - 142 + (mant > 0x7fe000u ? 1 : 0);
+  return e < -126 ? -126 : (e > 127 ? 127 : e);
+}
+
+__global__ void __launch_bounds__(kThreads)
+quant_pack_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K,
+                  const int32_t* __restrict__ types, int T, const int32_t* __restrict__ slot_of,
+                  const uint32_t* __restrict__ amax_bits, uint2* __restrict__ payload,
+                  float* __restrict__ scale, WsHeader* ws) {
+  extern __shared__ float s_inv[];
+  for (int t = threadIdx.x; t < T; t += kThreads) {
+    const uint32_t a = amax_bits[t];
+    const int e = scale_exponent_from_bits(a);
+    // 2^-e is a normal float for every e a finite amax can produce
+    s_inv[t] = (e <= 126) ? __uint_as_float((uint32_t)(127 - e) << 23) : 0.0f;
+    if (blockIdx.x == 0) {
+      scale[t] = __uint_as_float((uint32_t)(127 + e) << 23);
+      if (a >= 0x7f800000u) record_fault(ws, kFaultNonFinite);
+    }
+  }
+  __syncthreads();
+  const int lane = threadIdx.x % 32;
+  for (int64_t i = global_warp(); i < n_atoms; i += total_warps()) {
+    int t = types[i];
+    if (t < 0 || t >= T) t = 0;                // recorded by the amax pass
+    const float inv = s_inv[t];
+    const int my_slot = lane < K ? slot_of[i * K + lane] : 0;
+    const float4* src = x + i * d4;
+    for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
+      uint2 q[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < d4) {
+          const float4 v = __ldcs(src + c);
+          // exact power-of-two scaling, then one round-to-nearest-even
+          const __half2 lo = __floats2half2_rn(v.x * inv, v.y * inv);
+          const __half2 hi = __floats2half2_rn(v.z * inv, v.w * inv);
+          q[u].x = *reinterpret_cast<const uint32_t*>(&lo);
+          q[u].y = *reinterpret_cast<const uint32_t*>(&hi);
+        }
+      }
+      for (int k = 0; k < K; ++k) {
+        const int64_t p = K <= 32 ? __shfl_sync(0xffffffffu, my_slot, k) : slot_of[i * K + k];
+        uint2* dst = payload + p * d4;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int c = c0 + u * 32 + lane;
+          if (c < d4) dst[c] = q[u];
+        }
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+dequant_kernel(const uint2* __restrict__ payload, int64_t n_rows, int d4, int K,
+               const int32_t* __restrict__ types, int T, const int32_t* __restrict__ perm,
+               const float* __restrict__ scale, float4* __restrict__ xd) {
+  const int lane = threadIdx.x % 32;
+  for (int64_t p = global_warp(); p < n_rows; p += total_warps()) {
+    int t = types[perm[p] / K];
+    if (t < 0 || t >= T) t = 0;
+    const float s = scale[t];
+    const uint2* src = payload + p * d4;
+    float4* dst = xd + p * d4;
+    for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
+      uint2 q[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < d4) q[u] = __ldcs(src + c);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < d4) {
+          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&q[u].x));
+          const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&q[u].y));
+          dst[c] = make_float4(a.x * s, a.y * s, b.x * s, b.y * s);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+}  // namespace janus
+
+using namespace janus;
+
+static janus_status check_rows(int64_t n_atoms, int32_t d, int32_t top_k) {
+  JANUS_CHECK_ARG(n_atoms >= 0 && top_k >= 1 && top_k <= kMaxExperts);
+  JANUS_CHECK_ARG(d >= 1 && d <= kMaxDim);
+  JANUS_CHECK_ARG(n_atoms * (int64_t)top_k < (int64_t)INT32_MAX);
+  JANUS_CHECK_ALIGN(d % 4 == 0);
+  return JANUS_OK;
+}
+
+extern "C" janus_status janus_dispatch(const float* x, int64_t n_atoms, int32_t d, int32_t top_k,
+                                       const int32_t* slot_of, const float* topk_weight,
+                                       float* xd, janus_stream_t stream) {
+  janus_status st = check_rows(n_atoms, d, top_k);
+  if (st != JANUS_OK) return st;
+  if (n_atoms == 0) return JANUS_OK;
+  JANUS_CHECK_ARG(x && slot_of && xd);
+  JANUS_CHECK_ALIGN(aligned(x, 16) && aligned(xd, 16));
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  const unsigned grid = rows_grid(n_atoms, 8);
+  if (topk_weight)
+    dispatch_kernel<true><<<grid, kThreads, 0, (cudaStream_t)stream>>>(
+        (const float4*)x, n_atoms, d / 4, top_k, slot_of, topk_weight, (float4*)xd);
+  else
+    dispatch_kernel<false><<<grid, kThreads, 0, (cudaStream_t)stream>>>(
+        (const float4*)x, n_atoms, d / 4, top_k, slot_of, nullptr, (float4*)xd);
+  return launch_status();
+}
+
+extern "C" janus_status janus_combine(const float* yd, const int32_t* slot_of,
+                                      const float* topk_weight, int64_t n_atoms, int32_t top_k,
+                                      int32_t d, float* y, janus_stream_t stream) {
+  janus_status st = check_rows(n_atoms, d, top_k);
+  if (st != JANUS_OK) return st;
+  if (n_atoms == 0) return JANUS_OK;
+  JANUS_CHECK_ARG(yd && slot_of && y);
+  JANUS_CHECK_ALIGN(aligned(yd, 16) && aligned(y, 16));
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  const unsigned grid = rows_grid(n_atoms, 8);
+  if (topk_weight)
+    combine_kernel<true><<<grid, kThreads, 0, (cudaStream_t)stream>>>(
+        (const float4*)yd, slot_of, topk_weight, n_atoms, top_k, d / 4, (float4*)y);
+  else
+    combine_kernel<false><<<grid, kThreads, 0, (cudaStream_t)stream>>>(
+        (const float4*)yd, slot_of, nullptr, n_atoms, top_k, d / 4, (float4*)y);
+  return launch_status();
+}
+
+extern "C" janus_status janus_quant_by_type_workspace_size(int32_t n_types, size_t* bytes) {
+  JANUS_CHECK_ARG(bytes && n_types >= 1 && n_types <= kMaxTypes);
+  *bytes = sizeof(WsHeader) + align_up(sizeof(uint32_t) * (size_t)n_types, 256);
+  return JANUS_OK;
+}
+
+extern "C" janus_status janus_quant_by_type(const float* x, int64_t n_atoms, int32_t d,
+                                            int32_t top_k, const int32_t* types, int32_t n_types,
+                                            const int32_t* slot_of, uint16_t* payload,
+                                            float* scale, void* workspace,
+                                            size_t workspace_bytes, janus_stream_t stream_) {
+  cudaStream_t stream = (cudaStream_t)stream_;
+  janus_status st = check_rows(n_atoms, d, top_k);
+  if (st != JANUS_OK) return st;
+  size_t need = 0;
+  st = janus_quant_by_type_workspace_size(n_types, &need);
+  if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(scale && workspace && workspace_bytes >= need);
+  JANUS_CHECK_ARG(n_atoms == 0 || (x && types && slot_of && payload));
+  JANUS_CHECK_ALIGN(aligned(workspace, 256));
+  JANUS_CHECK_ALIGN(n_atoms == 0 || (aligned(x, 16) && aligned(payload, 8)));
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  WsHeader* hdr = (WsHeader*)workspace;
+  uint32_t* amax_bits = (uint32_t*)((char*)workspace + sizeof(WsHeader));
+  JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, need, stream));
+  const size_t smem = sizeof(uint32_t) * (size_t)n_types;
+  const unsigned grid = rows_grid(n_atoms, 8);
+  if (n_atoms > 0)
+    quant_amax_kernel<<<grid, kThreads, smem, stream>>>((const float4*)x, n_atoms, d / 4, types,
+                                                        n_types, amax_bits, hdr);
+  quant_pack_kernel<<<grid, kThreads, smem, stream>>>((const float4*)x, n_atoms, d / 4, top_k,
+                                                      types, n_types, slot_of, amax_bits,
+                                                      (uint2*)payload, scale, hdr);
+  return launch_status();
+}
+
+extern "C" janus_status janus_dequant_by_type(const uint16_t* payload, int64_t n_atoms, int32_t d,
+                                              int32_t top_k, const int32_t* types,
+                                              int32_t n_types, const int32_t* perm,
+                                              const float* scale, float* xd,
+                                              janus_stream_t stream) {
+  janus_status st = check_rows(n_atoms, d, top_k);
+  if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(n_types >= 1 && n_types <= kMaxTypes);
+  if (n_atoms == 0) return JANUS_OK;
+  JANUS_CHECK_ARG(payload && types && perm && scale && xd);
+  JANUS_CHECK_ALIGN(aligned(payload, 8) && aligned(xd, 16));
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  const int64_t R = n_atoms * top_k;
+  dequant_kernel<<<rows_grid(R, 8), kThreads, 0, (cudaStream_t)stream>>>(
+      (const uint2*)payload, R, d / 4, top_k, types, n_types, perm, scale, (float4*)xd);
+  return launch_status();
+}

@@ -1,0 +1,311 @@
+"""Thin ctypes binding over libjanus.so (the C ABI declared in include/janus.h).
+
+Argument marshalling only: every function checks tensor placement/dtype,
+allocates outputs and workspaces with PyTorch (device memory is PyTorch's
+job here), passes raw device pointers and the current CUDA stream, and turns a
+non-zero ``janus_status`` into ``JanusError``.  Every step of the computation
+runs in the library's CUDA kernels; there is no CPU or PyTorch fallback, and
+importing this module fails loudly when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libjanus.so")
+
+JANUS_OK = 0
+JANUS_ERR_INVALID_ARG = 1
+JANUS_ERR_MISALIGNED = 2
+JANUS_ERR_CUDA = 3
+JANUS_ERR_DATA = 4
+
+JANUS_FFN_FP32_SIMT = 0
+JANUS_FFN_3XTF32 = 1
+
+# Every entry point declared in include/janus.h.
+SYMBOLS = (
+    "janus_status_string", "janus_version", "janus_check",
+    "janus_route_workspace_size", "janus_route",
+    "janus_dispatch",
+    "janus_quant_by_type_workspace_size", "janus_quant_by_type", "janus_dequant_by_type",
+    "janus_expert_ffn_workspace_size", "janus_expert_ffn_fwd", "janus_expert_ffn_vjp",
+    "janus_combine", "janus_edge_aggregate",
+    "janus_debug_inject_launch_failures",
+)
+
+
+class JanusError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m element_routed_moe_b200.build`"
+                " (nvcc, sm_100a); there is no fallback implementation")
+        _lib = ctypes.CDLL(LIB_PATH)
+        _declare(_lib)
+    return _lib
+
+
+def _declare(L):
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    psz = ctypes.POINTER(ctypes.c_size_t)
+    st = ctypes.c_int
+    sig = {
+        "janus_status_string": (ctypes.c_char_p, [st]),
+        "janus_version": (i32, []),
+        "janus_check": (st, [vp, vp]),
+        "janus_route_workspace_size": (st, [i64, i32, i32, i32, psz]),
+        "janus_route": (st, [vp, i64, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "janus_dispatch": (st, [vp, i64, i32, i32, vp, vp, vp, vp]),
+        "janus_quant_by_type_workspace_size": (st, [i32, psz]),
+        "janus_quant_by_type": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp, sz, vp]),
+        "janus_dequant_by_type": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp]),
+        "janus_expert_ffn_workspace_size": (st, [i64, i32, i32, i32, i32, i32, ctypes.c_int, psz]),
+        "janus_expert_ffn_fwd": (st, [vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, ctypes.c_int,
+                                      vp, sz, vp]),
+        "janus_expert_ffn_vjp": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp,
+                                      ctypes.c_int, vp, sz, vp]),
+        "janus_combine": (st, [vp, vp, vp, i64, i32, i32, vp, vp]),
+        "janus_edge_aggregate": (st, [vp, vp, i64, i32, vp, vp]),
+        "janus_debug_inject_launch_failures": (None, [i32]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+
+
+def status_string(status: int) -> str:
+    return lib().janus_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return int(lib().janus_version())
+
+
+def _raise(status: int, where: str):
+    if status != JANUS_OK:
+        raise JanusError(status, where)
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _p(t, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr() if t.numel() > 0 else None
+
+
+def _empty(shape, dtype, device):
+    return torch.empty(shape, dtype=dtype, device=device)
+
+
+def _workspace(nbytes, device, ws):
+    if ws is not None:
+        if ws.numel() * ws.element_size() < nbytes:
+            raise ValueError("workspace too small")
+        return ws
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+# --------------------------------------------------------------------------
+# routing
+# --------------------------------------------------------------------------
+def janus_route_workspace_size(n_atoms: int, n_types: int, n_experts: int, top_k: int) -> int:
+    b = ctypes.c_size_t(0)
+    _raise(lib().janus_route_workspace_size(n_atoms, n_types, n_experts, top_k, ctypes.byref(b)),
+           "janus_route_workspace_size")
+    return b.value
+
+
+def janus_route(types, gate, top_k, *, out=None, workspace=None, stream=None):
+    """Static per-element top-K routing; returns a dict of device tensors
+    (topk_expert, topk_weight, counts, offsets, perm, slot_of, workspace)."""
+    dev = gate.device
+    N = types.shape[0]
+    T, E = gate.shape
+    K = int(top_k)
+    R = N * K
+    if out is None:
+        out = dict(topk_expert=_empty((N, K), torch.int32, dev),
+                   topk_weight=_empty((N, K), torch.float32, dev),
+                   counts=_empty((E,), torch.int32, dev),
+                   offsets=_empty((E + 1,), torch.int32, dev),
+                   perm=_empty((R,), torch.int32, dev),
+                   slot_of=_empty((R,), torch.int32, dev))
+    nb = janus_route_workspace_size(N, T, E, K)
+    ws = _workspace(nb, dev, workspace)
+    _raise(lib().janus_route(_p(types, torch.int32, "types"), N, _p(gate, torch.float32, "gate"),
+                             T, E, K, _p(out["topk_expert"]), _p(out["topk_weight"]),
+                             _p(out["counts"]), _p(out["offsets"]), _p(out["perm"]),
+                             _p(out["slot_of"]), _p(ws), nb, _stream(stream)), "janus_route")
+    out["workspace"] = ws
+    return out
+
+
+def janus_check(workspace, stream=None):
+    _raise(lib().janus_check(_p(workspace), _stream(stream)), "janus_check")
+
+
+# --------------------------------------------------------------------------
+# dispatch / combine
+# --------------------------------------------------------------------------
+def janus_dispatch(x, slot_of, top_k, topk_weight=None, *, out=None, stream=None):
+    N, d = x.shape
+    K = int(top_k)
+    if out is None:
+        out = _empty((N * K, d), torch.float32, x.device)
+    _raise(lib().janus_dispatch(_p(x, torch.float32, "x"), N, d, K,
+                                _p(slot_of, torch.int32, "slot_of"),
+                                _p(topk_weight, torch.float32, "topk_weight"),
+                                _p(out, torch.float32, "xd"), _stream(stream)), "janus_dispatch")
+    return out
+
+
+def janus_combine(yd, slot_of, top_k, topk_weight=None, *, out=None, stream=None):
+    K = int(top_k)
+    R, d = yd.shape
+    N = slot_of.shape[0] // K
+    if out is None:
+        out = _empty((N, d), torch.float32, yd.device)
+    _raise(lib().janus_combine(_p(yd, torch.float32, "yd"), _p(slot_of, torch.int32, "slot_of"),
+                               _p(topk_weight, torch.float32, "topk_weight"), N, K, d,
+                               _p(out, torch.float32, "y"), _stream(stream)), "janus_combine")
+    return out
+
+
+# --------------------------------------------------------------------------
+# per-element-type FP16 packing
+# --------------------------------------------------------------------------
+def janus_quant_by_type_workspace_size(n_types: int) -> int:
+    b = ctypes.c_size_t(0)
+    _raise(lib().janus_quant_by_type_workspace_size(n_types, ctypes.byref(b)),
+           "janus_quant_by_type_workspace_size")
+    return b.value
+
+
+def janus_quant_by_type(x, types, n_types, slot_of, top_k, *, payload=None, scale=None,
+                        workspace=None, stream=None):
+    """Returns (payload [R,d] float16 (binary16 bits), scale [T] float32, workspace)."""
+    N, d = x.shape
+    K = int(top_k)
+    if payload is None:
+        payload = _empty((N * K, d), torch.float16, x.device)
+    if scale is None:
+        scale = _empty((n_types,), torch.float32, x.device)
+    nb = janus_quant_by_type_workspace_size(n_types)
+    ws = _workspace(nb, x.device, workspace)
+    _raise(lib().janus_quant_by_type(_p(x, torch.float32, "x"), N, d, K,
+                                     _p(types, torch.int32, "types"), int(n_types),
+                                     _p(slot_of, torch.int32, "slot_of"), _p(payload, None, "payload"),
+                                     _p(scale, torch.float32, "scale"), _p(ws), nb,
+                                     _stream(stream)), "janus_quant_by_type")
+    return payload, scale, ws
+
+
+def janus_dequant_by_type(payload, types, n_types, perm, top_k, scale, *, out=None, stream=None):
+    R, d = payload.shape
+    K = int(top_k)
+    N = types.shape[0]
+    if out is None:
+        out = _empty((R, d), torch.float32, payload.device)
+    _raise(lib().janus_dequant_by_type(_p(payload, None, "payload"), N, d, K,
+                                       _p(types, torch.int32, "types"), int(n_types),
+                                       _p(perm, torch.int32, "perm"),
+                                       _p(scale, torch.float32, "scale"),
+                                       _p(out, torch.float32, "xd"), _stream(stream)),
+           "janus_dequant_by_type")
+    return out
+
+
+# --------------------------------------------------------------------------
+# grouped expert MLP
+# --------------------------------------------------------------------------
+def janus_expert_ffn_workspace_size(n_rows, d, h, n_experts, vjp, have_act,
+                                    mode=JANUS_FFN_FP32_SIMT) -> int:
+    b = ctypes.c_size_t(0)
+    _raise(lib().janus_expert_ffn_workspace_size(n_rows, d, h, n_experts, int(bool(vjp)),
+                                                 int(bool(have_act)), int(mode), ctypes.byref(b)),
+           "janus_expert_ffn_workspace_size")
+    return b.value
+
+
+def janus_expert_ffn_fwd(xd, offsets, w1, w2, *, mode=JANUS_FFN_FP32_SIMT, want_act=False,
+                         out=None, act=None, workspace=None, stream=None):
+    """yd = silu(xd W1[e]) W2[e] per expert segment; returns (yd, act-or-None)."""
+    R, d = xd.shape
+    E, _, h = w1.shape
+    if out is None:
+        out = _empty((R, d), torch.float32, xd.device)
+    if want_act and act is None:
+        act = _empty((R, h), torch.float32, xd.device)
+    nb = janus_expert_ffn_workspace_size(R, d, h, E, False, act is not None, mode)
+    ws = _workspace(nb, xd.device, workspace)
+    _raise(lib().janus_expert_ffn_fwd(_p(xd, torch.float32, "xd"),
+                                      _p(offsets, torch.int32, "offsets"), E, R, d, h,
+                                      _p(w1, torch.float32, "w1"), _p(w2, torch.float32, "w2"),
+                                      _p(out, torch.float32, "yd"), _p(act, torch.float32, "act"),
+                                      int(mode), _p(ws), nb, _stream(stream)),
+           "janus_expert_ffn_fwd")
+    return out, act
+
+
+def janus_expert_ffn_vjp(xd, gd, offsets, w1, w2, *, act=None, mode=JANUS_FFN_FP32_SIMT,
+                         out=None, workspace=None, stream=None):
+    R, d = xd.shape
+    E, _, h = w1.shape
+    if out is None:
+        out = _empty((R, d), torch.float32, xd.device)
+    nb = janus_expert_ffn_workspace_size(R, d, h, E, True, act is not None, mode)
+    ws = _workspace(nb, xd.device, workspace)
+    _raise(lib().janus_expert_ffn_vjp(_p(xd, torch.float32, "xd"), _p(gd, torch.float32, "gd"),
+                                      _p(act, torch.float32, "act"),
+                                      _p(offsets, torch.int32, "offsets"), E, R, d, h,
+                                      _p(w1, torch.float32, "w1"), _p(w2, torch.float32, "w2"),
+                                      _p(out, torch.float32, "dxd"), int(mode), _p(ws), nb,
+                                      _stream(stream)), "janus_expert_ffn_vjp")
+    return out
+
+
+# --------------------------------------------------------------------------
+# edge aggregation
+# --------------------------------------------------------------------------
+def janus_edge_aggregate(msg, row_ptr, *, out=None, stream=None):
+    N = row_ptr.shape[0] - 1
+    d = msg.shape[1]
+    if out is None:
+        out = _empty((N, d), torch.float32, msg.device)
+    _raise(lib().janus_edge_aggregate(_p(msg, torch.float32, "msg"),
+                                      _p(row_ptr, torch.int64, "row_ptr"), N, d,
+                                      _p(out, torch.float32, "out"), _stream(stream)),
+           "janus_edge_aggregate")
+    return out
+
+
+def janus_debug_inject_launch_failures(n_calls: int):
+    lib().janus_debug_inject_launch_failures(int(n_calls))

@@ -1,0 +1,213 @@
+/*
+ * janus.h - C ABI of libjanus.so: the element-type-routed sparse MoE layer over
+ * atom feature tokens and the edge-to-atom aggregation that feeds it, as
+ * hand-written CUDA kernels for B200 (sm_100a).
+ *
+ * Sources (web pages on the method, cited by title and section):
+ *   [Review]    "Breaking the Training Barrier of Billion-Parameter Universal
+ *               Machine Learning Interatomic Potentials" (xllm-io paper review)
+ *   [News]      "11.5B参数、1.2EFLOPS、训练从数周压到数小时" (ScienceAI)
+ *   [Blueprint] "MatRIS-MoE与Janus框架：构建百亿参数通用机器学习原子间势"
+ *
+ * Notation: N atoms, T element types, E experts, K experts per atom (top-K),
+ * R = N*K routed tokens ("slots"), d feature size, h expert hidden size,
+ * Ed edges.  Flat slot s = i*K + k is atom i's k-th expert.  The dispatch
+ * buffer holds one row per slot, grouped by expert: rows
+ * [offsets[e], offsets[e+1]) belong to expert e, atoms ascending inside.
+ *
+ * Conventions for every call:
+ *   - Every array argument is a DEVICE pointer (cudaMalloc'd or managed),
+ *     owned by the caller.  The library never allocates or frees memory; a
+ *     call that needs scratch space takes a caller-owned `workspace` whose
+ *     size is given by the matching *_workspace_size query.
+ *   - Every call is asynchronous on the given stream (0 = legacy default
+ *     stream), never synchronises (except janus_check), and is thread-safe.
+ *   - Arrays are dense row-major.  FP32 feature rows ([*, d]) need a 16-byte
+ *     aligned base and d % 4 == 0; FP16 payload rows need an 8-byte aligned
+ *     base (same d rule).  Otherwise JANUS_ERR_MISALIGNED.
+ *   - Limits: 1 <= K <= E <= 256, 1 <= T <= 4096, N*K < 2^31, 1 <= d, h <= 2^20.
+ *     Edge counts and feature element offsets are 64-bit.
+ *   - Arguments are checked before anything is launched: a failed check
+ *     returns an error and launches nothing.  Index arrays that a call takes
+ *     as input (perm, slot_of, offsets, row_ptr) must be what janus_route /
+ *     a valid CSR would produce; they are not re-validated on the device.
+ *   - Data-dependent faults (a type id outside [0,T), a non-finite feature
+ *     to be packed) are recorded in the workspace's error word and reported
+ *     by janus_check(); the call still writes every output (bad type ids are
+ *     treated as type 0) so no out-of-bounds access can follow.
+ */
+#ifndef JANUS_H_
+#define JANUS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* janus_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  JANUS_OK = 0,
+  JANUS_ERR_INVALID_ARG = 1, /* null pointer, size/limit violation, workspace too small */
+  JANUS_ERR_MISALIGNED = 2,  /* feature pointer not 16-byte (FP32) / 8-byte (FP16) aligned, or d % 4 != 0 */
+  JANUS_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed */
+  JANUS_ERR_DATA = 4         /* data-dependent fault recorded on the device (see janus_check) */
+} janus_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* janus_status_string(janus_status s);
+
+/* Library ABI version (major*10000 + minor*100 + patch). */
+int32_t janus_version(void);
+
+/* Synchronises `stream`, then reads the error word at the start of a
+ * workspace used by janus_route or janus_quant_by_type.  Returns JANUS_OK,
+ * JANUS_ERR_DATA if a kernel recorded a data fault, or JANUS_ERR_CUDA. */
+janus_status janus_check(const void* workspace, janus_stream_t stream);
+
+/* -------------------------------------------------------------------------
+ * Routing.  [Review] section 3.2 (sparse MoE design): each element type
+ * activates its own top-K experts, so the active set does not depend on the
+ * coordinates; [News] (model architecture paragraph) says the same.  [News]
+ * (training framework paragraph): JIT planning routes a batch before the
+ * step and counts the tokens per expert.
+ *
+ *   S_t = the K experts with the largest gate[t, :], descending logit, ties
+ *         to the lower expert id;
+ *   topk_expert[i,k] = S_{types[i]}[k];
+ *   topk_weight[i,k] = softmax over the K selected logits of gate[types[i],:];
+ *   counts[e]  = number of slots routed to e;  offsets = exclusive scan
+ *                (offsets[0] = 0, offsets[E] = R);
+ *   perm[p]    = the slot held by dispatch row p (stable: slots ascending
+ *                inside each expert);  slot_of[perm[p]] = p.
+ *
+ * in : types [N] int32, gate [T,E] float32 (finite)
+ * out: topk_expert [N,K] int32, topk_weight [N,K] float32, counts [E] int32,
+ *      offsets [E+1] int32, perm [R] int32, slot_of [R] int32
+ * workspace: janus_route_workspace_size() bytes; its error word records type
+ *      ids outside [0,T) (those atoms are routed as type 0).
+ * N == 0 is allowed (counts and offsets are zeroed).
+ * ------------------------------------------------------------------------- */
+janus_status janus_route_workspace_size(int64_t n_atoms, int32_t n_types,
+                                        int32_t n_experts, int32_t top_k,
+                                        size_t* bytes);
+janus_status janus_route(const int32_t* types, int64_t n_atoms, const float* gate,
+                         int32_t n_types, int32_t n_experts, int32_t top_k,
+                         int32_t* topk_expert, float* topk_weight, int32_t* counts,
+                         int32_t* offsets, int32_t* perm, int32_t* slot_of,
+                         void* workspace, size_t workspace_bytes,
+                         janus_stream_t stream);
+
+/* -------------------------------------------------------------------------
+ * Dispatch.  [Review] section 3.5 (CNIS kernels, MoE dispatch/combine).
+ *   xd[slot_of[i*K+k], :] = x[i, :] * (topk_weight ? topk_weight[i*K+k] : 1)
+ * The weighted form is the first step of the input VJP (upstream gradient
+ * times gate weight).  Each atom row is read once and written K times.
+ * in : x [N,d] float32, slot_of [R] int32, topk_weight [N,K] float32 or NULL
+ * out: xd [R,d] float32
+ * ------------------------------------------------------------------------- */
+janus_status janus_dispatch(const float* x, int64_t n_atoms, int32_t d, int32_t top_k,
+                            const int32_t* slot_of, const float* topk_weight,
+                            float* xd, janus_stream_t stream);
+
+/* -------------------------------------------------------------------------
+ * Atom-type-aware FP16 packing.  [Review] section 3.5 (CNIS, atom-type-aware
+ * FP16 compression): after routing, the dispatch buffer's tokens are grouped
+ * by atom type, quantised with one scale per type, carried as FP16 (half the
+ * FP32 bytes) and dequantised afterwards.
+ *   amax_t  = max |x[i,j]| over atoms i of type t;
+ *   scale_t = the smallest power of two 2^e with amax_t <= 65504 * 2^e,
+ *             e clamped to [-126, 127]; 1 if amax_t == 0 or type t is absent;
+ *   payload[slot_of[i*K+k], j] = binary16_rne(x[i,j] / scale_{types[i]}).
+ * Fused gather: x is read twice (amax pass, pack pass); payload is written in
+ * dispatch order.
+ * in : x [N,d] float32, types [N], slot_of [R]
+ * out: payload [R,d] IEEE binary16 bit patterns, scale [T] float32
+ * workspace: janus_quant_by_type_workspace_size() bytes; its error word
+ *      records bad type ids and non-finite features.
+ * ------------------------------------------------------------------------- */
+janus_status janus_quant_by_type_workspace_size(int32_t n_types, size_t* bytes);
+janus_status janus_quant_by_type(const float* x, int64_t n_atoms, int32_t d, int32_t top_k,
+                                 const int32_t* types, int32_t n_types,
+                                 const int32_t* slot_of, uint16_t* payload, float* scale,
+                                 void* workspace, size_t workspace_bytes,
+                                 janus_stream_t stream);
+
+/* Dequantisation of a packed dispatch buffer (same passage):
+ *   xd[p, j] = float(payload[p, j]) * scale[types[perm[p] / K]]   (exact)
+ * in : payload [R,d] binary16 bits, types [N], perm [R], scale [T]
+ * out: xd [R,d] float32 */
+janus_status janus_dequant_by_type(const uint16_t* payload, int64_t n_atoms, int32_t d,
+                                   int32_t top_k, const int32_t* types, int32_t n_types,
+                                   const int32_t* perm, const float* scale, float* xd,
+                                   janus_stream_t stream);
+
+/* -------------------------------------------------------------------------
+ * Grouped expert MLP.  [Review] section 3.1, Table II (MLP hidden size);
+ * each expert is read as bias-free Linear(d,h) -> SiLU -> Linear(h,d):
+ *   for rows p in [offsets[e], offsets[e+1]):
+ *     a = xd[p,:] W1[e]      (W1 [E,d,h] row-major)
+ *     yd[p,:] = silu(a) W2[e] (W2 [E,h,d] row-major),  silu(a) = a / (1 + exp(-a))
+ * Input VJP ([Review] section 3.3: forces and stress are autodiff gradients
+ * of the energy, so the layer's input gradient is needed):
+ *   dxd[p,:] = W1[e] ( (W2[e] gd[p,:]) * silu'(a) ),  silu'(a) = sig(a)(1 + a(1 - sig(a)))
+ * offsets stays on the device (the tile scheduler reads it there; no host
+ * synchronisation).  n_rows = R = offsets[E].
+ * FP32 inputs/outputs; accuracy mode:
+ *   JANUS_FFN_FP32_SIMT : FP32 FFMA on the CUDA cores;
+ *   JANUS_FFN_3XTF32    : tcgen05 tensor cores, each FP32 operand split into
+ *                         a TF32 high part and a TF32 residual, three products.
+ * fwd: act [R,h] (nullable) receives a; the workspace holds silu(a).
+ * vjp: act (nullable) is a from the forward; NULL recomputes it.
+ * ------------------------------------------------------------------------- */
+typedef enum { JANUS_FFN_FP32_SIMT = 0, JANUS_FFN_3XTF32 = 1 } janus_ffn_mode;
+
+janus_status janus_expert_ffn_workspace_size(int64_t n_rows, int32_t d, int32_t h,
+                                             int32_t n_experts, int32_t vjp,
+                                             int32_t have_act, janus_ffn_mode mode,
+                                             size_t* bytes);
+janus_status janus_expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t n_experts,
+                                  int64_t n_rows, int32_t d, int32_t h, const float* w1,
+                                  const float* w2, float* yd, float* act, janus_ffn_mode mode,
+                                  void* workspace, size_t workspace_bytes,
+                                  janus_stream_t stream);
+janus_status janus_expert_ffn_vjp(const float* xd, const float* gd, const float* act,
+                                  const int32_t* offsets, int32_t n_experts, int64_t n_rows,
+                                  int32_t d, int32_t h, const float* w1, const float* w2,
+                                  float* dxd, janus_ffn_mode mode, void* workspace,
+                                  size_t workspace_bytes, janus_stream_t stream);
+
+/* -------------------------------------------------------------------------
+ * Combine.  [Blueprint] section 3.2 (aggregation and output layer): the
+ * activated experts' outputs are summed with the gate weights.  Gather form
+ * of the weighted scatter-add (deterministic, no atomics):
+ *   y[i,:] = sum_{k = 0..K-1, ascending} w[i,k] * yd[slot_of[i*K+k], :]
+ * topk_weight == NULL means w = 1 (the VJP combine).
+ * in : yd [R,d], slot_of [R], topk_weight [N,K] or NULL;  out: y [N,d]
+ * ------------------------------------------------------------------------- */
+janus_status janus_combine(const float* yd, const int32_t* slot_of, const float* topk_weight,
+                           int64_t n_atoms, int32_t top_k, int32_t d, float* y,
+                           janus_stream_t stream);
+
+/* -------------------------------------------------------------------------
+ * Edge -> atom aggregation.  [Review] section 3.5 (CNIS kernels: neighbour
+ * aggregation with fused indexing, edge aggregation): edge messages are
+ * reduced into their receiver atoms.  Segment sum over a receiver-sorted CSR:
+ *   out[i,:] = sum_{e in [row_ptr[i], row_ptr[i+1])} msg[e,:]   (0 if empty)
+ * in : msg [Ed,d] float32 (Ed = row_ptr[N]), row_ptr [N+1] int64 (row_ptr[0]
+ *      = 0, non-decreasing);  out: out [N,d] float32
+ * ------------------------------------------------------------------------- */
+janus_status janus_edge_aggregate(const float* msg, const int64_t* row_ptr, int64_t n_atoms,
+                                  int32_t d, float* out, janus_stream_t stream);
+
+/* Host-side fault injection for tests: the next `n_calls` library calls that
+ * would launch work return JANUS_ERR_CUDA before launching anything. */
+void janus_debug_inject_launch_failures(int32_t n_calls);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JANUS_H_ */

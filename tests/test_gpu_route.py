@@ -1,0 +1,126 @@
+"""GPU parity: janus_route vs the oracle, bit-exact for indices/counts/offsets
+and the stable permutation (routing by element type: paper review 'Breaking
+the Training Barrier of Billion-Parameter Universal Machine Learning
+Interatomic Potentials', section 3.2)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from element_routed_moe_b200 import janus as J
+from element_routed_moe_b200 import synth
+from helpers import DEV, TOL_WEIGHT, host, poison_like, to_dev
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    # name: (N, T, E, K, dist)
+    "tiny": (512, 8, 8, 2, "uniform"),
+    "S": (8192, 89, 72, 4, "zipf"),
+    "M": (32768, 89, 40, 8, "zipf"),
+    "L": (16384, 89, 72, 16, "zipf"),
+    "slice": (65536, 89, 40, 8, "zipf"),
+    "K1": (3000, 89, 40, 1, "zipf"),
+    "K_eq_E": (2000, 13, 24, 24, "zipf"),
+    "single_type": (1500, 1, 16, 4, "zipf"),
+    "E256_K200": (700, 30, 256, 200, "uniform"),
+    "ragged_chunks": (64 * 7 + 13, 5, 9, 3, "uniform"),
+    "one_atom": (1, 3, 5, 2, "uniform"),
+    "large_N_multichunk": (300_000, 89, 40, 1, "zipf"),
+}
+
+
+def _inputs(N, T, E, K, dist, seed):
+    types = synth.types_uniform(N, T, seed) if dist == "uniform" else synth.types_zipf(N, T, seed=seed)
+    gate = synth.gate_table(T, E, seed + 1)
+    return types, gate
+
+
+def _gpu_route(types, gate, K):
+    N = types.shape[0]
+    T, E = gate.shape
+    R = N * K
+    out = dict(topk_expert=poison_like((N, K), torch.int32),
+               topk_weight=poison_like((N, K), torch.float32),
+               counts=poison_like((E,), torch.int32),
+               offsets=poison_like((E + 1,), torch.int32),
+               perm=poison_like((R,), torch.int32),
+               slot_of=poison_like((R,), torch.int32))
+    r = J.janus_route(to_dev(types), to_dev(gate), K, out=out)
+    J.janus_check(r["workspace"])
+    return {k: host(v) for k, v in r.items() if k != "workspace"}
+
+
+def _compare(g, o):
+    for k in ("topk_expert", "counts", "offsets", "perm", "slot_of"):
+        assert np.array_equal(g[k], o[k]), k
+    w_g, w_o = g["topk_weight"].astype(np.float64), o["topk_weight"].astype(np.float64)
+    assert np.all(np.abs(w_g - w_o) <= TOL_WEIGHT * np.abs(w_o))
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_route_parity(name):
+    N, T, E, K, dist = CASES[name]
+    types, gate = _inputs(N, T, E, K, dist, seed=10)
+    _compare(_gpu_route(types, gate, K), oracle.route(types, gate, K))
+
+
+@pytest.mark.parametrize("seed", [1, 2])
+def test_route_parity_more_seeds(seed):
+    N, T, E, K, dist = CASES["M"]
+    types, gate = _inputs(N, T, E, K, dist, seed=100 + seed)
+    _compare(_gpu_route(types, gate, K), oracle.route(types, gate, K))
+
+
+def test_route_ties_and_empty_experts():
+    gate = np.zeros((4, 12), np.float32)
+    gate[1, [3, 7, 9]] = 1.5               # ties at the top
+    gate[2, :] = -np.arange(12, dtype=np.float32)
+    gate[3, 5] = gate[3, 6] = 2.0
+    types = synth.types_uniform(5000, 4, 3)
+    for K in (1, 3, 5, 12):
+        _compare(_gpu_route(types, gate, K), oracle.route(types, gate, K))
+
+
+def test_route_zero_atoms():
+    gate = synth.gate_table(4, 6, 0)
+    r = J.janus_route(torch.empty(0, dtype=torch.int32, device=DEV), to_dev(gate), 2)
+    J.janus_check(r["workspace"])
+    assert np.all(host(r["counts"]) == 0) and np.all(host(r["offsets"]) == 0)
+
+
+def test_route_bad_type_sets_data_error():
+    gate = synth.gate_table(4, 6, 0)
+    types = np.array([0, 1, 7, 2, -3], np.int32)
+    r = J.janus_route(to_dev(types), to_dev(gate), 2)
+    with pytest.raises(J.JanusError) as e:
+        J.janus_check(r["workspace"])
+    assert e.value.status == J.JANUS_ERR_DATA
+    # outputs stay well-formed: bad ids are routed as type 0
+    fixed = np.where((types < 0) | (types >= 4), 0, types).astype(np.int32)
+    _compare({k: host(v) for k, v in r.items() if k != "workspace"}, oracle.route(fixed, gate, 2))
+    # the next good call clears the error word
+    r2 = J.janus_route(to_dev(fixed), to_dev(gate), 2, workspace=r["workspace"])
+    J.janus_check(r2["workspace"])
+
+
+def test_route_repeat_calls_reuse_workspace():
+    N, T, E, K, dist = CASES["S"]
+    types, gate = _inputs(N, T, E, K, dist, seed=5)
+    ref = oracle.route(types, gate, K)
+    ws = None
+    for _ in range(3):
+        r = J.janus_route(to_dev(types), to_dev(gate), K, workspace=ws)
+        ws = r["workspace"]
+        J.janus_check(ws)
+        _compare({k: host(v) for k, v in r.items() if k != "workspace"}, ref)
+
+
+def test_injected_failure_with_real_buffers():
+    types, gate = _inputs(100, 4, 6, 2, "uniform", 0)
+    J.janus_debug_inject_launch_failures(1)
+    with pytest.raises(J.JanusError) as e:
+        J.janus_route(to_dev(types), to_dev(gate), 2)
+    assert e.value.status == J.JANUS_ERR_CUDA
+    r = J.janus_route(to_dev(types), to_dev(gate), 2)
+    J.janus_check(r["workspace"])
