@@ -56,7 +56,19 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--atoms", type=int, default=None, help="override N (profiling small cases)")
+    ap.add_argument("--experts", type=int, default=None, help="override E (profiling small cases)")
     return ap.parse_args()
+
+
+def workload(args):
+    import dataclasses
+    cfg = synth.CONFIGS[args.workload]
+    if args.atoms:
+        cfg = dataclasses.replace(cfg, n_atoms=args.atoms)
+    if args.experts:
+        cfg = dataclasses.replace(cfg, n_experts=args.experts, top_k=min(cfg.top_k, args.experts))
+    return cfg
 
 
 # --------------------------------------------------------------------------
@@ -98,7 +110,7 @@ def describe(cfg) -> dict:
     w = {"tiny": "tiny layer", "S": "MatRIS-MoE(S)-shaped layer", "M": "MatRIS-MoE(M)-shaped layer",
          "L": "MatRIS-MoE(L)-shaped layer", "slice": "interaction-block slice at M shape"}[cfg.name]
     return {
-        "workload": f"{w}: N={cfg.n_atoms} atoms, T={cfg.n_types} element types "
+        "workload": f"{w}{'' if cfg == synth.CONFIGS[cfg.name] else ' (resized)'}: N={cfg.n_atoms} atoms, T={cfg.n_types} element types "
                     f"({'Zipf(1.1)' if cfg.type_dist == 'zipf' else 'uniform'}), E={cfg.n_experts}, "
                     f"K={cfg.top_k}, d=h={cfg.d}, FP32, fwd+input-VJP"
                     + (", edge aggregation + FP16 per-type packing" if cfg.name == "slice" else ""),
@@ -362,7 +374,7 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     import oracle
-    cfg = synth.CONFIGS[args.workload]
+    cfg = workload(args)
     inp = synth.layer_inputs(cfg, seed=args.seed, device="cpu", with_edges=False)
     host = dict(types=inp["types"], gate=inp["gate"], x=inp["x"].numpy(), g=inp["g"].numpy(),
                 w1=inp["w1"].numpy(), w2=inp["w2"].numpy())
@@ -395,7 +407,7 @@ def run_janus(args, world, rank, local):
     from element_routed_moe_b200 import janus as J
     J.lib()   # fails loudly if the CUDA library is missing
     dev = torch.device("cuda", local)
-    cfg = synth.CONFIGS[args.workload]
+    cfg = workload(args)
     mode = J.JANUS_FFN_3XTF32 if args.mode == "3xtf32" else J.JANUS_FFN_FP32_SIMT
     layer = Layer(cfg, mode, seed=args.seed + 1000 * rank, dev=dev)
     work = layer.work()
