@@ -48,10 +48,10 @@ FP32_LANES_PER_SM = 128
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="S", choices=list(synth.CONFIGS))
-    ap.add_argument("--mode", default="simt", choices=["simt", "3xtf32"])
+    ap.add_argument("--mode", default="3xtf32", choices=["simt", "3xtf32"])
     ap.add_argument("--impl", default="janus", choices=["janus", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

@@ -84,7 +84,9 @@ extern "C" janus_status janus_edge_aggregate(const float* msg, const int64_t* ro
   JANUS_CHECK_ARG(n_atoms >= 0 && d >= 1 && d <= kMaxDim);
   JANUS_CHECK_ALIGN(d % 4 == 0);
   if (n_atoms == 0) return JANUS_OK;
-  JANUS_CHECK_ARG(msg && row_ptr && out);
+  // msg may be NULL only for a CSR without edges: it is read at
+  // [row_ptr[i], row_ptr[i+1]) only.
+  JANUS_CHECK_ARG(row_ptr && out);
   JANUS_CHECK_ALIGN(aligned(msg, 16) && aligned(out, 16));
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
   const int64_t need = (n_atoms + 7) / 8;

@@ -94,8 +94,9 @@ extern "C" janus_status janus_expert_ffn_fwd(const float* xd, const int32_t* off
   float* H = (float*)((char*)workspace + L.off_h);
   const int64_t sw = (int64_t)d * h;
   if (mode == JANUS_FFN_3XTF32) {
+    JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
     st = tc::expert_ffn_fwd(xd, offsets, n_experts, n_rows, d, h, w1, w2, yd, act, H,
-                            (char*)workspace + L.total - tc::workspace_extra(), stream);
+                            &((WsHeader*)workspace)->error, stream);
     if (st != JANUS_OK) return st;
     return launch_status();
   }
@@ -126,8 +127,9 @@ extern "C" janus_status janus_expert_ffn_vjp(const float* xd, const float* gd, c
   float* A = act ? const_cast<float*>(act) : (float*)((char*)workspace + L.off_h + rh);
   const int64_t sw = (int64_t)d * h;
   if (mode == JANUS_FFN_3XTF32) {
+    JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
     st = tc::expert_ffn_vjp(xd, gd, act, A, offsets, n_experts, n_rows, d, h, w1, w2, dxd, dA,
-                            (char*)workspace + L.total - tc::workspace_extra(), stream);
+                            &((WsHeader*)workspace)->error, stream);
     if (st != JANUS_OK) return st;
     return launch_status();
   }

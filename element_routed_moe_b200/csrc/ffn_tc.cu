@@ -1,22 +1,553 @@
-// Tensor-core (tcgen05, 3xTF32) grouped expert MLP.  Not built yet: the
-// entry points report JANUS_ERR_INVALID_ARG for this mode.
+// Grouped expert-MLP GEMM on the 5th-generation tensor cores (tcgen05) with
+// the 3xTF32 split, for JANUS_FFN_3XTF32.
+//
+// FP32 accuracy from TF32 tensor cores (Ootomo & Yokota 2022, "Recovering
+// single precision accuracy from Tensor Cores while surpassing the FP32
+// theoretical peak performance"): every FP32 operand x is split into
+//   hi = x rounded to TF32 (10 fraction bits), lo = x - hi (exact in FP32),
+// and a*b is accumulated as a_lo*b_hi + a_hi*b_lo + a_hi*b_hi; the dropped
+// a_lo*b_lo term is below 2^-22 of the product.  The tensor core adds into its
+// FP32 accumulator with truncation, so a long reduction drifts (about 2e-5
+// relative at K = 2560 when accumulated in one pass).  As in the same paper,
+// accumulation is therefore split: each chunk of 4 k-blocks (K = 128) is
+// accumulated from zero in TMEM and then added, with round-to-nearest FP32
+// adds, into running sums held in the epilogue warps' registers.
+//
+//   C[p, :] = epilogue( A[p, :] * B_e )  for the rows p of expert e's segment
+//
+// Structure (one persistent CTA per SM, 16 warps = 4 warpgroups):
+//   warp 0       TMA producer: A tile 128x32 and B tile 256x32 (FP32, 128-byte
+//                swizzle; 32-byte swizzle atoms for an MN-major B) per k-block
+//                into a 2-stage ring;
+//   warp 1       TMEM allocator and MMA issuer: 3 products x 4 k-steps of
+//                tcgen05.mma.kind::tf32 (M=128, N=256, K=8) per k-block into
+//                one of two TMEM chunk buffers (2 x 256 columns);
+//   warps 2,3,12..15  splitters: rewrite each landed tile in place as hi and
+//                write lo into a twin buffer (same swizzled offsets);
+//   warps 4..11  epilogue (warpgroups 1 and 2, one 128-column half each):
+//                tcgen05.ld of each chunk (one TMEM lane quarter = 32 rows per
+//                warp), FP32 running sums in registers (setmaxnreg: 192 per
+//                thread here, 64 elsewhere), then fused SiLU / SiLU' / store.
+// Tiles come from a device-side list built from `offsets` (expert-major, then
+// 128-row block, then 256-column block), so the host never reads the routing.
+// Every mbarrier wait is bounded: on timeout the CTA records an error in the
+// workspace header, every role leaves its loop, issued MMAs and loads are
+// drained (bounded) and TMEM is freed.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "ffn_tc.cuh"
 
 namespace janus {
 namespace tc {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 32;
+constexpr int kStages = 2;
+constexpr int kThreads = 512;
+constexpr int kNumSplitWarps = 6;
+constexpr int kNumEpiWarps = 8;
+constexpr int kEpiCols = BN / 2;         // columns per epilogue thread
+constexpr int kChunkKb = 4;              // k-blocks accumulated per TMEM chunk
+constexpr int kEpiRegs = 192, kOtherRegs = 64;
+static_assert(2 * 128 * kEpiRegs + 2 * 128 * kOtherRegs == 65536, "register split must match the launch");
+constexpr uint32_t kTileABytes = BM * BK * 4;              // 16 KB
+constexpr uint32_t kTileBBytes = BN * BK * 4;              // 32 KB
+constexpr uint32_t kStageBytes = 2 * (kTileABytes + kTileBBytes);   // raw + lo
+constexpr uint32_t kTxBytes = kTileABytes + kTileBBytes;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kFaultTimeout = 3;
+constexpr long long kWaitLimitCycles = 4000000000LL;     // ~2 s at 2 GHz
+
+enum Epilogue : int { kEpiStore = 0, kEpiSilu = 1, kEpiDSilu = 2 };
+
+struct Args {
+  float* C;
+  float* C2;
+  const float* aux;
+  const int32_t* offsets;
+  int E, Kd, N;
+  int32_t* err;
+};
+
+struct Smem {
+  uint64_t full[kStages];     // TMA landed (tx count)
+  uint64_t split[kStages];    // hi/lo written (one arrive per splitter warp)
+  uint64_t empty[kStages];    // MMAs done reading the stage (tcgen05.commit)
+  uint64_t chunk_full[2];     // a k-chunk's partial product is in TMEM (tcgen05.commit)
+  uint64_t chunk_empty[2];    // the epilogue folded that chunk into its sums (8 warps)
+  uint64_t drain;             // final commit before TMEM is freed
+  uint32_t tmem_base;
+  int abort;
+  int off[kMaxExperts + 1];
+  int start[kMaxExperts + 1];
+};
+
+// ---- PTX wrappers ---------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false if the CTA aborted or the wait ran out (then aborts it).
+__device__ __forceinline__ bool mbar_wait(Smem* s, uint64_t* bar, uint32_t parity, int32_t* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*(volatile int*)&s->abort) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      *(volatile int*)&s->abort = 1;
+      atomicCAS(err, 0, kFaultTimeout);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* bar, void* dst, int c0, int c1,
+                                            int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05): start address, leading and
+// stride byte offsets (16-byte units), version 1, swizzle mode.
+// K-major operands use the 128-byte swizzle (mode 2; 16-byte granules XOR the
+// row mod 8).  An MN-major TF32 operand must use the 128-byte swizzle with
+// 32-byte atoms (mode 1; 32-byte granules XOR the row mod 4), which TMA writes
+// with CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B.
+constexpr uint32_t kSwizzle128B = 2, kSwizzle128B32B = 1;
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              uint32_t mode) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)mode << 61;
+  return d;
+}
+
+// Instruction descriptor: D=F32, A=B=TF32, A K-major, B K- or MN-major, M=128, N=256.
+__host__ __device__ constexpr uint32_t instr_desc(bool b_mn_major) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(BN >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + expf(-a)); }
+__device__ __forceinline__ float dsilu_f(float a) {
+  const float s = 1.0f / (1.0f + expf(-a));
+  return s * (1.0f + a * (1.0f - s));
+}
+
+// TF32 high part: round to nearest (ties away) to 10 fraction bits; values
+// whose rounding would overflow are truncated instead.
+__device__ __forceinline__ uint32_t tf32_hi_bits(uint32_t b) {
+  const uint32_t r = (b + 0x1000u) & 0xFFFFE000u;
+  return ((r & 0x7F800000u) == 0x7F800000u && (b & 0x7F800000u) != 0x7F800000u) ? (b & 0xFFFFE000u) : r;
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+struct TileCoord {
+  int e, m0, m_end, n0;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const Smem* s, int E, int n_tiles_n, int tile) {
+  const int mt = tile / n_tiles_n, nt = tile % n_tiles_n;
+  int lo = 0, hi = E;   // start[lo] <= mt < start[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s->start[mid] <= mt) lo = mid; else hi = mid;
+  }
+  TileCoord c;
+  c.e = lo;
+  c.m0 = s->off[lo] + (mt - s->start[lo]) * BM;
+  c.m_end = s->off[lo + 1];
+  c.n0 = nt * BN;
+  return c;
+}
+
+// Epilogue warpgroups: fold each TMEM chunk into FP32 running sums, then apply
+// the fused epilogue and store the tile.
+template <int kEpi>
+__device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_t tmem_base, int warp, int lane,
+                                              int n_tiles_n, int total, int nk) {
+  const int wg = warp / 4;
+  const int E = args.E, N = args.N;
+  const int q = warp % 4;                  // TMEM lane quarter = 32 rows
+  const int half = wg - 1;                // columns [128*half, 128*half + 128)
+  const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+  uint32_t ch = 0;
+  for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    const TileCoord c = decode_tile(s, E, n_tiles_n, tile);
+    float acc[kEpiCols];
+    bool ok = true;
+    for (int c0 = 0; c0 < nk; c0 += kChunkKb, ++ch) {
+      const uint32_t p = ch & 1, cuse = ch >> 1;
+      if (!mbar_wait(s, &s->chunk_full[p], cuse & 1, args.err)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + lane_addr + p * BN + half * kEpiCols;
+#pragma unroll
+      for (int j = 0; j < kEpiCols; j += 16) {
+        uint32_t r[16];
+        tmem_ld16(taddr + j, r);
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+          acc[j + t] = (c0 == 0) ? __uint_as_float(r[t]) : acc[j + t] + __uint_as_float(r[t]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s->chunk_empty[p]);
+    }
+    if (!ok) break;
+    const int row = c.m0 + q * 32 + lane;
+    const int colb = c.n0 + half * kEpiCols;
+    if (row < c.m_end && colb < N) {
+      const int64_t o = (int64_t)row * N + colb;
+#pragma unroll
+      for (int j = 0; j < kEpiCols; j += 4) {
+        if (colb + j < N) {
+          float4 v = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+          if (kEpi == kEpiSilu) {
+            if (args.C2) *reinterpret_cast<float4*>(args.C2 + o + j) = v;
+            v = make_float4(silu_f(v.x), silu_f(v.y), silu_f(v.z), silu_f(v.w));
+          } else if (kEpi == kEpiDSilu) {
+            const float4 a = __ldg(reinterpret_cast<const float4*>(args.aux + o + j));
+            v = make_float4(v.x * dsilu_f(a.x), v.y * dsilu_f(a.y), v.z * dsilu_f(a.z), v.w * dsilu_f(a.w));
+          }
+          *reinterpret_cast<float4*>(args.C + o + j) = v;
+        }
+      }
+    }
+  }
+}
+
+template <bool kNT, int kEpi>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, Args args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* tiles = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  Smem* s = (Smem*)(tiles + kStages * kStageBytes);
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int wg = warp / 4;
+  const int E = args.E, Kd = args.Kd, N = args.N;
+
+  for (int e = tid; e <= E; e += kThreads) s->off[e] = args.offsets[e];
+  if (tid == 0) {
+    s->abort = 0;
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&s->full[i], 1);
+      mbar_init(&s->split[i], kNumSplitWarps);
+      mbar_init(&s->empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s->chunk_full[i], 1);
+      mbar_init(&s->chunk_empty[i], kNumEpiWarps);
+    }
+    mbar_init(&s->drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s->tmem_base)),
+                 "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int e = 0; e < E; ++e) {
+      s->start[e] = acc;
+      acc += (s->off[e + 1] - s->off[e] + BM - 1) / BM;
+    }
+    s->start[E] = acc;
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = s->tmem_base;
+  const int n_tiles_n = (N + BN - 1) / BN;
+  const int total = s->start[E] * n_tiles_n;
+  const int nk = (Kd + BK - 1) / BK;
+
+  if (wg == 1 || wg == 2) {
+    // the epilogue warpgroups hold 128 FP32 running sums per thread
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
+    epilogue_role<kEpi>(s, args, tmem_base, warp, lane, n_tiles_n, total, nk);
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
+    if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileCoord c = decode_tile(s, E, n_tiles_n, tile);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t st = it % kStages, use = it / kStages;
+          if (!mbar_wait(s, &s->empty[st], (use & 1) ^ 1, args.err)) { ok = false; break; }
+          uint8_t* base = tiles + st * kStageBytes;
+          mbar_arrive_expect_tx(&s->full[st], kTxBytes);
+          tma_load_2d(&mapA, &s->full[st], base, kb * BK, c.m0);
+          if (kNT) {
+            tma_load_3d(&mapB, &s->full[st], base + kTileABytes, kb * BK, c.n0, c.e);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 32; ++j)
+              tma_load_3d(&mapB, &s->full[st], base + kTileABytes + j * (32 * BK * 4), c.n0 + 32 * j, kb * BK, c.e);
+          }
+        }
+      }
+      // the last issued loads must land before the CTA may exit
+      const uint32_t n_last = it < (uint32_t)kStages ? it : (uint32_t)kStages;
+      for (uint32_t j = 0; j < n_last; ++j) {
+        const uint32_t i2 = it - 1 - j, st = i2 % kStages, use = i2 / kStages;
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&s->full[st], use & 1) && clock64() - t0 < kWaitLimitCycles) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    // Each chunk of kChunkKb k-blocks is accumulated from zero into one of two
+    // TMEM buffers; the epilogue folds it into FP32 running sums.
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc(!kNT);
+      uint32_t it = 0, ch = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        for (int c0 = 0; c0 < nk && ok; c0 += kChunkKb, ++ch) {
+          const uint32_t p = ch & 1, cuse = ch >> 1;
+          if (!mbar_wait(s, &s->chunk_empty[p], (cuse & 1) ^ 1, args.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + p * BN;
+          const int c1 = min(c0 + kChunkKb, nk);
+          for (int kb = c0; kb < c1; ++kb, ++it) {
+            const uint32_t st = it % kStages, use = it / kStages;
+            if (!mbar_wait(s, &s->split[st], use & 1, args.err)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a_hi = smem_u32(tiles + st * kStageBytes);
+            const uint32_t b_hi = a_hi + kTileABytes;
+            const uint32_t a_lo = a_hi + kTxBytes, b_lo = b_hi + kTxBytes;
+#pragma unroll
+            for (int kk = 0; kk < BK / 8; ++kk) {
+              // K-major: 8 rows x 128 B per 1024-byte group (SBO), k-step = +32 B.
+              // MN-major B: 32-column chunks 32*BK*4 B apart (LBO), 4 k-rows per
+              // 512-byte group (SBO), k-step of 8 rows = +1024 B.
+              const uint64_t adh = smem_desc(a_hi + kk * 32, 16, 1024, kSwizzle128B);
+              const uint64_t adl = smem_desc(a_lo + kk * 32, 16, 1024, kSwizzle128B);
+              uint64_t bdh, bdl;
+              if (kNT) {
+                bdh = smem_desc(b_hi + kk * 32, 16, 1024, kSwizzle128B);
+                bdl = smem_desc(b_lo + kk * 32, 16, 1024, kSwizzle128B);
+              } else {
+                bdh = smem_desc(b_hi + kk * 1024, 32 * BK * 4, 512, kSwizzle128B32B);
+                bdl = smem_desc(b_lo + kk * 1024, 32 * BK * 4, 512, kSwizzle128B32B);
+              }
+              tc_mma_tf32(d_tmem, adl, bdh, idesc, (kb > c0 || kk > 0) ? 1u : 0u);
+              tc_mma_tf32(d_tmem, adh, bdl, idesc, 1u);
+              tc_mma_tf32(d_tmem, adh, bdh, idesc, 1u);
+            }
+            tc_commit(&s->empty[st]);
+          }
+          if (!ok) break;
+          tc_commit(&s->chunk_full[p]);
+        }
+      }
+      // every issued MMA completes before TMEM can be freed
+      tc_commit(&s->drain);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(&s->drain, 0) && clock64() - t0 < kWaitLimitCycles) {
+      }
+    }
+    } else {
+      // ---------------- splitters: x -> (hi in place, lo in the twin buffer) ----------------
+    const int ci = warp < 4 ? warp - 2 : warp - 10;
+    const int ct = ci * 32 + lane;
+    constexpr int kVec = (int)(kTxBytes / 16);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const uint32_t st = it % kStages, use = it / kStages;
+        if (!mbar_wait(s, &s->full[st], use & 1, args.err)) { ok = false; break; }
+        uint4* raw = reinterpret_cast<uint4*>(tiles + st * kStageBytes);
+        uint4* lo = reinterpret_cast<uint4*>(tiles + st * kStageBytes + kTxBytes);
+#pragma unroll 2
+        for (int i = ct; i < kVec; i += kNumSplitWarps * 32) {
+          const uint4 x = raw[i];
+          uint4 h, l;
+          h.x = tf32_hi_bits(x.x); h.y = tf32_hi_bits(x.y); h.z = tf32_hi_bits(x.z); h.w = tf32_hi_bits(x.w);
+          l.x = __float_as_uint(__uint_as_float(x.x) - __uint_as_float(h.x));
+          l.y = __float_as_uint(__uint_as_float(x.y) - __uint_as_float(h.y));
+          l.z = __float_as_uint(__uint_as_float(x.z) - __uint_as_float(h.z));
+          l.w = __float_as_uint(__uint_as_float(x.w) - __uint_as_float(h.w));
+          raw[i] = h;
+          lo[i] = l;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s->split[st]);
+      }
+    }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ---- host side -------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+  });
+  return fn;
+}
+
+// A: [R, Kd] row-major FP32, box 32 (k) x 128 (rows)
+bool map_a(CUtensorMap* m, const float* A, int64_t R, int Kd) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)Kd, (cuuint64_t)R};
+  cuuint64_t strides[1] = {(cuuint64_t)Kd * 4};
+  cuuint32_t box[2] = {BK, BM};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, (void*)A, dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// B for "x W": W [E, Kd, N] (N contiguous), box 32 (n) x 32 (k) x 1
+// B for "x W^T": W [E, N, Kd] (Kd contiguous), box 32 (k) x 256 (n) x 1
+bool map_b(CUtensorMap* m, const float* W, int E, int Kd, int N, bool nt) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3], es[3] = {1, 1, 1};
+  if (nt) {
+    dims[0] = Kd; dims[1] = N; dims[2] = E;
+    strides[0] = (cuuint64_t)Kd * 4; strides[1] = (cuuint64_t)Kd * N * 4;
+    box[0] = BK; box[1] = BN; box[2] = 1;
+  } else {
+    dims[0] = N; dims[1] = Kd; dims[2] = E;
+    strides[0] = (cuuint64_t)N * 4; strides[1] = (cuuint64_t)Kd * N * 4;
+    box[0] = 32; box[1] = BK; box[2] = 1;
+  }
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, (void*)W, dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE,
+             nt ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Smem);
+
+template <bool kNT, int kEpi>
+janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, int N, float* C, float* C2,
+                    const float* aux, const int32_t* offsets, int32_t* err, cudaStream_t stream) {
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [] {
+    attr = cudaFuncSetAttribute(tc_gemm_kernel<kNT, kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kSmemBytes);
+  });
+  if (attr != cudaSuccess) return JANUS_ERR_CUDA;
+  CUtensorMap ma, mb;
+  if (!map_a(&ma, A, R, Kd) || !map_b(&mb, W, E, Kd, N, kNT)) return JANUS_ERR_CUDA;
+  Args a;
+  a.C = C; a.C2 = C2; a.aux = aux; a.offsets = offsets; a.E = E; a.Kd = Kd; a.N = N; a.err = err;
+  tc_gemm_kernel<kNT, kEpi><<<num_sms(), kThreads, kSmemBytes, stream>>>(ma, mb, a);
+  return launch_status();
+}
+
+}  // namespace
 
 size_t workspace_extra() { return 0; }
 
-janus_status expert_ffn_fwd(const float*, const int32_t*, int32_t, int64_t, int32_t, int32_t,
-                            const float*, const float*, float*, float*, float*, void*,
-                            cudaStream_t) {
-  return JANUS_ERR_INVALID_ARG;
+janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, int64_t R, int32_t d,
+                            int32_t h, const float* w1, const float* w2, float* yd, float* act, float* H,
+                            int32_t* err, cudaStream_t stream) {
+  janus_status st = launch<false, kEpiSilu>(xd, w1, R, E, d, h, H, act, nullptr, offsets, err, stream);
+  if (st != JANUS_OK) return st;
+  return launch<false, kEpiStore>(H, w2, R, E, h, d, yd, nullptr, nullptr, offsets, err, stream);
 }
 
-janus_status expert_ffn_vjp(const float*, const float*, const float*, float*, const int32_t*,
-                            int32_t, int64_t, int32_t, int32_t, const float*, const float*,
-                            float*, float*, void*, cudaStream_t) {
-  return JANUS_ERR_INVALID_ARG;
+janus_status expert_ffn_vjp(const float* xd, const float* gd, const float* act_in, float* A,
+                            const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
+                            const float* w1, const float* w2, float* dxd, float* dA, int32_t* err,
+                            cudaStream_t stream) {
+  janus_status st;
+  if (!act_in) {
+    st = launch<false, kEpiStore>(xd, w1, R, E, d, h, A, nullptr, nullptr, offsets, err, stream);
+    if (st != JANUS_OK) return st;
+  }
+  st = launch<true, kEpiDSilu>(gd, w2, R, E, d, h, dA, nullptr, A, offsets, err, stream);
+  if (st != JANUS_OK) return st;
+  return launch<true, kEpiStore>(dA, w1, R, E, h, d, dxd, nullptr, nullptr, offsets, err, stream);
 }
 
 }  // namespace tc

@@ -10,13 +10,15 @@ namespace tc {
 // extra workspace bytes the tensor-core path needs beyond the activations
 size_t workspace_extra();
 
+// `err` is the workspace header's error word (a bounded wait that ran out
+// records a timeout there).
 janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, int64_t R,
                             int32_t d, int32_t h, const float* w1, const float* w2, float* yd,
-                            float* act, float* H, void* extra, cudaStream_t stream);
+                            float* act, float* H, int32_t* err, cudaStream_t stream);
 
 janus_status expert_ffn_vjp(const float* xd, const float* gd, const float* act_in, float* A,
                             const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
-                            const float* w1, const float* w2, float* dxd, float* dA, void* extra,
+                            const float* w1, const float* w2, float* dxd, float* dA, int32_t* err,
                             cudaStream_t stream);
 
 }  // namespace tc

@@ -196,8 +196,8 @@ janus_status janus_combine(const float* yd, const int32_t* slot_of, const float*
  * aggregation with fused indexing, edge aggregation): edge messages are
  * reduced into their receiver atoms.  Segment sum over a receiver-sorted CSR:
  *   out[i,:] = sum_{e in [row_ptr[i], row_ptr[i+1])} msg[e,:]   (0 if empty)
- * in : msg [Ed,d] float32 (Ed = row_ptr[N]), row_ptr [N+1] int64 (row_ptr[0]
- *      = 0, non-decreasing);  out: out [N,d] float32
+ * in : msg [Ed,d] float32 (Ed = row_ptr[N]; may be NULL only when Ed == 0),
+ *      row_ptr [N+1] int64 (row_ptr[0] = 0, non-decreasing);  out: out [N,d] float32
  * ------------------------------------------------------------------------- */
 janus_status janus_edge_aggregate(const float* msg, const int64_t* row_ptr, int64_t n_atoms,
                                   int32_t d, float* out, janus_stream_t stream);

@@ -54,7 +54,7 @@ def _oracle_chain(x, types, gate, T, K, w1, w2, g, quant):
     return dict(route=r, payload=p, scale=s, y=y, dx=dx)
 
 
-@pytest.mark.parametrize("mode", [J.JANUS_FFN_FP32_SIMT])
+@pytest.mark.parametrize("mode", [J.JANUS_FFN_FP32_SIMT, J.JANUS_FFN_3XTF32])
 def test_slice_chain_small(mode):
     N, T, E, K, d = 2048, 89, 40, 8, 256
     rp, _, _ = synth.edges_pbc(N, seed=1)
@@ -79,7 +79,7 @@ def test_slice_chain_small(mode):
     assert rel_fro(host(out["dx"]), f["dx"]) <= TOL_FP16_PATH
 
 
-@pytest.mark.parametrize("mode", [J.JANUS_FFN_FP32_SIMT])
+@pytest.mark.parametrize("mode", [J.JANUS_FFN_FP32_SIMT, J.JANUS_FFN_3XTF32])
 def test_slice_chain_full_size_sampled(mode):
     cfg = synth.CONFIGS["slice"]
     N, T, E, K, d = cfg.n_atoms, cfg.n_types, cfg.n_experts, cfg.top_k, cfg.d

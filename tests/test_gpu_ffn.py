@@ -13,7 +13,7 @@ from helpers import DEV, TOL_FP32, host, poison_like, rel_fro, sample_rows, to_d
 
 pytestmark = pytest.mark.gpu
 
-MODES = [J.JANUS_FFN_FP32_SIMT]
+MODES = [J.JANUS_FFN_FP32_SIMT, J.JANUS_FFN_3XTF32]
 
 
 def _offsets(counts):
