@@ -373,3 +373,84 @@ extern "C" janus_status janus_dequant_by_type(const uint16_t* payload, int64_t n
       (const uint2*)payload, R, d / 4, top_k, types, n_types, perm, scale, (float4*)xd);
   return launch_status();
 }
+
+// ---------------------------------------------------------------------------
+// janus_quant_by_type_noalloc: per-type FP16 packing for callers that cannot
+// allocate device memory.
+//
+// Some callers cannot call cudaMalloc (or any allocating routine) at the
+// point where they pack a dispatch buffer: code running under an allocator
+// that forbids allocation during a step, plug-ins handed fixed buffers by a
+// host framework, or host code that has already partitioned all device
+// memory.  This entry point needs nothing from them beyond the inputs and
+// outputs: its scratch (the error word and one absmax word per element type)
+// is a file-scope device array owned by this library, 256 + 4 * 4096 =
+// 16,640 bytes, which every GPU that loads the library keeps until the
+// process exits.
+// ---------------------------------------------------------------------------
+#include <mutex>
+#include <unordered_map>
+
+constexpr int kNoAllocMaxTypes = 4096;
+constexpr size_t kNoAllocScratchBytes = sizeof(janus::WsHeader) + sizeof(uint32_t) * kNoAllocMaxTypes;
+
+// The scratch itself.  Host code must not use this name as an address (on the
+// host it is only a stand-in); the address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_quant_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+std::unordered_map<int, void*> g_noalloc_addr;   // device ordinal -> scratch address
+
+// Device address of the scratch on the current device, looked up once per
+// device (cudaGetSymbolAddress may load the module on that device).
+janus_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return JANUS_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  auto it = g_noalloc_addr.find(dev);
+  if (it != g_noalloc_addr.end()) {
+    *out = it->second;
+    return JANUS_OK;
+  }
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_quant_noalloc_scratch) != cudaSuccess || p == nullptr)
+    return JANUS_ERR_CUDA;
+  g_noalloc_addr[dev] = p;
+  *out = p;
+  return JANUS_OK;
+}
+
+}  // namespace
+
+extern "C" janus_status janus_quant_by_type_noalloc(const float* x, int64_t n_atoms, int32_t d,
+                                                    int32_t top_k, const int32_t* types,
+                                                    int32_t n_types, const int32_t* slot_of,
+                                                    uint16_t* payload, float* scale,
+                                                    janus_stream_t stream_) {
+  cudaStream_t stream = (cudaStream_t)stream_;
+  janus_status st = check_rows(n_atoms, d, top_k);
+  if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(n_types >= 1 && n_types <= kNoAllocMaxTypes);
+  JANUS_CHECK_ARG(scale != nullptr);
+  JANUS_CHECK_ARG(n_atoms == 0 || (x && types && slot_of && payload));
+  JANUS_CHECK_ALIGN(n_atoms == 0 || (aligned(x, 16) && aligned(payload, 8)));
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != JANUS_OK) return st;
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  WsHeader* hdr = (WsHeader*)scratch;
+  uint32_t* amax_bits = (uint32_t*)((char*)scratch + sizeof(WsHeader));
+  // the previous call's absmax words are still there: clear what this call uses
+  JANUS_CUDA_TRY(cudaMemsetAsync(scratch, 0, sizeof(WsHeader) + sizeof(uint32_t) * (size_t)n_types, stream));
+  const size_t smem = sizeof(uint32_t) * (size_t)n_types;
+  const unsigned grid = rows_grid(n_atoms, 8);
+  if (n_atoms > 0)
+    quant_amax_kernel<<<grid, kThreads, smem, stream>>>((const float4*)x, n_atoms, d / 4, types, n_types,
+                                                        amax_bits, hdr);
+  quant_pack_kernel<<<grid, kThreads, smem, stream>>>((const float4*)x, n_atoms, d / 4, top_k, types,
+                                                      n_types, slot_of, amax_bits, (uint2*)payload, scale,
+                                                      hdr);
+  return launch_status();
+}

@@ -31,7 +31,8 @@ SYMBOLS = (
     "janus_status_string", "janus_version", "janus_check",
     "janus_route_workspace_size", "janus_route",
     "janus_dispatch",
-    "janus_quant_by_type_workspace_size", "janus_quant_by_type", "janus_dequant_by_type",
+    "janus_quant_by_type_workspace_size", "janus_quant_by_type", "janus_quant_by_type_noalloc",
+    "janus_dequant_by_type",
     "janus_expert_ffn_workspace_size", "janus_expert_ffn_fwd", "janus_expert_ffn_vjp",
     "janus_combine", "janus_edge_aggregate",
     "janus_debug_inject_launch_failures",
@@ -72,6 +73,7 @@ def _declare(L):
         "janus_dispatch": (st, [vp, i64, i32, i32, vp, vp, vp, vp]),
         "janus_quant_by_type_workspace_size": (st, [i32, psz]),
         "janus_quant_by_type": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp, sz, vp]),
+        "janus_quant_by_type_noalloc": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp]),
         "janus_dequant_by_type": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp]),
         "janus_expert_ffn_workspace_size": (st, [i64, i32, i32, i32, i32, i32, ctypes.c_int, psz]),
         "janus_expert_ffn_fwd": (st, [vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, ctypes.c_int,
@@ -226,6 +228,28 @@ def janus_quant_by_type(x, types, n_types, slot_of, top_k, *, payload=None, scal
                                      _p(scale, torch.float32, "scale"), _p(ws), nb,
                                      _stream(stream)), "janus_quant_by_type")
     return payload, scale, ws
+
+
+def janus_quant_by_type_noalloc(x, types, n_types, slot_of, top_k, *, payload=None, scale=None,
+                                stream=None):
+    """janus_quant_by_type without a workspace, for callers that cannot
+    allocate device memory where they pack.  The library keeps its own
+    16,640-byte scratch per GPU; calls that overlap on the GPU race.
+    payload/scale are allocated here only when not given (pass them to keep
+    the call allocation-free).  Returns (payload, scale)."""
+    N, d = x.shape
+    K = int(top_k)
+    if payload is None:
+        payload = _empty((N * K, d), torch.float16, x.device)
+    if scale is None:
+        scale = _empty((n_types,), torch.float32, x.device)
+    _raise(lib().janus_quant_by_type_noalloc(_p(x, torch.float32, "x"), N, d, K,
+                                             _p(types, torch.int32, "types"), int(n_types),
+                                             _p(slot_of, torch.int32, "slot_of"),
+                                             _p(payload, None, "payload"),
+                                             _p(scale, torch.float32, "scale"), _stream(stream)),
+           "janus_quant_by_type_noalloc")
+    return payload, scale
 
 
 def janus_dequant_by_type(payload, types, n_types, perm, top_k, scale, *, out=None, stream=None):

@@ -135,6 +135,30 @@ janus_status janus_quant_by_type(const float* x, int64_t n_atoms, int32_t d, int
                                  void* workspace, size_t workspace_bytes,
                                  janus_stream_t stream);
 
+/* Same packing as janus_quant_by_type, for callers that cannot allocate
+ * device memory (no workspace argument).  The paper has no counterpart: this
+ * is a library convenience.  It is meant for code that must not call
+ * cudaMalloc or any allocating routine where it packs (for example inside a
+ * step run under an allocator that forbids allocation, or a plug-in that is
+ * handed fixed buffers); the caller still provides x, types, slot_of, payload
+ * and scale.  Scratch lives in a library-owned device array of 16,640 bytes
+ * (a 256-byte header plus one 32-bit word per element type), which every GPU
+ * that loads the library keeps until the process exits.
+ *   - n_types must be <= 4096; larger values return JANUS_ERR_INVALID_ARG.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, once per device, with that device current); make
+ *     that first call before any stream capture.
+ *   - Every call clears and reuses the same array, so calls whose work
+ *     overlaps on the GPU (different streams, or different host threads on one
+ *     device) race and may produce wrong scales; serialise them.
+ *   - Data faults are not reported (there is no workspace to hand to
+ *     janus_check); bad type ids are packed as type 0.
+ * Calls no cudaMalloc/cudaFree and no allocating library routine. */
+janus_status janus_quant_by_type_noalloc(const float* x, int64_t n_atoms, int32_t d, int32_t top_k,
+                                         const int32_t* types, int32_t n_types,
+                                         const int32_t* slot_of, uint16_t* payload, float* scale,
+                                         janus_stream_t stream);
+
 /* Dequantisation of a packed dispatch buffer (same passage):
  *   xd[p, j] = float(payload[p, j]) * scale[types[perm[p] / K]]   (exact)
  * in : payload [R,d] binary16 bits, types [N], perm [R], scale [T]
