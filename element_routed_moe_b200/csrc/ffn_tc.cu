@@ -4,30 +4,31 @@
 // FP32 accuracy from TF32 tensor cores (Ootomo & Yokota 2022, "Recovering
 // single precision accuracy from Tensor Cores while surpassing the FP32
 // theoretical peak performance"): every FP32 operand x is split into
-//   hi = x rounded to TF32 (10 fraction bits), lo = x - hi (exact in FP32),
+//   hi = x truncated to TF32 (10 fraction bits), lo = x - hi (exact in FP32),
 // and a*b is accumulated as a_lo*b_hi + a_hi*b_lo + a_hi*b_hi; the dropped
-// a_lo*b_lo term is below 2^-22 of the product.  The tensor core adds into its
+// a_lo*b_lo term is below 2^-20 of the product.  The tensor core adds into its
 // FP32 accumulator with truncation, so a long reduction drifts (about 2e-5
 // relative at K = 2560 when accumulated in one pass).  As in the same paper,
-// accumulation is therefore split: each chunk of 4 k-blocks (K = 128) is
+// accumulation is therefore split: each chunk of 8 k-blocks (K = 128) is
 // accumulated from zero in TMEM and then added, with round-to-nearest FP32
 // adds, into running sums held in the epilogue warps' registers.
 //
 //   C[p, :] = epilogue( A[p, :] * B_e )  for the rows p of expert e's segment
 //
 // Structure (one persistent CTA per SM, 16 warps = 4 warpgroups):
-//   warp 0       TMA producer: A tile 128x32 and B tile 256x32 (FP32, 128-byte
-//                swizzle; 32-byte swizzle atoms for an MN-major B) per k-block
-//                into a 2-stage ring;
-//   warp 1       TMEM allocator and MMA issuer: 3 products x 4 k-steps of
+//   warp 0       TMA producer: A tile 128x16 and B tile 256x16 (FP32, 64-byte
+//                swizzle; 128-byte swizzle with 32-byte atoms for an MN-major
+//                B) per k-block into a 4-stage ring (48 KB per stage: raw + lo);
+//   warp 1       TMEM allocator and MMA issuer: 3 products x 2 k-steps of
 //                tcgen05.mma.kind::tf32 (M=128, N=256, K=8) per k-block into
 //                one of two TMEM chunk buffers (2 x 256 columns);
-//   warps 2,3,12..15  splitters: rewrite each landed tile in place as hi and
-//                write lo into a twin buffer (same swizzled offsets);
+//   warps 2,3,12..15  splitters: write each landed tile's residual lo = x - hi
+//                into a twin buffer (same swizzled offsets; the landed FP32
+//                tile is read by the MMA as hi);
 //   warps 4..11  epilogue (warpgroups 1 and 2, one 128-column half each):
 //                tcgen05.ld of each chunk (one TMEM lane quarter = 32 rows per
-//                warp), FP32 running sums in registers (setmaxnreg: 192 per
-//                thread here, 64 elsewhere), then fused SiLU / SiLU' / store.
+//                warp), FP32 running sums in registers (setmaxnreg: 184 per
+//                thread here, 72 elsewhere), then fused SiLU / SiLU' / store.
 // Tiles come from a device-side list built from `offsets` (expert-major, then
 // 128-row block, then 256-column block), so the host never reads the routing.
 // Every mbarrier wait is bounded: on timeout the CTA records an error in the
@@ -44,17 +45,17 @@ namespace janus {
 namespace tc {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 32;
-constexpr int kStages = 2;
+constexpr int BM = 128, BN = 256, BK = 16;
+constexpr int kStages = 4;
 constexpr int kThreads = 512;
 constexpr int kNumSplitWarps = 6;
 constexpr int kNumEpiWarps = 8;
 constexpr int kEpiCols = BN / 2;         // columns per epilogue thread
-constexpr int kChunkKb = 4;              // k-blocks accumulated per TMEM chunk
-constexpr int kEpiRegs = 192, kOtherRegs = 64;
+constexpr int kChunkKb = 128 / BK;       // k-blocks accumulated per TMEM chunk (K = 128)
+constexpr int kEpiRegs = 184, kOtherRegs = 72;
 static_assert(2 * 128 * kEpiRegs + 2 * 128 * kOtherRegs == 65536, "register split must match the launch");
-constexpr uint32_t kTileABytes = BM * BK * 4;              // 16 KB
-constexpr uint32_t kTileBBytes = BN * BK * 4;              // 32 KB
+constexpr uint32_t kTileABytes = BM * BK * 4;              // 8 KB
+constexpr uint32_t kTileBBytes = BN * BK * 4;              // 16 KB
 constexpr uint32_t kStageBytes = 2 * (kTileABytes + kTileBBytes);   // raw + lo
 constexpr uint32_t kTxBytes = kTileABytes + kTileBBytes;
 constexpr uint32_t kTmemCols = 512;
@@ -159,7 +160,7 @@ __device__ __forceinline__ void tc_mma_tf32(uint32_t d_tmem, uint64_t adesc, uin
 // row mod 8).  An MN-major TF32 operand must use the 128-byte swizzle with
 // 32-byte atoms (mode 1; 32-byte granules XOR the row mod 4), which TMA writes
 // with CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B.
-constexpr uint32_t kSwizzle128B = 2, kSwizzle128B32B = 1;
+constexpr uint32_t kSwizzle64B = 4, kSwizzle128B32B = 1;
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
                                               uint32_t mode) {
   uint64_t d = 0;
@@ -183,12 +184,13 @@ __device__ __forceinline__ float dsilu_f(float a) {
   return s * (1.0f + a * (1.0f - s));
 }
 
-// TF32 high part: round to nearest (ties away) to 10 fraction bits; values
-// whose rounding would overflow are truncated instead.
-__device__ __forceinline__ uint32_t tf32_hi_bits(uint32_t b) {
-  const uint32_t r = (b + 0x1000u) & 0xFFFFE000u;
-  return ((r & 0x7F800000u) == 0x7F800000u && (b & 0x7F800000u) != 0x7F800000u) ? (b & 0xFFFFE000u) : r;
-}
+// TF32 high part: the FP32 value with its 13 low fraction bits cleared (exact
+// for every input, no overflow); the residual x - hi is exact in FP32.
+// tcgen05.mma.kind::tf32 reads a 32-bit operand by ignoring those same 13
+// bits (checked on B200: results are bit-identical to feeding it the cleared
+// value), so the landed FP32 tile serves as the high part unchanged and only
+// the residual tile is written.
+constexpr uint32_t kTf32Mask = 0xFFFFE000u;
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -384,15 +386,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
             const uint32_t a_lo = a_hi + kTxBytes, b_lo = b_hi + kTxBytes;
 #pragma unroll
             for (int kk = 0; kk < BK / 8; ++kk) {
-              // K-major: 8 rows x 128 B per 1024-byte group (SBO), k-step = +32 B.
+              // K-major: 8 rows x 64 B per 512-byte group (SBO), k-step = +32 B.
               // MN-major B: 32-column chunks 32*BK*4 B apart (LBO), 4 k-rows per
               // 512-byte group (SBO), k-step of 8 rows = +1024 B.
-              const uint64_t adh = smem_desc(a_hi + kk * 32, 16, 1024, kSwizzle128B);
-              const uint64_t adl = smem_desc(a_lo + kk * 32, 16, 1024, kSwizzle128B);
+              const uint64_t adh = smem_desc(a_hi + kk * 32, 16, 512, kSwizzle64B);
+              const uint64_t adl = smem_desc(a_lo + kk * 32, 16, 512, kSwizzle64B);
               uint64_t bdh, bdl;
               if (kNT) {
-                bdh = smem_desc(b_hi + kk * 32, 16, 1024, kSwizzle128B);
-                bdl = smem_desc(b_lo + kk * 32, 16, 1024, kSwizzle128B);
+                bdh = smem_desc(b_hi + kk * 32, 16, 512, kSwizzle64B);
+                bdl = smem_desc(b_lo + kk * 32, 16, 512, kSwizzle64B);
               } else {
                 bdh = smem_desc(b_hi + kk * 1024, 32 * BK * 4, 512, kSwizzle128B32B);
                 bdl = smem_desc(b_lo + kk * 1024, 32 * BK * 4, 512, kSwizzle128B32B);
@@ -414,10 +416,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       }
     }
     } else {
-      // ---------------- splitters: x -> (hi in place, lo in the twin buffer) ----------------
+      // ---------------- splitters: x -> lo = x - hi in the twin buffer ----------------
     const int ci = warp < 4 ? warp - 2 : warp - 10;
     const int ct = ci * 32 + lane;
-    constexpr int kVec = (int)(kTxBytes / 16);
+    constexpr int kSplitPer = (int)(kTxBytes / 16) / (kNumSplitWarps * 32);
+    static_assert(kSplitPer * kNumSplitWarps * 32 * 16 == (int)kTxBytes, "split work divides evenly");
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
@@ -426,17 +429,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         if (!mbar_wait(s, &s->full[st], use & 1, args.err)) { ok = false; break; }
         uint4* raw = reinterpret_cast<uint4*>(tiles + st * kStageBytes);
         uint4* lo = reinterpret_cast<uint4*>(tiles + st * kStageBytes + kTxBytes);
-#pragma unroll 2
-        for (int i = ct; i < kVec; i += kNumSplitWarps * 32) {
-          const uint4 x = raw[i];
-          uint4 h, l;
-          h.x = tf32_hi_bits(x.x); h.y = tf32_hi_bits(x.y); h.z = tf32_hi_bits(x.z); h.w = tf32_hi_bits(x.w);
-          l.x = __float_as_uint(__uint_as_float(x.x) - __uint_as_float(h.x));
-          l.y = __float_as_uint(__uint_as_float(x.y) - __uint_as_float(h.y));
-          l.z = __float_as_uint(__uint_as_float(x.z) - __uint_as_float(h.z));
-          l.w = __float_as_uint(__uint_as_float(x.w) - __uint_as_float(h.w));
-          raw[i] = h;
-          lo[i] = l;
+        // all of this thread's 16-byte words are loaded first, then split; the
+        // raw tile itself is the high part (the MMA ignores the 13 low bits)
+        uint4 x[kSplitPer];
+#pragma unroll
+        for (int j = 0; j < kSplitPer; ++j) x[j] = raw[ct + j * kNumSplitWarps * 32];
+#pragma unroll
+        for (int j = 0; j < kSplitPer; ++j) {
+          const uint4 l = make_uint4(
+              __float_as_uint(__uint_as_float(x[j].x) - __uint_as_float(x[j].x & kTf32Mask)),
+              __float_as_uint(__uint_as_float(x[j].y) - __uint_as_float(x[j].y & kTf32Mask)),
+              __float_as_uint(__uint_as_float(x[j].z) - __uint_as_float(x[j].z & kTf32Mask)),
+              __float_as_uint(__uint_as_float(x[j].w) - __uint_as_float(x[j].w & kTf32Mask)));
+          lo[ct + j * kNumSplitWarps * 32] = l;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
@@ -469,7 +474,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// A: [R, Kd] row-major FP32, box 32 (k) x 128 (rows)
+// A: [R, Kd] row-major FP32, box 16 (k) x 128 (rows), 64-byte swizzle
 bool map_a(CUtensorMap* m, const float* A, int64_t R, int Kd) {
   auto enc = encode_fn();
   if (!enc) return false;
@@ -478,12 +483,13 @@ bool map_a(CUtensorMap* m, const float* A, int64_t R, int Kd) {
   cuuint32_t box[2] = {BK, BM};
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, (void*)A, dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// B for "x W": W [E, Kd, N] (N contiguous), box 32 (n) x 32 (k) x 1
-// B for "x W^T": W [E, N, Kd] (Kd contiguous), box 32 (k) x 256 (n) x 1
+// B for "x W": W [E, Kd, N] (N contiguous), box 32 (n) x 16 (k) x 1, 128-byte
+//   swizzle with 32-byte atoms (MN-major)
+// B for "x W^T": W [E, N, Kd] (Kd contiguous), box 16 (k) x 256 (n) x 1, 64-byte swizzle
 bool map_b(CUtensorMap* m, const float* W, int E, int Kd, int N, bool nt) {
   auto enc = encode_fn();
   if (!enc) return false;
@@ -500,7 +506,7 @@ bool map_b(CUtensorMap* m, const float* W, int E, int Kd, int N, bool nt) {
   }
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, (void*)W, dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE,
-             nt ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B,
+             nt ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
