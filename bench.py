@@ -177,6 +177,24 @@ class ClockSampler:
                 "power_w_max": max(pw) if pw else None, "reasons": reasons}
 
 
+# DRAM bytes per launch of the expert-MLP GEMM, from one ncu capture of the
+# S-shaped layer (profiles/expert_ffn_tc_gemm.md), valid only for the kernel
+# source it was taken on.
+GEMM_TRAFFIC = {("S", "3xtf32"): {"src": "element_routed_moe_b200/csrc/ffn_tc.cu",
+                                  "sha256_prefix": "93a3d1e8f6bbcfc0", "bytes_per_launch": 3.106e9}}
+
+
+def measured_traffic(workload: str, mode: str):
+    import hashlib
+    rec = GEMM_TRAFFIC.get((workload, mode))
+    if rec is None:
+        return None
+    with open(os.path.join(ROOT, rec["src"]), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != rec["sha256_prefix"]:
+            return None
+    return rec["bytes_per_launch"]
+
+
 def measured_peaks() -> tuple[dict, str]:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -463,7 +481,9 @@ def run_janus(args, world, rank, local):
         peak = peaks["bf16_tflops_sustained"] * (1.125 / 2.25) / 3.0
         roof = {"bound": "tensor", "peak_source": f"{peak_src} sustained bf16 x (TF32/BF16 nominal 1.125/2.25) / 3 products"}
     roof.update({"kernel": "grouped expert-MLP GEMM", "achieved": achieved, "peak": peak,
-                 "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                 "unit": "TFLOP/s", "frac": achieved / peak,
+                 "traffic": (measured_traffic(cfg.name, args.mode)
+                             if cfg == synth.CONFIGS[cfg.name] else None),
                  "algorithmic_flops_per_launch": ffn_flops / 4, "launches_per_step": 4})
 
     line = {
