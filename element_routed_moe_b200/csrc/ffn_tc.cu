@@ -15,16 +15,24 @@
 //
 //   C[p, :] = epilogue( A[p, :] * B_e )  for the rows p of expert e's segment
 //
-// Structure (one persistent CTA per SM, 16 warps = 4 warpgroups):
-//   warp 0       TMA producer: A tile 128x16 and B tile 256x16 (FP32, 64-byte
-//                swizzle; 128-byte swizzle with 32-byte atoms for an MN-major
-//                B) per k-block into a 4-stage ring (48 KB per stage: raw + lo);
-//   warp 1       TMEM allocator and MMA issuer: 3 products x 2 k-steps of
-//                tcgen05.mma.kind::tf32 (M=128, N=256, K=8) per k-block into
-//                one of two TMEM chunk buffers (2 x 256 columns);
-//   warps 2,3,12..15  splitters: write each landed tile's residual lo = x - hi
-//                into a twin buffer (same swizzled offsets; the landed FP32
-//                tile is read by the MMA as hi);
+// Structure: one persistent CTA per SM, clusters of two CTAs that share one
+// M=256 x N=256 output tile through tcgen05 cta_group::2 MMAs (each CTA holds
+// its 128 rows of A, 128 of the 256 B columns and its 128 accumulator rows,
+// so shared-memory traffic per CTA is a third lower than with 1-CTA MMAs).
+// 16 warps = 4 warpgroups per CTA:
+//   warp 0       TMA producer: this CTA's A tile 128x16 and B half 128x16
+//                (FP32, 64-byte swizzle; 128-byte swizzle with 32-byte atoms
+//                for an MN-major B) per k-block into a 6-stage ring (32 KB per
+//                stage: raw + lo);
+//   warp 1       TMEM allocator (paired) and, in the leader CTA, the MMA
+//                issuer: 3 products x 2 k-steps of tcgen05.mma.cta_group::2
+//                .kind::tf32 (M=256, N=256, K=8) per k-block into one of two
+//                TMEM chunk buffers (2 x 256 columns), commits signalling
+//                both CTAs; peers' splitters and epilogues arrive on the
+//                leader's barriers;
+//   warps 2,3,12..15  splitters, each owning every sixth k-block: write the
+//                landed tile's residual lo = x - hi into a twin buffer (same
+//                swizzled offsets; the landed FP32 tile is read by the MMA as hi);
 //   warps 4..11  epilogue (warpgroups 1 and 2, one 128-column half each):
 //                tcgen05.ld of each chunk (one TMEM lane quarter = 32 rows per
 //                warp), FP32 running sums in registers (setmaxnreg: 184 per
@@ -45,8 +53,12 @@ namespace janus {
 namespace tc {
 namespace {
 
+// A CTA pair (cluster of 2) computes a 256 x 256 output tile with M = 256
+// MMAs (tcgen05 cta_group::2): each CTA holds its own 128 rows of A, half of
+// the 256 B columns, and its 128 rows of the accumulator in its own TMEM.
 constexpr int BM = 128, BN = 256, BK = 16;
-constexpr int kStages = 4;
+constexpr int BNH = BN / 2;               // B columns held by one CTA
+constexpr int kStages = 6;
 constexpr int kThreads = 512;
 constexpr int kNumSplitWarps = 6;
 constexpr int kNumEpiWarps = 8;
@@ -55,7 +67,7 @@ constexpr int kChunkKb = 128 / BK;       // k-blocks accumulated per TMEM chunk 
 constexpr int kEpiRegs = 184, kOtherRegs = 72;
 static_assert(2 * 128 * kEpiRegs + 2 * 128 * kOtherRegs == 65536, "register split must match the launch");
 constexpr uint32_t kTileABytes = BM * BK * 4;              // 8 KB
-constexpr uint32_t kTileBBytes = BN * BK * 4;              // 16 KB
+constexpr uint32_t kTileBBytes = BNH * BK * 4;             // 8 KB (this CTA's half)
 constexpr uint32_t kStageBytes = 2 * (kTileABytes + kTileBBytes);   // raw + lo
 constexpr uint32_t kTxBytes = kTileABytes + kTileBBytes;
 constexpr uint32_t kTmemCols = 512;
@@ -74,12 +86,12 @@ struct Args {
 };
 
 struct Smem {
-  uint64_t full[kStages];     // TMA landed (tx count)
-  uint64_t split[kStages];    // hi/lo written (one arrive per splitter warp)
-  uint64_t empty[kStages];    // MMAs done reading the stage (tcgen05.commit)
-  uint64_t chunk_full[2];     // a k-chunk's partial product is in TMEM (tcgen05.commit)
-  uint64_t chunk_empty[2];    // the epilogue folded that chunk into its sums (8 warps)
-  uint64_t drain;             // final commit before TMEM is freed
+  uint64_t full[kStages];     // this CTA's TMA landed (tx count)
+  uint64_t split[kStages];    // leader: residuals written in both CTAs (1 warp x 2)
+  uint64_t empty[kStages];    // MMAs done reading the stage (commit to both CTAs)
+  uint64_t chunk_full[2];     // a k-chunk's partial product is in TMEM (commit to both)
+  uint64_t chunk_empty[2];    // leader: both epilogues folded that chunk (8 warps x 2)
+  uint64_t drain;             // final commit (both CTAs) before TMEM is freed
   uint32_t tmem_base;
   int abort;
   int off[kMaxExperts + 1];
@@ -92,9 +104,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 }
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
@@ -138,18 +147,43 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* ba
       ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on the barrier at the same shared-memory offset in the leader CTA of
+// the pair: a plain local arrive in the leader itself, a remote arrive (default
+// release semantics) from the peer.  The data behind these arrivals is read
+// by the arriving CTA's own tensor core, so a cluster-scope release (about a
+// thousand cycles per arrive on B200) is not needed.
+__device__ __forceinline__ void mbar_arrive_leader(uint64_t* bar, uint32_t rank) {
+  if (rank == 0) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+  } else {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(bar)), "r"(0));
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+  }
+}
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
+// completion of the pair's MMAs arrives on the barrier at this offset in both CTAs
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+      ::"r"(smem_u32(bar)), "h"((uint16_t)0x3)
+      : "memory");
 }
-__device__ __forceinline__ void tc_mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                            uint32_t accumulate) {
+__device__ __forceinline__ void tc_mma_tf32_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n"
+      "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n"
       ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -172,10 +206,11 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
-// Instruction descriptor: D=F32, A=B=TF32, A K-major, B K- or MN-major, M=128, N=256.
+// Instruction descriptor: D=F32, A=B=TF32, A K-major, B K- or MN-major,
+// M=256 (the CTA pair), N=256.
 __host__ __device__ constexpr uint32_t instr_desc(bool b_mn_major) {
   return (1u << 4) | (2u << 7) | (2u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(BN >> 3) << 17) |
-         ((uint32_t)(BM >> 4) << 24);
+         ((uint32_t)((2 * BM) >> 4) << 24);
 }
 
 __device__ __forceinline__ float silu_f(float a) { return a / (1.0f + expf(-a)); }
@@ -207,7 +242,9 @@ struct TileCoord {
   int e, m0, m_end, n0;
 };
 
-__device__ __forceinline__ TileCoord decode_tile(const Smem* s, int E, int n_tiles_n, int tile) {
+// Pair tile `tile` -> expert, this CTA's 128-row block and the 256-column block.
+// start[e] counts 256-row blocks (one per CTA pair).
+__device__ __forceinline__ TileCoord decode_tile(const Smem* s, int E, int n_tiles_n, int tile, uint32_t rank) {
   const int mt = tile / n_tiles_n, nt = tile % n_tiles_n;
   int lo = 0, hi = E;   // start[lo] <= mt < start[hi]
   while (hi - lo > 1) {
@@ -216,25 +253,25 @@ __device__ __forceinline__ TileCoord decode_tile(const Smem* s, int E, int n_til
   }
   TileCoord c;
   c.e = lo;
-  c.m0 = s->off[lo] + (mt - s->start[lo]) * BM;
+  c.m0 = s->off[lo] + ((mt - s->start[lo]) * 2 + (int)rank) * BM;
   c.m_end = s->off[lo + 1];
   c.n0 = nt * BN;
   return c;
 }
 
 // Epilogue warpgroups: fold each TMEM chunk into FP32 running sums, then apply
-// the fused epilogue and store the tile.
+// the fused epilogue and store this CTA's 128 x 256 part of the tile.
 template <int kEpi>
 __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_t tmem_base, int warp, int lane,
-                                              int n_tiles_n, int total, int nk) {
+                                              int n_tiles_n, int total, int nk, uint32_t rank, int n_pairs) {
   const int wg = warp / 4;
   const int E = args.E, N = args.N;
   const int q = warp % 4;                  // TMEM lane quarter = 32 rows
-  const int half = wg - 1;                // columns [128*half, 128*half + 128)
+  const int half = wg - 1;                 // columns [128*half, 128*half + 128)
   const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
   uint32_t ch = 0;
-  for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-    const TileCoord c = decode_tile(s, E, n_tiles_n, tile);
+  for (int tile = blockIdx.x / 2; tile < total; tile += n_pairs) {
+    const TileCoord c = decode_tile(s, E, n_tiles_n, tile, rank);
     float acc[kEpiCols];
     bool ok = true;
     for (int c0 = 0; c0 < nk; c0 += kChunkKb, ++ch) {
@@ -252,7 +289,7 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s->chunk_empty[p]);
+      if (lane == 0) mbar_arrive_leader(&s->chunk_empty[p], rank);
     }
     if (!ok) break;
     const int row = c.m0 + q * 32 + lane;
@@ -285,6 +322,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   Smem* s = (Smem*)(tiles + kStages * kStageBytes);
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int wg = warp / 4;
+  const uint32_t rank = cluster_rank();       // 0 = leader (issues the MMAs)
+  const int n_pairs = gridDim.x / 2;
   const int E = args.E, Kd = args.Kd, N = args.N;
 
   for (int e = tid; e <= E; e += kThreads) s->off[e] = args.offsets[e];
@@ -292,21 +331,22 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     s->abort = 0;
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&s->full[i], 1);
-      mbar_init(&s->split[i], kNumSplitWarps);
+      mbar_init(&s->split[i], 2);   // one splitter warp per CTA per stage
       mbar_init(&s->empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s->chunk_full[i], 1);
-      mbar_init(&s->chunk_empty[i], kNumEpiWarps);
+      mbar_init(&s->chunk_empty[i], 2 * kNumEpiWarps);
     }
     mbar_init(&s->drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s->tmem_base)),
+    // the pair's TMEM: same column range in both CTAs
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s->tmem_base)),
                  "r"(kTmemCols) : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     tc_fence_before();
   }
   __syncthreads();
@@ -314,11 +354,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     int acc = 0;
     for (int e = 0; e < E; ++e) {
       s->start[e] = acc;
-      acc += (s->off[e + 1] - s->off[e] + BM - 1) / BM;
+      acc += (s->off[e + 1] - s->off[e] + 2 * BM - 1) / (2 * BM);
     }
     s->start[E] = acc;
   }
-  __syncthreads();
+  // both CTAs' barriers are initialised before any remote arrive
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = s->tmem_base;
   const int n_tiles_n = (N + BN - 1) / BN;
@@ -328,133 +369,142 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   if (wg == 1 || wg == 2) {
     // the epilogue warpgroups hold 128 FP32 running sums per thread
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
-    epilogue_role<kEpi>(s, args, tmem_base, warp, lane, n_tiles_n, total, nk);
+    epilogue_role<kEpi>(s, args, tmem_base, warp, lane, n_tiles_n, total, nk, rank, n_pairs);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
     if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      uint32_t it = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const TileCoord c = decode_tile(s, E, n_tiles_n, tile);
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const uint32_t st = it % kStages, use = it / kStages;
-          if (!mbar_wait(s, &s->empty[st], (use & 1) ^ 1, args.err)) { ok = false; break; }
-          uint8_t* base = tiles + st * kStageBytes;
-          mbar_arrive_expect_tx(&s->full[st], kTxBytes);
-          tma_load_2d(&mapA, &s->full[st], base, kb * BK, c.m0);
-          if (kNT) {
-            tma_load_3d(&mapB, &s->full[st], base + kTileABytes, kb * BK, c.n0, c.e);
-          } else {
-#pragma unroll
-            for (int j = 0; j < BN / 32; ++j)
-              tma_load_3d(&mapB, &s->full[st], base + kTileABytes + j * (32 * BK * 4), c.n0 + 32 * j, kb * BK, c.e);
-          }
-        }
-      }
-      // the last issued loads must land before the CTA may exit
-      const uint32_t n_last = it < (uint32_t)kStages ? it : (uint32_t)kStages;
-      for (uint32_t j = 0; j < n_last; ++j) {
-        const uint32_t i2 = it - 1 - j, st = i2 % kStages, use = i2 / kStages;
-        const long long t0 = clock64();
-        while (!mbar_try_wait(&s->full[st], use & 1) && clock64() - t0 < kWaitLimitCycles) {
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    // Each chunk of kChunkKb k-blocks is accumulated from zero into one of two
-    // TMEM buffers; the epilogue folds it into FP32 running sums.
-    if (lane == 0) {
-      constexpr uint32_t idesc = instr_desc(!kNT);
-      uint32_t it = 0, ch = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        for (int c0 = 0; c0 < nk && ok; c0 += kChunkKb, ++ch) {
-          const uint32_t p = ch & 1, cuse = ch >> 1;
-          if (!mbar_wait(s, &s->chunk_empty[p], (cuse & 1) ^ 1, args.err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t d_tmem = tmem_base + p * BN;
-          const int c1 = min(c0 + kChunkKb, nk);
-          for (int kb = c0; kb < c1; ++kb, ++it) {
+      // ---------------- TMA producer (each CTA loads its own A rows and B half) ----------------
+      if (lane == 0) {
+        uint32_t it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x / 2; tile < total && ok; tile += n_pairs) {
+          const TileCoord c = decode_tile(s, E, n_tiles_n, tile, rank);
+          const int nb = c.n0 + (int)rank * BNH;
+          for (int kb = 0; kb < nk; ++kb, ++it) {
             const uint32_t st = it % kStages, use = it / kStages;
-            if (!mbar_wait(s, &s->split[st], use & 1, args.err)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t a_hi = smem_u32(tiles + st * kStageBytes);
-            const uint32_t b_hi = a_hi + kTileABytes;
-            const uint32_t a_lo = a_hi + kTxBytes, b_lo = b_hi + kTxBytes;
+            if (!mbar_wait(s, &s->empty[st], (use & 1) ^ 1, args.err)) { ok = false; break; }
+            uint8_t* base = tiles + st * kStageBytes;
+            mbar_arrive_expect_tx(&s->full[st], kTxBytes);
+            tma_load_2d(&mapA, &s->full[st], base, kb * BK, c.m0);
+            if (kNT) {
+              tma_load_3d(&mapB, &s->full[st], base + kTileABytes, kb * BK, nb, c.e);
+            } else {
 #pragma unroll
-            for (int kk = 0; kk < BK / 8; ++kk) {
-              // K-major: 8 rows x 64 B per 512-byte group (SBO), k-step = +32 B.
-              // MN-major B: 32-column chunks 32*BK*4 B apart (LBO), 4 k-rows per
-              // 512-byte group (SBO), k-step of 8 rows = +1024 B.
-              const uint64_t adh = smem_desc(a_hi + kk * 32, 16, 512, kSwizzle64B);
-              const uint64_t adl = smem_desc(a_lo + kk * 32, 16, 512, kSwizzle64B);
-              uint64_t bdh, bdl;
-              if (kNT) {
-                bdh = smem_desc(b_hi + kk * 32, 16, 512, kSwizzle64B);
-                bdl = smem_desc(b_lo + kk * 32, 16, 512, kSwizzle64B);
-              } else {
-                bdh = smem_desc(b_hi + kk * 1024, 32 * BK * 4, 512, kSwizzle128B32B);
-                bdl = smem_desc(b_lo + kk * 1024, 32 * BK * 4, 512, kSwizzle128B32B);
-              }
-              tc_mma_tf32(d_tmem, adl, bdh, idesc, (kb > c0 || kk > 0) ? 1u : 0u);
-              tc_mma_tf32(d_tmem, adh, bdl, idesc, 1u);
-              tc_mma_tf32(d_tmem, adh, bdh, idesc, 1u);
+              for (int j = 0; j < BNH / 32; ++j)
+                tma_load_3d(&mapB, &s->full[st], base + kTileABytes + j * (32 * BK * 4), nb + 32 * j, kb * BK, c.e);
             }
-            tc_commit(&s->empty[st]);
           }
-          if (!ok) break;
-          tc_commit(&s->chunk_full[p]);
+        }
+        // the last issued loads must land before the CTA may exit
+        const uint32_t n_last = it < (uint32_t)kStages ? it : (uint32_t)kStages;
+        for (uint32_t j = 0; j < n_last; ++j) {
+          const uint32_t i2 = it - 1 - j, st = i2 % kStages, use = i2 / kStages;
+          const long long t0 = clock64();
+          while (!mbar_try_wait(&s->full[st], use & 1) && clock64() - t0 < kWaitLimitCycles) {
+          }
         }
       }
-      // every issued MMA completes before TMEM can be freed
-      tc_commit(&s->drain);
-      const long long t0 = clock64();
-      while (!mbar_try_wait(&s->drain, 0) && clock64() - t0 < kWaitLimitCycles) {
+    } else if (warp == 1) {
+      // ---------------- MMA issuer (leader CTA only) ----------------
+      // Each chunk of kChunkKb k-blocks is accumulated from zero into one of two
+      // TMEM buffers; the epilogues of both CTAs fold it into FP32 running sums.
+      if (lane == 0 && rank == 0) {
+        constexpr uint32_t idesc = instr_desc(!kNT);
+        uint32_t it = 0, ch = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x / 2; tile < total && ok; tile += n_pairs) {
+          for (int c0 = 0; c0 < nk && ok; c0 += kChunkKb, ++ch) {
+            const uint32_t p = ch & 1, cuse = ch >> 1;
+            if (!mbar_wait(s, &s->chunk_empty[p], (cuse & 1) ^ 1, args.err)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + p * BN;
+            const int c1 = min(c0 + kChunkKb, nk);
+            for (int kb = c0; kb < c1; ++kb, ++it) {
+              const uint32_t st = it % kStages, use = it / kStages;
+              if (!mbar_wait(s, &s->split[st], use & 1, args.err)) { ok = false; break; }
+              tc_fence_after();
+              const uint32_t a_hi = smem_u32(tiles + st * kStageBytes);
+              const uint32_t b_hi = a_hi + kTileABytes;
+              const uint32_t a_lo = a_hi + kTxBytes, b_lo = b_hi + kTxBytes;
+#pragma unroll
+              for (int kk = 0; kk < BK / 8; ++kk) {
+                // K-major: 8 rows x 64 B per 512-byte group (SBO), k-step = +32 B.
+                // MN-major B: 32-column chunks 32*BK*4 B apart (LBO), 4 k-rows per
+                // 512-byte group (SBO), k-step of 8 rows = +1024 B.
+                const uint64_t adh = smem_desc(a_hi + kk * 32, 16, 512, kSwizzle64B);
+                const uint64_t adl = smem_desc(a_lo + kk * 32, 16, 512, kSwizzle64B);
+                uint64_t bdh, bdl;
+                if (kNT) {
+                  bdh = smem_desc(b_hi + kk * 32, 16, 512, kSwizzle64B);
+                  bdl = smem_desc(b_lo + kk * 32, 16, 512, kSwizzle64B);
+                } else {
+                  bdh = smem_desc(b_hi + kk * 1024, 32 * BK * 4, 512, kSwizzle128B32B);
+                  bdl = smem_desc(b_lo + kk * 1024, 32 * BK * 4, 512, kSwizzle128B32B);
+                }
+                tc_mma_tf32_pair(d_tmem, adl, bdh, idesc, (kb > c0 || kk > 0) ? 1u : 0u);
+                tc_mma_tf32_pair(d_tmem, adh, bdl, idesc, 1u);
+                tc_mma_tf32_pair(d_tmem, adh, bdh, idesc, 1u);
+              }
+              tc_commit_pair(&s->empty[st]);
+            }
+            if (!ok) break;
+            tc_commit_pair(&s->chunk_full[p]);
+          }
+        }
+        // every issued MMA completes before TMEM can be freed (in both CTAs)
+        tc_commit_pair(&s->drain);
       }
-    }
+      if (lane == 0) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&s->drain, 0) && clock64() - t0 < kWaitLimitCycles) {
+        }
+      }
     } else {
       // ---------------- splitters: x -> lo = x - hi in the twin buffer ----------------
-    const int ci = warp < 4 ? warp - 2 : warp - 10;
-    const int ct = ci * 32 + lane;
-    constexpr int kSplitPer = (int)(kTxBytes / 16) / (kNumSplitWarps * 32);
-    static_assert(kSplitPer * kNumSplitWarps * 32 * 16 == (int)kTxBytes, "split work divides evenly");
-    uint32_t it = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      for (int kb = 0; kb < nk; ++kb, ++it) {
-        const uint32_t st = it % kStages, use = it / kStages;
-        if (!mbar_wait(s, &s->full[st], use & 1, args.err)) { ok = false; break; }
-        uint4* raw = reinterpret_cast<uint4*>(tiles + st * kStageBytes);
-        uint4* lo = reinterpret_cast<uint4*>(tiles + st * kStageBytes + kTxBytes);
-        // all of this thread's 16-byte words are loaded first, then split; the
-        // raw tile itself is the high part (the MMA ignores the 13 low bits)
-        uint4 x[kSplitPer];
+      // Each splitter warp owns whole k-blocks (every kNumSplitWarps-th), so a
+      // stage costs one proxy fence and one arrive, and the ring depth hides a
+      // warp's latency.  The raw tile itself is the high part (the MMA ignores
+      // the 13 low bits of an FP32 operand).
+      const int ci = warp < 4 ? warp - 2 : warp - 10;
+      constexpr int kVec = (int)(kTxBytes / 16);
+      constexpr int kBatch = 8;
+      static_assert(kVec % (32 * kBatch) == 0, "split batches divide the stage");
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x / 2; tile < total && ok; tile += n_pairs) {
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          if ((int)(it % kNumSplitWarps) != ci) continue;
+          const uint32_t st = it % kStages, use = it / kStages;
+          if (!mbar_wait(s, &s->full[st], use & 1, args.err)) { ok = false; break; }
+          uint4* raw = reinterpret_cast<uint4*>(tiles + st * kStageBytes);
+          uint4* lo = reinterpret_cast<uint4*>(tiles + st * kStageBytes + kTxBytes);
+#pragma unroll 1
+          for (int b0 = lane; b0 < kVec; b0 += 32 * kBatch) {
+            uint4 x[kBatch];
 #pragma unroll
-        for (int j = 0; j < kSplitPer; ++j) x[j] = raw[ct + j * kNumSplitWarps * 32];
+            for (int j = 0; j < kBatch; ++j) x[j] = raw[b0 + 32 * j];
 #pragma unroll
-        for (int j = 0; j < kSplitPer; ++j) {
-          const uint4 l = make_uint4(
-              __float_as_uint(__uint_as_float(x[j].x) - __uint_as_float(x[j].x & kTf32Mask)),
-              __float_as_uint(__uint_as_float(x[j].y) - __uint_as_float(x[j].y & kTf32Mask)),
-              __float_as_uint(__uint_as_float(x[j].z) - __uint_as_float(x[j].z & kTf32Mask)),
-              __float_as_uint(__uint_as_float(x[j].w) - __uint_as_float(x[j].w & kTf32Mask)));
-          lo[ct + j * kNumSplitWarps * 32] = l;
+            for (int j = 0; j < kBatch; ++j)
+              lo[b0 + 32 * j] = make_uint4(
+                  __float_as_uint(__uint_as_float(x[j].x) - __uint_as_float(x[j].x & kTf32Mask)),
+                  __float_as_uint(__uint_as_float(x[j].y) - __uint_as_float(x[j].y & kTf32Mask)),
+                  __float_as_uint(__uint_as_float(x[j].z) - __uint_as_float(x[j].z & kTf32Mask)),
+                  __float_as_uint(__uint_as_float(x[j].w) - __uint_as_float(x[j].w & kTf32Mask)));
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) mbar_arrive_leader(&s->split[st], rank);
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s->split[st]);
       }
-    }
     }
   }
 
+  // no CTA leaves (or frees TMEM) while its peer may still signal its barriers
   __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
                  : "memory");
   }
 }
@@ -488,8 +538,8 @@ bool map_a(CUtensorMap* m, const float* A, int64_t R, int Kd) {
 }
 
 // B for "x W": W [E, Kd, N] (N contiguous), box 32 (n) x 16 (k) x 1, 128-byte
-//   swizzle with 32-byte atoms (MN-major)
-// B for "x W^T": W [E, N, Kd] (Kd contiguous), box 16 (k) x 256 (n) x 1, 64-byte swizzle
+//   swizzle with 32-byte atoms (MN-major); 4 boxes per CTA and k-block
+// B for "x W^T": W [E, N, Kd] (Kd contiguous), box 16 (k) x 128 (n) x 1, 64-byte swizzle
 bool map_b(CUtensorMap* m, const float* W, int E, int Kd, int N, bool nt) {
   auto enc = encode_fn();
   if (!enc) return false;
@@ -498,7 +548,7 @@ bool map_b(CUtensorMap* m, const float* W, int E, int Kd, int N, bool nt) {
   if (nt) {
     dims[0] = Kd; dims[1] = N; dims[2] = E;
     strides[0] = (cuuint64_t)Kd * 4; strides[1] = (cuuint64_t)Kd * N * 4;
-    box[0] = BK; box[1] = BN; box[2] = 1;
+    box[0] = BK; box[1] = BNH; box[2] = 1;
   } else {
     dims[0] = N; dims[1] = Kd; dims[2] = E;
     strides[0] = (cuuint64_t)N * 4; strides[1] = (cuuint64_t)Kd * N * 4;
@@ -526,7 +576,20 @@ janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, in
   if (!map_a(&ma, A, R, Kd) || !map_b(&mb, W, E, Kd, N, kNT)) return JANUS_ERR_CUDA;
   Args a;
   a.C = C; a.C2 = C2; a.aux = aux; a.offsets = offsets; a.E = E; a.Kd = Kd; a.N = N; a.err = err;
-  tc_gemm_kernel<kNT, kEpi><<<num_sms(), kThreads, kSmemBytes, stream>>>(ma, mb, a);
+  // one CTA per SM, in clusters of two (the MMA pairs)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(num_sms() / 2 * 2));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute cluster_attr[1];
+  cluster_attr[0].id = cudaLaunchAttributeClusterDimension;
+  cluster_attr[0].val.clusterDim.x = 2;
+  cluster_attr[0].val.clusterDim.y = 1;
+  cluster_attr[0].val.clusterDim.z = 1;
+  cfg.attrs = cluster_attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, tc_gemm_kernel<kNT, kEpi>, ma, mb, a) != cudaSuccess) return JANUS_ERR_CUDA;
   return launch_status();
 }
 
