@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--atoms", type=int, default=None, help="override N (profiling small cases)")
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling small cases)")
+    ap.add_argument("--ref-seconds", type=float, default=None,
+                    help="reference arm: target seconds of oracle work per step")
     return ap.parse_args()
 
 
@@ -396,7 +398,7 @@ def run_reference(args, world, rank):
     inp = synth.layer_inputs(cfg, seed=args.seed, device="cpu", with_edges=False)
     host = dict(types=inp["types"], gate=inp["gate"], x=inp["x"].numpy(), g=inp["g"].numpy(),
                 w1=inp["w1"].numpy(), w2=inp["w2"].numpy())
-    per_step = max(2.0, min(15.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step = args.ref_seconds or max(2.0, min(15.0, 150.0 / max(1, args.steps + args.warmup)))
     n_s = oracle_calibrate(cfg, host, per_step)
     times = []
     for i in range(args.warmup + args.steps):
