@@ -42,6 +42,7 @@ def _setup(L):
     L.orc_dequant_by_type.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp]
     L.orc_expert_ffn_fwd.argtypes = [vp, vp, i32, i64, i32, i32, vp, vp, vp, i64, vp, vp]
     L.orc_expert_ffn_vjp.argtypes = [vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, i64, vp]
+    L.orc_expert_ffn_weight_grad.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp, vp]
     L.orc_combine.argtypes = [vp, vp, vp, i64, i32, i32, vp]
     L.orc_edge_aggregate.argtypes = [vp, vp, i64, i32, vp]
 
@@ -151,6 +152,22 @@ def expert_ffn_vjp(xd, gd, offsets, w1, w2, rows=None):
     lib().orc_expert_ffn_vjp(_p(xd), _p(gd), _p(offsets), E, R, d, h, _p(w1), _p(w2),
                              _p(r), 0 if r is None else r.shape[0], _p(dxd))
     return dxd
+
+
+def expert_ffn_weight_grad(xd, gd, offsets, w1, w2):
+    """Per-expert weight gradients (dW1 [E,d,h], dW2 [E,h,d]) of
+    L = sum_p <yd[p], gd[p]> for the bias-free Linear-SiLU-Linear experts."""
+    xd = _c(xd, np.float32)
+    gd = _c(gd, np.float32)
+    offsets = _c(offsets, np.int32)
+    w1 = _c(w1, np.float32)
+    w2 = _c(w2, np.float32)
+    E, d, h = w1.shape
+    dw1 = np.empty((E, d, h), np.float32)
+    dw2 = np.empty((E, h, d), np.float32)
+    lib().orc_expert_ffn_weight_grad(_p(xd), _p(gd), _p(offsets), E, d, h, _p(w1), _p(w2),
+                                     _p(dw1), _p(dw2))
+    return dw1, dw2
 
 
 def combine(yd, slot_of, top_k, topk_weight=None):

@@ -296,6 +296,45 @@ void orc_expert_ffn_vjp(const float* xd, const float* gd, const int32_t* offsets
 }
 
 // ---------------------------------------------------------------------------
+// Expert weight gradients (the layer's parameters, needed by force training:
+// [Review] section 3.3).  With L = sum_p <Yd[p,:], Gd[p,:]> over the rows of
+// expert e and a = x W1, hh = silu(a):
+//   dW2[e][j][c] = sum_p hh[p][j] * gd[p][c]
+//   dW1[e][k][j] = sum_p x[p][k] * dA[p][j],  dA = (W2 g) * silu'(a)
+// An expert with no rows gets zero gradients.  a and dA are recomputed in FP64.
+// ---------------------------------------------------------------------------
+void orc_expert_ffn_weight_grad(const float* xd, const float* gd, const int32_t* offsets,
+                                int32_t n_experts, int32_t d, int32_t h, const float* w1,
+                                const float* w2, float* dw1, float* dw2) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int e = 0; e < n_experts; ++e) {
+    const float* W1 = w1 + (int64_t)e * d * h;
+    const float* W2 = w2 + (int64_t)e * h * d;
+    std::vector<double> g1((size_t)d * h, 0.0), g2((size_t)h * d, 0.0), a(h), hh(h), da(h);
+    for (int64_t p = offsets[e]; p < offsets[e + 1]; ++p) {
+      std::fill(a.begin(), a.end(), 0.0);
+      for (int k = 0; k < d; ++k) {
+        const double xk = xd[p * d + k];
+        for (int j = 0; j < h; ++j) a[j] += xk * (double)W1[(int64_t)k * h + j];
+      }
+      for (int j = 0; j < h; ++j) {
+        double dh = 0.0;
+        for (int c = 0; c < d; ++c) dh += (double)W2[(int64_t)j * d + c] * (double)gd[p * d + c];
+        const double sg = 1.0 / (1.0 + std::exp(-a[j]));
+        hh[j] = a[j] * sg;
+        da[j] = dh * sg * (1.0 + a[j] * (1.0 - sg));
+      }
+      for (int j = 0; j < h; ++j)
+        for (int c = 0; c < d; ++c) g2[(size_t)j * d + c] += hh[j] * (double)gd[p * d + c];
+      for (int k = 0; k < d; ++k)
+        for (int j = 0; j < h; ++j) g1[(size_t)k * h + j] += (double)xd[p * d + k] * da[j];
+    }
+    for (size_t i = 0; i < g1.size(); ++i) dw1[(int64_t)e * d * h + i] = (float)g1[i];
+    for (size_t i = 0; i < g2.size(); ++i) dw2[(int64_t)e * h * d + i] = (float)g2[i];
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Combine.  [Blueprint] §3.2: the activated experts' outputs are summed with
 // the gate weights.  Gather form: Y[i,:] = sum_{k ascending} w[i,k] *
 // Yd[slot_of[i*K+k],:]; topk_weight == NULL means weight 1 (the VJP combine).

@@ -28,12 +28,14 @@ def _np_forward(xd, offsets, w1, w2, dtype=np.float64):
     for e in range(w1.shape[0]):
         a, b = offsets[e], offsets[e + 1]
         if b > a:
-            pre = xd[a:b].astype(dtype) @ w1[e].astype(np.float64)
+            w1e = w1[e] if np.iscomplexobj(w1) else w1[e].astype(np.float64)
+            w2e = w2[e] if np.iscomplexobj(w2) else w2[e].astype(np.float64)
+            pre = xd[a:b].astype(dtype) @ w1e
             if np.iscomplexobj(pre):
                 hh = pre / (1.0 + np.exp(-pre))
             else:
                 hh = pre * scipy.special.expit(pre)
-            y[a:b] = hh @ w2[e].astype(np.float64)
+            y[a:b] = hh @ w2e
     return y
 
 
@@ -124,3 +126,41 @@ def test_layer_vjp_finite_differences():
     dd = layer(x.astype(np.float64) + 1j * 1e-30 * v).imag / 1e-30
     got = np.sum(dx.astype(np.float64) * v)
     assert abs(got - dd) <= 1e-6 * abs(dd)
+
+
+def test_weight_grad_complex_step():
+    # d/dt <Y(W + t V), G> = <dW, V>: complex step through the pinned forward
+    counts = [6, 0, 9, 4]
+    offs = _offsets(counts)
+    E, d, h = 4, 8, 12
+    w1, w2 = _experts(E, d, h, seed=12)
+    R = offs[-1]
+    xd = synth.normal((R, d), 13).numpy()
+    gd = synth.normal((R, d), 14).numpy()
+    dw1, dw2 = oracle.expert_ffn_weight_grad(xd, gd, offs, w1, w2)
+    assert np.all(dw1[1] == 0) and np.all(dw2[1] == 0)        # expert without rows
+    g = np.random.default_rng(5)
+    for _ in range(3):
+        v1 = g.standard_normal(w1.shape)
+        v2 = g.standard_normal(w2.shape)
+        hcs = 1e-30
+        y1 = _np_forward(xd.astype(np.complex128), offs, w1 + 1j * hcs * v1, w2, np.complex128)
+        y2 = _np_forward(xd.astype(np.complex128), offs, w1, w2 + 1j * hcs * v2, np.complex128)
+        d1 = np.sum(y1.imag * gd) / hcs
+        d2 = np.sum(y2.imag * gd) / hcs
+        assert abs(np.sum(dw1.astype(np.float64) * v1) - d1) <= 1e-6 * abs(d1)
+        assert abs(np.sum(dw2.astype(np.float64) * v2) - d2) <= 1e-6 * abs(d2)
+
+
+def test_weight_grad_dw2_is_numpy_outer_sum():
+    counts = [5, 7]
+    offs = _offsets(counts)
+    w1, w2 = _experts(2, 6, 10, seed=21)
+    xd = synth.normal((12, 6), 22).numpy()
+    gd = synth.normal((12, 6), 23).numpy()
+    _, dw2 = oracle.expert_ffn_weight_grad(xd, gd, offs, w1, w2)
+    for e in range(2):
+        a, b = offs[e], offs[e + 1]
+        pre = xd[a:b].astype(np.float64) @ w1[e]
+        hh = pre * scipy.special.expit(pre)
+        np.testing.assert_allclose(dw2[e], hh.T @ gd[a:b].astype(np.float64), rtol=1e-6, atol=1e-7)
