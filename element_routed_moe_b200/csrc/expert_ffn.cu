@@ -14,6 +14,8 @@
 //   G0: a = xd W1[e]          (only when the forward's act is not supplied)
 //   G3: dA = (gd W2[e]^T) * silu'(a)   (workspace)
 //   G4: dxd = dA W1[e]^T
+// Weight gradients (G3 also writes H = silu(a)):
+//   G5: dW1[e] = Xd_e^T dA_e,  G6: dW2[e] = H_e^T Gd_e  (sums over expert e's rows)
 #include "common.cuh"
 #include "ffn_simt.cuh"
 #include "ffn_tc.cuh"
@@ -137,5 +139,61 @@ extern "C" janus_status janus_expert_ffn_vjp(const float* xd, const float* gd, c
     launch_simt<false, simt::kEpiStore>(make_args(xd, w1, sw, A, nullptr, nullptr, offsets, n_experts, d, h), stream);
   launch_simt<true, simt::kEpiDSilu>(make_args(gd, w2, sw, dA, nullptr, A, offsets, n_experts, d, h), stream);
   launch_simt<true, simt::kEpiStore>(make_args(dA, w1, sw, dxd, nullptr, nullptr, offsets, n_experts, h, d), stream);
+  return launch_status();
+}
+
+extern "C" janus_status janus_expert_ffn_weight_grad_workspace_size(int64_t n_rows, int32_t h,
+                                                                    int32_t have_act, size_t* bytes) {
+  JANUS_CHECK_ARG(bytes && n_rows >= 0 && h >= 1);
+  const size_t rh = align_up(sizeof(float) * (size_t)n_rows * (size_t)h, 256);
+  *bytes = sizeof(WsHeader) + (have_act ? 2 : 3) * rh;
+  return JANUS_OK;
+}
+
+extern "C" janus_status janus_expert_ffn_weight_grad(const float* xd, const float* gd, const float* act,
+                                                     const int32_t* offsets, int32_t n_experts,
+                                                     int64_t n_rows, int32_t d, int32_t h,
+                                                     const float* w1, const float* w2, float* dw1,
+                                                     float* dw2, janus_ffn_mode mode, void* workspace,
+                                                     size_t workspace_bytes, janus_stream_t stream_) {
+  cudaStream_t stream = (cudaStream_t)stream_;
+  janus_status st = check_ffn(xd, offsets, n_experts, n_rows, d, h, w1, w2, dw1, mode);
+  if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(dw1 && dw2 && (n_rows == 0 || gd));
+  JANUS_CHECK_ALIGN(aligned(dw1, 16) && aligned(dw2, 16));
+  JANUS_CHECK_ALIGN(n_rows == 0 || aligned(gd, 16));
+  JANUS_CHECK_ALIGN(act == nullptr || aligned(act, 16));
+  size_t need = 0;
+  st = janus_expert_ffn_weight_grad_workspace_size(n_rows, h, act != nullptr, &need);
+  if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(workspace && workspace_bytes >= need);
+  JANUS_CHECK_ALIGN(aligned(workspace, 256));
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  const size_t wbytes = sizeof(float) * (size_t)n_experts * (size_t)d * (size_t)h;
+  if (n_rows == 0) {   // no rows routed anywhere: every gradient is zero
+    JANUS_CUDA_TRY(cudaMemsetAsync(dw1, 0, wbytes, stream));
+    JANUS_CUDA_TRY(cudaMemsetAsync(dw2, 0, wbytes, stream));
+    return JANUS_OK;
+  }
+  const size_t rh = align_up(sizeof(float) * (size_t)n_rows * (size_t)h, 256);
+  char* w = (char*)workspace + sizeof(WsHeader);
+  float* dA = (float*)w;
+  float* H = (float*)(w + rh);
+  float* A = act ? const_cast<float*>(act) : (float*)(w + 2 * rh);
+  if (mode == JANUS_FFN_3XTF32) {
+    JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
+    st = tc::expert_ffn_weight_grad(xd, gd, act, A, offsets, n_experts, n_rows, d, h, w1, w2, dw1, dw2, dA,
+                                    H, &((WsHeader*)workspace)->error, stream);
+    if (st != JANUS_OK) return st;
+    return launch_status();
+  }
+  const int64_t sw = (int64_t)d * h;
+  if (!act)
+    launch_simt<false, simt::kEpiStore>(make_args(xd, w1, sw, A, nullptr, nullptr, offsets, n_experts, d, h), stream);
+  launch_simt<true, simt::kEpiDSilu>(make_args(gd, w2, sw, dA, H, A, offsets, n_experts, d, h), stream);
+  simt::TnArgs t1{xd, dA, dw1, offsets, n_experts, d, h};
+  simt::grouped_tn_kernel<<<num_sms() * 2, simt::kThreads, 0, stream>>>(t1);
+  simt::TnArgs t2{H, gd, dw2, offsets, n_experts, h, d};
+  simt::grouped_tn_kernel<<<num_sms() * 2, simt::kThreads, 0, stream>>>(t2);
   return launch_status();
 }

@@ -203,8 +203,105 @@ __global__ void __launch_bounds__(kThreads, 2) grouped_gemm_kernel(Args args) {
         } else if (kEpi == kEpiDSilu) {
           const float4 a = __ldg(reinterpret_cast<const float4*>(args.aux + o));
           v = make_float4(v.x * dsilu_f(a.x), v.y * dsilu_f(a.y), v.z * dsilu_f(a.z), v.w * dsilu_f(a.w));
+          if (args.C2)   // H = silu(a) for the second weight gradient
+            *reinterpret_cast<float4*>(args.C2 + o) = make_float4(silu_f(a.x), silu_f(a.y), silu_f(a.z), silu_f(a.w));
         }
         *reinterpret_cast<float4*>(args.C + o) = v;
+      }
+    }
+  }
+}
+
+// Per-expert weight gradient on the CUDA cores:
+//   C[e] [M,N] = sum over rows p of expert e of X[p, :]^T Y[p, :]
+// X [R,M] and Y [R,N] row-major; both tiles are loaded along their contiguous
+// dimension (k = row), rows past the expert's segment are zero; an expert
+// without rows gets a zero matrix.  Same 128x128x16 register tiling.
+struct TnArgs {
+  const float* X;
+  const float* Y;
+  float* C;
+  const int32_t* offsets;
+  int E, M, N;
+};
+
+__global__ void __launch_bounds__(kThreads, 2) grouped_tn_kernel(TnArgs args) {
+  __shared__ __align__(16) float As[2][BK][BM];
+  __shared__ __align__(16) float Bs[2][BK][BN];
+  const int tid = threadIdx.x;
+  const int tx = tid % 16, ty = tid / 16;
+  const int M = args.M, N = args.N;
+  const int n_tm = (M + BM - 1) / BM, n_tn = (N + BN - 1) / BN;
+  const int total = args.E * n_tm * n_tn;
+  for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    const int e = tile / (n_tm * n_tn);
+    const int rem = tile % (n_tm * n_tn);
+    const int m0 = (rem / n_tn) * BM, n0 = (rem % n_tn) * BN;
+    const int p0 = args.offsets[e], p1 = args.offsets[e + 1];
+    const int nk = (p1 - p0 + BK - 1) / BK;
+    float4 ra[2], rb[2];
+    auto load_tile = [&](int kt) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int idx = tid + j * kThreads;
+        const int kr = idx / (BM / 4), q = idx % (BM / 4);
+        const int p = p0 + kt * BK + kr;
+        const bool okr = p < p1;
+        ra[j] = (okr && m0 + q * 4 < M) ? __ldg(reinterpret_cast<const float4*>(args.X + (int64_t)p * M + m0 + q * 4))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        rb[j] = (okr && n0 + q * 4 < N) ? __ldg(reinterpret_cast<const float4*>(args.Y + (int64_t)p * N + n0 + q * 4))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    auto store_tile = [&](int buf) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int idx = tid + j * kThreads;
+        const int kr = idx / (BM / 4), q = idx % (BM / 4);
+        *reinterpret_cast<float4*>(&As[buf][kr][q * 4]) = ra[j];
+        *reinterpret_cast<float4*>(&Bs[buf][kr][q * 4]) = rb[j];
+      }
+    };
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    if (nk > 0) {
+      load_tile(0);
+      store_tile(0);
+    }
+    __syncthreads();
+    for (int kt = 0; kt < nk; ++kt) {
+      const int cur = kt & 1;
+      if (kt + 1 < nk) load_tile(kt + 1);
+#pragma unroll
+      for (int k = 0; k < BK; ++k) {
+        const float4 a0 = *reinterpret_cast<const float4*>(&As[cur][k][ty * 4]);
+        const float4 a1 = *reinterpret_cast<const float4*>(&As[cur][k][64 + ty * 4]);
+        const float4 b0 = *reinterpret_cast<const float4*>(&Bs[cur][k][tx * 4]);
+        const float4 b1 = *reinterpret_cast<const float4*>(&Bs[cur][k][64 + tx * 4]);
+        const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+      }
+      if (kt + 1 < nk) store_tile(cur ^ 1);
+      __syncthreads();
+    }
+    float* C = args.C + (int64_t)e * M * N;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+      if (r >= M) continue;
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        const int c = n0 + g * 64 + tx * 4;
+        if (c >= N) continue;
+        *reinterpret_cast<float4*>(C + (int64_t)r * N + c) =
+            make_float4(acc[i][g * 4 + 0], acc[i][g * 4 + 1], acc[i][g * 4 + 2], acc[i][g * 4 + 3]);
       }
     }
   }

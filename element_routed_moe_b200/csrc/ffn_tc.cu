@@ -76,12 +76,19 @@ constexpr long long kWaitLimitCycles = 4000000000LL;     // ~2 s at 2 GHz
 
 enum Epilogue : int { kEpiStore = 0, kEpiSilu = 1, kEpiDSilu = 2 };
 
+// Operand layouts:  kModeNN  C = A W       (W stored [E][Kd][N], MN-major B)
+//                   kModeNT  C = A W^T     (W stored [E][N][Kd], K-major B)
+//                   kModeTN  C_e = X_e^T Y_e per expert (weight gradient; both
+//                            operands MN-major, K = the expert's row segment)
+enum Mode : int { kModeNN = 0, kModeNT = 1, kModeTN = 2 };
+
 struct Args {
   float* C;
   float* C2;
   const float* aux;
   const int32_t* offsets;
   int E, Kd, N;
+  int M;            // kModeTN: rows of each expert's output (C is [E][M][N])
   int32_t* err;
 };
 
@@ -206,11 +213,11 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
-// Instruction descriptor: D=F32, A=B=TF32, A K-major, B K- or MN-major,
+// Instruction descriptor: D=F32, A=B=TF32, A and B K- or MN-major,
 // M=256 (the CTA pair), N=256.
-__host__ __device__ constexpr uint32_t instr_desc(bool b_mn_major) {
-  return (1u << 4) | (2u << 7) | (2u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(BN >> 3) << 17) |
-         ((uint32_t)((2 * BM) >> 4) << 24);
+__host__ __device__ constexpr uint32_t instr_desc(bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)((2 * BM) >> 4) << 24);
 }
 
 __device__ __forceinline__ float silu_f(float a) { return a / (1.0f + expf(-a)); }
@@ -240,41 +247,62 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 
 struct TileCoord {
   int e, m0, m_end, n0;
+  int k_row0;       // kModeTN: first row of the expert's segment (the K range)
+  int k_rows;       // kModeTN: rows in the segment
+  int nk;           // k-blocks of this tile
 };
 
 // Pair tile `tile` -> expert, this CTA's 128-row block and the 256-column block.
-// start[e] counts 256-row blocks (one per CTA pair).
-__device__ __forceinline__ TileCoord decode_tile(const Smem* s, int E, int n_tiles_n, int tile, uint32_t rank) {
-  const int mt = tile / n_tiles_n, nt = tile % n_tiles_n;
-  int lo = 0, hi = E;   // start[lo] <= mt < start[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (s->start[mid] <= mt) lo = mid; else hi = mid;
-  }
+//   kModeNN/NT: start[e] counts 256-row blocks of expert e's row segment.
+//   kModeTN:    every expert has ceil(M/256) row blocks of its [M x N] output.
+template <int kMode>
+__device__ __forceinline__ TileCoord decode_tile(const Smem* s, const Args& args, int n_tiles_n, int nk_fixed,
+                                                 int tile, uint32_t rank) {
   TileCoord c;
-  c.e = lo;
-  c.m0 = s->off[lo] + ((mt - s->start[lo]) * 2 + (int)rank) * BM;
-  c.m_end = s->off[lo + 1];
+  const int mt = tile / n_tiles_n, nt = tile % n_tiles_n;
   c.n0 = nt * BN;
+  if (kMode == kModeTN) {
+    const int n_mp = (args.M + 2 * BM - 1) / (2 * BM);
+    c.e = mt / n_mp;
+    c.m0 = ((mt % n_mp) * 2 + (int)rank) * BM;
+    c.m_end = args.M;
+    c.k_row0 = s->off[c.e];
+    c.k_rows = s->off[c.e + 1] - c.k_row0;
+    c.nk = (c.k_rows + BK - 1) / BK;
+  } else {
+    int lo = 0, hi = args.E;   // start[lo] <= mt < start[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s->start[mid] <= mt) lo = mid; else hi = mid;
+    }
+    c.e = lo;
+    c.m0 = s->off[lo] + ((mt - s->start[lo]) * 2 + (int)rank) * BM;
+    c.m_end = s->off[lo + 1];
+    c.k_row0 = 0;
+    c.k_rows = 0;
+    c.nk = nk_fixed;
+  }
   return c;
 }
 
 // Epilogue warpgroups: fold each TMEM chunk into FP32 running sums, then apply
 // the fused epilogue and store this CTA's 128 x 256 part of the tile.
-template <int kEpi>
+template <int kMode, int kEpi>
 __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_t tmem_base, int warp, int lane,
-                                              int n_tiles_n, int total, int nk, uint32_t rank, int n_pairs) {
+                                              int n_tiles_n, int total, int nk_fixed, uint32_t rank, int n_pairs) {
   const int wg = warp / 4;
-  const int E = args.E, N = args.N;
+  const int N = args.N;
   const int q = warp % 4;                  // TMEM lane quarter = 32 rows
   const int half = wg - 1;                 // columns [128*half, 128*half + 128)
   const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
   uint32_t ch = 0;
   for (int tile = blockIdx.x / 2; tile < total; tile += n_pairs) {
-    const TileCoord c = decode_tile(s, E, n_tiles_n, tile, rank);
+    const TileCoord c = decode_tile<kMode>(s, args, n_tiles_n, nk_fixed, tile, rank);
     float acc[kEpiCols];
+#pragma unroll
+    for (int j = 0; j < kEpiCols; ++j) acc[j] = 0.f;     // a tile with no k-blocks stores zeros
     bool ok = true;
-    for (int c0 = 0; c0 < nk; c0 += kChunkKb, ++ch) {
+    for (int c0 = 0; c0 < c.nk; c0 += kChunkKb, ++ch) {
       const uint32_t p = ch & 1, cuse = ch >> 1;
       if (!mbar_wait(s, &s->chunk_full[p], cuse & 1, args.err)) { ok = false; break; }
       tc_fence_after();
@@ -285,7 +313,7 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
         tmem_ld16(taddr + j, r);
 #pragma unroll
         for (int t = 0; t < 16; ++t)
-          acc[j + t] = (c0 == 0) ? __uint_as_float(r[t]) : acc[j + t] + __uint_as_float(r[t]);
+          acc[j + t] += __uint_as_float(r[t]);
       }
       tc_fence_before();
       __syncwarp();
@@ -295,7 +323,7 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
     const int row = c.m0 + q * 32 + lane;
     const int colb = c.n0 + half * kEpiCols;
     if (row < c.m_end && colb < N) {
-      const int64_t o = (int64_t)row * N + colb;
+      const int64_t o = (kMode == kModeTN ? (int64_t)c.e * args.M * N : 0) + (int64_t)row * N + colb;
 #pragma unroll
       for (int j = 0; j < kEpiCols; j += 4) {
         if (colb + j < N) {
@@ -306,6 +334,9 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
           } else if (kEpi == kEpiDSilu) {
             const float4 a = __ldg(reinterpret_cast<const float4*>(args.aux + o + j));
             v = make_float4(v.x * dsilu_f(a.x), v.y * dsilu_f(a.y), v.z * dsilu_f(a.z), v.w * dsilu_f(a.w));
+            if (args.C2)   // H = silu(a) for the second weight gradient
+              *reinterpret_cast<float4*>(args.C2 + o + j) =
+                  make_float4(silu_f(a.x), silu_f(a.y), silu_f(a.z), silu_f(a.w));
           }
           *reinterpret_cast<float4*>(args.C + o + j) = v;
         }
@@ -314,7 +345,7 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
   }
 }
 
-template <bool kNT, int kEpi>
+template <int kMode, int kEpi>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, Args args) {
   extern __shared__ uint8_t smem_raw[];
@@ -354,7 +385,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     int acc = 0;
     for (int e = 0; e < E; ++e) {
       s->start[e] = acc;
-      acc += (s->off[e + 1] - s->off[e] + 2 * BM - 1) / (2 * BM);
+      acc += kMode == kModeTN ? (args.M + 2 * BM - 1) / (2 * BM)
+                              : (s->off[e + 1] - s->off[e] + 2 * BM - 1) / (2 * BM);
     }
     s->start[E] = acc;
   }
@@ -369,7 +401,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   if (wg == 1 || wg == 2) {
     // the epilogue warpgroups hold 128 FP32 running sums per thread
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
-    epilogue_role<kEpi>(s, args, tmem_base, warp, lane, n_tiles_n, total, nk, rank, n_pairs);
+    epilogue_role<kMode, kEpi>(s, args, tmem_base, warp, lane, n_tiles_n, total, nk, rank, n_pairs);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
     if (warp == 0) {
@@ -378,20 +410,32 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         uint32_t it = 0;
         bool ok = true;
         for (int tile = blockIdx.x / 2; tile < total && ok; tile += n_pairs) {
-          const TileCoord c = decode_tile(s, E, n_tiles_n, tile, rank);
+          const TileCoord c = decode_tile<kMode>(s, args, n_tiles_n, nk, tile, rank);
           const int nb = c.n0 + (int)rank * BNH;
-          for (int kb = 0; kb < nk; ++kb, ++it) {
+          for (int kb = 0; kb < c.nk; ++kb, ++it) {
             const uint32_t st = it % kStages, use = it / kStages;
             if (!mbar_wait(s, &s->empty[st], (use & 1) ^ 1, args.err)) { ok = false; break; }
             uint8_t* base = tiles + st * kStageBytes;
             mbar_arrive_expect_tx(&s->full[st], kTxBytes);
-            tma_load_2d(&mapA, &s->full[st], base, kb * BK, c.m0);
-            if (kNT) {
-              tma_load_3d(&mapB, &s->full[st], base + kTileABytes, kb * BK, nb, c.e);
-            } else {
+            if (kMode == kModeTN) {
+              // both operands MN-major: 32-column boxes of 16 segment rows
+              const int row = c.k_row0 + kb * BK;
+#pragma unroll
+              for (int j = 0; j < BM / 32; ++j)
+                tma_load_2d(&mapA, &s->full[st], base + j * (32 * BK * 4), c.m0 + 32 * j, row);
 #pragma unroll
               for (int j = 0; j < BNH / 32; ++j)
-                tma_load_3d(&mapB, &s->full[st], base + kTileABytes + j * (32 * BK * 4), nb + 32 * j, kb * BK, c.e);
+                tma_load_2d(&mapB, &s->full[st], base + kTileABytes + j * (32 * BK * 4), nb + 32 * j, row);
+            } else {
+              tma_load_2d(&mapA, &s->full[st], base, kb * BK, c.m0);
+              if (kMode == kModeNT) {
+                tma_load_3d(&mapB, &s->full[st], base + kTileABytes, kb * BK, nb, c.e);
+              } else {
+#pragma unroll
+                for (int j = 0; j < BNH / 32; ++j)
+                  tma_load_3d(&mapB, &s->full[st], base + kTileABytes + j * (32 * BK * 4), nb + 32 * j, kb * BK,
+                              c.e);
+              }
             }
           }
         }
@@ -409,16 +453,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       // Each chunk of kChunkKb k-blocks is accumulated from zero into one of two
       // TMEM buffers; the epilogues of both CTAs fold it into FP32 running sums.
       if (lane == 0 && rank == 0) {
-        constexpr uint32_t idesc = instr_desc(!kNT);
+        constexpr uint32_t idesc = instr_desc(kMode == kModeTN, kMode != kModeNT);
         uint32_t it = 0, ch = 0;
         bool ok = true;
         for (int tile = blockIdx.x / 2; tile < total && ok; tile += n_pairs) {
-          for (int c0 = 0; c0 < nk && ok; c0 += kChunkKb, ++ch) {
+          const int tnk = decode_tile<kMode>(s, args, n_tiles_n, nk, tile, rank).nk;
+          for (int c0 = 0; c0 < tnk && ok; c0 += kChunkKb, ++ch) {
             const uint32_t p = ch & 1, cuse = ch >> 1;
             if (!mbar_wait(s, &s->chunk_empty[p], (cuse & 1) ^ 1, args.err)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + p * BN;
-            const int c1 = min(c0 + kChunkKb, nk);
+            const int c1 = min(c0 + kChunkKb, tnk);
             for (int kb = c0; kb < c1; ++kb, ++it) {
               const uint32_t st = it % kStages, use = it / kStages;
               if (!mbar_wait(s, &s->split[st], use & 1, args.err)) { ok = false; break; }
@@ -431,10 +476,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                 // K-major: 8 rows x 64 B per 512-byte group (SBO), k-step = +32 B.
                 // MN-major B: 32-column chunks 32*BK*4 B apart (LBO), 4 k-rows per
                 // 512-byte group (SBO), k-step of 8 rows = +1024 B.
-                const uint64_t adh = smem_desc(a_hi + kk * 32, 16, 512, kSwizzle64B);
-                const uint64_t adl = smem_desc(a_lo + kk * 32, 16, 512, kSwizzle64B);
-                uint64_t bdh, bdl;
-                if (kNT) {
+                uint64_t adh, adl, bdh, bdl;
+                if (kMode == kModeTN) {
+                  adh = smem_desc(a_hi + kk * 1024, 32 * BK * 4, 512, kSwizzle128B32B);
+                  adl = smem_desc(a_lo + kk * 1024, 32 * BK * 4, 512, kSwizzle128B32B);
+                } else {
+                  adh = smem_desc(a_hi + kk * 32, 16, 512, kSwizzle64B);
+                  adl = smem_desc(a_lo + kk * 32, 16, 512, kSwizzle64B);
+                }
+                if (kMode == kModeNT) {
                   bdh = smem_desc(b_hi + kk * 32, 16, 512, kSwizzle64B);
                   bdl = smem_desc(b_lo + kk * 32, 16, 512, kSwizzle64B);
                 } else {
@@ -472,8 +522,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x / 2; tile < total && ok; tile += n_pairs) {
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        const TileCoord c = decode_tile<kMode>(s, args, n_tiles_n, nk, tile, rank);
+        for (int kb = 0; kb < c.nk; ++kb, ++it) {
           if ((int)(it % kNumSplitWarps) != ci) continue;
+          // kModeTN: rows past the expert's segment belong to the next expert
+          const int k_valid = kMode == kModeTN ? c.k_rows - kb * BK : BK;
           const uint32_t st = it % kStages, use = it / kStages;
           if (!mbar_wait(s, &s->full[st], use & 1, args.err)) { ok = false; break; }
           uint4* raw = reinterpret_cast<uint4*>(tiles + st * kStageBytes);
@@ -483,6 +536,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
             uint4 x[kBatch];
 #pragma unroll
             for (int j = 0; j < kBatch; ++j) x[j] = raw[b0 + 32 * j];
+            if (kMode == kModeTN && k_valid < BK) {
+              // MN-major tiles are [chunk][16 k-rows][128 B]: zero k-rows >= k_valid
+#pragma unroll
+              for (int j = 0; j < kBatch; ++j)
+                if ((((b0 + 32 * j) >> 3) & (BK - 1)) >= k_valid) {
+                  x[j] = make_uint4(0u, 0u, 0u, 0u);
+                  raw[b0 + 32 * j] = x[j];
+                }
+            }
 #pragma unroll
             for (int j = 0; j < kBatch; ++j)
               lo[b0 + 32 * j] = make_uint4(
@@ -560,22 +622,42 @@ bool map_b(CUtensorMap* m, const float* W, int E, int Kd, int N, bool nt) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// kModeTN operands: X [R, M] and Y [R, N] row-major, read as MN-major 32-column
+// boxes of 16 rows (128-byte swizzle with 32-byte atoms)
+bool map_rows_mn(CUtensorMap* m, const float* X, int64_t R, int cols) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)R};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+  cuuint32_t box[2] = {32, BK};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, (void*)X, dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Smem);
 
-template <bool kNT, int kEpi>
+// kModeNN/NT: C [R,N] = A [R,Kd] x W_e;  kModeTN: C [E,M,N] with C_e = A_e^T W_e
+// over expert e's rows of A [R,M] and W [R,N] (Kd unused).
+template <int kMode, int kEpi>
 janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, int N, float* C, float* C2,
-                    const float* aux, const int32_t* offsets, int32_t* err, cudaStream_t stream) {
+                    const float* aux, const int32_t* offsets, int32_t* err, cudaStream_t stream, int M = 0) {
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(tc_gemm_kernel<kNT, kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr = cudaFuncSetAttribute(tc_gemm_kernel<kMode, kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kSmemBytes);
   });
   if (attr != cudaSuccess) return JANUS_ERR_CUDA;
   CUtensorMap ma, mb;
-  if (!map_a(&ma, A, R, Kd) || !map_b(&mb, W, E, Kd, N, kNT)) return JANUS_ERR_CUDA;
+  if (kMode == kModeTN) {
+    if (!map_rows_mn(&ma, A, R, M) || !map_rows_mn(&mb, W, R, N)) return JANUS_ERR_CUDA;
+  } else if (!map_a(&ma, A, R, Kd) || !map_b(&mb, W, E, Kd, N, kMode == kModeNT)) {
+    return JANUS_ERR_CUDA;
+  }
   Args a;
-  a.C = C; a.C2 = C2; a.aux = aux; a.offsets = offsets; a.E = E; a.Kd = Kd; a.N = N; a.err = err;
+  a.C = C; a.C2 = C2; a.aux = aux; a.offsets = offsets; a.E = E; a.Kd = Kd; a.N = N; a.M = M; a.err = err;
   // one CTA per SM, in clusters of two (the MMA pairs)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(num_sms() / 2 * 2));
@@ -589,7 +671,7 @@ janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, in
   cluster_attr[0].val.clusterDim.z = 1;
   cfg.attrs = cluster_attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, tc_gemm_kernel<kNT, kEpi>, ma, mb, a) != cudaSuccess) return JANUS_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, tc_gemm_kernel<kMode, kEpi>, ma, mb, a) != cudaSuccess) return JANUS_ERR_CUDA;
   return launch_status();
 }
 
@@ -600,9 +682,9 @@ size_t workspace_extra() { return 0; }
 janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, int64_t R, int32_t d,
                             int32_t h, const float* w1, const float* w2, float* yd, float* act, float* H,
                             int32_t* err, cudaStream_t stream) {
-  janus_status st = launch<false, kEpiSilu>(xd, w1, R, E, d, h, H, act, nullptr, offsets, err, stream);
+  janus_status st = launch<kModeNN, kEpiSilu>(xd, w1, R, E, d, h, H, act, nullptr, offsets, err, stream);
   if (st != JANUS_OK) return st;
-  return launch<false, kEpiStore>(H, w2, R, E, h, d, yd, nullptr, nullptr, offsets, err, stream);
+  return launch<kModeNN, kEpiStore>(H, w2, R, E, h, d, yd, nullptr, nullptr, offsets, err, stream);
 }
 
 janus_status expert_ffn_vjp(const float* xd, const float* gd, const float* act_in, float* A,
@@ -611,12 +693,29 @@ janus_status expert_ffn_vjp(const float* xd, const float* gd, const float* act_i
                             cudaStream_t stream) {
   janus_status st;
   if (!act_in) {
-    st = launch<false, kEpiStore>(xd, w1, R, E, d, h, A, nullptr, nullptr, offsets, err, stream);
+    st = launch<kModeNN, kEpiStore>(xd, w1, R, E, d, h, A, nullptr, nullptr, offsets, err, stream);
     if (st != JANUS_OK) return st;
   }
-  st = launch<true, kEpiDSilu>(gd, w2, R, E, d, h, dA, nullptr, A, offsets, err, stream);
+  st = launch<kModeNT, kEpiDSilu>(gd, w2, R, E, d, h, dA, nullptr, A, offsets, err, stream);
   if (st != JANUS_OK) return st;
-  return launch<true, kEpiStore>(dA, w1, R, E, h, d, dxd, nullptr, nullptr, offsets, err, stream);
+  return launch<kModeNT, kEpiStore>(dA, w1, R, E, h, d, dxd, nullptr, nullptr, offsets, err, stream);
+}
+
+janus_status expert_ffn_weight_grad(const float* xd, const float* gd, const float* act_in, float* A,
+                                    const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
+                                    const float* w1, const float* w2, float* dw1, float* dw2, float* dA,
+                                    float* H, int32_t* err, cudaStream_t stream) {
+  janus_status st;
+  if (!act_in) {
+    st = launch<kModeNN, kEpiStore>(xd, w1, R, E, d, h, A, nullptr, nullptr, offsets, err, stream);
+    if (st != JANUS_OK) return st;
+  }
+  // dA = (gd W2^T) * silu'(a), and H = silu(a)
+  st = launch<kModeNT, kEpiDSilu>(gd, w2, R, E, d, h, dA, H, A, offsets, err, stream);
+  if (st != JANUS_OK) return st;
+  st = launch<kModeTN, kEpiStore>(xd, dA, R, E, 0, h, dw1, nullptr, nullptr, offsets, err, stream, d);
+  if (st != JANUS_OK) return st;
+  return launch<kModeTN, kEpiStore>(H, gd, R, E, 0, d, dw2, nullptr, nullptr, offsets, err, stream, h);
 }
 
 }  // namespace tc

@@ -21,5 +21,12 @@ janus_status expert_ffn_vjp(const float* xd, const float* gd, const float* act_i
                             const float* w1, const float* w2, float* dxd, float* dA, int32_t* err,
                             cudaStream_t stream);
 
+// Per-expert weight gradients: dW1[e] = Xd_e^T dA_e, dW2[e] = H_e^T Gd_e with
+// dA = (gd W2^T) * silu'(a) and H = silu(a) computed into dA and H.
+janus_status expert_ffn_weight_grad(const float* xd, const float* gd, const float* act_in, float* A,
+                                    const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
+                                    const float* w1, const float* w2, float* dw1, float* dw2, float* dA,
+                                    float* H, int32_t* err, cudaStream_t stream);
+
 }  // namespace tc
 }  // namespace janus

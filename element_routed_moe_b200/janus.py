@@ -34,6 +34,7 @@ SYMBOLS = (
     "janus_quant_by_type_workspace_size", "janus_quant_by_type", "janus_quant_by_type_noalloc",
     "janus_dequant_by_type",
     "janus_expert_ffn_workspace_size", "janus_expert_ffn_fwd", "janus_expert_ffn_vjp",
+    "janus_expert_ffn_weight_grad_workspace_size", "janus_expert_ffn_weight_grad",
     "janus_combine", "janus_edge_aggregate",
     "janus_debug_inject_launch_failures",
 )
@@ -80,6 +81,9 @@ def _declare(L):
                                       vp, sz, vp]),
         "janus_expert_ffn_vjp": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp,
                                       ctypes.c_int, vp, sz, vp]),
+        "janus_expert_ffn_weight_grad_workspace_size": (st, [i64, i32, i32, psz]),
+        "janus_expert_ffn_weight_grad": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp,
+                                              ctypes.c_int, vp, sz, vp]),
         "janus_combine": (st, [vp, vp, vp, i64, i32, i32, vp, vp]),
         "janus_edge_aggregate": (st, [vp, vp, i64, i32, vp, vp]),
         "janus_debug_inject_launch_failures": (None, [i32]),
@@ -314,6 +318,35 @@ def janus_expert_ffn_vjp(xd, gd, offsets, w1, w2, *, act=None, mode=JANUS_FFN_FP
                                       _p(out, torch.float32, "dxd"), int(mode), _p(ws), nb,
                                       _stream(stream)), "janus_expert_ffn_vjp")
     return out
+
+
+def janus_expert_ffn_weight_grad_workspace_size(n_rows, h, have_act) -> int:
+    b = ctypes.c_size_t(0)
+    _raise(lib().janus_expert_ffn_weight_grad_workspace_size(n_rows, h, int(bool(have_act)),
+                                                             ctypes.byref(b)),
+           "janus_expert_ffn_weight_grad_workspace_size")
+    return b.value
+
+
+def janus_expert_ffn_weight_grad(xd, gd, offsets, w1, w2, *, act=None, mode=JANUS_FFN_FP32_SIMT,
+                                 dw1=None, dw2=None, workspace=None, stream=None):
+    """Per-expert weight gradients; returns (dw1 [E,d,h], dw2 [E,h,d])."""
+    R, d = xd.shape
+    E, _, h = w1.shape
+    if dw1 is None:
+        dw1 = _empty((E, d, h), torch.float32, w1.device)
+    if dw2 is None:
+        dw2 = _empty((E, h, d), torch.float32, w1.device)
+    nb = janus_expert_ffn_weight_grad_workspace_size(R, h, act is not None)
+    ws = _workspace(nb, w1.device, workspace)
+    _raise(lib().janus_expert_ffn_weight_grad(_p(xd, torch.float32, "xd"), _p(gd, torch.float32, "gd"),
+                                              _p(act, torch.float32, "act"),
+                                              _p(offsets, torch.int32, "offsets"), E, R, d, h,
+                                              _p(w1, torch.float32, "w1"), _p(w2, torch.float32, "w2"),
+                                              _p(dw1, torch.float32, "dw1"), _p(dw2, torch.float32, "dw2"),
+                                              int(mode), _p(ws), nb, _stream(stream)),
+           "janus_expert_ffn_weight_grad")
+    return dw1, dw2
 
 
 # --------------------------------------------------------------------------

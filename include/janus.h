@@ -203,6 +203,23 @@ janus_status janus_expert_ffn_vjp(const float* xd, const float* gd, const float*
                                   float* dxd, janus_ffn_mode mode, void* workspace,
                                   size_t workspace_bytes, janus_stream_t stream);
 
+/* Expert weight gradients, the parameter side of the same backward pass
+ * (force training differentiates the energy w.r.t. inputs and weights,
+ * [Review] section 3.3).  For L = sum_p <yd[p,:], gd[p,:]>:
+ *   dW1[e] = sum_{p in expert e} xd[p,:]^T dA[p,:],  dA = (gd W2[e]^T) * silu'(a)
+ *   dW2[e] = sum_{p in expert e} silu(a[p,:])^T gd[p,:]
+ * out: dw1 [E,d,h], dw2 [E,h,d] float32 (overwritten; experts without rows
+ * get zeros).  act (nullable) is a from the forward; NULL recomputes it.
+ * workspace: janus_expert_ffn_weight_grad_workspace_size() bytes (dA, silu(a)
+ * and, without act, a: [R,h] each). */
+janus_status janus_expert_ffn_weight_grad_workspace_size(int64_t n_rows, int32_t h, int32_t have_act,
+                                                         size_t* bytes);
+janus_status janus_expert_ffn_weight_grad(const float* xd, const float* gd, const float* act,
+                                          const int32_t* offsets, int32_t n_experts, int64_t n_rows,
+                                          int32_t d, int32_t h, const float* w1, const float* w2,
+                                          float* dw1, float* dw2, janus_ffn_mode mode, void* workspace,
+                                          size_t workspace_bytes, janus_stream_t stream);
+
 /* -------------------------------------------------------------------------
  * Combine.  [Blueprint] section 3.2 (aggregation and output layer): the
  * activated experts' outputs are summed with the gate weights.  Gather form

@@ -306,13 +306,16 @@ void orc_expert_ffn_vjp(const float* xd, const float* gd, const int32_t* offsets
 void orc_expert_ffn_weight_grad(const float* xd, const float* gd, const int32_t* offsets,
                                 int32_t n_experts, int32_t d, int32_t h, const float* w1,
                                 const float* w2, float* dw1, float* dw2) {
-#pragma omp parallel for schedule(dynamic, 1)
   for (int e = 0; e < n_experts; ++e) {
     const float* W1 = w1 + (int64_t)e * d * h;
     const float* W2 = w2 + (int64_t)e * h * d;
-    std::vector<double> g1((size_t)d * h, 0.0), g2((size_t)h * d, 0.0), a(h), hh(h), da(h);
-    for (int64_t p = offsets[e]; p < offsets[e + 1]; ++p) {
-      std::fill(a.begin(), a.end(), 0.0);
+    const int64_t p0 = offsets[e], n = offsets[e + 1] - offsets[e];
+    // per row of the expert: hh = silu(a) and dA, in FP64
+    std::vector<double> hh((size_t)n * h), da((size_t)n * h);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n; ++r) {
+      const int64_t p = p0 + r;
+      std::vector<double> a(h, 0.0);
       for (int k = 0; k < d; ++k) {
         const double xk = xd[p * d + k];
         for (int j = 0; j < h; ++j) a[j] += xk * (double)W1[(int64_t)k * h + j];
@@ -321,16 +324,29 @@ void orc_expert_ffn_weight_grad(const float* xd, const float* gd, const int32_t*
         double dh = 0.0;
         for (int c = 0; c < d; ++c) dh += (double)W2[(int64_t)j * d + c] * (double)gd[p * d + c];
         const double sg = 1.0 / (1.0 + std::exp(-a[j]));
-        hh[j] = a[j] * sg;
-        da[j] = dh * sg * (1.0 + a[j] * (1.0 - sg));
+        hh[(size_t)r * h + j] = a[j] * sg;
+        da[(size_t)r * h + j] = dh * sg * (1.0 + a[j] * (1.0 - sg));
       }
-      for (int j = 0; j < h; ++j)
-        for (int c = 0; c < d; ++c) g2[(size_t)j * d + c] += hh[j] * (double)gd[p * d + c];
-      for (int k = 0; k < d; ++k)
-        for (int j = 0; j < h; ++j) g1[(size_t)k * h + j] += (double)xd[p * d + k] * da[j];
     }
-    for (size_t i = 0; i < g1.size(); ++i) dw1[(int64_t)e * d * h + i] = (float)g1[i];
-    for (size_t i = 0; i < g2.size(); ++i) dw2[(int64_t)e * h * d + i] = (float)g2[i];
+    // sums over the expert's rows in row order
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int k = 0; k < d; ++k) {
+      std::vector<double> acc(h, 0.0);
+      for (int64_t r = 0; r < n; ++r) {
+        const double xk = xd[(p0 + r) * d + k];
+        for (int j = 0; j < h; ++j) acc[j] += xk * da[(size_t)r * h + j];
+      }
+      for (int j = 0; j < h; ++j) dw1[(int64_t)e * d * h + (int64_t)k * h + j] = (float)acc[j];
+    }
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int j = 0; j < h; ++j) {
+      std::vector<double> acc(d, 0.0);
+      for (int64_t r = 0; r < n; ++r) {
+        const double hj = hh[(size_t)r * h + j];
+        for (int c = 0; c < d; ++c) acc[c] += hj * (double)gd[(p0 + r) * d + c];
+      }
+      for (int c = 0; c < d; ++c) dw2[(int64_t)e * h * d + (int64_t)j * d + c] = (float)acc[c];
+    }
   }
 }
 
