@@ -45,6 +45,9 @@ def _setup(L):
     L.orc_expert_ffn_weight_grad.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp, vp]
     L.orc_combine.argtypes = [vp, vp, vp, i64, i32, i32, vp]
     L.orc_edge_aggregate.argtypes = [vp, vp, i64, i32, vp]
+    L.orc_edge_broadcast.argtypes = [vp, vp, i64, i32, vp]
+    L.orc_neighbor_aggregate.argtypes = [vp, vp, vp, i64, i32, vp]
+    L.orc_neighbor_aggregate.restype = ctypes.c_int
 
 
 def _c(a, dtype):
@@ -189,4 +192,26 @@ def edge_aggregate(msg, row_ptr):
     d = msg.shape[1]
     out = np.empty((N, d), np.float32)
     lib().orc_edge_aggregate(_p(msg), _p(row_ptr), N, d, _p(out))
+    return out
+
+
+def edge_broadcast(dx, row_ptr):
+    """dmsg[e] = dx[receiver(e)] (the gradient of the edge aggregation)."""
+    dx = _c(dx, np.float32)
+    row_ptr = _c(row_ptr, np.int64)
+    N, d = dx.shape
+    dmsg = np.empty((int(row_ptr[-1]), d), np.float32)
+    lib().orc_edge_broadcast(_p(dx), _p(row_ptr), N, d, _p(dmsg))
+    return dmsg
+
+
+def neighbor_aggregate(x, row_ptr, senders):
+    """out[i] = sum over row i's edges of x[senders[e]]."""
+    x = _c(x, np.float32)
+    row_ptr = _c(row_ptr, np.int64)
+    senders = _c(senders, np.int32)
+    N, d = x.shape
+    out = np.empty((N, d), np.float32)
+    if lib().orc_neighbor_aggregate(_p(x), _p(row_ptr), _p(senders), N, d, _p(out)) != 0:
+        raise ValueError("oracle neighbor_aggregate: sender index out of range")
     return out

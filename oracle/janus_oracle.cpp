@@ -387,4 +387,33 @@ void orc_edge_aggregate(const float* msg, const int64_t* row_ptr, int64_t n_atom
   }
 }
 
+// ---------------------------------------------------------------------------
+// Edge-side neighbour operations ([Review] §3.5, CNIS kernels: neighbour
+// aggregation with fused indexing).  Reading: with the receiver-sorted CSR
+// (row_ptr, senders),
+//   gradient of the edge aggregation:  dmsg[e,:] = dX[i,:] for e in row i;
+//   neighbour aggregation by sender:   out[i,:] = sum_{e in row i} x[senders[e],:].
+// ---------------------------------------------------------------------------
+void orc_edge_broadcast(const float* dx, const int64_t* row_ptr, int64_t n_atoms, int32_t d,
+                        float* dmsg) {
+  for (int64_t i = 0; i < n_atoms; ++i)
+    for (int64_t e = row_ptr[i]; e < row_ptr[i + 1]; ++e)
+      for (int j = 0; j < d; ++j) dmsg[e * d + j] = dx[i * d + j];
+}
+
+int orc_neighbor_aggregate(const float* x, const int64_t* row_ptr, const int32_t* senders,
+                           int64_t n_atoms, int32_t d, float* out) {
+  std::vector<double> acc(d);
+  for (int64_t i = 0; i < n_atoms; ++i) {
+    std::fill(acc.begin(), acc.end(), 0.0);
+    for (int64_t e = row_ptr[i]; e < row_ptr[i + 1]; ++e) {
+      const int64_t s = senders[e];
+      if (s < 0 || s >= n_atoms) return -1;
+      for (int j = 0; j < d; ++j) acc[j] += (double)x[s * d + j];
+    }
+    for (int j = 0; j < d; ++j) out[i * d + j] = (float)acc[j];
+  }
+  return 0;
+}
+
 }  // extern "C"

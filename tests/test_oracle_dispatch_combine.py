@@ -85,3 +85,32 @@ def test_edge_aggregate_pbc_degrees():
     assert abs(deg.mean() - expect * (1999 / 2000)) < 0.05 * expect
     assert np.all(recv[:-1] <= recv[1:])
     assert not np.any(send == recv)
+
+
+def test_edge_broadcast_is_adjoint_of_edge_aggregate():
+    N, d = 300, 10
+    rp, send, recv = synth.edges_random(N, 12, seed=7)
+    msg = synth.normal((int(rp[-1]), d), 8).numpy()
+    dx = synth.normal((N, d), 9).numpy()
+    dmsg = oracle.edge_broadcast(dx, rp)
+    assert np.array_equal(dmsg, dx[recv])                 # NumPy gather, bit-exact
+    lhs = np.sum(oracle.edge_aggregate(msg, rp).astype(np.float64) * dx)
+    rhs = np.sum(msg.astype(np.float64) * dmsg)
+    assert abs(lhs - rhs) <= 1e-6 * (abs(lhs) + 1.0)
+
+
+def test_neighbor_aggregate_brute_force():
+    N, d = 257, 12
+    rp, send, recv = synth.edges_random(N, 16, seed=10)
+    x = synth.normal((N, d), 11).numpy()
+    out = oracle.neighbor_aggregate(x, rp, send.astype(np.int32))
+    ref = np.zeros((N, d), np.float64)
+    np.add.at(ref, recv, x[send].astype(np.float64))
+    assert np.array_equal(out, ref.astype(np.float32))
+    # the same as aggregating the gathered messages
+    assert np.array_equal(out, oracle.edge_aggregate(x[send], rp))
+    import pytest
+    bad = send.astype(np.int32).copy()
+    bad[3] = N
+    with pytest.raises(ValueError):
+        oracle.neighbor_aggregate(x, rp, bad)
