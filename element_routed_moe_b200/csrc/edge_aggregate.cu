@@ -13,7 +13,9 @@
 //     streaming load (evict-first, the messages are read exactly once);
 //   * one warp per atom, U = 4 column float4s per lane and the edge loop
 //     unrolled by 4 -> up to 16 independent 16-byte loads per lane in flight;
-//   * FP32 accumulation in edge order, each output row written once;
+//   * FP32 accumulation: each group of 4 edges is summed pairwise and then
+//     added to the running sum (edge order otherwise); each output row is
+//     written once;
 //   * 64-bit element offsets (Ed*d exceeds 2^31 at production sizes).
 #include "common.cuh"
 
@@ -23,6 +25,11 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kU = 4;
 constexpr int kEdgeUnroll = 4;
+static_assert(kEdgeUnroll == 4, "the pairwise group sum below is written for 4 edges");
+
+__device__ __forceinline__ float4 f4add(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
 
 __global__ void __launch_bounds__(kThreads)
 edge_aggregate_kernel(const float4* __restrict__ msg, const int64_t* __restrict__ row_ptr,
@@ -45,13 +52,13 @@ edge_aggregate_kernel(const float4* __restrict__ msg, const int64_t* __restrict_
             const int c = c0 + u * 32 + lane;
             v[r][u] = c < d4 ? __ldcs(msg + (e + r) * d4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
           }
+        // pairwise within the group of 4, then one add into the running sum
+        // (a 4x shorter rounding chain for high-degree receivers)
 #pragma unroll
-        for (int r = 0; r < kEdgeUnroll; ++r)
-#pragma unroll
-          for (int u = 0; u < kU; ++u) {
-            acc[u].x += v[r][u].x; acc[u].y += v[r][u].y;
-            acc[u].z += v[r][u].z; acc[u].w += v[r][u].w;
-          }
+        for (int u = 0; u < kU; ++u) {
+          const float4 a = f4add(v[0][u], v[1][u]), b = f4add(v[2][u], v[3][u]);
+          acc[u] = f4add(acc[u], f4add(a, b));
+        }
       }
       for (; e < e1; ++e) {
 #pragma unroll
@@ -60,6 +67,88 @@ edge_aggregate_kernel(const float4* __restrict__ msg, const int64_t* __restrict_
           if (c < d4) {
             const float4 v = __ldcs(msg + e * d4 + c);
             acc[u].x += v.x; acc[u].y += v.y; acc[u].z += v.z; acc[u].w += v.w;
+          }
+        }
+      }
+      float4* dst = out + i * d4;
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < d4) dst[c] = acc[u];
+      }
+    }
+  }
+}
+
+// Gradient of the edge aggregation: every edge of receiver i gets dX[i,:].
+// One warp per receiver: the dX row chunk is loaded once and written to the
+// receiver's contiguous block of edge rows with streaming stores.
+__global__ void __launch_bounds__(kThreads)
+edge_broadcast_kernel(const float4* __restrict__ dx, const int64_t* __restrict__ row_ptr, int64_t n_atoms,
+                      int d4, float4* __restrict__ dmsg) {
+  const int lane = threadIdx.x % 32;
+  const int64_t nwarps = (int64_t)gridDim.x * kThreads / 32;
+  for (int64_t i = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / 32; i < n_atoms; i += nwarps) {
+    const int64_t e0 = row_ptr[i], e1 = row_ptr[i + 1];
+    if (e1 <= e0) continue;
+    for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
+      float4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + u * 32 + lane;
+        v[u] = c < d4 ? __ldg(dx + i * d4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      for (int64_t e = e0; e < e1; ++e) {
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int c = c0 + u * 32 + lane;
+          if (c < d4) __stcs(dmsg + e * d4 + c, v[u]);
+        }
+      }
+    }
+  }
+}
+
+// Neighbour aggregation through the sender index: out[i,:] = sum over the
+// receiver's edges of x[senders[e],:].  One warp per receiver; the sender ids
+// of 32 edges are read with one coalesced load and broadcast by shuffles;
+// rows are gathered 4 edges at a time (U float4s each) for memory-level
+// parallelism; FP32 accumulation as in edge_aggregate_kernel.  Senders outside [0, N) are
+// skipped (they contribute nothing), so a bad index cannot read out of bounds.
+__global__ void __launch_bounds__(kThreads)
+neighbor_aggregate_kernel(const float4* __restrict__ x, const int64_t* __restrict__ row_ptr,
+                          const int32_t* __restrict__ senders, int64_t n_atoms, int d4,
+                          float4* __restrict__ out) {
+  const int lane = threadIdx.x % 32;
+  const int64_t nwarps = (int64_t)gridDim.x * kThreads / 32;
+  for (int64_t i = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / 32; i < n_atoms; i += nwarps) {
+    const int64_t e0 = row_ptr[i], e1 = row_ptr[i + 1];
+    for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
+      float4 acc[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int64_t eb = e0; eb < e1; eb += 32) {
+        const int64_t my_e = eb + lane;
+        int32_t my_s = my_e < e1 ? senders[my_e] : -1;
+        if (my_s >= n_atoms) my_s = -1;
+        const int n_here = (int)min((int64_t)32, e1 - eb);
+        for (int t = 0; t < n_here; t += 4) {
+          int32_t s4[4];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) s4[r] = __shfl_sync(0xffffffffu, my_s, (t + r) & 31);
+          float4 v[4][kU];
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+              const int c = c0 + u * 32 + lane;
+              const bool ok = (t + r < n_here) && s4[r] >= 0 && c < d4;
+              v[r][u] = ok ? __ldg(x + (int64_t)s4[r] * d4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const float4 a = f4add(v[0][u], v[1][u]), b = f4add(v[2][u], v[3][u]);
+            acc[u] = f4add(acc[u], f4add(a, b));
           }
         }
       }
@@ -94,5 +183,38 @@ extern "C" janus_status janus_edge_aggregate(const float* msg, const int64_t* ro
   const unsigned grid = (unsigned)(need < cap ? need : cap);
   edge_aggregate_kernel<<<grid, kThreads, 0, (cudaStream_t)stream>>>(
       (const float4*)msg, row_ptr, n_atoms, d / 4, (float4*)out);
+  return launch_status();
+}
+
+extern "C" janus_status janus_edge_broadcast(const float* dx, const int64_t* row_ptr, int64_t n_atoms,
+                                             int32_t d, float* dmsg, janus_stream_t stream) {
+  JANUS_CHECK_ARG(n_atoms >= 0 && d >= 1 && d <= kMaxDim);
+  JANUS_CHECK_ALIGN(d % 4 == 0);
+  if (n_atoms == 0) return JANUS_OK;
+  // dmsg may be NULL only for a CSR without edges
+  JANUS_CHECK_ARG(dx && row_ptr);
+  JANUS_CHECK_ALIGN(aligned(dx, 16) && aligned(dmsg, 16));
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  const int64_t need = (n_atoms + 7) / 8;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  edge_broadcast_kernel<<<(unsigned)(need < cap ? need : cap), kThreads, 0, (cudaStream_t)stream>>>(
+      (const float4*)dx, row_ptr, n_atoms, d / 4, (float4*)dmsg);
+  return launch_status();
+}
+
+extern "C" janus_status janus_neighbor_aggregate(const float* x, const int64_t* row_ptr,
+                                                 const int32_t* senders, int64_t n_atoms, int32_t d,
+                                                 float* out, janus_stream_t stream) {
+  JANUS_CHECK_ARG(n_atoms >= 0 && n_atoms < (int64_t)INT32_MAX && d >= 1 && d <= kMaxDim);
+  JANUS_CHECK_ALIGN(d % 4 == 0);
+  if (n_atoms == 0) return JANUS_OK;
+  // senders may be NULL only for a CSR without edges
+  JANUS_CHECK_ARG(x && row_ptr && out);
+  JANUS_CHECK_ALIGN(aligned(x, 16) && aligned(out, 16));
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  const int64_t need = (n_atoms + 7) / 8;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  neighbor_aggregate_kernel<<<(unsigned)(need < cap ? need : cap), kThreads, 0, (cudaStream_t)stream>>>(
+      (const float4*)x, row_ptr, senders, n_atoms, d / 4, (float4*)out);
   return launch_status();
 }

@@ -35,7 +35,7 @@ SYMBOLS = (
     "janus_dequant_by_type",
     "janus_expert_ffn_workspace_size", "janus_expert_ffn_fwd", "janus_expert_ffn_vjp",
     "janus_expert_ffn_weight_grad_workspace_size", "janus_expert_ffn_weight_grad",
-    "janus_combine", "janus_edge_aggregate",
+    "janus_combine", "janus_edge_aggregate", "janus_edge_broadcast", "janus_neighbor_aggregate",
     "janus_debug_inject_launch_failures",
 )
 
@@ -86,6 +86,8 @@ def _declare(L):
                                               ctypes.c_int, vp, sz, vp]),
         "janus_combine": (st, [vp, vp, vp, i64, i32, i32, vp, vp]),
         "janus_edge_aggregate": (st, [vp, vp, i64, i32, vp, vp]),
+        "janus_edge_broadcast": (st, [vp, vp, i64, i32, vp, vp]),
+        "janus_neighbor_aggregate": (st, [vp, vp, vp, i64, i32, vp, vp]),
         "janus_debug_inject_launch_failures": (None, [i32]),
     }
     for name, (res, args) in sig.items():
@@ -361,6 +363,29 @@ def janus_edge_aggregate(msg, row_ptr, *, out=None, stream=None):
                                       _p(row_ptr, torch.int64, "row_ptr"), N, d,
                                       _p(out, torch.float32, "out"), _stream(stream)),
            "janus_edge_aggregate")
+    return out
+
+
+def janus_edge_broadcast(dx, row_ptr, *, out=None, stream=None):
+    """dmsg[e] = dx[receiver(e)] over a receiver-sorted CSR."""
+    N, d = dx.shape
+    if out is None:
+        out = _empty((int(row_ptr[-1].item()) if row_ptr.numel() else 0, d), torch.float32, dx.device)
+    _raise(lib().janus_edge_broadcast(_p(dx, torch.float32, "dx"), _p(row_ptr, torch.int64, "row_ptr"),
+                                      N, d, _p(out, torch.float32, "dmsg"), _stream(stream)),
+           "janus_edge_broadcast")
+    return out
+
+
+def janus_neighbor_aggregate(x, row_ptr, senders, *, out=None, stream=None):
+    """out[i] = sum over row i's edges of x[senders[e]]."""
+    N, d = x.shape
+    if out is None:
+        out = _empty((N, d), torch.float32, x.device)
+    _raise(lib().janus_neighbor_aggregate(_p(x, torch.float32, "x"), _p(row_ptr, torch.int64, "row_ptr"),
+                                          _p(senders, torch.int32, "senders"), N, d,
+                                          _p(out, torch.float32, "out"), _stream(stream)),
+           "janus_neighbor_aggregate")
     return out
 
 

@@ -243,6 +243,23 @@ janus_status janus_combine(const float* yd, const int32_t* slot_of, const float*
 janus_status janus_edge_aggregate(const float* msg, const int64_t* row_ptr, int64_t n_atoms,
                                   int32_t d, float* out, janus_stream_t stream);
 
+/* Gradient of the edge aggregation (same passage): every edge of receiver i
+ * receives that atom's gradient row,  dmsg[e,:] = dx[i,:]  for e in
+ * [row_ptr[i], row_ptr[i+1]).  in : dx [N,d], row_ptr [N+1];  out: dmsg [Ed,d]
+ * (may be NULL only when Ed == 0). */
+janus_status janus_edge_broadcast(const float* dx, const int64_t* row_ptr, int64_t n_atoms,
+                                  int32_t d, float* dmsg, janus_stream_t stream);
+
+/* Neighbour aggregation with fused indexing ([Review] section 3.5, CNIS
+ * kernels): node features are gathered through the sender index instead of a
+ * materialised message buffer,
+ *   out[i,:] = sum_{e in [row_ptr[i], row_ptr[i+1])} x[senders[e], :]
+ * in : x [N,d] float32, row_ptr [N+1] int64, senders [Ed] int32 (may be NULL
+ * only when Ed == 0);  out: out [N,d].  Sender ids outside [0,N) are skipped
+ * (they add nothing).  N < 2^31. */
+janus_status janus_neighbor_aggregate(const float* x, const int64_t* row_ptr, const int32_t* senders,
+                                      int64_t n_atoms, int32_t d, float* out, janus_stream_t stream);
+
 /* Host-side fault injection for tests: the next `n_calls` library calls that
  * would launch work return JANUS_ERR_CUDA before launching anything. */
 void janus_debug_inject_launch_failures(int32_t n_calls);

@@ -81,3 +81,66 @@ def _colsum64(t, chunk=1 << 18):
     for i in range(0, t.shape[0], chunk):
         acc += t[i:i + chunk].to(torch.float64).sum(0)
     return acc
+
+
+# ---- gradient of the edge aggregation, and neighbour aggregation by sender ----
+
+def test_edge_broadcast_bit_exact():
+    deg = np.array([0, 1, 4096, 0, 3, 5, 7, 0, 2, 9, 0], np.int64)
+    rp = np.concatenate([[0], np.cumsum(deg)]).astype(np.int64)
+    for d in (4, 4 * 37, 4 * 300):
+        dx = synth.normal((len(deg), d), 5, DEV)
+        out = poison_like((int(rp[-1]), d), torch.float32)
+        J.janus_edge_broadcast(dx, to_dev(rp), out=out)
+        assert np.array_equal(host(out), oracle.edge_broadcast(host(dx), rp))
+
+
+def test_edge_broadcast_adjoint_on_gpu():
+    rp, _, _ = synth.edges_random(512, 16, seed=6)
+    msg = synth.normal((int(rp[-1]), 64), 8, DEV)
+    dx = synth.normal((512, 64), 9, DEV)
+    x = J.janus_edge_aggregate(msg, to_dev(rp))
+    dmsg = J.janus_edge_broadcast(dx, to_dev(rp))
+    lhs = float((x.double() * dx.double()).sum())
+    rhs = float((msg.double() * dmsg.double()).sum())
+    assert abs(lhs - rhs) <= 1e-5 * (abs(lhs) + 1.0)
+
+
+@pytest.mark.parametrize("d", [4, 64, 4 * 37, 4 * 300])
+def test_neighbor_aggregate_small(d):
+    rp, send, _ = synth.edges_random(700, 16, seed=12)
+    x = synth.normal((700, d), 13, DEV)
+    out = poison_like((700, d), torch.float32)
+    J.janus_neighbor_aggregate(x, to_dev(rp), to_dev(send.astype(np.int32)), out=out)
+    ref = oracle.neighbor_aggregate(host(x), rp, send.astype(np.int32))
+    assert rel_fro(host(out), ref) <= TOL_FP32
+    deg = np.diff(rp)
+    assert np.all(host(out)[deg == 0] == 0)
+
+
+def test_neighbor_aggregate_degenerate_and_bad_senders():
+    deg = np.array([0, 1, 4096, 0, 33, 31, 32, 64, 0], np.int64)
+    rp = np.concatenate([[0], np.cumsum(deg)]).astype(np.int64)
+    N = len(deg)
+    send = np.random.default_rng(3).integers(0, N, int(rp[-1])).astype(np.int32)
+    x = synth.normal((N, 4 * 40), 14, DEV)
+    out = J.janus_neighbor_aggregate(x, to_dev(rp), to_dev(send))
+    assert rel_fro(host(out), oracle.neighbor_aggregate(host(x), rp, send)) <= TOL_FP32
+    # out-of-range senders add nothing
+    bad = send.copy()
+    bad[5] = N + 7
+    bad[100] = -2
+    out2 = J.janus_neighbor_aggregate(x, to_dev(rp), to_dev(bad))
+    mask = (bad < 0) | (bad >= N)
+    xs = np.vstack([host(x), np.zeros((1, x.shape[1]), np.float32)])   # row N is zero
+    ref2 = oracle.edge_aggregate(xs[np.where(mask, N, bad)], rp)
+    assert rel_fro(host(out2), ref2) <= TOL_FP32
+
+
+def test_neighbor_aggregate_full_size_L():
+    cfg = synth.CONFIGS["L"]
+    rp, send, _ = synth.edges_pbc(cfg.n_atoms, seed=6)
+    x = synth.normal((cfg.n_atoms, cfg.d), 8, DEV)
+    out = J.janus_neighbor_aggregate(x, to_dev(rp), to_dev(send.astype(np.int32)))
+    ref = oracle.neighbor_aggregate(host(x), rp, send.astype(np.int32))
+    assert rel_fro(host(out), ref) <= TOL_FP32
