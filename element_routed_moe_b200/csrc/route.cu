@@ -6,6 +6,10 @@
 // type activates its own top-K experts); ScienceAI article (JIT planning:
 // route before the step, count per-expert token load).
 //
+// janus_route_layers routes several MoE layers' gate tables for the same atoms
+// in the same four launches (grid dimension y = layer), as JIT planning does
+// for all layers of a step before it runs.
+//
 // Design (four launches, no host sync, no inter-CTA spin-wait):
 //   1. route_table   one warp per element type: top-K of the gate row by K
 //                    rounds of warp argmax, softmax weights in FP64.  The
@@ -30,25 +34,29 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxBlocks = 2048;       // route_scan handles up to 8 per thread
 
+// Workspace: header | per-layer ticket counters [nl] | per-type tables
+// [nl][T][K] (experts, weights) | per-block expert counts [nl][E][n_blocks].
 struct RouteLayout {
   int64_t atoms_per_block;
   int64_t n_blocks;
-  size_t off_table_e, off_table_w, off_blockcnt, total;
+  size_t off_done, off_table_e, off_table_w, off_blockcnt, total;
 };
 
-RouteLayout route_layout(int64_t n_atoms, int32_t T, int32_t E, int32_t K) {
+RouteLayout route_layout(int64_t n_atoms, int32_t T, int32_t E, int32_t K, int32_t nl) {
   RouteLayout L;
   int64_t apb = 64;
   if (n_atoms > apb * kMaxBlocks) apb = (n_atoms + kMaxBlocks - 1) / kMaxBlocks;
   L.atoms_per_block = apb;
   L.n_blocks = n_atoms > 0 ? (n_atoms + apb - 1) / apb : 0;
   size_t off = sizeof(WsHeader);
+  L.off_done = off;
+  off = align_up(off + sizeof(uint32_t) * (size_t)nl, 256);
   L.off_table_e = off;
-  off = align_up(off + sizeof(int32_t) * (size_t)T * K, 256);
+  off = align_up(off + sizeof(int32_t) * (size_t)nl * T * K, 256);
   L.off_table_w = off;
-  off = align_up(off + sizeof(float) * (size_t)T * K, 256);
+  off = align_up(off + sizeof(float) * (size_t)nl * T * K, 256);
   L.off_blockcnt = off;
-  off = align_up(off + sizeof(int32_t) * (size_t)E * (L.n_blocks > 0 ? L.n_blocks : 1), 256);
+  off = align_up(off + sizeof(int32_t) * (size_t)nl * E * (L.n_blocks > 0 ? L.n_blocks : 1), 256);
   L.total = off;
   return L;
 }
@@ -62,6 +70,10 @@ __global__ void __launch_bounds__(kThreads)
 route_table(const float* __restrict__ gate, int32_t T, int32_t E, int32_t K,
             int32_t* __restrict__ table_e, float* __restrict__ table_w) {
   __shared__ float sel_logit[kWarps][kMaxExperts];
+  // layer blockIdx.y: gate [T,E] and tables [T,K] of that layer
+  gate += (int64_t)blockIdx.y * T * E;
+  table_e += (int64_t)blockIdx.y * T * K;
+  table_w += (int64_t)blockIdx.y * T * K;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int t = blockIdx.x * kWarps + warp;
   if (t >= T) return;
@@ -118,6 +130,14 @@ route_count(const int32_t* __restrict__ types, int64_t n_atoms, int32_t T, int32
             int64_t atoms_per_block, int64_t n_blocks, int32_t* __restrict__ topk_e,
             float* __restrict__ topk_w, int32_t* __restrict__ blockcnt, WsHeader* ws) {
   __shared__ int32_t cnt[kMaxExperts];
+  {  // layer blockIdx.y (types are shared by all layers)
+    const int64_t l = blockIdx.y;
+    table_e += l * T * K;
+    table_w += l * T * K;
+    topk_e += l * n_atoms * K;
+    topk_w += l * n_atoms * K;
+    blockcnt += l * E * n_blocks;
+  }
   for (int e = threadIdx.x; e < E; e += kThreads) cnt[e] = 0;
   __syncthreads();
   const int64_t a0 = (int64_t)blockIdx.x * atoms_per_block;
@@ -166,8 +186,15 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* total) {
 
 __global__ void __launch_bounds__(kThreads)
 route_scan(int32_t E, int64_t n_blocks, int32_t* __restrict__ blockcnt,
-           int32_t* __restrict__ counts, int32_t* __restrict__ offsets, WsHeader* ws) {
+           int32_t* __restrict__ counts, int32_t* __restrict__ offsets, uint32_t* done) {
   __shared__ bool is_last;
+  {  // layer blockIdx.y
+    const int64_t l = blockIdx.y;
+    blockcnt += l * E * n_blocks;
+    counts += l * E;
+    offsets += l * (E + 1);
+    done += l;
+  }
   const int e = blockIdx.x;
   int32_t* col = blockcnt + (int64_t)e * n_blocks;
   const int per = (int)((n_blocks + kThreads - 1) / kThreads);   // <= 8
@@ -189,7 +216,7 @@ route_scan(int32_t E, int64_t n_blocks, int32_t* __restrict__ blockcnt,
   if (threadIdx.x == 0) {
     counts[e] = total;
     __threadfence();
-    is_last = (atomicAdd(&ws->done, 1u) == (unsigned)E - 1);
+    is_last = (atomicAdd(done, 1u) == (unsigned)E - 1);
   }
   __syncthreads();
   if (!is_last) return;
@@ -201,7 +228,7 @@ route_scan(int32_t E, int64_t n_blocks, int32_t* __restrict__ blockcnt,
   if (threadIdx.x < E) offsets[threadIdx.x] = pre;
   if (threadIdx.x == 0) {
     offsets[E] = tot;
-    ws->done = 0;
+    *done = 0;
   }
 }
 
@@ -212,6 +239,14 @@ route_scatter(int64_t n_atoms, int32_t E, int32_t K, int64_t atoms_per_block, in
               int32_t* __restrict__ slot_of) {
   __shared__ int32_t wcnt[kWarps][kMaxExperts];
   __shared__ int32_t base[kMaxExperts];
+  {  // layer blockIdx.y
+    const int64_t l = blockIdx.y, R = n_atoms * K;
+    topk_e += l * R;
+    blockcnt += l * E * n_blocks;
+    offsets += l * (E + 1);
+    perm += l * R;
+    slot_of += l * R;
+  }
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   for (int e = threadIdx.x; e < E; e += kThreads) {
     base[e] = offsets[e] + blockcnt[(int64_t)e * n_blocks + blockIdx.x];
@@ -255,14 +290,61 @@ route_scatter(int64_t n_atoms, int32_t E, int32_t K, int64_t atoms_per_block, in
 
 using namespace janus;
 
+static janus_status route_check(int64_t n_atoms, int32_t n_types, int32_t n_experts, int32_t top_k,
+                                int32_t n_layers) {
+  JANUS_CHECK_ARG(n_atoms >= 0 && n_types >= 1 && n_types <= kMaxTypes);
+  JANUS_CHECK_ARG(n_experts >= 1 && n_experts <= kMaxExperts && top_k >= 1 && top_k <= n_experts);
+  JANUS_CHECK_ARG(n_atoms * (int64_t)top_k < (int64_t)INT32_MAX);
+  JANUS_CHECK_ARG(n_layers >= 1 && n_layers <= 65535);
+  return JANUS_OK;
+}
+
+// Routes n_layers gate tables [nl][T][E] for the same atoms in one set of four
+// launches (grid dimension y = layer); outputs are stacked per layer.
+static janus_status route_impl(const int32_t* types, int64_t n_atoms, const float* gates, int32_t nl,
+                               int32_t T, int32_t E, int32_t K, int32_t* topk_expert, float* topk_weight,
+                               int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* slot_of,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  janus_status st = route_check(n_atoms, T, E, K, nl);
+  if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(gates && counts && offsets && workspace);
+  JANUS_CHECK_ARG(n_atoms == 0 || (types && topk_expert && topk_weight && perm && slot_of));
+  const RouteLayout L = route_layout(n_atoms, T, E, K, nl);
+  JANUS_CHECK_ARG(workspace_bytes >= L.total);
+  JANUS_CHECK_ALIGN(aligned(workspace, 256));
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+
+  char* w = (char*)workspace;
+  WsHeader* hdr = (WsHeader*)w;
+  uint32_t* done = (uint32_t*)(w + L.off_done);
+  int32_t* table_e = (int32_t*)(w + L.off_table_e);
+  float* table_w = (float*)(w + L.off_table_w);
+  int32_t* blockcnt = (int32_t*)(w + L.off_blockcnt);
+
+  JANUS_CUDA_TRY(cudaMemsetAsync(hdr, 0, L.off_table_e, stream));   // header + ticket counters
+  if (n_atoms == 0) {
+    JANUS_CUDA_TRY(cudaMemsetAsync(counts, 0, sizeof(int32_t) * E * nl, stream));
+    JANUS_CUDA_TRY(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1) * nl, stream));
+    return JANUS_OK;
+  }
+  const unsigned nb = (unsigned)L.n_blocks, ly = (unsigned)nl;
+  route_table<<<dim3((T + kWarps - 1) / kWarps, ly), kThreads, 0, stream>>>(gates, T, E, K, table_e, table_w);
+  route_count<<<dim3(nb, ly), kThreads, 0, stream>>>(types, n_atoms, T, E, K, table_e, table_w,
+                                                      L.atoms_per_block, L.n_blocks, topk_expert,
+                                                      topk_weight, blockcnt, hdr);
+  route_scan<<<dim3(E, ly), kThreads, 0, stream>>>(E, L.n_blocks, blockcnt, counts, offsets, done);
+  route_scatter<<<dim3(nb, ly), kThreads, 0, stream>>>(n_atoms, E, K, L.atoms_per_block, L.n_blocks,
+                                                        topk_expert, blockcnt, offsets, perm, slot_of);
+  return launch_status();
+}
+
 extern "C" janus_status janus_route_workspace_size(int64_t n_atoms, int32_t n_types,
                                                    int32_t n_experts, int32_t top_k,
                                                    size_t* bytes) {
   JANUS_CHECK_ARG(bytes != nullptr);
-  JANUS_CHECK_ARG(n_atoms >= 0 && n_types >= 1 && n_types <= kMaxTypes);
-  JANUS_CHECK_ARG(n_experts >= 1 && n_experts <= kMaxExperts && top_k >= 1 && top_k <= n_experts);
-  JANUS_CHECK_ARG(n_atoms * (int64_t)top_k < (int64_t)INT32_MAX);
-  *bytes = route_layout(n_atoms, n_types, n_experts, top_k).total;
+  janus_status st = route_check(n_atoms, n_types, n_experts, top_k, 1);
+  if (st != JANUS_OK) return st;
+  *bytes = route_layout(n_atoms, n_types, n_experts, top_k, 1).total;
   return JANUS_OK;
 }
 
@@ -271,37 +353,27 @@ extern "C" janus_status janus_route(const int32_t* types, int64_t n_atoms, const
                                     int32_t* topk_expert, float* topk_weight, int32_t* counts,
                                     int32_t* offsets, int32_t* perm, int32_t* slot_of,
                                     void* workspace, size_t workspace_bytes,
-                                    janus_stream_t stream_) {
-  cudaStream_t stream = (cudaStream_t)stream_;
-  size_t need = 0;
-  janus_status st = janus_route_workspace_size(n_atoms, n_types, n_experts, top_k, &need);
+                                    janus_stream_t stream) {
+  return route_impl(types, n_atoms, gate, 1, n_types, n_experts, top_k, topk_expert, topk_weight,
+                    counts, offsets, perm, slot_of, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+extern "C" janus_status janus_route_layers_workspace_size(int64_t n_atoms, int32_t n_types,
+                                                          int32_t n_experts, int32_t top_k,
+                                                          int32_t n_layers, size_t* bytes) {
+  JANUS_CHECK_ARG(bytes != nullptr);
+  janus_status st = route_check(n_atoms, n_types, n_experts, top_k, n_layers);
   if (st != JANUS_OK) return st;
-  JANUS_CHECK_ARG(gate && counts && offsets && workspace);
-  JANUS_CHECK_ARG(n_atoms == 0 || (types && topk_expert && topk_weight && perm && slot_of));
-  JANUS_CHECK_ARG(workspace_bytes >= need);
-  JANUS_CHECK_ALIGN(aligned(workspace, 256));
-  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  *bytes = route_layout(n_atoms, n_types, n_experts, top_k, n_layers).total;
+  return JANUS_OK;
+}
 
-  const int32_t T = n_types, E = n_experts, K = top_k;
-  RouteLayout L = route_layout(n_atoms, T, E, K);
-  char* w = (char*)workspace;
-  WsHeader* hdr = (WsHeader*)w;
-  int32_t* table_e = (int32_t*)(w + L.off_table_e);
-  float* table_w = (float*)(w + L.off_table_w);
-  int32_t* blockcnt = (int32_t*)(w + L.off_blockcnt);
-
-  JANUS_CUDA_TRY(cudaMemsetAsync(hdr, 0, sizeof(WsHeader), stream));
-  if (n_atoms == 0) {
-    JANUS_CUDA_TRY(cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, stream));
-    JANUS_CUDA_TRY(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), stream));
-    return JANUS_OK;
-  }
-  route_table<<<(T + kWarps - 1) / kWarps, kThreads, 0, stream>>>(gate, T, E, K, table_e, table_w);
-  route_count<<<(unsigned)L.n_blocks, kThreads, 0, stream>>>(
-      types, n_atoms, T, E, K, table_e, table_w, L.atoms_per_block, L.n_blocks, topk_expert,
-      topk_weight, blockcnt, hdr);
-  route_scan<<<E, kThreads, 0, stream>>>(E, L.n_blocks, blockcnt, counts, offsets, hdr);
-  route_scatter<<<(unsigned)L.n_blocks, kThreads, 0, stream>>>(
-      n_atoms, E, K, L.atoms_per_block, L.n_blocks, topk_expert, blockcnt, offsets, perm, slot_of);
-  return launch_status();
+extern "C" janus_status janus_route_layers(const int32_t* types, int64_t n_atoms, const float* gates,
+                                           int32_t n_layers, int32_t n_types, int32_t n_experts,
+                                           int32_t top_k, int32_t* topk_expert, float* topk_weight,
+                                           int32_t* counts, int32_t* offsets, int32_t* perm,
+                                           int32_t* slot_of, void* workspace, size_t workspace_bytes,
+                                           janus_stream_t stream) {
+  return route_impl(types, n_atoms, gates, n_layers, n_types, n_experts, top_k, topk_expert, topk_weight,
+                    counts, offsets, perm, slot_of, workspace, workspace_bytes, (cudaStream_t)stream);
 }

@@ -30,6 +30,7 @@ JANUS_FFN_3XTF32 = 1
 SYMBOLS = (
     "janus_status_string", "janus_version", "janus_check",
     "janus_route_workspace_size", "janus_route",
+    "janus_route_layers_workspace_size", "janus_route_layers",
     "janus_dispatch",
     "janus_quant_by_type_workspace_size", "janus_quant_by_type", "janus_quant_by_type_noalloc",
     "janus_dequant_by_type",
@@ -71,6 +72,9 @@ def _declare(L):
         "janus_check": (st, [vp, vp]),
         "janus_route_workspace_size": (st, [i64, i32, i32, i32, psz]),
         "janus_route": (st, [vp, i64, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "janus_route_layers_workspace_size": (st, [i64, i32, i32, i32, i32, psz]),
+        "janus_route_layers": (st, [vp, i64, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz,
+                                    vp]),
         "janus_dispatch": (st, [vp, i64, i32, i32, vp, vp, vp, vp]),
         "janus_quant_by_type_workspace_size": (st, [i32, psz]),
         "janus_quant_by_type": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp, sz, vp]),
@@ -172,6 +176,37 @@ def janus_route(types, gate, top_k, *, out=None, workspace=None, stream=None):
                              T, E, K, _p(out["topk_expert"]), _p(out["topk_weight"]),
                              _p(out["counts"]), _p(out["offsets"]), _p(out["perm"]),
                              _p(out["slot_of"]), _p(ws), nb, _stream(stream)), "janus_route")
+    out["workspace"] = ws
+    return out
+
+
+def janus_route_layers_workspace_size(n_atoms, n_types, n_experts, top_k, n_layers) -> int:
+    b = ctypes.c_size_t(0)
+    _raise(lib().janus_route_layers_workspace_size(n_atoms, n_types, n_experts, top_k, n_layers,
+                                                   ctypes.byref(b)), "janus_route_layers_workspace_size")
+    return b.value
+
+
+def janus_route_layers(types, gates, top_k, *, workspace=None, stream=None):
+    """Routes gates [L,T,E] for the same atoms; returns per-layer stacked
+    device tensors (topk_expert [L,N,K], ..., offsets [L,E+1], perm [L,R])."""
+    dev = gates.device
+    N = types.shape[0]
+    L, T, E = gates.shape
+    K = int(top_k)
+    R = N * K
+    out = dict(topk_expert=_empty((L, N, K), torch.int32, dev),
+               topk_weight=_empty((L, N, K), torch.float32, dev),
+               counts=_empty((L, E), torch.int32, dev),
+               offsets=_empty((L, E + 1), torch.int32, dev),
+               perm=_empty((L, R), torch.int32, dev),
+               slot_of=_empty((L, R), torch.int32, dev))
+    nb = janus_route_layers_workspace_size(N, T, E, K, L)
+    ws = _workspace(nb, dev, workspace)
+    _raise(lib().janus_route_layers(_p(types, torch.int32, "types"), N, _p(gates, torch.float32, "gates"),
+                                    L, T, E, K, _p(out["topk_expert"]), _p(out["topk_weight"]),
+                                    _p(out["counts"]), _p(out["offsets"]), _p(out["perm"]),
+                                    _p(out["slot_of"]), _p(ws), nb, _stream(stream)), "janus_route_layers")
     out["workspace"] = ws
     return out
 

@@ -100,6 +100,21 @@ janus_status janus_route(const int32_t* types, int64_t n_atoms, const float* gat
                          void* workspace, size_t workspace_bytes,
                          janus_stream_t stream);
 
+/* Routing of several MoE layers at once, as JIT planning does for every MoE
+ * layer of a step before it runs ([News], training-framework paragraph: route
+ * all layers in a batch, count each expert's token load).  gates is
+ * [L][T][E]; every output is stacked per layer: topk_expert/topk_weight
+ * [L][N][K], counts [L][E], offsets [L][E+1], perm/slot_of [L][R].  Layer l's
+ * outputs equal janus_route(types, gates[l]).  1 <= L <= 65535; the workspace
+ * grows with L (janus_route_layers_workspace_size). */
+janus_status janus_route_layers_workspace_size(int64_t n_atoms, int32_t n_types, int32_t n_experts,
+                                               int32_t top_k, int32_t n_layers, size_t* bytes);
+janus_status janus_route_layers(const int32_t* types, int64_t n_atoms, const float* gates,
+                                int32_t n_layers, int32_t n_types, int32_t n_experts, int32_t top_k,
+                                int32_t* topk_expert, float* topk_weight, int32_t* counts,
+                                int32_t* offsets, int32_t* perm, int32_t* slot_of, void* workspace,
+                                size_t workspace_bytes, janus_stream_t stream);
+
 /* -------------------------------------------------------------------------
  * Dispatch.  [Review] section 3.5 (CNIS kernels, MoE dispatch/combine).
  *   xd[slot_of[i*K+k], :] = x[i, :] * (topk_weight ? topk_weight[i*K+k] : 1)

@@ -124,3 +124,31 @@ def test_injected_failure_with_real_buffers():
     assert e.value.status == J.JANUS_ERR_CUDA
     r = J.janus_route(to_dev(types), to_dev(gate), 2)
     J.janus_check(r["workspace"])
+
+
+# ---- several MoE layers routed at once (JIT planning) ----
+
+@pytest.mark.parametrize("shape", [(8192, 89, 72, 4, 12), (3001, 13, 24, 7, 3), (700, 30, 256, 200, 2)])
+def test_route_layers_match_per_layer_oracle(shape):
+    N, T, E, K, L = shape
+    types = synth.types_zipf(N, T, seed=3)
+    gates = np.stack([synth.gate_table(T, E, 100 + l) for l in range(L)])
+    r = J.janus_route_layers(to_dev(types), to_dev(gates), K)
+    J.janus_check(r["workspace"])
+    for l in range(L):
+        ref = oracle.route(types, gates[l], K)
+        got = {k: host(v[l]) for k, v in r.items() if k != "workspace"}
+        got["topk_expert"] = got["topk_expert"].reshape(N, K)
+        got["topk_weight"] = got["topk_weight"].reshape(N, K)
+        _compare(got, ref)
+
+
+def test_route_layers_zero_atoms_and_bad_type():
+    gates = np.stack([synth.gate_table(4, 6, l) for l in range(3)])
+    r = J.janus_route_layers(torch.empty(0, dtype=torch.int32, device=DEV), to_dev(gates), 2)
+    J.janus_check(r["workspace"])
+    assert np.all(host(r["counts"]) == 0) and np.all(host(r["offsets"]) == 0)
+    r = J.janus_route_layers(to_dev(np.array([0, 9, 1], np.int32)), to_dev(gates), 2)
+    with pytest.raises(J.JanusError) as e:
+        J.janus_check(r["workspace"])
+    assert e.value.status == J.JANUS_ERR_DATA
