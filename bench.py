@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--atoms", type=int, default=None, help="override N (profiling small cases)")
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling small cases)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip timing the weight-gradient, multi-layer routing and edge-side calls")
     ap.add_argument("--ref-seconds", type=float, default=None,
                     help="reference arm: target seconds of oracle work per step")
     return ap.parse_args()
@@ -505,6 +507,8 @@ def run_janus(args, world, rank, local):
 
     if not args.no_e2e and not layer.slice:
         line["e2e"] = run_e2e(layer, args)
+    if not args.no_extras:
+        line["extras"] = run_extras(layer, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host = host_inputs(cfg, layer)
         n_s = oracle_calibrate(cfg, host, 15.0)
@@ -517,6 +521,61 @@ def run_janus(args, world, rank, local):
                       f"full expert weights, {dt:.1f} s; host {cpu_descr()}"}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def _time_ms(fn, reps=5):
+    fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def run_extras(layer, peaks):
+    """Calls outside the layer pass, timed separately (not part of `value`):
+    expert weight gradients, routing of 12 MoE layers at once vs one by one,
+    and (slice workload) the edge-side gradient and sender-indexed gather."""
+    J = layer.J
+    cfg = layer.cfg
+    N, R, d, h, E, K, T = cfg.n_atoms, cfg.n_rows, cfg.d, cfg.h, cfg.n_experts, cfg.top_k, cfg.n_types
+    r = layer.route_out
+    out = {}
+    dw1 = torch.empty_like(layer.w1)
+    dw2 = torch.empty_like(layer.w2)
+    ws = torch.empty(J.janus_expert_ffn_weight_grad_workspace_size(R, h, True), dtype=torch.uint8,
+                     device=layer.x.device)
+    ms = _time_ms(lambda: J.janus_expert_ffn_weight_grad(layer.xd, layer.gd, r["offsets"], layer.w1, layer.w2,
+                                                          act=layer.act, mode=layer.mode, dw1=dw1, dw2=dw2,
+                                                          workspace=ws))
+    out["expert_weight_grad"] = {"ms": ms, "gemms": 3, "TFLOP/s": 6 * R * d * h / (ms * 1e-3) / 1e12}
+    del dw1, dw2, ws
+    L = 12   # 6 interaction blocks x 2 MoE layers
+    gates = torch.as_tensor(np.stack([synth.gate_table(T, E, 500 + l) for l in range(L)]), device=layer.x.device)
+    ws_l = torch.empty(J.janus_route_layers_workspace_size(N, T, E, K, L), dtype=torch.uint8,
+                       device=layer.x.device)
+    ms_layers = _time_ms(lambda: J.janus_route_layers(layer.types, gates, K, workspace=ws_l))
+    ms_single = _time_ms(lambda: [J.janus_route(layer.types, gates[l], K, out=r, workspace=layer.route_ws)
+                                  for l in range(L)])
+    out["route_12_layers"] = {"ms_one_call": ms_layers, "ms_12_calls": ms_single}
+    if layer.slice:
+        Ed = int(layer.inp["row_ptr"][-1])
+        dmsg = torch.empty_like(layer.msg)
+        ms_b = _time_ms(lambda: J.janus_edge_broadcast(layer.dx, layer.row_ptr, out=dmsg), reps=3)
+        bb = 4 * N * d + 4 * Ed * d + 8 * (N + 1)
+        out["edge_broadcast"] = {"ms": ms_b, "GB/s": bb / (ms_b * 1e-3) / 1e9,
+                                 "frac_hbm": bb / (ms_b * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+        senders = torch.as_tensor(layer.inp["senders"].astype(np.int32), device=layer.x.device)
+        y = torch.empty_like(layer.xagg)
+        ms_n = _time_ms(lambda: J.janus_neighbor_aggregate(layer.xagg, layer.row_ptr, senders, out=y), reps=3)
+        gathered = 4 * Ed * d + 4 * Ed + 8 * (N + 1) + 4 * N * d
+        out["neighbor_aggregate"] = {"ms": ms_n, "gathered_GB/s": gathered / (ms_n * 1e-3) / 1e9,
+                                     "note": "gathered bytes (rows re-read through L2) per second"}
+        del dmsg, y
+    return out
 
 
 def run_e2e(layer, args):
