@@ -76,10 +76,14 @@ constexpr long long kWaitLimitCycles = 4000000000LL;     // ~2 s at 2 GHz
 
 enum Epilogue : int { kEpiStore = 0, kEpiSilu = 1, kEpiDSilu = 2 };
 
-// Operand layouts:  kModeNN  C = A W       (W stored [E][Kd][N], MN-major B)
-//                   kModeNT  C = A W^T     (W stored [E][N][Kd], K-major B)
+// Operand layouts:  kModeNN  C = X W       (W stored [E][Kd][N])
+//                   kModeNT  C = X W^T     (W stored [E][N][Kd])
 //                   kModeTN  C_e = X_e^T Y_e per expert (weight gradient; both
 //                            operands MN-major, K = the expert's row segment)
+// NN and NT run with the operands swapped (C^T = W^T X^T): the MMA's M is the
+// output feature (256 per CTA pair: the weights fill it without padding) and
+// its N is the expert's rows, chosen per tile as the valid rows rounded up to
+// 32, so a small expert wastes at most 31 rows instead of up to 255.
 enum Mode : int { kModeNN = 0, kModeNT = 1, kModeTN = 2 };
 
 struct Args {
@@ -215,16 +219,19 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 
 // Instruction descriptor: D=F32, A=B=TF32, A and B K- or MN-major,
 // M=256 (the CTA pair), N=256.
-__host__ __device__ constexpr uint32_t instr_desc(bool a_mn_major, bool b_mn_major) {
+__host__ __device__ constexpr uint32_t instr_desc(bool a_mn_major, bool b_mn_major, uint32_t n = BN) {
   return (1u << 4) | (2u << 7) | (2u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
-         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)((2 * BM) >> 4) << 24);
+         ((n >> 3) << 17) | ((uint32_t)((2 * BM) >> 4) << 24);
 }
 
-__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + expf(-a)); }
-__device__ __forceinline__ float dsilu_f(float a) {
-  const float s = 1.0f / (1.0f + expf(-a));
-  return s * (1.0f + a * (1.0f - s));
-}
+// Epilogue activations.  The store phase is unrolled over 128 columns per
+// thread, so every instruction here is repeated 128 times in the kernel's code;
+// a long sequence (an accurate expf plus an IEEE divide, twice) overflows the
+// instruction cache and stalls the MMA-issuing warp with it.  The sigmoid is
+// therefore computed once per element with the fast exponential and divide
+// (relative error a few 1e-7 against ~1e-6 from the 3xTF32 products).
+__device__ __forceinline__ float sigmoid_fast(float a) { return __fdividef(1.0f, 1.0f + __expf(-a)); }
+__device__ __forceinline__ float silu_f(float a) { return a * sigmoid_fast(a); }
 
 // TF32 high part: the FP32 value with its 13 low fraction bits cleared (exact
 // for every input, no overflow); the residual x - hi is exact in FP32.
@@ -246,7 +253,11 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 
 struct TileCoord {
-  int e, m0, m_end, n0;
+  int e;
+  int m0, m_end;    // MMA M: this CTA's first row (TN: output row; NN/NT: output feature) and bound
+  int n0;           // MMA N: TN: first output column; NN/NT: first dispatch row of the tile
+  int n_valid;      // NN/NT: valid rows in the tile
+  int n_mma;        // the MMA's N for this tile
   int k_row0;       // kModeTN: first row of the expert's segment (the K range)
   int k_rows;       // kModeTN: rows in the segment
   int nk;           // k-blocks of this tile
@@ -260,24 +271,30 @@ __device__ __forceinline__ TileCoord decode_tile(const Smem* s, const Args& args
                                                  int tile, uint32_t rank) {
   TileCoord c;
   const int mt = tile / n_tiles_n, nt = tile % n_tiles_n;
-  c.n0 = nt * BN;
   if (kMode == kModeTN) {
     const int n_mp = (args.M + 2 * BM - 1) / (2 * BM);
     c.e = mt / n_mp;
     c.m0 = ((mt % n_mp) * 2 + (int)rank) * BM;
     c.m_end = args.M;
+    c.n0 = nt * BN;
+    c.n_valid = min(BN, args.N - c.n0);
+    c.n_mma = BN;
     c.k_row0 = s->off[c.e];
     c.k_rows = s->off[c.e + 1] - c.k_row0;
     c.nk = (c.k_rows + BK - 1) / BK;
   } else {
+    // mt: 256-row block of the expert's segment; nt: 256-feature block
     int lo = 0, hi = args.E;   // start[lo] <= mt < start[hi]
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (s->start[mid] <= mt) lo = mid; else hi = mid;
     }
     c.e = lo;
-    c.m0 = s->off[lo] + ((mt - s->start[lo]) * 2 + (int)rank) * BM;
-    c.m_end = s->off[lo + 1];
+    c.n0 = s->off[lo] + (mt - s->start[lo]) * (2 * BM);
+    c.n_valid = min(2 * BM, s->off[lo + 1] - c.n0);
+    c.n_mma = (c.n_valid + 31) & ~31;
+    c.m0 = nt * BN + (int)rank * BNH;
+    c.m_end = args.N;
     c.k_row0 = 0;
     c.k_rows = 0;
     c.nk = nk_fixed;
@@ -320,25 +337,54 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
       if (lane == 0) mbar_arrive_leader(&s->chunk_empty[p], rank);
     }
     if (!ok) break;
+    if (kMode != kModeTN) {
+      // TMEM lane = output feature, column = dispatch row: for one row the 32
+      // lanes of a warp write 32 consecutive features (128-byte stores)
+      const int f = c.m0 + q * 32 + lane;
+      const int j0 = half * kEpiCols;
+      if (f < c.m_end) {
+        // batches of 16 columns: every load of a batch is issued before any
+        // use, so the pre-activation reads overlap instead of serialising
+        constexpr int kB = 16;
+#pragma unroll
+        for (int jb = 0; jb < kEpiCols; jb += kB) {
+          float a[kB];
+          if (kEpi == kEpiDSilu) {
+#pragma unroll
+            for (int j = 0; j < kB; ++j)
+              a[j] = (j0 + jb + j < c.n_valid) ? __ldg(args.aux + (int64_t)(c.n0 + j0 + jb + j) * N + f) : 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < kB; ++j) {
+            if (j0 + jb + j < c.n_valid) {
+              const int64_t o = (int64_t)(c.n0 + j0 + jb + j) * N + f;
+              float v = acc[jb + j];
+              if (kEpi == kEpiSilu) {
+                if (args.C2) args.C2[o] = v;
+                v = silu_f(v);
+              } else if (kEpi == kEpiDSilu) {
+                // silu'(a) = s (1 + a (1 - s)), s = sigmoid(a); C2 = silu(a) = a s
+                const float sg = sigmoid_fast(a[j]);
+                v *= sg * (1.0f + a[j] * (1.0f - sg));
+                if (args.C2) args.C2[o] = a[j] * sg;
+              }
+              args.C[o] = v;
+            }
+          }
+        }
+      }
+      continue;
+    }
+    // weight gradient (plain store): TMEM lane = output row, columns along it
+    static_assert(kMode != kModeTN || kEpi == kEpiStore, "the weight-gradient GEMM has no fused activation");
     const int row = c.m0 + q * 32 + lane;
     const int colb = c.n0 + half * kEpiCols;
     if (row < c.m_end && colb < N) {
-      const int64_t o = (kMode == kModeTN ? (int64_t)c.e * args.M * N : 0) + (int64_t)row * N + colb;
+      const int64_t o = (int64_t)c.e * args.M * N + (int64_t)row * N + colb;
 #pragma unroll
       for (int j = 0; j < kEpiCols; j += 4) {
         if (colb + j < N) {
-          float4 v = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-          if (kEpi == kEpiSilu) {
-            if (args.C2) *reinterpret_cast<float4*>(args.C2 + o + j) = v;
-            v = make_float4(silu_f(v.x), silu_f(v.y), silu_f(v.z), silu_f(v.w));
-          } else if (kEpi == kEpiDSilu) {
-            const float4 a = __ldg(reinterpret_cast<const float4*>(args.aux + o + j));
-            v = make_float4(v.x * dsilu_f(a.x), v.y * dsilu_f(a.y), v.z * dsilu_f(a.z), v.w * dsilu_f(a.w));
-            if (args.C2)   // H = silu(a) for the second weight gradient
-              *reinterpret_cast<float4*>(args.C2 + o + j) =
-                  make_float4(silu_f(a.x), silu_f(a.y), silu_f(a.z), silu_f(a.w));
-          }
-          *reinterpret_cast<float4*>(args.C + o + j) = v;
+          *reinterpret_cast<float4*>(args.C + o + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
         }
       }
     }
@@ -411,7 +457,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         bool ok = true;
         for (int tile = blockIdx.x / 2; tile < total && ok; tile += n_pairs) {
           const TileCoord c = decode_tile<kMode>(s, args, n_tiles_n, nk, tile, rank);
-          const int nb = c.n0 + (int)rank * BNH;
+          const int nb = c.n0 + (int)rank * BNH;   // kModeTN: this CTA's B columns
           for (int kb = 0; kb < c.nk; ++kb, ++it) {
             const uint32_t st = it % kStages, use = it / kStages;
             if (!mbar_wait(s, &s->empty[st], (use & 1) ^ 1, args.err)) { ok = false; break; }
@@ -427,15 +473,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
               for (int j = 0; j < BNH / 32; ++j)
                 tma_load_2d(&mapB, &s->full[st], base + kTileABytes + j * (32 * BK * 4), nb + 32 * j, row);
             } else {
-              tma_load_2d(&mapA, &s->full[st], base, kb * BK, c.m0);
+              // A: this CTA's 128 features of expert e's weights
               if (kMode == kModeNT) {
-                tma_load_3d(&mapB, &s->full[st], base + kTileABytes, kb * BK, nb, c.e);
+                tma_load_3d(&mapA, &s->full[st], base, kb * BK, c.m0, c.e);
               } else {
 #pragma unroll
-                for (int j = 0; j < BNH / 32; ++j)
-                  tma_load_3d(&mapB, &s->full[st], base + kTileABytes + j * (32 * BK * 4), nb + 32 * j, kb * BK,
-                              c.e);
+                for (int j = 0; j < BM / 32; ++j)
+                  tma_load_3d(&mapA, &s->full[st], base + j * (32 * BK * 4), c.m0 + 32 * j, kb * BK, c.e);
               }
+              // B: this CTA's half of the tile's dispatch rows (n_mma / 2 of them)
+              tma_load_2d(&mapB, &s->full[st], base + kTileABytes, kb * BK, c.n0 + (int)rank * (c.n_mma / 2));
             }
           }
         }
@@ -453,11 +500,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       // Each chunk of kChunkKb k-blocks is accumulated from zero into one of two
       // TMEM buffers; the epilogues of both CTAs fold it into FP32 running sums.
       if (lane == 0 && rank == 0) {
-        constexpr uint32_t idesc = instr_desc(kMode == kModeTN, kMode != kModeNT);
+        constexpr bool kAMN = kMode != kModeNT;       // TN: X^T; NN: W (features contiguous)
+        constexpr bool kBMN = kMode == kModeTN;       // NN/NT: dispatch rows, K-major
         uint32_t it = 0, ch = 0;
         bool ok = true;
         for (int tile = blockIdx.x / 2; tile < total && ok; tile += n_pairs) {
-          const int tnk = decode_tile<kMode>(s, args, n_tiles_n, nk, tile, rank).nk;
+          const TileCoord tc = decode_tile<kMode>(s, args, n_tiles_n, nk, tile, rank);
+          const int tnk = tc.nk;
+          const uint32_t idesc = instr_desc(kAMN, kBMN, (uint32_t)tc.n_mma);
           for (int c0 = 0; c0 < tnk && ok; c0 += kChunkKb, ++ch) {
             const uint32_t p = ch & 1, cuse = ch >> 1;
             if (!mbar_wait(s, &s->chunk_empty[p], (cuse & 1) ^ 1, args.err)) { ok = false; break; }
@@ -477,19 +527,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                 // MN-major B: 32-column chunks 32*BK*4 B apart (LBO), 4 k-rows per
                 // 512-byte group (SBO), k-step of 8 rows = +1024 B.
                 uint64_t adh, adl, bdh, bdl;
-                if (kMode == kModeTN) {
+                if (kAMN) {
                   adh = smem_desc(a_hi + kk * 1024, 32 * BK * 4, 512, kSwizzle128B32B);
                   adl = smem_desc(a_lo + kk * 1024, 32 * BK * 4, 512, kSwizzle128B32B);
                 } else {
                   adh = smem_desc(a_hi + kk * 32, 16, 512, kSwizzle64B);
                   adl = smem_desc(a_lo + kk * 32, 16, 512, kSwizzle64B);
                 }
-                if (kMode == kModeNT) {
-                  bdh = smem_desc(b_hi + kk * 32, 16, 512, kSwizzle64B);
-                  bdl = smem_desc(b_lo + kk * 32, 16, 512, kSwizzle64B);
-                } else {
+                if (kBMN) {
                   bdh = smem_desc(b_hi + kk * 1024, 32 * BK * 4, 512, kSwizzle128B32B);
                   bdl = smem_desc(b_lo + kk * 1024, 32 * BK * 4, 512, kSwizzle128B32B);
+                } else {
+                  bdh = smem_desc(b_hi + kk * 32, 16, 512, kSwizzle64B);
+                  bdl = smem_desc(b_lo + kk * 32, 16, 512, kSwizzle64B);
                 }
                 tc_mma_tf32_pair(d_tmem, adl, bdh, idesc, (kb > c0 || kk > 0) ? 1u : 0u);
                 tc_mma_tf32_pair(d_tmem, adh, bdl, idesc, 1u);
@@ -653,7 +703,8 @@ janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, in
   CUtensorMap ma, mb;
   if (kMode == kModeTN) {
     if (!map_rows_mn(&ma, A, R, M) || !map_rows_mn(&mb, W, R, N)) return JANUS_ERR_CUDA;
-  } else if (!map_a(&ma, A, R, Kd) || !map_b(&mb, W, E, Kd, N, kMode == kModeNT)) {
+  } else if (!map_b(&ma, W, E, Kd, N, kMode == kModeNT) || !map_a(&mb, A, R, Kd)) {
+    // operands swapped: the weights are the MMA's A, the dispatch rows its B
     return JANUS_ERR_CUDA;
   }
   Args a;
