@@ -185,7 +185,7 @@ class ClockSampler:
 # S-shaped layer (profiles/expert_ffn_tc_gemm.md), valid only for the kernel
 # source it was taken on.
 GEMM_TRAFFIC = {("S", "3xtf32"): {"src": "element_routed_moe_b200/csrc/ffn_tc.cu",
-                                  "sha256_prefix": "93a3d1e8f6bbcfc0", "bytes_per_launch": 3.106e9}}
+                                  "sha256_prefix": "9d27d43dc69b134d", "bytes_per_launch": 3.167e9}}
 
 
 def measured_traffic(workload: str, mode: str):
@@ -482,8 +482,11 @@ def run_janus(args, world, rank, local):
         peak = SM_COUNT * FP32_LANES_PER_SM * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
         roof = {"bound": "alu", "peak_source": "148 SMs x 128 FP32 lanes x 2 FLOP x max SM clock"}
     else:
-        peak = peaks["bf16_tflops_sustained"] * (1.125 / 2.25) / 3.0
-        roof = {"bound": "tensor", "peak_source": f"{peak_src} sustained bf16 x (TF32/BF16 nominal 1.125/2.25) / 3 products"}
+        # burst figure: the GEMM runs at the maximum SM clock inside this step
+        # (the clocks record shows it), unlike the power-capped seconds-long
+        # bf16 loop behind the sustained figure; the burst one is the stricter
+        peak = peaks["bf16_tflops"] * (1.125 / 2.25) / 3.0
+        roof = {"bound": "tensor", "peak_source": f"{peak_src} burst bf16 x (TF32/BF16 nominal 1.125/2.25) / 3 products"}
     roof.update({"kernel": "grouped expert-MLP GEMM", "achieved": achieved, "peak": peak,
                  "unit": "TFLOP/s", "frac": achieved / peak,
                  "traffic": (measured_traffic(cfg.name, args.mode)

@@ -335,6 +335,16 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader(&s->chunk_empty[p], rank);
+      if (kMode != kModeTN && kEpi == kEpiDSilu && c0 == 0) {
+        // the tile's pre-activations travel to L2 while its chunks accumulate
+        const int f = c.m0 + q * 32 + lane;
+        const int jn = min(kEpiCols, c.n_valid - half * kEpiCols);
+        if (f < c.m_end) {
+#pragma unroll 1
+          for (int j = 0; j < jn; ++j)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(args.aux + (int64_t)(c.n0 + half * kEpiCols + j) * N + f));
+        }
+      }
     }
     if (!ok) break;
     if (kMode != kModeTN) {
@@ -343,16 +353,21 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
       const int f = c.m0 + q * 32 + lane;
       const int j0 = half * kEpiCols;
       if (f < c.m_end) {
-        // batches of 16 columns: every load of a batch is issued before any
-        // use, so the pre-activation reads overlap instead of serialising
-        constexpr int kB = 16;
+        // batches of 8 columns; the pre-activations of batch b + 1 are in
+        // flight while batch b is finished, so two loads per column overlap
+        constexpr int kB = 8;
+        const float* arow = args.aux + (int64_t)(c.n0 + j0) * N + f;
+        float a_cur[kB], a_nxt[kB];
+        if (kEpi == kEpiDSilu) {
+#pragma unroll
+          for (int j = 0; j < kB; ++j) a_cur[j] = (j0 + j < c.n_valid) ? __ldg(arow + (int64_t)j * N) : 0.f;
+        }
 #pragma unroll
         for (int jb = 0; jb < kEpiCols; jb += kB) {
-          float a[kB];
-          if (kEpi == kEpiDSilu) {
+          if (kEpi == kEpiDSilu && jb + kB < kEpiCols) {
 #pragma unroll
             for (int j = 0; j < kB; ++j)
-              a[j] = (j0 + jb + j < c.n_valid) ? __ldg(args.aux + (int64_t)(c.n0 + j0 + jb + j) * N + f) : 0.f;
+              a_nxt[j] = (j0 + jb + kB + j < c.n_valid) ? __ldg(arow + (int64_t)(jb + kB + j) * N) : 0.f;
           }
 #pragma unroll
           for (int j = 0; j < kB; ++j) {
@@ -364,12 +379,17 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
                 v = silu_f(v);
               } else if (kEpi == kEpiDSilu) {
                 // silu'(a) = s (1 + a (1 - s)), s = sigmoid(a); C2 = silu(a) = a s
-                const float sg = sigmoid_fast(a[j]);
-                v *= sg * (1.0f + a[j] * (1.0f - sg));
-                if (args.C2) args.C2[o] = a[j] * sg;
+                const float a = a_cur[j];
+                const float sg = sigmoid_fast(a);
+                v *= sg * (1.0f + a * (1.0f - sg));
+                if (args.C2) args.C2[o] = a * sg;
               }
               args.C[o] = v;
             }
+          }
+          if (kEpi == kEpiDSilu) {
+#pragma unroll
+            for (int j = 0; j < kB; ++j) a_cur[j] = a_nxt[j];
           }
         }
       }
