@@ -43,6 +43,8 @@ def _setup(L):
     L.orc_expert_ffn_fwd.argtypes = [vp, vp, i32, i64, i32, i32, vp, vp, vp, i64, vp, vp]
     L.orc_expert_ffn_vjp.argtypes = [vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, i64, vp]
     L.orc_expert_ffn_weight_grad.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp, vp]
+    L.orc_expert_ffn_vjp_vjp.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, i64, vp, vp]
+    L.orc_expert_ffn_vjp_vjp_weight_grad.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp]
     L.orc_combine.argtypes = [vp, vp, vp, i64, i32, i32, vp]
     L.orc_edge_aggregate.argtypes = [vp, vp, i64, i32, vp]
     L.orc_edge_broadcast.argtypes = [vp, vp, i64, i32, vp]
@@ -170,6 +172,37 @@ def expert_ffn_weight_grad(xd, gd, offsets, w1, w2):
     dw2 = np.empty((E, h, d), np.float32)
     lib().orc_expert_ffn_weight_grad(_p(xd), _p(gd), _p(offsets), E, d, h, _p(w1), _p(w2),
                                      _p(dw1), _p(dw2))
+    return dw1, dw2
+
+
+def expert_ffn_vjp_vjp(xd, gd, vd, offsets, w1, w2, rows=None):
+    """Second-order pass: gradients w.r.t. xd and gd of L = <dxd(xd, gd), vd>,
+    where dxd is the expert MLP's input VJP.  Returns (d_xd, d_gd), [n_out, d]."""
+    xd, gd, vd = _c(xd, np.float32), _c(gd, np.float32), _c(vd, np.float32)
+    offsets = _c(offsets, np.int32)
+    w1, w2 = _c(w1, np.float32), _c(w2, np.float32)
+    R, d = xd.shape
+    E, _, h = w1.shape
+    r = None if rows is None else _c(rows, np.int64)
+    n_out = R if r is None else r.shape[0]
+    d_xd = np.empty((n_out, d), np.float32)
+    d_gd = np.empty((n_out, d), np.float32)
+    lib().orc_expert_ffn_vjp_vjp(_p(xd), _p(gd), _p(vd), _p(offsets), E, R, d, h, _p(w1), _p(w2),
+                                 _p(r), 0 if r is None else r.shape[0], _p(d_xd), _p(d_gd))
+    return d_xd, d_gd
+
+
+def expert_ffn_vjp_vjp_weight_grad(xd, gd, vd, offsets, w1, w2):
+    """Weight part of the second-order pass: (dW1 [E,d,h], dW2 [E,h,d]) of
+    L = <dxd(xd, gd; W1, W2), vd>."""
+    xd, gd, vd = _c(xd, np.float32), _c(gd, np.float32), _c(vd, np.float32)
+    offsets = _c(offsets, np.int32)
+    w1, w2 = _c(w1, np.float32), _c(w2, np.float32)
+    E, d, h = w1.shape
+    dw1 = np.empty((E, d, h), np.float32)
+    dw2 = np.empty((E, h, d), np.float32)
+    lib().orc_expert_ffn_vjp_vjp_weight_grad(_p(xd), _p(gd), _p(vd), _p(offsets), E, d, h,
+                                             _p(w1), _p(w2), _p(dw1), _p(dw2))
     return dw1, dw2
 
 

@@ -351,6 +351,120 @@ void orc_expert_ffn_weight_grad(const float* xd, const float* gd, const int32_t*
 }
 
 // ---------------------------------------------------------------------------
+// Second-order pass: the VJP of the input VJP.  Force training ([Review]
+// section 3.3: forces are -dE/dx, fitted by a loss) differentiates the forces,
+// so the gradient of a loss on the layer's input VJP is on the path.  Per row,
+// with a = x W1, sig = sigmoid(a):
+//   s1 = silu'(a)  = sig (1 + a (1 - sig))
+//   s2 = silu''(a) = sig (1 - sig) (2 + a (1 - 2 sig))
+//   dh = W2 g,  u = dh * s1,  dx = W1 u                (the input VJP)
+// and for L = <dx, v> with v the cotangent of dx:
+//   ub = W1^T v,  t1 = ub * s1,  t2 = ub * dh * s2
+//   dL/dx = W1 t2,  dL/dg = W2^T t1
+//   dL/dW1[k][j] = sum_p v[k] u[j] + x[k] t2[j],  dL/dW2[j][c] = sum_p t1[j] g[c]
+// Everything per row in FP64 (a recomputed), outputs rounded once to FP32.
+// ---------------------------------------------------------------------------
+namespace {
+struct RowTerms {
+  std::vector<double> a, dh, s1, s2, u, t1, t2;
+  explicit RowTerms(int h) : a(h), dh(h), s1(h), s2(h), u(h), t1(h), t2(h) {}
+  void compute(const float* x, const float* g, const float* v, const float* W1, const float* W2, int d,
+               int h) {
+    std::fill(a.begin(), a.end(), 0.0);
+    for (int k = 0; k < d; ++k) {
+      const double xk = x[k];
+      for (int j = 0; j < h; ++j) a[j] += xk * (double)W1[(int64_t)k * h + j];
+    }
+    for (int j = 0; j < h; ++j) {
+      double acc = 0.0, ub = 0.0;
+      for (int c = 0; c < d; ++c) acc += (double)W2[(int64_t)j * d + c] * (double)g[c];
+      for (int k = 0; k < d; ++k) ub += (double)W1[(int64_t)k * h + j] * (double)v[k];
+      const double sg = 1.0 / (1.0 + std::exp(-a[j]));
+      dh[j] = acc;
+      s1[j] = sg * (1.0 + a[j] * (1.0 - sg));
+      s2[j] = sg * (1.0 - sg) * (2.0 + a[j] * (1.0 - 2.0 * sg));
+      u[j] = dh[j] * s1[j];
+      t1[j] = ub * s1[j];
+      t2[j] = ub * dh[j] * s2[j];
+    }
+  }
+};
+}  // namespace
+
+void orc_expert_ffn_vjp_vjp(const float* xd, const float* gd, const float* vd, const int32_t* offsets,
+                            int32_t n_experts, int64_t n_rows, int32_t d, int32_t h, const float* w1,
+                            const float* w2, const int64_t* rows, int64_t n_sel, float* d_xd, float* d_gd) {
+  const int64_t n_out = rows ? n_sel : n_rows;
+#pragma omp parallel
+  {
+    RowTerms t(h);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t q = 0; q < n_out; ++q) {
+      const int64_t p = rows ? rows[q] : q;
+      const int e = expert_of_row(offsets, n_experts, p);
+      const float* W1 = w1 + (int64_t)e * d * h;
+      const float* W2 = w2 + (int64_t)e * h * d;
+      t.compute(xd + p * d, gd + p * d, vd + p * d, W1, W2, d, h);
+      for (int k = 0; k < d; ++k) {
+        double acc = 0.0;
+        for (int j = 0; j < h; ++j) acc += (double)W1[(int64_t)k * h + j] * t.t2[j];
+        d_xd[q * d + k] = (float)acc;
+      }
+      for (int c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (int j = 0; j < h; ++j) acc += (double)W2[(int64_t)j * d + c] * t.t1[j];
+        d_gd[q * d + c] = (float)acc;
+      }
+    }
+  }
+}
+
+// Weight part of the second-order pass (sums over each expert's rows, in row
+// order); an expert with no rows gets zeros.
+void orc_expert_ffn_vjp_vjp_weight_grad(const float* xd, const float* gd, const float* vd,
+                                        const int32_t* offsets, int32_t n_experts, int32_t d, int32_t h,
+                                        const float* w1, const float* w2, float* dw1, float* dw2) {
+  for (int e = 0; e < n_experts; ++e) {
+    const float* W1 = w1 + (int64_t)e * d * h;
+    const float* W2 = w2 + (int64_t)e * h * d;
+    const int64_t p0 = offsets[e], n = offsets[e + 1] - offsets[e];
+    std::vector<double> u((size_t)n * h), t1((size_t)n * h), t2((size_t)n * h);
+#pragma omp parallel
+    {
+      RowTerms t(h);
+#pragma omp for schedule(dynamic, 1)
+      for (int64_t r = 0; r < n; ++r) {
+        const int64_t p = p0 + r;
+        t.compute(xd + p * d, gd + p * d, vd + p * d, W1, W2, d, h);
+        for (int j = 0; j < h; ++j) {
+          u[(size_t)r * h + j] = t.u[j];
+          t1[(size_t)r * h + j] = t.t1[j];
+          t2[(size_t)r * h + j] = t.t2[j];
+        }
+      }
+    }
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int k = 0; k < d; ++k) {
+      std::vector<double> acc(h, 0.0);
+      for (int64_t r = 0; r < n; ++r) {
+        const double vk = vd[(p0 + r) * d + k], xk = xd[(p0 + r) * d + k];
+        for (int j = 0; j < h; ++j) acc[j] += vk * u[(size_t)r * h + j] + xk * t2[(size_t)r * h + j];
+      }
+      for (int j = 0; j < h; ++j) dw1[(int64_t)e * d * h + (int64_t)k * h + j] = (float)acc[j];
+    }
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int j = 0; j < h; ++j) {
+      std::vector<double> acc(d, 0.0);
+      for (int64_t r = 0; r < n; ++r) {
+        const double tj = t1[(size_t)r * h + j];
+        for (int c = 0; c < d; ++c) acc[c] += tj * (double)gd[(p0 + r) * d + c];
+      }
+      for (int c = 0; c < d; ++c) dw2[(int64_t)e * h * d + (int64_t)j * d + c] = (float)acc[c];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Combine.  [Blueprint] §3.2: the activated experts' outputs are summed with
 // the gate weights.  Gather form: Y[i,:] = sum_{k ascending} w[i,k] *
 // Yd[slot_of[i*K+k],:]; topk_weight == NULL means weight 1 (the VJP combine).
