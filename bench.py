@@ -555,7 +555,18 @@ def run_extras(layer, peaks):
                                                           act=layer.act, mode=layer.mode, dw1=dw1, dw2=dw2,
                                                           workspace=ws))
     out["expert_weight_grad"] = {"ms": ms, "gemms": 3, "TFLOP/s": 6 * R * d * h / (ms * 1e-3) / 1e12}
-    del dw1, dw2, ws
+    # second-order pass (VJP of the input VJP) with its weight part: 7 GEMMs
+    # of 2*R*d*h each (dh, v W1, t1 W2, t2 W1^T, T1^T Gd, Vd^T U, Xd^T T2)
+    vd = synth.normal((R, d), 77, layer.x.device)    # cotangent of the input VJP
+    d_x = torch.empty_like(layer.xd)
+    d_g = torch.empty_like(layer.xd)
+    ws2 = torch.empty(J.janus_expert_ffn_vjp_vjp_workspace_size(R, h, True, True), dtype=torch.uint8,
+                      device=layer.x.device)
+    ms2 = _time_ms(lambda: J.janus_expert_ffn_vjp_vjp(layer.xd, layer.gd, vd, r["offsets"], layer.w1,
+                                                      layer.w2, act=layer.act, mode=layer.mode, weight_grad=True,
+                                                      d_xd=d_x, d_gd=d_g, dw1=dw1, dw2=dw2, workspace=ws2))
+    out["expert_second_order"] = {"ms": ms2, "gemms": 7, "TFLOP/s": 14 * R * d * h / (ms2 * 1e-3) / 1e12}
+    del dw1, dw2, ws, d_x, d_g, ws2, vd
     L = 12   # 6 interaction blocks x 2 MoE layers
     gates = torch.as_tensor(np.stack([synth.gate_table(T, E, 500 + l) for l in range(L)]), device=layer.x.device)
     ws_l = torch.empty(J.janus_route_layers_workspace_size(N, T, E, K, L), dtype=torch.uint8,

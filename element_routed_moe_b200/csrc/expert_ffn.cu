@@ -60,6 +60,7 @@ simt::Args make_args(const float* A, const float* B, int64_t bstride, float* C, 
                      const float* aux, const int32_t* offsets, int E, int Kd, int N) {
   simt::Args a;
   a.A = A; a.B = B; a.b_expert_stride = bstride; a.C = C; a.C2 = C2; a.aux = aux;
+  a.aux2 = nullptr; a.C3 = nullptr;
   a.offsets = offsets; a.E = E; a.Kd = Kd; a.N = N;
   return a;
 }
@@ -191,9 +192,92 @@ extern "C" janus_status janus_expert_ffn_weight_grad(const float* xd, const floa
   if (!act)
     launch_simt<false, simt::kEpiStore>(make_args(xd, w1, sw, A, nullptr, nullptr, offsets, n_experts, d, h), stream);
   launch_simt<true, simt::kEpiDSilu>(make_args(gd, w2, sw, dA, H, A, offsets, n_experts, d, h), stream);
-  simt::TnArgs t1{xd, dA, dw1, offsets, n_experts, d, h};
+  simt::TnArgs t1{xd, dA, dw1, offsets, n_experts, d, h, 0};
   simt::grouped_tn_kernel<<<num_sms() * 2, simt::kThreads, 0, stream>>>(t1);
-  simt::TnArgs t2{H, gd, dw2, offsets, n_experts, h, d};
+  simt::TnArgs t2{H, gd, dw2, offsets, n_experts, h, d, 0};
   simt::grouped_tn_kernel<<<num_sms() * 2, simt::kThreads, 0, stream>>>(t2);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// Second-order pass: gradients of L = <dxd(xd, gd; W1, W2), vd> (the VJP of
+// the input VJP, which force training differentiates).
+//   G0: a = xd W1                  (only without the forward's act)
+//   G1: dh = gd W2^T
+//   G2: ub = vd W1 -> t1 = ub silu'(a), t2 = ub dh silu''(a), u = dh silu'(a)
+//   G3: d_gd = t1 W2,  G4: d_xd = t2 W1^T
+//   G5: dW2[e] = T1_e^T Gd_e,  G6/G7: dW1[e] = Vd_e^T U_e + Xd_e^T T2_e
+// Workspace: header | dh | t1 | t2 | u (weight gradients) | a (no act), each
+// [R,h] FP32 rounded up to 256 bytes.
+// ---------------------------------------------------------------------------
+extern "C" janus_status janus_expert_ffn_vjp_vjp_workspace_size(int64_t n_rows, int32_t h, int32_t have_act,
+                                                                int32_t want_weight_grad, size_t* bytes) {
+  JANUS_CHECK_ARG(bytes && n_rows >= 0 && h >= 1);
+  const size_t rh = align_up(sizeof(float) * (size_t)n_rows * (size_t)h, 256);
+  *bytes = sizeof(WsHeader) + (3 + (want_weight_grad ? 1 : 0) + (have_act ? 0 : 1)) * rh;
+  return JANUS_OK;
+}
+
+extern "C" janus_status janus_expert_ffn_vjp_vjp(const float* xd, const float* gd, const float* vd,
+                                                 const float* act, const int32_t* offsets, int32_t n_experts,
+                                                 int64_t n_rows, int32_t d, int32_t h, const float* w1,
+                                                 const float* w2, float* d_xd, float* d_gd, float* dw1,
+                                                 float* dw2, janus_ffn_mode mode, void* workspace,
+                                                 size_t workspace_bytes, janus_stream_t stream_) {
+  cudaStream_t stream = (cudaStream_t)stream_;
+  janus_status st = check_ffn(xd, offsets, n_experts, n_rows, d, h, w1, w2, d_xd, mode);
+  if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(n_rows == 0 || (gd && vd && d_gd));
+  JANUS_CHECK_ARG((dw1 == nullptr) == (dw2 == nullptr));
+  JANUS_CHECK_ALIGN(n_rows == 0 || (aligned(gd, 16) && aligned(vd, 16) && aligned(d_gd, 16)));
+  JANUS_CHECK_ALIGN(act == nullptr || aligned(act, 16));
+  JANUS_CHECK_ALIGN(dw1 == nullptr || (aligned(dw1, 16) && aligned(dw2, 16)));
+  const bool wg = dw1 != nullptr;
+  size_t need = 0;
+  st = janus_expert_ffn_vjp_vjp_workspace_size(n_rows, h, act != nullptr, wg, &need);
+  if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(workspace && workspace_bytes >= need);
+  JANUS_CHECK_ALIGN(aligned(workspace, 256));
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  if (n_rows == 0) {   // no rows: the weight gradients are zero, nothing else to write
+    if (wg) {
+      const size_t wbytes = sizeof(float) * (size_t)n_experts * (size_t)d * (size_t)h;
+      JANUS_CUDA_TRY(cudaMemsetAsync(dw1, 0, wbytes, stream));
+      JANUS_CUDA_TRY(cudaMemsetAsync(dw2, 0, wbytes, stream));
+    }
+    return JANUS_OK;
+  }
+  const size_t rh = align_up(sizeof(float) * (size_t)n_rows * (size_t)h, 256);
+  char* w = (char*)workspace + sizeof(WsHeader);
+  float* dh = (float*)w;
+  float* t1 = (float*)(w + rh);
+  float* t2 = (float*)(w + 2 * rh);
+  float* u = wg ? (float*)(w + 3 * rh) : nullptr;
+  float* A = act ? const_cast<float*>(act) : (float*)(w + (wg ? 4 : 3) * rh);
+  if (mode == JANUS_FFN_3XTF32) {
+    JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
+    st = tc::expert_ffn_vjp_vjp(xd, gd, vd, act, A, offsets, n_experts, n_rows, d, h, w1, w2, d_xd, d_gd, dw1,
+                                dw2, dh, t1, t2, u, &((WsHeader*)workspace)->error, stream);
+    if (st != JANUS_OK) return st;
+    return launch_status();
+  }
+  const int64_t sw = (int64_t)d * h;
+  if (!act)
+    launch_simt<false, simt::kEpiStore>(make_args(xd, w1, sw, A, nullptr, nullptr, offsets, n_experts, d, h), stream);
+  launch_simt<true, simt::kEpiStore>(make_args(gd, w2, sw, dh, nullptr, nullptr, offsets, n_experts, d, h), stream);
+  simt::Args a2 = make_args(vd, w1, sw, t1, t2, A, offsets, n_experts, d, h);
+  a2.aux2 = dh;
+  a2.C3 = u;
+  launch_simt<false, simt::kEpiD2>(a2, stream);
+  launch_simt<false, simt::kEpiStore>(make_args(t1, w2, sw, d_gd, nullptr, nullptr, offsets, n_experts, h, d), stream);
+  launch_simt<true, simt::kEpiStore>(make_args(t2, w1, sw, d_xd, nullptr, nullptr, offsets, n_experts, h, d), stream);
+  if (wg) {
+    simt::TnArgs g2{t1, gd, dw2, offsets, n_experts, h, d, 0};
+    simt::grouped_tn_kernel<<<num_sms() * 2, simt::kThreads, 0, stream>>>(g2);
+    simt::TnArgs g1a{vd, u, dw1, offsets, n_experts, d, h, 0};
+    simt::grouped_tn_kernel<<<num_sms() * 2, simt::kThreads, 0, stream>>>(g1a);
+    simt::TnArgs g1b{xd, t2, dw1, offsets, n_experts, d, h, 1};
+    simt::grouped_tn_kernel<<<num_sms() * 2, simt::kThreads, 0, stream>>>(g1b);
+  }
   return launch_status();
 }

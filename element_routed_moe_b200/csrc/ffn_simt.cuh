@@ -25,7 +25,9 @@ constexpr int BM = 128, BN = 128, BK = 16, kThreads = 256;
 enum Epilogue : int {
   kEpiStore = 0,   // C = acc
   kEpiSilu = 1,    // C2 = acc (if C2), C = silu(acc)
-  kEpiDSilu = 2    // C = acc * silu'(aux)
+  kEpiDSilu = 2,   // C = acc * silu'(aux)
+  kEpiD2 = 3       // second-order pass, acc = v W1, aux = a, aux2 = dh:
+                   //   C = acc * silu'(a), C2 = acc * dh * silu''(a), C3 = dh * silu'(a) (if C3)
 };
 
 struct Args {
@@ -34,7 +36,9 @@ struct Args {
   int64_t b_expert_stride;   // elements between experts' weights
   float* C;
   float* C2;                 // optional second output (pre-activation)
-  const float* aux;          // pre-activation for kEpiDSilu, [R, N]
+  const float* aux;          // pre-activation for kEpiDSilu / kEpiD2, [R, N]
+  const float* aux2;         // kEpiD2: dh = gd W2^T, [R, N]
+  float* C3;                 // kEpiD2: optional third output
   const int32_t* offsets;
   int E;
   int Kd;                    // reduction length
@@ -45,6 +49,15 @@ __device__ __forceinline__ float silu_f(float a) { return a / (1.0f + expf(-a));
 __device__ __forceinline__ float dsilu_f(float a) {
   const float s = 1.0f / (1.0f + expf(-a));
   return s * (1.0f + a * (1.0f - s));
+}
+// silu''(a) = sig (1 - sig) (2 + a (1 - 2 sig))
+__device__ __forceinline__ void d2_terms(float acc, float a, float dh, float& t1, float& t2, float& u) {
+  const float s = 1.0f / (1.0f + expf(-a));
+  const float s1 = s * (1.0f + a * (1.0f - s));
+  const float s2 = s * (1.0f - s) * (2.0f + a * (1.0f - 2.0f * s));
+  t1 = acc * s1;
+  t2 = acc * dh * s2;
+  u = dh * s1;
 }
 
 // Expert-major tile list: tile_start[e] = sum_{e'<e} ceil(count_e'/BM).
@@ -205,6 +218,16 @@ __global__ void __launch_bounds__(kThreads, 2) grouped_gemm_kernel(Args args) {
           v = make_float4(v.x * dsilu_f(a.x), v.y * dsilu_f(a.y), v.z * dsilu_f(a.z), v.w * dsilu_f(a.w));
           if (args.C2)   // H = silu(a) for the second weight gradient
             *reinterpret_cast<float4*>(args.C2 + o) = make_float4(silu_f(a.x), silu_f(a.y), silu_f(a.z), silu_f(a.w));
+        } else if (kEpi == kEpiD2) {
+          const float4 a = __ldg(reinterpret_cast<const float4*>(args.aux + o));
+          const float4 g = __ldg(reinterpret_cast<const float4*>(args.aux2 + o));
+          float4 t2, u;
+          d2_terms(v.x, a.x, g.x, v.x, t2.x, u.x);
+          d2_terms(v.y, a.y, g.y, v.y, t2.y, u.y);
+          d2_terms(v.z, a.z, g.z, v.z, t2.z, u.z);
+          d2_terms(v.w, a.w, g.w, v.w, t2.w, u.w);
+          *reinterpret_cast<float4*>(args.C2 + o) = t2;
+          if (args.C3) *reinterpret_cast<float4*>(args.C3 + o) = u;
         }
         *reinterpret_cast<float4*>(args.C + o) = v;
       }
@@ -223,6 +246,7 @@ struct TnArgs {
   float* C;
   const int32_t* offsets;
   int E, M, N;
+  int accumulate;   // nonzero: C += X^T Y
 };
 
 __global__ void __launch_bounds__(kThreads, 2) grouped_tn_kernel(TnArgs args) {
@@ -300,8 +324,13 @@ __global__ void __launch_bounds__(kThreads, 2) grouped_tn_kernel(TnArgs args) {
       for (int g = 0; g < 2; ++g) {
         const int c = n0 + g * 64 + tx * 4;
         if (c >= N) continue;
-        *reinterpret_cast<float4*>(C + (int64_t)r * N + c) =
-            make_float4(acc[i][g * 4 + 0], acc[i][g * 4 + 1], acc[i][g * 4 + 2], acc[i][g * 4 + 3]);
+        float4 v = make_float4(acc[i][g * 4 + 0], acc[i][g * 4 + 1], acc[i][g * 4 + 2], acc[i][g * 4 + 3]);
+        float4* dst = reinterpret_cast<float4*>(C + (int64_t)r * N + c);
+        if (args.accumulate) {
+          const float4 o = *dst;
+          v = make_float4(o.x + v.x, o.y + v.y, o.z + v.z, o.w + v.w);
+        }
+        *dst = v;
       }
     }
   }

@@ -74,7 +74,10 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kFaultTimeout = 3;
 constexpr long long kWaitLimitCycles = 4000000000LL;     // ~2 s at 2 GHz
 
-enum Epilogue : int { kEpiStore = 0, kEpiSilu = 1, kEpiDSilu = 2 };
+// kEpiD2 (second-order pass, x·W): acc = v W1, aux = a, aux2 = dh;
+//   C = acc silu'(a), C2 = acc dh silu''(a), C3 = dh silu'(a) (if C3).
+// kEpiAccum (weight-gradient layout only): C += acc.
+enum Epilogue : int { kEpiStore = 0, kEpiSilu = 1, kEpiDSilu = 2, kEpiD2 = 3, kEpiAccum = 4 };
 
 // Operand layouts:  kModeNN  C = X W       (W stored [E][Kd][N])
 //                   kModeNT  C = X W^T     (W stored [E][N][Kd])
@@ -89,7 +92,9 @@ enum Mode : int { kModeNN = 0, kModeNT = 1, kModeTN = 2 };
 struct Args {
   float* C;
   float* C2;
+  float* C3;
   const float* aux;
+  const float* aux2;
   const int32_t* offsets;
   int E, Kd, N;
   int M;            // kModeTN: rows of each expert's output (C is [E][M][N])
@@ -302,6 +307,38 @@ __device__ __forceinline__ TileCoord decode_tile(const Smem* s, const Args& args
   return c;
 }
 
+// Second-order epilogue for one thread's 128 columns (swapped layout: output
+// feature f of dispatch rows n0 + j0 + j), 4 columns per batch with both
+// inputs loaded before use.
+__device__ __forceinline__ void d2_store(const Args& args, const float (&acc)[kEpiCols], const TileCoord& c,
+                                         int j0, int f, int N) {
+  constexpr int kB = 4;
+#pragma unroll
+  for (int jb = 0; jb < kEpiCols; jb += kB) {
+    float a[kB], g[kB];
+#pragma unroll
+    for (int j = 0; j < kB; ++j) {
+      const bool ok = j0 + jb + j < c.n_valid;
+      const int64_t o = (int64_t)(c.n0 + j0 + jb + j) * N + f;
+      a[j] = ok ? __ldg(args.aux + o) : 0.f;
+      g[j] = ok ? __ldg(args.aux2 + o) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < kB; ++j) {
+      if (j0 + jb + j < c.n_valid) {
+        const int64_t o = (int64_t)(c.n0 + j0 + jb + j) * N + f;
+        // silu'(a) = s (1 + a (1 - s)), silu''(a) = s (1 - s) (2 + a (1 - 2 s))
+        const float sg = sigmoid_fast(a[j]);
+        const float s1 = sg * (1.0f + a[j] * (1.0f - sg));
+        const float s2 = sg * (1.0f - sg) * (2.0f + a[j] * (1.0f - 2.0f * sg));
+        args.C[o] = acc[jb + j] * s1;
+        args.C2[o] = acc[jb + j] * g[j] * s2;
+        if (args.C3) args.C3[o] = g[j] * s1;
+      }
+    }
+  }
+}
+
 // Epilogue warpgroups: fold each TMEM chunk into FP32 running sums, then apply
 // the fused epilogue and store this CTA's 128 x 256 part of the tile.
 template <int kMode, int kEpi>
@@ -335,14 +372,17 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader(&s->chunk_empty[p], rank);
-      if (kMode != kModeTN && kEpi == kEpiDSilu && c0 == 0) {
+      if (kMode != kModeTN && (kEpi == kEpiDSilu || kEpi == kEpiD2) && c0 == 0) {
         // the tile's pre-activations travel to L2 while its chunks accumulate
         const int f = c.m0 + q * 32 + lane;
         const int jn = min(kEpiCols, c.n_valid - half * kEpiCols);
         if (f < c.m_end) {
 #pragma unroll 1
-          for (int j = 0; j < jn; ++j)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(args.aux + (int64_t)(c.n0 + half * kEpiCols + j) * N + f));
+          for (int j = 0; j < jn; ++j) {
+            const int64_t o = (int64_t)(c.n0 + half * kEpiCols + j) * N + f;
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(args.aux + o));
+            if (kEpi == kEpiD2) asm volatile("prefetch.global.L2 [%0];" ::"l"(args.aux2 + o));
+          }
         }
       }
     }
@@ -352,6 +392,10 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
       // lanes of a warp write 32 consecutive features (128-byte stores)
       const int f = c.m0 + q * 32 + lane;
       const int j0 = half * kEpiCols;
+      if (kEpi == kEpiD2) {
+        if (f < c.m_end) d2_store(args, acc, c, j0, f, N);
+        continue;
+      }
       if (f < c.m_end) {
         // batches of 8 columns; the pre-activations of batch b + 1 are in
         // flight while batch b is finished, so two loads per column overlap
@@ -396,7 +440,8 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
       continue;
     }
     // weight gradient (plain store): TMEM lane = output row, columns along it
-    static_assert(kMode != kModeTN || kEpi == kEpiStore, "the weight-gradient GEMM has no fused activation");
+    static_assert(kMode != kModeTN || kEpi == kEpiStore || kEpi == kEpiAccum,
+                  "the weight-gradient GEMM has no fused activation");
     const int row = c.m0 + q * 32 + lane;
     const int colb = c.n0 + half * kEpiCols;
     if (row < c.m_end && colb < N) {
@@ -404,7 +449,12 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
 #pragma unroll
       for (int j = 0; j < kEpiCols; j += 4) {
         if (colb + j < N) {
-          *reinterpret_cast<float4*>(args.C + o + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+          float4 v = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+          if (kEpi == kEpiAccum) {
+            const float4 old = *reinterpret_cast<const float4*>(args.C + o + j);
+            v = make_float4(old.x + v.x, old.y + v.y, old.z + v.z, old.w + v.w);
+          }
+          *reinterpret_cast<float4*>(args.C + o + j) = v;
         }
       }
     }
@@ -712,7 +762,8 @@ constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Smem
 // over expert e's rows of A [R,M] and W [R,N] (Kd unused).
 template <int kMode, int kEpi>
 janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, int N, float* C, float* C2,
-                    const float* aux, const int32_t* offsets, int32_t* err, cudaStream_t stream, int M = 0) {
+                    const float* aux, const int32_t* offsets, int32_t* err, cudaStream_t stream, int M = 0,
+                    const float* aux2 = nullptr, float* C3 = nullptr) {
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
@@ -728,7 +779,8 @@ janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, in
     return JANUS_ERR_CUDA;
   }
   Args a;
-  a.C = C; a.C2 = C2; a.aux = aux; a.offsets = offsets; a.E = E; a.Kd = Kd; a.N = N; a.M = M; a.err = err;
+  a.C = C; a.C2 = C2; a.C3 = C3; a.aux = aux; a.aux2 = aux2;
+  a.offsets = offsets; a.E = E; a.Kd = Kd; a.N = N; a.M = M; a.err = err;
   // one CTA per SM, in clusters of two (the MMA pairs)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(num_sms() / 2 * 2));
@@ -787,6 +839,35 @@ janus_status expert_ffn_weight_grad(const float* xd, const float* gd, const floa
   st = launch<kModeTN, kEpiStore>(xd, dA, R, E, 0, h, dw1, nullptr, nullptr, offsets, err, stream, d);
   if (st != JANUS_OK) return st;
   return launch<kModeTN, kEpiStore>(H, gd, R, E, 0, d, dw2, nullptr, nullptr, offsets, err, stream, h);
+}
+
+janus_status expert_ffn_vjp_vjp(const float* xd, const float* gd, const float* vd, const float* act_in, float* A,
+                                const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
+                                const float* w1, const float* w2, float* d_xd, float* d_gd, float* dw1,
+                                float* dw2, float* dh, float* t1, float* t2, float* u, int32_t* err,
+                                cudaStream_t stream) {
+  janus_status st;
+  if (!act_in) {
+    st = launch<kModeNN, kEpiStore>(xd, w1, R, E, d, h, A, nullptr, nullptr, offsets, err, stream);
+    if (st != JANUS_OK) return st;
+  }
+  // dh = gd W2^T
+  st = launch<kModeNT, kEpiStore>(gd, w2, R, E, d, h, dh, nullptr, nullptr, offsets, err, stream);
+  if (st != JANUS_OK) return st;
+  // ub = vd W1 -> t1 = ub silu'(a), t2 = ub dh silu''(a), u = dh silu'(a)
+  st = launch<kModeNN, kEpiD2>(vd, w1, R, E, d, h, t1, t2, A, offsets, err, stream, 0, dh, dw1 ? u : nullptr);
+  if (st != JANUS_OK) return st;
+  // d_gd = t1 W2, d_xd = t2 W1^T
+  st = launch<kModeNN, kEpiStore>(t1, w2, R, E, h, d, d_gd, nullptr, nullptr, offsets, err, stream);
+  if (st != JANUS_OK) return st;
+  st = launch<kModeNT, kEpiStore>(t2, w1, R, E, h, d, d_xd, nullptr, nullptr, offsets, err, stream);
+  if (st != JANUS_OK || !dw1) return st;
+  // dW2 = t1^T gd;  dW1 = vd^T u + xd^T t2
+  st = launch<kModeTN, kEpiStore>(t1, gd, R, E, 0, d, dw2, nullptr, nullptr, offsets, err, stream, h);
+  if (st != JANUS_OK) return st;
+  st = launch<kModeTN, kEpiStore>(vd, u, R, E, 0, h, dw1, nullptr, nullptr, offsets, err, stream, d);
+  if (st != JANUS_OK) return st;
+  return launch<kModeTN, kEpiAccum>(xd, t2, R, E, 0, h, dw1, nullptr, nullptr, offsets, err, stream, d);
 }
 
 }  // namespace tc

@@ -28,5 +28,17 @@ janus_status expert_ffn_weight_grad(const float* xd, const float* gd, const floa
                                     const float* w1, const float* w2, float* dw1, float* dw2, float* dA,
                                     float* H, int32_t* err, cudaStream_t stream);
 
+// Second-order pass (the VJP of the input VJP) for the cotangent vd of dxd:
+//   dh = gd W2^T, t1 = (vd W1) silu'(a), t2 = (vd W1) dh silu''(a), u = dh silu'(a)
+//   d_gd = t1 W2, d_xd = t2 W1^T;  with dw1/dw2 (both or neither):
+//   dW2[e] = T1_e^T Gd_e, dW1[e] = Vd_e^T U_e + Xd_e^T T2_e.
+// dh, t1, t2 (and u with the weight gradients) are [R,h] scratch; A receives a
+// when act_in is NULL.
+janus_status expert_ffn_vjp_vjp(const float* xd, const float* gd, const float* vd, const float* act_in, float* A,
+                                const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
+                                const float* w1, const float* w2, float* d_xd, float* d_gd, float* dw1,
+                                float* dw2, float* dh, float* t1, float* t2, float* u, int32_t* err,
+                                cudaStream_t stream);
+
 }  // namespace tc
 }  // namespace janus

@@ -36,6 +36,7 @@ SYMBOLS = (
     "janus_dequant_by_type",
     "janus_expert_ffn_workspace_size", "janus_expert_ffn_fwd", "janus_expert_ffn_vjp",
     "janus_expert_ffn_weight_grad_workspace_size", "janus_expert_ffn_weight_grad",
+    "janus_expert_ffn_vjp_vjp_workspace_size", "janus_expert_ffn_vjp_vjp",
     "janus_combine", "janus_edge_aggregate", "janus_edge_broadcast", "janus_neighbor_aggregate",
     "janus_debug_inject_launch_failures",
 )
@@ -88,6 +89,9 @@ def _declare(L):
         "janus_expert_ffn_weight_grad_workspace_size": (st, [i64, i32, i32, psz]),
         "janus_expert_ffn_weight_grad": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp,
                                               ctypes.c_int, vp, sz, vp]),
+        "janus_expert_ffn_vjp_vjp_workspace_size": (st, [i64, i32, i32, i32, psz]),
+        "janus_expert_ffn_vjp_vjp": (st, [vp, vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, vp,
+                                          i32, vp, sz, vp]),
         "janus_combine": (st, [vp, vp, vp, i64, i32, i32, vp, vp]),
         "janus_edge_aggregate": (st, [vp, vp, i64, i32, vp, vp]),
         "janus_edge_broadcast": (st, [vp, vp, i64, i32, vp, vp]),
@@ -384,6 +388,46 @@ def janus_expert_ffn_weight_grad(xd, gd, offsets, w1, w2, *, act=None, mode=JANU
                                               int(mode), _p(ws), nb, _stream(stream)),
            "janus_expert_ffn_weight_grad")
     return dw1, dw2
+
+
+def janus_expert_ffn_vjp_vjp_workspace_size(n_rows, h, have_act, want_weight_grad) -> int:
+    b = ctypes.c_size_t(0)
+    _raise(lib().janus_expert_ffn_vjp_vjp_workspace_size(n_rows, h, int(bool(have_act)),
+                                                         int(bool(want_weight_grad)), ctypes.byref(b)),
+           "janus_expert_ffn_vjp_vjp_workspace_size")
+    return b.value
+
+
+def janus_expert_ffn_vjp_vjp(xd, gd, vd, offsets, w1, w2, *, act=None, mode=JANUS_FFN_FP32_SIMT,
+                             weight_grad=False, d_xd=None, d_gd=None, dw1=None, dw2=None,
+                             workspace=None, stream=None):
+    """Second-order pass for the cotangent vd of the input VJP; returns
+    (d_xd, d_gd) or, with weight_grad, (d_xd, d_gd, dw1, dw2)."""
+    R, d = xd.shape
+    E, _, h = w1.shape
+    if d_xd is None:
+        d_xd = _empty((R, d), torch.float32, xd.device)
+    if d_gd is None:
+        d_gd = _empty((R, d), torch.float32, xd.device)
+    if weight_grad:
+        if dw1 is None:
+            dw1 = _empty((E, d, h), torch.float32, w1.device)
+        if dw2 is None:
+            dw2 = _empty((E, h, d), torch.float32, w1.device)
+    nb = janus_expert_ffn_vjp_vjp_workspace_size(R, h, act is not None, weight_grad)
+    ws = _workspace(nb, w1.device, workspace)
+    _raise(lib().janus_expert_ffn_vjp_vjp(_p(xd, torch.float32, "xd"), _p(gd, torch.float32, "gd"),
+                                          _p(vd, torch.float32, "vd"), _p(act, torch.float32, "act"),
+                                          _p(offsets, torch.int32, "offsets"), E, R, d, h,
+                                          _p(w1, torch.float32, "w1"), _p(w2, torch.float32, "w2"),
+                                          _p(d_xd, torch.float32, "d_xd"), _p(d_gd, torch.float32, "d_gd"),
+                                          _p(dw1 if weight_grad else None, torch.float32, "dw1"),
+                                          _p(dw2 if weight_grad else None, torch.float32, "dw2"),
+                                          int(mode), _p(ws), nb, _stream(stream)),
+           "janus_expert_ffn_vjp_vjp")
+    if weight_grad:
+        return d_xd, d_gd, dw1, dw2
+    return d_xd, d_gd
 
 
 # --------------------------------------------------------------------------

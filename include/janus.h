@@ -235,6 +235,34 @@ janus_status janus_expert_ffn_weight_grad(const float* xd, const float* gd, cons
                                           float* dw1, float* dw2, janus_ffn_mode mode, void* workspace,
                                           size_t workspace_bytes, janus_stream_t stream);
 
+/* Second-order pass: the VJP of the input VJP.  Force training fits forces,
+ * which are input gradients of the energy ([Review] section 3.3), so a loss on
+ * them sends its gradient back through janus_expert_ffn_vjp.  With
+ * dxd = W1((W2 gd) * silu'(a)), a = xd W1, per row, and vd the cotangent of dxd
+ * (L = sum_p <dxd[p,:], vd[p,:]>):
+ *   ub = vd W1,  t1 = ub * silu'(a),  t2 = ub * (gd W2^T) * silu''(a)
+ *   d_xd = dL/dxd = t2 W1^T,  d_gd = dL/dgd = t1 W2
+ *   dW1[e] = sum_{p in e} vd[p]^T u[p] + xd[p]^T t2[p],  u = (gd W2^T) * silu'(a)
+ *   dW2[e] = sum_{p in e} t1[p]^T gd[p]
+ *   silu''(a) = sig(a) (1 - sig(a)) (2 + a (1 - 2 sig(a))).
+ * in : xd, gd, vd [R,d]; act [R,h] from the forward, or NULL to recompute;
+ *      offsets [E+1]; w1 [E,d,h], w2 [E,h,d] (all device, float32, 16-byte
+ *      aligned, d and h multiples of 4)
+ * out: d_xd, d_gd [R,d]; dw1 [E,d,h] and dw2 [E,h,d], both or neither
+ *      (NULL skips the weight part; experts without rows get zeros).
+ * workspace: janus_expert_ffn_vjp_vjp_workspace_size() bytes, 256-byte
+ *      aligned (dh, t1, t2, u with the weight part, a without act: [R,h]
+ *      each).  Errors as janus_expert_ffn_fwd; JANUS_ERR_INVALID_ARG if only one
+ *      of dw1, dw2 is given.  3xTF32 timeouts are reported by janus_check. */
+janus_status janus_expert_ffn_vjp_vjp_workspace_size(int64_t n_rows, int32_t h, int32_t have_act,
+                                                     int32_t want_weight_grad, size_t* bytes);
+janus_status janus_expert_ffn_vjp_vjp(const float* xd, const float* gd, const float* vd,
+                                      const float* act, const int32_t* offsets, int32_t n_experts,
+                                      int64_t n_rows, int32_t d, int32_t h, const float* w1,
+                                      const float* w2, float* d_xd, float* d_gd, float* dw1, float* dw2,
+                                      janus_ffn_mode mode, void* workspace, size_t workspace_bytes,
+                                      janus_stream_t stream);
+
 /* -------------------------------------------------------------------------
  * Combine.  [Blueprint] section 3.2 (aggregation and output layer): the
  * activated experts' outputs are summed with the gate weights.  Gather form
