@@ -46,6 +46,8 @@ def _setup(L):
     L.orc_expert_ffn_vjp_vjp.argtypes = [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, i64, vp, vp]
     L.orc_expert_ffn_vjp_vjp_weight_grad.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp]
     L.orc_combine.argtypes = [vp, vp, vp, i64, i32, i32, vp]
+    L.orc_ep_layout.argtypes = [vp, i32, i32, vp, vp, vp]
+    L.orc_ep_layout.restype = ctypes.c_int
     L.orc_edge_aggregate.argtypes = [vp, vp, i64, i32, vp]
     L.orc_edge_broadcast.argtypes = [vp, vp, i64, i32, vp]
     L.orc_neighbor_aggregate.argtypes = [vp, vp, vp, i64, i32, vp]
@@ -204,6 +206,21 @@ def expert_ffn_vjp_vjp_weight_grad(xd, gd, vd, offsets, w1, w2):
     lib().orc_expert_ffn_vjp_vjp_weight_grad(_p(xd), _p(gd), _p(vd), _p(offsets), E, d, h,
                                              _p(w1), _p(w2), _p(dw1), _p(dw2))
     return dw1, dw2
+
+
+def ep_layout(counts_all):
+    """Expert-parallel exchange layout from the all-gathered counts [P, E]:
+    (src_off [P, E+1], dst_off [P, E], recv_off [P, E/P+1])."""
+    c = _c(counts_all, np.int32)
+    P, E = c.shape
+    if E % P:
+        raise ValueError("E must be a multiple of the number of ranks")
+    src = np.empty((P, E + 1), np.int32)
+    dst = np.empty((P, E), np.int32)
+    recv = np.empty((P, E // P + 1), np.int32)
+    if lib().orc_ep_layout(_p(c), P, E, _p(src), _p(dst), _p(recv)) != 0:
+        raise ValueError("bad layout arguments")
+    return src, dst, recv
 
 
 def combine(yd, slot_of, top_k, topk_weight=None):

@@ -465,6 +465,50 @@ void orc_expert_ffn_vjp_vjp_weight_grad(const float* xd, const float* gd, const 
 }
 
 // ---------------------------------------------------------------------------
+// Expert-parallel exchange layout.  [Review] section 3.4 (FSEP: experts are
+// sharded over ranks) and section 3.5 (the dispatch all-to-all of the packed
+// rows).  P ranks; rank o owns experts [o*E/P, (o+1)*E/P) (E divisible by P).
+// counts_all[s][e] = rows rank s routed to expert e.  Definitions:
+//   src_off[s][e]  = sum_{e' < e} counts_all[s][e']        (sender's local dispatch
+//                    order is expert-major; src_off[s][E] = its row count)
+//   recv_off[o][j] = sum_{local experts j' < j of o} sum_s counts_all[s][o*E/P + j']
+//                    (the owner groups received rows by local expert, then sender)
+//   dst_off[s][e]  = recv_off[owner(e)][e - owner(e)*E/P] + sum_{s' < s} counts_all[s'][e]
+// Row i of (s, e) travels from sender row src_off[s][e] + i to owner row
+// dst_off[s][e] + i.  Returns 0, or -1 if E is not a multiple of P.
+// ---------------------------------------------------------------------------
+int orc_ep_layout(const int32_t* counts_all, int32_t P, int32_t E, int32_t* src_off, int32_t* dst_off,
+                  int32_t* recv_off) {
+  if (P < 1 || E < P || E % P != 0) return -1;
+  const int El = E / P;
+  for (int s = 0; s < P; ++s) {
+    int64_t acc = 0;
+    for (int e = 0; e < E; ++e) {
+      src_off[s * (E + 1) + e] = (int32_t)acc;
+      acc += counts_all[s * E + e];
+    }
+    src_off[s * (E + 1) + E] = (int32_t)acc;
+  }
+  for (int o = 0; o < P; ++o) {
+    int64_t acc = 0;
+    for (int j = 0; j < El; ++j) {
+      recv_off[o * (El + 1) + j] = (int32_t)acc;
+      for (int s = 0; s < P; ++s) acc += counts_all[s * E + o * El + j];
+    }
+    recv_off[o * (El + 1) + El] = (int32_t)acc;
+  }
+  for (int e = 0; e < E; ++e) {
+    const int o = e / El, j = e - o * El;
+    int64_t acc = recv_off[o * (El + 1) + j];
+    for (int s = 0; s < P; ++s) {
+      dst_off[s * E + e] = (int32_t)acc;
+      acc += counts_all[s * E + e];
+    }
+  }
+  return 0;
+}
+
+// ---------------------------------------------------------------------------
 // Combine.  [Blueprint] §3.2: the activated experts' outputs are summed with
 // the gate weights.  Gather form: Y[i,:] = sum_{k ascending} w[i,k] *
 // Yd[slot_of[i*K+k],:]; topk_weight == NULL means weight 1 (the VJP combine).
