@@ -38,8 +38,19 @@ SYMBOLS = (
     "janus_expert_ffn_weight_grad_workspace_size", "janus_expert_ffn_weight_grad",
     "janus_expert_ffn_vjp_vjp_workspace_size", "janus_expert_ffn_vjp_vjp",
     "janus_combine", "janus_edge_aggregate", "janus_edge_broadcast", "janus_neighbor_aggregate",
+    "janus_ep_layout", "janus_ep_dispatch_quant", "janus_ep_dispatch", "janus_ep_dequant_rows",
+    "janus_ep_return", "janus_ipc_get_handle", "janus_ipc_open_handle", "janus_ipc_close_handle",
     "janus_debug_inject_launch_failures",
 )
+
+
+JANUS_EP_MAX_RANKS = 8
+
+
+class IpcHandle(ctypes.Structure):
+    """janus_ipc_handle: the allocation's CUDA IPC handle and the byte offset
+    of the pointer inside it."""
+    _fields_ = [("bytes", ctypes.c_ubyte * 64), ("offset", ctypes.c_uint64)]
 
 
 class JanusError(RuntimeError):
@@ -96,6 +107,15 @@ def _declare(L):
         "janus_edge_aggregate": (st, [vp, vp, i64, i32, vp, vp]),
         "janus_edge_broadcast": (st, [vp, vp, i64, i32, vp, vp]),
         "janus_neighbor_aggregate": (st, [vp, vp, vp, i64, i32, vp, vp]),
+        "janus_ep_layout": (st, [vp, i32, i32, vp, vp, vp, vp]),
+        "janus_ep_dispatch_quant": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp,
+                                         vp, sz, vp]),
+        "janus_ep_dispatch": (st, [vp, i64, i32, i32, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp]),
+        "janus_ep_dequant_rows": (st, [vp, vp, vp, i32, i32, i32, i64, i32, vp, vp]),
+        "janus_ep_return": (st, [vp, vp, vp, vp, vp, i32, i32, i32, i64, i32, vp, vp]),
+        "janus_ipc_get_handle": (st, [vp, ctypes.POINTER(IpcHandle)]),
+        "janus_ipc_open_handle": (st, [ctypes.POINTER(IpcHandle), ctypes.POINTER(ctypes.c_void_p)]),
+        "janus_ipc_close_handle": (st, [vp, ctypes.c_uint64]),
         "janus_debug_inject_launch_failures": (None, [i32]),
     }
     for name, (res, args) in sig.items():
@@ -244,6 +264,113 @@ def janus_combine(yd, slot_of, top_k, topk_weight=None, *, out=None, stream=None
                                _p(topk_weight, torch.float32, "topk_weight"), N, K, d,
                                _p(out, torch.float32, "y"), _stream(stream)), "janus_combine")
     return out
+
+
+# --------------------------------------------------------------------------
+# expert-parallel exchange (rank o owns experts [o*E/P, (o+1)*E/P))
+# --------------------------------------------------------------------------
+def _ptr_array(ptrs):
+    """Host array of device pointers (index = rank) from tensors or ints."""
+    vals = [t.data_ptr() if isinstance(t, torch.Tensor) else int(t) for t in ptrs]
+    return (ctypes.c_void_p * len(vals))(*vals)
+
+
+def janus_ep_layout(counts_all, n_experts, *, src_off=None, dst_off=None, recv_off=None, stream=None):
+    """Exchange layout from the gathered counts [P, E]: (src_off [P, E+1],
+    dst_off [P, E], recv_off [P, E/P+1]), device int32."""
+    P = counts_all.shape[0]
+    E = int(n_experts)
+    dev = counts_all.device
+    if src_off is None:
+        src_off = _empty((P, E + 1), torch.int32, dev)
+    if dst_off is None:
+        dst_off = _empty((P, E), torch.int32, dev)
+    if recv_off is None:
+        recv_off = _empty((P, E // max(P, 1) + 1), torch.int32, dev)
+    _raise(lib().janus_ep_layout(_p(counts_all, torch.int32, "counts_all"), P, E,
+                                 _p(src_off, torch.int32, "src_off"), _p(dst_off, torch.int32, "dst_off"),
+                                 _p(recv_off, torch.int32, "recv_off"), _stream(stream)), "janus_ep_layout")
+    return src_off, dst_off, recv_off
+
+
+def janus_ep_dispatch_quant(x, types, n_types, route, layout, rank, recv_payload, recv_scale, *,
+                            scale=None, workspace=None, stream=None):
+    """FP16-pack this rank's routed rows and store them in their owners'
+    receive buffers (recv_payload / recv_scale: one per rank, index = rank).
+    Returns (scale [T], workspace)."""
+    N, d = x.shape
+    K = route["topk_expert"].shape[1]
+    src_off, dst_off, _ = layout
+    P, E = dst_off.shape
+    if scale is None:
+        scale = _empty((int(n_types),), torch.float32, x.device)
+    nb = janus_quant_by_type_workspace_size(n_types)
+    ws = _workspace(nb, x.device, workspace)
+    _raise(lib().janus_ep_dispatch_quant(_p(x, torch.float32, "x"), N, d, K, _p(types, torch.int32, "types"),
+                                         int(n_types), _p(route["slot_of"], torch.int32, "slot_of"),
+                                         _p(route["topk_expert"], torch.int32, "topk_expert"),
+                                         _p(src_off, torch.int32, "src_off"), _p(dst_off, torch.int32, "dst_off"),
+                                         int(rank), P, E, _ptr_array(recv_payload), _ptr_array(recv_scale),
+                                         _p(scale, torch.float32, "scale"), _p(ws), nb, _stream(stream)),
+           "janus_ep_dispatch_quant")
+    return scale, ws
+
+
+def janus_ep_dispatch(x, route, layout, rank, recv_rows, *, weighted=False, stream=None):
+    """FP32 send of this rank's rows (times the gate weight when weighted) to
+    their owners' receive buffers."""
+    N, d = x.shape
+    K = route["topk_expert"].shape[1]
+    src_off, dst_off, _ = layout
+    P, E = dst_off.shape
+    _raise(lib().janus_ep_dispatch(_p(x, torch.float32, "x"), N, d, K, _p(route["slot_of"], torch.int32, "slot_of"),
+                                   _p(route["topk_expert"], torch.int32, "topk_expert"),
+                                   _p(route["topk_weight"] if weighted else None, torch.float32, "topk_weight"),
+                                   _p(src_off, torch.int32, "src_off"), _p(dst_off, torch.int32, "dst_off"),
+                                   int(rank), P, E, _ptr_array(recv_rows), _stream(stream)), "janus_ep_dispatch")
+
+
+def janus_ep_dequant_rows(payload, row_scale, layout, rank, *, out=None, stream=None):
+    """Owner side of the FP16 send: received rows times their scales."""
+    max_rows, d = payload.shape
+    _, dst_off, recv_off = layout
+    P, E = dst_off.shape
+    if out is None:
+        out = _empty((max_rows, d), torch.float32, payload.device)
+    _raise(lib().janus_ep_dequant_rows(_p(payload, torch.float16, "payload"), _p(row_scale, torch.float32, "row_scale"),
+                                       _p(recv_off, torch.int32, "recv_off"), int(rank), P, E, max_rows, d,
+                                       _p(out, torch.float32, "xd"), _stream(stream)), "janus_ep_dequant_rows")
+    return out
+
+
+def janus_ep_return(yd, counts_all, layout, rank, ret_rows, *, stream=None):
+    """Owner side of the return: each received row's result to its sender."""
+    max_rows, d = yd.shape
+    src_off, dst_off, recv_off = layout
+    P, E = dst_off.shape
+    _raise(lib().janus_ep_return(_p(yd, torch.float32, "yd"), _p(counts_all, torch.int32, "counts_all"),
+                                 _p(src_off, torch.int32, "src_off"), _p(dst_off, torch.int32, "dst_off"),
+                                 _p(recv_off, torch.int32, "recv_off"), int(rank), P, E, max_rows, d,
+                                 _ptr_array(ret_rows), _stream(stream)), "janus_ep_return")
+
+
+def janus_ipc_get_handle(t) -> bytes:
+    """Serialised janus_ipc_handle of a device tensor's storage."""
+    h = IpcHandle()
+    _raise(lib().janus_ipc_get_handle(ctypes.c_void_p(t.data_ptr()), ctypes.byref(h)), "janus_ipc_get_handle")
+    return bytes(h)
+
+
+def janus_ipc_open_handle(blob: bytes) -> tuple:
+    """Map another process's buffer: returns (device pointer, offset)."""
+    h = IpcHandle.from_buffer_copy(blob)
+    p = ctypes.c_void_p(0)
+    _raise(lib().janus_ipc_open_handle(ctypes.byref(h), ctypes.byref(p)), "janus_ipc_open_handle")
+    return p.value, int(h.offset)
+
+
+def janus_ipc_close_handle(ptr: int, offset: int):
+    _raise(lib().janus_ipc_close_handle(ctypes.c_void_p(ptr), ctypes.c_uint64(offset)), "janus_ipc_close_handle")
 
 
 # --------------------------------------------------------------------------

@@ -264,6 +264,92 @@ janus_status janus_expert_ffn_vjp_vjp(const float* xd, const float* gd, const fl
                                       janus_stream_t stream);
 
 /* -------------------------------------------------------------------------
+ * Expert-parallel exchange.  [Review] section 3.4 (FSEP: experts sharded over
+ * ranks) and section 3.5 (the MoE all-to-all moves atom-type-aware FP16 rows,
+ * half the FP32 volume).  P ranks, one process per GPU of a node; rank o owns
+ * experts [o*E/P, (o+1)*E/P) (E a multiple of P, P <= JANUS_EP_MAX_RANKS).
+ * Every rank calls janus_route on its own atoms; the counts of all ranks,
+ * gathered in rank order into counts_all [P,E] (device int32), fix the layout:
+ *   src_off [P,E+1]: src_off[s][e] = sum_{e'<e} counts_all[s][e'] (sender s's
+ *                    local dispatch order; equals its janus_route offsets)
+ *   recv_off [P,E/P+1]: owner o's rows per local expert, summed over senders
+ *                    (o's receive buffer: grouped by local expert, then sender;
+ *                    the expert MLP runs on recv_off[o] directly)
+ *   dst_off [P,E]:  dst_off[s][e] = recv_off[owner(e)][e - owner(e)*E/P]
+ *                    + sum_{s'<s} counts_all[s'][e]
+ * Row i of (s, e) moves from sender row src_off[s][e] + i to owner row
+ * dst_off[s][e] + i, and back.
+ *
+ * The send and return calls store straight into the other ranks' buffers:
+ * the pointer arrays (host arrays of P device pointers, index = rank) hold the
+ * local buffer at this rank's index and peer-mapped buffers elsewhere
+ * (janus_ipc_open_handle).  No call waits on another rank: a call's stores are
+ * complete when its stream work is, and the caller orders the phases (a
+ * collective barrier after each send/return, before the receiver reads).
+ * Buffers are sized by the caller: a receive buffer holds at least the
+ * owner's recv_off[o][E/P] rows (max_rows is its capacity); rows past the
+ * received count are left untouched.  top_k <= 32 for the send calls.
+ * ------------------------------------------------------------------------- */
+#define JANUS_EP_MAX_RANKS 8
+
+/* One CTA; writes src_off, dst_off, recv_off (device int32, layouts above). */
+janus_status janus_ep_layout(const int32_t* counts_all, int32_t world, int32_t n_experts,
+                             int32_t* src_off, int32_t* dst_off, int32_t* recv_off,
+                             janus_stream_t stream);
+
+/* Forward send with the FP16 packing of janus_quant_by_type (this rank's
+ * per-type power-of-two absmax scales, written to scale [T]): for each of
+ * this rank's atoms i and k < K, with e = topk_expert[i*K+k] and
+ * p = slot_of[i*K+k], owner o = e/(E/P), row r = dst_off[rank][e] + p -
+ * src_off[rank][e]:  recv_payload[o][r,:] = fp16(x[i,:] / scale[types[i]]),
+ * recv_scale[o][r] = scale[types[i]].  recv_payload[o]: 8-byte aligned.
+ * workspace: janus_quant_by_type_workspace_size(n_types) bytes; bad type ids
+ * and non-finite rows are reported by janus_check as in janus_quant_by_type. */
+janus_status janus_ep_dispatch_quant(const float* x, int64_t n_atoms, int32_t d, int32_t top_k,
+                                     const int32_t* types, int32_t n_types, const int32_t* slot_of,
+                                     const int32_t* topk_expert, const int32_t* src_off,
+                                     const int32_t* dst_off, int32_t rank, int32_t world,
+                                     int32_t n_experts, uint16_t* const* recv_payload,
+                                     float* const* recv_scale, float* scale, void* workspace,
+                                     size_t workspace_bytes, janus_stream_t stream);
+
+/* FP32 send (the gradient direction): recv_rows[o][r,:] = w * x[i,:] with
+ * w = topk_weight[i*K+k] (1 when topk_weight is NULL), same (o, r) as above. */
+janus_status janus_ep_dispatch(const float* x, int64_t n_atoms, int32_t d, int32_t top_k,
+                               const int32_t* slot_of, const int32_t* topk_expert,
+                               const float* topk_weight, const int32_t* src_off, const int32_t* dst_off,
+                               int32_t rank, int32_t world, int32_t n_experts, float* const* recv_rows,
+                               janus_stream_t stream);
+
+/* Owner side of the FP16 send: xd[r,:] = f32(payload[r,:]) * row_scale[r] for
+ * r < recv_off[rank][E/P] (read on the device; at most max_rows). */
+janus_status janus_ep_dequant_rows(const uint16_t* payload, const float* row_scale, const int32_t* recv_off,
+                                   int32_t rank, int32_t world, int32_t n_experts, int64_t max_rows,
+                                   int32_t d, float* xd, janus_stream_t stream);
+
+/* Owner side of the return: for each received row r (r < recv_off[rank][E/P],
+ * at most max_rows) of sender s and expert e, ret_rows[s][src_off[s][e] + r -
+ * dst_off[s][e], :] = yd[r,:].  The sender then runs janus_combine on its
+ * return buffer as on a local expert output. */
+janus_status janus_ep_return(const float* yd, const int32_t* counts_all, const int32_t* src_off,
+                             const int32_t* dst_off, const int32_t* recv_off, int32_t rank, int32_t world,
+                             int32_t n_experts, int64_t max_rows, int32_t d, float* const* ret_rows,
+                             janus_stream_t stream);
+
+/* CUDA IPC, so ranks on one node can map each other's buffers.  A handle names
+ * the allocation that holds dev_ptr plus dev_ptr's byte offset in it (callers
+ * may pass pointers into a caching allocator's blocks).  Open returns the
+ * mapped pointer with the offset applied; close takes that pointer and the
+ * same offset.  Opening a handle in the process that created it fails. */
+typedef struct {
+  unsigned char bytes[64];
+  uint64_t offset;
+} janus_ipc_handle;
+janus_status janus_ipc_get_handle(const void* dev_ptr, janus_ipc_handle* out);
+janus_status janus_ipc_open_handle(const janus_ipc_handle* handle, void** dev_ptr);
+janus_status janus_ipc_close_handle(void* dev_ptr, uint64_t offset);
+
+/* -------------------------------------------------------------------------
  * Combine.  [Blueprint] section 3.2 (aggregation and output layer): the
  * activated experts' outputs are summed with the gate weights.  Gather form
  * of the weighted scatter-add (deterministic, no atomics):
