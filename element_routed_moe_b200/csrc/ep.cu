@@ -136,6 +136,8 @@ ep_pack_send_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K
       }
     }
   }
+  // the peer stores are visible system-wide before this kernel completes
+  __threadfence_system();
 }
 
 // FP32 send (the gradient direction): row x[i] (times the gate weight when
@@ -176,6 +178,8 @@ ep_send_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K, con
       }
     }
   }
+  // the peer stores are visible system-wide before this kernel completes
+  __threadfence_system();
 }
 
 // Owner side: received FP16 rows times their own scale (exact: powers of two).
@@ -245,6 +249,8 @@ ep_return_kernel(const float4* __restrict__ yd, const int32_t* __restrict__ coun
       }
     }
   }
+  // the peer stores are visible system-wide before this kernel completes
+  __threadfence_system();
 }
 
 janus_status check_ep(int32_t rank, int32_t world, int32_t n_experts) {

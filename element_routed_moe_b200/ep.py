@@ -1,0 +1,140 @@
+"""Expert-parallel MoE layer over the ranks of one node (one process per GPU).
+
+Paper review "Breaking the Training Barrier of Billion-Parameter Universal
+Machine Learning Interatomic Potentials", section 3.4 (FSEP: experts sharded
+over ranks) and section 3.5 (the MoE all-to-all of atom-type-aware FP16
+rows).  Rank o holds the weights of experts [o*E/P, (o+1)*E/P) and its own
+atoms.  One layer pass:
+
+  forward:  route (local) -> gather counts -> layout -> FP16 pack-and-send to
+            the owners -> barrier -> owner: unpack, experts -> return to the
+            senders -> barrier -> combine (local)
+  VJP:      weighted FP32 send of dY -> barrier -> owner: input VJP of its
+            experts -> return -> barrier -> combine (local)
+
+Every step is a kernel of libjanus; torch.distributed carries only the
+counts, the IPC handles (once) and the phase barriers.  The receive and return
+buffers are allocated once at their worst-case size (all routed rows of all
+ranks), so no step waits for the host to learn a count.  With NCCL a barrier
+is a one-element all-reduce on the current stream (stream-ordered: every
+rank's send kernel has finished before any rank passes it); with gloo it is a
+stream synchronize plus a host barrier.
+"""
+import torch
+import torch.distributed as dist
+
+from . import janus as J
+
+
+class ExpertParallelLayer:
+    """Buffers, peer mappings and the ordered calls of one EP layer pass."""
+
+    def __init__(self, n_atoms_max, d, h, n_types, n_experts, top_k, w1_local, w2_local, *,
+                 mode=J.JANUS_FFN_3XTF32, group=None, device=None):
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        if self.world > J.JANUS_EP_MAX_RANKS:
+            raise ValueError(f"at most {J.JANUS_EP_MAX_RANKS} ranks (one node)")
+        if n_experts % self.world:
+            raise ValueError("the number of experts must be a multiple of the number of ranks")
+        self.dev = torch.device(device) if device is not None else w1_local.device
+        self.d, self.h, self.T, self.E, self.K = d, h, n_types, n_experts, top_k
+        self.El = n_experts // self.world
+        if w1_local.shape != (self.El, d, h) or w2_local.shape != (self.El, h, d):
+            raise ValueError("w1_local / w2_local must hold this rank's E/P experts")
+        self.w1, self.w2, self.mode = w1_local, w2_local, mode
+        self.nccl = dist.get_backend(group) == "nccl"
+        # worst case: every routed row of every rank lands on this rank
+        self.n_atoms_max = int(n_atoms_max)
+        cap = max(self.world * self.n_atoms_max * top_k, 1)
+        rows = max(self.n_atoms_max * top_k, 1)
+        f32 = dict(dtype=torch.float32, device=self.dev)
+        self.cap = cap
+        self.payload = torch.empty((cap, d), dtype=torch.float16, device=self.dev)
+        self.row_scale = torch.empty((cap,), **f32)
+        self.recv_rows = torch.empty((cap, d), **f32)       # gradients in, outputs out
+        self.xd = torch.empty((cap, d), **f32)
+        self.act = torch.empty((cap, h), **f32)
+        self.yd = torch.empty((cap, d), **f32)
+        self.ret = torch.empty((rows, d), **f32)             # this rank's rows coming back
+        self.counts_all = torch.empty((self.world, n_experts), dtype=torch.int32, device=self.dev)
+        self._token = torch.zeros(1, **f32)
+        self._opened = []
+        self.peer_payload = self._exchange(self.payload)
+        self.peer_scale = self._exchange(self.row_scale)
+        self.peer_rows = self._exchange(self.recv_rows)
+        self.peer_ret = self._exchange(self.ret)
+
+    # -- plumbing ------------------------------------------------------------
+    def _exchange(self, t):
+        """Device pointers of every rank's copy of buffer t (index = rank)."""
+        blob = J.janus_ipc_get_handle(t) if self.world > 1 else b""
+        blobs = [None] * self.world
+        dist.all_gather_object(blobs, blob, group=self.group)
+        ptrs = []
+        for r, b in enumerate(blobs):
+            if r == self.rank:
+                ptrs.append(t.data_ptr())
+            else:
+                p, off = J.janus_ipc_open_handle(b)
+                self._opened.append((p, off))
+                ptrs.append(p)
+        return ptrs
+
+    def barrier(self):
+        """Every rank's work queued so far (its peer stores included) is done
+        before any rank's next step runs."""
+        if self.nccl:
+            dist.all_reduce(self._token, group=self.group)
+        else:
+            torch.cuda.current_stream(self.dev).synchronize()
+            dist.barrier(group=self.group)
+
+    def _gather_counts(self, counts):
+        if self.nccl:
+            dist.all_gather_into_tensor(self.counts_all, counts, group=self.group)
+        else:
+            parts = [torch.empty_like(counts.cpu()) for _ in range(self.world)]
+            dist.all_gather(parts, counts.cpu(), group=self.group)
+            self.counts_all.copy_(torch.stack(parts))
+
+    def close(self):
+        torch.cuda.synchronize(self.dev)
+        dist.barrier(group=self.group)          # no rank still writes into a mapping
+        for p, off in self._opened:
+            J.janus_ipc_close_handle(p, off)
+        self._opened = []
+
+    # -- the layer -------------------------------------------------------------
+    def forward(self, x, types, gate):
+        """y [N,d] for this rank's atoms (FP16-packed dispatch)."""
+        if x.shape[0] > self.n_atoms_max:
+            raise ValueError("more atoms than the buffers were sized for")
+        self.x_shape = x.shape
+        self.route = J.janus_route(types, gate, self.K)
+        self._gather_counts(self.route["counts"])
+        self.layout = J.janus_ep_layout(self.counts_all, self.E)
+        J.janus_ep_dispatch_quant(x, types, self.T, self.route, self.layout, self.rank,
+                                  self.peer_payload, self.peer_scale)
+        self.barrier()
+        recv_off = self.layout[2][self.rank]
+        J.janus_ep_dequant_rows(self.payload, self.row_scale, self.layout, self.rank, out=self.xd)
+        J.janus_expert_ffn_fwd(self.xd, recv_off, self.w1, self.w2, mode=self.mode, out=self.yd, act=self.act)
+        J.janus_ep_return(self.yd, self.counts_all, self.layout, self.rank, self.peer_ret)
+        self.barrier()
+        R = x.shape[0] * self.K
+        return J.janus_combine(self.ret[:R], self.route["slot_of"], self.K, self.route["topk_weight"])
+
+    def vjp(self, g):
+        """dx [N,d] for the upstream gradient g [N,d] of forward's output."""
+        r = self.route
+        J.janus_ep_dispatch(g, r, self.layout, self.rank, self.peer_rows, weighted=True)
+        self.barrier()
+        recv_off = self.layout[2][self.rank]
+        J.janus_expert_ffn_vjp(self.xd, self.recv_rows, recv_off, self.w1, self.w2, act=self.act,
+                               mode=self.mode, out=self.yd)
+        J.janus_ep_return(self.yd, self.counts_all, self.layout, self.rank, self.peer_ret)
+        self.barrier()
+        R = self.x_shape[0] * self.K
+        return J.janus_combine(self.ret[:R], r["slot_of"], self.K)

@@ -1,0 +1,91 @@
+"""The expert-parallel layer across two processes ([Review] 'Breaking the
+Training Barrier of Billion-Parameter Universal Machine Learning Interatomic
+Potentials', sections 3.4-3.5), with the rank-to-rank stores going through
+real CUDA IPC mappings of the other process's buffers.
+
+Both processes share one GPU (each has its own context); the phases are
+ordered by stream synchronisation plus a gloo barrier, and no kernel waits on
+another.  Each rank's forward and input-VJP results must equal its own
+single-GPU chain with all experts local.
+"""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, mode, q):
+    try:
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        sys.path.insert(0, ROOT)
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        import datetime
+        import torch
+        import torch.distributed as dist
+        from element_routed_moe_b200 import janus as J
+        from element_routed_moe_b200 import synth
+        from element_routed_moe_b200.ep import ExpertParallelLayer
+        from helpers import rel_fro
+        dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+        dev = torch.device("cuda:0")
+        torch.cuda.set_device(dev)
+        N, T, E, K, d, h = 257 + 31 * rank, 89, 8, 2, 128, 96
+        El = E // world
+        gate = torch.as_tensor(synth.gate_table(T, E, 1), device=dev)
+        w1, w2 = synth.expert_weights(E, d, h, 2, dev)
+        x = synth.normal((N, d), 10 + rank, dev)
+        types = torch.as_tensor(synth.types_zipf(N, T, seed=20 + rank), device=dev)
+        g = synth.normal((N, d), 30 + rank, dev)
+        layer = ExpertParallelLayer(400, d, h, T, E, K, w1[rank * El:(rank + 1) * El].contiguous(),
+                                    w2[rank * El:(rank + 1) * El].contiguous(), mode=mode, device=dev)
+        errs = []
+        for _ in range(2):                                  # buffers reused across passes
+            y = layer.forward(x, types, gate)
+            dx = layer.vjp(g)
+            torch.cuda.synchronize()
+            # local chain, all experts on this rank
+            r = J.janus_route(types, gate, K)
+            payload, scale, _ = J.janus_quant_by_type(x, types, T, r["slot_of"], K)
+            xd = J.janus_dequant_by_type(payload, types, T, r["perm"], K, scale)
+            yd, act = J.janus_expert_ffn_fwd(xd, r["offsets"], w1, w2, mode=mode, want_act=True)
+            y_ref = J.janus_combine(yd, r["slot_of"], K, r["topk_weight"])
+            gd = J.janus_dispatch(g, r["slot_of"], K, r["topk_weight"])
+            dxd = J.janus_expert_ffn_vjp(xd, gd, r["offsets"], w1, w2, act=act, mode=mode)
+            dx_ref = J.janus_combine(dxd, r["slot_of"], K)
+            errs.append((rel_fro(y.cpu().numpy(), y_ref.cpu().numpy()),
+                         rel_fro(dx.cpu().numpy(), dx_ref.cpu().numpy())))
+        layer.close()
+        dist.destroy_process_group()
+        q.put((rank, "ok", errs))
+    except Exception as e:  # report, do not hang the parent
+        q.put((rank, "error", repr(e)))
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_ep_layer_two_processes_through_ipc(mode):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, mode, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=300) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+    for rank, status, payload in results:
+        assert status == "ok", (rank, payload)
+        for ey, edx in payload:
+            assert ey <= 1e-6 and edx <= 1e-6, (rank, ey, edx)
+    assert all(p.exitcode == 0 for p in procs)
