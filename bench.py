@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--atoms", type=int, default=None, help="override N (profiling small cases)")
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling small cases)")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism over the ranks (experts split, FP16 all-to-all by peer "
+                         "stores) instead of independent replicas")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip timing the weight-gradient, multi-layer routing and edge-side calls")
     ap.add_argument("--ref-seconds", type=float, default=None,
@@ -526,6 +529,87 @@ def run_janus(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_ep(args, world, rank, local):
+    """The layer pass with experts split over the ranks (each rank: its own
+    N atoms, E/P experts); same metric, whole-job tokens per second."""
+    from element_routed_moe_b200 import janus as J
+    from element_routed_moe_b200.ep import ExpertParallelLayer
+    J.lib()
+    dev = torch.device("cuda", local)
+    cfg = workload(args)
+    N, T, E, K, d, h = cfg.n_atoms, cfg.n_types, cfg.n_experts, cfg.top_k, cfg.d, cfg.h
+    if E % world:
+        raise SystemExit(f"--ep needs E ({E}) divisible by the number of ranks ({world})")
+    mode = J.JANUS_FFN_3XTF32 if args.mode == "3xtf32" else J.JANUS_FFN_FP32_SIMT
+    inp = synth.layer_inputs(cfg, seed=args.seed + 1000 * rank, device=dev, with_edges=False)
+    gate = torch.as_tensor(synth.gate_table(T, E, args.seed + 2), device=dev)     # the same on every rank
+    w1, w2 = synth.expert_weights(E, d, h, args.seed + 3, dev)
+    El = E // world
+    w1l, w2l = w1[rank * El:(rank + 1) * El].contiguous(), w2[rank * El:(rank + 1) * El].contiguous()
+    del w1, w2, inp["w1"], inp["w2"]
+    types = torch.as_tensor(inp["types"], device=dev)
+    x, g = inp["x"], inp["g"]
+    layer = ExpertParallelLayer(N, d, h, T, E, K, w1l, w2l, mode=mode, device=dev)
+    peaks, peak_src = measured_peaks()
+    for _ in range(args.warmup):
+        layer.forward(x, types, gate)
+        layer.vjp(g)
+    torch.cuda.synchronize()
+    phases = ExpertParallelLayer.PHASES_FWD + ExpertParallelLayer.PHASES_VJP
+    ev = [{ph: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for ph in phases}
+          for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local))
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    t_start.record()
+    for k in range(args.steps):
+        layer.forward(x, types, gate, events=ev[k])
+        layer.vjp(g, events=ev[k])
+    t_end.record()
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    clocks = sampler.stop(wall0, wall1)
+    barrier(world)
+    elapsed = t_start.elapsed_time(t_end) / 1e3
+    t_max = max_over_ranks(elapsed, world)
+    value = N * K * world * args.steps / t_max
+    ph_ms = {ph: float(np.mean([e[ph][0].elapsed_time(e[ph][1]) for e in ev])) for ph in phases}
+    # this rank's expert GEMMs: 4 of 2 * R_recv * d * h FLOPs each (fwd + VJP)
+    r_recv = int(layer.layout[2][rank][-1].item())
+    ffn_flops = 8.0 * r_recv * d * h
+    ffn_ms = ph_ms["ffn_fwd"] + ph_ms["ffn_vjp"]
+    achieved = ffn_flops / (ffn_ms * 1e-3) / 1e12 if ffn_ms > 0 else 0.0
+    if mode == J.JANUS_FFN_FP32_SIMT:
+        peak = SM_COUNT * FP32_LANES_PER_SM * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+        roof = {"bound": "alu", "peak_source": "148 SMs x 128 FP32 lanes x 2 FLOP x max SM clock"}
+    else:
+        peak = peaks["bf16_tflops"] * (1.125 / 2.25) / 3.0
+        roof = {"bound": "tensor", "peak_source": f"{peak_src} burst bf16 x (TF32/BF16 nominal 1.125/2.25) / 3 products"}
+    roof.update({"kernel": "grouped expert-MLP GEMM (rank 0's experts; ffn phases include the FP16 unpack)",
+                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                 "algorithmic_flops_per_launch": ffn_flops / 4, "launches_per_step": 4})
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_max / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {**describe(cfg), "ffn_mode": args.mode, "parallelism": f"ep{world}",
+                   "experts_per_rank": El, "received_rows_rank0": r_recv,
+                   "l2": "no flush: per-step working set far above the 126 MB L2"},
+        "roofline": roof,
+        "breakdown_ms": ph_ms,
+        "gpu_launches": 18 * args.steps,
+        "clocks": clocks,
+    }
+    layer.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def _time_ms(fn, reps=5):
     fn()
     torch.cuda.synchronize()
@@ -633,6 +717,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.ep:
+            run_ep(args, world, rank, local)
         else:
             run_janus(args, world, rank, local)
     finally:

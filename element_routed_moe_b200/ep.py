@@ -32,8 +32,10 @@ class ExpertParallelLayer:
     def __init__(self, n_atoms_max, d, h, n_types, n_experts, top_k, w1_local, w2_local, *,
                  mode=J.JANUS_FFN_3XTF32, group=None, device=None):
         self.group = group
-        self.world = dist.get_world_size(group)
-        self.rank = dist.get_rank(group)
+        self.dist = dist.is_available() and dist.is_initialized()
+        # without a process group the layer is a single rank owning every expert
+        self.world = dist.get_world_size(group) if self.dist else 1
+        self.rank = dist.get_rank(group) if self.dist else 0
         if self.world > J.JANUS_EP_MAX_RANKS:
             raise ValueError(f"at most {J.JANUS_EP_MAX_RANKS} ranks (one node)")
         if n_experts % self.world:
@@ -44,7 +46,7 @@ class ExpertParallelLayer:
         if w1_local.shape != (self.El, d, h) or w2_local.shape != (self.El, h, d):
             raise ValueError("w1_local / w2_local must hold this rank's E/P experts")
         self.w1, self.w2, self.mode = w1_local, w2_local, mode
-        self.nccl = dist.get_backend(group) == "nccl"
+        self.nccl = self.dist and dist.get_backend(group) == "nccl"
         # worst case: every routed row of every rank lands on this rank
         self.n_atoms_max = int(n_atoms_max)
         cap = max(self.world * self.n_atoms_max * top_k, 1)
@@ -69,7 +71,9 @@ class ExpertParallelLayer:
     # -- plumbing ------------------------------------------------------------
     def _exchange(self, t):
         """Device pointers of every rank's copy of buffer t (index = rank)."""
-        blob = J.janus_ipc_get_handle(t) if self.world > 1 else b""
+        if self.world == 1:
+            return [t.data_ptr()]
+        blob = J.janus_ipc_get_handle(t)
         blobs = [None] * self.world
         dist.all_gather_object(blobs, blob, group=self.group)
         ptrs = []
@@ -85,6 +89,8 @@ class ExpertParallelLayer:
     def barrier(self):
         """Every rank's work queued so far (its peer stores included) is done
         before any rank's next step runs."""
+        if self.world == 1:
+            return
         if self.nccl:
             dist.all_reduce(self._token, group=self.group)
         else:
@@ -92,7 +98,9 @@ class ExpertParallelLayer:
             dist.barrier(group=self.group)
 
     def _gather_counts(self, counts):
-        if self.nccl:
+        if self.world == 1:
+            self.counts_all[0].copy_(counts)
+        elif self.nccl:
             dist.all_gather_into_tensor(self.counts_all, counts, group=self.group)
         else:
             parts = [torch.empty_like(counts.cpu()) for _ in range(self.world)]
@@ -101,40 +109,74 @@ class ExpertParallelLayer:
 
     def close(self):
         torch.cuda.synchronize(self.dev)
-        dist.barrier(group=self.group)          # no rank still writes into a mapping
+        if self.world > 1:
+            dist.barrier(group=self.group)      # no rank still writes into a mapping
         for p, off in self._opened:
             J.janus_ipc_close_handle(p, off)
         self._opened = []
 
     # -- the layer -------------------------------------------------------------
-    def forward(self, x, types, gate):
-        """y [N,d] for this rank's atoms (FP16-packed dispatch)."""
+    PHASES_FWD = ("route", "layout", "send", "ffn_fwd", "return", "combine")
+    PHASES_VJP = ("send_vjp", "ffn_vjp", "return_vjp", "combine_vjp")
+
+    @staticmethod
+    def _mark(events, name, i):
+        if events is not None:
+            events[name][i].record()
+
+    def forward(self, x, types, gate, events=None):
+        """y [N,d] for this rank's atoms (FP16-packed dispatch).  events: an
+        optional dict phase -> (start, end) CUDA events to record."""
         if x.shape[0] > self.n_atoms_max:
             raise ValueError("more atoms than the buffers were sized for")
+        m = self._mark
         self.x_shape = x.shape
+        m(events, "route", 0)
         self.route = J.janus_route(types, gate, self.K)
+        m(events, "route", 1)
+        m(events, "layout", 0)
         self._gather_counts(self.route["counts"])
         self.layout = J.janus_ep_layout(self.counts_all, self.E)
+        m(events, "layout", 1)
+        m(events, "send", 0)
         J.janus_ep_dispatch_quant(x, types, self.T, self.route, self.layout, self.rank,
                                   self.peer_payload, self.peer_scale)
         self.barrier()
+        m(events, "send", 1)
         recv_off = self.layout[2][self.rank]
+        m(events, "ffn_fwd", 0)
         J.janus_ep_dequant_rows(self.payload, self.row_scale, self.layout, self.rank, out=self.xd)
         J.janus_expert_ffn_fwd(self.xd, recv_off, self.w1, self.w2, mode=self.mode, out=self.yd, act=self.act)
+        m(events, "ffn_fwd", 1)
+        m(events, "return", 0)
         J.janus_ep_return(self.yd, self.counts_all, self.layout, self.rank, self.peer_ret)
         self.barrier()
+        m(events, "return", 1)
         R = x.shape[0] * self.K
-        return J.janus_combine(self.ret[:R], self.route["slot_of"], self.K, self.route["topk_weight"])
+        m(events, "combine", 0)
+        y = J.janus_combine(self.ret[:R], self.route["slot_of"], self.K, self.route["topk_weight"])
+        m(events, "combine", 1)
+        return y
 
-    def vjp(self, g):
+    def vjp(self, g, events=None):
         """dx [N,d] for the upstream gradient g [N,d] of forward's output."""
+        m = self._mark
         r = self.route
+        m(events, "send_vjp", 0)
         J.janus_ep_dispatch(g, r, self.layout, self.rank, self.peer_rows, weighted=True)
         self.barrier()
+        m(events, "send_vjp", 1)
         recv_off = self.layout[2][self.rank]
+        m(events, "ffn_vjp", 0)
         J.janus_expert_ffn_vjp(self.xd, self.recv_rows, recv_off, self.w1, self.w2, act=self.act,
                                mode=self.mode, out=self.yd)
+        m(events, "ffn_vjp", 1)
+        m(events, "return_vjp", 0)
         J.janus_ep_return(self.yd, self.counts_all, self.layout, self.rank, self.peer_ret)
         self.barrier()
+        m(events, "return_vjp", 1)
         R = self.x_shape[0] * self.K
-        return J.janus_combine(self.ret[:R], r["slot_of"], self.K)
+        m(events, "combine_vjp", 0)
+        dx = J.janus_combine(self.ret[:R], r["slot_of"], self.K)
+        m(events, "combine_vjp", 1)
+        return dx

@@ -63,3 +63,41 @@ def test_reference_arm_two_ranks_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def _ep_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from element_routed_moe_b200.ep import ExpertParallelLayer
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    out = []
+    w1, w2 = torch.zeros((4, 8, 12)), torch.zeros((4, 12, 8))
+    for E, a, b in ((9, w1, w2), (8, w1[:3], w2[:3]), (8, w2, w1)):
+        try:
+            ExpertParallelLayer(16, 8, 12, 5, E, 2, a, b)
+            out.append("accepted")
+        except ValueError as e:
+            out.append(str(e))
+    q.put((rank, out))
+    dist.destroy_process_group()
+
+
+def test_ep_layer_validates_the_expert_split_on_every_rank():
+    # two gloo ranks: 9 experts cannot be split, each rank must pass its E/P = 4
+    # experts in the [E/P, d, h] / [E/P, h, d] layout; nothing reaches CUDA
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ep_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = sorted(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, msgs in got:
+        assert "multiple of the number of ranks" in msgs[0]
+        assert "E/P experts" in msgs[1] and "E/P experts" in msgs[2]
