@@ -215,18 +215,14 @@ def measured_peaks() -> tuple[dict, str]:
 # the layer pass through the C ABI (device-resident inputs)
 # --------------------------------------------------------------------------
 class Layer:
-    """Preallocated buffers and the ordered ABI calls of one layer pass."""
-
-    OPS_FWD = ("route", "dispatch", "ffn_fwd", "combine")
-    OPS_VJP = ("dispatch_w", "ffn_vjp", "combine_vjp")
+    """Synthetic inputs of one workload and the library's MoELayer over them."""
 
     def __init__(self, cfg, mode: int, seed: int, dev):
         from element_routed_moe_b200 import janus as J
+        from element_routed_moe_b200.layer import MoELayer
         self.J = J
         self.cfg = cfg
         self.mode = mode
-        N, T, E, K, d, h = cfg.n_atoms, cfg.n_types, cfg.n_experts, cfg.top_k, cfg.d, cfg.h
-        R = N * K
         self.slice = cfg.name == "slice"
         inp = synth.layer_inputs(cfg, seed=seed, device=dev, with_edges=self.slice)
         self.inp = inp
@@ -237,90 +233,22 @@ class Layer:
         if self.slice:
             self.msg = inp["msg"]
             self.row_ptr = torch.as_tensor(inp["row_ptr"], device=dev)
-        f32 = dict(dtype=torch.float32, device=dev)
-        i32 = dict(dtype=torch.int32, device=dev)
-        self.route_out = dict(topk_expert=torch.empty((N, K), **i32),
-                              topk_weight=torch.empty((N, K), **f32),
-                              counts=torch.empty((E,), **i32), offsets=torch.empty((E + 1,), **i32),
-                              perm=torch.empty((R,), **i32), slot_of=torch.empty((R,), **i32))
-        self.route_ws = torch.empty(J.janus_route_workspace_size(N, T, E, K), dtype=torch.uint8, device=dev)
-        self.xd = torch.empty((R, d), **f32)
-        self.yd = torch.empty((R, d), **f32)
-        self.act = torch.empty((R, h), **f32)
-        self.y = torch.empty((N, d), **f32)
-        self.gd = torch.empty((R, d), **f32)
-        self.dxd = torch.empty((R, d), **f32)
-        self.dx = torch.empty((N, d), **f32)
-        nb = max(J.janus_expert_ffn_workspace_size(R, d, h, E, False, True, mode),
-                 J.janus_expert_ffn_workspace_size(R, d, h, E, True, True, mode))
-        self.ffn_ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        self.core = MoELayer(cfg.n_atoms, cfg.top_k, self.gate, self.w1, self.w2, mode=mode, packed=self.slice,
+                             row_ptr=self.row_ptr if self.slice else None)
+        c = self.core
+        self.route_out, self.route_ws = c.route_out, c.route_ws
+        self.xd, self.gd, self.act, self.y, self.dx = c.xd, c.gd, c.act, c.y, c.dx
         if self.slice:
-            self.xagg = torch.empty((N, d), **f32)
-            self.payload = torch.empty((R, d), dtype=torch.float16, device=dev)
-            self.scale = torch.empty((T,), **f32)
-            self.quant_ws = torch.empty(J.janus_quant_by_type_workspace_size(T), dtype=torch.uint8,
-                                        device=dev)
-        if self.slice:
-            self.ops = ("edge_aggregate", "route", "quant", "dequant", "ffn_fwd", "combine") + self.OPS_VJP
-        else:
-            self.ops = self.OPS_FWD + self.OPS_VJP
-        # our kernels per step (see each call's launches in csrc/)
-        per = {"edge_aggregate": 1, "quant": 2, "dequant": 1, "route": 4, "dispatch": 1,
-               "ffn_fwd": 2, "combine": 1, "dispatch_w": 1, "ffn_vjp": 2, "combine_vjp": 1}
-        self.launches_per_step = sum(per[o] for o in self.ops)
+            self.xagg = c.xagg
+        self.ops = c.ops
+        self.launches_per_step = c.launches_per_call
 
     def step(self, x=None, g=None, types=None, events=None):
         """One layer pass.  events: dict op -> (start, end) CUDA events, or None."""
-        J = self.J
-        cfg = self.cfg
-        T, K = cfg.n_types, cfg.top_k
-        x = self.x if x is None else x
+        x = (self.msg if self.slice else self.x) if x is None else x
         g = self.g if g is None else g
         types = self.types if types is None else types
-        r = self.route_out
-
-        def mark(op, i):
-            if events is not None:
-                events[op][i].record()
-
-        if self.slice:
-            mark("edge_aggregate", 0)
-            J.janus_edge_aggregate(self.msg, self.row_ptr, out=self.xagg)
-            mark("edge_aggregate", 1)
-            x = self.xagg
-        mark("route", 0)
-        J.janus_route(types, self.gate, K, out=r, workspace=self.route_ws)
-        mark("route", 1)
-        if self.slice:
-            mark("quant", 0)
-            J.janus_quant_by_type(x, types, T, r["slot_of"], K, payload=self.payload,
-                                  scale=self.scale, workspace=self.quant_ws)
-            mark("quant", 1)
-            mark("dequant", 0)
-            J.janus_dequant_by_type(self.payload, types, T, r["perm"], K, self.scale, out=self.xd)
-            mark("dequant", 1)
-        else:
-            mark("dispatch", 0)
-            J.janus_dispatch(x, r["slot_of"], K, out=self.xd)
-            mark("dispatch", 1)
-        mark("ffn_fwd", 0)
-        J.janus_expert_ffn_fwd(self.xd, r["offsets"], self.w1, self.w2, mode=self.mode, out=self.yd,
-                               act=self.act, workspace=self.ffn_ws)
-        mark("ffn_fwd", 1)
-        mark("combine", 0)
-        J.janus_combine(self.yd, r["slot_of"], K, r["topk_weight"], out=self.y)
-        mark("combine", 1)
-        mark("dispatch_w", 0)
-        J.janus_dispatch(g, r["slot_of"], K, r["topk_weight"], out=self.gd)
-        mark("dispatch_w", 1)
-        mark("ffn_vjp", 0)
-        J.janus_expert_ffn_vjp(self.xd, self.gd, r["offsets"], self.w1, self.w2, act=self.act,
-                               mode=self.mode, out=self.dxd, workspace=self.ffn_ws)
-        mark("ffn_vjp", 1)
-        mark("combine_vjp", 0)
-        J.janus_combine(self.dxd, r["slot_of"], K, out=self.dx)
-        mark("combine_vjp", 1)
-        return self.y, self.dx
+        return self.core.forward_vjp(x, g, types, events=events)
 
     # algorithmic bytes (memory-bound ops) and FLOPs (expert MLP) per call
     def work(self):
@@ -677,39 +605,34 @@ def run_extras(layer, peaks):
 
 
 def run_e2e(layer, args):
-    """Same metric through the public API with the step's inputs in pinned
-    host memory: H2D of (x, dY, types) and D2H of (y, dX) inside the timing."""
-    dev = layer.x.device
+    """Same metric through the library's MoELayer.run_host with the step's
+    inputs in pinned host memory: every step uploads (x, dY, types) and
+    downloads (y, dX) inside the timed region.  The copies run on their own
+    streams: dY's upload overlaps the forward, y's download the VJP, and the
+    next step's upload this step's compute."""
+    core = layer.core
     x_h = layer.x.cpu().pin_memory()
     g_h = layer.g.cpu().pin_memory()
     t_h = layer.types.cpu().pin_memory()
     y_h = torch.empty(layer.y.shape, dtype=torch.float32).pin_memory()
     dx_h = torch.empty(layer.dx.shape, dtype=torch.float32).pin_memory()
-    x_d, g_d, t_d = torch.empty_like(layer.x), torch.empty_like(layer.g), torch.empty_like(layer.types)
-
-    def step():
-        x_d.copy_(x_h, non_blocking=True)
-        g_d.copy_(g_h, non_blocking=True)
-        t_d.copy_(t_h, non_blocking=True)
-        y, dx = layer.step(x_d, g_d, t_d)
-        y_h.copy_(y, non_blocking=True)
-        dx_h.copy_(dx, non_blocking=True)
-
     for _ in range(args.warmup):
-        step()
+        core.run_host(x_h, g_h, t_h, y_h, dx_h)
+    core.host_sync()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(args.steps):
-        step()
+        core.run_host(x_h, g_h, t_h, y_h, dx_h)
+    core.host_sync()
     b.record()
     torch.cuda.synchronize()
     t = a.elapsed_time(b) / 1e3
     h2d = x_h.numel() * 4 + g_h.numel() * 4 + t_h.numel() * 4
     d2h = y_h.numel() * 4 + dx_h.numel() * 4
     return {"value": layer.cfg.n_rows * args.steps / t, "unit": UNIT,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "overlap": "uploads and downloads on their own streams, double-buffered on the device"}
 
 def main():
     args = parse()

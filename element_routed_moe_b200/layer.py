@@ -1,0 +1,199 @@
+"""One element-routed MoE layer on one GPU: forward and input VJP through the
+C ABI, with preallocated buffers.
+
+Sources: paper review "Breaking the Training Barrier of Billion-Parameter
+Universal Machine Learning Interatomic Potentials" sections 3.1-3.5 (static
+per-element routing, Linear-SiLU-Linear experts, forces by autodiff, FP16
+packing of the dispatch, edge aggregation in front of the MoE block) and
+"MatRIS-MoE与Janus框架" section 3.2 (gate-weighted sum of the experts).
+
+One pass, all on the current stream:
+    [edge_aggregate]  X = segment sums of the edge messages (row_ptr given)
+    route             per-type top-K, counts, offsets, permutation
+    dispatch          Xd = X rows in expert order   (or FP16 pack + unpack)
+    ffn_fwd           Yd = silu(Xd W1[e]) W2[e]      (a saved)
+    combine           Y  = sum_k w * Yd
+    dispatch_w        Gd = w * G rows in expert order
+    ffn_vjp           dXd = ((Gd W2^T) * silu'(a)) W1^T
+    combine_vjp       dX = sum_k dXd
+
+`run_host` runs the pass from and to pinned host memory with the copies on
+their own streams: the upload of G overlaps the forward, the download of Y
+overlaps the VJP, and the next call's upload overlaps this call's compute
+(inputs and outputs are double-buffered on the device).
+"""
+import torch
+
+from . import janus as J
+
+
+class MoELayer:
+    OPS_FWD = ("route", "dispatch", "ffn_fwd", "combine")
+    OPS_VJP = ("dispatch_w", "ffn_vjp", "combine_vjp")
+    # this library's kernels per call (see each entry point's launches)
+    LAUNCHES = {"edge_aggregate": 1, "quant": 2, "dequant": 1, "route": 4, "dispatch": 1,
+                "ffn_fwd": 2, "combine": 1, "dispatch_w": 1, "ffn_vjp": 2, "combine_vjp": 1}
+
+    def __init__(self, n_atoms, top_k, gate, w1, w2, *, mode=J.JANUS_FFN_3XTF32, packed=False,
+                 row_ptr=None):
+        """gate [T,E], w1 [E,d,h], w2 [E,h,d] on the layer's device.  packed:
+        FP16 per-type packing of the dispatch.  row_ptr [N+1] (int64): the
+        input is edge messages [Ed,d], aggregated per receiver first."""
+        dev = w1.device
+        self.dev = dev
+        self.N, self.K = int(n_atoms), int(top_k)
+        self.T, self.E = gate.shape
+        _, self.d, self.h = w1.shape
+        self.gate, self.w1, self.w2, self.mode = gate, w1, w2, mode
+        self.packed, self.row_ptr = packed, row_ptr
+        N, K, T, E, d, h = self.N, self.K, self.T, self.E, self.d, self.h
+        R = N * K
+        f32 = dict(dtype=torch.float32, device=dev)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.route_out = dict(topk_expert=torch.empty((N, K), **i32),
+                              topk_weight=torch.empty((N, K), **f32),
+                              counts=torch.empty((E,), **i32), offsets=torch.empty((E + 1,), **i32),
+                              perm=torch.empty((R,), **i32), slot_of=torch.empty((R,), **i32))
+        self.route_ws = torch.empty(J.janus_route_workspace_size(N, T, E, K), dtype=torch.uint8, device=dev)
+        self.xd = torch.empty((R, d), **f32)
+        self.yd = torch.empty((R, d), **f32)
+        self.act = torch.empty((R, h), **f32)
+        self.gd = torch.empty((R, d), **f32)
+        self.dxd = torch.empty((R, d), **f32)
+        self.y = torch.empty((N, d), **f32)
+        self.dx = torch.empty((N, d), **f32)
+        nb = max(J.janus_expert_ffn_workspace_size(R, d, h, E, False, True, mode),
+                 J.janus_expert_ffn_workspace_size(R, d, h, E, True, True, mode))
+        self.ffn_ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        if row_ptr is not None:
+            self.xagg = torch.empty((N, d), **f32)
+        if packed:
+            self.payload = torch.empty((R, d), dtype=torch.float16, device=dev)
+            self.scale = torch.empty((T,), **f32)
+            self.quant_ws = torch.empty(J.janus_quant_by_type_workspace_size(T), dtype=torch.uint8, device=dev)
+        front = ("edge_aggregate",) if row_ptr is not None else ()
+        mid = ("route", "quant", "dequant") if packed else ("route", "dispatch")
+        self.ops = front + mid + ("ffn_fwd", "combine") + self.OPS_VJP
+        self.launches_per_call = sum(self.LAUNCHES[o] for o in self.ops)
+        self._host = None
+
+    # -- device-resident pass ----------------------------------------------------
+    def forward_vjp(self, x, g, types, events=None, y=None, dx=None, after_forward=None):
+        """One pass on device tensors; returns (y, dx) (the layer's own buffers
+        unless y / dx are given).  events: dict op -> (start, end) CUDA events;
+        after_forward: called once y is enqueued, before the VJP."""
+        K, T, r = self.K, self.T, self.route_out
+        y = self.y if y is None else y
+        dx = self.dx if dx is None else dx
+
+        def mark(op, i):
+            if events is not None:
+                events[op][i].record()
+
+        if self.row_ptr is not None:
+            mark("edge_aggregate", 0)
+            J.janus_edge_aggregate(x, self.row_ptr, out=self.xagg)
+            mark("edge_aggregate", 1)
+            x = self.xagg
+        mark("route", 0)
+        J.janus_route(types, self.gate, K, out=r, workspace=self.route_ws)
+        mark("route", 1)
+        if self.packed:
+            mark("quant", 0)
+            J.janus_quant_by_type(x, types, T, r["slot_of"], K, payload=self.payload, scale=self.scale,
+                                  workspace=self.quant_ws)
+            mark("quant", 1)
+            mark("dequant", 0)
+            J.janus_dequant_by_type(self.payload, types, T, r["perm"], K, self.scale, out=self.xd)
+            mark("dequant", 1)
+        else:
+            mark("dispatch", 0)
+            J.janus_dispatch(x, r["slot_of"], K, out=self.xd)
+            mark("dispatch", 1)
+        mark("ffn_fwd", 0)
+        J.janus_expert_ffn_fwd(self.xd, r["offsets"], self.w1, self.w2, mode=self.mode, out=self.yd,
+                               act=self.act, workspace=self.ffn_ws)
+        mark("ffn_fwd", 1)
+        mark("combine", 0)
+        J.janus_combine(self.yd, r["slot_of"], K, r["topk_weight"], out=y)
+        mark("combine", 1)
+        if after_forward is not None:
+            after_forward()
+        mark("dispatch_w", 0)
+        J.janus_dispatch(g, r["slot_of"], K, r["topk_weight"], out=self.gd)
+        mark("dispatch_w", 1)
+        mark("ffn_vjp", 0)
+        J.janus_expert_ffn_vjp(self.xd, self.gd, r["offsets"], self.w1, self.w2, act=self.act,
+                               mode=self.mode, out=self.dxd, workspace=self.ffn_ws)
+        mark("ffn_vjp", 1)
+        mark("combine_vjp", 0)
+        J.janus_combine(self.dxd, r["slot_of"], K, out=dx)
+        mark("combine_vjp", 1)
+        return y, dx
+
+    # -- pass from and to pinned host memory, copies overlapped -------------------
+    def _host_state(self, x_shape):
+        dev = self.dev
+        f32 = dict(dtype=torch.float32, device=dev)
+        st = {
+            "copy_in": torch.cuda.Stream(dev), "copy_out": torch.cuda.Stream(dev), "k": 0,
+            "x": [torch.empty(x_shape, **f32) for _ in range(2)],
+            "g": [torch.empty((self.N, self.d), **f32) for _ in range(2)],
+            "types": [torch.empty((self.N,), dtype=torch.int32, device=dev) for _ in range(2)],
+            "y": [torch.empty((self.N, self.d), **f32) for _ in range(2)],
+            "dx": [torch.empty((self.N, self.d), **f32) for _ in range(2)],
+        }
+        for name in ("x_in", "g_in", "in_free", "y_done", "dx_done", "y_out", "dx_out"):
+            st[name] = [torch.cuda.Event() for _ in range(2)]
+        for b in range(2):      # nothing is in flight yet
+            for name in ("in_free", "y_out", "dx_out"):
+                st[name][b].record(torch.cuda.current_stream(dev))
+        return st
+
+    def run_host(self, x_h, g_h, types_h, y_h, dx_h):
+        """Enqueue one pass from pinned host inputs (x [N,d] or the edge
+        messages, g [N,d], types [N]) into pinned host outputs y_h, dx_h.
+        Returns at once; the outputs are complete after `host_sync()`."""
+        if self._host is None:
+            self._host = self._host_state(tuple(x_h.shape))
+        st = self._host
+        b = st["k"] % 2
+        st["k"] += 1
+        s = torch.cuda.current_stream(self.dev)
+        cin, cout = st["copy_in"], st["copy_out"]
+        # inputs: buffer set b is free once the pass that last used it is done
+        cin.wait_event(st["in_free"][b])
+        with torch.cuda.stream(cin):
+            st["types"][b].copy_(types_h, non_blocking=True)
+            st["x"][b].copy_(x_h, non_blocking=True)
+            st["x_in"][b].record(cin)
+            st["g"][b].copy_(g_h, non_blocking=True)
+            st["g_in"][b].record(cin)
+        s.wait_event(st["x_in"][b])
+        s.wait_event(st["y_out"][b])           # y buffer b downloaded by its previous pass
+        s.wait_event(st["dx_out"][b])
+
+        def after_fwd():                        # y is final: download it during the VJP
+            st["y_done"][b].record(s)
+            cout.wait_event(st["y_done"][b])
+            with torch.cuda.stream(cout):
+                y_h.copy_(st["y"][b], non_blocking=True)
+                st["y_out"][b].record(cout)
+            s.wait_event(st["g_in"][b])
+
+        self.forward_vjp(st["x"][b], st["g"][b], st["types"][b], y=st["y"][b], dx=st["dx"][b],
+                         after_forward=after_fwd)
+        st["in_free"][b].record(s)
+        st["dx_done"][b].record(s)
+        cout.wait_event(st["dx_done"][b])
+        with torch.cuda.stream(cout):
+            dx_h.copy_(st["dx"][b], non_blocking=True)
+            st["dx_out"][b].record(cout)
+
+    def host_sync(self):
+        """Make the current stream wait for every enqueued host pass's copies."""
+        if self._host is not None:
+            s = torch.cuda.current_stream(self.dev)
+            for b in range(2):
+                s.wait_event(self._host["y_out"][b])
+                s.wait_event(self._host["dx_out"][b])
