@@ -13,35 +13,41 @@
 // accumulated from zero in TMEM and then added, with round-to-nearest FP32
 // adds, into running sums held in the epilogue warps' registers.
 //
-//   C[p, :] = epilogue( A[p, :] * B_e )  for the rows p of expert e's segment
-//
-// Structure: one persistent CTA per SM, clusters of two CTAs that share one
-// M=256 x N=256 output tile through tcgen05 cta_group::2 MMAs (each CTA holds
-// its 128 rows of A, 128 of the 256 B columns and its 128 accumulator rows,
-// so shared-memory traffic per CTA is a third lower than with 1-CTA MMAs).
-// 16 warps = 4 warpgroups per CTA:
-//   warp 0       TMA producer: this CTA's A tile 128x16 and B half 128x16
-//                (FP32, 64-byte swizzle; 128-byte swizzle with 32-byte atoms
-//                for an MN-major B) per k-block into a 6-stage ring (32 KB per
-//                stage: raw + lo);
+// Three operand layouts share the kernel:
+//   x W   (forward)  and  x W^T (input VJP) run swapped, C^T = W^T X^T: the
+//         MMA's A is the expert's weights (128 output features per CTA, so
+//         M = 256 per pair is always full) and its B is the tile's dispatch
+//         rows (N = the valid rows rounded up to 32, half of them per CTA), so
+//         a Zipf-small expert pads at most 31 rows;
+//   X^T Y (weight gradients) runs direct, both operands MN-major, K = the
+//         expert's rows.
+// Structure: one persistent CTA per SM, clusters of two CTAs sharing each
+// output tile through tcgen05 cta_group::2 MMAs (each CTA holds its 128 rows
+// of A, its half of B and its 128 accumulator lanes, so shared-memory traffic
+// per CTA is a third lower than with 1-CTA MMAs).  16 warps:
+//   warp 0       TMA producer: this CTA's A and B tiles per 16-wide k-block
+//                into a 6-stage ring (32 KB per stage: raw + lo; 64-byte
+//                swizzle for K-major, 128-byte swizzle with 32-byte atoms for
+//                MN-major operands);
 //   warp 1       TMEM allocator (paired) and, in the leader CTA, the MMA
 //                issuer: 3 products x 2 k-steps of tcgen05.mma.cta_group::2
-//                .kind::tf32 (M=256, N=256, K=8) per k-block into one of two
-//                TMEM chunk buffers (2 x 256 columns), commits signalling
-//                both CTAs; peers' splitters and epilogues arrive on the
-//                leader's barriers;
+//                .kind::tf32 per k-block into one of two 256-column TMEM chunk
+//                buffers, commits signalling both CTAs; the peer's splitters
+//                and epilogues arrive on the leader's barriers;
 //   warps 2,3,12..15  splitters, each owning every sixth k-block: write the
 //                landed tile's residual lo = x - hi into a twin buffer (same
 //                swizzled offsets; the landed FP32 tile is read by the MMA as hi);
-//   warps 4..11  epilogue (warpgroups 1 and 2, one 128-column half each):
-//                tcgen05.ld of each chunk (one TMEM lane quarter = 32 rows per
-//                warp), FP32 running sums in registers (setmaxnreg: 184 per
-//                thread here, 72 elsewhere), then fused SiLU / SiLU' / store.
-// Tiles come from a device-side list built from `offsets` (expert-major, then
-// 128-row block, then 256-column block), so the host never reads the routing.
-// Every mbarrier wait is bounded: on timeout the CTA records an error in the
-// workspace header, every role leaves its loop, issued MMAs and loads are
-// drained (bounded) and TMEM is freed.
+//   warps 4..11  epilogue (two warpgroups, one half of the tile each):
+//                tcgen05.ld of each chunk, FP32 running sums in registers
+//                (setmaxnreg: 184 per thread here, 72 elsewhere), then the
+//                fused epilogue: SiLU (a and silu(a)), SiLU' (pre-activation
+//                reads pipelined and prefetched to L2), the second-order
+//                silu'/silu'' terms, a plain store, or an accumulating store.
+// Tiles come from per-expert block counts built on the device from `offsets`
+// (expert, then 256-row block, then 256-feature block), so the host never
+// reads the routing.  Every mbarrier wait is bounded: on timeout the CTA
+// records an error in the workspace header, every role leaves its loop,
+// issued MMAs and loads are drained (bounded) and TMEM is freed.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
