@@ -66,3 +66,30 @@ def test_device_pass_matches_oracle(packed):
     gd = oracle.dispatch(host(g), r["perm"], K, r["topk_weight"])
     dxd = oracle.expert_ffn_vjp(xd, gd, r["offsets"], host(w1), host(w2))
     assert rel_fro(host(dx), oracle.combine(dxd, r["slot_of"], K)) <= TOL_FP32
+
+
+def test_edge_fed_packed_layer_matches_oracle():
+    # the interaction-block slice form: edge messages aggregated per receiver,
+    # FP16 per-type packing of the dispatch, then the layer
+    from element_routed_moe_b200.synth import edges_random
+    N, T, E, K, d, h = 700, 11, 12, 3, 96, 64
+    rp, send, recv = edges_random(N, 9, seed=11)
+    msg = synth.normal((int(rp[-1]), d), 12, DEV)
+    gate_np = synth.gate_table(T, E, 13)
+    w1, w2 = synth.expert_weights(E, d, h, 14, DEV)
+    types_np = synth.types_zipf(N, T, seed=15)
+    g = synth.normal((N, d), 16, DEV)
+    layer = MoELayer(N, K, to_dev(gate_np), w1, w2, mode=J.JANUS_FFN_3XTF32, packed=True,
+                     row_ptr=torch.as_tensor(rp, device=DEV))
+    assert layer.ops[0] == "edge_aggregate" and "quant" in layer.ops
+    y, dx = layer.forward_vjp(msg, g, to_dev(types_np))
+    torch.cuda.synchronize()
+    x = oracle.edge_aggregate(host(msg), rp)
+    r = oracle.route(types_np, gate_np, K)
+    q, sc = oracle.quant_by_type(x, types_np, T, r["perm"], K)
+    xd = oracle.dequant_by_type(q, types_np, r["perm"], K, sc)
+    yd = oracle.expert_ffn_fwd(xd, r["offsets"], host(w1), host(w2))
+    assert rel_fro(host(y), oracle.combine(yd, r["slot_of"], K, r["topk_weight"])) <= TOL_FP32
+    gd = oracle.dispatch(host(g), r["perm"], K, r["topk_weight"])
+    dxd = oracle.expert_ffn_vjp(xd, gd, r["offsets"], host(w1), host(w2))
+    assert rel_fro(host(dx), oracle.combine(dxd, r["slot_of"], K)) <= TOL_FP32
