@@ -67,6 +67,13 @@ constexpr int BNH = BN / 2;               // B columns held by one CTA
 constexpr int kStages = 6;
 constexpr int kThreads = 512;
 constexpr int kNumSplitWarps = 6;
+// Splitter warp i splits every k-block with (k-block index) % kNumSplitWarps
+// == i, i.e. always the same stages.  That is what makes its parity wait on a
+// stage's `full` barrier safe: a parity wait cannot tell the phase it wants
+// from the one two phases later, so each stage's consecutive uses must be
+// waited for by one warp, in order.  (A 7-stage ring with 6 splitters, where
+// uses rotate between warps, split tiles before they had landed.)
+static_assert(kStages % kNumSplitWarps == 0, "every stage is split by one fixed warp");
 constexpr int kNumEpiWarps = 8;
 constexpr int kEpiCols = BN / 2;         // columns per epilogue thread
 constexpr int kChunkKb = 128 / BK;       // k-blocks accumulated per TMEM chunk (K = 128)
