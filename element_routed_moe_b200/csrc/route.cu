@@ -377,3 +377,43 @@ extern "C" janus_status janus_route_layers(const int32_t* types, int64_t n_atoms
   return route_impl(types, n_atoms, gates, n_layers, n_types, n_experts, top_k, topk_expert, topk_weight,
                     counts, offsets, perm, slot_of, workspace, workspace_bytes, (cudaStream_t)stream);
 }
+
+// ---------------------------------------------------------------------------
+// Active-expert lists: per layer, the ids of the experts with routed rows, in
+// ascending order (a stable compaction of counts > 0).  One CTA per layer,
+// one thread per expert; the rank of each active expert is its warp's ballot
+// prefix plus the active experts of the warps before it.
+// ---------------------------------------------------------------------------
+namespace janus {
+namespace {
+__global__ void __launch_bounds__(kMaxExperts) active_experts_kernel(const int32_t* __restrict__ counts, int E,
+                                                                    int32_t* __restrict__ active,
+                                                                    int32_t* __restrict__ n_active) {
+  __shared__ int warp_sum[kMaxExperts / 32];
+  const int l = blockIdx.x, e = threadIdx.x, lane = e % 32, w = e / 32;
+  const bool on = e < E && counts[(int64_t)l * E + e] > 0;
+  const unsigned bal = __ballot_sync(0xffffffffu, on);
+  if (lane == 0) warp_sum[w] = __popc(bal);
+  __syncthreads();
+  int base = 0;
+  for (int i = 0; i < w; ++i) base += warp_sum[i];
+  if (on) active[(int64_t)l * E + base + __popc(bal & ((1u << lane) - 1u))] = e;
+  if (e == 0) {
+    int tot = 0;
+    for (int i = 0; i < kMaxExperts / 32; ++i) tot += warp_sum[i];
+    n_active[l] = tot;
+  }
+}
+}  // namespace
+}  // namespace janus
+
+extern "C" janus_status janus_active_experts(const int32_t* counts, int32_t n_layers, int32_t n_experts,
+                                             int32_t* active, int32_t* n_active, janus_stream_t stream) {
+  using namespace janus;
+  JANUS_CHECK_ARG(n_layers >= 0 && n_experts >= 1 && n_experts <= kMaxExperts);
+  if (n_layers == 0) return JANUS_OK;
+  JANUS_CHECK_ARG(counts && active && n_active);
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  active_experts_kernel<<<n_layers, kMaxExperts, 0, (cudaStream_t)stream>>>(counts, n_experts, active, n_active);
+  return launch_status();
+}

@@ -30,7 +30,7 @@ JANUS_FFN_3XTF32 = 1
 SYMBOLS = (
     "janus_status_string", "janus_version", "janus_check",
     "janus_route_workspace_size", "janus_route",
-    "janus_route_layers_workspace_size", "janus_route_layers",
+    "janus_route_layers_workspace_size", "janus_route_layers", "janus_active_experts",
     "janus_dispatch",
     "janus_quant_by_type_workspace_size", "janus_quant_by_type", "janus_quant_by_type_noalloc",
     "janus_dequant_by_type",
@@ -87,6 +87,7 @@ def _declare(L):
         "janus_route_layers_workspace_size": (st, [i64, i32, i32, i32, i32, psz]),
         "janus_route_layers": (st, [vp, i64, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz,
                                     vp]),
+        "janus_active_experts": (st, [vp, i32, i32, vp, vp, vp]),
         "janus_dispatch": (st, [vp, i64, i32, i32, vp, vp, vp, vp]),
         "janus_quant_by_type_workspace_size": (st, [i32, psz]),
         "janus_quant_by_type": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp, sz, vp]),
@@ -242,6 +243,21 @@ def janus_check(workspace, stream=None):
 # --------------------------------------------------------------------------
 # dispatch / combine
 # --------------------------------------------------------------------------
+def janus_active_experts(counts, *, active=None, n_active=None, stream=None):
+    """Per layer, the ids of the experts with routed rows (ascending) and their
+    number: (active [L,E] (first n_active[l] valid), n_active [L])."""
+    c = counts.reshape(-1, counts.shape[-1])
+    L, E = c.shape
+    if active is None:
+        active = torch.full((L, E), -1, dtype=torch.int32, device=counts.device)
+    if n_active is None:
+        n_active = _empty((L,), torch.int32, counts.device)
+    _raise(lib().janus_active_experts(_p(c.contiguous(), torch.int32, "counts"), L, E,
+                                      _p(active, torch.int32, "active"), _p(n_active, torch.int32, "n_active"),
+                                      _stream(stream)), "janus_active_experts")
+    return active, n_active
+
+
 def janus_dispatch(x, slot_of, top_k, topk_weight=None, *, out=None, stream=None):
     N, d = x.shape
     K = int(top_k)

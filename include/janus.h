@@ -115,6 +115,16 @@ janus_status janus_route_layers(const int32_t* types, int64_t n_atoms, const flo
                                 int32_t* offsets, int32_t* perm, int32_t* slot_of, void* workspace,
                                 size_t workspace_bytes, janus_stream_t stream);
 
+/* Active-expert lists ([News], JIT planning: the experts a batch activates are
+ * restored before the expert stage).  For each of L layers, the experts with
+ * at least one routed row, in ascending id order:
+ *   active[l*E + j] = the j-th e with counts[l*E + e] > 0, j < n_active[l]
+ * in : counts [L,E] (device int32, e.g. janus_route_layers' counts)
+ * out: active [L,E] (entries past n_active[l] untouched), n_active [L]
+ * One CTA per layer; E <= 256.  Errors: JANUS_ERR_INVALID_ARG on bad sizes. */
+janus_status janus_active_experts(const int32_t* counts, int32_t n_layers, int32_t n_experts,
+                                  int32_t* active, int32_t* n_active, janus_stream_t stream);
+
 /* -------------------------------------------------------------------------
  * Dispatch.  [Review] section 3.5 (CNIS kernels, MoE dispatch/combine).
  *   xd[slot_of[i*K+k], :] = x[i, :] * (topk_weight ? topk_weight[i*K+k] : 1)

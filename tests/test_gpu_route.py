@@ -152,3 +152,33 @@ def test_route_layers_zero_atoms_and_bad_type():
     with pytest.raises(J.JanusError) as e:
         J.janus_check(r["workspace"])
     assert e.value.status == J.JANUS_ERR_DATA
+
+
+# ---- active-expert lists (JIT planning: the experts a batch activates) ----
+
+@pytest.mark.parametrize("E", [1, 7, 32, 72, 256])
+def test_active_experts_match_numpy_nonzero(E):
+    g = np.random.default_rng(E)
+    L = 13
+    counts = g.integers(0, 4, size=(L, E)).astype(np.int32)
+    counts[g.random((L, E)) < 0.5] = 0
+    counts[0] = 0                     # a layer with no active expert
+    counts[1] = 1                     # a layer with every expert active
+    active, n_active = J.janus_active_experts(to_dev(counts))
+    a, n = host(active), host(n_active)
+    for l in range(L):
+        ref = np.nonzero(counts[l])[0]
+        assert n[l] == ref.size
+        assert np.array_equal(a[l, :n[l]], ref)
+        assert np.all(a[l, n[l]:] == -1)     # entries past the count untouched
+
+
+def test_active_experts_of_routed_layers():
+    N, T, E, K, L = 3000, 13, 24, 3, 4
+    types = synth.types_zipf(N, T, seed=9)
+    gates = np.stack([synth.gate_table(T, E, 300 + l) for l in range(L)])
+    r = J.janus_route_layers(to_dev(types), to_dev(gates), K)
+    active, n_active = J.janus_active_experts(r["counts"])
+    for l in range(L):
+        ref = np.nonzero(oracle.route(types, gates[l], K)["counts"])[0]
+        assert np.array_equal(host(active)[l, :host(n_active)[l]], ref)
