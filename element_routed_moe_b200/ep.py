@@ -107,6 +107,13 @@ class ExpertParallelLayer:
             dist.all_gather(parts, counts.cpu(), group=self.group)
             self.counts_all.copy_(torch.stack(parts))
 
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+        return False
+
     def close(self):
         torch.cuda.synchronize(self.dev)
         if self.world > 1:
