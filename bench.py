@@ -61,6 +61,9 @@ def parse():
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism over the ranks (experts split, FP16 all-to-all by peer "
                          "stores) instead of independent replicas")
+    ap.add_argument("--ep-return", choices=("fused", "copy"), default="fused",
+                    help="--ep: the experts' last GEMM stores into the senders' return buffers (fused) or "
+                         "a separate kernel copies the rows back (copy)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip timing the weight-gradient, multi-layer routing and edge-side calls")
     ap.add_argument("--ref-seconds", type=float, default=None,
@@ -477,7 +480,8 @@ def run_ep(args, world, rank, local):
     del w1, w2, inp["w1"], inp["w2"]
     types = torch.as_tensor(inp["types"], device=dev)
     x, g = inp["x"], inp["g"]
-    layer = ExpertParallelLayer(N, d, h, T, E, K, w1l, w2l, mode=mode, device=dev)
+    layer = ExpertParallelLayer(N, d, h, T, E, K, w1l, w2l, mode=mode, device=dev,
+                                fused_return=args.ep_return == "fused")
     peaks, peak_src = measured_peaks()
     for _ in range(args.warmup):
         layer.forward(x, types, gate)
@@ -526,11 +530,11 @@ def run_ep(args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": t_max / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {**describe(cfg), "ffn_mode": args.mode, "parallelism": f"ep{world}",
-                   "experts_per_rank": El, "received_rows_rank0": r_recv,
+                   "experts_per_rank": El, "received_rows_rank0": r_recv, "ep_return": args.ep_return,
                    "l2": "no flush: per-step working set far above the 126 MB L2"},
         "roofline": roof,
         "breakdown_ms": ph_ms,
-        "gpu_launches": 18 * args.steps,
+        "gpu_launches": layer.launches_per_step * args.steps,
         "clocks": clocks,
     }
     layer.close()

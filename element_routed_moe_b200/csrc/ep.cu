@@ -214,25 +214,35 @@ ep_dequant_rows_kernel(const uint2* __restrict__ payload, const float* __restric
   }
 }
 
+// Where owner row j (j < the received count) came from: its sender s and
+// the row in the sender's local expert order.
+__device__ __forceinline__ int64_t sender_row(const int32_t* __restrict__ src_off,
+                                              const int32_t* __restrict__ dst_off,
+                                              const int32_t* __restrict__ recv_off_r, int rank, int P, int E,
+                                              int64_t j, int* sender) {
+  const int El = E / P;
+  int lo = 0, hi = El;                         // recv_off_r[lo] <= j < recv_off_r[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (recv_off_r[mid] <= j) lo = mid; else hi = mid;
+  }
+  const int e = rank * El + lo;
+  int s = 0;                                   // the last sender whose block starts at or before j
+  while (s + 1 < P && dst_off[(s + 1) * E + e] <= j) ++s;
+  *sender = s;
+  return (int64_t)src_off[s * (E + 1) + e] + (j - dst_off[s * E + e]);
+}
+
 // Owner side: each received row's result back to its sender's local row.
 __global__ void __launch_bounds__(kThreads)
-ep_return_kernel(const float4* __restrict__ yd, const int32_t* __restrict__ counts_all,
-                 const int32_t* __restrict__ src_off, const int32_t* __restrict__ dst_off,
-                 const int32_t* __restrict__ recv_off_r, int rank, int P, int E, int64_t max_rows, int d4,
-                 PeerRows peers) {
-  const int El = E / P;
-  const int64_t n = min((int64_t)recv_off_r[El], max_rows);
+ep_return_kernel(const float4* __restrict__ yd, const int32_t* __restrict__ src_off,
+                 const int32_t* __restrict__ dst_off, const int32_t* __restrict__ recv_off_r, int rank,
+                 int P, int E, int64_t max_rows, int d4, PeerRows peers) {
+  const int64_t n = min((int64_t)recv_off_r[E / P], max_rows);
   const int lane = threadIdx.x % 32;
   for (int64_t j = global_warp(); j < n; j += total_warps()) {
-    int lo = 0, hi = El;                       // recv_off_r[lo] <= j < recv_off_r[hi]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (recv_off_r[mid] <= j) lo = mid; else hi = mid;
-    }
-    const int e = rank * El + lo;
-    int s = 0;
-    while (s + 1 < P && dst_off[(s + 1) * E + e] <= j) ++s;
-    const int64_t row = (int64_t)src_off[s * (E + 1) + e] + (j - dst_off[s * E + e]);
+    int s;
+    const int64_t row = sender_row(src_off, dst_off, recv_off_r, rank, P, E, j, &s);
     const float4* src = yd + j * d4;
     float4* dst = reinterpret_cast<float4*>(peers.ptr[s]) + row * d4;
     for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
@@ -251,6 +261,21 @@ ep_return_kernel(const float4* __restrict__ yd, const int32_t* __restrict__ coun
   }
   // the peer stores are visible system-wide before this kernel completes
   __threadfence_system();
+}
+
+// Owner side of the fused return: the address in its sender's return buffer
+// of every received row, for a GEMM epilogue that stores through the table.
+__global__ void __launch_bounds__(kThreads)
+ep_return_rows_kernel(const int32_t* __restrict__ src_off, const int32_t* __restrict__ dst_off,
+                      const int32_t* __restrict__ recv_off_r, int rank, int P, int E, int64_t max_rows, int d,
+                      PeerRows peers, float** __restrict__ rows) {
+  const int64_t n = min((int64_t)recv_off_r[E / P], max_rows);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n; j += stride) {
+    int s;
+    const int64_t row = sender_row(src_off, dst_off, recv_off_r, rank, P, E, j, &s);
+    rows[j] = reinterpret_cast<float*>(peers.ptr[s]) + row * d;
+  }
 }
 
 janus_status check_ep(int32_t rank, int32_t world, int32_t n_experts) {
@@ -397,8 +422,30 @@ extern "C" janus_status janus_ep_return(const float* yd, const int32_t* counts_a
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
   const int El = n_experts / world;
   ep_return_kernel<<<rows_grid(max_rows, 8), kThreads, 0, (cudaStream_t)stream>>>(
-      (const float4*)yd, counts_all, src_off, dst_off, recv_off + (size_t)rank * (El + 1), rank, world, n_experts,
+      (const float4*)yd, src_off, dst_off, recv_off + (size_t)rank * (El + 1), rank, world, n_experts,
       max_rows, d / 4, peers);
+  return launch_status();
+}
+
+extern "C" janus_status janus_ep_return_rows(const int32_t* src_off, const int32_t* dst_off,
+                                             const int32_t* recv_off, int32_t rank, int32_t world,
+                                             int32_t n_experts, int64_t max_rows, int32_t d,
+                                             float* const* ret_rows, float** rows, janus_stream_t stream) {
+  janus_status st = check_ep(rank, world, n_experts);
+  if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(max_rows >= 0 && d >= 1 && d <= kMaxDim);
+  JANUS_CHECK_ALIGN(d % 4 == 0);
+  PeerRows peers;
+  st = peer_table(reinterpret_cast<void* const*>(ret_rows), nullptr, world, 16, &peers);
+  if (st != JANUS_OK) return st;
+  if (max_rows == 0) return JANUS_OK;
+  JANUS_CHECK_ARG(rows && src_off && dst_off && recv_off);
+  JANUS_CHECK_ALIGN(aligned(rows, 8));
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  const int El = n_experts / world;
+  const int64_t blocks = std::min<int64_t>((max_rows + kThreads - 1) / kThreads, (int64_t)num_sms() * 8);
+  ep_return_rows_kernel<<<(unsigned)blocks, kThreads, 0, (cudaStream_t)stream>>>(
+      src_off, dst_off, recv_off + (size_t)rank * (El + 1), rank, world, n_experts, max_rows, d, peers, rows);
   return launch_status();
 }
 

@@ -60,7 +60,7 @@ simt::Args make_args(const float* A, const float* B, int64_t bstride, float* C, 
                      const float* aux, const int32_t* offsets, int E, int Kd, int N) {
   simt::Args a;
   a.A = A; a.B = B; a.b_expert_stride = bstride; a.C = C; a.C2 = C2; a.aux = aux;
-  a.aux2 = nullptr; a.C3 = nullptr;
+  a.aux2 = nullptr; a.C3 = nullptr; a.c_rows = nullptr;
   a.offsets = offsets; a.E = E; a.Kd = Kd; a.N = N;
   return a;
 }
@@ -80,14 +80,15 @@ extern "C" janus_status janus_expert_ffn_workspace_size(int64_t n_rows, int32_t 
   return JANUS_OK;
 }
 
-extern "C" janus_status janus_expert_ffn_fwd(const float* xd, const int32_t* offsets,
-                                             int32_t n_experts, int64_t n_rows, int32_t d,
-                                             int32_t h, const float* w1, const float* w2,
-                                             float* yd, float* act, janus_ffn_mode mode,
-                                             void* workspace, size_t workspace_bytes,
-                                             janus_stream_t stream_) {
+namespace {
+
+// yd_rows (device array of n_rows row pointers) replaces yd when set.
+janus_status ffn_fwd(const float* xd, const int32_t* offsets, int32_t n_experts, int64_t n_rows, int32_t d,
+                     int32_t h, const float* w1, const float* w2, float* yd, float* const* yd_rows, float* act,
+                     janus_ffn_mode mode, void* workspace, size_t workspace_bytes, janus_stream_t stream_) {
   cudaStream_t stream = (cudaStream_t)stream_;
-  janus_status st = check_ffn(xd, offsets, n_experts, n_rows, d, h, w1, w2, yd, mode);
+  janus_status st = check_ffn(xd, offsets, n_experts, n_rows, d, h, w1, w2,
+                              yd_rows ? reinterpret_cast<const float*>(yd_rows) : yd, mode);
   if (st != JANUS_OK) return st;
   const FfnLayout L = ffn_layout(n_rows, h, false, act != nullptr);
   JANUS_CHECK_ARG(workspace && workspace_bytes >= L.total);
@@ -99,23 +100,25 @@ extern "C" janus_status janus_expert_ffn_fwd(const float* xd, const int32_t* off
   if (mode == JANUS_FFN_3XTF32) {
     JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
     st = tc::expert_ffn_fwd(xd, offsets, n_experts, n_rows, d, h, w1, w2, yd, act, H,
-                            &((WsHeader*)workspace)->error, stream);
+                            &((WsHeader*)workspace)->error, stream, yd_rows);
     if (st != JANUS_OK) return st;
     return launch_status();
   }
   launch_simt<false, simt::kEpiSilu>(make_args(xd, w1, sw, H, act, nullptr, offsets, n_experts, d, h), stream);
-  launch_simt<false, simt::kEpiStore>(make_args(H, w2, sw, yd, nullptr, nullptr, offsets, n_experts, h, d), stream);
+  simt::Args a2 = make_args(H, w2, sw, yd, nullptr, nullptr, offsets, n_experts, h, d);
+  a2.c_rows = yd_rows;
+  launch_simt<false, simt::kEpiStore>(a2, stream);
   return launch_status();
 }
 
-extern "C" janus_status janus_expert_ffn_vjp(const float* xd, const float* gd, const float* act,
-                                             const int32_t* offsets, int32_t n_experts,
-                                             int64_t n_rows, int32_t d, int32_t h,
-                                             const float* w1, const float* w2, float* dxd,
-                                             janus_ffn_mode mode, void* workspace,
-                                             size_t workspace_bytes, janus_stream_t stream_) {
+// dxd_rows (device array of n_rows row pointers) replaces dxd when set.
+janus_status ffn_vjp(const float* xd, const float* gd, const float* act, const int32_t* offsets,
+                     int32_t n_experts, int64_t n_rows, int32_t d, int32_t h, const float* w1, const float* w2,
+                     float* dxd, float* const* dxd_rows, janus_ffn_mode mode, void* workspace,
+                     size_t workspace_bytes, janus_stream_t stream_) {
   cudaStream_t stream = (cudaStream_t)stream_;
-  janus_status st = check_ffn(xd, offsets, n_experts, n_rows, d, h, w1, w2, dxd, mode);
+  janus_status st = check_ffn(xd, offsets, n_experts, n_rows, d, h, w1, w2,
+                              dxd_rows ? reinterpret_cast<const float*>(dxd_rows) : dxd, mode);
   if (st != JANUS_OK) return st;
   JANUS_CHECK_ARG(n_rows == 0 || gd);
   JANUS_CHECK_ALIGN(n_rows == 0 || aligned(gd, 16));
@@ -132,15 +135,61 @@ extern "C" janus_status janus_expert_ffn_vjp(const float* xd, const float* gd, c
   if (mode == JANUS_FFN_3XTF32) {
     JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
     st = tc::expert_ffn_vjp(xd, gd, act, A, offsets, n_experts, n_rows, d, h, w1, w2, dxd, dA,
-                            &((WsHeader*)workspace)->error, stream);
+                            &((WsHeader*)workspace)->error, stream, dxd_rows);
     if (st != JANUS_OK) return st;
     return launch_status();
   }
   if (!act)
     launch_simt<false, simt::kEpiStore>(make_args(xd, w1, sw, A, nullptr, nullptr, offsets, n_experts, d, h), stream);
   launch_simt<true, simt::kEpiDSilu>(make_args(gd, w2, sw, dA, nullptr, A, offsets, n_experts, d, h), stream);
-  launch_simt<true, simt::kEpiStore>(make_args(dA, w1, sw, dxd, nullptr, nullptr, offsets, n_experts, h, d), stream);
+  simt::Args a4 = make_args(dA, w1, sw, dxd, nullptr, nullptr, offsets, n_experts, h, d);
+  a4.c_rows = dxd_rows;
+  launch_simt<true, simt::kEpiStore>(a4, stream);
   return launch_status();
+}
+
+}  // namespace
+
+extern "C" janus_status janus_expert_ffn_fwd(const float* xd, const int32_t* offsets,
+                                             int32_t n_experts, int64_t n_rows, int32_t d,
+                                             int32_t h, const float* w1, const float* w2,
+                                             float* yd, float* act, janus_ffn_mode mode,
+                                             void* workspace, size_t workspace_bytes,
+                                             janus_stream_t stream) {
+  return ffn_fwd(xd, offsets, n_experts, n_rows, d, h, w1, w2, yd, nullptr, act, mode, workspace,
+                 workspace_bytes, stream);
+}
+
+extern "C" janus_status janus_expert_ffn_fwd_rows(const float* xd, const int32_t* offsets,
+                                                  int32_t n_experts, int64_t n_rows, int32_t d,
+                                                  int32_t h, const float* w1, const float* w2,
+                                                  float* const* yd_rows, float* act, janus_ffn_mode mode,
+                                                  void* workspace, size_t workspace_bytes,
+                                                  janus_stream_t stream) {
+  JANUS_CHECK_ARG(n_rows == 0 || yd_rows);
+  return ffn_fwd(xd, offsets, n_experts, n_rows, d, h, w1, w2, nullptr, yd_rows, act, mode, workspace,
+                 workspace_bytes, stream);
+}
+
+extern "C" janus_status janus_expert_ffn_vjp(const float* xd, const float* gd, const float* act,
+                                             const int32_t* offsets, int32_t n_experts,
+                                             int64_t n_rows, int32_t d, int32_t h,
+                                             const float* w1, const float* w2, float* dxd,
+                                             janus_ffn_mode mode, void* workspace,
+                                             size_t workspace_bytes, janus_stream_t stream) {
+  return ffn_vjp(xd, gd, act, offsets, n_experts, n_rows, d, h, w1, w2, dxd, nullptr, mode, workspace,
+                 workspace_bytes, stream);
+}
+
+extern "C" janus_status janus_expert_ffn_vjp_rows(const float* xd, const float* gd, const float* act,
+                                                  const int32_t* offsets, int32_t n_experts,
+                                                  int64_t n_rows, int32_t d, int32_t h,
+                                                  const float* w1, const float* w2, float* const* dxd_rows,
+                                                  janus_ffn_mode mode, void* workspace,
+                                                  size_t workspace_bytes, janus_stream_t stream) {
+  JANUS_CHECK_ARG(n_rows == 0 || dxd_rows);
+  return ffn_vjp(xd, gd, act, offsets, n_experts, n_rows, d, h, w1, w2, nullptr, dxd_rows, mode, workspace,
+                 workspace_bytes, stream);
 }
 
 extern "C" janus_status janus_expert_ffn_weight_grad_workspace_size(int64_t n_rows, int32_t h,

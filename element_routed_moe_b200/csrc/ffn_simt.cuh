@@ -39,6 +39,7 @@ struct Args {
   const float* aux;          // pre-activation for kEpiDSilu / kEpiD2, [R, N]
   const float* aux2;         // kEpiD2: dh = gd W2^T, [R, N]
   float* C3;                 // kEpiD2: optional third output
+  float* const* c_rows;      // kEpiStore: if set, row p is stored at c_rows[p] (not C + p N)
   const int32_t* offsets;
   int E;
   int Kd;                    // reduction length
@@ -229,10 +230,13 @@ __global__ void __launch_bounds__(kThreads, 2) grouped_gemm_kernel(Args args) {
           *reinterpret_cast<float4*>(args.C2 + o) = t2;
           if (args.C3) *reinterpret_cast<float4*>(args.C3 + o) = u;
         }
-        *reinterpret_cast<float4*>(args.C + o) = v;
+        float* dst = (kEpi == kEpiStore && args.c_rows) ? args.c_rows[r] + c : args.C + o;
+        *reinterpret_cast<float4*>(dst) = v;
       }
     }
   }
+  // rows stored through c_rows may sit in another GPU's memory
+  if (kEpi == kEpiStore && args.c_rows) __threadfence_system();
 }
 
 // Per-expert weight gradient on the CUDA cores:

@@ -108,6 +108,7 @@ struct Args {
   float* C3;
   const float* aux;
   const float* aux2;
+  float* const* c_rows;   // NN/NT plain store: if set, row p goes to c_rows[p] (e.g. a peer's buffer)
   const int32_t* offsets;
   int E, Kd, N;
   int M;            // kModeTN: rows of each expert's output (C is [E][M][N])
@@ -431,6 +432,10 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
             if (j0 + jb + j < c.n_valid) {
               const int64_t o = (int64_t)(c.n0 + j0 + jb + j) * N + f;
               float v = acc[jb + j];
+              if (kEpi == kEpiStore && args.c_rows) {   // the row's own destination
+                args.c_rows[c.n0 + j0 + jb + j][f] = v;
+                continue;
+              }
               if (kEpi == kEpiSilu) {
                 if (args.C2) args.C2[o] = v;
                 v = silu_f(v);
@@ -472,6 +477,9 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
       }
     }
   }
+  // rows stored through c_rows may sit in another GPU's memory: make them
+  // visible system-wide before the kernel completes
+  if (kEpi == kEpiStore && args.c_rows) __threadfence_system();
 }
 
 template <int kMode, int kEpi>
@@ -776,7 +784,7 @@ constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Smem
 template <int kMode, int kEpi>
 janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, int N, float* C, float* C2,
                     const float* aux, const int32_t* offsets, int32_t* err, cudaStream_t stream, int M = 0,
-                    const float* aux2 = nullptr, float* C3 = nullptr) {
+                    const float* aux2 = nullptr, float* C3 = nullptr, float* const* c_rows = nullptr) {
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
@@ -792,7 +800,7 @@ janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, in
     return JANUS_ERR_CUDA;
   }
   Args a;
-  a.C = C; a.C2 = C2; a.C3 = C3; a.aux = aux; a.aux2 = aux2;
+  a.C = C; a.C2 = C2; a.C3 = C3; a.aux = aux; a.aux2 = aux2; a.c_rows = c_rows;
   a.offsets = offsets; a.E = E; a.Kd = Kd; a.N = N; a.M = M; a.err = err;
   // one CTA per SM, in clusters of two (the MMA pairs)
   cudaLaunchConfig_t cfg = {};
@@ -817,16 +825,17 @@ size_t workspace_extra() { return 0; }
 
 janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, int64_t R, int32_t d,
                             int32_t h, const float* w1, const float* w2, float* yd, float* act, float* H,
-                            int32_t* err, cudaStream_t stream) {
+                            int32_t* err, cudaStream_t stream, float* const* yd_rows) {
   janus_status st = launch<kModeNN, kEpiSilu>(xd, w1, R, E, d, h, H, act, nullptr, offsets, err, stream);
   if (st != JANUS_OK) return st;
-  return launch<kModeNN, kEpiStore>(H, w2, R, E, h, d, yd, nullptr, nullptr, offsets, err, stream);
+  return launch<kModeNN, kEpiStore>(H, w2, R, E, h, d, yd, nullptr, nullptr, offsets, err, stream, 0, nullptr,
+                                    nullptr, yd_rows);
 }
 
 janus_status expert_ffn_vjp(const float* xd, const float* gd, const float* act_in, float* A,
                             const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
                             const float* w1, const float* w2, float* dxd, float* dA, int32_t* err,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, float* const* dxd_rows) {
   janus_status st;
   if (!act_in) {
     st = launch<kModeNN, kEpiStore>(xd, w1, R, E, d, h, A, nullptr, nullptr, offsets, err, stream);
@@ -834,7 +843,8 @@ janus_status expert_ffn_vjp(const float* xd, const float* gd, const float* act_i
   }
   st = launch<kModeNT, kEpiDSilu>(gd, w2, R, E, d, h, dA, nullptr, A, offsets, err, stream);
   if (st != JANUS_OK) return st;
-  return launch<kModeNT, kEpiStore>(dA, w1, R, E, h, d, dxd, nullptr, nullptr, offsets, err, stream);
+  return launch<kModeNT, kEpiStore>(dA, w1, R, E, h, d, dxd, nullptr, nullptr, offsets, err, stream, 0, nullptr,
+                                    nullptr, dxd_rows);
 }
 
 janus_status expert_ffn_weight_grad(const float* xd, const float* gd, const float* act_in, float* A,

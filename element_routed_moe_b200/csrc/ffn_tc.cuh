@@ -12,14 +12,16 @@ size_t workspace_extra();
 
 // `err` is the workspace header's error word (a bounded wait that ran out
 // records a timeout there).
+// yd_rows (nullable): row p of yd is written to yd_rows[p] instead of yd + p d.
 janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, int64_t R,
                             int32_t d, int32_t h, const float* w1, const float* w2, float* yd,
-                            float* act, float* H, int32_t* err, cudaStream_t stream);
+                            float* act, float* H, int32_t* err, cudaStream_t stream,
+                            float* const* yd_rows = nullptr);
 
 janus_status expert_ffn_vjp(const float* xd, const float* gd, const float* act_in, float* A,
                             const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
                             const float* w1, const float* w2, float* dxd, float* dA, int32_t* err,
-                            cudaStream_t stream);
+                            cudaStream_t stream, float* const* dxd_rows = nullptr);
 
 // Per-expert weight gradients: dW1[e] = Xd_e^T dA_e, dW2[e] = H_e^T Gd_e with
 // dA = (gd W2^T) * silu'(a) and H = silu(a) computed into dA and H.

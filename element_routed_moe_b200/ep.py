@@ -12,6 +12,12 @@ atoms.  One layer pass:
   VJP:      weighted FP32 send of dY -> barrier -> owner: input VJP of its
             experts -> return -> barrier -> combine (local)
 
+The return is fused into the experts' last GEMM by default: its epilogue
+stores each output row straight into the sender's return buffer through a row
+table (janus_ep_return_rows), so the rows cross NVLink as the tiles finish and
+no separate copy kernel runs.  fused_return=False keeps the copy kernel
+(janus_ep_return) after the GEMM.
+
 Every step is a kernel of libjanus; torch.distributed carries only the
 counts, the IPC handles (once) and the phase barriers.  The receive and return
 buffers are allocated once at their worst-case size (all routed rows of all
@@ -30,7 +36,7 @@ class ExpertParallelLayer:
     """Buffers, peer mappings and the ordered calls of one EP layer pass."""
 
     def __init__(self, n_atoms_max, d, h, n_types, n_experts, top_k, w1_local, w2_local, *,
-                 mode=J.JANUS_FFN_3XTF32, group=None, device=None):
+                 mode=J.JANUS_FFN_3XTF32, group=None, device=None, fused_return=True):
         self.group = group
         self.dist = dist.is_available() and dist.is_initialized()
         # without a process group the layer is a single rank owning every expert
@@ -46,6 +52,11 @@ class ExpertParallelLayer:
         if w1_local.shape != (self.El, d, h) or w2_local.shape != (self.El, h, d):
             raise ValueError("w1_local / w2_local must hold this rank's E/P experts")
         self.w1, self.w2, self.mode = w1_local, w2_local, mode
+        self.fused_return = bool(fused_return)
+        # this library's kernels per forward + VJP: route 4, layout 1, pack 2,
+        # unpack 1, expert MLP 2 + 2, FP32 send 1, combine 1 + 1, and the
+        # return table (fused) or the return copy twice (not fused)
+        self.launches_per_step = 15 + (1 if self.fused_return else 2)
         self.nccl = self.dist and dist.get_backend(group) == "nccl"
         # worst case: every routed row of every rank lands on this rank
         self.n_atoms_max = int(n_atoms_max)
@@ -60,6 +71,7 @@ class ExpertParallelLayer:
         self.act = torch.empty((cap, h), **f32)
         self.yd = torch.empty((cap, d), **f32)
         self.ret = torch.empty((rows, d), **f32)             # this rank's rows coming back
+        self.ret_rows = torch.zeros((cap,), dtype=torch.int64, device=self.dev)   # fused-return row table
         self.counts_all = torch.empty((self.world, n_experts), dtype=torch.int32, device=self.dev)
         self._token = torch.zeros(1, **f32)
         self._opened = []
@@ -153,10 +165,17 @@ class ExpertParallelLayer:
         recv_off = self.layout[2][self.rank]
         m(events, "ffn_fwd", 0)
         J.janus_ep_dequant_rows(self.payload, self.row_scale, self.layout, self.rank, out=self.xd)
-        J.janus_expert_ffn_fwd(self.xd, recv_off, self.w1, self.w2, mode=self.mode, out=self.yd, act=self.act)
+        if self.fused_return:
+            # the table depends only on the layout: the VJP reuses it
+            J.janus_ep_return_rows(self.layout, self.rank, self.peer_ret, self.cap, self.d, out=self.ret_rows)
+            J.janus_expert_ffn_fwd_rows(self.xd, recv_off, self.w1, self.w2, self.ret_rows, mode=self.mode,
+                                        act=self.act)
+        else:
+            J.janus_expert_ffn_fwd(self.xd, recv_off, self.w1, self.w2, mode=self.mode, out=self.yd, act=self.act)
         m(events, "ffn_fwd", 1)
         m(events, "return", 0)
-        J.janus_ep_return(self.yd, self.counts_all, self.layout, self.rank, self.peer_ret)
+        if not self.fused_return:
+            J.janus_ep_return(self.yd, self.counts_all, self.layout, self.rank, self.peer_ret)
         self.barrier()
         m(events, "return", 1)
         R = x.shape[0] * self.K
@@ -175,11 +194,16 @@ class ExpertParallelLayer:
         m(events, "send_vjp", 1)
         recv_off = self.layout[2][self.rank]
         m(events, "ffn_vjp", 0)
-        J.janus_expert_ffn_vjp(self.xd, self.recv_rows, recv_off, self.w1, self.w2, act=self.act,
-                               mode=self.mode, out=self.yd)
+        if self.fused_return:
+            J.janus_expert_ffn_vjp_rows(self.xd, self.recv_rows, recv_off, self.w1, self.w2, self.ret_rows,
+                                        act=self.act, mode=self.mode)
+        else:
+            J.janus_expert_ffn_vjp(self.xd, self.recv_rows, recv_off, self.w1, self.w2, act=self.act,
+                                   mode=self.mode, out=self.yd)
         m(events, "ffn_vjp", 1)
         m(events, "return_vjp", 0)
-        J.janus_ep_return(self.yd, self.counts_all, self.layout, self.rank, self.peer_ret)
+        if not self.fused_return:
+            J.janus_ep_return(self.yd, self.counts_all, self.layout, self.rank, self.peer_ret)
         self.barrier()
         m(events, "return_vjp", 1)
         R = self.x_shape[0] * self.K

@@ -35,11 +35,12 @@ SYMBOLS = (
     "janus_quant_by_type_workspace_size", "janus_quant_by_type", "janus_quant_by_type_noalloc",
     "janus_dequant_by_type",
     "janus_expert_ffn_workspace_size", "janus_expert_ffn_fwd", "janus_expert_ffn_vjp",
+    "janus_expert_ffn_fwd_rows", "janus_expert_ffn_vjp_rows",
     "janus_expert_ffn_weight_grad_workspace_size", "janus_expert_ffn_weight_grad",
     "janus_expert_ffn_vjp_vjp_workspace_size", "janus_expert_ffn_vjp_vjp",
     "janus_combine", "janus_edge_aggregate", "janus_edge_broadcast", "janus_neighbor_aggregate",
     "janus_ep_layout", "janus_ep_dispatch_quant", "janus_ep_dispatch", "janus_ep_dequant_rows",
-    "janus_ep_return", "janus_ipc_get_handle", "janus_ipc_open_handle", "janus_ipc_close_handle",
+    "janus_ep_return", "janus_ep_return_rows", "janus_ipc_get_handle", "janus_ipc_open_handle", "janus_ipc_close_handle",
     "janus_debug_inject_launch_failures",
 )
 
@@ -98,6 +99,10 @@ def _declare(L):
                                       vp, sz, vp]),
         "janus_expert_ffn_vjp": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp,
                                       ctypes.c_int, vp, sz, vp]),
+        "janus_expert_ffn_fwd_rows": (st, [vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, ctypes.c_int,
+                                           vp, sz, vp]),
+        "janus_expert_ffn_vjp_rows": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp,
+                                           ctypes.c_int, vp, sz, vp]),
         "janus_expert_ffn_weight_grad_workspace_size": (st, [i64, i32, i32, psz]),
         "janus_expert_ffn_weight_grad": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp,
                                               ctypes.c_int, vp, sz, vp]),
@@ -114,6 +119,7 @@ def _declare(L):
         "janus_ep_dispatch": (st, [vp, i64, i32, i32, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp]),
         "janus_ep_dequant_rows": (st, [vp, vp, vp, i32, i32, i32, i64, i32, vp, vp]),
         "janus_ep_return": (st, [vp, vp, vp, vp, vp, i32, i32, i32, i64, i32, vp, vp]),
+        "janus_ep_return_rows": (st, [vp, vp, vp, i32, i32, i32, i64, i32, vp, vp, vp]),
         "janus_ipc_get_handle": (st, [vp, ctypes.POINTER(IpcHandle)]),
         "janus_ipc_open_handle": (st, [ctypes.POINTER(IpcHandle), ctypes.POINTER(ctypes.c_void_p)]),
         "janus_ipc_close_handle": (st, [vp, ctypes.c_uint64]),
@@ -370,6 +376,23 @@ def janus_ep_return(yd, counts_all, layout, rank, ret_rows, *, stream=None):
                                  _ptr_array(ret_rows), _stream(stream)), "janus_ep_return")
 
 
+def janus_ep_return_rows(layout, rank, ret_rows, max_rows, d, *, out=None, stream=None):
+    """Row table of the fused return: int64 device tensor [max_rows] holding,
+    for each received row, its address in the sender's return buffer (entries
+    past the received count stay as they were; a new table starts at 0)."""
+    src_off, dst_off, recv_off = layout
+    P, E = dst_off.shape
+    if out is None:
+        out = torch.zeros((max_rows,), dtype=torch.int64, device=src_off.device)
+    if out.dtype != torch.int64 or out.numel() < max_rows:
+        raise ValueError("out must be an int64 tensor of at least max_rows entries")
+    _raise(lib().janus_ep_return_rows(_p(src_off, torch.int32, "src_off"), _p(dst_off, torch.int32, "dst_off"),
+                                      _p(recv_off, torch.int32, "recv_off"), int(rank), P, E, int(max_rows),
+                                      int(d), _ptr_array(ret_rows), _p(out, torch.int64, "rows"),
+                                      _stream(stream)), "janus_ep_return_rows")
+    return out
+
+
 def janus_ipc_get_handle(t) -> bytes:
     """Serialised janus_ipc_handle of a device tensor's storage."""
     h = IpcHandle()
@@ -502,6 +525,46 @@ def janus_expert_ffn_vjp(xd, gd, offsets, w1, w2, *, act=None, mode=JANUS_FFN_FP
                                       _p(out, torch.float32, "dxd"), int(mode), _p(ws), nb,
                                       _stream(stream)), "janus_expert_ffn_vjp")
     return out
+
+
+def _row_table(rows, R):
+    if rows.dtype != torch.int64 or rows.dim() != 1 or rows.numel() < R:
+        raise ValueError("the row table must be a 1-D int64 tensor of at least n_rows addresses")
+    return _p(rows, torch.int64, "rows")
+
+
+def janus_expert_ffn_fwd_rows(xd, offsets, w1, w2, yd_rows, *, mode=JANUS_FFN_FP32_SIMT, want_act=False,
+                              act=None, workspace=None, stream=None):
+    """janus_expert_ffn_fwd with output row p stored at address yd_rows[p]
+    (int64 device tensor); returns act-or-None."""
+    R, d = xd.shape
+    E, _, h = w1.shape
+    if want_act and act is None:
+        act = _empty((R, h), torch.float32, xd.device)
+    nb = janus_expert_ffn_workspace_size(R, d, h, E, False, act is not None, mode)
+    ws = _workspace(nb, xd.device, workspace)
+    _raise(lib().janus_expert_ffn_fwd_rows(_p(xd, torch.float32, "xd"),
+                                           _p(offsets, torch.int32, "offsets"), E, R, d, h,
+                                           _p(w1, torch.float32, "w1"), _p(w2, torch.float32, "w2"),
+                                           _row_table(yd_rows, R), _p(act, torch.float32, "act"),
+                                           int(mode), _p(ws), nb, _stream(stream)),
+           "janus_expert_ffn_fwd_rows")
+    return act
+
+
+def janus_expert_ffn_vjp_rows(xd, gd, offsets, w1, w2, dxd_rows, *, act=None, mode=JANUS_FFN_FP32_SIMT,
+                              workspace=None, stream=None):
+    """janus_expert_ffn_vjp with row p of dxd stored at address dxd_rows[p]."""
+    R, d = xd.shape
+    E, _, h = w1.shape
+    nb = janus_expert_ffn_workspace_size(R, d, h, E, True, act is not None, mode)
+    ws = _workspace(nb, xd.device, workspace)
+    _raise(lib().janus_expert_ffn_vjp_rows(_p(xd, torch.float32, "xd"), _p(gd, torch.float32, "gd"),
+                                           _p(act, torch.float32, "act"),
+                                           _p(offsets, torch.int32, "offsets"), E, R, d, h,
+                                           _p(w1, torch.float32, "w1"), _p(w2, torch.float32, "w2"),
+                                           _row_table(dxd_rows, R), int(mode), _p(ws), nb,
+                                           _stream(stream)), "janus_expert_ffn_vjp_rows")
 
 
 def janus_expert_ffn_weight_grad_workspace_size(n_rows, h, have_act) -> int:

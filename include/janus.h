@@ -228,6 +228,25 @@ janus_status janus_expert_ffn_vjp(const float* xd, const float* gd, const float*
                                   float* dxd, janus_ffn_mode mode, void* workspace,
                                   size_t workspace_bytes, janus_stream_t stream);
 
+/* The same two calls with each output row stored at its own address:
+ * row p of yd (dxd) goes to yd_rows[p][0..d) (dxd_rows[p][0..d)) instead of
+ * yd + p d.  yd_rows / dxd_rows: device array of n_rows pointers (16-byte
+ * aligned array); each pointer 16-byte aligned with room for d floats,
+ * possibly in a peer GPU's mapped memory (janus_ep_return_rows builds the
+ * expert-parallel return table).  Only the rows of the offsets' segments are
+ * read from the table.  The final GEMM's stores are made visible system-wide
+ * before it completes. */
+janus_status janus_expert_ffn_fwd_rows(const float* xd, const int32_t* offsets, int32_t n_experts,
+                                       int64_t n_rows, int32_t d, int32_t h, const float* w1,
+                                       const float* w2, float* const* yd_rows, float* act,
+                                       janus_ffn_mode mode, void* workspace, size_t workspace_bytes,
+                                       janus_stream_t stream);
+janus_status janus_expert_ffn_vjp_rows(const float* xd, const float* gd, const float* act,
+                                       const int32_t* offsets, int32_t n_experts, int64_t n_rows,
+                                       int32_t d, int32_t h, const float* w1, const float* w2,
+                                       float* const* dxd_rows, janus_ffn_mode mode, void* workspace,
+                                       size_t workspace_bytes, janus_stream_t stream);
+
 /* Expert weight gradients, the parameter side of the same backward pass
  * (force training differentiates the energy w.r.t. inputs and weights,
  * [Review] section 3.3).  For L = sum_p <yd[p,:], gd[p,:]>:
@@ -345,6 +364,19 @@ janus_status janus_ep_return(const float* yd, const int32_t* counts_all, const i
                              const int32_t* dst_off, const int32_t* recv_off, int32_t rank, int32_t world,
                              int32_t n_experts, int64_t max_rows, int32_t d, float* const* ret_rows,
                              janus_stream_t stream);
+
+/* The fused return: instead of copying yd, the owner's expert MLP stores each
+ * output row straight into its sender's return buffer.  This call writes the
+ * row table for janus_expert_ffn_fwd_rows / janus_expert_ffn_vjp_rows:
+ * rows[r] = ret_rows[s] + (src_off[s][e] + r - dst_off[s][e]) * d for every
+ * received row r (r < recv_off[rank][E/P], at most max_rows) of sender s and
+ * expert e; rows[r] past the received count are left untouched.  rows: device
+ * array of max_rows pointers, 8-byte aligned.  ret_rows: as in
+ * janus_ep_return (16-byte aligned buffers).  The table depends only on the
+ * layout, so one table serves the forward and the VJP of a layer pass. */
+janus_status janus_ep_return_rows(const int32_t* src_off, const int32_t* dst_off, const int32_t* recv_off,
+                                  int32_t rank, int32_t world, int32_t n_experts, int64_t max_rows, int32_t d,
+                                  float* const* ret_rows, float** rows, janus_stream_t stream);
 
 /* CUDA IPC, so ranks on one node can map each other's buffers.  A handle names
  * the allocation that holds dev_ptr plus dev_ptr's byte offset in it (callers

@@ -110,6 +110,21 @@ def test_argument_validation_before_launch(J):
                                   1024, null) == J.JANUS_ERR_INVALID_ARG
     assert L.janus_expert_ffn_vjp(FAKE, null, null, FAKE, 4, 100, 64, 64, FAKE, FAKE, FAKE, 0,
                                   FAKE, 1 << 30, null) == J.JANUS_ERR_INVALID_ARG
+    # ffn with a row table: table missing, table misaligned
+    assert L.janus_expert_ffn_fwd_rows(FAKE, FAKE, 4, 100, 64, 64, FAKE, FAKE, null, null, 0, FAKE,
+                                       1 << 30, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_expert_ffn_fwd_rows(FAKE, FAKE, 4, 100, 64, 64, FAKE, FAKE, FAKE + 8, null, 0, FAKE,
+                                       1 << 30, null) == J.JANUS_ERR_MISALIGNED
+    assert L.janus_expert_ffn_vjp_rows(FAKE, FAKE, null, FAKE, 4, 100, 64, 64, FAKE, FAKE, null, 0,
+                                       FAKE, 1 << 30, null) == J.JANUS_ERR_INVALID_ARG
+    # EP return table: E not a multiple of P, missing peer buffer, d % 4, misaligned table
+    two = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    assert L.janus_ep_return_rows(FAKE, FAKE, FAKE, 0, 2, 5, 10, 8, two, FAKE, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_ep_return_rows(FAKE, FAKE, FAKE, 0, 2, 4, 10, 8, (ctypes.c_void_p * 2)(FAKE, 0), FAKE,
+                                  null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_ep_return_rows(FAKE, FAKE, FAKE, 0, 2, 4, 10, 6, two, FAKE, null) == J.JANUS_ERR_MISALIGNED
+    assert L.janus_ep_return_rows(FAKE, FAKE, FAKE, 0, 2, 4, 10, 8, two, FAKE + 4, null) == J.JANUS_ERR_MISALIGNED
+    assert L.janus_ep_return_rows(FAKE, FAKE, FAKE, 0, 2, 4, 0, 8, two, null, null) == J.JANUS_OK
     # edge aggregate
     assert L.janus_edge_aggregate(FAKE, null, 10, 8, FAKE, null) == J.JANUS_ERR_INVALID_ARG
     assert L.janus_edge_aggregate(FAKE, FAKE, 10, 10, FAKE, null) == J.JANUS_ERR_MISALIGNED

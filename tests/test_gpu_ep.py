@@ -32,8 +32,10 @@ def _shards(P, N, T, d, seed):
     return out
 
 
-def _ep_pass(shards, gate, K, w1, w2, mode, grads=None):
-    """Forward (and with grads, the input VJP) of the emulated EP layer."""
+def _ep_pass(shards, gate, K, w1, w2, mode, grads=None, fused=False):
+    """Forward (and with grads, the input VJP) of the emulated EP layer.  With
+    fused, each owner's expert MLP stores its output rows straight into the
+    senders' return buffers through the janus_ep_return_rows table."""
     P = len(shards)
     T, E = gate.shape
     El = E // P
@@ -47,18 +49,25 @@ def _ep_pass(shards, gate, K, w1, w2, mode, grads=None):
     for s, (x, t) in enumerate(shards):
         J.janus_ep_dispatch_quant(x, t, T, routes[s], layout, s, payload, rscale)
     recv_off = layout[2]
+    # a rank without atoms still passes a (never written) buffer
+    ret = [torch.full((max(x.shape[0] * K, 1), d), float("nan"), device=DEV) for x, _ in shards]
+    dret = [torch.full((max(x.shape[0] * K, 1), d), float("nan"), device=DEV) for x, _ in shards]
     xd_recv, act_recv, yd_recv = [], [], []
     for o in range(P):
         xr = J.janus_ep_dequant_rows(payload[o], rscale[o], layout, o)
-        yr, ar = J.janus_expert_ffn_fwd(xr, recv_off[o], w1[o * El:(o + 1) * El].contiguous(),
-                                        w2[o * El:(o + 1) * El].contiguous(), mode=mode, want_act=True)
+        w1o, w2o = w1[o * El:(o + 1) * El].contiguous(), w2[o * El:(o + 1) * El].contiguous()
+        if fused:
+            ar = J.janus_expert_ffn_fwd_rows(xr, recv_off[o], w1o, w2o,
+                                             J.janus_ep_return_rows(layout, o, ret, cap, d),
+                                             mode=mode, want_act=True)
+        else:
+            yr, ar = J.janus_expert_ffn_fwd(xr, recv_off[o], w1o, w2o, mode=mode, want_act=True)
+            yd_recv.append(yr)
         xd_recv.append(xr)
         act_recv.append(ar)
-        yd_recv.append(yr)
-    # a rank without atoms still passes a (never written) buffer
-    ret = [torch.full((max(x.shape[0] * K, 1), d), float("nan"), device=DEV) for x, _ in shards]
-    for o in range(P):
-        J.janus_ep_return(yd_recv[o], counts_all, layout, o, ret)
+    if not fused:
+        for o in range(P):
+            J.janus_ep_return(yd_recv[o], counts_all, layout, o, ret)
     ys = [J.janus_combine(ret[s][:shards[s][0].shape[0] * K], routes[s]["slot_of"], K, routes[s]["topk_weight"])
           for s in range(P)]
     if grads is None:
@@ -66,11 +75,15 @@ def _ep_pass(shards, gate, K, w1, w2, mode, grads=None):
     g_recv = [torch.full((cap, d), float("nan"), device=DEV) for _ in range(P)]
     for s in range(P):
         J.janus_ep_dispatch(grads[s], routes[s], layout, s, g_recv, weighted=True)
-    dret = [torch.full((max(x.shape[0] * K, 1), d), float("nan"), device=DEV) for x, _ in shards]
     for o in range(P):
-        dxr = J.janus_expert_ffn_vjp(xd_recv[o], g_recv[o], recv_off[o], w1[o * El:(o + 1) * El].contiguous(),
-                                     w2[o * El:(o + 1) * El].contiguous(), act=act_recv[o], mode=mode)
-        J.janus_ep_return(dxr, counts_all, layout, o, dret)
+        w1o, w2o = w1[o * El:(o + 1) * El].contiguous(), w2[o * El:(o + 1) * El].contiguous()
+        if fused:
+            J.janus_expert_ffn_vjp_rows(xd_recv[o], g_recv[o], recv_off[o], w1o, w2o,
+                                        J.janus_ep_return_rows(layout, o, dret, cap, d),
+                                        act=act_recv[o], mode=mode)
+        else:
+            dxr = J.janus_expert_ffn_vjp(xd_recv[o], g_recv[o], recv_off[o], w1o, w2o, act=act_recv[o], mode=mode)
+            J.janus_ep_return(dxr, counts_all, layout, o, dret)
     dxs = [J.janus_combine(dret[s][:shards[s][0].shape[0] * K], routes[s]["slot_of"], K) for s in range(P)]
     return ys, dxs, routes, layout
 
@@ -128,6 +141,76 @@ def test_ep_forward_and_vjp_equal_local_chains(name, mode):
         gd = oracle.dispatch(host(grads[s]), r["perm"], K, r["topk_weight"])
         dxd = oracle.expert_ffn_vjp(xd, gd, r["offsets"], hw1, hw2)
         assert rel_fro(host(dxs[s]), oracle.combine(dxd, r["slot_of"], K)) <= TOL_FP32
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("name", ["p2_small", "p4_ragged", "p8_s_shape", "p1"])
+def test_fused_return_equals_copy_return(name, mode):
+    # the GEMM epilogue storing through the row table writes the same values
+    # to the same sender rows as the separate return copy: bit-exact
+    P, N, T, E, K, d, h = CASES[name]
+    gate = to_dev(synth.gate_table(T, E, 4))
+    w1, w2 = synth.expert_weights(E, d, h, 5, DEV)
+    shards = _shards(P, N, T, d, 300)
+    grads = [synth.normal((x.shape[0], d), 700 + s, DEV) for s, (x, _) in enumerate(shards)]
+    ys, dxs, _, _ = _ep_pass(shards, gate, K, w1, w2, mode, grads)
+    ys_f, dxs_f, _, _ = _ep_pass(shards, gate, K, w1, w2, mode, grads, fused=True)
+    torch.cuda.synchronize()
+    for s in range(P):
+        assert torch.equal(ys[s], ys_f[s]) and torch.equal(dxs[s], dxs_f[s]), s
+
+
+def test_return_row_table_follows_the_layout():
+    # every received row's address is its sender's row in the sender's local
+    # order (owner row dst_off[s][e] + i <-> sender row src_off[s][e] + i)
+    P, N, T, E, K, d = 4, 120, 9, 12, 3, 36
+    gate = to_dev(synth.gate_table(T, E, 6))
+    shards = _shards(P, N, T, d, 400)
+    routes = [J.janus_route(t, gate, K) for _, t in shards]
+    counts_all = torch.stack([r["counts"] for r in routes]).contiguous()
+    layout = J.janus_ep_layout(counts_all, E)
+    cap = sum(x.shape[0] for x, _ in shards) * K
+    ret = [torch.empty((x.shape[0] * K, d), device=DEV) for x, _ in shards]
+    src_off, dst_off, recv_off = oracle.ep_layout(np.stack([host(r["counts"]) for r in routes]))
+    El = E // P
+    for o in range(P):
+        table = host(J.janus_ep_return_rows(layout, o, ret, cap, d))
+        expect = np.zeros(cap, np.int64)
+        for e in range(o * El, (o + 1) * El):
+            for s in range(P):
+                for i in range(int(src_off[s][e + 1] - src_off[s][e])):
+                    expect[dst_off[s][e] + i] = ret[s].data_ptr() + 4 * d * (int(src_off[s][e]) + i)
+        assert np.array_equal(table, expect), o
+        assert not table[recv_off[o][El]:].any()        # past the received rows: untouched
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_ffn_rows_store_equals_permuted_plain_store(mode):
+    # an arbitrary row table (a permutation into a larger buffer): row p of the
+    # plain output lands at its table address, nothing else is written
+    E, d, h = 7, 132, 68
+    counts = np.array([0, 5, 300, 1, 0, 129, 64])
+    offsets = to_dev(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32))
+    R = int(counts.sum())
+    xd = synth.normal((R, d), 31, DEV)
+    gd = synth.normal((R, d), 32, DEV)
+    w1, w2 = synth.expert_weights(E, d, h, 33, DEV)
+    dest = torch.full((R + 50, d), float("nan"), device=DEV)
+    slot = torch.as_tensor(np.random.default_rng(34).permutation(R + 50)[:R], device=DEV)
+    table = dest.data_ptr() + 4 * d * slot.to(torch.int64)
+    yd, act = J.janus_expert_ffn_fwd(xd, offsets, w1, w2, mode=mode, want_act=True)
+    J.janus_expert_ffn_fwd_rows(xd, offsets, w1, w2, table, mode=mode)
+    torch.cuda.synchronize()
+    assert torch.equal(dest[slot], yd)
+    untouched = torch.ones(R + 50, dtype=torch.bool, device=DEV)
+    untouched[slot] = False
+    assert torch.isnan(dest[untouched]).all()
+    dest.fill_(float("nan"))
+    dxd = J.janus_expert_ffn_vjp(xd, gd, offsets, w1, w2, act=act, mode=mode)
+    J.janus_expert_ffn_vjp_rows(xd, gd, offsets, w1, w2, table, act=act, mode=mode)
+    torch.cuda.synchronize()
+    assert torch.equal(dest[slot], dxd)
+    assert torch.isnan(dest[untouched]).all()
 
 
 def test_ep_send_places_rows_by_the_layout():

@@ -6,7 +6,9 @@ real CUDA IPC mappings of the other process's buffers.
 Both processes share one GPU (each has its own context); the phases are
 ordered by stream synchronisation plus a gloo barrier, and no kernel waits on
 another.  Each rank's forward and input-VJP results must equal its own
-single-GPU chain with all experts local.
+single-GPU chain with all experts local, with the return fused into the
+experts' last GEMM (its epilogue storing into the other process's mapped
+return buffer) and with the separate return copy.
 """
 import os
 import socket
@@ -26,7 +28,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, mode, q):
+def _worker(rank, world, port, mode, fused, q):
     try:
         os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
         sys.path.insert(0, ROOT)
@@ -49,7 +51,8 @@ def _worker(rank, world, port, mode, q):
         types = torch.as_tensor(synth.types_zipf(N, T, seed=20 + rank), device=dev)
         g = synth.normal((N, d), 30 + rank, dev)
         layer = ExpertParallelLayer(400, d, h, T, E, K, w1[rank * El:(rank + 1) * El].contiguous(),
-                                    w2[rank * El:(rank + 1) * El].contiguous(), mode=mode, device=dev)
+                                    w2[rank * El:(rank + 1) * El].contiguous(), mode=mode, device=dev,
+                                    fused_return=fused)
         errs = []
         for _ in range(2):                                  # buffers reused across passes
             y = layer.forward(x, types, gate)
@@ -73,12 +76,13 @@ def _worker(rank, world, port, mode, q):
         q.put((rank, "error", repr(e)))
 
 
+@pytest.mark.parametrize("fused", [True, False])
 @pytest.mark.parametrize("mode", [0, 1])
-def test_ep_layer_two_processes_through_ipc(mode):
+def test_ep_layer_two_processes_through_ipc(mode, fused):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, mode, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, mode, fused, q)) for r in range(2)]
     for p in procs:
         p.start()
     results = [q.get(timeout=300) for _ in range(2)]
