@@ -34,7 +34,9 @@ const char* janus_status_string(janus_status s) {
     case JANUS_ERR_INVALID_ARG: return "JANUS_ERR_INVALID_ARG: null pointer, size/limit violation or workspace too small";
     case JANUS_ERR_MISALIGNED: return "JANUS_ERR_MISALIGNED: feature pointer not 16/8-byte aligned or d % 4 != 0";
     case JANUS_ERR_CUDA: return "JANUS_ERR_CUDA: a CUDA launch or runtime call failed";
-    case JANUS_ERR_DATA: return "JANUS_ERR_DATA: a kernel recorded a data fault (bad type id or non-finite feature)";
+    case JANUS_ERR_DATA:
+      return "JANUS_ERR_DATA: a kernel recorded a data fault (bad type id, non-finite feature, a bounded "
+             "tensor-core wait that ran out, or rows that break JANUS_FFN_X_DEQUANTIZED)";
   }
   return "JANUS_ERR_UNKNOWN";
 }

@@ -85,7 +85,9 @@ namespace {
 // yd_rows (device array of n_rows row pointers) replaces yd when set.
 janus_status ffn_fwd(const float* xd, const int32_t* offsets, int32_t n_experts, int64_t n_rows, int32_t d,
                      int32_t h, const float* w1, const float* w2, float* yd, float* const* yd_rows, float* act,
-                     janus_ffn_mode mode, void* workspace, size_t workspace_bytes, janus_stream_t stream_) {
+                     uint32_t flags, janus_ffn_mode mode, void* workspace, size_t workspace_bytes,
+                     janus_stream_t stream_) {
+  JANUS_CHECK_ARG((flags & ~(uint32_t)JANUS_FFN_X_DEQUANTIZED) == 0);
   cudaStream_t stream = (cudaStream_t)stream_;
   janus_status st = check_ffn(xd, offsets, n_experts, n_rows, d, h, w1, w2,
                               yd_rows ? reinterpret_cast<const float*>(yd_rows) : yd, mode);
@@ -100,7 +102,8 @@ janus_status ffn_fwd(const float* xd, const int32_t* offsets, int32_t n_experts,
   if (mode == JANUS_FFN_3XTF32) {
     JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
     st = tc::expert_ffn_fwd(xd, offsets, n_experts, n_rows, d, h, w1, w2, yd, act, H,
-                            &((WsHeader*)workspace)->error, stream, yd_rows);
+                            &((WsHeader*)workspace)->error, stream, yd_rows,
+                            (flags & JANUS_FFN_X_DEQUANTIZED) != 0);
     if (st != JANUS_OK) return st;
     return launch_status();
   }
@@ -156,7 +159,7 @@ extern "C" janus_status janus_expert_ffn_fwd(const float* xd, const int32_t* off
                                              float* yd, float* act, janus_ffn_mode mode,
                                              void* workspace, size_t workspace_bytes,
                                              janus_stream_t stream) {
-  return ffn_fwd(xd, offsets, n_experts, n_rows, d, h, w1, w2, yd, nullptr, act, mode, workspace,
+  return ffn_fwd(xd, offsets, n_experts, n_rows, d, h, w1, w2, yd, nullptr, act, 0, mode, workspace,
                  workspace_bytes, stream);
 }
 
@@ -167,7 +170,17 @@ extern "C" janus_status janus_expert_ffn_fwd_rows(const float* xd, const int32_t
                                                   void* workspace, size_t workspace_bytes,
                                                   janus_stream_t stream) {
   JANUS_CHECK_ARG(n_rows == 0 || yd_rows);
-  return ffn_fwd(xd, offsets, n_experts, n_rows, d, h, w1, w2, nullptr, yd_rows, act, mode, workspace,
+  return ffn_fwd(xd, offsets, n_experts, n_rows, d, h, w1, w2, nullptr, yd_rows, act, 0, mode, workspace,
+                 workspace_bytes, stream);
+}
+
+extern "C" janus_status janus_expert_ffn_fwd_ex(const float* xd, const int32_t* offsets, int32_t n_experts,
+                                                int64_t n_rows, int32_t d, int32_t h, const float* w1,
+                                                const float* w2, float* yd, float* const* yd_rows, float* act,
+                                                uint32_t flags, janus_ffn_mode mode, void* workspace,
+                                                size_t workspace_bytes, janus_stream_t stream) {
+  JANUS_CHECK_ARG((yd == nullptr) != (yd_rows == nullptr) || n_rows == 0);
+  return ffn_fwd(xd, offsets, n_experts, n_rows, d, h, w1, w2, yd, yd_rows, act, flags, mode, workspace,
                  workspace_bytes, stream);
 }
 

@@ -88,6 +88,7 @@ constexpr uint32_t kStageBytes = 2 * (kTileABytes + kTileBBytes);   // raw + lo
 constexpr uint32_t kTxBytes = kTileABytes + kTileBBytes;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kFaultTimeout = 3;
+constexpr int kFaultNotTf32 = 4;    // kBExact: a B tile held bits below TF32 precision
 constexpr long long kWaitLimitCycles = 4000000000LL;     // ~2 s at 2 GHz
 
 // kEpiD2 (second-order pass, x·W): acc = v W1, aux = a, aux2 = dh;
@@ -485,7 +486,7 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
   if (kEpi == kEpiStore && args.c_rows) __threadfence_system();
 }
 
-template <int kMode, int kEpi>
+template <int kMode, int kEpi, bool kBExact>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, Args args) {
   extern __shared__ uint8_t smem_raw[];
@@ -636,7 +637,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                   bdl = smem_desc(b_lo + kk * 32, 16, 512, kSwizzle64B);
                 }
                 tc_mma_tf32_pair(d_tmem, adl, bdh, idesc, (kb > c0 || kk > 0) ? 1u : 0u);
-                tc_mma_tf32_pair(d_tmem, adh, bdl, idesc, 1u);
+                if (!kBExact) tc_mma_tf32_pair(d_tmem, adh, bdl, idesc, 1u);   // B's residual is zero otherwise
                 tc_mma_tf32_pair(d_tmem, adh, bdh, idesc, 1u);
               }
               tc_commit_pair(&s->empty[st]);
@@ -660,7 +661,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       // warp's latency.  The raw tile itself is the high part (the MMA ignores
       // the 13 low bits of an FP32 operand).
       const int ci = warp < 4 ? warp - 2 : warp - 10;
-      constexpr int kVec = (int)(kTxBytes / 16);
+      // kBExact: only A (the weights) is split; B's rows are exact in TF32 and
+      // are only checked (low 13 bits zero), a violation recorded as a fault
+      constexpr int kVec = (int)((kBExact ? kTileABytes : kTxBytes) / 16);
       constexpr int kBatch = 8;
       static_assert(kVec % (32 * kBatch) == 0, "split batches divide the stage");
       uint32_t it = 0;
@@ -696,6 +699,21 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                   __float_as_uint(__uint_as_float(x[j].y) - __uint_as_float(x[j].y & kTf32Mask)),
                   __float_as_uint(__uint_as_float(x[j].z) - __uint_as_float(x[j].z & kTf32Mask)),
                   __float_as_uint(__uint_as_float(x[j].w) - __uint_as_float(x[j].w & kTf32Mask)));
+          }
+          if (kBExact) {
+            // only the tile's own rows (a K-major row is 4 consecutive 16-byte
+            // chunks: the 64-byte swizzle permutes chunks within a row); the box
+            // may reach rows past the caller's data
+            const uint4* rb = raw + kTileABytes / 16;
+            const int half_rows = c.n_mma / 2;
+            const int vrows = max(0, min(half_rows, c.n_valid - (int)rank * half_rows));
+            uint32_t low = 0;
+#pragma unroll 4
+            for (int i = lane; i < 4 * vrows; i += 32) {
+              const uint4 x = rb[i];
+              low |= (x.x | x.y | x.z | x.w) & ~kTf32Mask;
+            }
+            if (__any_sync(0xffffffffu, low != 0) && lane == 0) atomicCAS(args.err, 0, kFaultNotTf32);
           }
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           __syncwarp();
@@ -784,14 +802,14 @@ constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Smem
 
 // kModeNN/NT: C [R,N] = A [R,Kd] x W_e;  kModeTN: C [E,M,N] with C_e = A_e^T W_e
 // over expert e's rows of A [R,M] and W [R,N] (Kd unused).
-template <int kMode, int kEpi>
+template <int kMode, int kEpi, bool kBExact = false>
 janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, int N, float* C, float* C2,
                     const float* aux, const int32_t* offsets, int32_t* err, cudaStream_t stream, int M = 0,
                     const float* aux2 = nullptr, float* C3 = nullptr, float* const* c_rows = nullptr) {
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(tc_gemm_kernel<kMode, kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr = cudaFuncSetAttribute(tc_gemm_kernel<kMode, kEpi, kBExact>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kSmemBytes);
   });
   if (attr != cudaSuccess) return JANUS_ERR_CUDA;
@@ -818,7 +836,8 @@ janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, in
   cluster_attr[0].val.clusterDim.z = 1;
   cfg.attrs = cluster_attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, tc_gemm_kernel<kMode, kEpi>, ma, mb, a) != cudaSuccess) return JANUS_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, tc_gemm_kernel<kMode, kEpi, kBExact>, ma, mb, a) != cudaSuccess)
+    return JANUS_ERR_CUDA;
   return launch_status();
 }
 
@@ -828,8 +847,10 @@ size_t workspace_extra() { return 0; }
 
 janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, int64_t R, int32_t d,
                             int32_t h, const float* w1, const float* w2, float* yd, float* act, float* H,
-                            int32_t* err, cudaStream_t stream, float* const* yd_rows) {
-  janus_status st = launch<kModeNN, kEpiSilu>(xd, w1, R, E, d, h, H, act, nullptr, offsets, err, stream);
+                            int32_t* err, cudaStream_t stream, float* const* yd_rows, bool x_tf32_exact) {
+  janus_status st = x_tf32_exact
+                        ? launch<kModeNN, kEpiSilu, true>(xd, w1, R, E, d, h, H, act, nullptr, offsets, err, stream)
+                        : launch<kModeNN, kEpiSilu>(xd, w1, R, E, d, h, H, act, nullptr, offsets, err, stream);
   if (st != JANUS_OK) return st;
   return launch<kModeNN, kEpiStore>(H, w2, R, E, h, d, yd, nullptr, nullptr, offsets, err, stream, 0, nullptr,
                                     nullptr, yd_rows);

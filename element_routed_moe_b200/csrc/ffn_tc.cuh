@@ -13,10 +13,13 @@ size_t workspace_extra();
 // `err` is the workspace header's error word (a bounded wait that ran out
 // records a timeout there).
 // yd_rows (nullable): row p of yd is written to yd_rows[p] instead of yd + p d.
+// x_tf32_exact: every xd value is exact in TF32 (dequantized FP16 rows), so the
+// first GEMM drops the product with xd's residual; inexact rows are reported
+// as a data fault.
 janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, int64_t R,
                             int32_t d, int32_t h, const float* w1, const float* w2, float* yd,
                             float* act, float* H, int32_t* err, cudaStream_t stream,
-                            float* const* yd_rows = nullptr);
+                            float* const* yd_rows = nullptr, bool x_tf32_exact = false);
 
 janus_status expert_ffn_vjp(const float* xd, const float* gd, const float* act_in, float* A,
                             const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,

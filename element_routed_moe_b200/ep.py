@@ -165,13 +165,16 @@ class ExpertParallelLayer:
         recv_off = self.layout[2][self.rank]
         m(events, "ffn_fwd", 0)
         J.janus_ep_dequant_rows(self.payload, self.row_scale, self.layout, self.rank, out=self.xd)
+        # the unpacked FP16 rows are exact in TF32: the first GEMM skips their residual
+        flags = J.JANUS_FFN_X_DEQUANTIZED
         if self.fused_return:
             # the table depends only on the layout: the VJP reuses it
             J.janus_ep_return_rows(self.layout, self.rank, self.peer_ret, self.cap, self.d, out=self.ret_rows)
-            J.janus_expert_ffn_fwd_rows(self.xd, recv_off, self.w1, self.w2, self.ret_rows, mode=self.mode,
-                                        act=self.act)
+            J.janus_expert_ffn_fwd_ex(self.xd, recv_off, self.w1, self.w2, out_rows=self.ret_rows, act=self.act,
+                                      flags=flags, mode=self.mode)
         else:
-            J.janus_expert_ffn_fwd(self.xd, recv_off, self.w1, self.w2, mode=self.mode, out=self.yd, act=self.act)
+            J.janus_expert_ffn_fwd_ex(self.xd, recv_off, self.w1, self.w2, out=self.yd, act=self.act, flags=flags,
+                                      mode=self.mode)
         m(events, "ffn_fwd", 1)
         m(events, "return", 0)
         if not self.fused_return:

@@ -35,7 +35,7 @@ SYMBOLS = (
     "janus_quant_by_type_workspace_size", "janus_quant_by_type", "janus_quant_by_type_noalloc",
     "janus_dequant_by_type",
     "janus_expert_ffn_workspace_size", "janus_expert_ffn_fwd", "janus_expert_ffn_vjp",
-    "janus_expert_ffn_fwd_rows", "janus_expert_ffn_vjp_rows",
+    "janus_expert_ffn_fwd_rows", "janus_expert_ffn_vjp_rows", "janus_expert_ffn_fwd_ex",
     "janus_expert_ffn_weight_grad_workspace_size", "janus_expert_ffn_weight_grad",
     "janus_expert_ffn_vjp_vjp_workspace_size", "janus_expert_ffn_vjp_vjp",
     "janus_combine", "janus_edge_aggregate", "janus_edge_broadcast", "janus_neighbor_aggregate",
@@ -103,6 +103,8 @@ def _declare(L):
                                            vp, sz, vp]),
         "janus_expert_ffn_vjp_rows": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp,
                                            ctypes.c_int, vp, sz, vp]),
+        "janus_expert_ffn_fwd_ex": (st, [vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, ctypes.c_uint32,
+                                         ctypes.c_int, vp, sz, vp]),
         "janus_expert_ffn_weight_grad_workspace_size": (st, [i64, i32, i32, psz]),
         "janus_expert_ffn_weight_grad": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp,
                                               ctypes.c_int, vp, sz, vp]),
@@ -550,6 +552,33 @@ def janus_expert_ffn_fwd_rows(xd, offsets, w1, w2, yd_rows, *, mode=JANUS_FFN_FP
                                            int(mode), _p(ws), nb, _stream(stream)),
            "janus_expert_ffn_fwd_rows")
     return act
+
+
+JANUS_FFN_X_DEQUANTIZED = 1
+
+
+def janus_expert_ffn_fwd_ex(xd, offsets, w1, w2, *, out=None, out_rows=None, flags=0, mode=JANUS_FFN_FP32_SIMT,
+                            want_act=False, act=None, workspace=None, stream=None):
+    """The general forward: output rows to `out` (allocated when both out and
+    out_rows are None) or to the addresses in `out_rows`; flags as in the C
+    header (JANUS_FFN_X_DEQUANTIZED).  Returns (out-or-None, act-or-None)."""
+    R, d = xd.shape
+    E, _, h = w1.shape
+    if out is not None and out_rows is not None:
+        raise ValueError("give out or out_rows, not both")
+    if out is None and out_rows is None:
+        out = _empty((R, d), torch.float32, xd.device)
+    if want_act and act is None:
+        act = _empty((R, h), torch.float32, xd.device)
+    nb = janus_expert_ffn_workspace_size(R, d, h, E, False, act is not None, mode)
+    ws = _workspace(nb, xd.device, workspace)
+    _raise(lib().janus_expert_ffn_fwd_ex(_p(xd, torch.float32, "xd"), _p(offsets, torch.int32, "offsets"), E, R, d,
+                                         h, _p(w1, torch.float32, "w1"), _p(w2, torch.float32, "w2"),
+                                         _p(out, torch.float32, "yd"),
+                                         None if out_rows is None else _row_table(out_rows, R),
+                                         _p(act, torch.float32, "act"), int(flags), int(mode), _p(ws), nb,
+                                         _stream(stream)), "janus_expert_ffn_fwd_ex")
+    return out, act
 
 
 def janus_expert_ffn_vjp_rows(xd, gd, offsets, w1, w2, dxd_rows, *, act=None, mode=JANUS_FFN_FP32_SIMT,

@@ -111,8 +111,10 @@ class MoELayer:
             J.janus_dispatch(x, r["slot_of"], K, out=self.xd)
             mark("dispatch", 1)
         mark("ffn_fwd", 0)
-        J.janus_expert_ffn_fwd(self.xd, r["offsets"], self.w1, self.w2, mode=self.mode, out=self.yd,
-                               act=self.act, workspace=self.ffn_ws)
+        # unpacked FP16 rows are exact in TF32: the first GEMM skips their residual
+        J.janus_expert_ffn_fwd_ex(self.xd, r["offsets"], self.w1, self.w2, out=self.yd, act=self.act,
+                                  flags=J.JANUS_FFN_X_DEQUANTIZED if self.packed else 0, mode=self.mode,
+                                  workspace=self.ffn_ws)
         mark("ffn_fwd", 1)
         mark("combine", 0)
         J.janus_combine(self.yd, r["slot_of"], K, r["topk_weight"], out=y)

@@ -32,7 +32,8 @@
  *     as input (perm, slot_of, offsets, row_ptr) must be what janus_route /
  *     a valid CSR would produce; they are not re-validated on the device.
  *   - Data-dependent faults (a type id outside [0,T), a non-finite feature
- *     to be packed) are recorded in the workspace's error word and reported
+ *     to be packed, a bounded tensor-core wait that ran out, rows that break
+ *     JANUS_FFN_X_DEQUANTIZED) are recorded in the workspace's error word and reported
  *     by janus_check(); the call still writes every output (bad type ids are
  *     treated as type 0) so no out-of-bounds access can follow.
  */
@@ -241,6 +242,20 @@ janus_status janus_expert_ffn_fwd_rows(const float* xd, const int32_t* offsets, 
                                        const float* w2, float* const* yd_rows, float* act,
                                        janus_ffn_mode mode, void* workspace, size_t workspace_bytes,
                                        janus_stream_t stream);
+/* The general forward: yd or yd_rows (exactly one non-NULL), and flags.
+ * JANUS_FFN_X_DEQUANTIZED: every xd value is an FP16 value times a power of
+ * two (rows written by janus_dequant_by_type or janus_ep_dequant_rows), hence
+ * exact in TF32; the 3xTF32 first GEMM then skips the product with xd's
+ * residual (two tensor-core products instead of three).  A row that breaks
+ * the promise is reported by janus_check as a data fault (its results then
+ * miss that product).  No effect in JANUS_FFN_FP32_SIMT.  Other flag bits:
+ * JANUS_ERR_INVALID_ARG. */
+#define JANUS_FFN_X_DEQUANTIZED 1u
+janus_status janus_expert_ffn_fwd_ex(const float* xd, const int32_t* offsets, int32_t n_experts,
+                                     int64_t n_rows, int32_t d, int32_t h, const float* w1,
+                                     const float* w2, float* yd, float* const* yd_rows, float* act,
+                                     uint32_t flags, janus_ffn_mode mode, void* workspace,
+                                     size_t workspace_bytes, janus_stream_t stream);
 janus_status janus_expert_ffn_vjp_rows(const float* xd, const float* gd, const float* act,
                                        const int32_t* offsets, int32_t n_experts, int64_t n_rows,
                                        int32_t d, int32_t h, const float* w1, const float* w2,

@@ -1,0 +1,89 @@
+"""The expert MLP forward on dequantized FP16-packed rows (paper review
+'Breaking the Training Barrier of Billion-Parameter Universal Machine Learning
+Interatomic Potentials', section 3.5: atom-type-aware FP16 packing of the
+dispatch).
+
+A dequantized row is an FP16 value times a power-of-two scale, so it is exact
+in TF32 and its 3xTF32 residual is zero.  JANUS_FFN_X_DEQUANTIZED lets the
+first GEMM skip the product with that residual.  Skipping a product that only
+adds zeros leaves every accumulator bit unchanged, so the flagged forward must
+equal the unflagged one bit for bit, and both the oracle within 1e-5.  Rows
+that are not exact in TF32 are reported as a data fault.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from element_routed_moe_b200 import janus as J
+from element_routed_moe_b200 import synth
+from helpers import DEV, TOL_FP32, host, rel_fro, sample_rows, to_dev
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = {
+    # name: (N, T, E, K, d, h)
+    "ragged": (700, 11, 12, 3, 132, 68),
+    "M_like": (4096, 89, 40, 8, 512, 384),
+}
+
+
+def _packed_rows(N, T, E, K, d, seed):
+    types = synth.types_zipf(N, T, seed=seed)
+    gate = synth.gate_table(T, E, seed + 1)
+    x = synth.normal((N, d), seed + 2, DEV)
+    r = J.janus_route(to_dev(types), to_dev(gate), K)
+    payload, scale, _ = J.janus_quant_by_type(x, to_dev(types), T, r["slot_of"], K)
+    xd = J.janus_dequant_by_type(payload, to_dev(types), T, r["perm"], K, scale)
+    return xd, r
+
+
+@pytest.mark.parametrize("mode", [J.JANUS_FFN_FP32_SIMT, J.JANUS_FFN_3XTF32])
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_dequantized_flag_is_bit_identical_and_matches_oracle(name, mode):
+    N, T, E, K, d, h = SHAPES[name]
+    xd, r = _packed_rows(N, T, E, K, d, 40)
+    w1, w2 = synth.expert_weights(E, d, h, 41, DEV)
+    y_plain, a_plain = J.janus_expert_ffn_fwd(xd, r["offsets"], w1, w2, mode=mode, want_act=True)
+    nb = J.janus_expert_ffn_workspace_size(xd.shape[0], d, h, E, False, True, mode)
+    ws = torch.zeros(nb, dtype=torch.uint8, device=DEV)
+    y_flag, a_flag = J.janus_expert_ffn_fwd_ex(xd, r["offsets"], w1, w2, flags=J.JANUS_FFN_X_DEQUANTIZED,
+                                               mode=mode, want_act=True, workspace=ws)
+    J.janus_check(ws)                                   # the rows kept the promise
+    assert torch.equal(y_flag, y_plain) and torch.equal(a_flag, a_plain)
+    offs = host(r["offsets"])
+    rows = sample_rows(offs, 96, seed=3, R=xd.shape[0])
+    ref = oracle.expert_ffn_fwd(host(xd), offs, host(w1), host(w2), rows=rows)
+    assert rel_fro(host(y_flag)[rows], ref) <= TOL_FP32
+
+
+def test_dequantized_flag_into_a_row_table():
+    # the flag combines with the row-table store of the expert-parallel return
+    N, T, E, K, d, h = SHAPES["ragged"]
+    xd, r = _packed_rows(N, T, E, K, d, 50)
+    w1, w2 = synth.expert_weights(E, d, h, 51, DEV)
+    R = xd.shape[0]
+    y_plain, _ = J.janus_expert_ffn_fwd(xd, r["offsets"], w1, w2, mode=J.JANUS_FFN_3XTF32)
+    dest = torch.full((R + 9, d), float("nan"), device=DEV)
+    slot = torch.as_tensor(np.random.default_rng(52).permutation(R + 9)[:R], device=DEV)
+    table = dest.data_ptr() + 4 * d * slot.to(torch.int64)
+    out, _ = J.janus_expert_ffn_fwd_ex(xd, r["offsets"], w1, w2, out_rows=table,
+                                       flags=J.JANUS_FFN_X_DEQUANTIZED, mode=J.JANUS_FFN_3XTF32)
+    torch.cuda.synchronize()
+    assert out is None and torch.equal(dest[slot], y_plain)
+
+
+def test_rows_that_break_the_promise_are_reported():
+    # plain FP32 rows carry bits below TF32 precision: the call still runs, and
+    # janus_check reports the broken promise as a data fault
+    E, d, h = 4, 64, 64
+    offs = to_dev(np.array([0, 100, 100, 250, 300], np.int32))
+    xd = synth.normal((300, d), 60, DEV)
+    w1, w2 = synth.expert_weights(E, d, h, 61, DEV)
+    nb = J.janus_expert_ffn_workspace_size(300, d, h, E, False, False, J.JANUS_FFN_3XTF32)
+    ws = torch.zeros(nb, dtype=torch.uint8, device=DEV)
+    J.janus_expert_ffn_fwd_ex(xd, offs, w1, w2, flags=J.JANUS_FFN_X_DEQUANTIZED, mode=J.JANUS_FFN_3XTF32,
+                              workspace=ws)
+    with pytest.raises(J.JanusError) as e:
+        J.janus_check(ws)
+    assert e.value.status == J.JANUS_ERR_DATA
