@@ -40,6 +40,10 @@
 //   warps 2,3,12..15  splitters, each owning every sixth k-block: write the
 //                landed tile's residual lo = x - hi into a twin buffer (same
 //                swizzled offsets; the landed FP32 tile is read by the MMA as hi);
+//                when the rows are dequantized FP16 values (exact in TF32,
+//                kBExact) only the weights are split, the rows are only
+//                checked, and the product with the rows' zero residual is
+//                not issued;
 //   warps 4..11  epilogue (two warpgroups, one half of the tile each):
 //                tcgen05.ld of each chunk, FP32 running sums in registers
 //                (setmaxnreg: 184 per thread here, 72 elsewhere), then the
