@@ -3,8 +3,9 @@
 One step = one pass of the MoE layer over one synthetic batch:
     route -> dispatch -> expert MLP fwd -> combine            (forward)
     weighted dispatch of dY -> expert MLP VJP -> combine      (input VJP)
-with the interaction-block slice workload also running the edge aggregation
-and the per-element-type FP16 packing (quant -> dequant) in front.
+with the edge aggregation in front where the workload has edges (tiny, L, the
+interaction-block slice) and the per-element-type FP16 packing (quant ->
+dequant) in place of the dispatch where it packs (M, the slice).
 
 Metric: routed atom-expert tokens/s (tokens = N*K routed rows) per layer pass.
 Default workload: MatRIS-MoE(S)-shaped layer (N=8192, T=89 Zipf(1.1), E=72,
@@ -123,7 +124,8 @@ def describe(cfg) -> dict:
         "workload": f"{w}{'' if cfg == synth.CONFIGS[cfg.name] else ' (resized)'}: N={cfg.n_atoms} atoms, T={cfg.n_types} element types "
                     f"({'Zipf(1.1)' if cfg.type_dist == 'zipf' else 'uniform'}), E={cfg.n_experts}, "
                     f"K={cfg.top_k}, d=h={cfg.d}, FP32, fwd+input-VJP"
-                    + (", edge aggregation + FP16 per-type packing" if cfg.name == "slice" else ""),
+                    + (", edge aggregation in front" if cfg.edges != "none" else "")
+                    + (", FP16 per-type packed dispatch" if cfg.quant else ""),
         "n_atoms": cfg.n_atoms, "n_types": cfg.n_types, "n_experts": cfg.n_experts,
         "top_k": cfg.top_k, "d": cfg.d, "h": cfg.h, "routed_tokens": cfg.n_rows,
     }
@@ -226,29 +228,30 @@ class Layer:
         self.J = J
         self.cfg = cfg
         self.mode = mode
-        self.slice = cfg.name == "slice"
-        inp = synth.layer_inputs(cfg, seed=seed, device=dev, with_edges=self.slice)
+        self.edges = cfg.edges != "none"  # the tiny, L and slice configs aggregate edge messages first
+        self.packed = cfg.quant           # the M and slice configs name the FP16-packed dispatch
+        inp = synth.layer_inputs(cfg, seed=seed, device=dev, with_edges=self.edges)
         self.inp = inp
         self.types = torch.as_tensor(inp["types"], device=dev)
         self.gate = torch.as_tensor(inp["gate"], device=dev)
         self.w1, self.w2 = inp["w1"], inp["w2"]
         self.x, self.g = inp["x"], inp["g"]
-        if self.slice:
+        if self.edges:
             self.msg = inp["msg"]
             self.row_ptr = torch.as_tensor(inp["row_ptr"], device=dev)
-        self.core = MoELayer(cfg.n_atoms, cfg.top_k, self.gate, self.w1, self.w2, mode=mode, packed=self.slice,
-                             row_ptr=self.row_ptr if self.slice else None)
+        self.core = MoELayer(cfg.n_atoms, cfg.top_k, self.gate, self.w1, self.w2, mode=mode, packed=self.packed,
+                             row_ptr=self.row_ptr if self.edges else None)
         c = self.core
         self.route_out, self.route_ws = c.route_out, c.route_ws
         self.xd, self.gd, self.act, self.y, self.dx = c.xd, c.gd, c.act, c.y, c.dx
-        if self.slice:
+        if self.edges:
             self.xagg = c.xagg
         self.ops = c.ops
         self.launches_per_step = c.launches_per_call
 
     def step(self, x=None, g=None, types=None, events=None):
         """One layer pass.  events: dict op -> (start, end) CUDA events, or None."""
-        x = (self.msg if self.slice else self.x) if x is None else x
+        x = (self.msg if self.edges else self.x) if x is None else x
         g = self.g if g is None else g
         types = self.types if types is None else types
         return self.core.forward_vjp(x, g, types, events=events)
@@ -266,9 +269,10 @@ class Layer:
             "ffn_vjp": ("flops", 4 * R * d * h),
             "route": ("bytes", 4 * N + 8 * R * 2 + 8 * R),
         }
-        if self.slice:
+        if self.edges:
             Ed = int(self.inp["row_ptr"][-1])
             w["edge_aggregate"] = ("bytes", 4 * Ed * d + 4 * N * d + 8 * (N + 1))
+        if self.packed:
             w["quant"] = ("bytes", 4 * N * d * 2 + 2 * R * d + 4 * R)
             w["dequant"] = ("bytes", 2 * R * d + 4 * R * d + 8 * R)
         return w
@@ -278,17 +282,29 @@ class Layer:
 # CPU oracle timing (the reported CPU baseline; never the product path)
 # --------------------------------------------------------------------------
 def oracle_pass(cfg, host_inp, n: int) -> float:
-    """Wall time of the oracle's layer pass (route, dispatch, FFN fwd,
-    combine, weighted dispatch, FFN VJP, combine) on the first n atoms of the
-    workload, with the full expert weights."""
+    """Wall time of the oracle's layer pass on the first n atoms of the
+    workload, with the full expert weights: the same chain as the GPU step
+    (edge aggregation first where there are edges, FP16 pack and unpack in place of
+    the dispatch where the config packs; route, FFN fwd, combine, weighted
+    dispatch, FFN VJP, combine)."""
     import oracle
     types = host_inp["types"][:n]
     x, g = host_inp["x"][:n], host_inp["g"][:n]
     w1, w2 = host_inp["w1"], host_inp["w2"]
     K = cfg.top_k
+    msg = rp = None
+    if "row_ptr" in host_inp:            # the first n receivers' edge messages (copied before timing)
+        rp = host_inp["row_ptr"][:n + 1]
+        msg = host_inp["msg"][:int(rp[-1])].cpu().numpy()
     t0 = time.perf_counter()
+    if msg is not None:
+        x = oracle.edge_aggregate(msg, rp)
     r = oracle.route(types, host_inp["gate"], K)
-    xd = oracle.dispatch(x, r["perm"], K)
+    if cfg.quant:
+        q, sc = oracle.quant_by_type(x, types, cfg.n_types, r["perm"], K)
+        xd = oracle.dequant_by_type(q, types, r["perm"], K, sc)
+    else:
+        xd = oracle.dispatch(x, r["perm"], K)
     yd = oracle.expert_ffn_fwd(xd, r["offsets"], w1, w2)
     oracle.combine(yd, r["slot_of"], K, r["topk_weight"])
     gd = oracle.dispatch(g, r["perm"], K, r["topk_weight"])
@@ -298,19 +314,24 @@ def oracle_pass(cfg, host_inp, n: int) -> float:
 
 
 def oracle_calibrate(cfg, host_inp, target_s: float) -> int:
-    """Number of atoms whose oracle pass takes about target_s seconds."""
-    n = 4
+    """Number of atoms whose oracle pass takes about target_s seconds (at
+    most host_inp["max_atoms"] when given)."""
+    n_max = int(host_inp.get("max_atoms", cfg.n_atoms))
+    n = min(4, n_max)
     dt = oracle_pass(cfg, host_inp, n)
-    while dt < 0.1 * target_s and n < cfg.n_atoms:
-        n = min(cfg.n_atoms, n * 4)
+    while dt < 0.1 * target_s and n < n_max:
+        n = min(n_max, n * 4)
         dt = oracle_pass(cfg, host_inp, n)
-    return int(min(cfg.n_atoms, max(1, n * target_s / max(dt, 1e-6))))
+    return int(min(n_max, max(1, n * target_s / max(dt, 1e-6))))
 
 
 def host_inputs(cfg, layer):
-    return dict(types=np.asarray(layer.inp["types"]), gate=np.asarray(layer.inp["gate"]),
-                x=layer.x.cpu().numpy(), g=layer.g.cpu().numpy(),
-                w1=layer.w1.cpu().numpy(), w2=layer.w2.cpu().numpy())
+    h = dict(types=np.asarray(layer.inp["types"]), gate=np.asarray(layer.inp["gate"]),
+             x=layer.x.cpu().numpy(), g=layer.g.cpu().numpy(),
+             w1=layer.w1.cpu().numpy(), w2=layer.w2.cpu().numpy())
+    if layer.edges:   # the messages stay on the device; a sample's rows are copied when timed
+        h.update(row_ptr=np.asarray(layer.inp["row_ptr"]), msg=layer.msg)
+    return h
 
 
 def cpu_descr():
@@ -334,6 +355,15 @@ def run_reference(args, world, rank):
     inp = synth.layer_inputs(cfg, seed=args.seed, device="cpu", with_edges=False)
     host = dict(types=inp["types"], gate=inp["gate"], x=inp["x"].numpy(), g=inp["g"].numpy(),
                 w1=inp["w1"].numpy(), w2=inp["w2"].numpy())
+    if cfg.edges != "none":
+        # the same receiver-sorted CSR as the GPU arm; messages only for the
+        # first atoms the sample can reach (the full tensor is 9-29 GB)
+        if cfg.edges == "random":
+            rp, _, _ = synth.edges_random(cfg.n_atoms, cfg.edges_per_atom, args.seed + 6)
+        else:
+            rp, _, _ = synth.edges_pbc(cfg.n_atoms, args.seed + 6)
+        cap = min(cfg.n_atoms, 2048)
+        host.update(row_ptr=rp, msg=synth.normal((int(rp[cap]), cfg.d), args.seed + 8), max_atoms=cap)
     per_step = args.ref_seconds or max(2.0, min(15.0, 150.0 / max(1, args.steps + args.warmup)))
     n_s = oracle_calibrate(cfg, host, per_step)
     times = []
@@ -442,7 +472,7 @@ def run_janus(args, world, rank, local):
         "clocks": clocks,
     }
 
-    if not args.no_e2e and not layer.slice:
+    if not args.no_e2e and not layer.edges:   # host-side edge messages would be 9-29 GB per step
         line["e2e"] = run_e2e(layer, args)
     if not args.no_extras:
         line["extras"] = run_extras(layer, peaks)
@@ -557,7 +587,7 @@ def _time_ms(fn, reps=5):
 def run_extras(layer, peaks):
     """Calls outside the layer pass, timed separately (not part of `value`):
     expert weight gradients, routing of 12 MoE layers at once vs one by one,
-    and (slice workload) the edge-side gradient and sender-indexed gather."""
+    and (workloads with edges) the edge-side gradient and sender-indexed gather."""
     J = layer.J
     cfg = layer.cfg
     N, R, d, h, E, K, T = cfg.n_atoms, cfg.n_rows, cfg.d, cfg.h, cfg.n_experts, cfg.top_k, cfg.n_types
@@ -591,7 +621,7 @@ def run_extras(layer, peaks):
     ms_single = _time_ms(lambda: [J.janus_route(layer.types, gates[l], K, out=r, workspace=layer.route_ws)
                                   for l in range(L)])
     out["route_12_layers"] = {"ms_one_call": ms_layers, "ms_12_calls": ms_single}
-    if layer.slice:
+    if layer.edges:
         Ed = int(layer.inp["row_ptr"][-1])
         dmsg = torch.empty_like(layer.msg)
         ms_b = _time_ms(lambda: J.janus_edge_broadcast(layer.dx, layer.row_ptr, out=dmsg), reps=3)
