@@ -394,8 +394,11 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader(&s->chunk_empty[p], rank);
-      if (kMode != kModeTN && (kEpi == kEpiDSilu || kEpi == kEpiD2) && c0 == 0) {
-        // the tile's pre-activations travel to L2 while its chunks accumulate
+      // the tile's pre-activations travel to L2 while its last two chunks
+      // accumulate (late enough that they are still there for the store
+      // phase: 1-3 % faster than prefetching at the first chunk)
+      const int pf_c0 = max(0, ((c.nk - 1) / kChunkKb - 1) * kChunkKb);
+      if (kMode != kModeTN && (kEpi == kEpiDSilu || kEpi == kEpiD2) && c0 == pf_c0) {
         const int f = c.m0 + q * 32 + lane;
         const int jn = min(kEpiCols, c.n_valid - half * kEpiCols);
         if (f < c.m_end) {
