@@ -102,8 +102,9 @@ enum Epilogue : int { kEpiStore = 0, kEpiSilu = 1, kEpiDSilu = 2, kEpiD2 = 3, kE
 
 // Operand layouts:  kModeNN  C = X W       (W stored [E][Kd][N])
 //                   kModeNT  C = X W^T     (W stored [E][N][Kd])
-//                   kModeTN  C_e = X_e^T Y_e per expert (weight gradient; both
-//                            operands MN-major, K = the expert's row segment)
+//                   kModeTN  C_e = (X_e^T Y_e)^T = Y_e^T X_e per expert (weight
+//                            gradient; both operands MN-major, K = the expert's
+//                            row segment; the X^T Y product is stored transposed)
 // NN and NT run with the operands swapped (C^T = W^T X^T): the MMA's M is the
 // output feature (256 per CTA pair: the weights fill it without padding) and
 // its N is the expert's rows, chosen per tile as the valid rows rounded up to
@@ -119,7 +120,7 @@ struct Args {
   float* const* c_rows;   // NN/NT plain store: if set, row p goes to c_rows[p] (e.g. a peer's buffer)
   const int32_t* offsets;
   int E, Kd, N;
-  int M;            // kModeTN: rows of each expert's output (C is [E][M][N])
+  int M;            // kModeTN: MMA rows of each expert's product; C is [E][N][M] (stored transposed)
   int32_t* err;
 };
 
@@ -468,23 +469,28 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
       }
       continue;
     }
-    // weight gradient (plain store): TMEM lane = output row, columns along it
+    // weight gradient: TMEM lane = MMA row i (< M), column = j (< N).  The
+    // product is stored transposed, C[e][j][i], so the 32 lanes of a warp
+    // write 32 consecutive floats (one 128-byte segment) of one output row per
+    // instruction; row-per-lane float4 stores touched 32 rows per instruction
+    // and bound the short-K tiles of small experts.
     static_assert(kMode != kModeTN || kEpi == kEpiStore || kEpi == kEpiAccum,
                   "the weight-gradient GEMM has no fused activation");
     const int row = c.m0 + q * 32 + lane;
     const int colb = c.n0 + half * kEpiCols;
     if (row < c.m_end && colb < N) {
-      const int64_t o = (int64_t)c.e * args.M * N + (int64_t)row * N + colb;
+      float* base = args.C + (int64_t)c.e * args.M * N + (int64_t)colb * args.M + row;
+      constexpr int kB = 8;
 #pragma unroll
-      for (int j = 0; j < kEpiCols; j += 4) {
-        if (colb + j < N) {
-          float4 v = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-          if (kEpi == kEpiAccum) {
-            const float4 old = *reinterpret_cast<const float4*>(args.C + o + j);
-            v = make_float4(old.x + v.x, old.y + v.y, old.z + v.z, old.w + v.w);
-          }
-          *reinterpret_cast<float4*>(args.C + o + j) = v;
+      for (int jb = 0; jb < kEpiCols; jb += kB) {
+        float old[kB];
+        if (kEpi == kEpiAccum) {
+#pragma unroll
+          for (int j = 0; j < kB; ++j) old[j] = colb + jb + j < N ? base[(int64_t)(jb + j) * args.M] : 0.f;
         }
+#pragma unroll
+        for (int j = 0; j < kB; ++j)
+          if (colb + jb + j < N) base[(int64_t)(jb + j) * args.M] = kEpi == kEpiAccum ? old[j] + acc[jb + j] : acc[jb + j];
       }
     }
   }
@@ -807,8 +813,9 @@ bool map_rows_mn(CUtensorMap* m, const float* X, int64_t R, int cols) {
 
 constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Smem);
 
-// kModeNN/NT: C [R,N] = A [R,Kd] x W_e;  kModeTN: C [E,M,N] with C_e = A_e^T W_e
-// over expert e's rows of A [R,M] and W [R,N] (Kd unused).
+// kModeNN/NT: C [R,N] = A [R,Kd] x W_e;  kModeTN: C [E,N,M] with C_e = W_e^T A_e
+// (the product A_e^T W_e stored transposed) over expert e's rows of A [R,M] and
+// W [R,N] (Kd unused).
 template <int kMode, int kEpi, bool kBExact = false>
 janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, int N, float* C, float* C2,
                     const float* aux, const int32_t* offsets, int32_t* err, cudaStream_t stream, int M = 0,
@@ -890,9 +897,11 @@ janus_status expert_ffn_weight_grad(const float* xd, const float* gd, const floa
   // dA = (gd W2^T) * silu'(a), and H = silu(a)
   st = launch<kModeNT, kEpiDSilu>(gd, w2, R, E, d, h, dA, H, A, offsets, err, stream);
   if (st != JANUS_OK) return st;
-  st = launch<kModeTN, kEpiStore>(xd, dA, R, E, 0, h, dw1, nullptr, nullptr, offsets, err, stream, d);
+  // dW1 = xd^T dA [d][h]: the product dA^T xd, stored transposed
+  st = launch<kModeTN, kEpiStore>(dA, xd, R, E, 0, d, dw1, nullptr, nullptr, offsets, err, stream, h);
   if (st != JANUS_OK) return st;
-  return launch<kModeTN, kEpiStore>(H, gd, R, E, 0, d, dw2, nullptr, nullptr, offsets, err, stream, h);
+  // dW2 = H^T gd [h][d]
+  return launch<kModeTN, kEpiStore>(gd, H, R, E, 0, h, dw2, nullptr, nullptr, offsets, err, stream, d);
 }
 
 janus_status expert_ffn_vjp_vjp(const float* xd, const float* gd, const float* vd, const float* act_in, float* A,
@@ -917,11 +926,13 @@ janus_status expert_ffn_vjp_vjp(const float* xd, const float* gd, const float* v
   st = launch<kModeNT, kEpiStore>(t2, w1, R, E, h, d, d_xd, nullptr, nullptr, offsets, err, stream);
   if (st != JANUS_OK || !dw1) return st;
   // dW2 = t1^T gd;  dW1 = vd^T u + xd^T t2
-  st = launch<kModeTN, kEpiStore>(t1, gd, R, E, 0, d, dw2, nullptr, nullptr, offsets, err, stream, h);
+  // (each product stored transposed: the first operand's columns index the
+  // output's columns)
+  st = launch<kModeTN, kEpiStore>(gd, t1, R, E, 0, h, dw2, nullptr, nullptr, offsets, err, stream, d);
   if (st != JANUS_OK) return st;
-  st = launch<kModeTN, kEpiStore>(vd, u, R, E, 0, h, dw1, nullptr, nullptr, offsets, err, stream, d);
+  st = launch<kModeTN, kEpiStore>(u, vd, R, E, 0, d, dw1, nullptr, nullptr, offsets, err, stream, h);
   if (st != JANUS_OK) return st;
-  return launch<kModeTN, kEpiAccum>(xd, t2, R, E, 0, h, dw1, nullptr, nullptr, offsets, err, stream, d);
+  return launch<kModeTN, kEpiAccum>(t2, xd, R, E, 0, d, dw1, nullptr, nullptr, offsets, err, stream, h);
 }
 
 }  // namespace tc
