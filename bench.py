@@ -121,7 +121,8 @@ def describe(cfg) -> dict:
     w = {"tiny": "tiny layer", "S": "MatRIS-MoE(S)-shaped layer", "M": "MatRIS-MoE(M)-shaped layer",
          "L": "MatRIS-MoE(L)-shaped layer", "slice": "interaction-block slice at M shape"}[cfg.name]
     return {
-        "workload": f"{w}{'' if cfg == synth.CONFIGS[cfg.name] else ' (resized)'}: N={cfg.n_atoms} atoms, T={cfg.n_types} element types "
+        "workload": f"{w}{'' if cfg == synth.CONFIGS[cfg.name] else ' (resized)'}: "
+                    f"N={cfg.n_atoms} atoms, T={cfg.n_types} element types "
                     f"({'Zipf(1.1)' if cfg.type_dist == 'zipf' else 'uniform'}), E={cfg.n_experts}, "
                     f"K={cfg.top_k}, d=h={cfg.d}, FP32, fwd+input-VJP"
                     + (", edge aggregation in front" if cfg.edges != "none" else "")

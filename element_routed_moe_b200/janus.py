@@ -40,7 +40,8 @@ SYMBOLS = (
     "janus_expert_ffn_vjp_vjp_workspace_size", "janus_expert_ffn_vjp_vjp",
     "janus_combine", "janus_edge_aggregate", "janus_edge_broadcast", "janus_neighbor_aggregate",
     "janus_ep_layout", "janus_ep_dispatch_quant", "janus_ep_dispatch", "janus_ep_dequant_rows",
-    "janus_ep_return", "janus_ep_return_rows", "janus_ipc_get_handle", "janus_ipc_open_handle", "janus_ipc_close_handle",
+    "janus_ep_return", "janus_ep_return_rows",
+    "janus_ipc_get_handle", "janus_ipc_open_handle", "janus_ipc_close_handle",
     "janus_debug_inject_launch_failures",
 )
 
@@ -538,7 +539,8 @@ def _row_table(rows, R):
 def janus_expert_ffn_fwd_rows(xd, offsets, w1, w2, yd_rows, *, mode=JANUS_FFN_FP32_SIMT, want_act=False,
                               act=None, workspace=None, stream=None):
     """janus_expert_ffn_fwd with output row p stored at address yd_rows[p]
-    (int64 device tensor); returns act-or-None."""
+    (int64 device tensor of 16-byte aligned device addresses with room for d
+    floats each, e.g. from janus_ep_return_rows); returns act-or-None."""
     R, d = xd.shape
     E, _, h = w1.shape
     if want_act and act is None:
