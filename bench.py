@@ -276,6 +276,7 @@ class Layer:
         if self.packed:
             w["quant"] = ("bytes", 4 * N * d * 2 + 2 * R * d + 4 * R)
             w["dequant"] = ("bytes", 2 * R * d + 4 * R * d + 8 * R)
+            w["row_scales"] = ("bytes", 12 * R)      # perm + the row's type + the scale written
         return w
 
 
@@ -594,6 +595,10 @@ def run_extras(layer, peaks):
     N, R, d, h, E, K, T = cfg.n_atoms, cfg.n_rows, cfg.d, cfg.h, cfg.n_experts, cfg.top_k, cfg.n_types
     r = layer.route_out
     out = {}
+    if layer.core.packed and layer.core.fused_unpack:
+        # the step never writes xd (its first GEMM reads the FP16 rows): the
+        # weight-gradient extras need the unpacked rows, written here untimed
+        J.janus_dequant_by_type(layer.core.payload, layer.types, T, r["perm"], K, layer.core.scale, out=layer.xd)
     dw1 = torch.empty_like(layer.w1)
     dw2 = torch.empty_like(layer.w2)
     ws = torch.empty(J.janus_expert_ffn_weight_grad_workspace_size(R, h, True), dtype=torch.uint8,

@@ -16,6 +16,10 @@
 //   G4: dxd = dA W1[e]^T
 // Weight gradients (G3 also writes H = silu(a)):
 //   G5: dW1[e] = Xd_e^T dA_e,  G6: dW2[e] = H_e^T Gd_e  (sums over expert e's rows)
+#include <cuda_fp16.h>
+
+#include <algorithm>
+
 #include "common.cuh"
 #include "ffn_simt.cuh"
 #include "ffn_tc.cuh"
@@ -65,10 +69,83 @@ simt::Args make_args(const float* A, const float* B, int64_t bstride, float* C, 
   return a;
 }
 
+// xd[p,:] = f32(payload[p,:]) * row_scale[p]: one warp per row, four values
+// (8 bytes in, 16 out) per lane and step.  The SIMT path of the packed forward.
+__global__ void __launch_bounds__(256)
+unpack_rows_kernel(const uint2* __restrict__ payload, const float* __restrict__ row_scale, int64_t R, int d4,
+                   float4* __restrict__ xd) {
+  const int lane = threadIdx.x % 32;
+  const int64_t nw = (int64_t)gridDim.x * (blockDim.x / 32);
+  for (int64_t p = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32; p < R; p += nw) {
+    const float sc = __ldg(row_scale + p);
+    for (int c = lane; c < d4; c += 32) {
+      const uint2 q = __ldcs(payload + p * d4 + c);
+      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&q.x));
+      const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&q.y));
+      xd[p * d4 + c] = make_float4(a.x * sc, a.y * sc, b.x * sc, b.y * sc);
+    }
+  }
+}
+
+size_t packed_extra(int64_t R, int32_t d, janus_ffn_mode mode) {
+  return mode == JANUS_FFN_FP32_SIMT ? align_up(sizeof(float) * (size_t)R * (size_t)d, 256) : 0;
+}
+
 }  // namespace
 }  // namespace janus
 
 using namespace janus;
+
+extern "C" janus_status janus_expert_ffn_packed_workspace_size(int64_t n_rows, int32_t d, int32_t h,
+                                                               janus_ffn_mode mode, size_t* bytes) {
+  JANUS_CHECK_ARG(bytes && n_rows >= 0 && d >= 1 && h >= 1);
+  JANUS_CHECK_ARG(mode == JANUS_FFN_FP32_SIMT || mode == JANUS_FFN_3XTF32);
+  *bytes = ffn_layout(n_rows, h, false, true).total + packed_extra(n_rows, d, mode);
+  return JANUS_OK;
+}
+
+extern "C" janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, const float* row_scale,
+                                                    const int32_t* offsets, int32_t n_experts, int64_t n_rows,
+                                                    int32_t d, int32_t h, const float* w1, const float* w2,
+                                                    float* yd, float* const* yd_rows, float* act,
+                                                    janus_ffn_mode mode, void* workspace, size_t workspace_bytes,
+                                                    janus_stream_t stream_) {
+  cudaStream_t stream = (cudaStream_t)stream_;
+  JANUS_CHECK_ARG((yd == nullptr) != (yd_rows == nullptr) || n_rows == 0);
+  const float* outp = yd_rows ? reinterpret_cast<const float*>(yd_rows) : yd;
+  // check_ffn validates the shapes, weights and output; the payload is checked here
+  janus_status st = check_ffn(reinterpret_cast<const float*>(payload), offsets, n_experts, n_rows, d, h, w1, w2,
+                              outp, mode);
+  if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(n_rows == 0 || row_scale);
+  JANUS_CHECK_ALIGN(mode != JANUS_FFN_3XTF32 || d % 8 == 0);   // FP16 rows: 16-byte TMA strides
+  JANUS_CHECK_ALIGN(act == nullptr || aligned(act, 16));
+  const FfnLayout L = ffn_layout(n_rows, h, false, true);
+  const size_t extra = packed_extra(n_rows, d, mode);
+  JANUS_CHECK_ARG(workspace && workspace_bytes >= L.total + extra);
+  JANUS_CHECK_ALIGN(aligned(workspace, 256));
+  if (n_rows == 0) return JANUS_OK;
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  float* H = (float*)((char*)workspace + L.off_h);
+  if (mode == JANUS_FFN_3XTF32) {
+    JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
+    st = tc::expert_ffn_fwd_packed(payload, row_scale, offsets, n_experts, n_rows, d, h, w1, w2, yd, act, H,
+                                   &((WsHeader*)workspace)->error, stream, yd_rows);
+    if (st != JANUS_OK) return st;
+    return launch_status();
+  }
+  // FP32 SIMT: unpack into the workspace, then the plain forward
+  float* xd = (float*)((char*)workspace + L.total);
+  const int64_t blocks = std::min<int64_t>((n_rows + 7) / 8, (int64_t)num_sms() * 8);
+  unpack_rows_kernel<<<(unsigned)blocks, 256, 0, stream>>>((const uint2*)payload, row_scale, n_rows, d / 4,
+                                                         (float4*)xd);
+  const int64_t sw = (int64_t)d * h;
+  launch_simt<false, simt::kEpiSilu>(make_args(xd, w1, sw, H, act, nullptr, offsets, n_experts, d, h), stream);
+  simt::Args a2 = make_args(H, w2, sw, yd, nullptr, nullptr, offsets, n_experts, h, d);
+  a2.c_rows = yd_rows;
+  launch_simt<false, simt::kEpiStore>(a2, stream);
+  return launch_status();
+}
 
 extern "C" janus_status janus_expert_ffn_workspace_size(int64_t n_rows, int32_t d, int32_t h,
                                                         int32_t n_experts, int32_t vjp,

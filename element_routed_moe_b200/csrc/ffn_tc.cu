@@ -57,6 +57,7 @@
 // issued MMAs and loads are drained (bounded) and TMEM is freed.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_fp16.h>
 
 #include <mutex>
 
@@ -111,6 +112,17 @@ enum Epilogue : int { kEpiStore = 0, kEpiSilu = 1, kEpiDSilu = 2, kEpiD2 = 3, kE
 // 32, so a small expert wastes at most 31 rows instead of up to 255.
 enum Mode : int { kModeNN = 0, kModeNT = 1, kModeTN = 2 };
 
+// What the B tile (the dispatch rows, kModeNN) holds:
+//   kBSplit   FP32 rows, split into hi and lo by the splitters (3 products);
+//   kBExact   FP32 rows exact in TF32 (dequantized FP16): no lo, 2 products,
+//             the splitters only check the rows;
+//   kBHalf    the FP16 payload itself plus a per-row power-of-two scale: TMA
+//             lands the FP16 tile in the (unused) lo slot of B and the
+//             splitters write the FP32 rows, f32(q) * scale, into the B tile
+//             (exact, so again 2 products).  The unpack is fused into the GEMM.
+enum BKind : int { kBSplit = 0, kBExact = 1, kBHalf = 2 };
+constexpr uint32_t kTileBHalfBytes = BNH * BK * 2;       // 4 KB of FP16 rows per CTA
+
 struct Args {
   float* C;
   float* C2;
@@ -118,6 +130,8 @@ struct Args {
   const float* aux;
   const float* aux2;
   float* const* c_rows;   // NN/NT plain store: if set, row p goes to c_rows[p] (e.g. a peer's buffer)
+  const float* row_scale; // kBHalf: scale of dispatch row p
+  int64_t rows;           // kBHalf: rows of the payload (row_scale's length)
   const int32_t* offsets;
   int E, Kd, N;
   int M;            // kModeTN: MMA rows of each expert's product; C is [E][N][M] (stored transposed)
@@ -135,6 +149,7 @@ struct Smem {
   int abort;
   int off[kMaxExperts + 1];
   int start[kMaxExperts + 1];
+  float rscale[kNumSplitWarps][BNH];   // kBHalf: each splitter warp's row scales for its current tile
 };
 
 // ---- PTX wrappers ---------------------------------------------------------
@@ -499,7 +514,7 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
   if (kEpi == kEpiStore && args.c_rows) __threadfence_system();
 }
 
-template <int kMode, int kEpi, bool kBExact>
+template <int kMode, int kEpi, int kBK>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, Args args) {
   extern __shared__ uint8_t smem_raw[];
@@ -570,7 +585,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
             const uint32_t st = it % kStages, use = it / kStages;
             if (!mbar_wait(s, &s->empty[st], (use & 1) ^ 1, args.err)) { ok = false; break; }
             uint8_t* base = tiles + st * kStageBytes;
-            mbar_arrive_expect_tx(&s->full[st], kTxBytes);
+            mbar_arrive_expect_tx(&s->full[st], kBK == kBHalf ? kTileABytes + kTileBHalfBytes : kTxBytes);
             if (kMode == kModeTN) {
               // both operands MN-major: 32-column boxes of 16 segment rows
               const int row = c.k_row0 + kb * BK;
@@ -589,8 +604,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                 for (int j = 0; j < BM / 32; ++j)
                   tma_load_3d(&mapA, &s->full[st], base + j * (32 * BK * 4), c.m0 + 32 * j, kb * BK, c.e);
               }
-              // B: this CTA's half of the tile's dispatch rows (n_mma / 2 of them)
-              tma_load_2d(&mapB, &s->full[st], base + kTileABytes, kb * BK, c.n0 + (int)rank * (c.n_mma / 2));
+              // B: this CTA's half of the tile's dispatch rows (n_mma / 2 of them);
+              // FP16 rows land in B's lo slot, for the splitters to unpack
+              tma_load_2d(&mapB, &s->full[st], base + (kBK == kBHalf ? kTxBytes + kTileABytes : kTileABytes),
+                          kb * BK, c.n0 + (int)rank * (c.n_mma / 2));
             }
           }
         }
@@ -650,7 +667,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                   bdl = smem_desc(b_lo + kk * 32, 16, 512, kSwizzle64B);
                 }
                 tc_mma_tf32_pair(d_tmem, adl, bdh, idesc, (kb > c0 || kk > 0) ? 1u : 0u);
-                if (!kBExact) tc_mma_tf32_pair(d_tmem, adh, bdl, idesc, 1u);   // B's residual is zero otherwise
+                if (kBK == kBSplit) tc_mma_tf32_pair(d_tmem, adh, bdl, idesc, 1u);   // B's residual is zero otherwise
                 tc_mma_tf32_pair(d_tmem, adh, bdh, idesc, 1u);
               }
               tc_commit_pair(&s->empty[st]);
@@ -675,16 +692,30 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       // the 13 low bits of an FP32 operand).
       const int ci = warp < 4 ? warp - 2 : warp - 10;
       // kBExact: only A (the weights) is split; B's rows are exact in TF32 and
-      // are only checked (low 13 bits zero), a violation recorded as a fault
-      constexpr int kVec = (int)((kBExact ? kTileABytes : kTxBytes) / 16);
+      // are only checked (low 13 bits zero), a violation recorded as a fault.
+      // kBHalf: only A is split; B's FP16 rows are unpacked into the B tile.
+      constexpr int kVec = (int)((kBK != kBSplit ? kTileABytes : kTxBytes) / 16);
       constexpr int kBatch = 8;
       static_assert(kVec % (32 * kBatch) == 0, "split batches divide the stage");
       uint32_t it = 0;
       bool ok = true;
+      int scaled_tile = -1;    // kBHalf: the tile whose row scales this warp holds
       for (int tile = blockIdx.x / 2; tile < total && ok; tile += n_pairs) {
         const TileCoord c = decode_tile<kMode>(s, args, n_tiles_n, nk, tile, rank);
         for (int kb = 0; kb < c.nk; ++kb, ++it) {
           if ((int)(it % kNumSplitWarps) != ci) continue;
+          if (kBK == kBHalf && scaled_tile != tile) {
+            // this CTA's B rows of the tile: row0 .. row0 + 127 (past the
+            // payload: scale 0, the TMA fill is 0 too)
+            const int64_t row0 = (int64_t)c.n0 + (int64_t)rank * (c.n_mma / 2);
+#pragma unroll
+            for (int i = lane; i < BNH; i += 32) {
+              const int64_t p = row0 + i;
+              s->rscale[ci][i] = p < args.rows ? __ldg(args.row_scale + p) : 0.f;
+            }
+            __syncwarp();
+            scaled_tile = tile;
+          }
           // kModeTN: rows past the expert's segment belong to the next expert
           const int k_valid = kMode == kModeTN ? c.k_rows - kb * BK : BK;
           const uint32_t st = it % kStages, use = it / kStages;
@@ -713,7 +744,24 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                   __float_as_uint(__uint_as_float(x[j].z) - __uint_as_float(x[j].z & kTf32Mask)),
                   __float_as_uint(__uint_as_float(x[j].w) - __uint_as_float(x[j].w & kTf32Mask)));
           }
-          if (kBExact) {
+          if (kBK == kBHalf) {
+            // FP16 tile [128 rows][16] (32 bytes a row, no swizzle) -> FP32 B
+            // tile in the 64-byte swizzle TMA would have written: 16-byte chunk
+            // c of row r sits at chunk c ^ ((r >> 1) & 3) of the row
+            const uint2* hs = reinterpret_cast<const uint2*>(tiles + st * kStageBytes + kTxBytes + kTileABytes);
+            float4* rbw = reinterpret_cast<float4*>(tiles + st * kStageBytes + kTileABytes);
+            const float* rs = s->rscale[ci];
+#pragma unroll 4
+            for (int i = lane; i < BNH * 4; i += 32) {
+              const int r = i >> 2, cc = i & 3;
+              const uint2 h = hs[i];
+              const float sc = rs[r];
+              const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
+              const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
+              rbw[r * 4 + (cc ^ ((r >> 1) & 3))] = make_float4(f0.x * sc, f0.y * sc, f1.x * sc, f1.y * sc);
+            }
+          }
+          if (kBK == kBExact) {
             // only the tile's own rows (a K-major row is 4 consecutive 16-byte
             // chunks: the 64-byte swizzle permutes chunks within a row); the box
             // may reach rows past the caller's data
@@ -774,6 +822,20 @@ bool map_a(CUtensorMap* m, const float* A, int64_t R, int Kd) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A of the FP16-row forward: the payload [R, Kd] FP16, box 16 (k) x 128 (rows),
+// no swizzle (32-byte rows; the splitters unpack them)
+bool map_a_half(CUtensorMap* m, const uint16_t* A, int64_t R, int Kd) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)Kd, (cuuint64_t)R};
+  cuuint64_t strides[1] = {(cuuint64_t)Kd * 2};
+  cuuint32_t box[2] = {BK, BM};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void*)A, dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // B for "x W": W [E, Kd, N] (N contiguous), box 32 (n) x 16 (k) x 1, 128-byte
 //   swizzle with 32-byte atoms (MN-major); 4 boxes per CTA and k-block
 // B for "x W^T": W [E, N, Kd] (Kd contiguous), box 16 (k) x 128 (n) x 1, 64-byte swizzle
@@ -816,26 +878,30 @@ constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Smem
 // kModeNN/NT: C [R,N] = A [R,Kd] x W_e;  kModeTN: C [E,N,M] with C_e = W_e^T A_e
 // (the product A_e^T W_e stored transposed) over expert e's rows of A [R,M] and
 // W [R,N] (Kd unused).
-template <int kMode, int kEpi, bool kBExact = false>
+template <int kMode, int kEpi, int kBK = kBSplit>
 janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, int N, float* C, float* C2,
                     const float* aux, const int32_t* offsets, int32_t* err, cudaStream_t stream, int M = 0,
-                    const float* aux2 = nullptr, float* C3 = nullptr, float* const* c_rows = nullptr) {
+                    const float* aux2 = nullptr, float* C3 = nullptr, float* const* c_rows = nullptr,
+                    const float* row_scale = nullptr) {
+  static_assert(kBK == kBSplit || kMode == kModeNN, "exact or FP16 rows: the forward layout only");
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(tc_gemm_kernel<kMode, kEpi, kBExact>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr = cudaFuncSetAttribute(tc_gemm_kernel<kMode, kEpi, kBK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kSmemBytes);
   });
   if (attr != cudaSuccess) return JANUS_ERR_CUDA;
   CUtensorMap ma, mb;
   if (kMode == kModeTN) {
     if (!map_rows_mn(&ma, A, R, M) || !map_rows_mn(&mb, W, R, N)) return JANUS_ERR_CUDA;
-  } else if (!map_b(&ma, W, E, Kd, N, kMode == kModeNT) || !map_a(&mb, A, R, Kd)) {
+  } else if (!map_b(&ma, W, E, Kd, N, kMode == kModeNT) ||
+             !(kBK == kBHalf ? map_a_half(&mb, reinterpret_cast<const uint16_t*>(A), R, Kd) : map_a(&mb, A, R, Kd))) {
     // operands swapped: the weights are the MMA's A, the dispatch rows its B
     return JANUS_ERR_CUDA;
   }
   Args a;
   a.C = C; a.C2 = C2; a.C3 = C3; a.aux = aux; a.aux2 = aux2; a.c_rows = c_rows;
+  a.row_scale = row_scale; a.rows = R;
   a.offsets = offsets; a.E = E; a.Kd = Kd; a.N = N; a.M = M; a.err = err;
   // one CTA per SM, in clusters of two (the MMA pairs)
   cudaLaunchConfig_t cfg = {};
@@ -850,7 +916,7 @@ janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, in
   cluster_attr[0].val.clusterDim.z = 1;
   cfg.attrs = cluster_attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, tc_gemm_kernel<kMode, kEpi, kBExact>, ma, mb, a) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, tc_gemm_kernel<kMode, kEpi, kBK>, ma, mb, a) != cudaSuccess)
     return JANUS_ERR_CUDA;
   return launch_status();
 }
@@ -863,8 +929,20 @@ janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, 
                             int32_t h, const float* w1, const float* w2, float* yd, float* act, float* H,
                             int32_t* err, cudaStream_t stream, float* const* yd_rows, bool x_tf32_exact) {
   janus_status st = x_tf32_exact
-                        ? launch<kModeNN, kEpiSilu, true>(xd, w1, R, E, d, h, H, act, nullptr, offsets, err, stream)
+                        ? launch<kModeNN, kEpiSilu, kBExact>(xd, w1, R, E, d, h, H, act, nullptr, offsets, err, stream)
                         : launch<kModeNN, kEpiSilu>(xd, w1, R, E, d, h, H, act, nullptr, offsets, err, stream);
+  if (st != JANUS_OK) return st;
+  return launch<kModeNN, kEpiStore>(H, w2, R, E, h, d, yd, nullptr, nullptr, offsets, err, stream, 0, nullptr,
+                                    nullptr, yd_rows);
+}
+
+janus_status expert_ffn_fwd_packed(const uint16_t* payload, const float* row_scale, const int32_t* offsets,
+                                   int32_t E, int64_t R, int32_t d, int32_t h, const float* w1, const float* w2,
+                                   float* yd, float* act, float* H, int32_t* err, cudaStream_t stream,
+                                   float* const* yd_rows) {
+  janus_status st = launch<kModeNN, kEpiSilu, kBHalf>(reinterpret_cast<const float*>(payload), w1, R, E, d, h, H,
+                                                      act, nullptr, offsets, err, stream, 0, nullptr, nullptr,
+                                                      nullptr, row_scale);
   if (st != JANUS_OK) return st;
   return launch<kModeNN, kEpiStore>(H, w2, R, E, h, d, yd, nullptr, nullptr, offsets, err, stream, 0, nullptr,
                                     nullptr, yd_rows);

@@ -21,6 +21,12 @@ janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, 
                             float* act, float* H, int32_t* err, cudaStream_t stream,
                             float* const* yd_rows = nullptr, bool x_tf32_exact = false);
 
+// The forward on the FP16 payload itself: row p of xd is f32(payload[p]) *
+// row_scale[p], unpacked by the GEMM (d % 8 == 0, payload 16-byte aligned).
+janus_status expert_ffn_fwd_packed(const uint16_t* payload, const float* row_scale, const int32_t* offsets,
+                                   int32_t E, int64_t R, int32_t d, int32_t h, const float* w1, const float* w2,
+                                   float* yd, float* act, float* H, int32_t* err, cudaStream_t stream,
+                                   float* const* yd_rows = nullptr);
 janus_status expert_ffn_vjp(const float* xd, const float* gd, const float* act_in, float* A,
                             const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
                             const float* w1, const float* w2, float* dxd, float* dA, int32_t* err,

@@ -17,6 +17,8 @@
 //   * grids are a multiple of the SM count with grid-stride loops over rows.
 #include <cuda_fp16.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "rows.cuh"
 
@@ -201,6 +203,19 @@ dequant_kernel(const uint2* __restrict__ payload, int64_t n_rows, int d4, int K,
   }
 }
 
+// row_scale[p] = scale[type of dispatch row p] (bad type ids as type 0, as in
+// the dequant kernel).
+__global__ void __launch_bounds__(kThreads)
+row_scale_kernel(int64_t n_rows, int K, const int32_t* __restrict__ types, int T,
+                 const int32_t* __restrict__ perm, const float* __restrict__ scale, float* __restrict__ row_scale) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < n_rows; p += stride) {
+    int t = types[perm[p] / K];
+    if (t < 0 || t >= T) t = 0;
+    row_scale[p] = scale[t];
+  }
+}
+
 }  // namespace
 }  // namespace janus
 
@@ -303,6 +318,22 @@ extern "C" janus_status janus_dequant_by_type(const uint16_t* payload, int64_t n
   const int64_t R = n_atoms * top_k;
   dequant_kernel<<<rows_grid(R, 8), kThreads, 0, (cudaStream_t)stream>>>(
       (const uint2*)payload, R, d / 4, top_k, types, n_types, perm, scale, (float4*)xd);
+  return launch_status();
+}
+
+extern "C" janus_status janus_dispatch_row_scales(int64_t n_atoms, int32_t top_k, const int32_t* types,
+                                                  int32_t n_types, const int32_t* perm, const float* scale,
+                                                  float* row_scale, janus_stream_t stream) {
+  JANUS_CHECK_ARG(n_atoms >= 0 && top_k >= 1 && top_k <= kMaxExperts);
+  JANUS_CHECK_ARG(n_atoms * (int64_t)top_k < (int64_t)INT32_MAX);
+  JANUS_CHECK_ARG(n_types >= 1 && n_types <= kMaxTypes);
+  if (n_atoms == 0) return JANUS_OK;
+  JANUS_CHECK_ARG(types && perm && scale && row_scale);
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  const int64_t R = n_atoms * top_k;
+  const int64_t blocks = std::min<int64_t>((R + kThreads - 1) / kThreads, (int64_t)num_sms() * 8);
+  row_scale_kernel<<<(unsigned)blocks, kThreads, 0, (cudaStream_t)stream>>>(R, top_k, types, n_types, perm, scale,
+                                                                             row_scale);
   return launch_status();
 }
 

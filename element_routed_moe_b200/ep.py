@@ -12,6 +12,8 @@ atoms.  One layer pass:
   VJP:      weighted FP32 send of dY -> barrier -> owner: input VJP of its
             experts -> return -> barrier -> combine (local)
 
+The owner's unpack is fused into the experts' first GEMM: it loads the
+received FP16 rows and their scales itself (janus_expert_ffn_fwd_packed).
 The return is fused into the experts' last GEMM by default: its epilogue
 stores each output row straight into the sender's return buffer through a row
 table (janus_ep_return_rows), so the rows cross NVLink as the tiles finish and
@@ -53,10 +55,13 @@ class ExpertParallelLayer:
             raise ValueError("w1_local / w2_local must hold this rank's E/P experts")
         self.w1, self.w2, self.mode = w1_local, w2_local, mode
         self.fused_return = bool(fused_return)
+        # the received FP16 rows go straight into the first GEMM (its
+        # tensor-core form needs d % 8 == 0; otherwise they are unpacked first)
+        self.fused_unpack = mode == J.JANUS_FFN_FP32_SIMT or d % 8 == 0
         # this library's kernels per forward + VJP: route 4, layout 1, pack 2,
-        # unpack 1, expert MLP 2 + 2, FP32 send 1, combine 1 + 1, and the
-        # return table (fused) or the return copy twice (not fused)
-        self.launches_per_step = 15 + (1 if self.fused_return else 2)
+        # expert MLP 2 + 2, FP32 send 1, combine 1 + 1, the unpack 1 (when not
+        # fused), and the return table (fused) or the return copy twice
+        self.launches_per_step = 14 + (0 if self.fused_unpack else 1) + (1 if self.fused_return else 2)
         self.nccl = self.dist and dist.get_backend(group) == "nccl"
         # worst case: every routed row of every rank lands on this rank
         self.n_atoms_max = int(n_atoms_max)
@@ -164,17 +169,19 @@ class ExpertParallelLayer:
         m(events, "send", 1)
         recv_off = self.layout[2][self.rank]
         m(events, "ffn_fwd", 0)
-        J.janus_ep_dequant_rows(self.payload, self.row_scale, self.layout, self.rank, out=self.xd)
-        # the unpacked FP16 rows are exact in TF32: the first GEMM skips their residual
-        flags = J.JANUS_FFN_X_DEQUANTIZED
+        out = dict(out=self.yd)
         if self.fused_return:
             # the table depends only on the layout: the VJP reuses it
             J.janus_ep_return_rows(self.layout, self.rank, self.peer_ret, self.cap, self.d, out=self.ret_rows)
-            J.janus_expert_ffn_fwd_ex(self.xd, recv_off, self.w1, self.w2, out_rows=self.ret_rows, act=self.act,
-                                      flags=flags, mode=self.mode)
+            out = dict(out_rows=self.ret_rows)
+        if self.fused_unpack:
+            J.janus_expert_ffn_fwd_packed(self.payload, self.row_scale, recv_off, self.w1, self.w2, act=self.act,
+                                          mode=self.mode, **out)
         else:
-            J.janus_expert_ffn_fwd_ex(self.xd, recv_off, self.w1, self.w2, out=self.yd, act=self.act, flags=flags,
-                                      mode=self.mode)
+            # the unpacked FP16 rows are exact in TF32: the first GEMM skips their residual
+            J.janus_ep_dequant_rows(self.payload, self.row_scale, self.layout, self.rank, out=self.xd)
+            J.janus_expert_ffn_fwd_ex(self.xd, recv_off, self.w1, self.w2, act=self.act,
+                                      flags=J.JANUS_FFN_X_DEQUANTIZED, mode=self.mode, **out)
         m(events, "ffn_fwd", 1)
         m(events, "return", 0)
         if not self.fused_return:

@@ -33,9 +33,10 @@ SYMBOLS = (
     "janus_route_layers_workspace_size", "janus_route_layers", "janus_active_experts",
     "janus_dispatch",
     "janus_quant_by_type_workspace_size", "janus_quant_by_type", "janus_quant_by_type_noalloc",
-    "janus_dequant_by_type",
+    "janus_dequant_by_type", "janus_dispatch_row_scales",
     "janus_expert_ffn_workspace_size", "janus_expert_ffn_fwd", "janus_expert_ffn_vjp",
     "janus_expert_ffn_fwd_rows", "janus_expert_ffn_vjp_rows", "janus_expert_ffn_fwd_ex",
+    "janus_expert_ffn_packed_workspace_size", "janus_expert_ffn_fwd_packed",
     "janus_expert_ffn_weight_grad_workspace_size", "janus_expert_ffn_weight_grad",
     "janus_expert_ffn_vjp_vjp_workspace_size", "janus_expert_ffn_vjp_vjp",
     "janus_combine", "janus_edge_aggregate", "janus_edge_broadcast", "janus_neighbor_aggregate",
@@ -95,6 +96,7 @@ def _declare(L):
         "janus_quant_by_type": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp, sz, vp]),
         "janus_quant_by_type_noalloc": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp]),
         "janus_dequant_by_type": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp]),
+        "janus_dispatch_row_scales": (st, [i64, i32, vp, i32, vp, vp, vp, vp]),
         "janus_expert_ffn_workspace_size": (st, [i64, i32, i32, i32, i32, i32, ctypes.c_int, psz]),
         "janus_expert_ffn_fwd": (st, [vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, ctypes.c_int,
                                       vp, sz, vp]),
@@ -106,6 +108,9 @@ def _declare(L):
                                            ctypes.c_int, vp, sz, vp]),
         "janus_expert_ffn_fwd_ex": (st, [vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, ctypes.c_uint32,
                                          ctypes.c_int, vp, sz, vp]),
+        "janus_expert_ffn_packed_workspace_size": (st, [i64, i32, i32, ctypes.c_int, psz]),
+        "janus_expert_ffn_fwd_packed": (st, [vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, ctypes.c_int,
+                                             vp, sz, vp]),
         "janus_expert_ffn_weight_grad_workspace_size": (st, [i64, i32, i32, psz]),
         "janus_expert_ffn_weight_grad": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp,
                                               ctypes.c_int, vp, sz, vp]),
@@ -481,6 +486,20 @@ def janus_dequant_by_type(payload, types, n_types, perm, top_k, scale, *, out=No
     return out
 
 
+def janus_dispatch_row_scales(types, n_types, perm, top_k, scale, *, out=None, stream=None):
+    """row_scale [R] = scale[type of dispatch row p] (the per-row scales the
+    packed forward takes)."""
+    K = int(top_k)
+    N = types.shape[0]
+    if out is None:
+        out = _empty((N * K,), torch.float32, types.device)
+    _raise(lib().janus_dispatch_row_scales(N, K, _p(types, torch.int32, "types"), int(n_types),
+                                           _p(perm, torch.int32, "perm"), _p(scale, torch.float32, "scale"),
+                                           _p(out, torch.float32, "row_scale"), _stream(stream)),
+           "janus_dispatch_row_scales")
+    return out
+
+
 # --------------------------------------------------------------------------
 # grouped expert MLP
 # --------------------------------------------------------------------------
@@ -580,6 +599,40 @@ def janus_expert_ffn_fwd_ex(xd, offsets, w1, w2, *, out=None, out_rows=None, fla
                                          None if out_rows is None else _row_table(out_rows, R),
                                          _p(act, torch.float32, "act"), int(flags), int(mode), _p(ws), nb,
                                          _stream(stream)), "janus_expert_ffn_fwd_ex")
+    return out, act
+
+
+def janus_expert_ffn_packed_workspace_size(n_rows, d, h, mode=JANUS_FFN_FP32_SIMT) -> int:
+    b = ctypes.c_size_t(0)
+    _raise(lib().janus_expert_ffn_packed_workspace_size(n_rows, d, h, int(mode), ctypes.byref(b)),
+           "janus_expert_ffn_packed_workspace_size")
+    return b.value
+
+
+def janus_expert_ffn_fwd_packed(payload, row_scale, offsets, w1, w2, *, out=None, out_rows=None,
+                                mode=JANUS_FFN_FP32_SIMT, want_act=False, act=None, workspace=None, stream=None):
+    """The forward on the FP16 payload [R,d] with per-row scales [R] (the
+    unpack fused into the GEMM); output as in janus_expert_ffn_fwd_ex.
+    Returns (out-or-None, act-or-None)."""
+    R, d = payload.shape
+    E, _, h = w1.shape
+    if payload.dtype not in (torch.float16, torch.int16, torch.uint16):
+        raise ValueError("payload must hold 16-bit FP16 words")
+    if out is not None and out_rows is not None:
+        raise ValueError("give out or out_rows, not both")
+    if out is None and out_rows is None:
+        out = _empty((R, d), torch.float32, payload.device)
+    if want_act and act is None:
+        act = _empty((R, h), torch.float32, payload.device)
+    nb = janus_expert_ffn_packed_workspace_size(R, d, h, mode)
+    ws = _workspace(nb, payload.device, workspace)
+    _raise(lib().janus_expert_ffn_fwd_packed(_p(payload, None, "payload"), _p(row_scale, torch.float32, "row_scale"),
+                                             _p(offsets, torch.int32, "offsets"), E, R, d, h,
+                                             _p(w1, torch.float32, "w1"), _p(w2, torch.float32, "w2"),
+                                             _p(out, torch.float32, "yd"),
+                                             None if out_rows is None else _row_table(out_rows, R),
+                                             _p(act, torch.float32, "act"), int(mode), _p(ws), nb, _stream(stream)),
+           "janus_expert_ffn_fwd_packed")
     return out, act
 
 

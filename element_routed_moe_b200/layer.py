@@ -31,7 +31,7 @@ class MoELayer:
     OPS_FWD = ("route", "dispatch", "ffn_fwd", "combine")
     OPS_VJP = ("dispatch_w", "ffn_vjp", "combine_vjp")
     # this library's kernels per call (see each entry point's launches)
-    LAUNCHES = {"edge_aggregate": 1, "quant": 2, "dequant": 1, "route": 4, "dispatch": 1,
+    LAUNCHES = {"edge_aggregate": 1, "quant": 2, "dequant": 1, "row_scales": 1, "route": 4, "dispatch": 1,
                 "ffn_fwd": 2, "combine": 1, "dispatch_w": 1, "ffn_vjp": 2, "combine_vjp": 1}
 
     def __init__(self, n_atoms, top_k, gate, w1, w2, *, mode=J.JANUS_FFN_3XTF32, packed=False,
@@ -62,17 +62,25 @@ class MoELayer:
         self.dxd = torch.empty((R, d), **f32)
         self.y = torch.empty((N, d), **f32)
         self.dx = torch.empty((N, d), **f32)
+        # packed: the first GEMM reads the FP16 payload itself (the unpack is
+        # fused into it); its tensor-core form needs d % 8 == 0
+        self.fused_unpack = packed and (mode == J.JANUS_FFN_FP32_SIMT or d % 8 == 0)
         nb = max(J.janus_expert_ffn_workspace_size(R, d, h, E, False, True, mode),
-                 J.janus_expert_ffn_workspace_size(R, d, h, E, True, True, mode))
+                 J.janus_expert_ffn_workspace_size(R, d, h, E, True, True, mode),
+                 J.janus_expert_ffn_packed_workspace_size(R, d, h, mode) if self.fused_unpack else 0)
         self.ffn_ws = torch.empty(nb, dtype=torch.uint8, device=dev)
         if row_ptr is not None:
             self.xagg = torch.empty((N, d), **f32)
         if packed:
             self.payload = torch.empty((R, d), dtype=torch.float16, device=dev)
             self.scale = torch.empty((T,), **f32)
+            self.row_scale = torch.empty((R,), **f32)
             self.quant_ws = torch.empty(J.janus_quant_by_type_workspace_size(T), dtype=torch.uint8, device=dev)
         front = ("edge_aggregate",) if row_ptr is not None else ()
-        mid = ("route", "quant", "dequant") if packed else ("route", "dispatch")
+        if packed:
+            mid = ("route", "quant", "row_scales" if self.fused_unpack else "dequant")
+        else:
+            mid = ("route", "dispatch")
         self.ops = front + mid + ("ffn_fwd", "combine") + self.OPS_VJP
         self.launches_per_call = sum(self.LAUNCHES[o] for o in self.ops)
         self._host = None
@@ -103,18 +111,28 @@ class MoELayer:
             J.janus_quant_by_type(x, types, T, r["slot_of"], K, payload=self.payload, scale=self.scale,
                                   workspace=self.quant_ws)
             mark("quant", 1)
-            mark("dequant", 0)
-            J.janus_dequant_by_type(self.payload, types, T, r["perm"], K, self.scale, out=self.xd)
-            mark("dequant", 1)
+            if self.fused_unpack:
+                mark("row_scales", 0)
+                J.janus_dispatch_row_scales(types, T, r["perm"], K, self.scale, out=self.row_scale)
+                mark("row_scales", 1)
+            else:
+                mark("dequant", 0)
+                J.janus_dequant_by_type(self.payload, types, T, r["perm"], K, self.scale, out=self.xd)
+                mark("dequant", 1)
         else:
             mark("dispatch", 0)
             J.janus_dispatch(x, r["slot_of"], K, out=self.xd)
             mark("dispatch", 1)
         mark("ffn_fwd", 0)
-        # unpacked FP16 rows are exact in TF32: the first GEMM skips their residual
-        J.janus_expert_ffn_fwd_ex(self.xd, r["offsets"], self.w1, self.w2, out=self.yd, act=self.act,
-                                  flags=J.JANUS_FFN_X_DEQUANTIZED if self.packed else 0, mode=self.mode,
-                                  workspace=self.ffn_ws)
+        if self.fused_unpack:
+            # the FP16 rows go straight into the first GEMM (xd is not written)
+            J.janus_expert_ffn_fwd_packed(self.payload, self.row_scale, r["offsets"], self.w1, self.w2, out=self.yd,
+                                          act=self.act, mode=self.mode, workspace=self.ffn_ws)
+        else:
+            # unpacked FP16 rows are exact in TF32: the first GEMM skips their residual
+            J.janus_expert_ffn_fwd_ex(self.xd, r["offsets"], self.w1, self.w2, out=self.yd, act=self.act,
+                                      flags=J.JANUS_FFN_X_DEQUANTIZED if self.packed else 0, mode=self.mode,
+                                      workspace=self.ffn_ws)
         mark("ffn_fwd", 1)
         mark("combine", 0)
         J.janus_combine(self.yd, r["slot_of"], K, r["topk_weight"], out=y)
@@ -125,6 +143,7 @@ class MoELayer:
         J.janus_dispatch(g, r["slot_of"], K, r["topk_weight"], out=self.gd)
         mark("dispatch_w", 1)
         mark("ffn_vjp", 0)
+        # (xd is read only when the pre-activations are not saved; here they are)
         J.janus_expert_ffn_vjp(self.xd, self.gd, r["offsets"], self.w1, self.w2, act=self.act,
                                mode=self.mode, out=self.dxd, workspace=self.ffn_ws)
         mark("ffn_vjp", 1)

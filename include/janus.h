@@ -194,6 +194,14 @@ janus_status janus_dequant_by_type(const uint16_t* payload, int64_t n_atoms, int
                                    const int32_t* perm, const float* scale, float* xd,
                                    janus_stream_t stream);
 
+/* Per-row scales of the packed dispatch: row_scale[p] = scale[types[perm[p] /
+ * top_k]] for the R = n_atoms * top_k dispatch rows (bad type ids as type 0),
+ * the per-row form janus_expert_ffn_fwd_packed takes.  row_scale: device
+ * float [R]. */
+janus_status janus_dispatch_row_scales(int64_t n_atoms, int32_t top_k, const int32_t* types, int32_t n_types,
+                                       const int32_t* perm, const float* scale, float* row_scale,
+                                       janus_stream_t stream);
+
 /* -------------------------------------------------------------------------
  * Grouped expert MLP.  [Review] section 3.1, Table II (MLP hidden size);
  * each expert is read as bias-free Linear(d,h) -> SiLU -> Linear(h,d):
@@ -256,6 +264,26 @@ janus_status janus_expert_ffn_fwd_ex(const float* xd, const int32_t* offsets, in
                                      const float* w2, float* yd, float* const* yd_rows, float* act,
                                      uint32_t flags, janus_ffn_mode mode, void* workspace,
                                      size_t workspace_bytes, janus_stream_t stream);
+/* The forward on the FP16 payload itself (the unpack fused into the GEMM):
+ * row p of xd is f32(payload[p,:]) * row_scale[p] (payload from
+ * janus_quant_by_type or an expert-parallel receive buffer; row_scale from
+ * janus_dispatch_row_scales or the receive buffer's scales).  yd or yd_rows
+ * (exactly one non-NULL) as in janus_expert_ffn_fwd_ex.  In
+ * JANUS_FFN_3XTF32 the first GEMM loads the FP16 rows by TMA, unpacks them in
+ * shared memory and runs two tensor-core products (the rows are exact in
+ * TF32); d must be a multiple of 8 (JANUS_ERR_MISALIGNED otherwise) and the
+ * payload 16-byte aligned.  In JANUS_FFN_FP32_SIMT the rows are unpacked
+ * into the workspace first.  The result is bit-identical to
+ * janus_dequant_by_type followed by janus_expert_ffn_fwd_ex with
+ * JANUS_FFN_X_DEQUANTIZED.  workspace: janus_expert_ffn_packed_workspace_size
+ * bytes, 256-byte aligned. */
+janus_status janus_expert_ffn_packed_workspace_size(int64_t n_rows, int32_t d, int32_t h, janus_ffn_mode mode,
+                                                    size_t* bytes);
+janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, const float* row_scale, const int32_t* offsets,
+                                         int32_t n_experts, int64_t n_rows, int32_t d, int32_t h, const float* w1,
+                                         const float* w2, float* yd, float* const* yd_rows, float* act,
+                                         janus_ffn_mode mode, void* workspace, size_t workspace_bytes,
+                                         janus_stream_t stream);
 janus_status janus_expert_ffn_vjp_rows(const float* xd, const float* gd, const float* act,
                                        const int32_t* offsets, int32_t n_experts, int64_t n_rows,
                                        int32_t d, int32_t h, const float* w1, const float* w2,

@@ -122,6 +122,14 @@ def test_argument_validation_before_launch(J):
                                      1 << 30, null) == J.JANUS_ERR_INVALID_ARG
     assert L.janus_expert_ffn_fwd_ex(FAKE, FAKE, 4, 100, 64, 64, FAKE, FAKE, FAKE, null, null, 6, 1, FAKE,
                                      1 << 30, null) == J.JANUS_ERR_INVALID_ARG
+    # packed forward: d % 8 on the tensor cores, workspace too small, no row scales
+    assert L.janus_expert_ffn_fwd_packed(FAKE, FAKE, FAKE, 4, 100, 12, 64, FAKE, FAKE, FAKE, null, null, 1, FAKE,
+                                         1 << 30, null) == J.JANUS_ERR_MISALIGNED
+    assert L.janus_expert_ffn_fwd_packed(FAKE, FAKE, FAKE, 4, 100, 64, 64, FAKE, FAKE, FAKE, null, null, 0, FAKE,
+                                         1024, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_expert_ffn_fwd_packed(FAKE, null, FAKE, 4, 100, 64, 64, FAKE, FAKE, FAKE, null, null, 1, FAKE,
+                                         1 << 30, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_dispatch_row_scales(10, 2, FAKE, 0, FAKE, FAKE, FAKE, null) == J.JANUS_ERR_INVALID_ARG
     # EP return table: E not a multiple of P, missing peer buffer, d % 4, misaligned table
     two = (ctypes.c_void_p * 2)(FAKE, FAKE)
     assert L.janus_ep_return_rows(FAKE, FAKE, FAKE, 0, 2, 5, 10, 8, two, FAKE, null) == J.JANUS_ERR_INVALID_ARG

@@ -87,3 +87,79 @@ def test_rows_that_break_the_promise_are_reported():
     with pytest.raises(J.JanusError) as e:
         J.janus_check(ws)
     assert e.value.status == J.JANUS_ERR_DATA
+
+
+# ---------------------------------------------------------------------------
+# the forward on the FP16 payload itself: the unpack fused into the GEMM
+# ---------------------------------------------------------------------------
+PACKED = {
+    # name: (N, T, E, K, d, h)
+    "ragged8": (700, 11, 12, 3, 136, 68),
+    "M_like": (4096, 89, 40, 8, 512, 384),
+    "tails": (257, 5, 9, 2, 8, 4),
+}
+
+
+def _packed_inputs(N, T, E, K, d, seed):
+    types = to_dev(synth.types_zipf(N, T, seed=seed))
+    gate = to_dev(synth.gate_table(T, E, seed + 1))
+    x = synth.normal((N, d), seed + 2, DEV)
+    r = J.janus_route(types, gate, K)
+    payload, scale, _ = J.janus_quant_by_type(x, types, T, r["slot_of"], K)
+    return types, r, payload, scale
+
+
+@pytest.mark.parametrize("mode", [J.JANUS_FFN_FP32_SIMT, J.JANUS_FFN_3XTF32])
+@pytest.mark.parametrize("name", list(PACKED))
+def test_packed_forward_equals_unpack_then_forward(name, mode):
+    N, T, E, K, d, h = PACKED[name]
+    types, r, payload, scale = _packed_inputs(N, T, E, K, d, 70)
+    w1, w2 = synth.expert_weights(E, d, h, 71, DEV)
+    row_scale = J.janus_dispatch_row_scales(types, T, r["perm"], K, scale)
+    # the per-row scales are the per-type scales of each row's atom
+    ht, hp = host(types), host(r["perm"])
+    assert np.array_equal(host(row_scale), host(scale)[ht[hp // K]])
+    xd = J.janus_dequant_by_type(payload, types, T, r["perm"], K, scale)
+    y_ref, a_ref = J.janus_expert_ffn_fwd_ex(xd, r["offsets"], w1, w2, flags=J.JANUS_FFN_X_DEQUANTIZED, mode=mode,
+                                             want_act=True)
+    nb = J.janus_expert_ffn_packed_workspace_size(xd.shape[0], d, h, mode)
+    ws = torch.zeros(nb, dtype=torch.uint8, device=DEV)
+    y, a = J.janus_expert_ffn_fwd_packed(payload, row_scale, r["offsets"], w1, w2, mode=mode, want_act=True,
+                                         workspace=ws)
+    J.janus_check(ws)
+    assert torch.equal(y, y_ref) and torch.equal(a, a_ref)
+    offs = host(r["offsets"])
+    rows = sample_rows(offs, 64, seed=5, R=xd.shape[0])
+    ref = oracle.expert_ffn_fwd(host(xd), offs, host(w1), host(w2), rows=rows)
+    assert rel_fro(host(y)[rows], ref) <= TOL_FP32
+
+
+def test_packed_forward_into_a_row_table():
+    N, T, E, K, d, h = PACKED["ragged8"]
+    types, r, payload, scale = _packed_inputs(N, T, E, K, d, 80)
+    w1, w2 = synth.expert_weights(E, d, h, 81, DEV)
+    row_scale = J.janus_dispatch_row_scales(types, T, r["perm"], K, scale)
+    R = payload.shape[0]
+    y_ref, _ = J.janus_expert_ffn_fwd_packed(payload, row_scale, r["offsets"], w1, w2, mode=J.JANUS_FFN_3XTF32)
+    dest = torch.full((R + 5, d), float("nan"), device=DEV)
+    slot = torch.as_tensor(np.random.default_rng(82).permutation(R + 5)[:R], device=DEV)
+    table = dest.data_ptr() + 4 * d * slot.to(torch.int64)
+    out, _ = J.janus_expert_ffn_fwd_packed(payload, row_scale, r["offsets"], w1, w2, out_rows=table,
+                                           mode=J.JANUS_FFN_3XTF32)
+    torch.cuda.synchronize()
+    assert out is None and torch.equal(dest[slot], y_ref)
+
+
+def test_packed_forward_needs_d_multiple_of_8_on_the_tensor_cores():
+    N, T, E, K, d, h = 64, 3, 4, 2, 12, 8
+    types, r, payload, scale = _packed_inputs(N, T, E, K, d, 90)
+    w1, w2 = synth.expert_weights(E, d, h, 91, DEV)
+    row_scale = J.janus_dispatch_row_scales(types, T, r["perm"], K, scale)
+    with pytest.raises(J.JanusError) as e:
+        J.janus_expert_ffn_fwd_packed(payload, row_scale, r["offsets"], w1, w2, mode=J.JANUS_FFN_3XTF32)
+    assert e.value.status == J.JANUS_ERR_MISALIGNED
+    # the SIMT path takes any d % 4 == 0
+    y, _ = J.janus_expert_ffn_fwd_packed(payload, row_scale, r["offsets"], w1, w2, mode=J.JANUS_FFN_FP32_SIMT)
+    xd = J.janus_dequant_by_type(payload, types, T, r["perm"], K, scale)
+    y_ref, _ = J.janus_expert_ffn_fwd(xd, r["offsets"], w1, w2, mode=J.JANUS_FFN_FP32_SIMT)
+    assert torch.equal(y, y_ref)
