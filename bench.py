@@ -194,7 +194,7 @@ class ClockSampler:
 # S-shaped layer (profiles/expert_ffn_tc_gemm.md), valid only for the kernel
 # source it was taken on.
 GEMM_TRAFFIC = {("S", "3xtf32"): {"src": "element_routed_moe_b200/csrc/ffn_tc.cu",
-                                  "sha256_prefix": "0515a5eaee71c330", "bytes_per_launch": 3.235e9}}
+                                  "sha256_prefix": "045bb1478b54cb10", "bytes_per_launch": 3.258e9}}
 
 
 def measured_traffic(workload: str, mode: str):
