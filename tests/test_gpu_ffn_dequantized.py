@@ -163,3 +163,22 @@ def test_packed_forward_needs_d_multiple_of_8_on_the_tensor_cores():
     xd = J.janus_dequant_by_type(payload, types, T, r["perm"], K, scale)
     y_ref, _ = J.janus_expert_ffn_fwd(xd, r["offsets"], w1, w2, mode=J.JANUS_FFN_FP32_SIMT)
     assert torch.equal(y, y_ref)
+
+
+def test_row_scales_treat_bad_type_ids_as_type_0_like_the_unpack():
+    # the per-row scales and janus_dequant_by_type agree on every row,
+    # including atoms whose type id is outside [0, T)
+    N, T, E, K, d = 300, 6, 5, 2, 16
+    types_np = synth.types_uniform(N, T, 7).astype(np.int32)
+    types_np[[3, 50, 299]] = [-1, T, 1000]
+    types = to_dev(types_np)
+    gate = to_dev(synth.gate_table(T, E, 8))
+    r = J.janus_route(to_dev(np.clip(types_np, 0, T - 1)), gate, K)
+    scale = to_dev(np.exp2(np.arange(T, dtype=np.float32) - 3.0).astype(np.float32))
+    row_scale = J.janus_dispatch_row_scales(types, T, r["perm"], K, scale)
+    t_row = types_np[host(r["perm"]) // K]
+    t_row = np.where((t_row < 0) | (t_row >= T), 0, t_row)
+    assert np.array_equal(host(row_scale), host(scale)[t_row])
+    payload = torch.ones((N * K, d), dtype=torch.float16, device=DEV)
+    xd = J.janus_dequant_by_type(payload, types, T, r["perm"], K, scale)
+    assert np.array_equal(host(xd)[:, 0], host(row_scale))
