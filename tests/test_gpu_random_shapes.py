@@ -3,7 +3,9 @@ Barrier of Billion-Parameter Universal Machine Learning Interatomic
 Potentials', sections 3.1-3.5): each case draws N, T, E, K, d, h and the
 edge count, including empty layers, one type, K up to 32, E up to 256, and
 d, h at odd multiples of 4, then checks the path step by step against the
-oracle: routing and packing bit-exact, features within 1e-5.
+oracle: routing and packing bit-exact, features within 1e-5; the forward on
+the FP16 rows (unpack fused into the GEMM) and with the exact-row flag must
+equal the plain forward on the unpacked rows bit for bit.
 """
 import numpy as np
 import pytest
@@ -67,6 +69,17 @@ def test_random_shape_chain(seed):
         dxd = J.janus_expert_ffn_vjp(xd, gd, r["offsets"], w1, w2, act=act, mode=mode)
         assert rel_fro(host(yd), oyd) <= TOL_FP32, (mode, seed)
         assert rel_fro(host(dxd), odxd) <= TOL_FP32, (mode, seed)
+    # the forward on the FP16 rows themselves (unpack fused into the GEMM) and on
+    # the unpacked rows with the exact-TF32 flag: both bit-identical to the plain
+    # forward on the unpacked rows
+    row_scale = J.janus_dispatch_row_scales(to_dev(types), T, r["perm"], K, scale)
+    for mode in (J.JANUS_FFN_FP32_SIMT, J.JANUS_FFN_3XTF32):
+        yq, _ = J.janus_expert_ffn_fwd(xq, r["offsets"], w1, w2, mode=mode)
+        yf, _ = J.janus_expert_ffn_fwd_ex(xq, r["offsets"], w1, w2, flags=J.JANUS_FFN_X_DEQUANTIZED, mode=mode)
+        assert torch.equal(yf, yq), (mode, seed)
+        if mode == J.JANUS_FFN_FP32_SIMT or d % 8 == 0:
+            yp, _ = J.janus_expert_ffn_fwd_packed(payload, row_scale, r["offsets"], w1, w2, mode=mode)
+            assert torch.equal(yp, yq), (mode, seed)
     y = J.janus_combine(yd, r["slot_of"], K, r["topk_weight"])
     assert rel_fro(host(y), oracle.combine(host(yd), o["slot_of"], K, o["topk_weight"])) <= TOL_FP32
     dx = J.janus_combine(dxd, r["slot_of"], K)
