@@ -474,7 +474,10 @@ def run_janus(args, world, rank, local):
         "clocks": clocks,
     }
 
-    if not args.no_e2e and not layer.edges:   # host-side edge messages would be 9-29 GB per step
+    # (skipped where the step's input is the edge messages of L or the slice:
+    # 9-29 GB to upload per step)
+    msg_bytes = layer.msg.numel() * 4 if layer.edges else 0
+    if not args.no_e2e and msg_bytes <= (1 << 30):
         line["e2e"] = run_e2e(layer, args)
     if not args.no_extras:
         line["extras"] = run_extras(layer, peaks)
@@ -651,7 +654,8 @@ def run_e2e(layer, args):
     streams: dY's upload overlaps the forward, y's download the VJP, and the
     next step's upload this step's compute."""
     core = layer.core
-    x_h = layer.x.cpu().pin_memory()
+    # the step's input: the edge messages where the workload aggregates them
+    x_h = (layer.msg if layer.edges else layer.x).cpu().pin_memory()
     g_h = layer.g.cpu().pin_memory()
     t_h = layer.types.cpu().pin_memory()
     y_h = torch.empty(layer.y.shape, dtype=torch.float32).pin_memory()
