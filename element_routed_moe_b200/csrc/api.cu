@@ -1,6 +1,9 @@
-// Library-wide entry points: status strings, version, janus_check, and the
-// host-side launch-failure injection used by the tests.
+// Library-wide entry points: status strings, version, janus_check, the debug
+// build's fault word (janus_debug_build, janus_debug_check), and the host-side
+// launch-failure injection used by the tests.
 #include <atomic>
+#include <mutex>
+#include <unordered_map>
 
 #include "common.cuh"
 
@@ -23,6 +26,29 @@ int num_sms() {
     return 148;
   return n;
 }
+
+#ifdef JANUS_DEBUG
+// The debug build's fault word for calls without a workspace (one per GPU that
+// loads the library).  Host code takes its address with cudaGetSymbolAddress.
+static __device__ __align__(256) int32_t g_debug_fault[64];
+
+static std::mutex g_debug_mu;
+static std::unordered_map<int, int32_t*> g_debug_addr;   // device ordinal -> address
+
+int32_t* debug_fault_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lock(g_debug_mu);
+  auto it = g_debug_addr.find(dev);
+  if (it != g_debug_addr.end()) return it->second;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_debug_fault) != cudaSuccess) return nullptr;
+  g_debug_addr[dev] = (int32_t*)p;
+  return (int32_t*)p;
+}
+#else
+int32_t* debug_fault_word() { return nullptr; }
+#endif
 
 }  // namespace janus
 
@@ -49,6 +75,18 @@ janus_status janus_check(const void* workspace, janus_stream_t stream) {
   int32_t err = 0;
   if (cudaMemcpy(&err, workspace, sizeof(err), cudaMemcpyDeviceToHost) != cudaSuccess)
     return JANUS_ERR_CUDA;
+  return err == 0 ? JANUS_OK : JANUS_ERR_DATA;
+}
+
+int32_t janus_debug_build(void) { return janus::kDebug ? 1 : 0; }
+
+janus_status janus_debug_check(janus_stream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return JANUS_ERR_CUDA;
+  int32_t* w = janus::debug_fault_word();
+  if (!w) return JANUS_OK;   // release build: nothing is recorded here
+  int32_t err = 0;
+  if (cudaMemcpy(&err, w, sizeof(err), cudaMemcpyDeviceToHost) != cudaSuccess) return JANUS_ERR_CUDA;
+  if (err != 0 && cudaMemset(w, 0, sizeof(int32_t)) != cudaSuccess) return JANUS_ERR_CUDA;
   return err == 0 ? JANUS_OK : JANUS_ERR_DATA;
 }
 

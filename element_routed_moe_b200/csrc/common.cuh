@@ -16,7 +16,28 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 
-enum DataFault : int32_t { kFaultBadType = 1, kFaultNonFinite = 2 };
+// Data-fault codes written to a workspace's error word (first fault wins).
+enum DataFault : int32_t {
+  kFaultBadType = 1,     // element type id outside [0, T)
+  kFaultNonFinite = 2,   // non-finite feature to pack, or non-finite gate logit
+  kFaultTimeout = 3,     // a bounded tensor-core pipeline wait ran out
+  kFaultNotTf32 = 4,     // JANUS_FFN_X_DEQUANTIZED rows with bits below TF32 precision
+  kFaultIndex = 5,       // debug builds: a caller-supplied index outside its range
+  kFaultCapacity = 6,    // expert-parallel receive buffer too small for the routed rows
+};
+
+// Debug builds (compiled with -DJANUS_DEBUG) check every caller-supplied index
+// (slot_of, perm, offsets, row_ptr, senders, exchange tables) on the device
+// before using it, record kFaultIndex and skip the access instead.
+#ifdef JANUS_DEBUG
+constexpr bool kDebug = true;
+#else
+constexpr bool kDebug = false;
+#endif
+
+// Debug builds: device address, on the current device, of the library's fault
+// word for calls that take no workspace; release builds: nullptr.
+int32_t* debug_fault_word();
 
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTypes = 4096;
@@ -42,6 +63,15 @@ inline janus_status launch_status() {
 __device__ __forceinline__ void record_fault(WsHeader* ws, int32_t code) {
   atomicCAS(&ws->error, 0, code);
 }
+
+// Debug builds: record an index fault in `word` (the library's debug fault
+// word or a workspace's error word); a no-op in release builds.
+__device__ __forceinline__ void debug_fault(int32_t* word) {
+  if (kDebug && word) atomicCAS(word, 0, (int32_t)kFaultIndex);
+}
+
+// 0 <= v < n
+__device__ __forceinline__ bool in_range(int64_t v, int64_t n) { return (uint64_t)v < (uint64_t)n; }
 
 }  // namespace janus
 

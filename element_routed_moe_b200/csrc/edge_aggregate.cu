@@ -16,7 +16,13 @@
 //   * FP32 accumulation: each group of 4 edges is summed pairwise and then
 //     added to the running sum (edge order otherwise); each output row is
 //     written once;
-//   * 64-bit element offsets (Ed*d exceeds 2^31 at production sizes).
+//   * 64-bit element offsets (Ed*d exceeds 2^31 at production sizes);
+//   * message row 0 is edge row_ptr[0], so a receiver range of a larger CSR
+//     runs as it stands (the pinned-host pipeline streams the messages in
+//     such chunks);
+//   * every edge range is clamped to [0, n_edges), so a malformed row_ptr
+//     cannot make a kernel read or write outside the message buffer (debug
+//     builds also record the fault).
 #include "common.cuh"
 
 namespace janus {
@@ -31,13 +37,29 @@ __device__ __forceinline__ float4 f4add(float4 a, float4 b) {
   return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
 
+// Receiver i's rows of the message buffer, [*e0, *e1): msg row 0 is edge
+// row_ptr[0], so a receiver range of a larger CSR (row_ptr + i0 with the
+// messages of edges [row_ptr[i0], row_ptr[i1])) is processed as it stands.
+// The range is clamped to [0, n_edges]: a row_ptr that decreases or runs past
+// the edge count gives a shorter (possibly empty) range instead of an
+// out-of-bounds access; debug builds record it.
+__device__ __forceinline__ void edge_range(const int64_t* __restrict__ row_ptr, int64_t i, int64_t n_edges,
+                                           int32_t* dbg, int64_t* e0, int64_t* e1) {
+  const int64_t base = row_ptr[0];
+  const int64_t a = row_ptr[i] - base, b = row_ptr[i + 1] - base;
+  if (kDebug && (a < 0 || b < a || b > n_edges) && (threadIdx.x % 32) == 0) debug_fault(dbg);
+  *e0 = min(max(a, (int64_t)0), n_edges);
+  *e1 = min(max(b, *e0), n_edges);
+}
+
 __global__ void __launch_bounds__(kThreads)
 edge_aggregate_kernel(const float4* __restrict__ msg, const int64_t* __restrict__ row_ptr,
-                      int64_t n_atoms, int d4, float4* __restrict__ out) {
+                      int64_t n_atoms, int64_t n_edges, int d4, float4* __restrict__ out, int32_t* dbg) {
   const int lane = threadIdx.x % 32;
   const int64_t nwarps = (int64_t)gridDim.x * kThreads / 32;
   for (int64_t i = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / 32; i < n_atoms; i += nwarps) {
-    const int64_t e0 = row_ptr[i], e1 = row_ptr[i + 1];
+    int64_t e0, e1;
+    edge_range(row_ptr, i, n_edges, dbg, &e0, &e1);
     for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
       float4 acc[kU];
 #pragma unroll
@@ -85,11 +107,12 @@ edge_aggregate_kernel(const float4* __restrict__ msg, const int64_t* __restrict_
 // receiver's contiguous block of edge rows with streaming stores.
 __global__ void __launch_bounds__(kThreads)
 edge_broadcast_kernel(const float4* __restrict__ dx, const int64_t* __restrict__ row_ptr, int64_t n_atoms,
-                      int d4, float4* __restrict__ dmsg) {
+                      int64_t n_edges, int d4, float4* __restrict__ dmsg, int32_t* dbg) {
   const int lane = threadIdx.x % 32;
   const int64_t nwarps = (int64_t)gridDim.x * kThreads / 32;
   for (int64_t i = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / 32; i < n_atoms; i += nwarps) {
-    const int64_t e0 = row_ptr[i], e1 = row_ptr[i + 1];
+    int64_t e0, e1;
+    edge_range(row_ptr, i, n_edges, dbg, &e0, &e1);
     if (e1 <= e0) continue;
     for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
       float4 v[kU];
@@ -114,15 +137,17 @@ edge_broadcast_kernel(const float4* __restrict__ dx, const int64_t* __restrict__
 // of 32 edges are read with one coalesced load and broadcast by shuffles;
 // rows are gathered 4 edges at a time (U float4s each) for memory-level
 // parallelism; FP32 accumulation as in edge_aggregate_kernel.  Senders outside [0, N) are
-// skipped (they contribute nothing), so a bad index cannot read out of bounds.
+// skipped (they contribute nothing; debug builds record them), so a bad index
+// cannot read out of bounds.
 __global__ void __launch_bounds__(kThreads)
 neighbor_aggregate_kernel(const float4* __restrict__ x, const int64_t* __restrict__ row_ptr,
-                          const int32_t* __restrict__ senders, int64_t n_atoms, int d4,
-                          float4* __restrict__ out) {
+                          const int32_t* __restrict__ senders, int64_t n_atoms, int64_t n_edges, int d4,
+                          float4* __restrict__ out, int32_t* dbg) {
   const int lane = threadIdx.x % 32;
   const int64_t nwarps = (int64_t)gridDim.x * kThreads / 32;
   for (int64_t i = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / 32; i < n_atoms; i += nwarps) {
-    const int64_t e0 = row_ptr[i], e1 = row_ptr[i + 1];
+    int64_t e0, e1;
+    edge_range(row_ptr, i, n_edges, dbg, &e0, &e1);
     for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
       float4 acc[kU];
 #pragma unroll
@@ -130,7 +155,10 @@ neighbor_aggregate_kernel(const float4* __restrict__ x, const int64_t* __restric
       for (int64_t eb = e0; eb < e1; eb += 32) {
         const int64_t my_e = eb + lane;
         int32_t my_s = my_e < e1 ? senders[my_e] : -1;
-        if (my_s >= n_atoms) my_s = -1;
+        if (my_e < e1 && !in_range(my_s, n_atoms)) {
+          debug_fault(dbg);
+          my_s = -1;
+        }
         const int n_here = (int)min((int64_t)32, e1 - eb);
         for (int t = 0; t < n_here; t += 4) {
           int32_t s4[4];
@@ -167,54 +195,50 @@ neighbor_aggregate_kernel(const float4* __restrict__ x, const int64_t* __restric
 
 using namespace janus;
 
-extern "C" janus_status janus_edge_aggregate(const float* msg, const int64_t* row_ptr,
+extern "C" janus_status janus_edge_aggregate(const float* msg, int64_t n_edges, const int64_t* row_ptr,
                                              int64_t n_atoms, int32_t d, float* out,
                                              janus_stream_t stream) {
-  JANUS_CHECK_ARG(n_atoms >= 0 && d >= 1 && d <= kMaxDim);
+  JANUS_CHECK_ARG(n_atoms >= 0 && n_edges >= 0 && d >= 1 && d <= kMaxDim);
   JANUS_CHECK_ALIGN(d % 4 == 0);
   if (n_atoms == 0) return JANUS_OK;
-  // msg may be NULL only for a CSR without edges: it is read at
-  // [row_ptr[i], row_ptr[i+1]) only.
-  JANUS_CHECK_ARG(row_ptr && out);
+  JANUS_CHECK_ARG(row_ptr && out && (msg || n_edges == 0));
   JANUS_CHECK_ALIGN(aligned(msg, 16) && aligned(out, 16));
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
   const int64_t need = (n_atoms + 7) / 8;
   const int64_t cap = (int64_t)num_sms() * 8;
   const unsigned grid = (unsigned)(need < cap ? need : cap);
   edge_aggregate_kernel<<<grid, kThreads, 0, (cudaStream_t)stream>>>(
-      (const float4*)msg, row_ptr, n_atoms, d / 4, (float4*)out);
+      (const float4*)msg, row_ptr, n_atoms, n_edges, d / 4, (float4*)out, debug_fault_word());
   return launch_status();
 }
 
 extern "C" janus_status janus_edge_broadcast(const float* dx, const int64_t* row_ptr, int64_t n_atoms,
-                                             int32_t d, float* dmsg, janus_stream_t stream) {
-  JANUS_CHECK_ARG(n_atoms >= 0 && d >= 1 && d <= kMaxDim);
+                                             int32_t d, float* dmsg, int64_t n_edges, janus_stream_t stream) {
+  JANUS_CHECK_ARG(n_atoms >= 0 && n_edges >= 0 && d >= 1 && d <= kMaxDim);
   JANUS_CHECK_ALIGN(d % 4 == 0);
   if (n_atoms == 0) return JANUS_OK;
-  // dmsg may be NULL only for a CSR without edges
-  JANUS_CHECK_ARG(dx && row_ptr);
+  JANUS_CHECK_ARG(dx && row_ptr && (dmsg || n_edges == 0));
   JANUS_CHECK_ALIGN(aligned(dx, 16) && aligned(dmsg, 16));
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
   const int64_t need = (n_atoms + 7) / 8;
   const int64_t cap = (int64_t)num_sms() * 8;
   edge_broadcast_kernel<<<(unsigned)(need < cap ? need : cap), kThreads, 0, (cudaStream_t)stream>>>(
-      (const float4*)dx, row_ptr, n_atoms, d / 4, (float4*)dmsg);
+      (const float4*)dx, row_ptr, n_atoms, n_edges, d / 4, (float4*)dmsg, debug_fault_word());
   return launch_status();
 }
 
 extern "C" janus_status janus_neighbor_aggregate(const float* x, const int64_t* row_ptr,
-                                                 const int32_t* senders, int64_t n_atoms, int32_t d,
-                                                 float* out, janus_stream_t stream) {
-  JANUS_CHECK_ARG(n_atoms >= 0 && n_atoms < (int64_t)INT32_MAX && d >= 1 && d <= kMaxDim);
+                                                 const int32_t* senders, int64_t n_edges, int64_t n_atoms,
+                                                 int32_t d, float* out, janus_stream_t stream) {
+  JANUS_CHECK_ARG(n_atoms >= 0 && n_atoms < (int64_t)INT32_MAX && n_edges >= 0 && d >= 1 && d <= kMaxDim);
   JANUS_CHECK_ALIGN(d % 4 == 0);
   if (n_atoms == 0) return JANUS_OK;
-  // senders may be NULL only for a CSR without edges
-  JANUS_CHECK_ARG(x && row_ptr && out);
+  JANUS_CHECK_ARG(x && row_ptr && out && (senders || n_edges == 0));
   JANUS_CHECK_ALIGN(aligned(x, 16) && aligned(out, 16));
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
   const int64_t need = (n_atoms + 7) / 8;
   const int64_t cap = (int64_t)num_sms() * 8;
   neighbor_aggregate_kernel<<<(unsigned)(need < cap ? need : cap), kThreads, 0, (cudaStream_t)stream>>>(
-      (const float4*)x, row_ptr, senders, n_atoms, d / 4, (float4*)out);
+      (const float4*)x, row_ptr, senders, n_atoms, n_edges, d / 4, (float4*)out, debug_fault_word());
   return launch_status();
 }

@@ -21,6 +21,13 @@
 // Row i of (s, e) goes from sender row src_off[s][e] + i to owner row
 // dst_off[s][e] + i; the owner's rows are grouped by local expert, then sender,
 // so its expert MLP runs on recv_off[o] unchanged.
+//
+// Capacity: every receive buffer holds `cap` rows (a capacity factor times a
+// rank's fair share, chosen by the caller).  recv_off is clamped to cap, so the
+// owner's kernels never touch a row past it; a send whose owner row would be
+// at or past cap is skipped and recorded as kFaultCapacity in the send's
+// workspace error word (the layer's result is then incomplete, never an
+// out-of-bounds store).
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -41,7 +48,9 @@ struct PeerRows {          // one device pointer per rank (local or peer-mapped)
 };
 
 // One CTA: the whole layout is at most kMaxRanks x kMaxExperts entries.
-__global__ void ep_layout_kernel(const int32_t* __restrict__ counts_all, int P, int E,
+// recv_off is clamped to cap; dst_off keeps the unclamped positions (a send
+// compares them with cap).
+__global__ void ep_layout_kernel(const int32_t* __restrict__ counts_all, int P, int E, int64_t cap,
                                  int32_t* __restrict__ src_off, int32_t* __restrict__ dst_off,
                                  int32_t* __restrict__ recv_off) {
   const int El = E / P;
@@ -54,17 +63,18 @@ __global__ void ep_layout_kernel(const int32_t* __restrict__ counts_all, int P, 
     src_off[s * (E + 1) + E] = acc;
   }
   for (int o = threadIdx.x; o < P; o += blockDim.x) {
-    int32_t acc = 0;
+    int64_t acc = 0;
     for (int j = 0; j < El; ++j) {
-      recv_off[o * (El + 1) + j] = acc;
+      recv_off[o * (El + 1) + j] = (int32_t)min(acc, cap);
       for (int s = 0; s < P; ++s) acc += counts_all[s * E + o * El + j];
     }
-    recv_off[o * (El + 1) + El] = acc;
+    recv_off[o * (El + 1) + El] = (int32_t)min(acc, cap);
   }
-  __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int o = e / El, j = e - o * El;
-    int32_t acc = recv_off[o * (El + 1) + j];
+    int32_t acc = 0;        // rows of the owner's local experts before j
+    for (int jj = 0; jj < j; ++jj)
+      for (int s = 0; s < P; ++s) acc += counts_all[s * E + o * El + jj];
     for (int s = 0; s < P; ++s) {
       dst_off[s * E + e] = acc;
       acc += counts_all[s * E + e];
@@ -72,11 +82,29 @@ __global__ void ep_layout_kernel(const int32_t* __restrict__ counts_all, int P, 
   }
 }
 
-// Destination of local dispatch row p of expert e: (owner, owner row).
-__device__ __forceinline__ void ep_dest(int p, int e, int El, const int32_t* __restrict__ src_off_r,
-                                        const int32_t* __restrict__ dst_off_r, int* owner, int64_t* row) {
+// Destination of flat slot s (atom i's k-th expert): (owner, owner row), or
+// row -1 when the owner's receive buffer has no room for it (recorded as
+// kFaultCapacity) or, in debug builds, when slot_of / topk_expert hold an
+// index outside its range (recorded as kFaultIndex).  p = slot_of[s] is the
+// slot's row in this rank's local dispatch order, e = topk_expert[s].
+__device__ __forceinline__ void ep_dest(int64_t s, int64_t R, int E, int El, const int32_t* __restrict__ slot_of,
+                                        const int32_t* __restrict__ topk_expert,
+                                        const int32_t* __restrict__ src_off_r, const int32_t* __restrict__ dst_off_r,
+                                        int64_t cap, WsHeader* ws, int* owner, int64_t* row) {
+  const int32_t p = slot_of[s], e = topk_expert[s];
+  *owner = 0;
+  *row = -1;
+  if (kDebug && !(in_range(p, R) && in_range(e, E) && p >= src_off_r[e] && p < src_off_r[e + 1])) {
+    if (ws) debug_fault(&ws->error);
+    return;
+  }
+  const int64_t r = (int64_t)dst_off_r[e] + (p - src_off_r[e]);
+  if (r < 0 || r >= cap) {
+    if (ws) record_fault(ws, kFaultCapacity);
+    return;
+  }
   *owner = e / El;
-  *row = (int64_t)dst_off_r[e] + (p - src_off_r[e]);
+  *row = r;
 }
 
 // Pack-and-send: quant_pack_kernel's scatter form with the K destinations in
@@ -85,8 +113,9 @@ __global__ void __launch_bounds__(kThreads)
 ep_pack_send_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K,
                     const int32_t* __restrict__ types, int T, const int32_t* __restrict__ slot_of,
                     const int32_t* __restrict__ topk_expert, const uint32_t* __restrict__ amax_bits,
-                    const int32_t* __restrict__ src_off_r, const int32_t* __restrict__ dst_off_r, int El,
-                    PeerRows peers, float* __restrict__ scale, WsHeader* ws) {
+                    const int32_t* __restrict__ src_off_r, const int32_t* __restrict__ dst_off_r, int E, int El,
+                    int64_t cap, PeerRows peers, float* __restrict__ scale, WsHeader* ws) {
+  const int64_t R = n_atoms * K;
   extern __shared__ float s_tab[];            // [T] inverse scales, [T] scales
   float* s_inv = s_tab;
   float* s_scale = s_tab + T;
@@ -107,9 +136,10 @@ ep_pack_send_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K
     if (t < 0 || t >= T) t = 0;                // recorded by the amax pass
     const float inv = s_inv[t];
     int my_owner = 0;
-    int64_t my_row = 0;
-    if (lane < K) ep_dest(slot_of[i * K + lane], topk_expert[i * K + lane], El, src_off_r, dst_off_r, &my_owner, &my_row);
-    if (lane < K) peers.scale[my_owner][my_row] = s_scale[t];
+    int64_t my_row = -1;
+    if (lane < K)
+      ep_dest(i * K + lane, R, E, El, slot_of, topk_expert, src_off_r, dst_off_r, cap, ws, &my_owner, &my_row);
+    if (lane < K && my_row >= 0) peers.scale[my_owner][my_row] = s_scale[t];
     const float4* src = x + i * d4;
     for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
       uint2 q[kU];
@@ -127,6 +157,7 @@ ep_pack_send_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K
       for (int k = 0; k < K; ++k) {
         const int o = __shfl_sync(0xffffffffu, my_owner, k);
         const int64_t row = __shfl_sync(0xffffffffu, (long long)my_row, k);
+        if (row < 0) continue;                 // no room at the owner (same in every lane)
         uint2* dst = reinterpret_cast<uint2*>(peers.ptr[o]) + row * d4;
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
@@ -146,15 +177,16 @@ template <bool kWeighted>
 __global__ void __launch_bounds__(kThreads)
 ep_send_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K, const int32_t* __restrict__ slot_of,
                const int32_t* __restrict__ topk_expert, const float* __restrict__ w,
-               const int32_t* __restrict__ src_off_r, const int32_t* __restrict__ dst_off_r, int El,
-               PeerRows peers) {
+               const int32_t* __restrict__ src_off_r, const int32_t* __restrict__ dst_off_r, int E, int El,
+               int64_t cap, PeerRows peers, WsHeader* ws) {
   const int lane = threadIdx.x % 32;
+  const int64_t R = n_atoms * K;
   for (int64_t i = global_warp(); i < n_atoms; i += total_warps()) {
     int my_owner = 0;
-    int64_t my_row = 0;
+    int64_t my_row = -1;
     float my_w = 1.0f;
     if (lane < K) {
-      ep_dest(slot_of[i * K + lane], topk_expert[i * K + lane], El, src_off_r, dst_off_r, &my_owner, &my_row);
+      ep_dest(i * K + lane, R, E, El, slot_of, topk_expert, src_off_r, dst_off_r, cap, ws, &my_owner, &my_row);
       if (kWeighted) my_w = w[i * K + lane];
     }
     const float4* src = x + i * d4;
@@ -169,6 +201,7 @@ ep_send_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K, con
         const int o = __shfl_sync(0xffffffffu, my_owner, k);
         const int64_t row = __shfl_sync(0xffffffffu, (long long)my_row, k);
         const float wk = kWeighted ? __shfl_sync(0xffffffffu, my_w, k) : 1.0f;
+        if (row < 0) continue;                 // no room at the owner (same in every lane)
         float4* dst = reinterpret_cast<float4*>(peers.ptr[o]) + row * d4;
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
@@ -237,12 +270,16 @@ __device__ __forceinline__ int64_t sender_row(const int32_t* __restrict__ src_of
 __global__ void __launch_bounds__(kThreads)
 ep_return_kernel(const float4* __restrict__ yd, const int32_t* __restrict__ src_off,
                  const int32_t* __restrict__ dst_off, const int32_t* __restrict__ recv_off_r, int rank,
-                 int P, int E, int64_t max_rows, int d4, PeerRows peers) {
+                 int P, int E, int64_t max_rows, int d4, PeerRows peers, int32_t* dbg) {
   const int64_t n = min((int64_t)recv_off_r[E / P], max_rows);
   const int lane = threadIdx.x % 32;
   for (int64_t j = global_warp(); j < n; j += total_warps()) {
     int s;
     const int64_t row = sender_row(src_off, dst_off, recv_off_r, rank, P, E, j, &s);
+    if (kDebug && !in_range(row, src_off[s * (E + 1) + E])) {   // past the sender's routed rows
+      if (lane == 0) debug_fault(dbg);
+      continue;
+    }
     const float4* src = yd + j * d4;
     float4* dst = reinterpret_cast<float4*>(peers.ptr[s]) + row * d4;
     for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
@@ -268,12 +305,16 @@ ep_return_kernel(const float4* __restrict__ yd, const int32_t* __restrict__ src_
 __global__ void __launch_bounds__(kThreads)
 ep_return_rows_kernel(const int32_t* __restrict__ src_off, const int32_t* __restrict__ dst_off,
                       const int32_t* __restrict__ recv_off_r, int rank, int P, int E, int64_t max_rows, int d,
-                      PeerRows peers, float** __restrict__ rows) {
+                      PeerRows peers, float** __restrict__ rows, int32_t* dbg) {
   const int64_t n = min((int64_t)recv_off_r[E / P], max_rows);
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n; j += stride) {
     int s;
     const int64_t row = sender_row(src_off, dst_off, recv_off_r, rank, P, E, j, &s);
+    if (kDebug && !in_range(row, src_off[s * (E + 1) + E])) {
+      debug_fault(dbg);
+      continue;
+    }
     rows[j] = reinterpret_cast<float*>(peers.ptr[s]) + row * d;
   }
 }
@@ -308,13 +349,15 @@ janus_status peer_table(void* const* ptrs, float* const* scales, int32_t world, 
 using namespace janus;
 
 extern "C" janus_status janus_ep_layout(const int32_t* counts_all, int32_t world, int32_t n_experts,
-                                        int32_t* src_off, int32_t* dst_off, int32_t* recv_off,
+                                        int64_t recv_cap, int32_t* src_off, int32_t* dst_off, int32_t* recv_off,
                                         janus_stream_t stream) {
   janus_status st = check_ep(0, world, n_experts);
   if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(recv_cap >= 0 && recv_cap < (int64_t)INT32_MAX);
   JANUS_CHECK_ARG(counts_all && src_off && dst_off && recv_off);
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
-  ep_layout_kernel<<<1, 256, 0, (cudaStream_t)stream>>>(counts_all, world, n_experts, src_off, dst_off, recv_off);
+  ep_layout_kernel<<<1, 256, 0, (cudaStream_t)stream>>>(counts_all, world, n_experts, recv_cap, src_off, dst_off,
+                                                        recv_off);
   return launch_status();
 }
 
@@ -322,12 +365,13 @@ extern "C" janus_status janus_ep_dispatch_quant(const float* x, int64_t n_atoms,
                                                 const int32_t* types, int32_t n_types, const int32_t* slot_of,
                                                 const int32_t* topk_expert, const int32_t* src_off,
                                                 const int32_t* dst_off, int32_t rank, int32_t world,
-                                                int32_t n_experts, uint16_t* const* recv_payload,
+                                                int32_t n_experts, int64_t recv_cap, uint16_t* const* recv_payload,
                                                 float* const* recv_scale, float* scale, void* workspace,
                                                 size_t workspace_bytes, janus_stream_t stream_) {
   cudaStream_t stream = (cudaStream_t)stream_;
   janus_status st = check_ep(rank, world, n_experts);
   if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(recv_cap >= 0 && recv_cap < (int64_t)INT32_MAX);
   JANUS_CHECK_ARG(n_atoms >= 0 && top_k >= 1 && top_k <= 32 && top_k <= n_experts);
   JANUS_CHECK_ARG(d >= 1 && d <= kMaxDim && n_types >= 1 && n_types <= kMaxTypes);
   JANUS_CHECK_ALIGN(d % 4 == 0);
@@ -352,18 +396,20 @@ extern "C" janus_status janus_ep_dispatch_quant(const float* x, int64_t n_atoms,
                                                                               types, n_types, amax_bits, hdr);
   ep_pack_send_kernel<<<grid, kThreads, 2 * sizeof(float) * n_types, stream>>>(
       (const float4*)x, n_atoms, d / 4, top_k, types, n_types, slot_of, topk_expert, amax_bits,
-      src_off + (size_t)rank * (n_experts + 1), dst_off + (size_t)rank * n_experts, n_experts / world, peers,
-      scale, hdr);
+      src_off + (size_t)rank * (n_experts + 1), dst_off + (size_t)rank * n_experts, n_experts, n_experts / world,
+      recv_cap, peers, scale, hdr);
   return launch_status();
 }
 
 extern "C" janus_status janus_ep_dispatch(const float* x, int64_t n_atoms, int32_t d, int32_t top_k,
                                           const int32_t* slot_of, const int32_t* topk_expert,
                                           const float* topk_weight, const int32_t* src_off, const int32_t* dst_off,
-                                          int32_t rank, int32_t world, int32_t n_experts, float* const* recv_rows,
-                                          janus_stream_t stream) {
+                                          int32_t rank, int32_t world, int32_t n_experts, int64_t recv_cap,
+                                          float* const* recv_rows, void* workspace, janus_stream_t stream) {
   janus_status st = check_ep(rank, world, n_experts);
   if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(recv_cap >= 0 && recv_cap < (int64_t)INT32_MAX);
+  JANUS_CHECK_ALIGN(aligned(workspace, 256));
   JANUS_CHECK_ARG(n_atoms >= 0 && top_k >= 1 && top_k <= 32 && top_k <= n_experts);
   JANUS_CHECK_ARG(d >= 1 && d <= kMaxDim);
   JANUS_CHECK_ALIGN(d % 4 == 0);
@@ -378,12 +424,15 @@ extern "C" janus_status janus_ep_dispatch(const float* x, int64_t n_atoms, int32
   const unsigned grid = rows_grid(n_atoms, 8);
   const int32_t* so = src_off + (size_t)rank * (n_experts + 1);
   const int32_t* dof = dst_off + (size_t)rank * n_experts;
+  WsHeader* hdr = (WsHeader*)workspace;   // may be NULL: faults are then not recorded
   if (topk_weight)
     ep_send_kernel<true><<<grid, kThreads, 0, (cudaStream_t)stream>>>(
-        (const float4*)x, n_atoms, d / 4, top_k, slot_of, topk_expert, topk_weight, so, dof, n_experts / world, peers);
+        (const float4*)x, n_atoms, d / 4, top_k, slot_of, topk_expert, topk_weight, so, dof, n_experts,
+        n_experts / world, recv_cap, peers, hdr);
   else
     ep_send_kernel<false><<<grid, kThreads, 0, (cudaStream_t)stream>>>(
-        (const float4*)x, n_atoms, d / 4, top_k, slot_of, topk_expert, nullptr, so, dof, n_experts / world, peers);
+        (const float4*)x, n_atoms, d / 4, top_k, slot_of, topk_expert, nullptr, so, dof, n_experts,
+        n_experts / world, recv_cap, peers, hdr);
   return launch_status();
 }
 
@@ -423,7 +472,7 @@ extern "C" janus_status janus_ep_return(const float* yd, const int32_t* counts_a
   const int El = n_experts / world;
   ep_return_kernel<<<rows_grid(max_rows, 8), kThreads, 0, (cudaStream_t)stream>>>(
       (const float4*)yd, src_off, dst_off, recv_off + (size_t)rank * (El + 1), rank, world, n_experts,
-      max_rows, d / 4, peers);
+      max_rows, d / 4, peers, debug_fault_word());
   return launch_status();
 }
 
@@ -445,7 +494,8 @@ extern "C" janus_status janus_ep_return_rows(const int32_t* src_off, const int32
   const int El = n_experts / world;
   const int64_t blocks = std::min<int64_t>((max_rows + kThreads - 1) / kThreads, (int64_t)num_sms() * 8);
   ep_return_rows_kernel<<<(unsigned)blocks, kThreads, 0, (cudaStream_t)stream>>>(
-      src_off, dst_off, recv_off + (size_t)rank * (El + 1), rank, world, n_experts, max_rows, d, peers, rows);
+      src_off, dst_off, recv_off + (size_t)rank * (El + 1), rank, world, n_experts, max_rows, d, peers, rows,
+      debug_fault_word());
   return launch_status();
 }
 

@@ -61,11 +61,12 @@ void launch_simt(const simt::Args& a, cudaStream_t s) {
 }
 
 simt::Args make_args(const float* A, const float* B, int64_t bstride, float* C, float* C2,
-                     const float* aux, const int32_t* offsets, int E, int Kd, int N) {
+                     const float* aux, const int32_t* offsets, int E, int Kd, int N, int64_t rows) {
   simt::Args a;
   a.A = A; a.B = B; a.b_expert_stride = bstride; a.C = C; a.C2 = C2; a.aux = aux;
   a.aux2 = nullptr; a.C3 = nullptr; a.c_rows = nullptr;
   a.offsets = offsets; a.E = E; a.Kd = Kd; a.N = N;
+  a.rows = rows; a.dbg = debug_fault_word();
   return a;
 }
 
@@ -140,8 +141,8 @@ extern "C" janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, con
   unpack_rows_kernel<<<(unsigned)blocks, 256, 0, stream>>>((const uint2*)payload, row_scale, n_rows, d / 4,
                                                          (float4*)xd);
   const int64_t sw = (int64_t)d * h;
-  launch_simt<false, simt::kEpiSilu>(make_args(xd, w1, sw, H, act, nullptr, offsets, n_experts, d, h), stream);
-  simt::Args a2 = make_args(H, w2, sw, yd, nullptr, nullptr, offsets, n_experts, h, d);
+  launch_simt<false, simt::kEpiSilu>(make_args(xd, w1, sw, H, act, nullptr, offsets, n_experts, d, h, n_rows), stream);
+  simt::Args a2 = make_args(H, w2, sw, yd, nullptr, nullptr, offsets, n_experts, h, d, n_rows);
   a2.c_rows = yd_rows;
   launch_simt<false, simt::kEpiStore>(a2, stream);
   return launch_status();
@@ -184,8 +185,8 @@ janus_status ffn_fwd(const float* xd, const int32_t* offsets, int32_t n_experts,
     if (st != JANUS_OK) return st;
     return launch_status();
   }
-  launch_simt<false, simt::kEpiSilu>(make_args(xd, w1, sw, H, act, nullptr, offsets, n_experts, d, h), stream);
-  simt::Args a2 = make_args(H, w2, sw, yd, nullptr, nullptr, offsets, n_experts, h, d);
+  launch_simt<false, simt::kEpiSilu>(make_args(xd, w1, sw, H, act, nullptr, offsets, n_experts, d, h, n_rows), stream);
+  simt::Args a2 = make_args(H, w2, sw, yd, nullptr, nullptr, offsets, n_experts, h, d, n_rows);
   a2.c_rows = yd_rows;
   launch_simt<false, simt::kEpiStore>(a2, stream);
   return launch_status();
@@ -220,9 +221,9 @@ janus_status ffn_vjp(const float* xd, const float* gd, const float* act, const i
     return launch_status();
   }
   if (!act)
-    launch_simt<false, simt::kEpiStore>(make_args(xd, w1, sw, A, nullptr, nullptr, offsets, n_experts, d, h), stream);
-  launch_simt<true, simt::kEpiDSilu>(make_args(gd, w2, sw, dA, nullptr, A, offsets, n_experts, d, h), stream);
-  simt::Args a4 = make_args(dA, w1, sw, dxd, nullptr, nullptr, offsets, n_experts, h, d);
+    launch_simt<false, simt::kEpiStore>(make_args(xd, w1, sw, A, nullptr, nullptr, offsets, n_experts, d, h, n_rows), stream);
+  launch_simt<true, simt::kEpiDSilu>(make_args(gd, w2, sw, dA, nullptr, A, offsets, n_experts, d, h, n_rows), stream);
+  simt::Args a4 = make_args(dA, w1, sw, dxd, nullptr, nullptr, offsets, n_experts, h, d, n_rows);
   a4.c_rows = dxd_rows;
   launch_simt<true, simt::kEpiStore>(a4, stream);
   return launch_status();
@@ -329,11 +330,11 @@ extern "C" janus_status janus_expert_ffn_weight_grad(const float* xd, const floa
   }
   const int64_t sw = (int64_t)d * h;
   if (!act)
-    launch_simt<false, simt::kEpiStore>(make_args(xd, w1, sw, A, nullptr, nullptr, offsets, n_experts, d, h), stream);
-  launch_simt<true, simt::kEpiDSilu>(make_args(gd, w2, sw, dA, H, A, offsets, n_experts, d, h), stream);
-  simt::TnArgs t1{xd, dA, dw1, offsets, n_experts, d, h, 0};
+    launch_simt<false, simt::kEpiStore>(make_args(xd, w1, sw, A, nullptr, nullptr, offsets, n_experts, d, h, n_rows), stream);
+  launch_simt<true, simt::kEpiDSilu>(make_args(gd, w2, sw, dA, H, A, offsets, n_experts, d, h, n_rows), stream);
+  simt::TnArgs t1{xd, dA, dw1, offsets, n_experts, d, h, 0, n_rows, debug_fault_word()};
   simt::grouped_tn_kernel<<<num_sms() * 2, simt::kThreads, 0, stream>>>(t1);
-  simt::TnArgs t2{H, gd, dw2, offsets, n_experts, h, d, 0};
+  simt::TnArgs t2{H, gd, dw2, offsets, n_experts, h, d, 0, n_rows, debug_fault_word()};
   simt::grouped_tn_kernel<<<num_sms() * 2, simt::kThreads, 0, stream>>>(t2);
   return launch_status();
 }
@@ -402,20 +403,20 @@ extern "C" janus_status janus_expert_ffn_vjp_vjp(const float* xd, const float* g
   }
   const int64_t sw = (int64_t)d * h;
   if (!act)
-    launch_simt<false, simt::kEpiStore>(make_args(xd, w1, sw, A, nullptr, nullptr, offsets, n_experts, d, h), stream);
-  launch_simt<true, simt::kEpiStore>(make_args(gd, w2, sw, dh, nullptr, nullptr, offsets, n_experts, d, h), stream);
-  simt::Args a2 = make_args(vd, w1, sw, t1, t2, A, offsets, n_experts, d, h);
+    launch_simt<false, simt::kEpiStore>(make_args(xd, w1, sw, A, nullptr, nullptr, offsets, n_experts, d, h, n_rows), stream);
+  launch_simt<true, simt::kEpiStore>(make_args(gd, w2, sw, dh, nullptr, nullptr, offsets, n_experts, d, h, n_rows), stream);
+  simt::Args a2 = make_args(vd, w1, sw, t1, t2, A, offsets, n_experts, d, h, n_rows);
   a2.aux2 = dh;
   a2.C3 = u;
   launch_simt<false, simt::kEpiD2>(a2, stream);
-  launch_simt<false, simt::kEpiStore>(make_args(t1, w2, sw, d_gd, nullptr, nullptr, offsets, n_experts, h, d), stream);
-  launch_simt<true, simt::kEpiStore>(make_args(t2, w1, sw, d_xd, nullptr, nullptr, offsets, n_experts, h, d), stream);
+  launch_simt<false, simt::kEpiStore>(make_args(t1, w2, sw, d_gd, nullptr, nullptr, offsets, n_experts, h, d, n_rows), stream);
+  launch_simt<true, simt::kEpiStore>(make_args(t2, w1, sw, d_xd, nullptr, nullptr, offsets, n_experts, h, d, n_rows), stream);
   if (wg) {
-    simt::TnArgs g2{t1, gd, dw2, offsets, n_experts, h, d, 0};
+    simt::TnArgs g2{t1, gd, dw2, offsets, n_experts, h, d, 0, n_rows, debug_fault_word()};
     simt::grouped_tn_kernel<<<num_sms() * 2, simt::kThreads, 0, stream>>>(g2);
-    simt::TnArgs g1a{vd, u, dw1, offsets, n_experts, d, h, 0};
+    simt::TnArgs g1a{vd, u, dw1, offsets, n_experts, d, h, 0, n_rows, debug_fault_word()};
     simt::grouped_tn_kernel<<<num_sms() * 2, simt::kThreads, 0, stream>>>(g1a);
-    simt::TnArgs g1b{xd, t2, dw1, offsets, n_experts, d, h, 1};
+    simt::TnArgs g1b{xd, t2, dw1, offsets, n_experts, d, h, 1, n_rows, debug_fault_word()};
     simt::grouped_tn_kernel<<<num_sms() * 2, simt::kThreads, 0, stream>>>(g1b);
   }
   return launch_status();

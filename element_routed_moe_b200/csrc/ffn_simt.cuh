@@ -44,6 +44,8 @@ struct Args {
   int E;
   int Kd;                    // reduction length
   int N;                     // output columns
+  int64_t rows;              // rows of A and C (offsets[E] <= rows; checked in debug builds)
+  int32_t* dbg;              // debug builds: fault word for a bad offsets array
 };
 
 __device__ __forceinline__ float silu_f(float a) { return a / (1.0f + expf(-a)); }
@@ -67,10 +69,21 @@ struct TileMap {
   int start[kMaxExperts + 1];
 };
 
-__device__ __forceinline__ void build_tile_map(TileMap& tm, const int32_t* offsets, int E) {
+__device__ __forceinline__ void build_tile_map(TileMap& tm, const int32_t* offsets, int E, int64_t rows,
+                                               int32_t* dbg) {
   for (int e = threadIdx.x; e <= E; e += blockDim.x) tm.off[e] = offsets[e];
   __syncthreads();
   if (threadIdx.x == 0) {
+    if (kDebug) {
+      // offsets must be non-decreasing inside [0, rows]; otherwise every
+      // expert is treated as empty (no tile touches memory) and the fault recorded
+      bool ok = tm.off[0] >= 0 && tm.off[E] <= rows;
+      for (int e = 0; e < E; ++e) ok = ok && tm.off[e + 1] >= tm.off[e];
+      if (!ok) {
+        debug_fault(dbg);
+        for (int e = 0; e <= E; ++e) tm.off[e] = 0;
+      }
+    }
     int acc = 0;
     for (int e = 0; e < E; ++e) {
       tm.start[e] = acc;
@@ -95,7 +108,7 @@ __global__ void __launch_bounds__(kThreads, 2) grouped_gemm_kernel(Args args) {
   __shared__ __align__(16) float As[2][BK][BM];
   __shared__ __align__(16) float Bs[2][BK][BN];
   __shared__ TileMap tm;
-  build_tile_map(tm, args.offsets, args.E);
+  build_tile_map(tm, args.offsets, args.E, args.rows, args.dbg);
 
   const int tid = threadIdx.x;
   const int tx = tid % 16, ty = tid / 16;
@@ -251,6 +264,8 @@ struct TnArgs {
   const int32_t* offsets;
   int E, M, N;
   int accumulate;   // nonzero: C += X^T Y
+  int64_t rows;     // rows of X and Y (offsets[E] <= rows; checked in debug builds)
+  int32_t* dbg;     // debug builds: fault word for a bad offsets array
 };
 
 __global__ void __launch_bounds__(kThreads, 2) grouped_tn_kernel(TnArgs args) {
@@ -265,7 +280,12 @@ __global__ void __launch_bounds__(kThreads, 2) grouped_tn_kernel(TnArgs args) {
     const int e = tile / (n_tm * n_tn);
     const int rem = tile % (n_tm * n_tn);
     const int m0 = (rem / n_tn) * BM, n0 = (rem % n_tn) * BN;
-    const int p0 = args.offsets[e], p1 = args.offsets[e + 1];
+    int p0 = args.offsets[e], p1 = args.offsets[e + 1];
+    if (kDebug && !(p0 >= 0 && p1 >= p0 && p1 <= args.rows)) {
+      // a bad segment is treated as empty (zero gradient, nothing read)
+      if (tid == 0) debug_fault(args.dbg);
+      p0 = p1 = 0;
+    }
     const int nk = (p1 - p0 + BK - 1) / BK;
     float4 ra[2], rb[2];
     auto load_tile = [&](int kt) {

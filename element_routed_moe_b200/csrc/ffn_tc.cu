@@ -92,8 +92,6 @@ constexpr uint32_t kTileBBytes = BNH * BK * 4;             // 8 KB (this CTA's h
 constexpr uint32_t kStageBytes = 2 * (kTileABytes + kTileBBytes);   // raw + lo
 constexpr uint32_t kTxBytes = kTileABytes + kTileBBytes;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kFaultTimeout = 3;
-constexpr int kFaultNotTf32 = 4;    // kBExact: a B tile held bits below TF32 precision
 constexpr long long kWaitLimitCycles = 4000000000LL;     // ~2 s at 2 GHz
 
 // kEpiD2 (second-order pass, x·W): acc = v W1, aux = a, aux2 = dh;
@@ -131,7 +129,7 @@ struct Args {
   const float* aux2;
   float* const* c_rows;   // NN/NT plain store: if set, row p goes to c_rows[p] (e.g. a peer's buffer)
   const float* row_scale; // kBHalf: scale of dispatch row p
-  int64_t rows;           // kBHalf: rows of the payload (row_scale's length)
+  int64_t rows;           // rows of the dispatch operand (kBHalf: row_scale's length); offsets[E] <= rows
   const int32_t* offsets;
   int E, Kd, N;
   int M;            // kModeTN: MMA rows of each expert's product; C is [E][N][M] (stored transposed)
@@ -551,6 +549,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   }
   __syncthreads();
   if (tid == 0) {
+    if (kDebug) {
+      // offsets must be non-decreasing inside [0, rows]; otherwise every
+      // expert is treated as empty (no tile touches memory) and the fault recorded
+      bool ok = s->off[0] >= 0 && s->off[E] <= args.rows;
+      for (int e = 0; e < E; ++e) ok = ok && s->off[e + 1] >= s->off[e];
+      if (!ok) {
+        debug_fault(args.err);
+        for (int e = 0; e <= E; ++e) s->off[e] = 0;
+      }
+    }
     int acc = 0;
     for (int e = 0; e < E; ++e) {
       s->start[e] = acc;

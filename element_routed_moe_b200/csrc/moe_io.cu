@@ -43,7 +43,8 @@ template <bool kWeighted>
 __global__ void __launch_bounds__(kThreads)
 dispatch_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K,
                 const int32_t* __restrict__ slot_of, const float* __restrict__ w,
-                float4* __restrict__ xd) {
+                float4* __restrict__ xd, int32_t* dbg) {
+  const int64_t R = n_atoms * K;
   const int lane = threadIdx.x % 32;
   for (int64_t i = global_warp(); i < n_atoms; i += total_warps()) {
     const int my_slot = lane < K ? slot_of[i * K + lane] : 0;
@@ -60,6 +61,10 @@ dispatch_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K,
         int64_t p;
         float wk;
         slot_k<kWeighted>(k, K, i, my_slot, my_w, slot_of, w, &p, &wk);
+        if (kDebug && !in_range(p, R)) {   // p is the same in every lane
+          if (lane == 0) debug_fault(dbg);
+          continue;
+        }
         float4* dst = xd + p * d4;
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
@@ -79,7 +84,8 @@ template <bool kWeighted>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(const float4* __restrict__ yd, const int32_t* __restrict__ slot_of,
                const float* __restrict__ w, int64_t n_atoms, int K, int d4,
-               float4* __restrict__ y) {
+               float4* __restrict__ y, int32_t* dbg) {
+  const int64_t R = n_atoms * K;
   const int lane = threadIdx.x % 32;
   for (int64_t i = global_warp(); i < n_atoms; i += total_warps()) {
     const int my_slot = lane < K ? slot_of[i * K + lane] : 0;
@@ -92,6 +98,10 @@ combine_kernel(const float4* __restrict__ yd, const int32_t* __restrict__ slot_o
         int64_t p;
         float wk;
         slot_k<kWeighted>(k, K, i, my_slot, my_w, slot_of, w, &p, &wk);
+        if (kDebug && !in_range(p, R)) {
+          if (lane == 0) debug_fault(dbg);
+          continue;
+        }
         const float4* src = yd + p * d4;
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
@@ -127,6 +137,7 @@ quant_pack_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K,
                   const uint32_t* __restrict__ amax_bits, uint2* __restrict__ payload,
                   float* __restrict__ scale, WsHeader* ws) {
   extern __shared__ float s_inv[];
+  const int64_t R = n_atoms * K;
   for (int t = threadIdx.x; t < T; t += kThreads) {
     const uint32_t a = amax_bits[t];
     const int e = scale_exponent_from_bits(a);
@@ -161,6 +172,10 @@ quant_pack_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K,
       }
       for (int k = 0; k < K; ++k) {
         const int64_t p = K <= 32 ? __shfl_sync(0xffffffffu, my_slot, k) : slot_of[i * K + k];
+        if (kDebug && !in_range(p, R)) {
+          if (lane == 0) debug_fault(&ws->error);
+          continue;
+        }
         uint2* dst = payload + p * d4;
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
@@ -175,10 +190,15 @@ quant_pack_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K,
 __global__ void __launch_bounds__(kThreads)
 dequant_kernel(const uint2* __restrict__ payload, int64_t n_rows, int d4, int K,
                const int32_t* __restrict__ types, int T, const int32_t* __restrict__ perm,
-               const float* __restrict__ scale, float4* __restrict__ xd) {
+               const float* __restrict__ scale, float4* __restrict__ xd, int32_t* dbg) {
   const int lane = threadIdx.x % 32;
   for (int64_t p = global_warp(); p < n_rows; p += total_warps()) {
-    int t = types[perm[p] / K];
+    const int32_t slot = perm[p];
+    if (kDebug && !in_range(slot, n_rows)) {
+      if (lane == 0) debug_fault(dbg);
+      continue;
+    }
+    int t = types[slot / K];
     if (t < 0 || t >= T) t = 0;
     const float s = scale[t];
     const uint2* src = payload + p * d4;
@@ -207,10 +227,16 @@ dequant_kernel(const uint2* __restrict__ payload, int64_t n_rows, int d4, int K,
 // the dequant kernel).
 __global__ void __launch_bounds__(kThreads)
 row_scale_kernel(int64_t n_rows, int K, const int32_t* __restrict__ types, int T,
-                 const int32_t* __restrict__ perm, const float* __restrict__ scale, float* __restrict__ row_scale) {
+                 const int32_t* __restrict__ perm, const float* __restrict__ scale, float* __restrict__ row_scale,
+                 int32_t* dbg) {
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < n_rows; p += stride) {
-    int t = types[perm[p] / K];
+    const int32_t slot = perm[p];
+    if (kDebug && !in_range(slot, n_rows)) {
+      debug_fault(dbg);
+      continue;
+    }
+    int t = types[slot / K];
     if (t < 0 || t >= T) t = 0;
     row_scale[p] = scale[t];
   }
@@ -241,10 +267,10 @@ extern "C" janus_status janus_dispatch(const float* x, int64_t n_atoms, int32_t 
   const unsigned grid = rows_grid(n_atoms, 8);
   if (topk_weight)
     dispatch_kernel<true><<<grid, kThreads, 0, (cudaStream_t)stream>>>(
-        (const float4*)x, n_atoms, d / 4, top_k, slot_of, topk_weight, (float4*)xd);
+        (const float4*)x, n_atoms, d / 4, top_k, slot_of, topk_weight, (float4*)xd, debug_fault_word());
   else
     dispatch_kernel<false><<<grid, kThreads, 0, (cudaStream_t)stream>>>(
-        (const float4*)x, n_atoms, d / 4, top_k, slot_of, nullptr, (float4*)xd);
+        (const float4*)x, n_atoms, d / 4, top_k, slot_of, nullptr, (float4*)xd, debug_fault_word());
   return launch_status();
 }
 
@@ -260,10 +286,10 @@ extern "C" janus_status janus_combine(const float* yd, const int32_t* slot_of,
   const unsigned grid = rows_grid(n_atoms, 8);
   if (topk_weight)
     combine_kernel<true><<<grid, kThreads, 0, (cudaStream_t)stream>>>(
-        (const float4*)yd, slot_of, topk_weight, n_atoms, top_k, d / 4, (float4*)y);
+        (const float4*)yd, slot_of, topk_weight, n_atoms, top_k, d / 4, (float4*)y, debug_fault_word());
   else
     combine_kernel<false><<<grid, kThreads, 0, (cudaStream_t)stream>>>(
-        (const float4*)yd, slot_of, nullptr, n_atoms, top_k, d / 4, (float4*)y);
+        (const float4*)yd, slot_of, nullptr, n_atoms, top_k, d / 4, (float4*)y, debug_fault_word());
   return launch_status();
 }
 
@@ -317,7 +343,7 @@ extern "C" janus_status janus_dequant_by_type(const uint16_t* payload, int64_t n
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
   const int64_t R = n_atoms * top_k;
   dequant_kernel<<<rows_grid(R, 8), kThreads, 0, (cudaStream_t)stream>>>(
-      (const uint2*)payload, R, d / 4, top_k, types, n_types, perm, scale, (float4*)xd);
+      (const uint2*)payload, R, d / 4, top_k, types, n_types, perm, scale, (float4*)xd, debug_fault_word());
   return launch_status();
 }
 
@@ -333,7 +359,7 @@ extern "C" janus_status janus_dispatch_row_scales(int64_t n_atoms, int32_t top_k
   const int64_t R = n_atoms * top_k;
   const int64_t blocks = std::min<int64_t>((R + kThreads - 1) / kThreads, (int64_t)num_sms() * 8);
   row_scale_kernel<<<(unsigned)blocks, kThreads, 0, (cudaStream_t)stream>>>(R, top_k, types, n_types, perm, scale,
-                                                                             row_scale);
+                                                                             row_scale, debug_fault_word());
   return launch_status();
 }
 
@@ -351,11 +377,14 @@ extern "C" janus_status janus_dispatch_row_scales(int64_t n_atoms, int32_t top_k
 // 16,640 bytes, which every GPU that loads the library keeps until the
 // process exits.
 // ---------------------------------------------------------------------------
+#include <cuda.h>
+
 #include <mutex>
 #include <unordered_map>
 
 constexpr int kNoAllocMaxTypes = 4096;
 constexpr size_t kNoAllocScratchBytes = sizeof(janus::WsHeader) + sizeof(uint32_t) * kNoAllocMaxTypes;
+static_assert(kNoAllocMaxTypes <= janus::kMaxTypes, "the scratch may not admit more types than the library");
 
 // The scratch itself.  Host code must not use this name as an address (on the
 // host it is only a stand-in); the address comes from cudaGetSymbolAddress.
@@ -363,16 +392,41 @@ static __device__ __align__(256) unsigned char g_quant_noalloc_scratch[kNoAllocS
 
 namespace {
 
-std::mutex g_noalloc_mu;
-std::unordered_map<int, void*> g_noalloc_addr;   // device ordinal -> scratch address
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (CtxGetCurrentFn)p;
+  });
+  return fn;
+}
 
-// Device address of the scratch on the current device, looked up once per
-// device (cudaGetSymbolAddress may load the module on that device).
+std::mutex g_noalloc_mu;
+std::unordered_map<CUcontext, void*> g_noalloc_addr;   // CUDA context -> scratch address
+
+// Device address of the scratch in the current CUDA context, looked up once
+// per context (cudaGetSymbolAddress may load the module into it).  Keying on
+// the context, not the device ordinal, keeps a driver-API context from using
+// the primary context's address.  A context destroyed and re-created at the
+// same handle (cudaDeviceReset) is not detected.
 janus_status noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return JANUS_ERR_CUDA;
+  CtxGetCurrentFn get = ctx_get_current_fn();
+  CUcontext ctx = nullptr;
+  if (!get || get(&ctx) != CUDA_SUCCESS) return JANUS_ERR_CUDA;
+  if (ctx == nullptr) {
+    // no context is current yet: initialise the current device's primary
+    // context (cudaSetDevice does so at once and allocates no memory)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return JANUS_ERR_CUDA;
+    if (get(&ctx) != CUDA_SUCCESS || ctx == nullptr) return JANUS_ERR_CUDA;
+  }
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  auto it = g_noalloc_addr.find(dev);
+  auto it = g_noalloc_addr.find(ctx);
   if (it != g_noalloc_addr.end()) {
     *out = it->second;
     return JANUS_OK;
@@ -380,7 +434,7 @@ janus_status noalloc_scratch(void** out) {
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_quant_noalloc_scratch) != cudaSuccess || p == nullptr)
     return JANUS_ERR_CUDA;
-  g_noalloc_addr[dev] = p;
+  g_noalloc_addr[ctx] = p;
   *out = p;
   return JANUS_OK;
 }

@@ -66,9 +66,12 @@ __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib)
   return va > vb || (va == vb && ia < ib);
 }
 
+// A gate row with a non-finite logit (NaN or +-inf) has no well-defined top-K
+// and softmax: route_table records kFaultNonFinite for it (the selection it
+// makes is still a valid set of K distinct experts).
 __global__ void __launch_bounds__(kThreads)
 route_table(const float* __restrict__ gate, int32_t T, int32_t E, int32_t K,
-            int32_t* __restrict__ table_e, float* __restrict__ table_w) {
+            int32_t* __restrict__ table_e, float* __restrict__ table_w, WsHeader* ws) {
   __shared__ float sel_logit[kWarps][kMaxExperts];
   // layer blockIdx.y: gate [T,E] and tables [T,K] of that layer
   gate += (int64_t)blockIdx.y * T * E;
@@ -80,11 +83,14 @@ route_table(const float* __restrict__ gate, int32_t T, int32_t E, int32_t K,
   constexpr int kPer = kMaxExperts / 32;
   float v[kPer];
   uint32_t taken = 0;   // bit j: expert lane + 32 j already selected
+  bool finite = true;
 #pragma unroll
   for (int j = 0; j < kPer; ++j) {
     const int e = lane + 32 * j;
     v[j] = e < E ? gate[(int64_t)t * E + e] : 0.0f;
+    finite = finite && isfinite(v[j]);
   }
+  if (!__all_sync(0xffffffffu, finite) && lane == 0) record_fault(ws, kFaultNonFinite);
   for (int k = 0; k < K; ++k) {
     // lane-local best among untaken experts
     float bv = 0.0f;
@@ -328,7 +334,8 @@ static janus_status route_impl(const int32_t* types, int64_t n_atoms, const floa
     return JANUS_OK;
   }
   const unsigned nb = (unsigned)L.n_blocks, ly = (unsigned)nl;
-  route_table<<<dim3((T + kWarps - 1) / kWarps, ly), kThreads, 0, stream>>>(gates, T, E, K, table_e, table_w);
+  route_table<<<dim3((T + kWarps - 1) / kWarps, ly), kThreads, 0, stream>>>(gates, T, E, K, table_e, table_w,
+                                                                            hdr);
   route_count<<<dim3(nb, ly), kThreads, 0, stream>>>(types, n_atoms, T, E, K, table_e, table_w,
                                                       L.atoms_per_block, L.n_blocks, topk_expert,
                                                       topk_weight, blockcnt, hdr);

@@ -21,9 +21,12 @@ no separate copy kernel runs.  fused_return=False keeps the copy kernel
 (janus_ep_return) after the GEMM.
 
 Every step is a kernel of libjanus; torch.distributed carries only the
-counts, the IPC handles (once) and the phase barriers.  The receive and return
-buffers are allocated once at their worst-case size (all routed rows of all
-ranks), so no step waits for the host to learn a count.  With NCCL a barrier
+counts, the IPC handles (once) and the phase barriers.  The receive buffers
+are allocated once for capacity_factor times a rank's fair share of rows
+(N_max*K; the worst case, every rank's rows on one owner, is P times that), so
+no step waits for the host to learn a count.  Rows that would land past the
+capacity are not sent: the send kernels record a data fault, which `check()`
+raises.  With NCCL a barrier
 is a one-element all-reduce on the current stream (stream-ordered: every
 rank's send kernel has finished before any rank passes it); with gloo it is a
 stream synchronize plus a host barrier.
@@ -38,7 +41,7 @@ class ExpertParallelLayer:
     """Buffers, peer mappings and the ordered calls of one EP layer pass."""
 
     def __init__(self, n_atoms_max, d, h, n_types, n_experts, top_k, w1_local, w2_local, *,
-                 mode=J.JANUS_FFN_3XTF32, group=None, device=None, fused_return=True):
+                 mode=J.JANUS_FFN_3XTF32, group=None, device=None, fused_return=True, capacity_factor=2.0):
         self.group = group
         self.dist = dist.is_available() and dist.is_initialized()
         # without a process group the layer is a single rank owning every expert
@@ -63,10 +66,13 @@ class ExpertParallelLayer:
         # fused), and the return table (fused) or the return copy twice
         self.launches_per_step = 14 + (0 if self.fused_unpack else 1) + (1 if self.fused_return else 2)
         self.nccl = self.dist and dist.get_backend(group) == "nccl"
-        # worst case: every routed row of every rank lands on this rank
+        # receive capacity: capacity_factor x the fair share (this rank's own
+        # routed rows), never more than the worst case (every rank's rows here)
         self.n_atoms_max = int(n_atoms_max)
-        cap = max(self.world * self.n_atoms_max * top_k, 1)
         rows = max(self.n_atoms_max * top_k, 1)
+        if capacity_factor <= 0:
+            raise ValueError("capacity_factor must be positive")
+        cap = max(1, min(self.world * rows, int(-(-capacity_factor * rows // 1))))
         f32 = dict(dtype=torch.float32, device=self.dev)
         self.cap = cap
         self.payload = torch.empty((cap, d), dtype=torch.float16, device=self.dev)
@@ -78,6 +84,9 @@ class ExpertParallelLayer:
         self.ret = torch.empty((rows, d), **f32)             # this rank's rows coming back
         self.ret_rows = torch.zeros((cap,), dtype=torch.int64, device=self.dev)   # fused-return row table
         self.counts_all = torch.empty((self.world, n_experts), dtype=torch.int32, device=self.dev)
+        # error word of the sends (both directions): rows past the capacity
+        self.send_ws = torch.empty(J.janus_quant_by_type_workspace_size(n_types), dtype=torch.uint8,
+                                   device=self.dev)
         self._token = torch.zeros(1, **f32)
         self._opened = []
         self.peer_payload = self._exchange(self.payload)
@@ -124,6 +133,12 @@ class ExpertParallelLayer:
             dist.all_gather(parts, counts.cpu(), group=self.group)
             self.counts_all.copy_(torch.stack(parts))
 
+    def check(self):
+        """Raise JanusError(JANUS_ERR_DATA) if this rank's sends met a data
+        fault since the last forward (bad type ids, non-finite features, or
+        rows past an owner's receive capacity).  Synchronises the stream."""
+        J.janus_check(self.send_ws)
+
     def __enter__(self):
         return self
 
@@ -160,11 +175,11 @@ class ExpertParallelLayer:
         m(events, "route", 1)
         m(events, "layout", 0)
         self._gather_counts(self.route["counts"])
-        self.layout = J.janus_ep_layout(self.counts_all, self.E)
+        self.layout = J.janus_ep_layout(self.counts_all, self.E, self.cap)
         m(events, "layout", 1)
         m(events, "send", 0)
-        J.janus_ep_dispatch_quant(x, types, self.T, self.route, self.layout, self.rank,
-                                  self.peer_payload, self.peer_scale)
+        J.janus_ep_dispatch_quant(x, types, self.T, self.route, self.layout, self.rank, self.cap,
+                                  self.peer_payload, self.peer_scale, workspace=self.send_ws)
         self.barrier()
         m(events, "send", 1)
         recv_off = self.layout[2][self.rank]
@@ -199,7 +214,8 @@ class ExpertParallelLayer:
         m = self._mark
         r = self.route
         m(events, "send_vjp", 0)
-        J.janus_ep_dispatch(g, r, self.layout, self.rank, self.peer_rows, weighted=True)
+        J.janus_ep_dispatch(g, r, self.layout, self.rank, self.cap, self.peer_rows, weighted=True,
+                            workspace=self.send_ws)
         self.barrier()
         m(events, "send_vjp", 1)
         recv_off = self.layout[2][self.rank]

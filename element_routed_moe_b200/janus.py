@@ -16,6 +16,8 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libjanus.so")
+# the debug build (index arrays checked on the device, see janus_debug_check)
+DEBUG_LIB_PATH = os.path.join(_HERE, "libjanus_debug.so")
 
 JANUS_OK = 0
 JANUS_ERR_INVALID_ARG = 1
@@ -43,7 +45,7 @@ SYMBOLS = (
     "janus_ep_layout", "janus_ep_dispatch_quant", "janus_ep_dispatch", "janus_ep_dequant_rows",
     "janus_ep_return", "janus_ep_return_rows",
     "janus_ipc_get_handle", "janus_ipc_open_handle", "janus_ipc_close_handle",
-    "janus_debug_inject_launch_failures",
+    "janus_debug_build", "janus_debug_check", "janus_debug_inject_launch_failures",
 )
 
 
@@ -63,17 +65,34 @@ class JanusError(RuntimeError):
 
 
 _lib = None
+_loaded = {}
+
+
+def _load(path: str) -> ctypes.CDLL:
+    if path not in _loaded:
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is missing: build it with `python -m element_routed_moe_b200.build`"
+                " (nvcc, sm_100a; --debug for the debug build); there is no fallback implementation")
+        L = ctypes.CDLL(path)
+        _declare(L)
+        _loaded[path] = L
+    return _loaded[path]
 
 
 def lib() -> ctypes.CDLL:
+    """The library every wrapper here calls: libjanus.so, or the debug build
+    when the environment sets JANUS_DEBUG_LIB=1 (or after use_library)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(
-                f"{LIB_PATH} is missing: build it with `python -m element_routed_moe_b200.build`"
-                " (nvcc, sm_100a); there is no fallback implementation")
-        _lib = ctypes.CDLL(LIB_PATH)
-        _declare(_lib)
+        _lib = _load(DEBUG_LIB_PATH if os.environ.get("JANUS_DEBUG_LIB") == "1" else LIB_PATH)
+    return _lib
+
+
+def use_library(debug: bool) -> ctypes.CDLL:
+    """Route every wrapper to the debug build (True) or the release build."""
+    global _lib
+    _lib = _load(DEBUG_LIB_PATH if debug else LIB_PATH)
     return _lib
 
 
@@ -118,19 +137,21 @@ def _declare(L):
         "janus_expert_ffn_vjp_vjp": (st, [vp, vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, vp,
                                           i32, vp, sz, vp]),
         "janus_combine": (st, [vp, vp, vp, i64, i32, i32, vp, vp]),
-        "janus_edge_aggregate": (st, [vp, vp, i64, i32, vp, vp]),
-        "janus_edge_broadcast": (st, [vp, vp, i64, i32, vp, vp]),
-        "janus_neighbor_aggregate": (st, [vp, vp, vp, i64, i32, vp, vp]),
-        "janus_ep_layout": (st, [vp, i32, i32, vp, vp, vp, vp]),
-        "janus_ep_dispatch_quant": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp,
-                                         vp, sz, vp]),
-        "janus_ep_dispatch": (st, [vp, i64, i32, i32, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp]),
+        "janus_edge_aggregate": (st, [vp, i64, vp, i64, i32, vp, vp]),
+        "janus_edge_broadcast": (st, [vp, vp, i64, i32, vp, i64, vp]),
+        "janus_neighbor_aggregate": (st, [vp, vp, vp, i64, i64, i32, vp, vp]),
+        "janus_ep_layout": (st, [vp, i32, i32, i64, vp, vp, vp, vp]),
+        "janus_ep_dispatch_quant": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp, i32, i32, i32, i64, vp, vp,
+                                         vp, vp, sz, vp]),
+        "janus_ep_dispatch": (st, [vp, i64, i32, i32, vp, vp, vp, vp, vp, i32, i32, i32, i64, vp, vp, vp]),
         "janus_ep_dequant_rows": (st, [vp, vp, vp, i32, i32, i32, i64, i32, vp, vp]),
         "janus_ep_return": (st, [vp, vp, vp, vp, vp, i32, i32, i32, i64, i32, vp, vp]),
         "janus_ep_return_rows": (st, [vp, vp, vp, i32, i32, i32, i64, i32, vp, vp, vp]),
         "janus_ipc_get_handle": (st, [vp, ctypes.POINTER(IpcHandle)]),
         "janus_ipc_open_handle": (st, [ctypes.POINTER(IpcHandle), ctypes.POINTER(ctypes.c_void_p)]),
         "janus_ipc_close_handle": (st, [vp, ctypes.c_uint64]),
+        "janus_debug_build": (i32, []),
+        "janus_debug_check": (st, [vp]),
         "janus_debug_inject_launch_failures": (None, [i32]),
     }
     for name, (res, args) in sig.items():
@@ -305,9 +326,10 @@ def _ptr_array(ptrs):
     return (ctypes.c_void_p * len(vals))(*vals)
 
 
-def janus_ep_layout(counts_all, n_experts, *, src_off=None, dst_off=None, recv_off=None, stream=None):
-    """Exchange layout from the gathered counts [P, E]: (src_off [P, E+1],
-    dst_off [P, E], recv_off [P, E/P+1]), device int32."""
+def janus_ep_layout(counts_all, n_experts, recv_cap, *, src_off=None, dst_off=None, recv_off=None, stream=None):
+    """Exchange layout from the gathered counts [P, E] for receive buffers of
+    recv_cap rows: (src_off [P, E+1], dst_off [P, E], recv_off [P, E/P+1]),
+    device int32 (recv_off clamped to recv_cap)."""
     P = counts_all.shape[0]
     E = int(n_experts)
     dev = counts_all.device
@@ -317,17 +339,18 @@ def janus_ep_layout(counts_all, n_experts, *, src_off=None, dst_off=None, recv_o
         dst_off = _empty((P, E), torch.int32, dev)
     if recv_off is None:
         recv_off = _empty((P, E // max(P, 1) + 1), torch.int32, dev)
-    _raise(lib().janus_ep_layout(_p(counts_all, torch.int32, "counts_all"), P, E,
+    _raise(lib().janus_ep_layout(_p(counts_all, torch.int32, "counts_all"), P, E, int(recv_cap),
                                  _p(src_off, torch.int32, "src_off"), _p(dst_off, torch.int32, "dst_off"),
                                  _p(recv_off, torch.int32, "recv_off"), _stream(stream)), "janus_ep_layout")
     return src_off, dst_off, recv_off
 
 
-def janus_ep_dispatch_quant(x, types, n_types, route, layout, rank, recv_payload, recv_scale, *,
+def janus_ep_dispatch_quant(x, types, n_types, route, layout, rank, recv_cap, recv_payload, recv_scale, *,
                             scale=None, workspace=None, stream=None):
     """FP16-pack this rank's routed rows and store them in their owners'
-    receive buffers (recv_payload / recv_scale: one per rank, index = rank).
-    Returns (scale [T], workspace)."""
+    receive buffers of recv_cap rows (recv_payload / recv_scale: one per rank,
+    index = rank).  Returns (scale [T], workspace); janus_check(workspace)
+    reports rows that did not fit."""
     N, d = x.shape
     K = route["topk_expert"].shape[1]
     src_off, dst_off, _ = layout
@@ -340,15 +363,17 @@ def janus_ep_dispatch_quant(x, types, n_types, route, layout, rank, recv_payload
                                          int(n_types), _p(route["slot_of"], torch.int32, "slot_of"),
                                          _p(route["topk_expert"], torch.int32, "topk_expert"),
                                          _p(src_off, torch.int32, "src_off"), _p(dst_off, torch.int32, "dst_off"),
-                                         int(rank), P, E, _ptr_array(recv_payload), _ptr_array(recv_scale),
+                                         int(rank), P, E, int(recv_cap), _ptr_array(recv_payload),
+                                         _ptr_array(recv_scale),
                                          _p(scale, torch.float32, "scale"), _p(ws), nb, _stream(stream)),
            "janus_ep_dispatch_quant")
     return scale, ws
 
 
-def janus_ep_dispatch(x, route, layout, rank, recv_rows, *, weighted=False, stream=None):
+def janus_ep_dispatch(x, route, layout, rank, recv_cap, recv_rows, *, weighted=False, workspace=None, stream=None):
     """FP32 send of this rank's rows (times the gate weight when weighted) to
-    their owners' receive buffers."""
+    their owners' receive buffers of recv_cap rows; rows that do not fit are
+    recorded in workspace's error word when a workspace is given."""
     N, d = x.shape
     K = route["topk_expert"].shape[1]
     src_off, dst_off, _ = layout
@@ -357,7 +382,8 @@ def janus_ep_dispatch(x, route, layout, rank, recv_rows, *, weighted=False, stre
                                    _p(route["topk_expert"], torch.int32, "topk_expert"),
                                    _p(route["topk_weight"] if weighted else None, torch.float32, "topk_weight"),
                                    _p(src_off, torch.int32, "src_off"), _p(dst_off, torch.int32, "dst_off"),
-                                   int(rank), P, E, _ptr_array(recv_rows), _stream(stream)), "janus_ep_dispatch")
+                                   int(rank), P, E, int(recv_cap), _ptr_array(recv_rows), _p(workspace),
+                                   _stream(stream)), "janus_ep_dispatch")
 
 
 def janus_ep_dequant_rows(payload, row_scale, layout, rank, *, out=None, stream=None):
@@ -724,11 +750,12 @@ def janus_expert_ffn_vjp_vjp(xd, gd, vd, offsets, w1, w2, *, act=None, mode=JANU
 # edge aggregation
 # --------------------------------------------------------------------------
 def janus_edge_aggregate(msg, row_ptr, *, out=None, stream=None):
+    """out[i] = sum of receiver i's edge messages (msg [Ed,d], row_ptr [N+1])."""
     N = row_ptr.shape[0] - 1
-    d = msg.shape[1]
+    Ed, d = msg.shape
     if out is None:
         out = _empty((N, d), torch.float32, msg.device)
-    _raise(lib().janus_edge_aggregate(_p(msg, torch.float32, "msg"),
+    _raise(lib().janus_edge_aggregate(_p(msg, torch.float32, "msg"), Ed,
                                       _p(row_ptr, torch.int64, "row_ptr"), N, d,
                                       _p(out, torch.float32, "out"), _stream(stream)),
            "janus_edge_aggregate")
@@ -741,7 +768,7 @@ def janus_edge_broadcast(dx, row_ptr, *, out=None, stream=None):
     if out is None:
         out = _empty((int(row_ptr[-1].item()) if row_ptr.numel() else 0, d), torch.float32, dx.device)
     _raise(lib().janus_edge_broadcast(_p(dx, torch.float32, "dx"), _p(row_ptr, torch.int64, "row_ptr"),
-                                      N, d, _p(out, torch.float32, "dmsg"), _stream(stream)),
+                                      N, d, _p(out, torch.float32, "dmsg"), out.shape[0], _stream(stream)),
            "janus_edge_broadcast")
     return out
 
@@ -752,10 +779,21 @@ def janus_neighbor_aggregate(x, row_ptr, senders, *, out=None, stream=None):
     if out is None:
         out = _empty((N, d), torch.float32, x.device)
     _raise(lib().janus_neighbor_aggregate(_p(x, torch.float32, "x"), _p(row_ptr, torch.int64, "row_ptr"),
-                                          _p(senders, torch.int32, "senders"), N, d,
+                                          _p(senders, torch.int32, "senders"), senders.shape[0], N, d,
                                           _p(out, torch.float32, "out"), _stream(stream)),
            "janus_neighbor_aggregate")
     return out
+
+
+def janus_debug_build() -> bool:
+    """True when the loaded library is the debug build."""
+    return bool(lib().janus_debug_build())
+
+
+def janus_debug_check(stream=None):
+    """Raise JanusError(JANUS_ERR_DATA) if a call without a workspace found a
+    bad index since the last check (debug build; never in the release build)."""
+    _raise(lib().janus_debug_check(_stream(stream)), "janus_debug_check")
 
 
 def janus_debug_inject_launch_failures(n_calls: int):

@@ -30,12 +30,16 @@
  *   - Arguments are checked before anything is launched: a failed check
  *     returns an error and launches nothing.  Index arrays that a call takes
  *     as input (perm, slot_of, offsets, row_ptr) must be what janus_route /
- *     a valid CSR would produce; they are not re-validated on the device.
- *   - Data-dependent faults (a type id outside [0,T), a non-finite feature
- *     to be packed, a bounded tensor-core wait that ran out, rows that break
- *     JANUS_FFN_X_DEQUANTIZED) are recorded in the workspace's error word and reported
- *     by janus_check(); the call still writes every output (bad type ids are
- *     treated as type 0) so no out-of-bounds access can follow.
+ *     a valid CSR would produce; the release build does not re-validate them
+ *     on the device (edge ranges are clamped), the debug build does (see
+ *     janus_debug_check).
+ *   - Data-dependent faults (a type id outside [0,T), a non-finite gate
+ *     logit, a non-finite feature to be packed, a bounded tensor-core wait
+ *     that ran out, rows that break JANUS_FFN_X_DEQUANTIZED, expert-parallel
+ *     rows beyond the receive capacity) are recorded in the workspace's error
+ *     word and reported by janus_check(); the call still writes every output
+ *     (bad type ids are treated as type 0) so no out-of-bounds access can
+ *     follow.
  */
 #ifndef JANUS_H_
 #define JANUS_H_
@@ -88,7 +92,9 @@ janus_status janus_check(const void* workspace, janus_stream_t stream);
  * out: topk_expert [N,K] int32, topk_weight [N,K] float32, counts [E] int32,
  *      offsets [E+1] int32, perm [R] int32, slot_of [R] int32
  * workspace: janus_route_workspace_size() bytes; its error word records type
- *      ids outside [0,T) (those atoms are routed as type 0).
+ *      ids outside [0,T) (those atoms are routed as type 0) and gate rows
+ *      holding a non-finite logit (their top-K is still K distinct experts,
+ *      but its order and weights are undefined).
  * N == 0 is allowed (counts and offsets are zeroed).
  * ------------------------------------------------------------------------- */
 janus_status janus_route_workspace_size(int64_t n_atoms, int32_t n_types,
@@ -171,9 +177,12 @@ janus_status janus_quant_by_type(const float* x, int64_t n_atoms, int32_t d, int
  * (a 256-byte header plus one 32-bit word per element type), which every GPU
  * that loads the library keeps until the process exits.
  *   - n_types must be <= 4096; larger values return JANUS_ERR_INVALID_ARG.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, once per device, with that device current); make
- *     that first call before any stream capture.
+ *   - The first call in each CUDA context (the device's primary context, or
+ *     a context the caller created with the driver API) looks up the array's
+ *     device address there (cudaGetSymbolAddress, once per context, with
+ *     that context current); make that first call before any stream capture.
+ *     The cached address does not survive cudaDeviceReset: after a reset,
+ *     do not call this entry point again in the same process.
  *   - Every call clears and reuses the same array, so calls whose work
  *     overlaps on the GPU (different streams, or different host threads on one
  *     device) race and may produce wrong scales; serialise them.
@@ -346,11 +355,19 @@ janus_status janus_expert_ffn_vjp_vjp(const float* xd, const float* gd, const fl
  *                    local dispatch order; equals its janus_route offsets)
  *   recv_off [P,E/P+1]: owner o's rows per local expert, summed over senders
  *                    (o's receive buffer: grouped by local expert, then sender;
- *                    the expert MLP runs on recv_off[o] directly)
- *   dst_off [P,E]:  dst_off[s][e] = recv_off[owner(e)][e - owner(e)*E/P]
- *                    + sum_{s'<s} counts_all[s'][e]
+ *                    the expert MLP runs on recv_off[o] directly), each entry
+ *                    clamped to recv_cap
+ *   dst_off [P,E]:  dst_off[s][e] = (unclamped) rows of owner(e)'s local
+ *                    experts before e + sum_{s'<s} counts_all[s'][e]
  * Row i of (s, e) moves from sender row src_off[s][e] + i to owner row
  * dst_off[s][e] + i, and back.
+ *
+ * Capacity: every rank's receive buffers hold recv_cap rows (the caller picks
+ * it, e.g. a capacity factor times the fair share N*K; the worst case is
+ * P*N*K).  A send whose owner row would be at or past recv_cap is skipped and
+ * recorded as a data fault (JANUS_ERR_DATA from janus_check on the send's
+ * workspace): no call ever stores past recv_cap, and the owner's kernels see
+ * at most recv_cap rows.  The layer's output is then incomplete.
  *
  * The send and return calls store straight into the other ranks' buffers:
  * the pointer arrays (host arrays of P device pointers, index = rank) hold the
@@ -364,9 +381,10 @@ janus_status janus_expert_ffn_vjp_vjp(const float* xd, const float* gd, const fl
  * ------------------------------------------------------------------------- */
 #define JANUS_EP_MAX_RANKS 8
 
-/* One CTA; writes src_off, dst_off, recv_off (device int32, layouts above). */
+/* One CTA; writes src_off, dst_off, recv_off (device int32, layouts above)
+ * for receive buffers of recv_cap rows (0 <= recv_cap < 2^31). */
 janus_status janus_ep_layout(const int32_t* counts_all, int32_t world, int32_t n_experts,
-                             int32_t* src_off, int32_t* dst_off, int32_t* recv_off,
+                             int64_t recv_cap, int32_t* src_off, int32_t* dst_off, int32_t* recv_off,
                              janus_stream_t stream);
 
 /* Forward send with the FP16 packing of janus_quant_by_type (this rank's
@@ -374,24 +392,29 @@ janus_status janus_ep_layout(const int32_t* counts_all, int32_t world, int32_t n
  * this rank's atoms i and k < K, with e = topk_expert[i*K+k] and
  * p = slot_of[i*K+k], owner o = e/(E/P), row r = dst_off[rank][e] + p -
  * src_off[rank][e]:  recv_payload[o][r,:] = fp16(x[i,:] / scale[types[i]]),
- * recv_scale[o][r] = scale[types[i]].  recv_payload[o]: 8-byte aligned.
- * workspace: janus_quant_by_type_workspace_size(n_types) bytes; bad type ids
- * and non-finite rows are reported by janus_check as in janus_quant_by_type. */
+ * recv_scale[o][r] = scale[types[i]], for every r < recv_cap (the owner's
+ * receive capacity, as given to janus_ep_layout).  recv_payload[o]: 8-byte
+ * aligned.  workspace: janus_quant_by_type_workspace_size(n_types) bytes
+ * (cleared by the call); bad type ids, non-finite rows and rows past recv_cap
+ * are reported by janus_check. */
 janus_status janus_ep_dispatch_quant(const float* x, int64_t n_atoms, int32_t d, int32_t top_k,
                                      const int32_t* types, int32_t n_types, const int32_t* slot_of,
                                      const int32_t* topk_expert, const int32_t* src_off,
                                      const int32_t* dst_off, int32_t rank, int32_t world,
-                                     int32_t n_experts, uint16_t* const* recv_payload,
+                                     int32_t n_experts, int64_t recv_cap, uint16_t* const* recv_payload,
                                      float* const* recv_scale, float* scale, void* workspace,
                                      size_t workspace_bytes, janus_stream_t stream);
 
 /* FP32 send (the gradient direction): recv_rows[o][r,:] = w * x[i,:] with
- * w = topk_weight[i*K+k] (1 when topk_weight is NULL), same (o, r) as above. */
+ * w = topk_weight[i*K+k] (1 when topk_weight is NULL), same (o, r) as above,
+ * r < recv_cap.  workspace: NULL, or a 256-byte aligned workspace whose error
+ * word receives a row past recv_cap (it is not cleared by this call, so the
+ * forward send's workspace can collect both directions). */
 janus_status janus_ep_dispatch(const float* x, int64_t n_atoms, int32_t d, int32_t top_k,
                                const int32_t* slot_of, const int32_t* topk_expert,
                                const float* topk_weight, const int32_t* src_off, const int32_t* dst_off,
-                               int32_t rank, int32_t world, int32_t n_experts, float* const* recv_rows,
-                               janus_stream_t stream);
+                               int32_t rank, int32_t world, int32_t n_experts, int64_t recv_cap,
+                               float* const* recv_rows, void* workspace, janus_stream_t stream);
 
 /* Owner side of the FP16 send: xd[r,:] = f32(payload[r,:]) * row_scale[r] for
  * r < recv_off[rank][E/P] (read on the device; at most max_rows). */
@@ -451,28 +474,64 @@ janus_status janus_combine(const float* yd, const int32_t* slot_of, const float*
  * aggregation with fused indexing, edge aggregation): edge messages are
  * reduced into their receiver atoms.  Segment sum over a receiver-sorted CSR:
  *   out[i,:] = sum_{e in [row_ptr[i], row_ptr[i+1])} msg[e,:]   (0 if empty)
- * in : msg [Ed,d] float32 (Ed = row_ptr[N]; may be NULL only when Ed == 0),
- *      row_ptr [N+1] int64 (row_ptr[0] = 0, non-decreasing);  out: out [N,d] float32
+ * in : msg [Ed,d] float32 with Ed = n_edges (NULL is accepted only when
+ *      n_edges == 0), row_ptr [N+1] int64 (non-decreasing, row_ptr[N] -
+ *      row_ptr[0] = n_edges);  out: out [N,d] float32.
+ * Message row 0 is edge row_ptr[0] (0 for a whole CSR), so a range of
+ * receivers [i0, i1) of a larger CSR is aggregated by passing row_ptr + i0,
+ * N = i1 - i0 and the messages of edges [row_ptr[i0], row_ptr[i1]).
+ * Every edge range is clamped to [0, n_edges], so a malformed row_ptr cannot
+ * make the kernel read outside msg (the debug build also reports it through
+ * janus_debug_check).  A NULL msg with n_edges > 0 is JANUS_ERR_INVALID_ARG.
  * ------------------------------------------------------------------------- */
-janus_status janus_edge_aggregate(const float* msg, const int64_t* row_ptr, int64_t n_atoms,
-                                  int32_t d, float* out, janus_stream_t stream);
+janus_status janus_edge_aggregate(const float* msg, int64_t n_edges, const int64_t* row_ptr,
+                                  int64_t n_atoms, int32_t d, float* out, janus_stream_t stream);
 
 /* Gradient of the edge aggregation (same passage): every edge of receiver i
  * receives that atom's gradient row,  dmsg[e,:] = dx[i,:]  for e in
- * [row_ptr[i], row_ptr[i+1]).  in : dx [N,d], row_ptr [N+1];  out: dmsg [Ed,d]
- * (may be NULL only when Ed == 0). */
+ * [row_ptr[i], row_ptr[i+1]).  in : dx [N,d], row_ptr [N+1];  out: dmsg
+ * [Ed,d] with Ed = n_edges (NULL accepted only when n_edges == 0; a NULL dmsg
+ * with n_edges > 0 is JANUS_ERR_INVALID_ARG).  As in janus_edge_aggregate,
+ * dmsg row 0 is edge row_ptr[0] and edge ranges are clamped to [0, n_edges]. */
 janus_status janus_edge_broadcast(const float* dx, const int64_t* row_ptr, int64_t n_atoms,
-                                  int32_t d, float* dmsg, janus_stream_t stream);
+                                  int32_t d, float* dmsg, int64_t n_edges, janus_stream_t stream);
 
 /* Neighbour aggregation with fused indexing ([Review] section 3.5, CNIS
  * kernels): node features are gathered through the sender index instead of a
  * materialised message buffer,
  *   out[i,:] = sum_{e in [row_ptr[i], row_ptr[i+1])} x[senders[e], :]
- * in : x [N,d] float32, row_ptr [N+1] int64, senders [Ed] int32 (may be NULL
- * only when Ed == 0);  out: out [N,d].  Sender ids outside [0,N) are skipped
- * (they add nothing).  N < 2^31. */
+ * in : x [N,d] float32, row_ptr [N+1] int64, senders [Ed] int32 with Ed =
+ * n_edges (NULL accepted only when n_edges == 0; a NULL senders with
+ * n_edges > 0 is JANUS_ERR_INVALID_ARG);  out: out [N,d].  Sender ids outside
+ * [0,N) are skipped (they add nothing; the debug build reports them).  As in
+ * janus_edge_aggregate, senders[0] is edge row_ptr[0] and edge ranges are
+ * clamped to [0, n_edges].  N < 2^31. */
 janus_status janus_neighbor_aggregate(const float* x, const int64_t* row_ptr, const int32_t* senders,
-                                      int64_t n_atoms, int32_t d, float* out, janus_stream_t stream);
+                                      int64_t n_edges, int64_t n_atoms, int32_t d, float* out,
+                                      janus_stream_t stream);
+
+/* -------------------------------------------------------------------------
+ * Debug build.  The library built with -DJANUS_DEBUG (libjanus_debug.so)
+ * checks, on the device and before using them, the index arrays that calls
+ * take as input: slot_of and perm in [0, R), offsets non-decreasing from 0
+ * with offsets[E] <= R, row_ptr non-decreasing inside [0, n_edges], senders in
+ * [0, N), and the expert-parallel tables.  A kernel that finds a bad index
+ * records a data fault and skips that access, so a corrupted index array
+ * cannot make it read or write outside its buffers.  Calls with a workspace
+ * record the fault there (janus_check); calls without one record it in the
+ * library's per-GPU debug fault word, which janus_debug_check reads.  Both
+ * builds export the same symbols; the release build records nothing in the
+ * debug word.
+ * ------------------------------------------------------------------------- */
+
+/* 1 for the debug build, 0 for the release build. */
+int32_t janus_debug_build(void);
+
+/* Synchronises `stream`, then reads and clears the debug fault word of the
+ * current device.  JANUS_ERR_DATA if a call without a workspace found a bad
+ * index since the last check, else JANUS_OK (always JANUS_OK in the release
+ * build); JANUS_ERR_CUDA if a CUDA call failed. */
+janus_status janus_debug_check(janus_stream_t stream);
 
 /* Host-side fault injection for tests: the next `n_calls` library calls that
  * would launch work return JANUS_ERR_CUDA before launching anything. */

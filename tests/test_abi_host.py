@@ -138,9 +138,16 @@ def test_argument_validation_before_launch(J):
     assert L.janus_ep_return_rows(FAKE, FAKE, FAKE, 0, 2, 4, 10, 6, two, FAKE, null) == J.JANUS_ERR_MISALIGNED
     assert L.janus_ep_return_rows(FAKE, FAKE, FAKE, 0, 2, 4, 10, 8, two, FAKE + 4, null) == J.JANUS_ERR_MISALIGNED
     assert L.janus_ep_return_rows(FAKE, FAKE, FAKE, 0, 2, 4, 0, 8, two, null, null) == J.JANUS_OK
-    # edge aggregate
-    assert L.janus_edge_aggregate(FAKE, null, 10, 8, FAKE, null) == J.JANUS_ERR_INVALID_ARG
-    assert L.janus_edge_aggregate(FAKE, FAKE, 10, 10, FAKE, null) == J.JANUS_ERR_MISALIGNED
+    # edge aggregate: null row_ptr, d % 4, and a null message / gradient /
+    # sender array while the CSR has edges (only an edge-free CSR may pass NULL)
+    assert L.janus_edge_aggregate(FAKE, 100, null, 10, 8, FAKE, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_edge_aggregate(FAKE, 100, FAKE, 10, 10, FAKE, null) == J.JANUS_ERR_MISALIGNED
+    assert L.janus_edge_aggregate(null, 100, FAKE, 10, 8, FAKE, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_edge_aggregate(FAKE, -1, FAKE, 10, 8, FAKE, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_edge_broadcast(FAKE, FAKE, 10, 8, null, 100, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_edge_broadcast(FAKE, null, 10, 8, FAKE, 100, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_neighbor_aggregate(FAKE, FAKE, null, 100, 10, 8, FAKE, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_neighbor_aggregate(FAKE, FAKE, FAKE, 100, 10, 6, FAKE, null) == J.JANUS_ERR_MISALIGNED
     # janus_check needs a workspace
     assert L.janus_check(null, null) == J.JANUS_ERR_INVALID_ARG
 
@@ -159,8 +166,14 @@ def test_empty_inputs_are_no_ops(J):
     # n_atoms == 0: nothing to launch, nothing dereferenced
     assert L.janus_dispatch(None, 0, 8, 2, None, None, None, None) == J.JANUS_OK
     assert L.janus_combine(None, None, None, 0, 2, 8, None, None) == J.JANUS_OK
-    assert L.janus_edge_aggregate(None, None, 0, 8, None, None) == J.JANUS_OK
+    assert L.janus_edge_aggregate(None, 0, None, 0, 8, None, None) == J.JANUS_OK
+    assert L.janus_edge_broadcast(None, None, 0, 8, None, 0, None) == J.JANUS_OK
+    assert L.janus_neighbor_aggregate(None, None, None, 0, 0, 8, None, None) == J.JANUS_OK
     assert L.janus_dequant_by_type(None, 0, 8, 2, None, 4, None, None, None, None) == J.JANUS_OK
+
+
+def test_release_build_reports_no_debug_faults(J):
+    assert J.janus_debug_build() is False
 
 
 def test_product_path_has_no_oracle_dependency():

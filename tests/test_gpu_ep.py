@@ -35,19 +35,21 @@ def _shards(P, N, T, d, seed):
 def _ep_pass(shards, gate, K, w1, w2, mode, grads=None, fused=False):
     """Forward (and with grads, the input VJP) of the emulated EP layer.  With
     fused, each owner's expert MLP stores its output rows straight into the
-    senders' return buffers through the janus_ep_return_rows table."""
+    senders' return buffers through the janus_ep_return_rows table.  The
+    receive buffers hold the worst case (every rank's rows on one owner)."""
     P = len(shards)
     T, E = gate.shape
     El = E // P
     d = shards[0][0].shape[1]
     routes = [J.janus_route(t, gate, K) for _, t in shards]
     counts_all = torch.stack([r["counts"] for r in routes]).contiguous()
-    layout = J.janus_ep_layout(counts_all, E)
     cap = sum(x.shape[0] for x, _ in shards) * K
+    layout = J.janus_ep_layout(counts_all, E, cap)
     payload = [torch.full((cap, d), float("nan"), dtype=torch.float16, device=DEV) for _ in range(P)]
     rscale = [torch.full((cap,), float("nan"), device=DEV) for _ in range(P)]
     for s, (x, t) in enumerate(shards):
-        J.janus_ep_dispatch_quant(x, t, T, routes[s], layout, s, payload, rscale)
+        _, ws = J.janus_ep_dispatch_quant(x, t, T, routes[s], layout, s, cap, payload, rscale)
+        J.janus_check(ws)
     recv_off = layout[2]
     # a rank without atoms still passes a (never written) buffer
     ret = [torch.full((max(x.shape[0] * K, 1), d), float("nan"), device=DEV) for x, _ in shards]
@@ -74,7 +76,7 @@ def _ep_pass(shards, gate, K, w1, w2, mode, grads=None, fused=False):
         return ys, routes, layout
     g_recv = [torch.full((cap, d), float("nan"), device=DEV) for _ in range(P)]
     for s in range(P):
-        J.janus_ep_dispatch(grads[s], routes[s], layout, s, g_recv, weighted=True)
+        J.janus_ep_dispatch(grads[s], routes[s], layout, s, cap, g_recv, weighted=True)
     for o in range(P):
         w1o, w2o = w1[o * El:(o + 1) * El].contiguous(), w2[o * El:(o + 1) * El].contiguous()
         if fused:
@@ -168,8 +170,8 @@ def test_return_row_table_follows_the_layout():
     shards = _shards(P, N, T, d, 400)
     routes = [J.janus_route(t, gate, K) for _, t in shards]
     counts_all = torch.stack([r["counts"] for r in routes]).contiguous()
-    layout = J.janus_ep_layout(counts_all, E)
     cap = sum(x.shape[0] for x, _ in shards) * K
+    layout = J.janus_ep_layout(counts_all, E, cap)
     ret = [torch.empty((x.shape[0] * K, d), device=DEV) for x, _ in shards]
     src_off, dst_off, recv_off = oracle.ep_layout(np.stack([host(r["counts"]) for r in routes]))
     El = E // P
@@ -220,11 +222,11 @@ def test_ep_send_places_rows_by_the_layout():
     shards = _shards(P, N, T, d, 200)
     routes = [J.janus_route(t, gate, K) for _, t in shards]
     counts_all = torch.stack([r["counts"] for r in routes]).contiguous()
-    layout = J.janus_ep_layout(counts_all, E)
     cap = sum(x.shape[0] for x, _ in shards) * K
+    layout = J.janus_ep_layout(counts_all, E, cap)
     recv = [torch.full((cap, d), float("nan"), device=DEV) for _ in range(P)]
     for s, (x, _) in enumerate(shards):
-        J.janus_ep_dispatch(x, routes[s], layout, s, recv, weighted=False)
+        J.janus_ep_dispatch(x, routes[s], layout, s, cap, recv, weighted=False)
     torch.cuda.synchronize()
     src_off, dst_off, recv_off = (host(a) for a in layout)
     El = E // P
@@ -257,7 +259,54 @@ def test_ep_argument_checks():
     E = 9
     counts = torch.zeros((2, E), dtype=torch.int32, device=DEV)
     with pytest.raises(J.JanusError) as e:
-        J.janus_ep_layout(counts, E)                        # 9 experts over 2 ranks
+        J.janus_ep_layout(counts, E, 100)                   # 9 experts over 2 ranks
     assert e.value.status == J.JANUS_ERR_INVALID_ARG
     with pytest.raises(J.JanusError):
-        J.janus_ep_layout(torch.zeros((9, 72), dtype=torch.int32, device=DEV), 72)   # > 8 ranks
+        J.janus_ep_layout(torch.zeros((9, 72), dtype=torch.int32, device=DEV), 72, 100)   # > 8 ranks
+    with pytest.raises(J.JanusError):
+        J.janus_ep_layout(torch.zeros((2, 8), dtype=torch.int32, device=DEV), 8, -1)     # negative capacity
+
+
+def test_ep_capacity_overflow_is_reported_and_stays_in_bounds():
+    # P = 8 emulated ranks with receive buffers smaller than the busiest
+    # owner's rows: the sends skip what does not fit and record a data fault;
+    # guard rows past the capacity stay untouched, recv_off is clamped, and
+    # every owner row below the capacity holds what the unbounded layout puts there
+    P, N, T, E, K, d = 8, 200, 89, 16, 4, 24
+    gate = to_dev(synth.gate_table(T, E, 8))
+    shards = _shards(P, N, T, d, 600)
+    routes = [J.janus_route(t, gate, K) for _, t in shards]
+    counts_all = torch.stack([r["counts"] for r in routes]).contiguous()
+    full = sum(x.shape[0] for x, _ in shards) * K
+    _, _, recv_ref = oracle.ep_layout(host(counts_all))
+    busiest = int(recv_ref[:, -1].max())
+    cap = busiest - 37                                    # the busiest owner overflows
+    guard = 64
+    lay_full = J.janus_ep_layout(counts_all, E, full)
+    lay = J.janus_ep_layout(counts_all, E, cap)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(lay[2]), np.minimum(recv_ref, cap))
+    assert np.array_equal(host(lay[0]), host(lay_full[0])) and np.array_equal(host(lay[1]), host(lay_full[1]))
+    pay = [torch.full((cap + guard, d), float("nan"), dtype=torch.float16, device=DEV) for _ in range(P)]
+    rsc = [torch.full((cap + guard,), float("nan"), device=DEV) for _ in range(P)]
+    rows = [torch.full((cap + guard, d), float("nan"), device=DEV) for _ in range(P)]
+    pay_f = [torch.full((full, d), float("nan"), dtype=torch.float16, device=DEV) for _ in range(P)]
+    rsc_f = [torch.full((full,), float("nan"), device=DEV) for _ in range(P)]
+    faults = 0
+    for s, (x, t) in enumerate(shards):
+        _, ws = J.janus_ep_dispatch_quant(x, t, T, routes[s], lay, s, cap, pay, rsc)
+        J.janus_ep_dispatch(x, routes[s], lay, s, cap, rows, weighted=True, workspace=ws)
+        try:
+            J.janus_check(ws)
+        except J.JanusError as err:
+            assert err.status == J.JANUS_ERR_DATA
+            faults += 1
+        J.janus_ep_dispatch_quant(x, t, T, routes[s], lay_full, s, full, pay_f, rsc_f)
+    torch.cuda.synchronize()
+    assert faults >= 1
+    for o in range(P):
+        assert torch.isnan(pay[o][cap:].float()).all() and torch.isnan(rsc[o][cap:]).all(), o
+        assert torch.isnan(rows[o][cap:]).all(), o
+        n = min(int(recv_ref[o, -1]), cap)
+        assert torch.equal(pay[o][:n].view(torch.int16), pay_f[o][:n].view(torch.int16)), o
+        assert torch.equal(rsc[o][:n], rsc_f[o][:n]), o

@@ -89,6 +89,26 @@ def test_route_zero_atoms():
     assert np.all(host(r["counts"]) == 0) and np.all(host(r["offsets"]) == 0)
 
 
+@pytest.mark.parametrize("bad", [float("nan"), float("inf"), -float("inf")])
+def test_route_non_finite_gate_logit_sets_data_error(bad):
+    # a gate row with a non-finite logit has no defined top-K: reported as a
+    # data fault, while the selection stays K distinct valid experts
+    gate = synth.gate_table(3, 6, 1)
+    gate[1, 4] = bad
+    types = np.array([1, 0, 2, 1], np.int32)
+    r = J.janus_route(to_dev(types), to_dev(gate), 3)
+    with pytest.raises(J.JanusError) as e:
+        J.janus_check(r["workspace"])
+    assert e.value.status == J.JANUS_ERR_DATA
+    te = host(r["topk_expert"])
+    assert ((te >= 0) & (te < 6)).all()
+    assert all(len(set(row)) == 3 for row in te)
+    assert np.array_equal(np.sort(host(r["perm"])), np.arange(12))
+    # the finite rows are routed as usual
+    o = oracle.route(np.array([0, 2], np.int32), np.where(np.isfinite(gate), gate, 0).astype(np.float32), 3)
+    assert np.array_equal(te[[1, 2]], o["topk_expert"])
+
+
 def test_route_bad_type_sets_data_error():
     gate = synth.gate_table(4, 6, 0)
     types = np.array([0, 1, 7, 2, -3], np.int32)

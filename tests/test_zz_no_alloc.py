@@ -64,6 +64,14 @@ def test_noalloc_binding_and_limits():
     ref_p, ref_s, _ = J.janus_quant_by_type(x, types, T, slot_of, K)
     torch.cuda.synchronize()
     assert torch.equal(s, ref_s) and torch.equal(p.view(torch.int16), ref_p.view(torch.int16))
+    # the largest type count the scratch holds is accepted and packs bit for bit
+    T_max = 4096
+    types_w = torch.as_tensor(synth.types_uniform(x.shape[0], T_max, 21), device=DEV)
+    p4, s4 = J.janus_quant_by_type_noalloc(x, types_w, T_max, slot_of, K)
+    ref_p4, ref_s4, ws4 = J.janus_quant_by_type(x, types_w, T_max, slot_of, K)
+    J.janus_check(ws4)
+    torch.cuda.synchronize()
+    assert torch.equal(s4, ref_s4) and torch.equal(p4.view(torch.int16), ref_p4.view(torch.int16))
     # more element types than the library-owned scratch holds: rejected before any launch
     big_scale = torch.empty(4097, dtype=torch.float32, device=DEV)
     st = J.lib().janus_quant_by_type_noalloc(x.data_ptr(), x.shape[0], x.shape[1], K, types.data_ptr(),
