@@ -8,13 +8,17 @@ interaction-block slice) and the per-element-type FP16 packing (quant ->
 dequant) in place of the dispatch where it packs (M, the slice).
 
 Metric: routed atom-expert tokens/s (tokens = N*K routed rows) per layer pass.
-Default workload: MatRIS-MoE(S)-shaped layer (N=8192, T=89 Zipf(1.1), E=72,
-K=4, d=h=2560), model table of the paper review 'Breaking the Training
-Barrier of Billion-Parameter Universal Machine Learning Interatomic
-Potentials', section 3.1 Table II.
+Default workload: the interaction-block slice at the MatRIS-MoE(M) shape
+(N=65,536 atoms in a periodic cell at 0.08 atoms/A^3, 6 A cutoff, ~4.74 M
+edges with d=1536 messages -> edge aggregation -> route -> FP16-packed
+dispatch -> expert MLP fwd + input VJP -> combine; T=89 Zipf(1.1), E=40, K=8,
+d=h=1536), the largest configuration that fits one GPU and the only one that
+chains every step.  Shapes: model table of the paper review 'Breaking the
+Training Barrier of Billion-Parameter Universal Machine Learning Interatomic
+Potentials', section 3.1 Table II; block order: section 3.4 Figure 3.
 
 Usage:
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload S|M|L|slice|tiny]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload slice|S|M|L|tiny]
                   [--mode simt|3xtf32] [--impl janus|reference] [--no-cpu-baseline]
 Multi-GPU (weak scaling, one independent layer per rank, no collective on the
 data path): python -m torch.distributed.run --nproc-per-node N bench.py --gpus N
@@ -51,11 +55,12 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="S", choices=list(synth.CONFIGS))
+    ap.add_argument("--workload", default="slice", choices=list(synth.CONFIGS))
     ap.add_argument("--mode", default="3xtf32", choices=["simt", "3xtf32"])
     ap.add_argument("--impl", default="janus", choices=["janus", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cold", action="store_true", help="skip the cold-L2 timing of the memory-bound kernels")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--atoms", type=int, default=None, help="override N (profiling small cases)")
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling small cases)")
@@ -136,65 +141,92 @@ def describe(cfg) -> dict:
 # clocks sampled during the timed region
 # --------------------------------------------------------------------------
 class ClockSampler:
-    Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons of one GPU, sampled every
+    `period` seconds by a host thread through NVML (nvidia-smi's own query as
+    a fallback) while the timed region runs.  Only samples taken inside the
+    timed window are summarised: reading the settings, never changing them."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    def __init__(self, uuid: str | None, index: int, period: float = 0.02):
+        self.uuid, self.index, self.period = uuid, index, period
+        self.samples = []
+        self._stop = None
+        self._thread = None
+        self.source = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.uuid:
+            try:
+                return pynvml, pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            except pynvml.NVMLError:
+                pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
 
     def start(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            nv, h = self._handle()
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception:   # no NVML here: no clock record
+            self._thread = None
+            return
+        self.source = "nvml"
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                t = time.time()
+                try:
+                    mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                    rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                    self.samples.append((t, mhz, pw, rs))
+                except Exception:
+                    pass
+                self._stop.wait(self.period)
+
+        self._nv, self._h = nv, h
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
+
+    def sample_now(self):
+        """One sample taken at once (the timed region of a small workload can
+        be shorter than the sampling period)."""
+        if self._thread is None:
+            return
+        nv, h = self._nv, self._h
+        try:
+            self.samples.append((time.time(), float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                 nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                 int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+        except Exception:
+            pass
 
     def stop(self, wall0: float, wall1: float) -> dict | None:
-        """Summary of the samples taken between wall0 and wall1 (time.time());
-        all samples if fewer than three fall inside the window."""
-        import datetime
-        if self.proc is None:
+        """Summary of the samples taken between wall0 and wall1 (time.time())."""
+        if self._thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        for line in open(self.path):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9 or not f[1].replace(".", "").isdigit():
-                continue
-            try:
-                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
-            except ValueError:
-                ts = None
-            rows.append((ts, f))
-        os.unlink(self.path)
-        inside = [f for ts, f in rows if ts is not None and wall0 <= ts <= wall1]
-        used = inside if len(inside) >= 3 else [f for _, f in rows]
-        if not used:
-            return None
-        sm = [float(r[1]) for r in used]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[j] for r in used for j in range(4) if r[5 + j].lower() == "active"})
-        pw = [float(r[3]) for r in used if r[3].replace(".", "").isdigit()]
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(used[0][2]),
-                "samples": len(used), "samples_in_timed_region": len(inside),
-                "power_w_max": max(pw) if pw else None, "reasons": reasons}
+        self._stop.set()
+        self._thread.join(timeout=5)
+        inside = [x for x in self.samples if wall0 <= x[0] <= wall1]
+        if not inside:
+            return {"samples_in_timed_region": 0, "source": self.source, "period_s": self.period,
+                    "note": "no sample fell inside the timed region"}
+        reasons = sorted({name for _, _, _, rs in inside for name, bit in self.REASONS if rs & bit})
+        return {"sm_mhz": statistics.median(x[1] for x in inside), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(x[1] for x in inside), "samples_in_timed_region": len(inside),
+                "power_w_max": max(x[2] for x in inside), "reasons": reasons,
+                "source": self.source, "period_s": self.period}
 
 
-# DRAM bytes per launch of the expert-MLP GEMM, from one ncu capture of the
-# S-shaped layer (profiles/expert_ffn_tc_gemm.md), valid only for the kernel
-# source it was taken on.
-GEMM_TRAFFIC = {("S", "3xtf32"): {"src": "element_routed_moe_b200/csrc/ffn_tc.cu",
-                                  "sha256_prefix": "045bb1478b54cb10", "bytes_per_launch": 3.258e9}}
+# DRAM bytes per launch of the expert-MLP GEMM (mean over a step's four
+# launches), from ncu captures of a smaller case of the same workload scaled
+# to full size by its routed rows; valid only for the kernel source it was
+# taken on (else reported as null).
+GEMM_TRAFFIC = {}
 
 
 def measured_traffic(workload: str, mode: str):
@@ -391,6 +423,41 @@ def run_reference(args, world, rank):
 # --------------------------------------------------------------------------
 # janus arm
 # --------------------------------------------------------------------------
+def gemm_roofline(J, mode, cfg, packed_first, peaks, peak_src, flops_per_gemm, ms_total, launches):
+    """Roofline of the grouped expert-MLP GEMM over a step's launches.
+
+    3xTF32: a GEMM that issues p tensor-core products per k-step has an
+    FP32-accurate peak of (TF32 peak) / p; TF32 peak = measured burst BF16 x the
+    nominal TF32/BF16 ratio (1.125 / 2.25).  The forward's first GEMM issues
+    p = 2 when its rows are FP16-packed (an unpacked FP16 row is exact in TF32:
+    its residual product is skipped), every other GEMM p = 3.  The combined
+    peak is the FLOP-weighted harmonic mean, so frac = (sum of each launch's
+    ideal time) / (measured time).  SIMT: 148 SMs x 128 FP32 lanes x 2 FLOP x
+    the maximum SM clock, the same for every launch."""
+    tf32 = peaks["bf16_tflops"] * (1.125 / 2.25)
+    if mode == J.JANUS_FFN_FP32_SIMT:
+        per = [SM_COUNT * FP32_LANES_PER_SM * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12] * launches
+        roof = {"bound": "alu", "peak_source": "148 SMs x 128 FP32 lanes x 2 FLOP x max SM clock"}
+    else:
+        products = [2 if (i == 0 and packed_first) else 3 for i in range(launches)]
+        per = [tf32 / p for p in products]
+        roof = {"bound": "tensor",
+                "peak_source": f"{peak_src} burst bf16 x (TF32/BF16 nominal 1.125/2.25) / products per GEMM "
+                               f"({products}: the FP16-packed forward's first GEMM skips the rows' zero "
+                               f"residual)",
+                "products_per_gemm": products}
+    flops = flops_per_gemm * launches
+    ideal_s = sum(flops_per_gemm / (pk * 1e12) for pk in per)
+    peak = flops / ideal_s / 1e12
+    achieved = flops / (ms_total * 1e-3) / 1e12
+    roof.update({"kernel": "grouped expert-MLP GEMM", "achieved": achieved, "peak": peak,
+                 "peak_per_gemm": per, "unit": "TFLOP/s", "frac": achieved / peak,
+                 "frac_of_sustained_peak": achieved / (peak * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+                                                       / peaks["bf16_tflops"]),
+                 "algorithmic_flops_per_launch": flops_per_gemm, "launches_per_step": launches})
+    return roof
+
+
 def run_janus(args, world, rank, local):
     from element_routed_moe_b200 import janus as J
     J.lib()   # fails loudly if the CUDA library is missing
@@ -410,9 +477,9 @@ def run_janus(args, world, rank, local):
            for op in layer.ops} for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     props = torch.cuda.get_device_properties(dev)
-    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local))
+    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else None, local)
     sampler.start()
-    time.sleep(0.3)
+    time.sleep(0.1)
     barrier(world)
     torch.cuda.synchronize()
     wall0 = time.time()
@@ -420,6 +487,7 @@ def run_janus(args, world, rank, local):
     for k in range(args.steps):
         layer.step(events=ev[k])
     t_end.record()
+    sampler.sample_now()        # while the enqueued steps run
     torch.cuda.synchronize()
     wall1 = time.time()
     clocks = sampler.stop(wall0, wall1)
@@ -440,44 +508,32 @@ def run_janus(args, world, rank, local):
     kernels["route"] = {"ms": op_ms["route"]}
 
     # roofline of the dominant kernel: the grouped expert-MLP GEMM (4 launches
-    # per step: two forward, two VJP, each 2*R*d*h FLOPs)
+    # per step: two forward, two VJP, each 2*R*d*h FLOPs), timed by CUDA
+    # events on the launching stream inside the timed steps
     ffn_ms = op_ms["ffn_fwd"] + op_ms["ffn_vjp"]
-    ffn_flops = work["ffn_fwd"][1] + work["ffn_vjp"][1]
-    achieved = ffn_flops / (ffn_ms * 1e-3) / 1e12
-    if mode == J.JANUS_FFN_FP32_SIMT:
-        peak = SM_COUNT * FP32_LANES_PER_SM * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
-        roof = {"bound": "alu", "peak_source": "148 SMs x 128 FP32 lanes x 2 FLOP x max SM clock"}
-    else:
-        # burst figure: the GEMM runs at the maximum SM clock inside this step
-        # (the clocks record shows it), unlike the power-capped seconds-long
-        # bf16 loop behind the sustained figure; the burst one is the stricter
-        peak = peaks["bf16_tflops"] * (1.125 / 2.25) / 3.0
-        roof = {"bound": "tensor", "peak_source": f"{peak_src} burst bf16 x (TF32/BF16 nominal 1.125/2.25) / 3 products"}
-    roof.update({"kernel": "grouped expert-MLP GEMM", "achieved": achieved, "peak": peak,
-                 "unit": "TFLOP/s", "frac": achieved / peak,
-                 "traffic": (measured_traffic(cfg.name, args.mode)
-                             if cfg == synth.CONFIGS[cfg.name] else None),
-                 "algorithmic_flops_per_launch": ffn_flops / 4, "launches_per_step": 4})
-
+    roof = gemm_roofline(J, mode, cfg, layer.packed, peaks, peak_src, work["ffn_fwd"][1] / 2, ffn_ms, 4)
+    roof["traffic"] = measured_traffic(cfg.name, args.mode) if cfg == synth.CONFIGS[cfg.name] else None
+    roof["traffic_unit"] = "DRAM bytes per launch (mean of the step's 4 launches)"
+    ws_gb = ((layer.w1.numel() + layer.w2.numel()) * 4 + cfg.n_rows * cfg.d * 4 * 4) / 1e9
+    if layer.edges:
+        ws_gb += layer.msg.numel() * 4 / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_max / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {**describe(cfg), "ffn_mode": args.mode, "parallelism": f"replicas x{world}",
-                   "l2": "no flush: per-step working set "
-                         f"{(layer.w1.numel() + layer.w2.numel()) * 4 / 2**30:.1f} GiB weights + "
-                         f"{cfg.n_rows * cfg.d * 4 * 4 / 2**30:.2f} GiB activations >> 126 MB L2"},
+                   "l2": f"no flush between steps: each step streams {ws_gb:.1f} GB (weights, activations"
+                         f"{', edge messages' if layer.edges else ''}) >> the 126 MB L2; cold-L2 figures of the "
+                         f"memory-bound kernels under kernels_cold_l2"},
         "roofline": roof,
         "kernels": kernels,
         "breakdown_ms": op_ms,
         "gpu_launches": layer.launches_per_step * args.steps,
         "clocks": clocks,
     }
-
-    # (skipped where the step's input is the edge messages of L or the slice:
-    # 9-29 GB to upload per step)
-    msg_bytes = layer.msg.numel() * 4 if layer.edges else 0
-    if not args.no_e2e and msg_bytes <= (1 << 30):
+    if not args.no_cold:
+        line["kernels_cold_l2"] = run_cold_l2(layer, peaks)
+    if not args.no_e2e:
         line["e2e"] = run_e2e(layer, args)
     if not args.no_extras:
         line["extras"] = run_extras(layer, peaks)
@@ -493,6 +549,51 @@ def run_janus(args, world, rank, local):
                       f"full expert weights, {dt:.1f} s; host {cpu_descr()}"}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def run_cold_l2(layer, peaks, reps=5):
+    """The memory-bound kernels of the step timed one call at a time with the
+    L2 flushed before each call (a 2x-L2 buffer written in between, outside
+    the timed events): median of `reps` calls, next to the in-step figures."""
+    J = layer.J
+    cfg = layer.cfg
+    K, T = cfg.top_k, cfg.n_types
+    r = layer.route_out
+    core = layer.core
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=layer.x.device)
+    x = core.xagg if layer.edges else layer.x
+    calls = {
+        "dispatch": lambda: J.janus_dispatch(x, r["slot_of"], K, out=layer.xd),
+        "dispatch_w": lambda: J.janus_dispatch(layer.g, r["slot_of"], K, r["topk_weight"], out=layer.gd),
+        "combine": lambda: J.janus_combine(core.yd, r["slot_of"], K, r["topk_weight"], out=layer.y),
+        "combine_vjp": lambda: J.janus_combine(core.dxd, r["slot_of"], K, out=layer.dx),
+    }
+    if layer.edges:
+        calls["edge_aggregate"] = lambda: J.janus_edge_aggregate(layer.msg, layer.row_ptr, out=core.xagg)
+    if layer.packed:
+        calls["quant"] = lambda: J.janus_quant_by_type(x, layer.types, T, r["slot_of"], K, payload=core.payload,
+                                                       scale=core.scale, workspace=core.quant_ws)
+        calls["dequant"] = lambda: J.janus_dequant_by_type(core.payload, layer.types, T, r["perm"], K, core.scale,
+                                                           out=layer.xd)
+    work = layer.work()
+    out = {}
+    for op, fn in calls.items():
+        fn()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ms = statistics.median(ts)
+        amount = work[op][1]
+        out[op] = {"ms": ms, "GB/s": amount / (ms * 1e-3) / 1e9,
+                   "frac_hbm": amount / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "algorithmic_bytes": amount}
+    del flush
+    return out
 
 
 def run_ep(args, world, rank, local):
@@ -527,9 +628,9 @@ def run_ep(args, world, rank, local):
           for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     props = torch.cuda.get_device_properties(dev)
-    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local))
+    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else None, local)
     sampler.start()
-    time.sleep(0.3)
+    time.sleep(0.1)
     barrier(world)
     torch.cuda.synchronize()
     wall0 = time.time()
@@ -538,6 +639,7 @@ def run_ep(args, world, rank, local):
         layer.forward(x, types, gate, events=ev[k])
         layer.vjp(g, events=ev[k])
     t_end.record()
+    sampler.sample_now()
     torch.cuda.synchronize()
     wall1 = time.time()
     clocks = sampler.stop(wall0, wall1)
@@ -548,18 +650,11 @@ def run_ep(args, world, rank, local):
     ph_ms = {ph: float(np.mean([e[ph][0].elapsed_time(e[ph][1]) for e in ev])) for ph in phases}
     # this rank's expert GEMMs: 4 of 2 * R_recv * d * h FLOPs each (fwd + VJP)
     r_recv = int(layer.layout[2][rank][-1].item())
-    ffn_flops = 8.0 * r_recv * d * h
     ffn_ms = ph_ms["ffn_fwd"] + ph_ms["ffn_vjp"]
-    achieved = ffn_flops / (ffn_ms * 1e-3) / 1e12 if ffn_ms > 0 else 0.0
-    if mode == J.JANUS_FFN_FP32_SIMT:
-        peak = SM_COUNT * FP32_LANES_PER_SM * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
-        roof = {"bound": "alu", "peak_source": "148 SMs x 128 FP32 lanes x 2 FLOP x max SM clock"}
-    else:
-        peak = peaks["bf16_tflops"] * (1.125 / 2.25) / 3.0
-        roof = {"bound": "tensor", "peak_source": f"{peak_src} burst bf16 x (TF32/BF16 nominal 1.125/2.25) / 3 products"}
+    # the owner's first forward GEMM runs on the received FP16 rows: 2 products
+    roof = gemm_roofline(J, mode, cfg, True, peaks, peak_src, 2.0 * r_recv * d * h, max(ffn_ms, 1e-9), 4)
     roof.update({"kernel": "grouped expert-MLP GEMM (rank 0's experts; ffn phases include the FP16 unpack)",
-                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-                 "algorithmic_flops_per_launch": ffn_flops / 4, "launches_per_step": 4})
+                 "traffic": None})
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_max / args.steps * 1e3, "higher_is_better": True,
@@ -647,36 +742,68 @@ def run_extras(layer, peaks):
     return out
 
 
+def _pinned_copy(t):
+    """Host copy of device tensor t in page-locked memory, registered in place
+    (cudaHostRegister: no rounding of the size, unlike the caching pinned
+    allocator); release with _unpin."""
+    h = torch.empty(t.shape, dtype=t.dtype)
+    err = torch.cuda.cudart().cudaHostRegister(h.data_ptr(), h.numel() * h.element_size(), 0)
+    if int(err) != 0:
+        raise RuntimeError(f"cudaHostRegister failed ({err})")
+    h.copy_(t)
+    return h
+
+
+def _unpin(*ts):
+    torch.cuda.synchronize()
+    for t in ts:
+        torch.cuda.cudart().cudaHostUnregister(t.data_ptr())
+
+
 def run_e2e(layer, args):
     """Same metric through the library's MoELayer.run_host with the step's
-    inputs in pinned host memory: every step uploads (x, dY, types) and
-    downloads (y, dX) inside the timed region.  The copies run on their own
-    streams: dY's upload overlaps the forward, y's download the VJP, and the
-    next step's upload this step's compute."""
+    inputs in pinned host memory: every step uploads its inputs (the node
+    features x, or the edge messages where the workload aggregates them; dY;
+    types) and downloads its results (y, dX) inside the timed region.  The
+    copies run on their own streams: dY's upload overlaps the forward, y's
+    download the VJP, the next step's upload this step's compute; edge
+    messages stream through a ring of device buffers, each chunk aggregated as
+    it lands.  The receiver graph (row_ptr, 8 (N+1) bytes) is the layer's own,
+    uploaded once when the layer is built."""
     core = layer.core
-    # the step's input: the edge messages where the workload aggregates them
-    x_h = (layer.msg if layer.edges else layer.x).cpu().pin_memory()
-    g_h = layer.g.cpu().pin_memory()
-    t_h = layer.types.cpu().pin_memory()
-    y_h = torch.empty(layer.y.shape, dtype=torch.float32).pin_memory()
-    dx_h = torch.empty(layer.dx.shape, dtype=torch.float32).pin_memory()
-    for _ in range(args.warmup):
-        core.run_host(x_h, g_h, t_h, y_h, dx_h)
-    core.host_sync()
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(args.steps):
-        core.run_host(x_h, g_h, t_h, y_h, dx_h)
-    core.host_sync()
-    b.record()
-    torch.cuda.synchronize()
-    t = a.elapsed_time(b) / 1e3
-    h2d = x_h.numel() * 4 + g_h.numel() * 4 + t_h.numel() * 4
-    d2h = y_h.numel() * 4 + dx_h.numel() * 4
-    return {"value": layer.cfg.n_rows * args.steps / t, "unit": UNIT,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "overlap": "uploads and downloads on their own streams, double-buffered on the device"}
+    x_h = _pinned_copy(layer.msg if layer.edges else layer.x)
+    g_h = _pinned_copy(layer.g)
+    t_h = _pinned_copy(layer.types)
+    y_h = _pinned_copy(layer.y)
+    dx_h = _pinned_copy(layer.dx)
+    try:
+        for _ in range(args.warmup):
+            core.run_host(x_h, g_h, t_h, y_h, dx_h)
+        core.host_sync()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            core.run_host(x_h, g_h, t_h, y_h, dx_h)
+        core.host_sync()
+        b.record()
+        torch.cuda.synchronize()
+        t = a.elapsed_time(b) / 1e3
+        h2d = x_h.numel() * 4 + g_h.numel() * 4 + t_h.numel() * 4
+        d2h = y_h.numel() * 4 + dx_h.numel() * 4
+        out = {"value": layer.cfg.n_rows * args.steps / t, "unit": UNIT, "ms_per_step": t / args.steps * 1e3,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "h2d_GB/s": h2d / (t / args.steps) / 1e9,
+               "overlap": "uploads and downloads on their own streams, double-buffered on the device"
+                          + ("; edge messages streamed through a device ring, aggregated chunk by chunk"
+                             if layer.edges else "")}
+        if layer.edges:
+            out["chunks_per_step"] = len(core._host["chunks"])
+    finally:
+        core._host = None      # the host pipeline's device buffers and ring
+        _unpin(x_h, g_h, t_h, y_h, dx_h)
+    return out
+
 
 def main():
     args = parse()

@@ -11,8 +11,10 @@
 //   * receiver-sorted CSR: atom i's messages are one contiguous block
 //     msg[row_ptr[i] : row_ptr[i+1], :], so every load is a coalesced 128-bit
 //     streaming load (evict-first, the messages are read exactly once);
-//   * one warp per atom, U = 4 column float4s per lane and the edge loop
-//     unrolled by 4 -> up to 16 independent 16-byte loads per lane in flight;
+//   * one warp per work item (receiver, chunk of 128 float4 columns), so a
+//     layer with fewer receivers than the grid has warps still fills them;
+//     U = 4 column float4s per lane and the edge loop unrolled by 4 -> up to
+//     16 independent 16-byte loads per lane in flight;
 //   * FP32 accumulation: each group of 4 edges is summed pairwise and then
 //     added to the running sum (edge order otherwise); each output row is
 //     written once;
@@ -30,6 +32,25 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kU = 4;
+constexpr int kChunk4 = 32 * kU;   // float4 columns of one work item (receiver, column chunk)
+
+// Warp w takes column chunk w % nch of receivers w / nch, w / nch + W / nch,
+// ... (W warps, nch chunks per row; the last W % nch warps stay idle): the
+// chunks of one receiver go to neighbouring warps, and no warp divides per item.
+struct ChunkWalk {
+  int64_t row0, stride;
+  int c0;
+};
+__device__ __forceinline__ ChunkWalk chunk_walk(int d4) {
+  const int nch = (d4 + kChunk4 - 1) / kChunk4;
+  const int64_t w = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / 32;
+  const int64_t W = (int64_t)gridDim.x * kThreads / 32;
+  ChunkWalk cw;
+  cw.stride = W / nch;
+  cw.row0 = w < cw.stride * nch ? w / nch : INT64_MAX;
+  cw.c0 = (int)(w % nch) * kChunk4;
+  return cw;
+}
 constexpr int kEdgeUnroll = 4;
 static_assert(kEdgeUnroll == 4, "the pairwise group sum below is written for 4 edges");
 
@@ -56,49 +77,46 @@ __global__ void __launch_bounds__(kThreads)
 edge_aggregate_kernel(const float4* __restrict__ msg, const int64_t* __restrict__ row_ptr,
                       int64_t n_atoms, int64_t n_edges, int d4, float4* __restrict__ out, int32_t* dbg) {
   const int lane = threadIdx.x % 32;
-  const int64_t nwarps = (int64_t)gridDim.x * kThreads / 32;
-  for (int64_t i = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / 32; i < n_atoms; i += nwarps) {
+  const ChunkWalk cw = chunk_walk(d4);
+  const int c0 = cw.c0;
+  // float4 columns of this lane inside the chunk (kU except in a ragged last chunk)
+  const int nu = min(kU, max(0, (d4 - c0 - lane + 31) / 32));
+  for (int64_t i = cw.row0; i < n_atoms; i += cw.stride) {
     int64_t e0, e1;
     edge_range(row_ptr, i, n_edges, dbg, &e0, &e1);
-    for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
-      float4 acc[kU];
+    float4 acc[kU];
 #pragma unroll
-      for (int u = 0; u < kU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      int64_t e = e0;
-      for (; e + kEdgeUnroll <= e1; e += kEdgeUnroll) {
-        float4 v[kEdgeUnroll][kU];
+    for (int u = 0; u < kU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4* p = msg + e0 * d4 + c0 + lane;     // edge e0, this lane's first column
+    int n = (int)(e1 - e0);
+    for (; n >= kEdgeUnroll; n -= kEdgeUnroll, p += (int64_t)kEdgeUnroll * d4) {
+      float4 v[kEdgeUnroll][kU];
 #pragma unroll
-        for (int r = 0; r < kEdgeUnroll; ++r)
+      for (int r = 0; r < kEdgeUnroll; ++r)
 #pragma unroll
-          for (int u = 0; u < kU; ++u) {
-            const int c = c0 + u * 32 + lane;
-            v[r][u] = c < d4 ? __ldcs(msg + (e + r) * d4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        // pairwise within the group of 4, then one add into the running sum
-        // (a 4x shorter rounding chain for high-degree receivers)
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const float4 a = f4add(v[0][u], v[1][u]), b = f4add(v[2][u], v[3][u]);
-          acc[u] = f4add(acc[u], f4add(a, b));
-        }
-      }
-      for (; e < e1; ++e) {
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int c = c0 + u * 32 + lane;
-          if (c < d4) {
-            const float4 v = __ldcs(msg + e * d4 + c);
-            acc[u].x += v.x; acc[u].y += v.y; acc[u].z += v.z; acc[u].w += v.w;
-          }
-        }
-      }
-      float4* dst = out + i * d4;
+        for (int u = 0; u < kU; ++u)
+          v[r][u] = u < nu ? __ldcs(p + r * d4 + u * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
+      // pairwise within the group of 4, then one add into the running sum
+      // (a 4x shorter rounding chain for high-degree receivers)
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
-        const int c = c0 + u * 32 + lane;
-        if (c < d4) dst[c] = acc[u];
+        const float4 a = f4add(v[0][u], v[1][u]), b = f4add(v[2][u], v[3][u]);
+        acc[u] = f4add(acc[u], f4add(a, b));
       }
     }
+    for (; n > 0; --n, p += d4) {
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        if (u < nu) {
+          const float4 v = __ldcs(p + u * 32);
+          acc[u].x += v.x; acc[u].y += v.y; acc[u].z += v.z; acc[u].w += v.w;
+        }
+      }
+    }
+    float4* dst = out + i * d4 + c0 + lane;
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (u < nu) dst[u * 32] = acc[u];
   }
 }
 
@@ -109,24 +127,23 @@ __global__ void __launch_bounds__(kThreads)
 edge_broadcast_kernel(const float4* __restrict__ dx, const int64_t* __restrict__ row_ptr, int64_t n_atoms,
                       int64_t n_edges, int d4, float4* __restrict__ dmsg, int32_t* dbg) {
   const int lane = threadIdx.x % 32;
-  const int64_t nwarps = (int64_t)gridDim.x * kThreads / 32;
-  for (int64_t i = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / 32; i < n_atoms; i += nwarps) {
+  const ChunkWalk cw = chunk_walk(d4);
+  const int c0 = cw.c0;
+  for (int64_t i = cw.row0; i < n_atoms; i += cw.stride) {
     int64_t e0, e1;
     edge_range(row_ptr, i, n_edges, dbg, &e0, &e1);
     if (e1 <= e0) continue;
-    for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
-      float4 v[kU];
+    float4 v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int c = c0 + u * 32 + lane;
+      v[u] = c < d4 ? __ldg(dx + i * d4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int64_t e = e0; e < e1; ++e) {
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
         const int c = c0 + u * 32 + lane;
-        v[u] = c < d4 ? __ldg(dx + i * d4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      for (int64_t e = e0; e < e1; ++e) {
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int c = c0 + u * 32 + lane;
-          if (c < d4) __stcs(dmsg + e * d4 + c, v[u]);
-        }
+        if (c < d4) __stcs(dmsg + e * d4 + c, v[u]);
       }
     }
   }
@@ -204,7 +221,7 @@ extern "C" janus_status janus_edge_aggregate(const float* msg, int64_t n_edges, 
   JANUS_CHECK_ARG(row_ptr && out && (msg || n_edges == 0));
   JANUS_CHECK_ALIGN(aligned(msg, 16) && aligned(out, 16));
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
-  const int64_t need = (n_atoms + 7) / 8;
+  const int64_t need = (n_atoms * ((d / 4 + kChunk4 - 1) / kChunk4) + 7) / 8;
   const int64_t cap = (int64_t)num_sms() * 8;
   const unsigned grid = (unsigned)(need < cap ? need : cap);
   edge_aggregate_kernel<<<grid, kThreads, 0, (cudaStream_t)stream>>>(
@@ -220,7 +237,7 @@ extern "C" janus_status janus_edge_broadcast(const float* dx, const int64_t* row
   JANUS_CHECK_ARG(dx && row_ptr && (dmsg || n_edges == 0));
   JANUS_CHECK_ALIGN(aligned(dx, 16) && aligned(dmsg, 16));
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
-  const int64_t need = (n_atoms + 7) / 8;
+  const int64_t need = (n_atoms * ((d / 4 + kChunk4 - 1) / kChunk4) + 7) / 8;
   const int64_t cap = (int64_t)num_sms() * 8;
   edge_broadcast_kernel<<<(unsigned)(need < cap ? need : cap), kThreads, 0, (cudaStream_t)stream>>>(
       (const float4*)dx, row_ptr, n_atoms, n_edges, d / 4, (float4*)dmsg, debug_fault_word());

@@ -392,8 +392,8 @@ extern "C" janus_status janus_ep_dispatch_quant(const float* x, int64_t n_atoms,
   JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, need, stream));
   const unsigned grid = rows_grid(n_atoms, 8);
   if (n_atoms > 0)
-    quant_amax_kernel<<<grid, kThreads, sizeof(uint32_t) * n_types, stream>>>((const float4*)x, n_atoms, d / 4,
-                                                                              types, n_types, amax_bits, hdr);
+    quant_amax_kernel<<<rows_grid(row_items(n_atoms, d / 4), 8), kThreads, sizeof(uint32_t) * n_types, stream>>>(
+        (const float4*)x, n_atoms, d / 4, types, n_types, amax_bits, hdr);
   ep_pack_send_kernel<<<grid, kThreads, 2 * sizeof(float) * n_types, stream>>>(
       (const float4*)x, n_atoms, d / 4, top_k, types, n_types, slot_of, topk_expert, amax_bits,
       src_off + (size_t)rank * (n_experts + 1), dst_off + (size_t)rank * n_experts, n_experts, n_experts / world,

@@ -128,8 +128,10 @@ extern "C" janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, con
   if (n_rows == 0) return JANUS_OK;
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
   float* H = (float*)((char*)workspace + L.off_h);
+  // the error word starts clear in both modes, so janus_check on this
+  // workspace reports only this call's faults
+  JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
   if (mode == JANUS_FFN_3XTF32) {
-    JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
     st = tc::expert_ffn_fwd_packed(payload, row_scale, offsets, n_experts, n_rows, d, h, w1, w2, yd, act, H,
                                    &((WsHeader*)workspace)->error, stream, yd_rows);
     if (st != JANUS_OK) return st;
@@ -177,8 +179,10 @@ janus_status ffn_fwd(const float* xd, const int32_t* offsets, int32_t n_experts,
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
   float* H = (float*)((char*)workspace + L.off_h);
   const int64_t sw = (int64_t)d * h;
+  // the error word starts clear in both modes, so janus_check on this
+  // workspace reports only this call's faults
+  JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
   if (mode == JANUS_FFN_3XTF32) {
-    JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
     st = tc::expert_ffn_fwd(xd, offsets, n_experts, n_rows, d, h, w1, w2, yd, act, H,
                             &((WsHeader*)workspace)->error, stream, yd_rows,
                             (flags & JANUS_FFN_X_DEQUANTIZED) != 0);
@@ -213,8 +217,10 @@ janus_status ffn_vjp(const float* xd, const float* gd, const float* act, const i
   float* dA = (float*)((char*)workspace + L.off_h);
   float* A = act ? const_cast<float*>(act) : (float*)((char*)workspace + L.off_h + rh);
   const int64_t sw = (int64_t)d * h;
+  // the error word starts clear in both modes, so janus_check on this
+  // workspace reports only this call's faults
+  JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
   if (mode == JANUS_FFN_3XTF32) {
-    JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
     st = tc::expert_ffn_vjp(xd, gd, act, A, offsets, n_experts, n_rows, d, h, w1, w2, dxd, dA,
                             &((WsHeader*)workspace)->error, stream, dxd_rows);
     if (st != JANUS_OK) return st;
@@ -321,8 +327,10 @@ extern "C" janus_status janus_expert_ffn_weight_grad(const float* xd, const floa
   float* dA = (float*)w;
   float* H = (float*)(w + rh);
   float* A = act ? const_cast<float*>(act) : (float*)(w + 2 * rh);
+  // the error word starts clear in both modes, so janus_check on this
+  // workspace reports only this call's faults
+  JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
   if (mode == JANUS_FFN_3XTF32) {
-    JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
     st = tc::expert_ffn_weight_grad(xd, gd, act, A, offsets, n_experts, n_rows, d, h, w1, w2, dw1, dw2, dA,
                                     H, &((WsHeader*)workspace)->error, stream);
     if (st != JANUS_OK) return st;
@@ -394,8 +402,10 @@ extern "C" janus_status janus_expert_ffn_vjp_vjp(const float* xd, const float* g
   float* t2 = (float*)(w + 2 * rh);
   float* u = wg ? (float*)(w + 3 * rh) : nullptr;
   float* A = act ? const_cast<float*>(act) : (float*)(w + (wg ? 4 : 3) * rh);
+  // the error word starts clear in both modes, so janus_check on this
+  // workspace reports only this call's faults
+  JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
   if (mode == JANUS_FFN_3XTF32) {
-    JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
     st = tc::expert_ffn_vjp_vjp(xd, gd, vd, act, A, offsets, n_experts, n_rows, d, h, w1, w2, d_xd, d_gd, dw1,
                                 dw2, dh, t1, t2, u, &((WsHeader*)workspace)->error, stream);
     if (st != JANUS_OK) return st;

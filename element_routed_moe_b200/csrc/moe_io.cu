@@ -7,8 +7,9 @@
 // "MatRIS-MoE与Janus框架" section 3.2 (gate-weighted sum of expert outputs).
 //
 // All four are HBM-bound streams.  Layout choices for B200:
-//   * one warp per atom row, 128-bit accesses, U = 4 independent 16-byte
-//     loads per lane in flight (2 KB per warp) before any store;
+//   * one warp per work item (row, chunk of 128 float4 columns), 128-bit
+//     accesses, U = 4 independent 16-byte loads per lane in flight (2 KB per
+//     warp) before any store;
 //   * dispatch and pack run in scatter form: the atom row is read once and
 //     written to its K dispatch rows (slot_of gives each destination; every
 //     destination is distinct, so no atomics and a deterministic result);
@@ -46,40 +47,55 @@ dispatch_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K,
                 float4* __restrict__ xd, int32_t* dbg) {
   const int64_t R = n_atoms * K;
   const int lane = threadIdx.x % 32;
-  for (int64_t i = global_warp(); i < n_atoms; i += total_warps()) {
+  const ChunkWalk cw = chunk_walk(d4);
+  const int c0 = cw.c0;
+  for (int64_t i = cw.row0; i < n_atoms; i += cw.stride) {
     const int my_slot = lane < K ? slot_of[i * K + lane] : 0;
     const float my_w = (kWeighted && lane < K) ? w[i * K + lane] : 1.0f;
     const float4* src = x + i * d4;
-    for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
-      float4 v[kU];
+    float4 v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int c = c0 + u * 32 + lane;
+      if (c < d4) v[u] = __ldcs(src + c);
+    }
+    for (int k = 0; k < K; ++k) {
+      int64_t p;
+      float wk;
+      slot_k<kWeighted>(k, K, i, my_slot, my_w, slot_of, w, &p, &wk);
+      if (kDebug && !in_range(p, R)) {   // p is the same in every lane
+        if (lane == 0) debug_fault(dbg);
+        continue;
+      }
+      float4* dst = xd + p * d4;
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
         const int c = c0 + u * 32 + lane;
-        if (c < d4) v[u] = __ldcs(src + c);
-      }
-      for (int k = 0; k < K; ++k) {
-        int64_t p;
-        float wk;
-        slot_k<kWeighted>(k, K, i, my_slot, my_w, slot_of, w, &p, &wk);
-        if (kDebug && !in_range(p, R)) {   // p is the same in every lane
-          if (lane == 0) debug_fault(dbg);
-          continue;
-        }
-        float4* dst = xd + p * d4;
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int c = c0 + u * 32 + lane;
-          if (c < d4) {
-            float4 o = v[u];
-            if (kWeighted) { o.x *= wk; o.y *= wk; o.z *= wk; o.w *= wk; }
-            dst[c] = o;
-          }
+        if (c < d4) {
+          float4 o = v[u];
+          if (kWeighted) { o.x *= wk; o.y *= wk; o.z *= wk; o.w *= wk; }
+          dst[c] = o;
         }
       }
     }
   }
 }
 
+// acc += wk * v (or acc += v), one FMA (add) per component, in the caller's k order
+template <bool kWeighted>
+__device__ __forceinline__ void accumulate(float4& acc, float wk, const float4& v) {
+  if (kWeighted) {
+    acc.x = fmaf(wk, v.x, acc.x);
+    acc.y = fmaf(wk, v.y, acc.y);
+    acc.z = fmaf(wk, v.z, acc.z);
+    acc.w = fmaf(wk, v.w, acc.w);
+  } else {
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+}
+
+// Gather form: the K expert rows of one (atom, column chunk) item are added
+// in ascending k.
 template <bool kWeighted>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(const float4* __restrict__ yd, const int32_t* __restrict__ slot_of,
@@ -87,45 +103,35 @@ combine_kernel(const float4* __restrict__ yd, const int32_t* __restrict__ slot_o
                float4* __restrict__ y, int32_t* dbg) {
   const int64_t R = n_atoms * K;
   const int lane = threadIdx.x % 32;
-  for (int64_t i = global_warp(); i < n_atoms; i += total_warps()) {
+  const ChunkWalk cw = chunk_walk(d4);
+  const int c0 = cw.c0;
+  const int nu = min(kU, max(0, (d4 - c0 - lane + 31) / 32));   // this lane's columns in the chunk
+  const float4* yl = yd + c0 + lane;
+  for (int64_t i = cw.row0; i < n_atoms; i += cw.stride) {
     const int my_slot = lane < K ? slot_of[i * K + lane] : 0;
     const float my_w = (kWeighted && lane < K) ? w[i * K + lane] : 1.0f;
-    for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
-      float4 acc[kU];
+    float4 acc[kU];
 #pragma unroll
-      for (int u = 0; u < kU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int k = 0; k < K; ++k) {
-        int64_t p;
-        float wk;
-        slot_k<kWeighted>(k, K, i, my_slot, my_w, slot_of, w, &p, &wk);
-        if (kDebug && !in_range(p, R)) {
-          if (lane == 0) debug_fault(dbg);
-          continue;
-        }
-        const float4* src = yd + p * d4;
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int c = c0 + u * 32 + lane;
-          if (c < d4) {
-            const float4 v = __ldcs(src + c);
-            if (kWeighted) {
-              acc[u].x = fmaf(wk, v.x, acc[u].x);
-              acc[u].y = fmaf(wk, v.y, acc[u].y);
-              acc[u].z = fmaf(wk, v.z, acc[u].z);
-              acc[u].w = fmaf(wk, v.w, acc[u].w);
-            } else {
-              acc[u].x += v.x; acc[u].y += v.y; acc[u].z += v.z; acc[u].w += v.w;
-            }
-          }
-        }
+    for (int u = 0; u < kU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < K; ++k) {
+      int64_t p;
+      float wk;
+      slot_k<kWeighted>(k, K, i, my_slot, my_w, slot_of, w, &p, &wk);
+      if (kDebug && !in_range(p, R)) {   // p is the same in every lane
+        if (lane == 0) debug_fault(dbg);
+        continue;
       }
-      float4* dst = y + i * d4;
+      const float4* src = yl + p * d4;
+      float4 v[kU];
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int c = c0 + u * 32 + lane;
-        if (c < d4) dst[c] = acc[u];
-      }
+      for (int u = 0; u < kU; ++u) v[u] = u < nu ? __ldcs(src + u * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) accumulate<kWeighted>(acc[u], wk, v[u]);
     }
+    float4* dst = y + i * d4 + c0 + lane;
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (u < nu) dst[u * 32] = acc[u];
   }
 }
 
@@ -150,38 +156,38 @@ quant_pack_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K,
   }
   __syncthreads();
   const int lane = threadIdx.x % 32;
-  for (int64_t i = global_warp(); i < n_atoms; i += total_warps()) {
+  const ChunkWalk cw = chunk_walk(d4);
+  const int c0 = cw.c0;
+  for (int64_t i = cw.row0; i < n_atoms; i += cw.stride) {
     int t = types[i];
     if (t < 0 || t >= T) t = 0;                // recorded by the amax pass
     const float inv = s_inv[t];
     const int my_slot = lane < K ? slot_of[i * K + lane] : 0;
     const float4* src = x + i * d4;
-    for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
-      uint2 q[kU];
+    uint2 q[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int c = c0 + u * 32 + lane;
+      if (c < d4) {
+        const float4 v = __ldcs(src + c);
+        // exact power-of-two scaling, then one round-to-nearest-even
+        const __half2 lo = __floats2half2_rn(v.x * inv, v.y * inv);
+        const __half2 hi = __floats2half2_rn(v.z * inv, v.w * inv);
+        q[u].x = *reinterpret_cast<const uint32_t*>(&lo);
+        q[u].y = *reinterpret_cast<const uint32_t*>(&hi);
+      }
+    }
+    for (int k = 0; k < K; ++k) {
+      const int64_t p = K <= 32 ? __shfl_sync(0xffffffffu, my_slot, k) : slot_of[i * K + k];
+      if (kDebug && !in_range(p, R)) {
+        if (lane == 0) debug_fault(&ws->error);
+        continue;
+      }
+      uint2* dst = payload + p * d4;
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
         const int c = c0 + u * 32 + lane;
-        if (c < d4) {
-          const float4 v = __ldcs(src + c);
-          // exact power-of-two scaling, then one round-to-nearest-even
-          const __half2 lo = __floats2half2_rn(v.x * inv, v.y * inv);
-          const __half2 hi = __floats2half2_rn(v.z * inv, v.w * inv);
-          q[u].x = *reinterpret_cast<const uint32_t*>(&lo);
-          q[u].y = *reinterpret_cast<const uint32_t*>(&hi);
-        }
-      }
-      for (int k = 0; k < K; ++k) {
-        const int64_t p = K <= 32 ? __shfl_sync(0xffffffffu, my_slot, k) : slot_of[i * K + k];
-        if (kDebug && !in_range(p, R)) {
-          if (lane == 0) debug_fault(&ws->error);
-          continue;
-        }
-        uint2* dst = payload + p * d4;
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int c = c0 + u * 32 + lane;
-          if (c < d4) dst[c] = q[u];
-        }
+        if (c < d4) dst[c] = q[u];
       }
     }
   }
@@ -192,7 +198,9 @@ dequant_kernel(const uint2* __restrict__ payload, int64_t n_rows, int d4, int K,
                const int32_t* __restrict__ types, int T, const int32_t* __restrict__ perm,
                const float* __restrict__ scale, float4* __restrict__ xd, int32_t* dbg) {
   const int lane = threadIdx.x % 32;
-  for (int64_t p = global_warp(); p < n_rows; p += total_warps()) {
+  const ChunkWalk cw = chunk_walk(d4);
+  const int c0 = cw.c0;
+  for (int64_t p = cw.row0; p < n_rows; p += cw.stride) {
     const int32_t slot = perm[p];
     if (kDebug && !in_range(slot, n_rows)) {
       if (lane == 0) debug_fault(dbg);
@@ -203,21 +211,19 @@ dequant_kernel(const uint2* __restrict__ payload, int64_t n_rows, int d4, int K,
     const float s = scale[t];
     const uint2* src = payload + p * d4;
     float4* dst = xd + p * d4;
-    for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
-      uint2 q[kU];
+    uint2 q[kU];
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int c = c0 + u * 32 + lane;
-        if (c < d4) q[u] = __ldcs(src + c);
-      }
+    for (int u = 0; u < kU; ++u) {
+      const int c = c0 + u * 32 + lane;
+      if (c < d4) q[u] = __ldcs(src + c);
+    }
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int c = c0 + u * 32 + lane;
-        if (c < d4) {
-          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&q[u].x));
-          const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&q[u].y));
-          dst[c] = make_float4(a.x * s, a.y * s, b.x * s, b.y * s);
-        }
+    for (int u = 0; u < kU; ++u) {
+      const int c = c0 + u * 32 + lane;
+      if (c < d4) {
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&q[u].x));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&q[u].y));
+        dst[c] = make_float4(a.x * s, a.y * s, b.x * s, b.y * s);
       }
     }
   }
@@ -264,7 +270,7 @@ extern "C" janus_status janus_dispatch(const float* x, int64_t n_atoms, int32_t 
   JANUS_CHECK_ARG(x && slot_of && xd);
   JANUS_CHECK_ALIGN(aligned(x, 16) && aligned(xd, 16));
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
-  const unsigned grid = rows_grid(n_atoms, 8);
+  const unsigned grid = rows_grid(row_items(n_atoms, d / 4), 8);
   if (topk_weight)
     dispatch_kernel<true><<<grid, kThreads, 0, (cudaStream_t)stream>>>(
         (const float4*)x, n_atoms, d / 4, top_k, slot_of, topk_weight, (float4*)xd, debug_fault_word());
@@ -283,7 +289,7 @@ extern "C" janus_status janus_combine(const float* yd, const int32_t* slot_of,
   JANUS_CHECK_ARG(yd && slot_of && y);
   JANUS_CHECK_ALIGN(aligned(yd, 16) && aligned(y, 16));
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
-  const unsigned grid = rows_grid(n_atoms, 8);
+  const unsigned grid = rows_grid(row_items(n_atoms, d / 4), 8);
   if (topk_weight)
     combine_kernel<true><<<grid, kThreads, 0, (cudaStream_t)stream>>>(
         (const float4*)yd, slot_of, topk_weight, n_atoms, top_k, d / 4, (float4*)y, debug_fault_word());
@@ -319,7 +325,7 @@ extern "C" janus_status janus_quant_by_type(const float* x, int64_t n_atoms, int
   uint32_t* amax_bits = (uint32_t*)((char*)workspace + sizeof(WsHeader));
   JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, need, stream));
   const size_t smem = sizeof(uint32_t) * (size_t)n_types;
-  const unsigned grid = rows_grid(n_atoms, 8);
+  const unsigned grid = rows_grid(row_items(n_atoms, d / 4), 8);
   if (n_atoms > 0)
     quant_amax_kernel<<<grid, kThreads, smem, stream>>>((const float4*)x, n_atoms, d / 4, types,
                                                         n_types, amax_bits, hdr);
@@ -342,7 +348,7 @@ extern "C" janus_status janus_dequant_by_type(const uint16_t* payload, int64_t n
   JANUS_CHECK_ALIGN(aligned(payload, 8) && aligned(xd, 16));
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
   const int64_t R = n_atoms * top_k;
-  dequant_kernel<<<rows_grid(R, 8), kThreads, 0, (cudaStream_t)stream>>>(
+  dequant_kernel<<<rows_grid(row_items(R, d / 4), 8), kThreads, 0, (cudaStream_t)stream>>>(
       (const uint2*)payload, R, d / 4, top_k, types, n_types, perm, scale, (float4*)xd, debug_fault_word());
   return launch_status();
 }
@@ -462,7 +468,7 @@ extern "C" janus_status janus_quant_by_type_noalloc(const float* x, int64_t n_at
   // the previous call's absmax words are still there: clear what this call uses
   JANUS_CUDA_TRY(cudaMemsetAsync(scratch, 0, sizeof(WsHeader) + sizeof(uint32_t) * (size_t)n_types, stream));
   const size_t smem = sizeof(uint32_t) * (size_t)n_types;
-  const unsigned grid = rows_grid(n_atoms, 8);
+  const unsigned grid = rows_grid(row_items(n_atoms, d / 4), 8);
   if (n_atoms > 0)
     quant_amax_kernel<<<grid, kThreads, smem, stream>>>((const float4*)x, n_atoms, d / 4, types, n_types,
                                                         amax_bits, hdr);

@@ -29,6 +29,30 @@ __device__ __forceinline__ int64_t total_warps() {
   return (int64_t)gridDim.x * blockDim.x / 32;
 }
 
+// Work items of the row-streaming kernels: (row, chunk of 32 * kU float4
+// columns).  Warp w of the grid always takes column chunk w % nch and strides
+// over the rows w / nch, w / nch + W / nch, ... (W warps, nch chunks per row),
+// so a layer with fewer rows than the grid has warps (the S layer's 8,192
+// atoms, the L layer's 16,384 receivers) still fills every warp, the chunks of
+// one row go to neighbouring warps at about the same time, and no warp divides
+// per item.  The last W % nch warps of the grid stay idle.
+constexpr int kChunk4 = 32 * kU;
+inline int64_t row_items(int64_t rows, int d4) { return rows * ((d4 + kChunk4 - 1) / kChunk4); }
+
+struct ChunkWalk {
+  int64_t row0, stride;   // first row, row stride (0 rows for an idle warp)
+  int c0;                 // first float4 column of the warp's chunk
+};
+__device__ __forceinline__ ChunkWalk chunk_walk(int d4) {
+  const int nch = (d4 + kChunk4 - 1) / kChunk4;
+  const int64_t w = global_warp(), W = total_warps();
+  ChunkWalk cw;
+  cw.stride = W / nch;
+  cw.row0 = w < cw.stride * nch ? w / nch : INT64_MAX;
+  cw.c0 = (int)(w % nch) * kChunk4;
+  return cw;
+}
+
 // ---- atom-type-aware FP16 packing: per-type absmax and scale ------------
 
 // |x| as ordered bits: for non-negative floats the integer order is the
@@ -43,7 +67,9 @@ quant_amax_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4,
   for (int t = threadIdx.x; t < T; t += kThreads) s_amax[t] = 0;
   __syncthreads();
   const int lane = threadIdx.x % 32;
-  for (int64_t i = global_warp(); i < n_atoms; i += total_warps()) {
+  const ChunkWalk cw = chunk_walk(d4);
+  const int c0 = cw.c0;
+  for (int64_t i = cw.row0; i < n_atoms; i += cw.stride) {
     int t = types[i];
     if (t < 0 || t >= T) {
       if (lane == 0) record_fault(ws, kFaultBadType);
@@ -51,17 +77,15 @@ quant_amax_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4,
     }
     const float4* src = x + i * d4;
     uint32_t m = 0;
-    for (int c0 = 0; c0 < d4; c0 += 32 * kU) {
-      float4 v[kU];
+    float4 v[kU];
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int c = c0 + u * 32 + lane;
-        v[u] = c < d4 ? __ldg(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < kU; ++u)
-        m = max(m, max(max(abs_bits(v[u].x), abs_bits(v[u].y)), max(abs_bits(v[u].z), abs_bits(v[u].w))));
+    for (int u = 0; u < kU; ++u) {
+      const int c = c0 + u * 32 + lane;
+      v[u] = c < d4 ? __ldg(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      m = max(m, max(max(abs_bits(v[u].x), abs_bits(v[u].y)), max(abs_bits(v[u].z), abs_bits(v[u].w))));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0 && m) atomicMax(&s_amax[t], m);

@@ -20,8 +20,14 @@ One pass, all on the current stream:
 `run_host` runs the pass from and to pinned host memory with the copies on
 their own streams: the upload of G overlaps the forward, the download of Y
 overlaps the VJP, and the next call's upload overlaps this call's compute
-(inputs and outputs are double-buffered on the device).
+(inputs and outputs are double-buffered on the device).  When the input is
+edge messages, they are streamed instead: the receivers are cut into chunks
+whose messages fit a ring of device buffers, each chunk's messages are
+uploaded into a free ring slot and aggregated from there as soon as they land,
+so the messages never need a device copy of their own and the upload of the
+next call's first chunks overlaps this call's MoE compute.
 """
+import numpy as np
 import torch
 
 from . import janus as J
@@ -33,6 +39,10 @@ class MoELayer:
     # this library's kernels per call (see each entry point's launches)
     LAUNCHES = {"edge_aggregate": 1, "quant": 2, "dequant": 1, "row_scales": 1, "route": 4, "dispatch": 1,
                 "ffn_fwd": 2, "combine": 1, "dispatch_w": 1, "ffn_vjp": 2, "combine_vjp": 1}
+
+    # pinned-host pipeline for edge-message inputs: ring of device buffers
+    RING_SLOTS = 8
+    RING_SLOT_BYTES = 512 << 20
 
     def __init__(self, n_atoms, top_k, gate, w1, w2, *, mode=J.JANUS_FFN_3XTF32, packed=False,
                  row_ptr=None):
@@ -86,10 +96,11 @@ class MoELayer:
         self._host = None
 
     # -- device-resident pass ----------------------------------------------------
-    def forward_vjp(self, x, g, types, events=None, y=None, dx=None, after_forward=None):
+    def forward_vjp(self, x, g, types, events=None, y=None, dx=None, after_forward=None, aggregated=False):
         """One pass on device tensors; returns (y, dx) (the layer's own buffers
         unless y / dx are given).  events: dict op -> (start, end) CUDA events;
-        after_forward: called once y is enqueued, before the VJP."""
+        after_forward: called once y is enqueued, before the VJP; aggregated:
+        the edge messages were already aggregated into self.xagg (x unused)."""
         K, T, r = self.K, self.T, self.route_out
         y = self.y if y is None else y
         dx = self.dx if dx is None else dx
@@ -98,7 +109,9 @@ class MoELayer:
             if events is not None:
                 events[op][i].record()
 
-        if self.row_ptr is not None:
+        if aggregated:
+            x = self.xagg
+        elif self.row_ptr is not None:
             mark("edge_aggregate", 0)
             J.janus_edge_aggregate(x, self.row_ptr, out=self.xagg)
             mark("edge_aggregate", 1)
@@ -153,17 +166,45 @@ class MoELayer:
         return y, dx
 
     # -- pass from and to pinned host memory, copies overlapped -------------------
+    def _edge_chunks(self, d):
+        """Receiver chunks [i0, i1) whose messages [e0, e1) fit one ring slot,
+        from the host copy of row_ptr (a receiver with more edges than a slot
+        holds gets a chunk, and the slots that size, of its own)."""
+        rp = self.row_ptr.cpu().numpy()
+        slot_rows = max(1, self.RING_SLOT_BYTES // (4 * d))
+        slot_rows = max(slot_rows, int((rp[1:] - rp[:-1]).max(initial=0)))
+        chunks, i0 = [], 0
+        N = rp.shape[0] - 1
+        while i0 < N:
+            # the last receiver i1 with rp[i1] - rp[i0] <= slot_rows
+            i1 = int(np.searchsorted(rp, rp[i0] + slot_rows, side="right")) - 1
+            i1 = max(i0 + 1, min(i1, N))
+            chunks.append((i0, i1, int(rp[i0]), int(rp[i1])))
+            i0 = i1
+        return chunks, slot_rows
+
     def _host_state(self, x_shape):
         dev = self.dev
         f32 = dict(dtype=torch.float32, device=dev)
         st = {
             "copy_in": torch.cuda.Stream(dev), "copy_out": torch.cuda.Stream(dev), "k": 0,
-            "x": [torch.empty(x_shape, **f32) for _ in range(2)],
             "g": [torch.empty((self.N, self.d), **f32) for _ in range(2)],
             "types": [torch.empty((self.N,), dtype=torch.int32, device=dev) for _ in range(2)],
             "y": [torch.empty((self.N, self.d), **f32) for _ in range(2)],
             "dx": [torch.empty((self.N, self.d), **f32) for _ in range(2)],
         }
+        if self.row_ptr is None:
+            st["x"] = [torch.empty(x_shape, **f32) for _ in range(2)]
+        else:
+            # edge messages: streamed through a ring of device buffers
+            st["chunks"], slot_rows = self._edge_chunks(x_shape[1])
+            n_slots = min(self.RING_SLOTS, max(1, len(st["chunks"])))
+            st["ring"] = [torch.empty((slot_rows, x_shape[1]), **f32) for _ in range(n_slots)]
+            st["ring_in"] = [torch.cuda.Event() for _ in range(n_slots)]
+            st["ring_free"] = [torch.cuda.Event() for _ in range(n_slots)]
+            st["ring_next"] = 0
+            for ev in st["ring_free"]:
+                ev.record(torch.cuda.current_stream(dev))
         for name in ("x_in", "g_in", "in_free", "y_done", "dx_done", "y_out", "dx_out"):
             st[name] = [torch.cuda.Event() for _ in range(2)]
         for b in range(2):      # nothing is in flight yet
@@ -171,10 +212,26 @@ class MoELayer:
                 st[name][b].record(torch.cuda.current_stream(dev))
         return st
 
+    def _stream_edges(self, st, msg_h, s, cin):
+        """Upload the edge messages chunk by chunk into the ring and aggregate
+        each chunk into self.xagg on stream s as soon as it has landed."""
+        ring = st["ring"]
+        n = len(ring)
+        for (i0, i1, e0, e1) in st["chunks"]:
+            j = st["ring_next"] % n
+            st["ring_next"] += 1
+            cin.wait_event(st["ring_free"][j])
+            with torch.cuda.stream(cin):
+                ring[j][:e1 - e0].copy_(msg_h[e0:e1], non_blocking=True)
+                st["ring_in"][j].record(cin)
+            s.wait_event(st["ring_in"][j])
+            J.janus_edge_aggregate(ring[j][:e1 - e0], self.row_ptr[i0:i1 + 1], out=self.xagg[i0:i1])
+            st["ring_free"][j].record(s)
+
     def run_host(self, x_h, g_h, types_h, y_h, dx_h):
         """Enqueue one pass from pinned host inputs (x [N,d] or the edge
-        messages, g [N,d], types [N]) into pinned host outputs y_h, dx_h.
-        Returns at once; the outputs are complete after `host_sync()`."""
+        messages [Ed,d], g [N,d], types [N]) into pinned host outputs y_h,
+        dx_h.  Returns at once; the outputs are complete after `host_sync()`."""
         if self._host is None:
             self._host = self._host_state(tuple(x_h.shape))
         st = self._host
@@ -183,14 +240,19 @@ class MoELayer:
         s = torch.cuda.current_stream(self.dev)
         cin, cout = st["copy_in"], st["copy_out"]
         # inputs: buffer set b is free once the pass that last used it is done
+        edges = self.row_ptr is not None
         cin.wait_event(st["in_free"][b])
         with torch.cuda.stream(cin):
             st["types"][b].copy_(types_h, non_blocking=True)
-            st["x"][b].copy_(x_h, non_blocking=True)
+            if not edges:
+                st["x"][b].copy_(x_h, non_blocking=True)
             st["x_in"][b].record(cin)
+        s.wait_event(st["x_in"][b])
+        if edges:
+            self._stream_edges(st, x_h, s, cin)
+        with torch.cuda.stream(cin):
             st["g"][b].copy_(g_h, non_blocking=True)
             st["g_in"][b].record(cin)
-        s.wait_event(st["x_in"][b])
         s.wait_event(st["y_out"][b])           # y buffer b downloaded by its previous pass
         s.wait_event(st["dx_out"][b])
 
@@ -202,8 +264,8 @@ class MoELayer:
                 st["y_out"][b].record(cout)
             s.wait_event(st["g_in"][b])
 
-        self.forward_vjp(st["x"][b], st["g"][b], st["types"][b], y=st["y"][b], dx=st["dx"][b],
-                         after_forward=after_fwd)
+        self.forward_vjp(None if edges else st["x"][b], st["g"][b], st["types"][b], y=st["y"][b],
+                         dx=st["dx"][b], after_forward=after_fwd, aggregated=edges)
         st["in_free"][b].record(s)
         st["dx_done"][b].record(s)
         cout.wait_event(st["dx_done"][b])

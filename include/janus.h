@@ -68,8 +68,10 @@ const char* janus_status_string(janus_status s);
 int32_t janus_version(void);
 
 /* Synchronises `stream`, then reads the error word at the start of a
- * workspace used by janus_route or janus_quant_by_type.  Returns JANUS_OK,
- * JANUS_ERR_DATA if a kernel recorded a data fault, or JANUS_ERR_CUDA. */
+ * workspace used by a call that takes one (routing, packing, the expert MLP
+ * calls, the expert-parallel sends); each such call clears the word when it
+ * starts (janus_ep_dispatch: see there).  Returns JANUS_OK, JANUS_ERR_DATA
+ * if a kernel recorded a data fault, or JANUS_ERR_CUDA. */
 janus_status janus_check(const void* workspace, janus_stream_t stream);
 
 /* -------------------------------------------------------------------------
@@ -228,6 +230,9 @@ janus_status janus_dispatch_row_scales(int64_t n_atoms, int32_t top_k, const int
  *                         a TF32 high part and a TF32 residual, three products.
  * fwd: act [R,h] (nullable) receives a; the workspace holds silu(a).
  * vjp: act (nullable) is a from the forward; NULL recomputes it.
+ * The workspace's error word (janus_check) is cleared by every call and
+ * receives a bounded tensor-core wait that ran out, rows that break
+ * JANUS_FFN_X_DEQUANTIZED, and (debug build) a malformed offsets array.
  * ------------------------------------------------------------------------- */
 typedef enum { JANUS_FFN_FP32_SIMT = 0, JANUS_FFN_3XTF32 = 1 } janus_ffn_mode;
 

@@ -23,6 +23,22 @@ def rel_fro(got, ref) -> float:
     return float(num / den) if den > 0 else float(num)
 
 
+def max_row_rel(got, ref) -> float:
+    """Largest per-row relative error ||got_i - ref_i|| / ||ref_i|| (a local
+    error that a norm over many rows would hide)."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    num = np.linalg.norm(got - ref, axis=1)
+    den = np.linalg.norm(ref, axis=1)
+    return float(np.max(np.where(den > 0, num / np.where(den > 0, den, 1.0), num)))
+
+
+# Per-row bound for the full-size sampled comparisons: the relative Frobenius
+# bar over the sample stays TOL_FP32, and no single row may be off by more
+# than ten times that.
+TOL_ROW = 1e-4
+
+
 def to_dev(a, dtype=None):
     t = torch.as_tensor(a)
     if dtype is not None:

@@ -32,6 +32,9 @@ def test_bench_line_carries_the_contract_keys():
     roof = d["roofline"]
     assert roof["bound"] in ("tensor", "hbm", "alu") and roof["peak"] > 0
     assert abs(roof["frac"] - roof["achieved"] / roof["peak"]) <= 1e-9 * max(1.0, roof["frac"])
+    assert len(roof["peak_per_gemm"]) == roof["launches_per_step"] == 4
+    cold = d["kernels_cold_l2"]
+    assert {"dispatch", "combine", "edge_aggregate"} <= set(cold) and all(v["ms"] > 0 for v in cold.values())
     e2e = d["e2e"]
     assert e2e["value"] > 0 and e2e["h2d_bytes_per_step"] > 0 and e2e["d2h_bytes_per_step"] > 0
     # this library's kernels: route 4, edge aggregation 1, dispatch 1, MLP 2 + 2,
@@ -39,7 +42,7 @@ def test_bench_line_carries_the_contract_keys():
     assert d["gpu_launches"] == 13 * d["steps"]
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] > 0
-    assert "sm_mhz" in d["clocks"] and "reasons" in d["clocks"]
+    assert "sm_mhz" in d["clocks"] and "reasons" in d["clocks"] and d["clocks"]["samples_in_timed_region"] >= 1
 
 
 def test_reference_arm_line():

@@ -9,7 +9,7 @@ import torch
 import oracle
 from element_routed_moe_b200 import janus as J
 from element_routed_moe_b200 import synth
-from helpers import DEV, TOL_FP32, host, poison_like, rel_fro, sample_rows, to_dev
+from helpers import DEV, TOL_FP32, TOL_ROW, host, max_row_rel, poison_like, rel_fro, sample_rows, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -99,5 +99,7 @@ def test_ffn_full_size_sampled_rows(name, mode):
     ref_dx = oracle.expert_ffn_vjp(host(xd), host(gd), offs, hw1, hw2, rows=rows)
     assert rel_fro(host(yd)[rows], ref_y) <= TOL_FP32
     assert rel_fro(host(dxd)[rows], ref_dx) <= TOL_FP32
+    assert max_row_rel(host(yd)[rows], ref_y) <= TOL_ROW
+    assert max_row_rel(host(dxd)[rows], ref_dx) <= TOL_ROW
     # every row was written
     assert torch.isfinite(yd).all().item() and torch.isfinite(dxd).all().item()
