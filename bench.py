@@ -226,7 +226,12 @@ class ClockSampler:
 # launches), from ncu captures of a smaller case of the same workload scaled
 # to full size by its routed rows; valid only for the kernel source it was
 # taken on (else reported as null).
-GEMM_TRAFFIC = {}
+GEMM_TRAFFIC = {
+    # slice-shaped MoE layer captured at 4,096 and 8,192 atoms, fitted as
+    # 0.41 GB (weights) + b * rows per launch and taken to R = 524,288
+    ("slice", "3xtf32"): {"src": "element_routed_moe_b200/csrc/ffn_tc.cu", "sha256_prefix": "2fbccd613e3b6b18",
+                          "bytes_per_launch": 7.92e9},
+}
 
 
 def measured_traffic(workload: str, mode: str):
