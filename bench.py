@@ -298,8 +298,11 @@ class Layer:
     def work(self):
         c = self.cfg
         N, R, d, h = c.n_atoms, c.n_rows, c.d, c.h
+        split = self.core.split
         w = {
-            "dispatch": ("bytes", 4 * d * (N + R) + 4 * R),
+            # split dispatch: a first pass reads X for the row maxima; the two
+            # FP16 planes are as many bytes as the FP32 rows, plus a scale per row
+            "dispatch": ("bytes", 4 * d * (N + R) + 4 * R + ((4 * N * d + 4 * R) if split else 0)),
             "dispatch_w": ("bytes", 4 * d * (N + R) + 8 * R),
             "combine": ("bytes", 4 * d * (R + N) + 8 * R),
             "combine_vjp": ("bytes", 4 * d * (R + N) + 4 * R),
@@ -428,37 +431,41 @@ def run_reference(args, world, rank):
 # --------------------------------------------------------------------------
 # janus arm
 # --------------------------------------------------------------------------
-def gemm_roofline(J, mode, cfg, packed_first, peaks, peak_src, flops_per_gemm, ms_total, launches):
+def gemm_roofline(J, mode, cfg, kinds, peaks, peak_src, flops_per_gemm, ms_total, launches):
     """Roofline of the grouped expert-MLP GEMM over a step's launches.
 
-    3xTF32: a GEMM that issues p tensor-core products per k-step has an
-    FP32-accurate peak of (TF32 peak) / p; TF32 peak = measured burst BF16 x the
-    nominal TF32/BF16 ratio (1.125 / 2.25).  The forward's first GEMM issues
-    p = 2 when its rows are FP16-packed (an unpacked FP16 row is exact in TF32:
-    its residual product is skipped), every other GEMM p = 3.  The combined
-    peak is the FLOP-weighted harmonic mean, so frac = (sum of each launch's
-    ideal time) / (measured time).  SIMT: 148 SMs x 128 FP32 lanes x 2 FLOP x
-    the maximum SM clock, the same for every launch."""
-    tf32 = peaks["bf16_tflops"] * (1.125 / 2.25)
+    Each launch's FP32-accurate peak is the tensor peak of the operand kind it
+    runs on divided by the products it issues per k-step:
+      3xTF32 (every GEMM on FP32 rows): TF32 peak / 3, with TF32 peak =
+        measured burst BF16 x the nominal TF32/BF16 ratio (1.125 / 2.25);
+      FP16 rows x two-term FP16 split of the weights (the packed forward's
+        first GEMM): FP16 peak / 2, FP16 peak = the measured burst BF16 figure
+        (the same nominal rate);
+      two-term FP16 rows x two-term FP16 weights (the first GEMM of each
+        direction on split rows): FP16 peak / 3;
+      unpacked FP16 rows on TF32 (packed layers with d % 8 != 0): TF32 / 2.
+    `kinds` lists each launch's (kind, products) in step order.
+    The combined peak is the FLOP-weighted harmonic mean, so frac = (sum of
+    each launch's ideal time) / (measured time).  SIMT: 148 SMs x 128 FP32
+    lanes x 2 FLOP x the maximum SM clock, the same for every launch."""
+    bf16 = peaks["bf16_tflops"]
+    tf32 = bf16 * (1.125 / 2.25)
     if mode == J.JANUS_FFN_FP32_SIMT:
         per = [SM_COUNT * FP32_LANES_PER_SM * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12] * launches
         roof = {"bound": "alu", "peak_source": "148 SMs x 128 FP32 lanes x 2 FLOP x max SM clock"}
     else:
-        products = [2 if (i == 0 and packed_first) else 3 for i in range(launches)]
-        per = [tf32 / p for p in products]
+        per = [(bf16 if k == "f16" else tf32) / p for k, p in kinds]
         roof = {"bound": "tensor",
-                "peak_source": f"{peak_src} burst bf16 x (TF32/BF16 nominal 1.125/2.25) / products per GEMM "
-                               f"({products}: the FP16-packed forward's first GEMM skips the rows' zero "
-                               f"residual)",
-                "products_per_gemm": products}
+                "peak_source": f"{peak_src} burst bf16 (FP16 kind; x 1.125/2.25 for TF32) / products per GEMM "
+                               f"{[f'{k}x{p}' for k, p in kinds]}",
+                "gemm_kinds": [f"{k}x{p}" for k, p in kinds]}
     flops = flops_per_gemm * launches
     ideal_s = sum(flops_per_gemm / (pk * 1e12) for pk in per)
     peak = flops / ideal_s / 1e12
     achieved = flops / (ms_total * 1e-3) / 1e12
     roof.update({"kernel": "grouped expert-MLP GEMM", "achieved": achieved, "peak": peak,
                  "peak_per_gemm": per, "unit": "TFLOP/s", "frac": achieved / peak,
-                 "frac_of_sustained_peak": achieved / (peak * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-                                                       / peaks["bf16_tflops"]),
+                 "frac_of_sustained_peak": achieved / (peak * peaks.get("bf16_tflops_sustained", bf16) / bf16),
                  "algorithmic_flops_per_launch": flops_per_gemm, "launches_per_step": launches})
     return roof
 
@@ -516,7 +523,13 @@ def run_janus(args, world, rank, local):
     # per step: two forward, two VJP, each 2*R*d*h FLOPs), timed by CUDA
     # events on the launching stream inside the timed steps
     ffn_ms = op_ms["ffn_fwd"] + op_ms["ffn_vjp"]
-    roof = gemm_roofline(J, mode, cfg, layer.packed, peaks, peak_src, work["ffn_fwd"][1] / 2, ffn_ms, 4)
+    core = layer.core
+    if core.packed:
+        first = ("f16", 2) if core.fused_unpack else ("tf32", 2)
+    else:
+        first = ("f16", 3) if core.split else ("tf32", 3)
+    kinds = [first, ("f16", 3) if core.f16_second else ("tf32", 3), ("tf32", 3), ("tf32", 3)]
+    roof = gemm_roofline(J, mode, cfg, kinds, peaks, peak_src, work["ffn_fwd"][1] / 2, ffn_ms, 4)
     roof["traffic"] = measured_traffic(cfg.name, args.mode) if cfg == synth.CONFIGS[cfg.name] else None
     roof["traffic_unit"] = "DRAM bytes per launch (mean of the step's 4 launches)"
     ws_gb = ((layer.w1.numel() + layer.w2.numel()) * 4 + cfg.n_rows * cfg.d * 4 * 4) / 1e9
@@ -657,7 +670,9 @@ def run_ep(args, world, rank, local):
     r_recv = int(layer.layout[2][rank][-1].item())
     ffn_ms = ph_ms["ffn_fwd"] + ph_ms["ffn_vjp"]
     # the owner's first forward GEMM runs on the received FP16 rows: 2 products
-    roof = gemm_roofline(J, mode, cfg, True, peaks, peak_src, 2.0 * r_recv * d * h, max(ffn_ms, 1e-9), 4)
+    kinds = [("f16", 2) if layer.fused_unpack else ("tf32", 2), ("f16", 3) if layer.f16_second else ("tf32", 3),
+             ("tf32", 3), ("tf32", 3)]
+    roof = gemm_roofline(J, mode, cfg, kinds, peaks, peak_src, 2.0 * r_recv * d * h, max(ffn_ms, 1e-9), 4)
     roof.update({"kernel": "grouped expert-MLP GEMM (rank 0's experts; ffn phases include the FP16 unpack)",
                  "traffic": None})
     line = {
@@ -698,10 +713,15 @@ def run_extras(layer, peaks):
     N, R, d, h, E, K, T = cfg.n_atoms, cfg.n_rows, cfg.d, cfg.h, cfg.n_experts, cfg.top_k, cfg.n_types
     r = layer.route_out
     out = {}
-    if layer.core.packed and layer.core.fused_unpack:
-        # the step never writes xd (its first GEMM reads the FP16 rows): the
-        # weight-gradient extras need the unpacked rows, written here untimed
+    # the weight-gradient extras take the FP32 dispatch rows, which the step
+    # does not write on its FP16 tensor path (FP16 payload or split rows):
+    # written here, untimed
+    x_in = layer.core.xagg if layer.edges else layer.x
+    if layer.core.packed:
         J.janus_dequant_by_type(layer.core.payload, layer.types, T, r["perm"], K, layer.core.scale, out=layer.xd)
+    else:
+        J.janus_dispatch(x_in, r["slot_of"], K, out=layer.xd)
+    J.janus_dispatch(layer.g, r["slot_of"], K, r["topk_weight"], out=layer.gd)
     dw1 = torch.empty_like(layer.w1)
     dw2 = torch.empty_like(layer.w2)
     ws = torch.empty(J.janus_expert_ffn_weight_grad_workspace_size(R, h, True), dtype=torch.uint8,

@@ -88,8 +88,40 @@ unpack_rows_kernel(const uint2* __restrict__ payload, const float* __restrict__ 
   }
 }
 
-size_t packed_extra(int64_t R, int32_t d, janus_ffn_mode mode) {
-  return mode == JANUS_FFN_FP32_SIMT ? align_up(sizeof(float) * (size_t)R * (size_t)d, 256) : 0;
+// The forward's second GEMM (H W2) runs on the kind::f16 path too when the
+// layer has at least this many routed rows per expert: its row split of H and
+// the per-call split of W2 then cost less than the GEMM saves.
+constexpr int64_t kF16SecondMinRowsPerExpert = 2048;
+bool use_f16_second(int64_t R, int32_t E, int32_t h) {
+  return h % 8 == 0 && R >= kF16SecondMinRowsPerExpert * E;
+}
+
+// Scratch of the FP16 second GEMM (see tc::F16Second), starting at `base`.
+size_t f16_second_bytes(int64_t R, int32_t E, int32_t d, int32_t h) {
+  return align_up(2 * sizeof(uint16_t) * (size_t)R * h, 256) + 2 * align_up(sizeof(float) * (size_t)R, 256) +
+         align_up(2 * sizeof(uint16_t) * (size_t)E * d * h, 256) + align_up(sizeof(float) * (size_t)E * d, 256);
+}
+tc::F16Second f16_second_at(char* base, int64_t R, int32_t E, int32_t d, int32_t h) {
+  tc::F16Second f;
+  f.h16 = (uint16_t*)base;
+  base += align_up(2 * sizeof(uint16_t) * (size_t)R * h, 256);
+  f.hscale = (float*)base;
+  base += align_up(sizeof(float) * (size_t)R, 256);
+  f.rowmax = (uint32_t*)base;
+  base += align_up(sizeof(float) * (size_t)R, 256);
+  f.w16 = (uint16_t*)base;
+  base += align_up(2 * sizeof(uint16_t) * (size_t)E * d * h, 256);
+  f.winv = (float*)base;
+  return f;
+}
+
+// Past the forward's activations: SIMT, the unpacked rows [R,d] FP32;
+// 3xTF32, the FP16 split of W1 (hi and mid, [E][h][d] each), 1 / S [E][h],
+// and the FP16 second GEMM's scratch when it is used.
+size_t packed_extra(int64_t R, int32_t E, int32_t d, int32_t h, janus_ffn_mode mode) {
+  if (mode == JANUS_FFN_FP32_SIMT) return align_up(sizeof(float) * (size_t)R * (size_t)d, 256);
+  return align_up(2 * sizeof(uint16_t) * (size_t)E * d * h, 256) + align_up(sizeof(float) * (size_t)E * h, 256) +
+         (use_f16_second(R, E, h) ? f16_second_bytes(R, E, d, h) : 0);
 }
 
 }  // namespace
@@ -97,11 +129,11 @@ size_t packed_extra(int64_t R, int32_t d, janus_ffn_mode mode) {
 
 using namespace janus;
 
-extern "C" janus_status janus_expert_ffn_packed_workspace_size(int64_t n_rows, int32_t d, int32_t h,
-                                                               janus_ffn_mode mode, size_t* bytes) {
-  JANUS_CHECK_ARG(bytes && n_rows >= 0 && d >= 1 && h >= 1);
+extern "C" janus_status janus_expert_ffn_packed_workspace_size(int64_t n_rows, int32_t n_experts, int32_t d,
+                                                               int32_t h, janus_ffn_mode mode, size_t* bytes) {
+  JANUS_CHECK_ARG(bytes && n_rows >= 0 && d >= 1 && h >= 1 && n_experts >= 1 && n_experts <= kMaxExperts);
   JANUS_CHECK_ARG(mode == JANUS_FFN_FP32_SIMT || mode == JANUS_FFN_3XTF32);
-  *bytes = ffn_layout(n_rows, h, false, true).total + packed_extra(n_rows, d, mode);
+  *bytes = ffn_layout(n_rows, h, false, true).total + packed_extra(n_rows, n_experts, d, h, mode);
   return JANUS_OK;
 }
 
@@ -122,7 +154,7 @@ extern "C" janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, con
   JANUS_CHECK_ALIGN(mode != JANUS_FFN_3XTF32 || d % 8 == 0);   // FP16 rows: 16-byte TMA strides
   JANUS_CHECK_ALIGN(act == nullptr || aligned(act, 16));
   const FfnLayout L = ffn_layout(n_rows, h, false, true);
-  const size_t extra = packed_extra(n_rows, d, mode);
+  const size_t extra = packed_extra(n_rows, n_experts, d, h, mode);
   JANUS_CHECK_ARG(workspace && workspace_bytes >= L.total + extra);
   JANUS_CHECK_ALIGN(aligned(workspace, 256));
   if (n_rows == 0) return JANUS_OK;
@@ -132,8 +164,14 @@ extern "C" janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, con
   // workspace reports only this call's faults
   JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
   if (mode == JANUS_FFN_3XTF32) {
-    st = tc::expert_ffn_fwd_packed(payload, row_scale, offsets, n_experts, n_rows, d, h, w1, w2, yd, act, H,
-                                   &((WsHeader*)workspace)->error, stream, yd_rows);
+    uint16_t* w16 = (uint16_t*)((char*)workspace + L.total);
+    const size_t w16_bytes = align_up(2 * sizeof(uint16_t) * (size_t)n_experts * d * h, 256);
+    float* winv = (float*)((char*)workspace + L.total + w16_bytes);
+    char* second_base = (char*)workspace + L.total + w16_bytes + align_up(sizeof(float) * (size_t)n_experts * h, 256);
+    const tc::F16Second second = f16_second_at(second_base, n_rows, n_experts, d, h);
+    st = tc::expert_ffn_fwd_packed(payload, row_scale, offsets, n_experts, n_rows, d, h, w1, w2, yd, act, H, w16,
+                                   winv, &((WsHeader*)workspace)->error, stream, yd_rows,
+                                   use_f16_second(n_rows, n_experts, h) ? &second : nullptr);
     if (st != JANUS_OK) return st;
     return launch_status();
   }
@@ -147,6 +185,102 @@ extern "C" janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, con
   simt::Args a2 = make_args(H, w2, sw, yd, nullptr, nullptr, offsets, n_experts, h, d, n_rows);
   a2.c_rows = yd_rows;
   launch_simt<false, simt::kEpiStore>(a2, stream);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// The expert MLP on rows given as two FP16 terms with a per-row scale
+// (janus_dispatch_split): the first GEMM of the forward (x W1) or of the VJP
+// (gd W2^T, dSiLU epilogue) on the kind::f16 tensor path, the second on
+// 3xTF32.  Workspace: header | H or dA [R,h] | the FP16 split of the first
+// GEMM's weights (hi and mid, [E][h][d] each) | 1 / S [E][h].
+// ---------------------------------------------------------------------------
+namespace {
+struct SplitLayout {
+  size_t off_h, off_w16, off_winv, off_second, total;
+};
+SplitLayout split_layout(int64_t R, int32_t E, int32_t d, int32_t h) {
+  SplitLayout L;
+  L.off_h = sizeof(WsHeader);
+  L.off_w16 = L.off_h + align_up(sizeof(float) * (size_t)R * (size_t)h, 256);
+  L.off_winv = L.off_w16 + align_up(2 * sizeof(uint16_t) * (size_t)E * d * h, 256);
+  L.off_second = L.off_winv + align_up(sizeof(float) * (size_t)E * h, 256);
+  L.total = L.off_second + (use_f16_second(R, E, h) ? f16_second_bytes(R, E, d, h) : 0);
+  return L;
+}
+
+janus_status check_split(const uint16_t* rows16, const float* row_scale, const int32_t* offsets, int32_t E,
+                         int64_t R, int32_t d, int32_t h, const float* w1, const float* w2, const void* out,
+                         void* workspace, size_t workspace_bytes) {
+  JANUS_CHECK_ARG(E >= 1 && E <= kMaxExperts);
+  JANUS_CHECK_ARG(R >= 0 && R < (int64_t)INT32_MAX / 2);
+  JANUS_CHECK_ARG(d >= 1 && d <= kMaxDim && h >= 1 && h <= kMaxDim);
+  JANUS_CHECK_ALIGN(d % 8 == 0 && h % 4 == 0);
+  JANUS_CHECK_ARG(offsets && w1 && w2);
+  JANUS_CHECK_ARG(R == 0 || (rows16 && row_scale && out));
+  JANUS_CHECK_ALIGN(aligned(w1, 16) && aligned(w2, 16));
+  JANUS_CHECK_ALIGN(R == 0 || (aligned(rows16, 16) && aligned(out, 16)));
+  JANUS_CHECK_ARG(workspace && workspace_bytes >= split_layout(R, E, d, h).total);
+  JANUS_CHECK_ALIGN(aligned(workspace, 256));
+  return JANUS_OK;
+}
+}  // namespace
+
+extern "C" janus_status janus_expert_ffn_split_workspace_size(int64_t n_rows, int32_t n_experts, int32_t d,
+                                                              int32_t h, size_t* bytes) {
+  JANUS_CHECK_ARG(bytes && n_rows >= 0 && d >= 1 && h >= 1 && n_experts >= 1 && n_experts <= kMaxExperts);
+  *bytes = split_layout(n_rows, n_experts, d, h).total;
+  return JANUS_OK;
+}
+
+extern "C" janus_status janus_expert_ffn_fwd_split(const uint16_t* rows16, const float* row_scale,
+                                                   const int32_t* offsets, int32_t n_experts, int64_t n_rows,
+                                                   int32_t d, int32_t h, const float* w1, const float* w2,
+                                                   float* yd, float* const* yd_rows, float* act, void* workspace,
+                                                   size_t workspace_bytes, janus_stream_t stream_) {
+  cudaStream_t stream = (cudaStream_t)stream_;
+  JANUS_CHECK_ARG((yd == nullptr) != (yd_rows == nullptr) || n_rows == 0);
+  const void* outp = yd_rows ? (const void*)yd_rows : (const void*)yd;
+  janus_status st = check_split(rows16, row_scale, offsets, n_experts, n_rows, d, h, w1, w2, outp, workspace,
+                                workspace_bytes);
+  if (st != JANUS_OK) return st;
+  JANUS_CHECK_ALIGN(act == nullptr || aligned(act, 16));
+  if (n_rows == 0) return JANUS_OK;
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  const SplitLayout L = split_layout(n_rows, n_experts, d, h);
+  char* w = (char*)workspace;
+  JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
+  const tc::F16Second second = f16_second_at(w + L.off_second, n_rows, n_experts, d, h);
+  st = tc::expert_ffn_fwd_split(rows16, row_scale, offsets, n_experts, n_rows, d, h, w1, w2, yd, act,
+                                (float*)(w + L.off_h), (uint16_t*)(w + L.off_w16), (float*)(w + L.off_winv),
+                                &((WsHeader*)workspace)->error, stream, yd_rows,
+                                use_f16_second(n_rows, n_experts, h) ? &second : nullptr);
+  if (st != JANUS_OK) return st;
+  return launch_status();
+}
+
+extern "C" janus_status janus_expert_ffn_vjp_split(const uint16_t* gd16, const float* gd_scale, const float* act,
+                                                   const int32_t* offsets, int32_t n_experts, int64_t n_rows,
+                                                   int32_t d, int32_t h, const float* w1, const float* w2,
+                                                   float* dxd, float* const* dxd_rows, void* workspace,
+                                                   size_t workspace_bytes, janus_stream_t stream_) {
+  cudaStream_t stream = (cudaStream_t)stream_;
+  JANUS_CHECK_ARG((dxd == nullptr) != (dxd_rows == nullptr) || n_rows == 0);
+  const void* outp = dxd_rows ? (const void*)dxd_rows : (const void*)dxd;
+  janus_status st = check_split(gd16, gd_scale, offsets, n_experts, n_rows, d, h, w1, w2, outp, workspace,
+                                workspace_bytes);
+  if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(n_rows == 0 || act);
+  JANUS_CHECK_ALIGN(act == nullptr || aligned(act, 16));
+  if (n_rows == 0) return JANUS_OK;
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  const SplitLayout L = split_layout(n_rows, n_experts, d, h);
+  char* w = (char*)workspace;
+  JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
+  st = tc::expert_ffn_vjp_split(gd16, gd_scale, act, offsets, n_experts, n_rows, d, h, w1, w2, dxd,
+                                (float*)(w + L.off_h), (uint16_t*)(w + L.off_w16), (float*)(w + L.off_winv),
+                                &((WsHeader*)workspace)->error, stream, dxd_rows);
+  if (st != JANUS_OK) return st;
   return launch_status();
 }
 

@@ -1,5 +1,7 @@
-// Grouped expert-MLP GEMM on the 5th-generation tensor cores (tcgen05) with
-// the 3xTF32 split, for JANUS_FFN_3XTF32.
+// Grouped expert-MLP GEMM on the 5th-generation tensor cores (tcgen05), for
+// JANUS_FFN_3XTF32: the 3xTF32 split on kind::tf32, and (kBF16W / kBF16S
+// below) an FP16 form on kind::f16 for rows that arrive as FP16 values or as
+// two FP16 terms: the FP16-packed dispatch and the split dispatch.
 //
 // FP32 accuracy from TF32 tensor cores (Ootomo & Yokota 2022, "Recovering
 // single precision accuracy from Tensor Cores while surpassing the FP32
@@ -59,6 +61,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "ffn_tc.cuh"
@@ -114,12 +117,46 @@ enum Mode : int { kModeNN = 0, kModeNT = 1, kModeTN = 2 };
 //   kBSplit   FP32 rows, split into hi and lo by the splitters (3 products);
 //   kBExact   FP32 rows exact in TF32 (dequantized FP16): no lo, 2 products,
 //             the splitters only check the rows;
-//   kBHalf    the FP16 payload itself plus a per-row power-of-two scale: TMA
-//             lands the FP16 tile in the (unused) lo slot of B and the
-//             splitters write the FP32 rows, f32(q) * scale, into the B tile
-//             (exact, so again 2 products).  The unpack is fused into the GEMM.
-enum BKind : int { kBSplit = 0, kBExact = 1, kBHalf = 2 };
-constexpr uint32_t kTileBHalfBytes = BNH * BK * 2;       // 4 KB of FP16 rows per CTA
+//   kBF16W    the FP16 payload against an FP16 split of the weights, on the
+//             kind::f16 tensor path (below): no splitter work, 2 products;
+//   kBF16S    FP32 rows given as two FP16 terms (hi and mid planes of a
+//             [2R][Kd] tensor, from janus_dispatch_split) with a per-row
+//             power-of-two scale, against the FP16 split of the weights:
+//             3 products, hi.hi + hi.mid + mid.hi (mid.mid, below 2^-22 of
+//             the product, is dropped as in 3xTF32).
+enum BKind : int { kBSplit = 0, kBExact = 1, kBF16W = 3, kBF16S = 4 };
+
+// kBF16W: FP16 rows x FP16-split weights on tcgen05 kind::f16.
+// A packed row is q * s (q binary16, s a power of two), exact in FP16 up to
+// its scale.  Each weight column f of expert e is scaled by a power of two S
+// that puts its largest magnitude in [2^14, 2^15) and split into two FP16
+// terms, w S = hi + mid + r with |r| <= 2^-22 |w S| (the split the weight
+// pass below writes).  The tensor core multiplies FP16 operands exactly and
+// accumulates in FP32, so
+//   a[p, f] = s_p / S_f * sum_k q[p, k] (hi[f, k] + mid[f, k])
+// is as accurate as the 3xTF32 product, with two kind::f16 MMAs per 16-wide
+// k-step (a kind::f16 MMA covers twice the K of a TF32 one in the same time).
+// Both operands are K-major FP16 tiles with the 128-byte swizzle: a k-block is
+// 64 wide (128 bytes per row), a stage holds the weights' hi and mid tiles and
+// this CTA's rows (3 x 16 KB), 4 stages.
+constexpr int BK16 = 64;
+constexpr int kStages16 = 4, kStages16S = 3;
+constexpr uint32_t kTile16Bytes = BM * BK16 * 2;          // 16 KB: 128 rows x 128 bytes
+constexpr uint32_t kStage16Bytes = 3 * kTile16Bytes;      // A hi | A mid | B
+constexpr uint32_t kStage16SBytes = 4 * kTile16Bytes;     // A hi | A mid | B hi | B mid
+static_assert(kStages16 * kStage16Bytes <= kStages * kStageBytes, "the FP16 ring fits the same shared memory");
+static_assert(kStages16S * kStage16SBytes <= kStages * kStageBytes, "the FP16 ring fits the same shared memory");
+static_assert(kStages16 <= kNumSplitWarps && kStages16S <= kNumSplitWarps, "one relay warp per FP16 stage");
+template <int kBK> __host__ __device__ constexpr bool f16_path() { return kBK == kBF16W || kBK == kBF16S; }
+template <int kBK> __host__ __device__ constexpr int ring_stages() {
+  return kBK == kBF16W ? kStages16 : (kBK == kBF16S ? kStages16S : kStages);
+}
+template <int kBK> __host__ __device__ constexpr uint32_t ring_stage_bytes() {
+  return kBK == kBF16W ? kStage16Bytes : (kBK == kBF16S ? kStage16SBytes : kStageBytes);
+}
+template <int kBK> __host__ __device__ constexpr int kblock_width() { return f16_path<kBK>() ? BK16 : BK; }
+// k-blocks per TMEM chunk (K = 256 in both geometries)
+template <int kBK> __host__ __device__ constexpr int chunk_kblocks() { return 256 / kblock_width<kBK>(); }
 
 struct Args {
   float* C;
@@ -128,8 +165,9 @@ struct Args {
   const float* aux;
   const float* aux2;
   float* const* c_rows;   // NN/NT plain store: if set, row p goes to c_rows[p] (e.g. a peer's buffer)
-  const float* row_scale; // kBHalf: scale of dispatch row p
-  int64_t rows;           // rows of the dispatch operand (kBHalf: row_scale's length); offsets[E] <= rows
+  const float* row_scale; // kBF16W, kBF16S: scale of dispatch row p
+  const float* col_scale; // kBF16W, kBF16S: 1 / S of output feature f of expert e, [E][N]
+  int64_t rows;           // rows of the dispatch operand; offsets[E] <= rows
   const int32_t* offsets;
   int E, Kd, N;
   int M;            // kModeTN: MMA rows of each expert's product; C is [E][N][M] (stored transposed)
@@ -147,7 +185,6 @@ struct Smem {
   int abort;
   int off[kMaxExperts + 1];
   int start[kMaxExperts + 1];
-  float rscale[kNumSplitWarps][BNH];   // kBHalf: each splitter warp's row scales for its current tile
 };
 
 // ---- PTX wrappers ---------------------------------------------------------
@@ -240,13 +277,23 @@ __device__ __forceinline__ void tc_mma_tf32_pair(uint32_t d_tmem, uint64_t adesc
       : "memory");
 }
 
+__device__ __forceinline__ void tc_mma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor (tcgen05): start address, leading and
 // stride byte offsets (16-byte units), version 1, swizzle mode.
 // K-major operands use the 128-byte swizzle (mode 2; 16-byte granules XOR the
 // row mod 8).  An MN-major TF32 operand must use the 128-byte swizzle with
 // 32-byte atoms (mode 1; 32-byte granules XOR the row mod 4), which TMA writes
 // with CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B.
-constexpr uint32_t kSwizzle64B = 4, kSwizzle128B32B = 1;
+constexpr uint32_t kSwizzle64B = 4, kSwizzle128B32B = 1, kSwizzle128B = 2;
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
                                               uint32_t mode) {
   uint64_t d = 0;
@@ -263,6 +310,12 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 __host__ __device__ constexpr uint32_t instr_desc(bool a_mn_major, bool b_mn_major, uint32_t n = BN) {
   return (1u << 4) | (2u << 7) | (2u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
          ((n >> 3) << 17) | ((uint32_t)((2 * BM) >> 4) << 24);
+}
+
+// kind::f16 instruction descriptor: D=F32, A=B=F16 (format 0), both K-major,
+// M=256 (the CTA pair), N = n.
+__host__ __device__ constexpr uint32_t instr_desc_f16(uint32_t n) {
+  return (1u << 4) | ((n >> 3) << 17) | ((uint32_t)((2 * BM) >> 4) << 24);
 }
 
 // Epilogue activations.  The store phase is unrolled over 128 columns per
@@ -377,9 +430,10 @@ __device__ __forceinline__ void d2_store(const Args& args, const float (&acc)[kE
 
 // Epilogue warpgroups: fold each TMEM chunk into FP32 running sums, then apply
 // the fused epilogue and store this CTA's 128 x 256 part of the tile.
-template <int kMode, int kEpi>
+template <int kMode, int kEpi, int kBK>
 __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_t tmem_base, int warp, int lane,
                                               int n_tiles_n, int total, int nk_fixed, uint32_t rank, int n_pairs) {
+  constexpr int kChunk = chunk_kblocks<kBK>();
   const int wg = warp / 4;
   const int N = args.N;
   const int q = warp % 4;                  // TMEM lane quarter = 32 rows
@@ -392,7 +446,7 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
 #pragma unroll
     for (int j = 0; j < kEpiCols; ++j) acc[j] = 0.f;     // a tile with no k-blocks stores zeros
     bool ok = true;
-    for (int c0 = 0; c0 < c.nk; c0 += kChunkKb, ++ch) {
+    for (int c0 = 0; c0 < c.nk; c0 += kChunk, ++ch) {
       const uint32_t p = ch & 1, cuse = ch >> 1;
       if (!mbar_wait(s, &s->chunk_full[p], cuse & 1, args.err)) { ok = false; break; }
       tc_fence_after();
@@ -411,7 +465,7 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
       // the tile's pre-activations travel to L2 while its last two chunks
       // accumulate (late enough that they are still there for the store
       // phase: 1-3 % faster than prefetching at the first chunk)
-      const int pf_c0 = max(0, ((c.nk - 1) / kChunkKb - 1) * kChunkKb);
+      const int pf_c0 = max(0, ((c.nk - 1) / kChunk - 1) * kChunk);
       if (kMode != kModeTN && (kEpi == kEpiDSilu || kEpi == kEpiD2) && c0 == pf_c0) {
         const int f = c.m0 + q * 32 + lane;
         const int jn = min(kEpiCols, c.n_valid - half * kEpiCols);
@@ -436,6 +490,10 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
         continue;
       }
       if (f < c.m_end) {
+        // FP16 path: the product is q (hi + mid) S (kBF16S: q = the row's
+        // two terms); scale column j by its row's s_p and this lane's feature
+        // by 1 / S (powers of two: exact)
+        const float cscale = f16_path<kBK>() ? __ldg(args.col_scale + (int64_t)c.e * N + f) : 1.0f;
         // batches of 8 columns; the pre-activations of batch b + 1 are in
         // flight while batch b is finished, so two loads per column overlap
         constexpr int kB = 8;
@@ -457,6 +515,7 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
             if (j0 + jb + j < c.n_valid) {
               const int64_t o = (int64_t)(c.n0 + j0 + jb + j) * N + f;
               float v = acc[jb + j];
+              if (f16_path<kBK>()) v = v * __ldg(args.row_scale + c.n0 + j0 + jb + j) * cscale;
               if (kEpi == kEpiStore && args.c_rows) {   // the row's own destination
                 args.c_rows[c.n0 + j0 + jb + j][f] = v;
                 continue;
@@ -573,12 +632,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   const uint32_t tmem_base = s->tmem_base;
   const int n_tiles_n = (N + BN - 1) / BN;
   const int total = s->start[E] * n_tiles_n;
-  const int nk = (Kd + BK - 1) / BK;
+  constexpr int kRing = ring_stages<kBK>();
+  constexpr uint32_t kRingBytes = ring_stage_bytes<kBK>();
+  constexpr int kKb = kblock_width<kBK>();
+  constexpr int kChunk = chunk_kblocks<kBK>();
+  const int nk = (Kd + kKb - 1) / kKb;
 
   if (wg == 1 || wg == 2) {
     // the epilogue warpgroups hold 128 FP32 running sums per thread
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
-    epilogue_role<kMode, kEpi>(s, args, tmem_base, warp, lane, n_tiles_n, total, nk, rank, n_pairs);
+    epilogue_role<kMode, kEpi, kBK>(s, args, tmem_base, warp, lane, n_tiles_n, total, nk, rank, n_pairs);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
     if (warp == 0) {
@@ -590,10 +653,23 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           const TileCoord c = decode_tile<kMode>(s, args, n_tiles_n, nk, tile, rank);
           const int nb = c.n0 + (int)rank * BNH;   // kModeTN: this CTA's B columns
           for (int kb = 0; kb < c.nk; ++kb, ++it) {
-            const uint32_t st = it % kStages, use = it / kStages;
+            const uint32_t st = it % kRing, use = it / kRing;
             if (!mbar_wait(s, &s->empty[st], (use & 1) ^ 1, args.err)) { ok = false; break; }
-            uint8_t* base = tiles + st * kStageBytes;
-            mbar_arrive_expect_tx(&s->full[st], kBK == kBHalf ? kTileABytes + kTileBHalfBytes : kTxBytes);
+            uint8_t* base = tiles + st * kRingBytes;
+            if (f16_path<kBK>()) {
+              // the weights' hi and mid tiles (expert e and E + e of the split
+              // tensor) and this CTA's rows (kBF16S: their hi and mid planes,
+              // rows r and R + r), 64 k wide, 128-byte swizzle
+              const int row = c.n0 + (int)rank * (c.n_mma / 2);
+              mbar_arrive_expect_tx(&s->full[st], kRingBytes);
+              tma_load_3d(&mapA, &s->full[st], base, kb * BK16, c.m0, c.e);
+              tma_load_3d(&mapA, &s->full[st], base + kTile16Bytes, kb * BK16, c.m0, E + c.e);
+              tma_load_2d(&mapB, &s->full[st], base + 2 * kTile16Bytes, kb * BK16, row);
+              if (kBK == kBF16S)
+                tma_load_2d(&mapB, &s->full[st], base + 3 * kTile16Bytes, kb * BK16, (int)args.rows + row);
+              continue;
+            }
+            mbar_arrive_expect_tx(&s->full[st], kTxBytes);
             if (kMode == kModeTN) {
               // both operands MN-major: 32-column boxes of 16 segment rows
               const int row = c.k_row0 + kb * BK;
@@ -612,17 +688,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                 for (int j = 0; j < BM / 32; ++j)
                   tma_load_3d(&mapA, &s->full[st], base + j * (32 * BK * 4), c.m0 + 32 * j, kb * BK, c.e);
               }
-              // B: this CTA's half of the tile's dispatch rows (n_mma / 2 of them);
-              // FP16 rows land in B's lo slot, for the splitters to unpack
-              tma_load_2d(&mapB, &s->full[st], base + (kBK == kBHalf ? kTxBytes + kTileABytes : kTileABytes),
-                          kb * BK, c.n0 + (int)rank * (c.n_mma / 2));
+              // B: this CTA's half of the tile's dispatch rows (n_mma / 2 of them)
+              tma_load_2d(&mapB, &s->full[st], base + kTileABytes, kb * BK, c.n0 + (int)rank * (c.n_mma / 2));
             }
           }
         }
         // the last issued loads must land before the CTA may exit
-        const uint32_t n_last = it < (uint32_t)kStages ? it : (uint32_t)kStages;
+        const uint32_t n_last = it < (uint32_t)kRing ? it : (uint32_t)kRing;
         for (uint32_t j = 0; j < n_last; ++j) {
-          const uint32_t i2 = it - 1 - j, st = i2 % kStages, use = i2 / kStages;
+          const uint32_t i2 = it - 1 - j, st = i2 % kRing, use = i2 / kRing;
           const long long t0 = clock64();
           while (!mbar_try_wait(&s->full[st], use & 1) && clock64() - t0 < kWaitLimitCycles) {
           }
@@ -640,17 +714,35 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         for (int tile = blockIdx.x / 2; tile < total && ok; tile += n_pairs) {
           const TileCoord tc = decode_tile<kMode>(s, args, n_tiles_n, nk, tile, rank);
           const int tnk = tc.nk;
-          const uint32_t idesc = instr_desc(kAMN, kBMN, (uint32_t)tc.n_mma);
-          for (int c0 = 0; c0 < tnk && ok; c0 += kChunkKb, ++ch) {
+          const uint32_t idesc = f16_path<kBK>() ? instr_desc_f16((uint32_t)tc.n_mma)
+                                                 : instr_desc(kAMN, kBMN, (uint32_t)tc.n_mma);
+          for (int c0 = 0; c0 < tnk && ok; c0 += kChunk, ++ch) {
             const uint32_t p = ch & 1, cuse = ch >> 1;
             if (!mbar_wait(s, &s->chunk_empty[p], (cuse & 1) ^ 1, args.err)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + p * BN;
-            const int c1 = min(c0 + kChunkKb, tnk);
+            const int c1 = min(c0 + kChunk, tnk);
             for (int kb = c0; kb < c1; ++kb, ++it) {
-              const uint32_t st = it % kStages, use = it / kStages;
+              const uint32_t st = it % kRing, use = it / kRing;
               if (!mbar_wait(s, &s->split[st], use & 1, args.err)) { ok = false; break; }
               tc_fence_after();
+              if (f16_path<kBK>()) {
+                // K-major FP16 tiles, 128-byte swizzle: 8-row groups 1024 B
+                // apart (SBO), a 16-wide k-step = +32 B inside the swizzle row
+                const uint32_t a16 = smem_u32(tiles + st * kRingBytes);
+                const uint32_t m16 = a16 + kTile16Bytes, b16 = a16 + 2 * kTile16Bytes, bm16 = a16 + 3 * kTile16Bytes;
+#pragma unroll
+                for (int kk = 0; kk < BK16 / 16; ++kk) {
+                  const uint64_t ad = smem_desc(a16 + kk * 32, 16, 1024, kSwizzle128B);
+                  const uint64_t bd = smem_desc(b16 + kk * 32, 16, 1024, kSwizzle128B);
+                  tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb > c0 || kk > 0) ? 1u : 0u);
+                  if (kBK == kBF16S)
+                    tc_mma_f16_pair(d_tmem, ad, smem_desc(bm16 + kk * 32, 16, 1024, kSwizzle128B), idesc, 1u);
+                  tc_mma_f16_pair(d_tmem, smem_desc(m16 + kk * 32, 16, 1024, kSwizzle128B), bd, idesc, 1u);
+                }
+                tc_commit_pair(&s->empty[st]);
+                continue;
+              }
               const uint32_t a_hi = smem_u32(tiles + st * kStageBytes);
               const uint32_t b_hi = a_hi + kTileABytes;
               const uint32_t a_lo = a_hi + kTxBytes, b_lo = b_hi + kTxBytes;
@@ -701,29 +793,29 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       const int ci = warp < 4 ? warp - 2 : warp - 10;
       // kBExact: only A (the weights) is split; B's rows are exact in TF32 and
       // are only checked (low 13 bits zero), a violation recorded as a fault.
-      // kBHalf: only A is split; B's FP16 rows are unpacked into the B tile.
       constexpr int kVec = (int)((kBK != kBSplit ? kTileABytes : kTxBytes) / 16);
       constexpr int kBatch = 8;
       static_assert(kVec % (32 * kBatch) == 0, "split batches divide the stage");
       uint32_t it = 0;
       bool ok = true;
-      int scaled_tile = -1;    // kBHalf: the tile whose row scales this warp holds
-      for (int tile = blockIdx.x / 2; tile < total && ok; tile += n_pairs) {
+      if (f16_path<kBK>()) {
+        // nothing to split: warp ci relays stage ci's landing (its own CTA's
+        // TMA) to the leader's MMA issuer, one fixed warp per stage
+        for (int tile = blockIdx.x / 2; tile < total && ok && ci < kRing; tile += n_pairs) {
+          const TileCoord c = decode_tile<kMode>(s, args, n_tiles_n, nk, tile, rank);
+          for (int kb = 0; kb < c.nk; ++kb, ++it) {
+            if ((int)(it % kRing) != ci) continue;
+            const uint32_t st = it % kRing, use = it / kRing;
+            if (!mbar_wait(s, &s->full[st], use & 1, args.err)) { ok = false; break; }
+            __syncwarp();
+            if (lane == 0) mbar_arrive_leader(&s->split[st], rank);
+          }
+        }
+      }
+      for (int tile = blockIdx.x / 2; !f16_path<kBK>() && tile < total && ok; tile += n_pairs) {
         const TileCoord c = decode_tile<kMode>(s, args, n_tiles_n, nk, tile, rank);
         for (int kb = 0; kb < c.nk; ++kb, ++it) {
           if ((int)(it % kNumSplitWarps) != ci) continue;
-          if (kBK == kBHalf && scaled_tile != tile) {
-            // this CTA's B rows of the tile: row0 .. row0 + 127 (past the
-            // payload: scale 0, the TMA fill is 0 too)
-            const int64_t row0 = (int64_t)c.n0 + (int64_t)rank * (c.n_mma / 2);
-#pragma unroll
-            for (int i = lane; i < BNH; i += 32) {
-              const int64_t p = row0 + i;
-              s->rscale[ci][i] = p < args.rows ? __ldg(args.row_scale + p) : 0.f;
-            }
-            __syncwarp();
-            scaled_tile = tile;
-          }
           // kModeTN: rows past the expert's segment belong to the next expert
           const int k_valid = kMode == kModeTN ? c.k_rows - kb * BK : BK;
           const uint32_t st = it % kStages, use = it / kStages;
@@ -751,23 +843,6 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                   __float_as_uint(__uint_as_float(x[j].y) - __uint_as_float(x[j].y & kTf32Mask)),
                   __float_as_uint(__uint_as_float(x[j].z) - __uint_as_float(x[j].z & kTf32Mask)),
                   __float_as_uint(__uint_as_float(x[j].w) - __uint_as_float(x[j].w & kTf32Mask)));
-          }
-          if (kBK == kBHalf) {
-            // FP16 tile [128 rows][16] (32 bytes a row, no swizzle) -> FP32 B
-            // tile in the 64-byte swizzle TMA would have written: 16-byte chunk
-            // c of row r sits at chunk c ^ ((r >> 1) & 3) of the row
-            const uint2* hs = reinterpret_cast<const uint2*>(tiles + st * kStageBytes + kTxBytes + kTileABytes);
-            float4* rbw = reinterpret_cast<float4*>(tiles + st * kStageBytes + kTileABytes);
-            const float* rs = s->rscale[ci];
-#pragma unroll 4
-            for (int i = lane; i < BNH * 4; i += 32) {
-              const int r = i >> 2, cc = i & 3;
-              const uint2 h = hs[i];
-              const float sc = rs[r];
-              const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
-              const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
-              rbw[r * 4 + (cc ^ ((r >> 1) & 3))] = make_float4(f0.x * sc, f0.y * sc, f1.x * sc, f1.y * sc);
-            }
           }
           if (kBK == kBExact) {
             // only the tile's own rows (a K-major row is 4 consecutive 16-byte
@@ -830,20 +905,6 @@ bool map_a(CUtensorMap* m, const float* A, int64_t R, int Kd) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// A of the FP16-row forward: the payload [R, Kd] FP16, box 16 (k) x 128 (rows),
-// no swizzle (32-byte rows; the splitters unpack them)
-bool map_a_half(CUtensorMap* m, const uint16_t* A, int64_t R, int Kd) {
-  auto enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)Kd, (cuuint64_t)R};
-  cuuint64_t strides[1] = {(cuuint64_t)Kd * 2};
-  cuuint32_t box[2] = {BK, BM};
-  cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void*)A, dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // B for "x W": W [E, Kd, N] (N contiguous), box 32 (n) x 16 (k) x 1, 128-byte
 //   swizzle with 32-byte atoms (MN-major); 4 boxes per CTA and k-block
 // B for "x W^T": W [E, N, Kd] (Kd contiguous), box 16 (k) x 128 (n) x 1, 64-byte swizzle
@@ -865,6 +926,32 @@ bool map_b(CUtensorMap* m, const float* W, int E, int Kd, int N, bool nt) {
              CU_TENSOR_MAP_INTERLEAVE_NONE,
              nt ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// kBF16W operands, both K-major FP16 with the 128-byte swizzle and a 64-wide
+// (128-byte) k-box: the split weights [2E][N][Kd] (box 64 x 128 x 1) and the
+// payload rows [R][Kd] (box 64 x 128).  Kd % 8 == 0 (16-byte strides).
+bool map_w16(CUtensorMap* m, const uint16_t* W16, int E, int Kd, int N) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)Kd, (cuuint64_t)N, (cuuint64_t)(2 * E)};
+  cuuint64_t strides[2] = {(cuuint64_t)Kd * 2, (cuuint64_t)Kd * N * 2};
+  cuuint32_t box[3] = {BK16, BM, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, (void*)W16, dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool map_rows16(CUtensorMap* m, const uint16_t* A, int64_t R, int Kd) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)Kd, (cuuint64_t)R};
+  cuuint64_t strides[1] = {(cuuint64_t)Kd * 2};
+  cuuint32_t box[2] = {BK16, BM};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void*)A, dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // kModeTN operands: X [R, M] and Y [R, N] row-major, read as MN-major 32-column
@@ -890,7 +977,7 @@ template <int kMode, int kEpi, int kBK = kBSplit>
 janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, int N, float* C, float* C2,
                     const float* aux, const int32_t* offsets, int32_t* err, cudaStream_t stream, int M = 0,
                     const float* aux2 = nullptr, float* C3 = nullptr, float* const* c_rows = nullptr,
-                    const float* row_scale = nullptr) {
+                    const float* row_scale = nullptr, const float* col_scale = nullptr) {
   static_assert(kBK == kBSplit || kMode == kModeNN, "exact or FP16 rows: the forward layout only");
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
@@ -900,16 +987,22 @@ janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, in
   });
   if (attr != cudaSuccess) return JANUS_ERR_CUDA;
   CUtensorMap ma, mb;
-  if (kMode == kModeTN) {
+  if (f16_path<kBK>()) {
+    // W: the split weights [2E][N][Kd] FP16 (hi for expert e, mid for E + e);
+    // A: the payload [R][Kd] (kBF16W) or the rows' hi and mid planes [2R][Kd] (kBF16S)
+    if (!map_w16(&ma, reinterpret_cast<const uint16_t*>(W), E, Kd, N) ||
+        !map_rows16(&mb, reinterpret_cast<const uint16_t*>(A), kBK == kBF16S ? 2 * R : R, Kd))
+      return JANUS_ERR_CUDA;
+  } else if (kMode == kModeTN) {
     if (!map_rows_mn(&ma, A, R, M) || !map_rows_mn(&mb, W, R, N)) return JANUS_ERR_CUDA;
   } else if (!map_b(&ma, W, E, Kd, N, kMode == kModeNT) ||
-             !(kBK == kBHalf ? map_a_half(&mb, reinterpret_cast<const uint16_t*>(A), R, Kd) : map_a(&mb, A, R, Kd))) {
+             !map_a(&mb, A, R, Kd)) {
     // operands swapped: the weights are the MMA's A, the dispatch rows its B
     return JANUS_ERR_CUDA;
   }
   Args a;
   a.C = C; a.C2 = C2; a.C3 = C3; a.aux = aux; a.aux2 = aux2; a.c_rows = c_rows;
-  a.row_scale = row_scale; a.rows = R;
+  a.row_scale = row_scale; a.col_scale = col_scale; a.rows = R;
   a.offsets = offsets; a.E = E; a.Kd = Kd; a.N = N; a.M = M; a.err = err;
   // one CTA per SM, in clusters of two (the MMA pairs)
   cudaLaunchConfig_t cfg = {};
@@ -929,7 +1022,132 @@ janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, in
   return launch_status();
 }
 
+// ---- the FP16 split of the weights for the kind::f16 GEMMs ------------------
+// x W (W [E][Kd][N]) or x W^T (W [E][N][Kd]) FP32 -> w16 = [hi | mid], each
+// [E][N][Kd] FP16 (K-major for the kind::f16 MMA: x W's weights are
+// transposed on the way), and winv [E][N] = 1 / S per output feature.
+// S = 2^(141 - b), b = the biased exponent of the column's largest magnitude,
+// so that magnitude times S lies in [2^14, 2^15) (below FP16's 65504); S is
+// clamped to [2^-126, 2^126] and is 1 for an all-zero column.  hi = fp16(w S)
+// and mid = fp16(w S - hi): w S - hi is exact in FP32 and the pair carries
+// 22 bits of w S.  Three passes: column maxima (as bits, into winv), the split
+// with the transpose through shared memory, maxima -> 1 / S.
+
+__device__ __forceinline__ int w16_scale_exp(uint32_t max_bits) {
+  if (max_bits == 0) return 0;
+  const int b = max((int)(max_bits >> 23), 1);
+  return min(max(141 - b, -126), 126);
+}
+
+__global__ void __launch_bounds__(256) w16_colmax_kernel(const float* __restrict__ w, int Kd, int N, int k_per,
+                                                         uint32_t* __restrict__ colmax) {
+  const int e = blockIdx.z, f = blockIdx.x * 256 + threadIdx.x, k0 = blockIdx.y * k_per;
+  if (f >= N) return;
+  const float* p = w + (int64_t)e * Kd * N + f;
+  const int k1 = min(k0 + k_per, Kd);
+  uint32_t m = 0;
+  for (int k = k0; k < k1; ++k) m = max(m, __float_as_uint(__ldcs(p + (int64_t)k * N)) & 0x7fffffffu);
+  if (m) atomicMax(colmax + (int64_t)e * N + f, m);
+}
+
+// tile: 32 features x 64 k of expert e; reads are 128-byte rows of W[e]
+// ([Kd][N], features contiguous), writes 128-byte rows of the K-major split
+// (two consecutive k per lane)
+__global__ void __launch_bounds__(256) w16_split_kernel(const float* __restrict__ w, int E, int Kd, int N,
+                                                        const uint32_t* __restrict__ colmax, __half* __restrict__ w16) {
+  __shared__ __half t_hi[32][66], t_mid[32][66];     // [feature][k] of a 32 x 64 tile
+  const int e = blockIdx.z, f0 = blockIdx.x * 32, k0 = blockIdx.y * 64;
+  const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;
+  const int f = f0 + tx;
+  const float S = f < N ? __uint_as_float((uint32_t)(127 + w16_scale_exp(colmax[(int64_t)e * N + f])) << 23) : 1.0f;
+#pragma unroll
+  for (int j = ty; j < 64; j += 8) {
+    const int k = k0 + j;
+    const float v = (f < N && k < Kd) ? __ldcs(w + ((int64_t)e * Kd + k) * N + f) * S : 0.0f;
+    const __half hi = __float2half_rn(v);
+    t_hi[tx][j] = hi;
+    t_mid[tx][j] = __float2half_rn(v - __half2float(hi));
+  }
+  __syncthreads();
+  const int64_t plane = (int64_t)E * N * Kd;        // mid follows hi
+#pragma unroll
+  for (int j = ty; j < 32; j += 8) {
+    const int fo = f0 + j, ko = k0 + 2 * tx;
+    if (fo >= N) continue;
+    const int64_t o = ((int64_t)e * N + fo) * Kd + ko;
+    if (ko + 1 < Kd && (o % 2) == 0) {
+      *reinterpret_cast<__half2*>(w16 + o) = __halves2half2(t_hi[j][2 * tx], t_hi[j][2 * tx + 1]);
+      *reinterpret_cast<__half2*>(w16 + plane + o) = __halves2half2(t_mid[j][2 * tx], t_mid[j][2 * tx + 1]);
+    } else {
+      for (int q = 0; q < 2; ++q)
+        if (ko + q < Kd) {
+          w16[o + q] = t_hi[j][2 * tx + q];
+          w16[plane + o + q] = t_mid[j][2 * tx + q];
+        }
+    }
+  }
+}
+
+// x W^T: output feature n is row n of W[e] ([N][Kd], K contiguous): one warp
+// per row for its maximum, then an elementwise split in place (no transpose).
+__global__ void __launch_bounds__(256) w16_rowmax_kernel(const float* __restrict__ w, int64_t rows, int Kd,
+                                                         uint32_t* __restrict__ rowmax) {
+  const int lane = threadIdx.x % 32;
+  for (int64_t r = ((int64_t)blockIdx.x * 256 + threadIdx.x) / 32; r < rows; r += (int64_t)gridDim.x * 8) {
+    const float* p = w + r * Kd;
+    uint32_t m = 0;
+    for (int k = lane; k < Kd; k += 32) m = max(m, __float_as_uint(__ldcs(p + k)) & 0x7fffffffu);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) rowmax[r] = m;
+  }
+}
+
+__global__ void __launch_bounds__(256) w16_split_rows_kernel(const float* __restrict__ w, int64_t rows, int Kd,
+                                                             const uint32_t* __restrict__ rowmax,
+                                                             __half* __restrict__ w16) {
+  const int64_t n = rows * Kd;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const float S = __uint_as_float((uint32_t)(127 + w16_scale_exp(rowmax[r])) << 23);
+    for (int k = threadIdx.x; k < Kd; k += 256) {
+      const int64_t i = r * Kd + k;
+      const float v = __ldcs(w + i) * S;
+      const __half hi = __float2half_rn(v);
+      w16[i] = hi;
+      w16[n + i] = __float2half_rn(v - __half2float(hi));
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) w16_inv_scale_kernel(uint32_t* __restrict__ colmax_to_inv, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (int64_t)gridDim.x * 256)
+    colmax_to_inv[i] = (uint32_t)(127 - w16_scale_exp(colmax_to_inv[i])) << 23;
+}
+
 }  // namespace
+
+janus_status split_weights_f16(const float* w, int32_t E, int32_t Kd, int32_t N, bool transposed, uint16_t* w16,
+                               float* winv, cudaStream_t stream) {
+  uint32_t* colmax = reinterpret_cast<uint32_t*>(winv);
+  const int64_t n = (int64_t)E * N;
+  if (!transposed) {
+    // x W^T: W [E][N][Kd] is already K-major
+    const int64_t blocks = std::min<int64_t>((n + 7) / 8, (int64_t)num_sms() * 8);
+    w16_rowmax_kernel<<<(unsigned)blocks, 256, 0, stream>>>(w, n, Kd, colmax);
+    const int64_t eb = std::min<int64_t>(n, (int64_t)num_sms() * 16);
+    w16_split_rows_kernel<<<(unsigned)eb, 256, 0, stream>>>(w, n, Kd, colmax, reinterpret_cast<__half*>(w16));
+    w16_inv_scale_kernel<<<(unsigned)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, stream>>>(colmax, n);
+    return launch_status();
+  }
+  JANUS_CUDA_TRY(cudaMemsetAsync(colmax, 0, sizeof(uint32_t) * (size_t)E * N, stream));
+  const int k_per = 64;
+  w16_colmax_kernel<<<dim3((N + 255) / 256, (Kd + k_per - 1) / k_per, E), 256, 0, stream>>>(w, Kd, N, k_per,
+                                                                                            colmax);
+  w16_split_kernel<<<dim3((N + 31) / 32, (Kd + 63) / 64, E), 256, 0, stream>>>(w, E, Kd, N, colmax,
+                                                                             reinterpret_cast<__half*>(w16));
+  w16_inv_scale_kernel<<<(unsigned)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, stream>>>(colmax, n);
+  return launch_status();
+}
 
 size_t workspace_extra() { return 0; }
 
@@ -944,16 +1162,67 @@ janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, 
                                     nullptr, yd_rows);
 }
 
+namespace {
+// The forward's second GEMM, yd = H W2: on 3xTF32, or (second given) on the
+// kind::f16 path with H split into two FP16 terms per row first.
+janus_status second_gemm(const float* H, const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
+                         const float* w2, float* yd, float* const* yd_rows, int32_t* err, cudaStream_t stream,
+                         const F16Second* second) {
+  if (!second)
+    return launch<kModeNN, kEpiStore>(H, w2, R, E, h, d, yd, nullptr, nullptr, offsets, err, stream, 0, nullptr,
+                                      nullptr, yd_rows);
+  janus_status st = rows_split_f16(H, R, h, second->h16, second->hscale, second->rowmax, stream);
+  if (st != JANUS_OK) return st;
+  st = split_weights_f16(w2, E, h, d, true, second->w16, second->winv, stream);
+  if (st != JANUS_OK) return st;
+  return launch<kModeNN, kEpiStore, kBF16S>(reinterpret_cast<const float*>(second->h16),
+                                            reinterpret_cast<const float*>(second->w16), R, E, h, d, yd, nullptr,
+                                            nullptr, offsets, err, stream, 0, nullptr, nullptr, yd_rows,
+                                            second->hscale, second->winv);
+}
+}  // namespace
+
 janus_status expert_ffn_fwd_packed(const uint16_t* payload, const float* row_scale, const int32_t* offsets,
                                    int32_t E, int64_t R, int32_t d, int32_t h, const float* w1, const float* w2,
-                                   float* yd, float* act, float* H, int32_t* err, cudaStream_t stream,
-                                   float* const* yd_rows) {
-  janus_status st = launch<kModeNN, kEpiSilu, kBHalf>(reinterpret_cast<const float*>(payload), w1, R, E, d, h, H,
-                                                      act, nullptr, offsets, err, stream, 0, nullptr, nullptr,
-                                                      nullptr, row_scale);
+                                   float* yd, float* act, float* H, uint16_t* w16, float* winv, int32_t* err,
+                                   cudaStream_t stream, float* const* yd_rows, const F16Second* second) {
+  // the FP16 split of W1 (transposed to [E][h][d], K-major), then the
+  // kind::f16 first GEMM on the payload, then the second GEMM
+  janus_status st = split_weights_f16(w1, E, d, h, true, w16, winv, stream);
   if (st != JANUS_OK) return st;
-  return launch<kModeNN, kEpiStore>(H, w2, R, E, h, d, yd, nullptr, nullptr, offsets, err, stream, 0, nullptr,
-                                    nullptr, yd_rows);
+  st = launch<kModeNN, kEpiSilu, kBF16W>(reinterpret_cast<const float*>(payload), reinterpret_cast<const float*>(w16),
+                                          R, E, d, h, H, act, nullptr, offsets, err, stream, 0, nullptr, nullptr,
+                                          nullptr, row_scale, winv);
+  if (st != JANUS_OK) return st;
+  return second_gemm(H, offsets, E, R, d, h, w2, yd, yd_rows, err, stream, second);
+}
+
+janus_status expert_ffn_fwd_split(const uint16_t* rows16, const float* row_scale, const int32_t* offsets, int32_t E,
+                                  int64_t R, int32_t d, int32_t h, const float* w1, const float* w2, float* yd,
+                                  float* act, float* H, uint16_t* w16, float* winv, int32_t* err,
+                                  cudaStream_t stream, float* const* yd_rows, const F16Second* second) {
+  janus_status st = split_weights_f16(w1, E, d, h, true, w16, winv, stream);
+  if (st != JANUS_OK) return st;
+  st = launch<kModeNN, kEpiSilu, kBF16S>(reinterpret_cast<const float*>(rows16), reinterpret_cast<const float*>(w16),
+                                          R, E, d, h, H, act, nullptr, offsets, err, stream, 0, nullptr, nullptr,
+                                          nullptr, row_scale, winv);
+  if (st != JANUS_OK) return st;
+  return second_gemm(H, offsets, E, R, d, h, w2, yd, yd_rows, err, stream, second);
+}
+
+janus_status expert_ffn_vjp_split(const uint16_t* gd16, const float* gd_scale, const float* act,
+                                  const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
+                                  const float* w1, const float* w2, float* dxd, float* dA, uint16_t* w16,
+                                  float* winv, int32_t* err, cudaStream_t stream, float* const* dxd_rows) {
+  // dA = (gd W2^T) * silu'(a): W2 [E][h][d] is K-major for this product as it stands
+  janus_status st = split_weights_f16(w2, E, d, h, false, w16, winv, stream);
+  if (st != JANUS_OK) return st;
+  st = launch<kModeNN, kEpiDSilu, kBF16S>(reinterpret_cast<const float*>(gd16), reinterpret_cast<const float*>(w16),
+                                           R, E, d, h, dA, nullptr, act, offsets, err, stream, 0, nullptr, nullptr,
+                                           nullptr, gd_scale, winv);
+  if (st != JANUS_OK) return st;
+  return launch<kModeNT, kEpiStore>(dA, w1, R, E, h, d, dxd, nullptr, nullptr, offsets, err, stream, 0, nullptr,
+                                    nullptr, dxd_rows);
 }
 
 janus_status expert_ffn_vjp(const float* xd, const float* gd, const float* act_in, float* A,

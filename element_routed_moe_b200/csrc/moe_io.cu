@@ -135,6 +135,129 @@ combine_kernel(const float4* __restrict__ yd, const int32_t* __restrict__ slot_o
   }
 }
 
+// ---- dispatch into two FP16 terms per value (the FP16 tensor-core GEMMs) ----
+//
+// Each dispatch row p (slot s = i K + k) is written as hi and mid binary16
+// planes with one power-of-two scale S_p per row:  v = (w_k) x[i, :] (the
+// same FP32 value janus_dispatch writes), hi = fp16(v S_p), mid =
+// fp16(v S_p - hi), row_scale[p] = 1 / S_p.  S_p puts the row's largest |v|,
+// |w_k| max_j |x[i, j]| (rounding is monotonic), in [2^14, 2^15); a value
+// within 2^18 of that maximum keeps 22 significant bits, smaller ones an
+// absolute error below 2^-40 of it.  The row maxima come from a first pass.
+
+// rowmax[i] = max_j |x[i, j]| as ordered bits (atomicMax per chunk item)
+__global__ void __launch_bounds__(kThreads)
+row_absmax_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, uint32_t* __restrict__ rowmax) {
+  const int lane = threadIdx.x % 32;
+  const ChunkWalk cw = chunk_walk(d4);
+  const int c0 = cw.c0;
+  for (int64_t i = cw.row0; i < n_atoms; i += cw.stride) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int c = c0 + u * 32 + lane;
+      if (c < d4) {
+        const float4 v = __ldg(x + i * d4 + c);
+        m = max(m, max(max(abs_bits(v.x), abs_bits(v.y)), max(abs_bits(v.z), abs_bits(v.w))));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0 && m) atomicMax(rowmax + i, m);
+  }
+}
+
+// exponent e of S = 2^e for a row maximum m (bits): m 2^e in [2^14, 2^15),
+// clamped to [-126, 126]; 0 for a zero row
+__device__ __forceinline__ int split_exp(uint32_t m) {
+  if (m == 0) return 0;
+  const int b = max((int)(m >> 23), 1);
+  return min(max(141 - b, -126), 126);
+}
+
+__device__ __forceinline__ uint2 halves(float a, float b, float c, float d) {
+  const __half2 lo = __floats2half2_rn(a, b), hi = __floats2half2_rn(c, d);
+  return make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+}
+
+template <bool kWeighted>
+__global__ void __launch_bounds__(kThreads)
+dispatch_split_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K, const int32_t* __restrict__ slot_of,
+                      const float* __restrict__ w, const uint32_t* __restrict__ rowmax, uint2* __restrict__ rows16,
+                      float* __restrict__ row_scale, int32_t* dbg) {
+  const int64_t R = n_atoms * K;
+  const int lane = threadIdx.x % 32;
+  uint2* mid_plane = rows16 + R * d4;
+  const ChunkWalk cw = chunk_walk(d4);
+  const int c0 = cw.c0;
+  for (int64_t i = cw.row0; i < n_atoms; i += cw.stride) {
+    const int my_slot = lane < K ? slot_of[i * K + lane] : 0;
+    const float my_w = (kWeighted && lane < K) ? w[i * K + lane] : 1.0f;
+    const float m = __uint_as_float(rowmax[i]);
+    float4 v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int c = c0 + u * 32 + lane;
+      if (c < d4) v[u] = __ldcs(x + i * d4 + c);
+    }
+    for (int k = 0; k < K; ++k) {
+      int64_t p;
+      float wk;
+      slot_k<kWeighted>(k, K, i, my_slot, my_w, slot_of, w, &p, &wk);
+      if (kDebug && !in_range(p, R)) {   // p is the same in every lane
+        if (lane == 0) debug_fault(dbg);
+        continue;
+      }
+      const int e = split_exp(__float_as_uint(kWeighted ? fabsf(wk) * m : m));
+      const float S = __uint_as_float((uint32_t)(127 + e) << 23);
+      if (c0 == 0 && lane == 0) row_scale[p] = __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < d4) {
+          float4 o = v[u];
+          if (kWeighted) { o.x *= wk; o.y *= wk; o.z *= wk; o.w *= wk; }
+          o.x *= S; o.y *= S; o.z *= S; o.w *= S;
+          const uint2 hq = halves(o.x, o.y, o.z, o.w);
+          const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hq.x));
+          const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hq.y));
+          rows16[p * d4 + c] = hq;
+          mid_plane[p * d4 + c] = halves(o.x - h0.x, o.y - h0.y, o.z - h1.x, o.w - h1.y);
+        }
+      }
+    }
+  }
+}
+
+// Rows in place (row i -> row i): the same two-term split for a buffer a
+// kernel of this library has just written (the expert MLP's H = silu(a)).
+__global__ void __launch_bounds__(kThreads)
+rows_split_kernel(const float4* __restrict__ x, int64_t rows, int d4, const uint32_t* __restrict__ rowmax,
+                  uint2* __restrict__ rows16, float* __restrict__ row_scale) {
+  const int lane = threadIdx.x % 32;
+  uint2* mid_plane = rows16 + rows * d4;
+  const ChunkWalk cw = chunk_walk(d4);
+  const int c0 = cw.c0;
+  for (int64_t i = cw.row0; i < rows; i += cw.stride) {
+    const int e = split_exp(rowmax[i]);
+    const float S = __uint_as_float((uint32_t)(127 + e) << 23);
+    if (c0 == 0 && lane == 0) row_scale[i] = __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int c = c0 + u * 32 + lane;
+      if (c < d4) {
+        float4 o = __ldcs(x + i * d4 + c);
+        o.x *= S; o.y *= S; o.z *= S; o.w *= S;
+        const uint2 hq = halves(o.x, o.y, o.z, o.w);
+        const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hq.x));
+        const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hq.y));
+        rows16[i * d4 + c] = hq;
+        mid_plane[i * d4 + c] = halves(o.x - h0.x, o.y - h0.y, o.z - h1.x, o.w - h1.y);
+      }
+    }
+  }
+}
+
 // ---- atom-type-aware FP16 packing ------------------------------------------
 
 __global__ void __launch_bounds__(kThreads)
@@ -296,6 +419,55 @@ extern "C" janus_status janus_combine(const float* yd, const int32_t* slot_of,
   else
     combine_kernel<false><<<grid, kThreads, 0, (cudaStream_t)stream>>>(
         (const float4*)yd, slot_of, nullptr, n_atoms, top_k, d / 4, (float4*)y, debug_fault_word());
+  return launch_status();
+}
+
+namespace janus {
+janus_status rows_split_f16(const float* x, int64_t rows, int32_t d, uint16_t* rows16, float* row_scale,
+                            uint32_t* rowmax, cudaStream_t stream) {
+  if (rows == 0) return JANUS_OK;
+  JANUS_CUDA_TRY(cudaMemsetAsync(rowmax, 0, sizeof(uint32_t) * (size_t)rows, stream));
+  const unsigned grid = rows_grid(row_items(rows, d / 4), 8);
+  row_absmax_kernel<<<grid, kThreads, 0, stream>>>((const float4*)x, rows, d / 4, rowmax);
+  rows_split_kernel<<<grid, kThreads, 0, stream>>>((const float4*)x, rows, d / 4, rowmax, (uint2*)rows16, row_scale);
+  return launch_status();
+}
+}  // namespace janus
+
+extern "C" janus_status janus_dispatch_split_workspace_size(int64_t n_atoms, size_t* bytes) {
+  JANUS_CHECK_ARG(bytes && n_atoms >= 0);
+  *bytes = sizeof(WsHeader) + align_up(sizeof(uint32_t) * (size_t)(n_atoms > 0 ? n_atoms : 1), 256);
+  return JANUS_OK;
+}
+
+extern "C" janus_status janus_dispatch_split(const float* x, int64_t n_atoms, int32_t d, int32_t top_k,
+                                             const int32_t* slot_of, const float* topk_weight, uint16_t* rows16,
+                                             float* row_scale, void* workspace, size_t workspace_bytes,
+                                             janus_stream_t stream_) {
+  cudaStream_t stream = (cudaStream_t)stream_;
+  janus_status st = check_rows(n_atoms, d, top_k);
+  if (st != JANUS_OK) return st;
+  size_t need = 0;
+  st = janus_dispatch_split_workspace_size(n_atoms, &need);
+  if (st != JANUS_OK) return st;
+  JANUS_CHECK_ARG(workspace && workspace_bytes >= need);
+  JANUS_CHECK_ALIGN(aligned(workspace, 256));
+  if (n_atoms == 0) return JANUS_OK;
+  JANUS_CHECK_ARG(x && slot_of && rows16 && row_scale);
+  JANUS_CHECK_ALIGN(aligned(x, 16) && aligned(rows16, 16));
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  uint32_t* rowmax = (uint32_t*)((char*)workspace + sizeof(WsHeader));
+  JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, need, stream));
+  const unsigned grid = rows_grid(row_items(n_atoms, d / 4), 8);
+  row_absmax_kernel<<<grid, kThreads, 0, stream>>>((const float4*)x, n_atoms, d / 4, rowmax);
+  if (topk_weight)
+    dispatch_split_kernel<true><<<grid, kThreads, 0, stream>>>((const float4*)x, n_atoms, d / 4, top_k, slot_of,
+                                                               topk_weight, rowmax, (uint2*)rows16, row_scale,
+                                                               debug_fault_word());
+  else
+    dispatch_split_kernel<false><<<grid, kThreads, 0, stream>>>((const float4*)x, n_atoms, d / 4, top_k, slot_of,
+                                                                nullptr, rowmax, (uint2*)rows16, row_scale,
+                                                                debug_fault_word());
   return launch_status();
 }
 

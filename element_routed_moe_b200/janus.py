@@ -33,12 +33,13 @@ SYMBOLS = (
     "janus_status_string", "janus_version", "janus_check",
     "janus_route_workspace_size", "janus_route",
     "janus_route_layers_workspace_size", "janus_route_layers", "janus_active_experts",
-    "janus_dispatch",
+    "janus_dispatch", "janus_dispatch_split_workspace_size", "janus_dispatch_split",
     "janus_quant_by_type_workspace_size", "janus_quant_by_type", "janus_quant_by_type_noalloc",
     "janus_dequant_by_type", "janus_dispatch_row_scales",
     "janus_expert_ffn_workspace_size", "janus_expert_ffn_fwd", "janus_expert_ffn_vjp",
     "janus_expert_ffn_fwd_rows", "janus_expert_ffn_vjp_rows", "janus_expert_ffn_fwd_ex",
     "janus_expert_ffn_packed_workspace_size", "janus_expert_ffn_fwd_packed",
+    "janus_expert_ffn_split_workspace_size", "janus_expert_ffn_fwd_split", "janus_expert_ffn_vjp_split",
     "janus_expert_ffn_weight_grad_workspace_size", "janus_expert_ffn_weight_grad",
     "janus_expert_ffn_vjp_vjp_workspace_size", "janus_expert_ffn_vjp_vjp",
     "janus_combine", "janus_edge_aggregate", "janus_edge_broadcast", "janus_neighbor_aggregate",
@@ -111,6 +112,8 @@ def _declare(L):
                                     vp]),
         "janus_active_experts": (st, [vp, i32, i32, vp, vp, vp]),
         "janus_dispatch": (st, [vp, i64, i32, i32, vp, vp, vp, vp]),
+        "janus_dispatch_split_workspace_size": (st, [i64, psz]),
+        "janus_dispatch_split": (st, [vp, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp]),
         "janus_quant_by_type_workspace_size": (st, [i32, psz]),
         "janus_quant_by_type": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp, sz, vp]),
         "janus_quant_by_type_noalloc": (st, [vp, i64, i32, i32, vp, i32, vp, vp, vp, vp]),
@@ -127,9 +130,12 @@ def _declare(L):
                                            ctypes.c_int, vp, sz, vp]),
         "janus_expert_ffn_fwd_ex": (st, [vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, ctypes.c_uint32,
                                          ctypes.c_int, vp, sz, vp]),
-        "janus_expert_ffn_packed_workspace_size": (st, [i64, i32, i32, ctypes.c_int, psz]),
+        "janus_expert_ffn_packed_workspace_size": (st, [i64, i32, i32, i32, ctypes.c_int, psz]),
         "janus_expert_ffn_fwd_packed": (st, [vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, ctypes.c_int,
                                              vp, sz, vp]),
+        "janus_expert_ffn_split_workspace_size": (st, [i64, i32, i32, i32, psz]),
+        "janus_expert_ffn_fwd_split": (st, [vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "janus_expert_ffn_vjp_split": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp]),
         "janus_expert_ffn_weight_grad_workspace_size": (st, [i64, i32, i32, psz]),
         "janus_expert_ffn_weight_grad": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp,
                                               ctypes.c_int, vp, sz, vp]),
@@ -303,6 +309,33 @@ def janus_dispatch(x, slot_of, top_k, topk_weight=None, *, out=None, stream=None
                                 _p(topk_weight, torch.float32, "topk_weight"),
                                 _p(out, torch.float32, "xd"), _stream(stream)), "janus_dispatch")
     return out
+
+
+def janus_dispatch_split_workspace_size(n_atoms) -> int:
+    b = ctypes.c_size_t(0)
+    _raise(lib().janus_dispatch_split_workspace_size(int(n_atoms), ctypes.byref(b)),
+           "janus_dispatch_split_workspace_size")
+    return b.value
+
+
+def janus_dispatch_split(x, slot_of, top_k, topk_weight=None, *, out=None, row_scale=None, workspace=None,
+                         stream=None):
+    """Dispatch into two FP16 terms per value with a per-row power-of-two
+    scale: returns (rows16 [2R, d] float16 = [hi | mid], row_scale [R])."""
+    N, d = x.shape
+    K = int(top_k)
+    R = N * K
+    if out is None:
+        out = _empty((2 * R, d), torch.float16, x.device)
+    if row_scale is None:
+        row_scale = _empty((R,), torch.float32, x.device)
+    nb = janus_dispatch_split_workspace_size(N)
+    ws = _workspace(nb, x.device, workspace)
+    _raise(lib().janus_dispatch_split(_p(x, torch.float32, "x"), N, d, K, _p(slot_of, torch.int32, "slot_of"),
+                                      _p(topk_weight, torch.float32, "topk_weight"), _p(out, torch.float16, "rows16"),
+                                      _p(row_scale, torch.float32, "row_scale"), _p(ws), nb, _stream(stream)),
+           "janus_dispatch_split")
+    return out, row_scale
 
 
 def janus_combine(yd, slot_of, top_k, topk_weight=None, *, out=None, stream=None):
@@ -628,18 +661,19 @@ def janus_expert_ffn_fwd_ex(xd, offsets, w1, w2, *, out=None, out_rows=None, fla
     return out, act
 
 
-def janus_expert_ffn_packed_workspace_size(n_rows, d, h, mode=JANUS_FFN_FP32_SIMT) -> int:
+def janus_expert_ffn_packed_workspace_size(n_rows, n_experts, d, h, mode=JANUS_FFN_FP32_SIMT) -> int:
     b = ctypes.c_size_t(0)
-    _raise(lib().janus_expert_ffn_packed_workspace_size(n_rows, d, h, int(mode), ctypes.byref(b)),
+    _raise(lib().janus_expert_ffn_packed_workspace_size(n_rows, n_experts, d, h, int(mode), ctypes.byref(b)),
            "janus_expert_ffn_packed_workspace_size")
     return b.value
 
 
 def janus_expert_ffn_fwd_packed(payload, row_scale, offsets, w1, w2, *, out=None, out_rows=None,
                                 mode=JANUS_FFN_FP32_SIMT, want_act=False, act=None, workspace=None, stream=None):
-    """The forward on the FP16 payload [R,d] with per-row scales [R] (the
-    unpack fused into the GEMM); output as in janus_expert_ffn_fwd_ex.
-    Returns (out-or-None, act-or-None)."""
+    """The forward on the FP16 payload [R,d] with per-row scales [R] (3xTF32
+    mode: the first GEMM on the FP16 tensor path against an FP16 split of
+    w1); output as in janus_expert_ffn_fwd_ex.  Returns (out-or-None,
+    act-or-None)."""
     R, d = payload.shape
     E, _, h = w1.shape
     if payload.dtype not in (torch.float16, torch.int16, torch.uint16):
@@ -650,7 +684,7 @@ def janus_expert_ffn_fwd_packed(payload, row_scale, offsets, w1, w2, *, out=None
         out = _empty((R, d), torch.float32, payload.device)
     if want_act and act is None:
         act = _empty((R, h), torch.float32, payload.device)
-    nb = janus_expert_ffn_packed_workspace_size(R, d, h, mode)
+    nb = janus_expert_ffn_packed_workspace_size(R, E, d, h, mode)
     ws = _workspace(nb, payload.device, workspace)
     _raise(lib().janus_expert_ffn_fwd_packed(_p(payload, None, "payload"), _p(row_scale, torch.float32, "row_scale"),
                                              _p(offsets, torch.int32, "offsets"), E, R, d, h,
@@ -660,6 +694,61 @@ def janus_expert_ffn_fwd_packed(payload, row_scale, offsets, w1, w2, *, out=None
                                              _p(act, torch.float32, "act"), int(mode), _p(ws), nb, _stream(stream)),
            "janus_expert_ffn_fwd_packed")
     return out, act
+
+
+def janus_expert_ffn_split_workspace_size(n_rows, n_experts, d, h) -> int:
+    b = ctypes.c_size_t(0)
+    _raise(lib().janus_expert_ffn_split_workspace_size(int(n_rows), int(n_experts), int(d), int(h),
+                                                       ctypes.byref(b)), "janus_expert_ffn_split_workspace_size")
+    return b.value
+
+
+def janus_expert_ffn_fwd_split(rows16, row_scale, offsets, w1, w2, *, out=None, out_rows=None, want_act=False,
+                               act=None, workspace=None, stream=None):
+    """The forward on split rows (janus_dispatch_split): the first GEMM on the
+    FP16 tensor path, the second on 3xTF32.  Returns (out-or-None, act-or-None)."""
+    R2, d = rows16.shape
+    R = R2 // 2
+    E, _, h = w1.shape
+    if out is not None and out_rows is not None:
+        raise ValueError("give out or out_rows, not both")
+    if out is None and out_rows is None:
+        out = _empty((R, d), torch.float32, rows16.device)
+    if want_act and act is None:
+        act = _empty((R, h), torch.float32, rows16.device)
+    nb = janus_expert_ffn_split_workspace_size(R, E, d, h)
+    ws = _workspace(nb, rows16.device, workspace)
+    _raise(lib().janus_expert_ffn_fwd_split(_p(rows16, torch.float16, "rows16"), _p(row_scale, torch.float32, "row_scale"),
+                                            _p(offsets, torch.int32, "offsets"), E, R, d, h,
+                                            _p(w1, torch.float32, "w1"), _p(w2, torch.float32, "w2"),
+                                            _p(out, torch.float32, "yd"),
+                                            None if out_rows is None else _row_table(out_rows, R),
+                                            _p(act, torch.float32, "act"), _p(ws), nb, _stream(stream)),
+           "janus_expert_ffn_fwd_split")
+    return out, act
+
+
+def janus_expert_ffn_vjp_split(gd16, gd_scale, offsets, w1, w2, act, *, out=None, out_rows=None, workspace=None,
+                               stream=None):
+    """The input VJP on split upstream-gradient rows (janus_dispatch_split,
+    weighted) and the forward's pre-activations: dA = (gd W2^T) silu'(a) on
+    the FP16 tensor path, dxd = dA W1^T on 3xTF32.  Returns out-or-None."""
+    R2, d = gd16.shape
+    R = R2 // 2
+    E, _, h = w1.shape
+    if out is not None and out_rows is not None:
+        raise ValueError("give out or out_rows, not both")
+    if out is None and out_rows is None:
+        out = _empty((R, d), torch.float32, gd16.device)
+    nb = janus_expert_ffn_split_workspace_size(R, E, d, h)
+    ws = _workspace(nb, gd16.device, workspace)
+    _raise(lib().janus_expert_ffn_vjp_split(_p(gd16, torch.float16, "gd16"), _p(gd_scale, torch.float32, "gd_scale"),
+                                            _p(act, torch.float32, "act"), _p(offsets, torch.int32, "offsets"), E, R,
+                                            d, h, _p(w1, torch.float32, "w1"), _p(w2, torch.float32, "w2"),
+                                            _p(out, torch.float32, "dxd"),
+                                            None if out_rows is None else _row_table(out_rows, R), _p(ws), nb,
+                                            _stream(stream)), "janus_expert_ffn_vjp_split")
+    return out
 
 
 def janus_expert_ffn_vjp_rows(xd, gd, offsets, w1, w2, dxd_rows, *, act=None, mode=JANUS_FFN_FP32_SIMT,

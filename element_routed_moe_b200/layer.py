@@ -10,12 +10,21 @@ packing of the dispatch, edge aggregation in front of the MoE block) and
 One pass, all on the current stream:
     [edge_aggregate]  X = segment sums of the edge messages (row_ptr given)
     route             per-type top-K, counts, offsets, permutation
-    dispatch          Xd = X rows in expert order   (or FP16 pack + unpack)
+    dispatch          Xd = X rows in expert order   (or FP16 pack, unpacked by the GEMM)
     ffn_fwd           Yd = silu(Xd W1[e]) W2[e]      (a saved)
     combine           Y  = sum_k w * Yd
     dispatch_w        Gd = w * G rows in expert order
     ffn_vjp           dXd = ((Gd W2^T) * silu'(a)) W1^T
     combine_vjp       dX = sum_k dXd
+
+In 3xTF32 mode the forward's first GEMM runs on the FP16 tensor path:
+FP16-packed rows go to janus_expert_ffn_fwd_packed as they are; unpacked rows
+are dispatched as two FP16 terms with a per-row scale (janus_dispatch_split)
+for janus_expert_ffn_fwd_split when the layer has at least SPLIT_MIN_ROWS_PER_EXPERT
+routed rows per expert (below that, re-splitting the weights every call costs
+more than the GEMM saves).  The VJP stays on 3xTF32: its first GEMM is bound
+by the dSiLU epilogue, and the FP16 form (janus_expert_ffn_vjp_split) measured
+no faster.
 
 `run_host` runs the pass from and to pinned host memory with the copies on
 their own streams: the upload of G overlaps the forward, the download of Y
@@ -39,6 +48,10 @@ class MoELayer:
     # this library's kernels per call (see each entry point's launches)
     LAUNCHES = {"edge_aggregate": 1, "quant": 2, "dequant": 1, "row_scales": 1, "route": 4, "dispatch": 1,
                 "ffn_fwd": 2, "combine": 1, "dispatch_w": 1, "ffn_vjp": 2, "combine_vjp": 1}
+    # the FP16 tensor path: row maxima + split dispatch; the weight split
+    # (3 kernels) in front of the two GEMMs
+    LAUNCHES_SPLIT = {"dispatch": 2, "ffn_fwd": 5}
+    SPLIT_MIN_ROWS_PER_EXPERT = 2048
 
     # pinned-host pipeline for edge-message inputs: ring of device buffers
     RING_SLOTS = 8
@@ -75,10 +88,20 @@ class MoELayer:
         # packed: the first GEMM reads the FP16 payload itself (the unpack is
         # fused into it); its tensor-core form needs d % 8 == 0
         self.fused_unpack = packed and (mode == J.JANUS_FFN_FP32_SIMT or d % 8 == 0)
+        # 3xTF32, unpacked rows: the forward's first GEMM on the FP16 tensor
+        # path (rows split into two FP16 terms by the dispatch; d % 8 == 0)
+        # when the rows per expert amortise the per-call weight split
+        self.split = (mode == J.JANUS_FFN_3XTF32 and not packed and d % 8 == 0
+                      and R >= self.SPLIT_MIN_ROWS_PER_EXPERT * E)
         nb = max(J.janus_expert_ffn_workspace_size(R, d, h, E, False, True, mode),
                  J.janus_expert_ffn_workspace_size(R, d, h, E, True, True, mode),
-                 J.janus_expert_ffn_packed_workspace_size(R, d, h, mode) if self.fused_unpack else 0)
+                 J.janus_expert_ffn_packed_workspace_size(R, E, d, h, mode) if self.fused_unpack else 0,
+                 J.janus_expert_ffn_split_workspace_size(R, E, d, h) if self.split else 0)
         self.ffn_ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        if self.split:
+            self.xd16 = torch.empty((2 * R, d), dtype=torch.float16, device=dev)
+            self.xd_scale = torch.empty((R,), **f32)
+            self.split_ws = torch.empty(J.janus_dispatch_split_workspace_size(N), dtype=torch.uint8, device=dev)
         if row_ptr is not None:
             self.xagg = torch.empty((N, d), **f32)
         if packed:
@@ -92,7 +115,19 @@ class MoELayer:
         else:
             mid = ("route", "dispatch")
         self.ops = front + mid + ("ffn_fwd", "combine") + self.OPS_VJP
-        self.launches_per_call = sum(self.LAUNCHES[o] for o in self.ops)
+        launches = dict(self.LAUNCHES)
+        if self.split:
+            launches.update(self.LAUNCHES_SPLIT)
+        if self.packed and self.fused_unpack and mode == J.JANUS_FFN_3XTF32:
+            launches["ffn_fwd"] = 5           # the weight split + the two GEMMs
+        # the library also runs the forward's second GEMM on the FP16 path
+        # (with H's row split and W2's split in front) at >= 2048 rows per
+        # expert and h % 8 == 0, after either FP16 first GEMM
+        fp16_first = self.split or (self.packed and self.fused_unpack and mode == J.JANUS_FFN_3XTF32)
+        self.f16_second = fp16_first and h % 8 == 0 and R >= 2048 * E
+        if self.f16_second:
+            launches["ffn_fwd"] += 5          # row maxima + row split + 3 weight-split kernels
+        self.launches_per_call = sum(launches[o] for o in self.ops)
         self._host = None
 
     # -- device-resident pass ----------------------------------------------------
@@ -132,12 +167,19 @@ class MoELayer:
                 mark("dequant", 0)
                 J.janus_dequant_by_type(self.payload, types, T, r["perm"], K, self.scale, out=self.xd)
                 mark("dequant", 1)
+        elif self.split:
+            mark("dispatch", 0)
+            J.janus_dispatch_split(x, r["slot_of"], K, out=self.xd16, row_scale=self.xd_scale, workspace=self.split_ws)
+            mark("dispatch", 1)
         else:
             mark("dispatch", 0)
             J.janus_dispatch(x, r["slot_of"], K, out=self.xd)
             mark("dispatch", 1)
         mark("ffn_fwd", 0)
-        if self.fused_unpack:
+        if self.split:
+            J.janus_expert_ffn_fwd_split(self.xd16, self.xd_scale, r["offsets"], self.w1, self.w2, out=self.yd,
+                                         act=self.act, workspace=self.ffn_ws)
+        elif self.fused_unpack:
             # the FP16 rows go straight into the first GEMM (xd is not written)
             J.janus_expert_ffn_fwd_packed(self.payload, self.row_scale, r["offsets"], self.w1, self.w2, out=self.yd,
                                           act=self.act, mode=self.mode, workspace=self.ffn_ws)

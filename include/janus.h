@@ -146,6 +146,27 @@ janus_status janus_dispatch(const float* x, int64_t n_atoms, int32_t d, int32_t 
                             const int32_t* slot_of, const float* topk_weight,
                             float* xd, janus_stream_t stream);
 
+/* Dispatch into two FP16 terms per value, for the expert MLP's FP16
+ * tensor-core GEMMs (janus_expert_ffn_fwd_split / _vjp_split).  Same rows
+ * and values as janus_dispatch, v = x[i,:] * (topk_weight[i*K+k] or 1) in
+ * FP32, written for dispatch row p = slot_of[i*K+k] as
+ *   hi[p,:] = fp16(v * S_p),  mid[p,:] = fp16(v * S_p - hi[p,:]),
+ *   row_scale[p] = 1 / S_p,
+ * with S_p the power of two that puts the row's largest |v| in [2^14, 2^15)
+ * (1 for a zero row; clamped to [2^-126, 2^126]).  hi + mid carries 22
+ * significant bits of every value within 2^18 of the row's largest; smaller
+ * values keep an absolute error below 2^-40 of it.  Not on the pages: an
+ * implementation layout of the dispatch buffer for the FP16 tensor path.
+ * out: rows16 = [hi | mid], 2 R rows of d binary16 (16-byte aligned),
+ *      row_scale [R] float32
+ * workspace: janus_dispatch_split_workspace_size bytes (the rows' maxima),
+ *      256-byte aligned.  Two passes over x (row maxima, then the dispatch). */
+janus_status janus_dispatch_split_workspace_size(int64_t n_atoms, size_t* bytes);
+janus_status janus_dispatch_split(const float* x, int64_t n_atoms, int32_t d, int32_t top_k,
+                                  const int32_t* slot_of, const float* topk_weight, uint16_t* rows16,
+                                  float* row_scale, void* workspace, size_t workspace_bytes,
+                                  janus_stream_t stream);
+
 /* -------------------------------------------------------------------------
  * Atom-type-aware FP16 packing.  [Review] section 3.5 (CNIS, atom-type-aware
  * FP16 compression): after routing, the dispatch buffer's tokens are grouped
@@ -282,17 +303,28 @@ janus_status janus_expert_ffn_fwd_ex(const float* xd, const int32_t* offsets, in
  * row p of xd is f32(payload[p,:]) * row_scale[p] (payload from
  * janus_quant_by_type or an expert-parallel receive buffer; row_scale from
  * janus_dispatch_row_scales or the receive buffer's scales).  yd or yd_rows
- * (exactly one non-NULL) as in janus_expert_ffn_fwd_ex.  In
- * JANUS_FFN_3XTF32 the first GEMM loads the FP16 rows by TMA, unpacks them in
- * shared memory and runs two tensor-core products (the rows are exact in
- * TF32); d must be a multiple of 8 (JANUS_ERR_MISALIGNED otherwise) and the
- * payload 16-byte aligned.  In JANUS_FFN_FP32_SIMT the rows are unpacked
- * into the workspace first.  The result is bit-identical to
- * janus_dequant_by_type followed by janus_expert_ffn_fwd_ex with
- * JANUS_FFN_X_DEQUANTIZED.  workspace: janus_expert_ffn_packed_workspace_size
- * bytes, 256-byte aligned. */
-janus_status janus_expert_ffn_packed_workspace_size(int64_t n_rows, int32_t d, int32_t h, janus_ffn_mode mode,
-                                                    size_t* bytes);
+ * (exactly one non-NULL) as in janus_expert_ffn_fwd_ex.
+ * JANUS_FFN_3XTF32: the first GEMM multiplies the FP16 rows, as they are,
+ * on the tcgen05 kind::f16 tensor path against an FP16 split of W1 that the
+ * call writes into the workspace first: per expert and output feature f, a
+ * power-of-two scale S_f puts the column's largest |w| in [2^14, 2^15), and
+ * w S_f = hi + mid (two binary16 terms, 22 bits), so
+ *   a[p,f] = row_scale[p] / S_f * sum_k payload[p,k] (hi[f,k] + mid[f,k])
+ * with exact FP16 products and FP32 accumulation (chunked as in the 3xTF32
+ * GEMM): FP32-accurate, within 1e-5 of the unpacked FP32 forward, at half
+ * the tensor-core work of the two-product TF32 form.  The second GEMM (H W2)
+ * runs on 3xTF32, or, when n_rows >= 2048 * n_experts and h % 8 == 0, on the
+ * same kind::f16 path with three products after H is split into two FP16
+ * terms per row in the workspace (as janus_dispatch_split does) and W2 is
+ * split like W1.  d must be a multiple of 8 (JANUS_ERR_MISALIGNED
+ * otherwise) and the payload 16-byte aligned.
+ * JANUS_FFN_FP32_SIMT: the rows are unpacked into the workspace first; the
+ * result is bit-identical to janus_dequant_by_type followed by
+ * janus_expert_ffn_fwd.
+ * workspace: janus_expert_ffn_packed_workspace_size bytes (it depends on
+ * n_experts through the weight split), 256-byte aligned. */
+janus_status janus_expert_ffn_packed_workspace_size(int64_t n_rows, int32_t n_experts, int32_t d, int32_t h,
+                                                    janus_ffn_mode mode, size_t* bytes);
 janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, const float* row_scale, const int32_t* offsets,
                                          int32_t n_experts, int64_t n_rows, int32_t d, int32_t h, const float* w1,
                                          const float* w2, float* yd, float* const* yd_rows, float* act,
@@ -303,6 +335,37 @@ janus_status janus_expert_ffn_vjp_rows(const float* xd, const float* gd, const f
                                        int32_t d, int32_t h, const float* w1, const float* w2,
                                        float* const* dxd_rows, janus_ffn_mode mode, void* workspace,
                                        size_t workspace_bytes, janus_stream_t stream);
+
+/* The expert MLP on dispatch rows given as two FP16 terms with a per-row
+ * scale (janus_dispatch_split), on the tensor cores: the first GEMM of the
+ * forward (a = xd W1 -> act, silu(a)) or of the input VJP (dA = (gd W2^T) *
+ * silu'(a)) runs on the tcgen05 kind::f16 path with three products,
+ *   hi_x hi_w + hi_x mid_w + mid_x hi_w,
+ * against an FP16 split of the weights written into the workspace first (per
+ * output feature a power-of-two scale and two binary16 terms, as in
+ * janus_expert_ffn_fwd_packed); products are exact and accumulate in FP32 in
+ * chunks of 256, the result is scaled by row_scale[p] and the feature's
+ * 1 / S.  The second GEMM runs on 3xTF32, or, in the forward with n_rows >=
+ * 2048 * n_experts and h % 8 == 0, on the same kind::f16 path after H is
+ * split into two FP16 terms per row in the workspace.  FP32-accurate as the
+ * 3xTF32 forms (within 1e-5), at half their tensor-core work per FP16 GEMM.
+ * fwd: rows16 = [hi | mid] of xd, act [R,h] nullable, yd or yd_rows (one).
+ * vjp: gd16 = [hi | mid] of the gate-weighted upstream gradient rows, act
+ *      = the forward's pre-activations (required), dxd or dxd_rows (one).
+ * d % 8 == 0, h % 4 == 0 (JANUS_ERR_MISALIGNED otherwise); N*K < 2^30.
+ * workspace: janus_expert_ffn_split_workspace_size bytes, 256-byte aligned;
+ * its error word reports as in janus_expert_ffn_fwd. */
+janus_status janus_expert_ffn_split_workspace_size(int64_t n_rows, int32_t n_experts, int32_t d, int32_t h,
+                                                   size_t* bytes);
+janus_status janus_expert_ffn_fwd_split(const uint16_t* rows16, const float* row_scale, const int32_t* offsets,
+                                        int32_t n_experts, int64_t n_rows, int32_t d, int32_t h, const float* w1,
+                                        const float* w2, float* yd, float* const* yd_rows, float* act,
+                                        void* workspace, size_t workspace_bytes, janus_stream_t stream);
+janus_status janus_expert_ffn_vjp_split(const uint16_t* gd16, const float* gd_scale, const float* act,
+                                        const int32_t* offsets, int32_t n_experts, int64_t n_rows, int32_t d,
+                                        int32_t h, const float* w1, const float* w2, float* dxd,
+                                        float* const* dxd_rows, void* workspace, size_t workspace_bytes,
+                                        janus_stream_t stream);
 
 /* Expert weight gradients, the parameter side of the same backward pass
  * (force training differentiates the energy w.r.t. inputs and weights,

@@ -17,7 +17,7 @@ import torch
 import oracle
 from element_routed_moe_b200 import janus as J
 from element_routed_moe_b200 import synth
-from helpers import DEV, TOL_FP32, host, rel_fro, sample_rows, to_dev
+from helpers import DEV, TOL_FP32, TOL_ROW, host, max_row_rel, rel_fro, sample_rows, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -90,13 +90,21 @@ def test_rows_that_break_the_promise_are_reported():
 
 
 # ---------------------------------------------------------------------------
-# the forward on the FP16 payload itself: the unpack fused into the GEMM
+# the forward on the FP16 payload itself.  SIMT: the rows are unpacked first,
+# bit-identical to unpack + forward.  3xTF32: the first GEMM multiplies the
+# FP16 rows on the kind::f16 tensor path against a two-term FP16 split of
+# W1 (per-feature power-of-two scale), so it is compared with the oracle and
+# with the unpacked 3xTF32 forward by tolerance, per row as well as overall.
 # ---------------------------------------------------------------------------
 PACKED = {
     # name: (N, T, E, K, d, h)
     "ragged8": (700, 11, 12, 3, 136, 68),
     "M_like": (4096, 89, 40, 8, 512, 384),
     "tails": (257, 5, 9, 2, 8, 4),
+    "wide_k": (300, 7, 3, 2, 1544, 200),       # 24 full 64-wide k-blocks + an 8-wide tail
+    # >= 2048 rows per expert and h % 8 == 0: the second GEMM (H W2) runs on
+    # the FP16 path too, over a 200-wide K (three 64-wide blocks + an 8 tail)
+    "second_f16": (3200, 9, 3, 2, 136, 200),
 }
 
 
@@ -111,7 +119,7 @@ def _packed_inputs(N, T, E, K, d, seed):
 
 @pytest.mark.parametrize("mode", [J.JANUS_FFN_FP32_SIMT, J.JANUS_FFN_3XTF32])
 @pytest.mark.parametrize("name", list(PACKED))
-def test_packed_forward_equals_unpack_then_forward(name, mode):
+def test_packed_forward_matches_unpack_then_forward(name, mode):
     N, T, E, K, d, h = PACKED[name]
     types, r, payload, scale = _packed_inputs(N, T, E, K, d, 70)
     w1, w2 = synth.expert_weights(E, d, h, 71, DEV)
@@ -122,16 +130,79 @@ def test_packed_forward_equals_unpack_then_forward(name, mode):
     xd = J.janus_dequant_by_type(payload, types, T, r["perm"], K, scale)
     y_ref, a_ref = J.janus_expert_ffn_fwd_ex(xd, r["offsets"], w1, w2, flags=J.JANUS_FFN_X_DEQUANTIZED, mode=mode,
                                              want_act=True)
-    nb = J.janus_expert_ffn_packed_workspace_size(xd.shape[0], d, h, mode)
+    nb = J.janus_expert_ffn_packed_workspace_size(xd.shape[0], E, d, h, mode)
     ws = torch.zeros(nb, dtype=torch.uint8, device=DEV)
     y, a = J.janus_expert_ffn_fwd_packed(payload, row_scale, r["offsets"], w1, w2, mode=mode, want_act=True,
                                          workspace=ws)
     J.janus_check(ws)
-    assert torch.equal(y, y_ref) and torch.equal(a, a_ref)
+    if mode == J.JANUS_FFN_FP32_SIMT:
+        assert torch.equal(y, y_ref) and torch.equal(a, a_ref)
+    else:
+        assert rel_fro(host(a), host(a_ref)) <= TOL_FP32 and rel_fro(host(y), host(y_ref)) <= TOL_FP32
+        assert max_row_rel(host(y), host(y_ref)) <= TOL_ROW
+        assert torch.isfinite(y).all().item()
     offs = host(r["offsets"])
     rows = sample_rows(offs, 64, seed=5, R=xd.shape[0])
-    ref = oracle.expert_ffn_fwd(host(xd), offs, host(w1), host(w2), rows=rows)
-    assert rel_fro(host(y)[rows], ref) <= TOL_FP32
+    ref, ref_a = oracle.expert_ffn_fwd(host(xd), offs, host(w1), host(w2), rows=rows, want_act=True)
+    assert rel_fro(host(y)[rows], ref) <= TOL_FP32 and rel_fro(host(a)[rows], ref_a) <= TOL_FP32
+    assert max_row_rel(host(y)[rows], ref) <= TOL_ROW
+
+
+def test_packed_forward_weight_split_handles_wide_column_ranges():
+    # the FP16 split scales each weight column on its own: a column a million
+    # times larger than the rest, an all-zero column, a column of values near
+    # 1e-32 and a column whose one entry is 40,000 times its others all stay
+    # within the FP32 tolerance of the oracle, column by column
+    N, T, E, K, d, h = 600, 7, 4, 2, 128, 72
+    types, r, payload, scale = _packed_inputs(N, T, E, K, d, 73)
+    w1, w2 = synth.expert_weights(E, d, h, 74, DEV)
+    w1[:, :, 3] *= 1.0e6
+    w1[:, :, 5] = 0.0
+    w1[:, :, 9] *= 1.0e-30
+    w1[1, 17, 11] = 1.0e3
+    row_scale = J.janus_dispatch_row_scales(types, T, r["perm"], K, scale)
+    y, a = J.janus_expert_ffn_fwd_packed(payload, row_scale, r["offsets"], w1, w2, mode=J.JANUS_FFN_3XTF32,
+                                         want_act=True)
+    torch.cuda.synchronize()
+    xd = J.janus_dequant_by_type(payload, types, T, r["perm"], K, scale)
+    offs = host(r["offsets"])
+    ref_y, ref_a = oracle.expert_ffn_fwd(host(xd), offs, host(w1), host(w2), want_act=True)
+    # per feature column of the pre-activation: each is scaled on its own
+    ha = host(a).astype(np.float64)
+    for f in (0, 3, 9, 11, 40):
+        col, rc = ha[:, f], ref_a[:, f].astype(np.float64)
+        assert np.linalg.norm(col - rc) <= TOL_FP32 * np.linalg.norm(rc), f
+    assert np.all(ha[:, 5] == 0.0)
+    assert rel_fro(host(y), ref_y) <= TOL_FP32
+
+
+def test_fp16_second_gemm_handles_wide_column_ranges_of_w2():
+    # the second GEMM's W2 split scales each output feature on its own, and
+    # H's split each row: W2 columns far apart in magnitude, an all-zero
+    # column and one large entry stay within the FP32 tolerance column by
+    # column (6,400 rows over 3 experts put it on the FP16 path)
+    N, T, E, K, d, h = 3200, 7, 3, 2, 128, 72
+    types, r, payload, scale = _packed_inputs(N, T, E, K, d, 75)
+    w1, w2 = synth.expert_weights(E, d, h, 76, DEV)
+    w2[:, :, 3] *= 1.0e6
+    w2[:, :, 5] = 0.0
+    w2[:, :, 9] *= 1.0e-30
+    w2[1, 17, 11] = 1.0e3
+    row_scale = J.janus_dispatch_row_scales(types, T, r["perm"], K, scale)
+    nb = J.janus_expert_ffn_packed_workspace_size(N * K, E, d, h, J.JANUS_FFN_3XTF32)
+    ws = torch.zeros(nb, dtype=torch.uint8, device=DEV)
+    y, _ = J.janus_expert_ffn_fwd_packed(payload, row_scale, r["offsets"], w1, w2, mode=J.JANUS_FFN_3XTF32,
+                                         workspace=ws)
+    J.janus_check(ws)
+    xd = J.janus_dequant_by_type(payload, types, T, r["perm"], K, scale)
+    offs = host(r["offsets"])
+    ref_y = oracle.expert_ffn_fwd(host(xd), offs, host(w1), host(w2))
+    hy = host(y).astype(np.float64)
+    for f in (0, 3, 9, 11, 40):
+        col, rc = hy[:, f], ref_y[:, f].astype(np.float64)
+        assert np.linalg.norm(col - rc) <= TOL_FP32 * np.linalg.norm(rc), f
+    assert np.all(hy[:, 5] == 0.0)
+    assert rel_fro(hy, ref_y) <= TOL_FP32
 
 
 def test_packed_forward_into_a_row_table():

@@ -69,17 +69,29 @@ def test_random_shape_chain(seed):
         dxd = J.janus_expert_ffn_vjp(xd, gd, r["offsets"], w1, w2, act=act, mode=mode)
         assert rel_fro(host(yd), oyd) <= TOL_FP32, (mode, seed)
         assert rel_fro(host(dxd), odxd) <= TOL_FP32, (mode, seed)
-    # the forward on the FP16 rows themselves (unpack fused into the GEMM) and on
-    # the unpacked rows with the exact-TF32 flag: both bit-identical to the plain
-    # forward on the unpacked rows
+    # the forward on the unpacked rows with the exact-TF32 flag: bit-identical
+    # to the plain forward on them; on the FP16 rows themselves: SIMT unpacks
+    # first (bit-identical), 3xTF32 runs the FP16 tensor path against a split
+    # of W1 (within the FP32 tolerance of the plain forward and the oracle);
+    # and the split-row forward and VJP (FP16 tensor path, d % 8 == 0)
     row_scale = J.janus_dispatch_row_scales(to_dev(types), T, r["perm"], K, scale)
+    oyq = oracle.expert_ffn_fwd(host(xq), o["offsets"], hw1, hw2)
     for mode in (J.JANUS_FFN_FP32_SIMT, J.JANUS_FFN_3XTF32):
         yq, _ = J.janus_expert_ffn_fwd(xq, r["offsets"], w1, w2, mode=mode)
         yf, _ = J.janus_expert_ffn_fwd_ex(xq, r["offsets"], w1, w2, flags=J.JANUS_FFN_X_DEQUANTIZED, mode=mode)
         assert torch.equal(yf, yq), (mode, seed)
         if mode == J.JANUS_FFN_FP32_SIMT or d % 8 == 0:
             yp, _ = J.janus_expert_ffn_fwd_packed(payload, row_scale, r["offsets"], w1, w2, mode=mode)
-            assert torch.equal(yp, yq), (mode, seed)
+            if mode == J.JANUS_FFN_FP32_SIMT:
+                assert torch.equal(yp, yq), (mode, seed)
+            else:
+                assert rel_fro(host(yp), host(yq)) <= TOL_FP32 and rel_fro(host(yp), oyq) <= TOL_FP32, (mode, seed)
+    if d % 8 == 0:
+        x16, xs = J.janus_dispatch_split(x, r["slot_of"], K)
+        g16, gs = J.janus_dispatch_split(g, r["slot_of"], K, r["topk_weight"])
+        ys, a_s = J.janus_expert_ffn_fwd_split(x16, xs, r["offsets"], w1, w2, want_act=True)
+        dxs = J.janus_expert_ffn_vjp_split(g16, gs, r["offsets"], w1, w2, a_s)
+        assert rel_fro(host(ys), oyd) <= TOL_FP32 and rel_fro(host(dxs), odxd) <= TOL_FP32, seed
     y = J.janus_combine(yd, r["slot_of"], K, r["topk_weight"])
     assert rel_fro(host(y), oracle.combine(host(yd), o["slot_of"], K, o["topk_weight"])) <= TOL_FP32
     dx = J.janus_combine(dxd, r["slot_of"], K)
