@@ -298,12 +298,12 @@ class Layer:
     def work(self):
         c = self.cfg
         N, R, d, h = c.n_atoms, c.n_rows, c.d, c.h
-        split = self.core.split
+        split, split_vjp = self.core.split, self.core.split_vjp
         w = {
             # split dispatch: a first pass reads X for the row maxima; the two
             # FP16 planes are as many bytes as the FP32 rows, plus a scale per row
             "dispatch": ("bytes", 4 * d * (N + R) + 4 * R + ((4 * N * d + 4 * R) if split else 0)),
-            "dispatch_w": ("bytes", 4 * d * (N + R) + 8 * R),
+            "dispatch_w": ("bytes", 4 * d * (N + R) + 8 * R + ((4 * N * d + 4 * R) if split_vjp else 0)),
             "combine": ("bytes", 4 * d * (R + N) + 8 * R),
             "combine_vjp": ("bytes", 4 * d * (R + N) + 4 * R),
             "ffn_fwd": ("flops", 4 * R * d * h),
@@ -528,7 +528,8 @@ def run_janus(args, world, rank, local):
         first = ("f16", 2) if core.fused_unpack else ("tf32", 2)
     else:
         first = ("f16", 3) if core.split else ("tf32", 3)
-    kinds = [first, ("f16", 3) if core.f16_second else ("tf32", 3), ("tf32", 3), ("tf32", 3)]
+    vjp = [("f16", 3)] * 2 if core.split_vjp else [("tf32", 3)] * 2
+    kinds = [first, ("f16", 3) if core.f16_second else ("tf32", 3)] + vjp
     roof = gemm_roofline(J, mode, cfg, kinds, peaks, peak_src, work["ffn_fwd"][1] / 2, ffn_ms, 4)
     roof["traffic"] = measured_traffic(cfg.name, args.mode) if cfg == synth.CONFIGS[cfg.name] else None
     roof["traffic_unit"] = "DRAM bytes per launch (mean of the step's 4 launches)"
@@ -583,9 +584,19 @@ def run_cold_l2(layer, peaks, reps=5):
     calls = {
         "dispatch": lambda: J.janus_dispatch(x, r["slot_of"], K, out=layer.xd),
         "dispatch_w": lambda: J.janus_dispatch(layer.g, r["slot_of"], K, r["topk_weight"], out=layer.gd),
+    }
+    # the calls the step makes: the split dispatch on the FP16 tensor path
+    if core.split:
+        calls["dispatch"] = lambda: J.janus_dispatch_split(x, r["slot_of"], K, out=core.xd16, row_scale=core.xd_scale,
+                                                           workspace=core.split_ws)
+    if core.split_vjp:
+        calls["dispatch_w"] = lambda: J.janus_dispatch_split(layer.g, r["slot_of"], K, r["topk_weight"],
+                                                             out=core.gd16, row_scale=core.gd_scale,
+                                                             workspace=core.split_ws)
+    calls.update({
         "combine": lambda: J.janus_combine(core.yd, r["slot_of"], K, r["topk_weight"], out=layer.y),
         "combine_vjp": lambda: J.janus_combine(core.dxd, r["slot_of"], K, out=layer.dx),
-    }
+    })
     if layer.edges:
         calls["edge_aggregate"] = lambda: J.janus_edge_aggregate(layer.msg, layer.row_ptr, out=core.xagg)
     if layer.packed:

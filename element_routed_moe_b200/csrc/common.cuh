@@ -55,13 +55,6 @@ bool consume_injected_failure();
 // Number of SMs of the current device.
 int num_sms();
 
-// Two-term FP16 split of `rows` rows of d floats in place of a dispatch (row
-// i -> row i, as janus_dispatch_split with an identity map): rows16 = [hi |
-// mid] planes, row_scale [rows], rowmax [rows] scratch.  d % 4 == 0, x and
-// rows16 16-byte aligned.
-janus_status rows_split_f16(const float* x, int64_t rows, int32_t d, uint16_t* rows16, float* row_scale,
-                            uint32_t* rowmax, cudaStream_t stream);
-
 inline janus_status launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? JANUS_OK : JANUS_ERR_CUDA;

@@ -88,9 +88,10 @@ unpack_rows_kernel(const uint2* __restrict__ payload, const float* __restrict__ 
   }
 }
 
-// The forward's second GEMM (H W2) runs on the kind::f16 path too when the
-// layer has at least this many routed rows per expert: its row split of H and
-// the per-call split of W2 then cost less than the GEMM saves.
+// The MLP's second GEMM (H W2 in the forward, dA W1^T in the split VJP)
+// runs on the kind::f16 path too when the layer has at least this many
+// routed rows per expert: the activation's row split and the per-call split
+// of the weights then cost less than the GEMM saves.
 constexpr int64_t kF16SecondMinRowsPerExpert = 2048;
 bool use_f16_second(int64_t R, int32_t E, int32_t h) {
   return h % 8 == 0 && R >= kF16SecondMinRowsPerExpert * E;
@@ -98,7 +99,7 @@ bool use_f16_second(int64_t R, int32_t E, int32_t h) {
 
 // Scratch of the FP16 second GEMM (see tc::F16Second), starting at `base`.
 size_t f16_second_bytes(int64_t R, int32_t E, int32_t d, int32_t h) {
-  return align_up(2 * sizeof(uint16_t) * (size_t)R * h, 256) + 2 * align_up(sizeof(float) * (size_t)R, 256) +
+  return align_up(2 * sizeof(uint16_t) * (size_t)R * h, 256) + align_up(sizeof(float) * (size_t)R, 256) +
          align_up(2 * sizeof(uint16_t) * (size_t)E * d * h, 256) + align_up(sizeof(float) * (size_t)E * d, 256);
 }
 tc::F16Second f16_second_at(char* base, int64_t R, int32_t E, int32_t d, int32_t h) {
@@ -106,8 +107,6 @@ tc::F16Second f16_second_at(char* base, int64_t R, int32_t E, int32_t d, int32_t
   f.h16 = (uint16_t*)base;
   base += align_up(2 * sizeof(uint16_t) * (size_t)R * h, 256);
   f.hscale = (float*)base;
-  base += align_up(sizeof(float) * (size_t)R, 256);
-  f.rowmax = (uint32_t*)base;
   base += align_up(sizeof(float) * (size_t)R, 256);
   f.w16 = (uint16_t*)base;
   base += align_up(2 * sizeof(uint16_t) * (size_t)E * d * h, 256);
@@ -191,9 +190,11 @@ extern "C" janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, con
 // ---------------------------------------------------------------------------
 // The expert MLP on rows given as two FP16 terms with a per-row scale
 // (janus_dispatch_split): the first GEMM of the forward (x W1) or of the VJP
-// (gd W2^T, dSiLU epilogue) on the kind::f16 tensor path, the second on
-// 3xTF32.  Workspace: header | H or dA [R,h] | the FP16 split of the first
-// GEMM's weights (hi and mid, [E][h][d] each) | 1 / S [E][h].
+// (gd W2^T) on the kind::f16 tensor path; the second on 3xTF32, or on the
+// kind::f16 path at >= 2048 rows per expert with h % 8 == 0.  Workspace:
+// header | H, dH or dA [R,h] | the FP16 split of the first GEMM's weights
+// (hi and mid, [E][h][d] each) | 1 / S [E][h] | the FP16 second GEMM's
+// scratch when it is used.
 // ---------------------------------------------------------------------------
 namespace {
 struct SplitLayout {
@@ -277,9 +278,11 @@ extern "C" janus_status janus_expert_ffn_vjp_split(const uint16_t* gd16, const f
   const SplitLayout L = split_layout(n_rows, n_experts, d, h);
   char* w = (char*)workspace;
   JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
+  const tc::F16Second second = f16_second_at(w + L.off_second, n_rows, n_experts, d, h);
   st = tc::expert_ffn_vjp_split(gd16, gd_scale, act, offsets, n_experts, n_rows, d, h, w1, w2, dxd,
                                 (float*)(w + L.off_h), (uint16_t*)(w + L.off_w16), (float*)(w + L.off_winv),
-                                &((WsHeader*)workspace)->error, stream, dxd_rows);
+                                &((WsHeader*)workspace)->error, stream, dxd_rows,
+                                use_f16_second(n_rows, n_experts, h) ? &second : nullptr);
   if (st != JANUS_OK) return st;
   return launch_status();
 }

@@ -1124,6 +1124,92 @@ __global__ void __launch_bounds__(256) w16_inv_scale_kernel(uint32_t* __restrict
     colmax_to_inv[i] = (uint32_t)(127 - w16_scale_exp(colmax_to_inv[i])) << 23;
 }
 
+// ---- the FP16 row split of an activation for a kind::f16 GEMM ---------------
+// v = silu(a) (kActSilu) or x silu'(a) (kActDSilu), with the SiLU arithmetic
+// of the GEMM epilogues, written as hi and mid binary16 planes ([rows][n]
+// each) with one power-of-two scale per row: S_p puts the row's largest |v|
+// in [2^14, 2^15), hi = fp16(v S_p), mid = fp16(v S_p - hi), row_scale[p] =
+// 1 / S_p.  One warp per row: a first sweep takes the row's maximum, a second
+// recomputes v and writes the two terms; the second sweep's loads find the
+// row in L1 / L2, so the activations are read from DRAM once and the FP32 v
+// is never stored.
+enum ActOp { kActSilu = 1, kActDSilu = 2 };
+constexpr int kActU = 4;       // float4 columns per lane in flight per sweep step
+
+template <int kOp, bool kLast>
+__device__ __forceinline__ float4 act_value(const float4* __restrict__ x, const float4* __restrict__ a, int64_t i) {
+  const float4 av = kLast ? __ldcs(a + i) : __ldg(a + i);
+  if (kOp == kActSilu) return make_float4(silu_f(av.x), silu_f(av.y), silu_f(av.z), silu_f(av.w));
+  const float4 xv = kLast ? __ldcs(x + i) : __ldg(x + i);
+  float4 v;
+  float sg;
+  sg = sigmoid_fast(av.x); v.x = xv.x * (sg * (1.0f + av.x * (1.0f - sg)));
+  sg = sigmoid_fast(av.y); v.y = xv.y * (sg * (1.0f + av.y * (1.0f - sg)));
+  sg = sigmoid_fast(av.z); v.z = xv.z * (sg * (1.0f + av.z * (1.0f - sg)));
+  sg = sigmoid_fast(av.w); v.w = xv.w * (sg * (1.0f + av.w * (1.0f - sg)));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int kOp>
+__global__ void __launch_bounds__(256)
+act_split_kernel(const float4* __restrict__ x, const float4* __restrict__ a, int64_t rows, int n4,
+                 uint2* __restrict__ rows16, float* __restrict__ row_scale) {
+  const int lane = threadIdx.x % 32;
+  const int64_t nw = (int64_t)gridDim.x * 8;
+  uint2* __restrict__ mid = rows16 + rows * n4;
+  for (int64_t p = ((int64_t)blockIdx.x * 256 + threadIdx.x) / 32; p < rows; p += nw) {
+    const int64_t base = p * n4;
+    uint32_t m = 0;
+    for (int c0 = 0; c0 < n4; c0 += 32 * kActU) {
+      float4 v[kActU];
+#pragma unroll
+      for (int u = 0; u < kActU; ++u) {
+        const int c = c0 + u * 32 + lane;
+        v[u] = c < n4 ? act_value<kOp, false>(x, a, base + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kActU; ++u)
+        m = max(m, max(max(__float_as_uint(v[u].x) & 0x7fffffffu, __float_as_uint(v[u].y) & 0x7fffffffu),
+                       max(__float_as_uint(v[u].z) & 0x7fffffffu, __float_as_uint(v[u].w) & 0x7fffffffu)));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const int e = w16_scale_exp(m);
+    const float S = __uint_as_float((uint32_t)(127 + e) << 23);
+    if (lane == 0) row_scale[p] = __uint_as_float((uint32_t)(127 - e) << 23);
+    for (int c0 = 0; c0 < n4; c0 += 32 * kActU) {
+#pragma unroll
+      for (int u = 0; u < kActU; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < n4) {
+          float4 o = act_value<kOp, true>(x, a, base + c);
+          o.x *= S; o.y *= S; o.z *= S; o.w *= S;
+          const uint2 hq = make_uint2(half2_bits(o.x, o.y), half2_bits(o.z, o.w));
+          const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hq.x));
+          const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hq.y));
+          __stcs(reinterpret_cast<uint2*>(rows16) + base + c, hq);
+          __stcs(mid + base + c, make_uint2(half2_bits(o.x - h0.x, o.y - h0.y), half2_bits(o.z - h1.x, o.w - h1.y)));
+        }
+      }
+    }
+  }
+}
+
+template <int kOp>
+janus_status act_split_f16(const float* x, const float* a, int64_t rows, int32_t n, uint16_t* rows16,
+                           float* row_scale, cudaStream_t stream) {
+  if (rows == 0) return JANUS_OK;
+  const int64_t blocks = std::min<int64_t>((rows + 7) / 8, (int64_t)num_sms() * 8);
+  act_split_kernel<kOp><<<(unsigned)blocks, 256, 0, stream>>>((const float4*)x, (const float4*)a, rows, n / 4,
+                                                               (uint2*)rows16, row_scale);
+  return launch_status();
+}
+
 }  // namespace
 
 janus_status split_weights_f16(const float* w, int32_t E, int32_t Kd, int32_t N, bool transposed, uint16_t* w16,
@@ -1163,15 +1249,35 @@ janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, 
 }
 
 namespace {
-// The forward's second GEMM, yd = H W2: on 3xTF32, or (second given) on the
-// kind::f16 path with H split into two FP16 terms per row first.
-janus_status second_gemm(const float* H, const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
-                         const float* w2, float* yd, float* const* yd_rows, int32_t* err, cudaStream_t stream,
-                         const F16Second* second) {
-  if (!second)
+// The forward behind the FP16 split of W1 (transposed to [E][h][d], K-major):
+// the kind::f16 first GEMM on FP16 rows (kBK = kBF16W: the packed payload;
+// kBF16S: two-term split rows), then the second GEMM, yd = H W2.  Without
+// `second` the first GEMM stores a and H = silu(a) and the second runs on
+// 3xTF32.  With it the first GEMM stores only a (into act, else the
+// workspace's H), one pass turns a into H's two FP16 terms per row, W2 is
+// split per output feature, and the second GEMM runs on the kind::f16 path
+// with three products.
+template <int kBK>
+janus_status fwd_f16(const uint16_t* rows, const float* row_scale, const int32_t* offsets, int32_t E, int64_t R,
+                     int32_t d, int32_t h, const float* w1, const float* w2, float* yd, float* act, float* H,
+                     uint16_t* w16, float* winv, int32_t* err, cudaStream_t stream, float* const* yd_rows,
+                     const F16Second* second) {
+  janus_status st = split_weights_f16(w1, E, d, h, true, w16, winv, stream);
+  if (st != JANUS_OK) return st;
+  const float* xq = reinterpret_cast<const float*>(rows);
+  const float* wq = reinterpret_cast<const float*>(w16);
+  if (!second) {
+    st = launch<kModeNN, kEpiSilu, kBK>(xq, wq, R, E, d, h, H, act, nullptr, offsets, err, stream, 0, nullptr,
+                                        nullptr, nullptr, row_scale, winv);
+    if (st != JANUS_OK) return st;
     return launch<kModeNN, kEpiStore>(H, w2, R, E, h, d, yd, nullptr, nullptr, offsets, err, stream, 0, nullptr,
                                       nullptr, yd_rows);
-  janus_status st = rows_split_f16(H, R, h, second->h16, second->hscale, second->rowmax, stream);
+  }
+  float* A = act ? act : H;
+  st = launch<kModeNN, kEpiStore, kBK>(xq, wq, R, E, d, h, A, nullptr, nullptr, offsets, err, stream, 0, nullptr,
+                                       nullptr, nullptr, row_scale, winv);
+  if (st != JANUS_OK) return st;
+  st = act_split_f16<kActSilu>(nullptr, A, R, h, second->h16, second->hscale, stream);
   if (st != JANUS_OK) return st;
   st = split_weights_f16(w2, E, h, d, true, second->w16, second->winv, stream);
   if (st != JANUS_OK) return st;
@@ -1186,43 +1292,49 @@ janus_status expert_ffn_fwd_packed(const uint16_t* payload, const float* row_sca
                                    int32_t E, int64_t R, int32_t d, int32_t h, const float* w1, const float* w2,
                                    float* yd, float* act, float* H, uint16_t* w16, float* winv, int32_t* err,
                                    cudaStream_t stream, float* const* yd_rows, const F16Second* second) {
-  // the FP16 split of W1 (transposed to [E][h][d], K-major), then the
-  // kind::f16 first GEMM on the payload, then the second GEMM
-  janus_status st = split_weights_f16(w1, E, d, h, true, w16, winv, stream);
-  if (st != JANUS_OK) return st;
-  st = launch<kModeNN, kEpiSilu, kBF16W>(reinterpret_cast<const float*>(payload), reinterpret_cast<const float*>(w16),
-                                          R, E, d, h, H, act, nullptr, offsets, err, stream, 0, nullptr, nullptr,
-                                          nullptr, row_scale, winv);
-  if (st != JANUS_OK) return st;
-  return second_gemm(H, offsets, E, R, d, h, w2, yd, yd_rows, err, stream, second);
+  return fwd_f16<kBF16W>(payload, row_scale, offsets, E, R, d, h, w1, w2, yd, act, H, w16, winv, err, stream,
+                         yd_rows, second);
 }
 
 janus_status expert_ffn_fwd_split(const uint16_t* rows16, const float* row_scale, const int32_t* offsets, int32_t E,
                                   int64_t R, int32_t d, int32_t h, const float* w1, const float* w2, float* yd,
                                   float* act, float* H, uint16_t* w16, float* winv, int32_t* err,
                                   cudaStream_t stream, float* const* yd_rows, const F16Second* second) {
-  janus_status st = split_weights_f16(w1, E, d, h, true, w16, winv, stream);
-  if (st != JANUS_OK) return st;
-  st = launch<kModeNN, kEpiSilu, kBF16S>(reinterpret_cast<const float*>(rows16), reinterpret_cast<const float*>(w16),
-                                          R, E, d, h, H, act, nullptr, offsets, err, stream, 0, nullptr, nullptr,
-                                          nullptr, row_scale, winv);
-  if (st != JANUS_OK) return st;
-  return second_gemm(H, offsets, E, R, d, h, w2, yd, yd_rows, err, stream, second);
+  return fwd_f16<kBF16S>(rows16, row_scale, offsets, E, R, d, h, w1, w2, yd, act, H, w16, winv, err, stream,
+                         yd_rows, second);
 }
 
 janus_status expert_ffn_vjp_split(const uint16_t* gd16, const float* gd_scale, const float* act,
                                   const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
                                   const float* w1, const float* w2, float* dxd, float* dA, uint16_t* w16,
-                                  float* winv, int32_t* err, cudaStream_t stream, float* const* dxd_rows) {
-  // dA = (gd W2^T) * silu'(a): W2 [E][h][d] is K-major for this product as it stands
+                                  float* winv, int32_t* err, cudaStream_t stream, float* const* dxd_rows,
+                                  const F16Second* second) {
+  // gd W2^T: W2 [E][h][d] is K-major for this product as it stands
   janus_status st = split_weights_f16(w2, E, d, h, false, w16, winv, stream);
   if (st != JANUS_OK) return st;
-  st = launch<kModeNN, kEpiDSilu, kBF16S>(reinterpret_cast<const float*>(gd16), reinterpret_cast<const float*>(w16),
-                                           R, E, d, h, dA, nullptr, act, offsets, err, stream, 0, nullptr, nullptr,
-                                           nullptr, gd_scale, winv);
+  const float* gq = reinterpret_cast<const float*>(gd16);
+  const float* wq = reinterpret_cast<const float*>(w16);
+  if (!second) {
+    // dA = (gd W2^T) * silu'(a) in the epilogue, then dxd = dA W1^T on 3xTF32
+    st = launch<kModeNN, kEpiDSilu, kBF16S>(gq, wq, R, E, d, h, dA, nullptr, act, offsets, err, stream, 0, nullptr,
+                                             nullptr, nullptr, gd_scale, winv);
+    if (st != JANUS_OK) return st;
+    return launch<kModeNT, kEpiStore>(dA, w1, R, E, h, d, dxd, nullptr, nullptr, offsets, err, stream, 0, nullptr,
+                                      nullptr, dxd_rows);
+  }
+  // dH = gd W2^T stored plain (in dA's buffer); one pass forms dA = dH *
+  // silu'(a) as two FP16 terms per row; W1 [E][d][h] is K-major for dA W1^T
+  st = launch<kModeNN, kEpiStore, kBF16S>(gq, wq, R, E, d, h, dA, nullptr, nullptr, offsets, err, stream, 0, nullptr,
+                                           nullptr, nullptr, gd_scale, winv);
   if (st != JANUS_OK) return st;
-  return launch<kModeNT, kEpiStore>(dA, w1, R, E, h, d, dxd, nullptr, nullptr, offsets, err, stream, 0, nullptr,
-                                    nullptr, dxd_rows);
+  st = act_split_f16<kActDSilu>(dA, act, R, h, second->h16, second->hscale, stream);
+  if (st != JANUS_OK) return st;
+  st = split_weights_f16(w1, E, h, d, false, second->w16, second->winv, stream);
+  if (st != JANUS_OK) return st;
+  return launch<kModeNN, kEpiStore, kBF16S>(reinterpret_cast<const float*>(second->h16),
+                                            reinterpret_cast<const float*>(second->w16), R, E, h, d, dxd, nullptr,
+                                            nullptr, offsets, err, stream, 0, nullptr, nullptr, dxd_rows,
+                                            second->hscale, second->winv);
 }
 
 janus_status expert_ffn_vjp(const float* xd, const float* gd, const float* act_in, float* A,

@@ -21,13 +21,13 @@ janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, 
                             float* act, float* H, int32_t* err, cudaStream_t stream,
                             float* const* yd_rows = nullptr, bool x_tf32_exact = false);
 
-// Scratch of the forward's second GEMM on the kind::f16 path (H W2 with H
-// split into two FP16 terms per row): H's planes [2R][h] and row scales [R],
-// the rows' maxima [R], the FP16 split of W2 ([2E][d][h]) and its 1 / S [E][d].
+// Scratch of the MLP's second GEMM on the kind::f16 path (H W2 in the
+// forward, dA W1^T in the VJP, the [R][h] activation split into two FP16
+// terms per row): the activation's planes [2R][h] and row scales [R], the
+// FP16 split of the weights ([2E][d][h]) and its 1 / S [E][d].
 struct F16Second {
   uint16_t* h16;
   float* hscale;
-  uint32_t* rowmax;
   uint16_t* w16;
   float* winv;
 };
@@ -40,9 +40,12 @@ janus_status split_weights_f16(const float* w, int32_t E, int32_t Kd, int32_t N,
 
 // Forward / input VJP on rows given as two FP16 terms (hi plane [R][d] then
 // mid plane [R][d]) with a per-row scale (janus_dispatch_split): the first
-// GEMM (x W1, or gd W2^T with the dSiLU epilogue) on the kind::f16 path with
-// three products against the FP16 split of W1 / W2 (written into w16 / winv),
-// the second GEMM on 3xTF32.  d % 8 == 0, h % 8 == 0 for the split weights.
+// GEMM (x W1, or gd W2^T) on the kind::f16 path with three products against
+// the FP16 split of W1 / W2 (written into w16 / winv).  The second GEMM runs
+// on 3xTF32 (the VJP's first GEMM then applies silu'(a) in its epilogue into
+// dA), or, with `second`, on the kind::f16 path after one pass splits the
+// activation (H = silu(a), or dA = dH silu'(a) with dH stored into dA's
+// buffer) into two FP16 terms per row.  d % 8 == 0; h % 8 == 0 with second.
 janus_status expert_ffn_fwd_split(const uint16_t* rows16, const float* row_scale, const int32_t* offsets, int32_t E,
                                   int64_t R, int32_t d, int32_t h, const float* w1, const float* w2, float* yd,
                                   float* act, float* H, uint16_t* w16, float* winv, int32_t* err,
@@ -51,7 +54,8 @@ janus_status expert_ffn_fwd_split(const uint16_t* rows16, const float* row_scale
 janus_status expert_ffn_vjp_split(const uint16_t* gd16, const float* gd_scale, const float* act,
                                   const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
                                   const float* w1, const float* w2, float* dxd, float* dA, uint16_t* w16,
-                                  float* winv, int32_t* err, cudaStream_t stream, float* const* dxd_rows = nullptr);
+                                  float* winv, int32_t* err, cudaStream_t stream, float* const* dxd_rows = nullptr,
+                                  const F16Second* second = nullptr);
 
 // The forward on the FP16 payload itself: row p of xd is f32(payload[p]) *
 // row_scale[p].  The first GEMM runs on the kind::f16 tensor path against the

@@ -229,35 +229,6 @@ dispatch_split_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int
   }
 }
 
-// Rows in place (row i -> row i): the same two-term split for a buffer a
-// kernel of this library has just written (the expert MLP's H = silu(a)).
-__global__ void __launch_bounds__(kThreads)
-rows_split_kernel(const float4* __restrict__ x, int64_t rows, int d4, const uint32_t* __restrict__ rowmax,
-                  uint2* __restrict__ rows16, float* __restrict__ row_scale) {
-  const int lane = threadIdx.x % 32;
-  uint2* mid_plane = rows16 + rows * d4;
-  const ChunkWalk cw = chunk_walk(d4);
-  const int c0 = cw.c0;
-  for (int64_t i = cw.row0; i < rows; i += cw.stride) {
-    const int e = split_exp(rowmax[i]);
-    const float S = __uint_as_float((uint32_t)(127 + e) << 23);
-    if (c0 == 0 && lane == 0) row_scale[i] = __uint_as_float((uint32_t)(127 - e) << 23);
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int c = c0 + u * 32 + lane;
-      if (c < d4) {
-        float4 o = __ldcs(x + i * d4 + c);
-        o.x *= S; o.y *= S; o.z *= S; o.w *= S;
-        const uint2 hq = halves(o.x, o.y, o.z, o.w);
-        const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hq.x));
-        const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hq.y));
-        rows16[i * d4 + c] = hq;
-        mid_plane[i * d4 + c] = halves(o.x - h0.x, o.y - h0.y, o.z - h1.x, o.w - h1.y);
-      }
-    }
-  }
-}
-
 // ---- atom-type-aware FP16 packing ------------------------------------------
 
 __global__ void __launch_bounds__(kThreads)
@@ -421,18 +392,6 @@ extern "C" janus_status janus_combine(const float* yd, const int32_t* slot_of,
         (const float4*)yd, slot_of, nullptr, n_atoms, top_k, d / 4, (float4*)y, debug_fault_word());
   return launch_status();
 }
-
-namespace janus {
-janus_status rows_split_f16(const float* x, int64_t rows, int32_t d, uint16_t* rows16, float* row_scale,
-                            uint32_t* rowmax, cudaStream_t stream) {
-  if (rows == 0) return JANUS_OK;
-  JANUS_CUDA_TRY(cudaMemsetAsync(rowmax, 0, sizeof(uint32_t) * (size_t)rows, stream));
-  const unsigned grid = rows_grid(row_items(rows, d / 4), 8);
-  row_absmax_kernel<<<grid, kThreads, 0, stream>>>((const float4*)x, rows, d / 4, rowmax);
-  rows_split_kernel<<<grid, kThreads, 0, stream>>>((const float4*)x, rows, d / 4, rowmax, (uint2*)rows16, row_scale);
-  return launch_status();
-}
-}  // namespace janus
 
 extern "C" janus_status janus_dispatch_split_workspace_size(int64_t n_atoms, size_t* bytes) {
   JANUS_CHECK_ARG(bytes && n_atoms >= 0);

@@ -706,7 +706,8 @@ def janus_expert_ffn_split_workspace_size(n_rows, n_experts, d, h) -> int:
 def janus_expert_ffn_fwd_split(rows16, row_scale, offsets, w1, w2, *, out=None, out_rows=None, want_act=False,
                                act=None, workspace=None, stream=None):
     """The forward on split rows (janus_dispatch_split): the first GEMM on the
-    FP16 tensor path, the second on 3xTF32.  Returns (out-or-None, act-or-None)."""
+    FP16 tensor path, the second on 3xTF32, or on the FP16 path too at >= 2048
+    rows per expert with h % 8 == 0.  Returns (out-or-None, act-or-None)."""
     R2, d = rows16.shape
     R = R2 // 2
     E, _, h = w1.shape
@@ -732,7 +733,8 @@ def janus_expert_ffn_vjp_split(gd16, gd_scale, offsets, w1, w2, act, *, out=None
                                stream=None):
     """The input VJP on split upstream-gradient rows (janus_dispatch_split,
     weighted) and the forward's pre-activations: dA = (gd W2^T) silu'(a) on
-    the FP16 tensor path, dxd = dA W1^T on 3xTF32.  Returns out-or-None."""
+    the FP16 tensor path, dxd = dA W1^T on 3xTF32, or on the FP16 path too at
+    >= 2048 rows per expert with h % 8 == 0.  Returns out-or-None."""
     R2, d = gd16.shape
     R = R2 // 2
     E, _, h = w1.shape

@@ -93,15 +93,23 @@ class MoELayer:
         # when the rows per expert amortise the per-call weight split
         self.split = (mode == J.JANUS_FFN_3XTF32 and not packed and d % 8 == 0
                       and R >= self.SPLIT_MIN_ROWS_PER_EXPERT * E)
+        # the input VJP on the FP16 tensor path (both GEMMs; the weighted
+        # dispatch writes the gradient rows as two FP16 terms) on the same rule
+        self.split_vjp = (mode == J.JANUS_FFN_3XTF32 and d % 8 == 0 and h % 8 == 0
+                          and R >= self.SPLIT_MIN_ROWS_PER_EXPERT * E)
         nb = max(J.janus_expert_ffn_workspace_size(R, d, h, E, False, True, mode),
                  J.janus_expert_ffn_workspace_size(R, d, h, E, True, True, mode),
                  J.janus_expert_ffn_packed_workspace_size(R, E, d, h, mode) if self.fused_unpack else 0,
-                 J.janus_expert_ffn_split_workspace_size(R, E, d, h) if self.split else 0)
+                 J.janus_expert_ffn_split_workspace_size(R, E, d, h) if self.split or self.split_vjp else 0)
         self.ffn_ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        if self.split or self.split_vjp:
+            self.split_ws = torch.empty(J.janus_dispatch_split_workspace_size(N), dtype=torch.uint8, device=dev)
         if self.split:
             self.xd16 = torch.empty((2 * R, d), dtype=torch.float16, device=dev)
             self.xd_scale = torch.empty((R,), **f32)
-            self.split_ws = torch.empty(J.janus_dispatch_split_workspace_size(N), dtype=torch.uint8, device=dev)
+        if self.split_vjp:
+            self.gd16 = torch.empty((2 * R, d), dtype=torch.float16, device=dev)
+            self.gd_scale = torch.empty((R,), **f32)
         if row_ptr is not None:
             self.xagg = torch.empty((N, d), **f32)
         if packed:
@@ -126,7 +134,12 @@ class MoELayer:
         fp16_first = self.split or (self.packed and self.fused_unpack and mode == J.JANUS_FFN_3XTF32)
         self.f16_second = fp16_first and h % 8 == 0 and R >= 2048 * E
         if self.f16_second:
-            launches["ffn_fwd"] += 5          # row maxima + row split + 3 weight-split kernels
+            launches["ffn_fwd"] += 4          # H's row split + 3 weight-split kernels
+        if self.split_vjp:
+            # weighted split dispatch: row maxima + split; VJP: W2 split (3),
+            # gd W2^T, dA's row split, W1 split (3), dA W1^T
+            launches["dispatch_w"] = 2
+            launches["ffn_vjp"] = 9
         self.launches_per_call = sum(launches[o] for o in self.ops)
         self._host = None
 
@@ -195,12 +208,20 @@ class MoELayer:
         if after_forward is not None:
             after_forward()
         mark("dispatch_w", 0)
-        J.janus_dispatch(g, r["slot_of"], K, r["topk_weight"], out=self.gd)
+        if self.split_vjp:
+            J.janus_dispatch_split(g, r["slot_of"], K, r["topk_weight"], out=self.gd16, row_scale=self.gd_scale,
+                                   workspace=self.split_ws)
+        else:
+            J.janus_dispatch(g, r["slot_of"], K, r["topk_weight"], out=self.gd)
         mark("dispatch_w", 1)
         mark("ffn_vjp", 0)
-        # (xd is read only when the pre-activations are not saved; here they are)
-        J.janus_expert_ffn_vjp(self.xd, self.gd, r["offsets"], self.w1, self.w2, act=self.act,
-                               mode=self.mode, out=self.dxd, workspace=self.ffn_ws)
+        if self.split_vjp:
+            J.janus_expert_ffn_vjp_split(self.gd16, self.gd_scale, r["offsets"], self.w1, self.w2, self.act,
+                                         out=self.dxd, workspace=self.ffn_ws)
+        else:
+            # (xd is read only when the pre-activations are not saved; here they are)
+            J.janus_expert_ffn_vjp(self.xd, self.gd, r["offsets"], self.w1, self.w2, act=self.act,
+                                   mode=self.mode, out=self.dxd, workspace=self.ffn_ws)
         mark("ffn_vjp", 1)
         mark("combine_vjp", 0)
         J.janus_combine(self.dxd, r["slot_of"], K, out=dx)

@@ -345,10 +345,14 @@ janus_status janus_expert_ffn_vjp_rows(const float* xd, const float* gd, const f
  * output feature a power-of-two scale and two binary16 terms, as in
  * janus_expert_ffn_fwd_packed); products are exact and accumulate in FP32 in
  * chunks of 256, the result is scaled by row_scale[p] and the feature's
- * 1 / S.  The second GEMM runs on 3xTF32, or, in the forward with n_rows >=
- * 2048 * n_experts and h % 8 == 0, on the same kind::f16 path after H is
- * split into two FP16 terms per row in the workspace.  FP32-accurate as the
- * 3xTF32 forms (within 1e-5), at half their tensor-core work per FP16 GEMM.
+ * 1 / S.  The second GEMM (H W2, or dA W1^T) runs on 3xTF32, or, with
+ * n_rows >= 2048 * n_experts and h % 8 == 0, on the same kind::f16 path: the
+ * first GEMM then stores a (fwd) or dH = gd W2^T (vjp) plainly, and one pass
+ * over each row writes H = silu(a), or dA = dH * silu'(a), as two FP16 terms
+ * with a per-row power-of-two scale into the workspace, after which the
+ * weights of the second GEMM are split per output feature.  FP32-accurate as
+ * the 3xTF32 forms (within 1e-5), at half their tensor-core work per FP16
+ * GEMM.
  * fwd: rows16 = [hi | mid] of xd, act [R,h] nullable, yd or yd_rows (one).
  * vjp: gd16 = [hi | mid] of the gate-weighted upstream gradient rows, act
  *      = the forward's pre-activations (required), dxd or dxd_rows (one).

@@ -157,6 +157,47 @@ def test_split_forward_full_size_sampled_rows():
     assert torch.isfinite(yd).all().item() and torch.isfinite(dxd).all().item()
 
 
+def test_fp16_second_gemms_handle_wide_ranges():
+    # at >= 2048 rows per expert both second GEMMs run on FP16: H W2 with W2
+    # split per output feature d, dA W1^T with W1 split per output feature d
+    # (a row of W1[e]).  Output features whose weights are 10^6 or 10^-30
+    # times the rest, or all zero, stay within the FP32 tolerance column by
+    # column; so do rows of the upstream gradient 10^9 times the rest
+    counts, d, h = [2100, 0, 2200, 2000], 128, 96
+    E = len(counts)
+    offs = _offsets(counts)
+    R = int(offs[-1])
+    w1, w2 = synth.expert_weights(E, d, h, 15, DEV)
+    w2[:, :, 3] *= 1.0e6
+    w2[:, :, 5] = 0.0
+    w2[:, :, 9] *= 1.0e-30
+    w1[:, 7, :] *= 1.0e6
+    w1[:, 11, :] = 0.0
+    w1[:, 13, :] *= 1.0e-30
+    xd = synth.normal((R, d), 16, DEV)
+    gd = synth.normal((R, d), 17, DEV)
+    gd[40] *= 1.0e9
+    o = to_dev(offs)
+    x16, xs = _split_rows(xd)
+    g16, gs = _split_rows(gd)
+    nb = J.janus_expert_ffn_split_workspace_size(R, E, d, h)
+    ws = torch.zeros(nb, dtype=torch.uint8, device=DEV)
+    yd, act = J.janus_expert_ffn_fwd_split(x16, xs, o, w1, w2, want_act=True, workspace=ws)
+    J.janus_check(ws)
+    dxd = J.janus_expert_ffn_vjp_split(g16, gs, o, w1, w2, act, workspace=ws)
+    J.janus_check(ws)
+    hw1, hw2 = host(w1), host(w2)
+    ref_y = oracle.expert_ffn_fwd(host(xd), offs, hw1, hw2)
+    ref_dx = oracle.expert_ffn_vjp(host(xd), host(gd), offs, hw1, hw2)
+    hy, hdx = host(yd).astype(np.float64), host(dxd).astype(np.float64)
+    for got, ref, cols, zero in ((hy, ref_y, (0, 3, 9, 40), 5), (hdx, ref_dx, (0, 7, 13, 40), 11)):
+        for f in cols:
+            col, rc = got[:, f], ref[:, f].astype(np.float64)
+            assert np.linalg.norm(col - rc) <= TOL_FP32 * np.linalg.norm(rc), f
+        assert np.all(got[:, zero] == 0.0)
+    assert max_row_rel(host(dxd), ref_dx) <= TOL_ROW and max_row_rel(host(yd), ref_y) <= TOL_ROW
+
+
 def test_split_calls_check_their_arguments():
     E, d, h = 3, 12, 8                              # d % 8 != 0
     offs = to_dev(_offsets([10, 0, 6]))
