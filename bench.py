@@ -431,6 +431,30 @@ def run_reference(args, world, rank):
 # --------------------------------------------------------------------------
 # janus arm
 # --------------------------------------------------------------------------
+TRACE_PER_STEP = 32     # traced launches per layer pass: 4 GEMMs + up to 6 splits, with room
+
+
+def trace_kind(name):
+    """(operand kind, products) from a GEMM's trace name, e.g. 'tc_gemm x.W
+    store f16x3' -> ('f16', 3)."""
+    ops = name.split()[-1]
+    return ("f16" if ops.startswith("f16") else "tf32"), int(ops[-1])
+
+
+def split_bytes(cfg, layer):
+    """Algorithmic bytes of one launch of each traced split kind: the
+    activation split reads a (and dH for dSiLU) once and writes the two FP16
+    planes and a scale per row; the weight split reads one expert matrix and
+    writes its two FP16 planes and a scale per output feature."""
+    R, d, h, E = cfg.n_rows, cfg.d, cfg.h, cfg.n_experts
+    return {
+        "act_split silu": 4 * R * h + 4 * R * h + 4 * R,
+        "act_split dsilu": 8 * R * h + 4 * R * h + 4 * R,
+        "w16_split transposed": 4 * E * d * h + 4 * E * d * h + 4 * E * max(d, h),
+        "w16_split rows": 4 * E * d * h + 4 * E * d * h + 4 * E * max(d, h),
+    }
+
+
 def gemm_roofline(J, mode, cfg, kinds, peaks, peak_src, flops_per_gemm, ms_total, launches):
     """Roofline of the grouped expert-MLP GEMM over a step's launches.
 
@@ -494,6 +518,10 @@ def run_janus(args, world, rank, local):
     time.sleep(0.1)
     barrier(world)
     torch.cuda.synchronize()
+    # the library's launch trace brackets each expert-MLP GEMM (and the
+    # weight / activation splits around them) with CUDA events on the
+    # launching stream, so the GEMM roofline uses the kernels' own durations
+    J.janus_trace_start(args.steps * TRACE_PER_STEP)
     wall0 = time.time()
     t_start.record()
     for k in range(args.steps):
@@ -502,6 +530,9 @@ def run_janus(args, world, rank, local):
     sampler.sample_now()        # while the enqueued steps run
     torch.cuda.synchronize()
     wall1 = time.time()
+    J.janus_trace_stop()
+    trace = J.janus_trace_records()
+    J.janus_trace_release()
     clocks = sampler.stop(wall0, wall1)
     barrier(world)
     elapsed = t_start.elapsed_time(t_end) / 1e3
@@ -520,17 +551,38 @@ def run_janus(args, world, rank, local):
     kernels["route"] = {"ms": op_ms["route"]}
 
     # roofline of the dominant kernel: the grouped expert-MLP GEMM (4 launches
-    # per step: two forward, two VJP, each 2*R*d*h FLOPs), timed by CUDA
-    # events on the launching stream inside the timed steps
+    # per step: two forward, two VJP, each 2*R*d*h FLOPs), each launch timed
+    # by the library's trace events on the launching stream inside the timed
+    # steps (the SIMT path is not traced: there the FFN calls' events)
     ffn_ms = op_ms["ffn_fwd"] + op_ms["ffn_vjp"]
-    core = layer.core
-    if core.packed:
-        first = ("f16", 2) if core.fused_unpack else ("tf32", 2)
+    flops_per_gemm = work["ffn_fwd"][1] / 2
+    gemms = [(n, ms) for n, ms in trace if n.startswith("tc_gemm")]
+    if mode == J.JANUS_FFN_3XTF32 and len(gemms) == 4 * args.steps:
+        kinds = [trace_kind(n) for n, _ in gemms[:4]]
+        gemm_ms = sum(ms for _, ms in gemms) / args.steps
+        roof = gemm_roofline(J, mode, cfg, kinds, peaks, peak_src, flops_per_gemm, gemm_ms, 4)
+        per_launch = []
+        for j in range(4):
+            ms_j = float(np.mean([gemms[4 * k + j][1] for k in range(args.steps)]))
+            tf = flops_per_gemm / (ms_j * 1e-3) / 1e12
+            per_launch.append({"kernel": gemms[j][0], "ms": ms_j, "TFLOP/s": tf,
+                               "frac": tf / roof["peak_per_gemm"][j]})
+        roof["per_launch"] = per_launch
+        roof["timing"] = "library trace events around each GEMM launch, mean over the timed steps"
+        roof["ffn_calls_ms"] = ffn_ms      # the MLP calls with their weight and activation splits
     else:
-        first = ("f16", 3) if core.split else ("tf32", 3)
-    vjp = [("f16", 3)] * 2 if core.split_vjp else [("tf32", 3)] * 2
-    kinds = [first, ("f16", 3) if core.f16_second else ("tf32", 3)] + vjp
-    roof = gemm_roofline(J, mode, cfg, kinds, peaks, peak_src, work["ffn_fwd"][1] / 2, ffn_ms, 4)
+        kinds = [("tf32", 3)] * 4
+        roof = gemm_roofline(J, mode, cfg, kinds, peaks, peak_src, flops_per_gemm, ffn_ms, 4)
+        roof["timing"] = "CUDA events around the expert-MLP calls"
+    # the splits around the FP16 GEMMs: memory-bound, from the same trace
+    for name, nbytes in split_bytes(cfg, layer).items():
+        rec = [ms for n, ms in trace if n == name]
+        if rec:
+            ms = float(np.sum(rec)) / args.steps
+            per = len(rec) // args.steps
+            gbs = nbytes * per / (ms * 1e-3) / 1e9
+            kernels[name] = {"ms": ms, "launches_per_step": per, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                             "algorithmic_bytes": nbytes * per}
     roof["traffic"] = measured_traffic(cfg.name, args.mode) if cfg == synth.CONFIGS[cfg.name] else None
     roof["traffic_unit"] = "DRAM bytes per launch (mean of the step's 4 launches)"
     ws_gb = ((layer.w1.numel() + layer.w2.numel()) * 4 + cfg.n_rows * cfg.d * 4 * 4) / 1e9

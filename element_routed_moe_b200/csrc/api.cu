@@ -1,9 +1,11 @@
 // Library-wide entry points: status strings, version, janus_check, the debug
-// build's fault word (janus_debug_build, janus_debug_check), and the host-side
-// launch-failure injection used by the tests.
+// build's fault word (janus_debug_build, janus_debug_check), the launch trace
+// (janus_trace_*), and the host-side launch-failure injection used by the
+// tests.
 #include <atomic>
 #include <mutex>
 #include <unordered_map>
+#include <vector>
 
 #include "common.cuh"
 
@@ -50,9 +52,98 @@ int32_t* debug_fault_word() {
 int32_t* debug_fault_word() { return nullptr; }
 #endif
 
+// ---- launch trace -------------------------------------------------------
+// Records of (kernel name, start event, end event), events created when the
+// trace starts (never inside a traced region); a launch past the capacity is
+// not recorded.
+namespace {
+struct TraceRec {
+  const char* name;
+  cudaEvent_t beg, end;
+};
+std::mutex g_trace_mu;
+std::vector<TraceRec> g_trace;
+int g_trace_used = 0;
+std::atomic<bool> g_trace_on{false};
+
+void trace_release() {
+  for (TraceRec& r : g_trace) {
+    cudaEventDestroy(r.beg);
+    cudaEventDestroy(r.end);
+  }
+  g_trace.clear();
+  g_trace_used = 0;
+}
+}  // namespace
+
+bool trace_on() { return g_trace_on.load(std::memory_order_relaxed); }
+
+int trace_begin(const char* name, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(g_trace_mu);
+  if (!g_trace_on.load() || g_trace_used >= (int)g_trace.size()) return -1;
+  const int slot = g_trace_used++;
+  g_trace[slot].name = name;
+  cudaEventRecord(g_trace[slot].beg, stream);
+  return slot;
+}
+
+void trace_end(int slot, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(g_trace_mu);
+  if (slot >= 0 && slot < (int)g_trace.size()) cudaEventRecord(g_trace[slot].end, stream);
+}
+
 }  // namespace janus
 
 extern "C" {
+
+janus_status janus_trace_start(int32_t capacity) {
+  JANUS_CHECK_ARG(capacity >= 1 && capacity <= (1 << 20));
+  std::lock_guard<std::mutex> lock(janus::g_trace_mu);
+  janus::g_trace_on.store(false);
+  janus::trace_release();
+  janus::g_trace.reserve((size_t)capacity);
+  for (int i = 0; i < capacity; ++i) {
+    janus::TraceRec r{nullptr, nullptr, nullptr};
+    if (cudaEventCreate(&r.beg) != cudaSuccess) return JANUS_ERR_CUDA;
+    if (cudaEventCreate(&r.end) != cudaSuccess) {
+      cudaEventDestroy(r.beg);
+      return JANUS_ERR_CUDA;
+    }
+    janus::g_trace.push_back(r);
+  }
+  janus::g_trace_on.store(true);
+  return JANUS_OK;
+}
+
+janus_status janus_trace_stop(void) {
+  janus::g_trace_on.store(false);
+  return JANUS_OK;
+}
+
+janus_status janus_trace_count(int32_t* n) {
+  JANUS_CHECK_ARG(n);
+  std::lock_guard<std::mutex> lock(janus::g_trace_mu);
+  *n = janus::g_trace_used;
+  return JANUS_OK;
+}
+
+janus_status janus_trace_get(int32_t i, const char** name, float* ms) {
+  JANUS_CHECK_ARG(name && ms);
+  std::lock_guard<std::mutex> lock(janus::g_trace_mu);
+  JANUS_CHECK_ARG(i >= 0 && i < janus::g_trace_used);
+  const janus::TraceRec& r = janus::g_trace[i];
+  if (cudaEventSynchronize(r.end) != cudaSuccess) return JANUS_ERR_CUDA;
+  if (cudaEventElapsedTime(ms, r.beg, r.end) != cudaSuccess) return JANUS_ERR_CUDA;
+  *name = r.name;
+  return JANUS_OK;
+}
+
+janus_status janus_trace_release(void) {
+  std::lock_guard<std::mutex> lock(janus::g_trace_mu);
+  janus::g_trace_on.store(false);
+  janus::trace_release();
+  return JANUS_OK;
+}
 
 const char* janus_status_string(janus_status s) {
   switch (s) {

@@ -55,6 +55,21 @@ bool consume_injected_failure();
 // Number of SMs of the current device.
 int num_sms();
 
+// Launch trace (janus_trace_*): while it records, a traced launch is
+// bracketed by two CUDA events on its stream.  trace_begin returns the record's
+// slot, or -1 when the trace is off or full.
+bool trace_on();
+int trace_begin(const char* name, cudaStream_t stream);
+void trace_end(int slot, cudaStream_t stream);
+struct TraceScope {
+  int slot;
+  cudaStream_t stream;
+  TraceScope(const char* name, cudaStream_t s) : slot(trace_on() ? trace_begin(name, s) : -1), stream(s) {}
+  ~TraceScope() {
+    if (slot >= 0) trace_end(slot, stream);
+  }
+};
+
 inline janus_status launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? JANUS_OK : JANUS_ERR_CUDA;

@@ -63,6 +63,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <string>
 
 #include "ffn_tc.cuh"
 
@@ -267,24 +268,65 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
       ::"r"(smem_u32(bar)), "h"((uint16_t)0x3)
       : "memory");
 }
+// A-operand collector use of an MMA: kCollNone reads A from shared memory;
+// kCollFill reads it and keeps it in the tensor core's A collector;
+// kCollLast takes A from the collector (filled by the MMA just before, with
+// the same A descriptor) instead of shared memory, and releases it.  Two
+// consecutive products with the same A (hi_w x hi_x, hi_w x lo_x) then fetch
+// the weights' tile once, which matters where operand fetch, not the MMA
+// rate, bounds a tile (few dispatch rows).
+enum Collector : int { kCollNone = 0, kCollFill = 1, kCollLast = 2 };
+
+template <int kColl = kCollNone>
 __device__ __forceinline__ void tc_mma_tf32_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                                  uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n"
-      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
+  if (kColl == kCollFill)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::tf32.collector::a::fill [%0], %1, %2, %3, p;\n\t}\n"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else if (kColl == kCollLast)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::tf32.collector::a::lastuse [%0], %1, %2, %3, p;\n\t}\n"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
+template <int kColl = kCollNone>
 __device__ __forceinline__ void tc_mma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                                 uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
-      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
+  if (kColl == kCollFill)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16.collector::a::fill [%0], %1, %2, %3, p;\n\t}\n"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else if (kColl == kCollLast)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16.collector::a::lastuse [%0], %1, %2, %3, p;\n\t}\n"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 // Shared-memory matrix descriptor (tcgen05): start address, leading and
@@ -445,10 +487,23 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
     float acc[kEpiCols];
 #pragma unroll
     for (int j = 0; j < kEpiCols; ++j) acc[j] = 0.f;     // a tile with no k-blocks stores zeros
+    // FP16 path: this half-tile's 128 row scales, four per lane, loaded while
+    // the tile accumulates; the store phase takes column j's from lane j % 32
+    // by a shuffle instead of a load per column (the dSiLU store phase, short
+    // of registers for them, loads each column's)
+    constexpr bool kShflScale = f16_path<kBK>() && kMode != kModeTN && kEpi != kEpiDSilu;
+    float rsr[kEpiCols / 32];
+#pragma unroll
+    for (int u = 0; u < kEpiCols / 32; ++u) {
+      const int col = (wg - 1) * kEpiCols + u * 32 + lane;
+      rsr[u] = (kShflScale && col < c.n_valid) ? __ldg(args.row_scale + c.n0 + col) : 0.f;
+    }
     bool ok = true;
     for (int c0 = 0; c0 < c.nk; c0 += kChunk, ++ch) {
       const uint32_t p = ch & 1, cuse = ch >> 1;
-      if (!mbar_wait(s, &s->chunk_full[p], cuse & 1, args.err)) { ok = false; break; }
+      // the warp leaves together (a timeout seen by one lane ends the tile for
+      // all 32: the TMEM loads and the row-scale shuffles are warp-wide)
+      if (!__all_sync(0xffffffffu, mbar_wait(s, &s->chunk_full[p], cuse & 1, args.err))) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr = tmem_base + lane_addr + p * BN + half * kEpiCols;
 #pragma unroll
@@ -489,11 +544,14 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
         if (f < c.m_end) d2_store(args, acc, c, j0, f, N);
         continue;
       }
-      if (f < c.m_end) {
+      // with the row-scale shuffles every lane runs the loop (they need the
+      // whole warp); lanes past the tile's last feature store nothing
+      const bool f_ok = f < c.m_end;
+      if (kShflScale || f_ok) {
         // FP16 path: the product is q (hi + mid) S (kBF16S: q = the row's
         // two terms); scale column j by its row's s_p and this lane's feature
         // by 1 / S (powers of two: exact)
-        const float cscale = f16_path<kBK>() ? __ldg(args.col_scale + (int64_t)c.e * N + f) : 1.0f;
+        const float cscale = (f16_path<kBK>() && f_ok) ? __ldg(args.col_scale + (int64_t)c.e * N + f) : 1.0f;
         // batches of 8 columns; the pre-activations of batch b + 1 are in
         // flight while batch b is finished, so two loads per column overlap
         constexpr int kB = 8;
@@ -501,21 +559,23 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
         float a_cur[kB], a_nxt[kB];
         if (kEpi == kEpiDSilu) {
 #pragma unroll
-          for (int j = 0; j < kB; ++j) a_cur[j] = (j0 + j < c.n_valid) ? __ldg(arow + (int64_t)j * N) : 0.f;
+          for (int j = 0; j < kB; ++j) a_cur[j] = (f_ok && j0 + j < c.n_valid) ? __ldg(arow + (int64_t)j * N) : 0.f;
         }
 #pragma unroll
         for (int jb = 0; jb < kEpiCols; jb += kB) {
           if (kEpi == kEpiDSilu && jb + kB < kEpiCols) {
 #pragma unroll
             for (int j = 0; j < kB; ++j)
-              a_nxt[j] = (j0 + jb + kB + j < c.n_valid) ? __ldg(arow + (int64_t)(jb + kB + j) * N) : 0.f;
+              a_nxt[j] = (f_ok && j0 + jb + kB + j < c.n_valid) ? __ldg(arow + (int64_t)(jb + kB + j) * N) : 0.f;
           }
 #pragma unroll
           for (int j = 0; j < kB; ++j) {
-            if (j0 + jb + j < c.n_valid) {
+            const float rs = kShflScale ? __shfl_sync(0xffffffffu, rsr[(jb + j) / 32], (jb + j) % 32) : 1.0f;
+            if (f_ok && j0 + jb + j < c.n_valid) {
               const int64_t o = (int64_t)(c.n0 + j0 + jb + j) * N + f;
               float v = acc[jb + j];
-              if (f16_path<kBK>()) v = v * __ldg(args.row_scale + c.n0 + j0 + jb + j) * cscale;
+              if (kShflScale) v = v * rs * cscale;
+              else if (f16_path<kBK>()) v = v * __ldg(args.row_scale + c.n0 + j0 + jb + j) * cscale;
               if (kEpi == kEpiStore && args.c_rows) {   // the row's own destination
                 args.c_rows[c.n0 + j0 + jb + j][f] = v;
                 continue;
@@ -716,6 +776,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           const int tnk = tc.nk;
           const uint32_t idesc = f16_path<kBK>() ? instr_desc_f16((uint32_t)tc.n_mma)
                                                  : instr_desc(kAMN, kBMN, (uint32_t)tc.n_mma);
+
           for (int c0 = 0; c0 < tnk && ok; c0 += kChunk, ++ch) {
             const uint32_t p = ch & 1, cuse = ch >> 1;
             if (!mbar_wait(s, &s->chunk_empty[p], (cuse & 1) ^ 1, args.err)) { ok = false; break; }
@@ -735,9 +796,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                 for (int kk = 0; kk < BK16 / 16; ++kk) {
                   const uint64_t ad = smem_desc(a16 + kk * 32, 16, 1024, kSwizzle128B);
                   const uint64_t bd = smem_desc(b16 + kk * 32, 16, 1024, kSwizzle128B);
-                  tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb > c0 || kk > 0) ? 1u : 0u);
-                  if (kBK == kBF16S)
-                    tc_mma_f16_pair(d_tmem, ad, smem_desc(bm16 + kk * 32, 16, 1024, kSwizzle128B), idesc, 1u);
+                  if (kBK == kBF16S) {
+                    // hi_w x hi_x and hi_w x mid_x share A: one fetch of hi_w
+                    tc_mma_f16_pair<kCollFill>(d_tmem, ad, bd, idesc, (kb > c0 || kk > 0) ? 1u : 0u);
+                    tc_mma_f16_pair<kCollLast>(d_tmem, ad, smem_desc(bm16 + kk * 32, 16, 1024, kSwizzle128B), idesc,
+                                               1u);
+                  } else {
+                    tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb > c0 || kk > 0) ? 1u : 0u);
+                  }
                   tc_mma_f16_pair(d_tmem, smem_desc(m16 + kk * 32, 16, 1024, kSwizzle128B), bd, idesc, 1u);
                 }
                 tc_commit_pair(&s->empty[st]);
@@ -767,8 +833,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                   bdl = smem_desc(b_lo + kk * 32, 16, 512, kSwizzle64B);
                 }
                 tc_mma_tf32_pair(d_tmem, adl, bdh, idesc, (kb > c0 || kk > 0) ? 1u : 0u);
-                if (kBK == kBSplit) tc_mma_tf32_pair(d_tmem, adh, bdl, idesc, 1u);   // B's residual is zero otherwise
-                tc_mma_tf32_pair(d_tmem, adh, bdh, idesc, 1u);
+                if (kBK == kBSplit) {
+                  // hi_a x lo_b and hi_a x hi_b share A: one fetch of hi_a
+                  // (a runtime choice per tile here cost 30 % on small
+                  // experts: the collector is used on every tile)
+                  tc_mma_tf32_pair<kCollFill>(d_tmem, adh, bdl, idesc, 1u);
+                  tc_mma_tf32_pair<kCollLast>(d_tmem, adh, bdh, idesc, 1u);
+                } else {
+                  tc_mma_tf32_pair(d_tmem, adh, bdh, idesc, 1u);   // B's residual is zero
+                }
               }
               tc_commit_pair(&s->empty[st]);
             }
@@ -973,6 +1046,21 @@ constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Smem
 // kModeNN/NT: C [R,N] = A [R,Kd] x W_e;  kModeTN: C [E,N,M] with C_e = W_e^T A_e
 // (the product A_e^T W_e stored transposed) over expert e's rows of A [R,M] and
 // W [R,N] (Kd unused).
+// Launch-trace name of a GEMM variant: "tc_gemm <product> <epilogue> <operands>",
+// products x.W / x.Wt / Xt.Y, operands tf32x3 (FP32 rows split in the
+// kernel), tf32x2 (rows exact in TF32), f16x2 (FP16 payload), f16x3 (two-term
+// FP16 rows).
+template <int kMode, int kEpi, int kBK>
+const char* gemm_trace_name() {
+  static const std::string name = [] {
+    static const char* modes[] = {"x.W", "x.Wt", "Xt.Y"};
+    static const char* epis[] = {"store", "silu", "dsilu", "d2", "accum"};
+    const char* ops = kBK == kBSplit ? "tf32x3" : kBK == kBExact ? "tf32x2" : kBK == kBF16W ? "f16x2" : "f16x3";
+    return std::string("tc_gemm ") + modes[kMode] + " " + epis[kEpi] + " " + ops;
+  }();
+  return name.c_str();
+}
+
 template <int kMode, int kEpi, int kBK = kBSplit>
 janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, int N, float* C, float* C2,
                     const float* aux, const int32_t* offsets, int32_t* err, cudaStream_t stream, int M = 0,
@@ -1017,6 +1105,7 @@ janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, in
   cluster_attr[0].val.clusterDim.z = 1;
   cfg.attrs = cluster_attr;
   cfg.numAttrs = 1;
+  TraceScope trace(gemm_trace_name<kMode, kEpi, kBK>(), stream);
   if (cudaLaunchKernelEx(&cfg, tc_gemm_kernel<kMode, kEpi, kBK>, ma, mb, a) != cudaSuccess)
     return JANUS_ERR_CUDA;
   return launch_status();
@@ -1030,8 +1119,14 @@ janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, in
 // so that magnitude times S lies in [2^14, 2^15) (below FP16's 65504); S is
 // clamped to [2^-126, 2^126] and is 1 for an all-zero column.  hi = fp16(w S)
 // and mid = fp16(w S - hi): w S - hi is exact in FP32 and the pair carries
-// 22 bits of w S.  Three passes: column maxima (as bits, into winv), the split
-// with the transpose through shared memory, maxima -> 1 / S.
+// 22 bits of w S.  x W: column maxima, the split with the transpose through
+// shared memory, maxima -> 1 / S; x W^T: one pass over each row.  N % 4 == 0
+// and Kd % 4 == 0 (JANUS_ERR_MISALIGNED otherwise).
+
+__device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
 
 __device__ __forceinline__ int w16_scale_exp(uint32_t max_bits) {
   if (max_bits == 0) return 0;
@@ -1039,6 +1134,8 @@ __device__ __forceinline__ int w16_scale_exp(uint32_t max_bits) {
   return min(max(141 - b, -126), 126);
 }
 
+// x W, three kernels: the column maxima (as ordered bits, into winv), the
+// split, and the maxima turned into 1 / S in place.
 __global__ void __launch_bounds__(256) w16_colmax_kernel(const float* __restrict__ w, int Kd, int N, int k_per,
                                                          uint32_t* __restrict__ colmax) {
   const int e = blockIdx.z, f = blockIdx.x * 256 + threadIdx.x, k0 = blockIdx.y * k_per;
@@ -1050,72 +1147,71 @@ __global__ void __launch_bounds__(256) w16_colmax_kernel(const float* __restrict
   if (m) atomicMax(colmax + (int64_t)e * N + f, m);
 }
 
-// tile: 32 features x 64 k of expert e; reads are 128-byte rows of W[e]
-// ([Kd][N], features contiguous), writes 128-byte rows of the K-major split
-// (two consecutive k per lane)
-__global__ void __launch_bounds__(256) w16_split_kernel(const float* __restrict__ w, int E, int Kd, int N,
-                                                        const uint32_t* __restrict__ colmax, __half* __restrict__ w16) {
-  __shared__ __half t_hi[32][66], t_mid[32][66];     // [feature][k] of a 32 x 64 tile
-  const int e = blockIdx.z, f0 = blockIdx.x * 32, k0 = blockIdx.y * 64;
-  const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;
-  const int f = f0 + tx;
-  const float S = f < N ? __uint_as_float((uint32_t)(127 + w16_scale_exp(colmax[(int64_t)e * N + f])) << 23) : 1.0f;
-#pragma unroll
-  for (int j = ty; j < 64; j += 8) {
-    const int k = k0 + j;
-    const float v = (f < N && k < Kd) ? __ldcs(w + ((int64_t)e * Kd + k) * N + f) * S : 0.0f;
-    const __half hi = __float2half_rn(v);
-    t_hi[tx][j] = hi;
-    t_mid[tx][j] = __float2half_rn(v - __half2float(hi));
-  }
-  __syncthreads();
-  const int64_t plane = (int64_t)E * N * Kd;        // mid follows hi
-#pragma unroll
-  for (int j = ty; j < 32; j += 8) {
-    const int fo = f0 + j, ko = k0 + 2 * tx;
-    if (fo >= N) continue;
-    const int64_t o = ((int64_t)e * N + fo) * Kd + ko;
-    if (ko + 1 < Kd && (o % 2) == 0) {
-      *reinterpret_cast<__half2*>(w16 + o) = __halves2half2(t_hi[j][2 * tx], t_hi[j][2 * tx + 1]);
-      *reinterpret_cast<__half2*>(w16 + plane + o) = __halves2half2(t_mid[j][2 * tx], t_mid[j][2 * tx + 1]);
-    } else {
-      for (int q = 0; q < 2; ++q)
-        if (ko + q < Kd) {
-          w16[o + q] = t_hi[j][2 * tx + q];
-          w16[plane + o + q] = t_mid[j][2 * tx + q];
-        }
-    }
-  }
-}
-
-// x W^T: output feature n is row n of W[e] ([N][Kd], K contiguous): one warp
-// per row for its maximum, then an elementwise split in place (no transpose).
-__global__ void __launch_bounds__(256) w16_rowmax_kernel(const float* __restrict__ w, int64_t rows, int Kd,
-                                                         uint32_t* __restrict__ rowmax) {
-  const int lane = threadIdx.x % 32;
-  for (int64_t r = ((int64_t)blockIdx.x * 256 + threadIdx.x) / 32; r < rows; r += (int64_t)gridDim.x * 8) {
-    const float* p = w + r * Kd;
-    uint32_t m = 0;
-    for (int k = lane; k < Kd; k += 32) m = max(m, __float_as_uint(__ldcs(p + k)) & 0x7fffffffu);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) rowmax[r] = m;
-  }
-}
-
-__global__ void __launch_bounds__(256) w16_split_rows_kernel(const float* __restrict__ w, int64_t rows, int Kd,
-                                                             const uint32_t* __restrict__ rowmax,
+// The split, over tiles of 32 features x 128 k of one expert (grid-stride):
+// each thread loads four float4 (128-byte row segments of W[e], [Kd][N]),
+// scales and splits them, the tile goes through shared memory, and each warp
+// writes four features' 128 k as half2 pairs into the K-major planes.  Many
+// blocks per SM keep enough loads in flight.  N % 4 == 0, Kd % 2 == 0.
+constexpr int kColTileK = 128;
+__global__ void __launch_bounds__(256) w16_split_tile_kernel(const float* __restrict__ w, int E, int Kd, int N,
+                                                             const uint32_t* __restrict__ colmax,
                                                              __half* __restrict__ w16) {
-  const int64_t n = rows * Kd;
-  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    const float S = __uint_as_float((uint32_t)(127 + w16_scale_exp(rowmax[r])) << 23);
-    for (int k = threadIdx.x; k < Kd; k += 256) {
-      const int64_t i = r * Kd + k;
-      const float v = __ldcs(w + i) * S;
-      const __half hi = __float2half_rn(v);
-      w16[i] = hi;
-      w16[n + i] = __float2half_rn(v - __half2float(hi));
+  __shared__ __align__(16) __half t_hi[32][kColTileK + 2];
+  __shared__ __align__(16) __half t_mid[32][kColTileK + 2];
+  const int tid = threadIdx.x, tx = tid % 8, ty = tid / 8;
+  const int warp = tid / 32, lane = tid % 32;
+  const int strips_n = (N + 31) / 32, ktiles = (Kd + kColTileK - 1) / kColTileK;
+  const int64_t n_tiles = (int64_t)E * strips_n * ktiles;
+  const int64_t plane = (int64_t)E * N * Kd;                 // mid follows hi
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    const int kt = (int)(t % ktiles);
+    const int64_t es = t / ktiles;
+    const int e = (int)(es / strips_n), f0 = (int)(es % strips_n) * 32, k0 = kt * kColTileK;
+    const float* we = w + (int64_t)e * Kd * N;
+    const int fc = f0 + 4 * tx;
+    const bool col_ok = fc < N;                              // N % 4 == 0: all four columns
+    float sc[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      sc[j] = col_ok ? __uint_as_float((uint32_t)(127 + w16_scale_exp(__ldg(colmax + (int64_t)e * N + fc + j))) << 23)
+                     : 0.f;
+    float4 v[kColTileK / 32];
+#pragma unroll
+    for (int u = 0; u < kColTileK / 32; ++u) {
+      const int k = k0 + ty + 32 * u;
+      v[u] = (col_ok && k < Kd) ? __ldcs(reinterpret_cast<const float4*>(we + (int64_t)k * N + fc)) : zero;
     }
+#pragma unroll
+    for (int u = 0; u < kColTileK / 32; ++u) {
+      const int kr = ty + 32 * u;
+      const float val[4] = {v[u].x * sc[0], v[u].y * sc[1], v[u].z * sc[2], v[u].w * sc[3]};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __half hi = __float2half_rn(val[j]);
+        t_hi[4 * tx + j][kr] = hi;
+        t_mid[4 * tx + j][kr] = __float2half_rn(val[j] - __half2float(hi));
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int fl = warp * 4 + j, fo = f0 + fl;
+      if (fo >= N) continue;
+      const int64_t row = ((int64_t)e * N + fo) * Kd;
+#pragma unroll
+      for (int q = 0; q < kColTileK / 64; ++q) {
+        const int kk = 2 * (lane + 32 * q), ko = k0 + kk;
+        if (ko + 1 < Kd) {
+          __stcs(reinterpret_cast<__half2*>(w16 + row + ko), *reinterpret_cast<const __half2*>(&t_hi[fl][kk]));
+          __stcs(reinterpret_cast<__half2*>(w16 + plane + row + ko), *reinterpret_cast<const __half2*>(&t_mid[fl][kk]));
+        } else if (ko < Kd) {
+          w16[row + ko] = t_hi[fl][kk];
+          w16[plane + row + ko] = t_mid[fl][kk];
+        }
+      }
+    }
+    __syncthreads();
   }
 }
 
@@ -1126,19 +1222,23 @@ __global__ void __launch_bounds__(256) w16_inv_scale_kernel(uint32_t* __restrict
 
 // ---- the FP16 row split of an activation for a kind::f16 GEMM ---------------
 // v = silu(a) (kActSilu) or x silu'(a) (kActDSilu), with the SiLU arithmetic
-// of the GEMM epilogues, written as hi and mid binary16 planes ([rows][n]
-// each) with one power-of-two scale per row: S_p puts the row's largest |v|
-// in [2^14, 2^15), hi = fp16(v S_p), mid = fp16(v S_p - hi), row_scale[p] =
-// 1 / S_p.  One warp per row: a first sweep takes the row's maximum, a second
-// recomputes v and writes the two terms; the second sweep's loads find the
-// row in L1 / L2, so the activations are read from DRAM once and the FP32 v
-// is never stored.
-enum ActOp { kActSilu = 1, kActDSilu = 2 };
+// of the GEMM epilogues, or v = a (kActPlain: the rows of a K-major weight
+// matrix, one per output feature), written as hi and mid binary16 planes
+// ([rows][n] each) with one power-of-two scale per row: S_p puts the row's
+// largest |v| in [2^14, 2^15), hi = fp16(v S_p), mid = fp16(v S_p - hi),
+// row_scale[p] = 1 / S_p.  Rows up to 4096 values stay in the registers of a
+// 128-thread block (act_split_blk_kernel); longer ones take one warp and two
+// sweeps, the first for the row's maximum, the second recomputing v and
+// writing the two terms with loads that find the row in L1 / L2
+// (act_split_kernel).  Either way the inputs are read from DRAM once and the
+// FP32 v is never stored.
+enum ActOp { kActPlain = 0, kActSilu = 1, kActDSilu = 2 };
 constexpr int kActU = 4;       // float4 columns per lane in flight per sweep step
 
 template <int kOp, bool kLast>
 __device__ __forceinline__ float4 act_value(const float4* __restrict__ x, const float4* __restrict__ a, int64_t i) {
   const float4 av = kLast ? __ldcs(a + i) : __ldg(a + i);
+  if (kOp == kActPlain) return av;
   if (kOp == kActSilu) return make_float4(silu_f(av.x), silu_f(av.y), silu_f(av.z), silu_f(av.w));
   const float4 xv = kLast ? __ldcs(x + i) : __ldg(x + i);
   float4 v;
@@ -1148,11 +1248,6 @@ __device__ __forceinline__ float4 act_value(const float4* __restrict__ x, const 
   sg = sigmoid_fast(av.z); v.z = xv.z * (sg * (1.0f + av.z * (1.0f - sg)));
   sg = sigmoid_fast(av.w); v.w = xv.w * (sg * (1.0f + av.w * (1.0f - sg)));
   return v;
-}
-
-__device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 template <int kOp>
@@ -1200,37 +1295,152 @@ act_split_kernel(const float4* __restrict__ x, const float4* __restrict__ a, int
   }
 }
 
+// Rows of at most 128 * kNU float4 (n <= 4096): a block of 128 threads per
+// row keeps it in registers, kNU float4 per thread (a and, for dSiLU, dH all
+// in flight at once), so each value is read once and the two terms are
+// written from registers; the row maximum goes through shared memory (two
+// slots by row parity, so one barrier per row suffices).
+constexpr int kActBlk = 128;
+template <int kOp, int kNU>
+__global__ void __launch_bounds__(kActBlk)
+act_split_blk_kernel(const float4* __restrict__ x, const float4* __restrict__ a, int64_t rows, int n4,
+                     uint2* __restrict__ rows16, float* __restrict__ row_scale) {
+  __shared__ uint32_t red[2][kActBlk / 32];
+  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  uint2* __restrict__ mid = rows16 + rows * n4;
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  int parity = 0;
+  for (int64_t p = blockIdx.x; p < rows; p += gridDim.x, parity ^= 1) {
+    const int64_t base = p * n4;
+    float4 v[kNU];
+#pragma unroll
+    for (int u = 0; u < kNU; ++u) {
+      const int c = u * kActBlk + tid;
+      v[u] = c < n4 ? __ldcs(a + base + c) : zero;
+    }
+    if (kOp == kActDSilu) {
+      float4 g[kNU];
+#pragma unroll
+      for (int u = 0; u < kNU; ++u) {
+        const int c = u * kActBlk + tid;
+        g[u] = c < n4 ? __ldcs(x + base + c) : zero;
+      }
+#pragma unroll
+      for (int u = 0; u < kNU; ++u) {
+        float sg;
+        sg = sigmoid_fast(v[u].x); v[u].x = g[u].x * (sg * (1.0f + v[u].x * (1.0f - sg)));
+        sg = sigmoid_fast(v[u].y); v[u].y = g[u].y * (sg * (1.0f + v[u].y * (1.0f - sg)));
+        sg = sigmoid_fast(v[u].z); v[u].z = g[u].z * (sg * (1.0f + v[u].z * (1.0f - sg)));
+        sg = sigmoid_fast(v[u].w); v[u].w = g[u].w * (sg * (1.0f + v[u].w * (1.0f - sg)));
+      }
+    } else if (kOp == kActSilu) {
+#pragma unroll
+      for (int u = 0; u < kNU; ++u) v[u] = make_float4(silu_f(v[u].x), silu_f(v[u].y), silu_f(v[u].z), silu_f(v[u].w));
+    }
+    uint32_t m = 0;
+#pragma unroll
+    for (int u = 0; u < kNU; ++u)
+      m = max(m, max(max(__float_as_uint(v[u].x) & 0x7fffffffu, __float_as_uint(v[u].y) & 0x7fffffffu),
+                     max(__float_as_uint(v[u].z) & 0x7fffffffu, __float_as_uint(v[u].w) & 0x7fffffffu)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) red[parity][warp] = m;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kActBlk / 32; ++w) m = max(m, red[parity][w]);
+    const int e = w16_scale_exp(m);
+    const float S = __uint_as_float((uint32_t)(127 + e) << 23);
+    if (tid == 0) row_scale[p] = __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+    for (int u = 0; u < kNU; ++u) {
+      const int c = u * kActBlk + tid;
+      if (c < n4) {
+        float4 o = v[u];
+        o.x *= S; o.y *= S; o.z *= S; o.w *= S;
+        const uint2 hq = make_uint2(half2_bits(o.x, o.y), half2_bits(o.z, o.w));
+        const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hq.x));
+        const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hq.y));
+        __stcs(rows16 + base + c, hq);
+        __stcs(mid + base + c, make_uint2(half2_bits(o.x - h0.x, o.y - h0.y), half2_bits(o.z - h1.x, o.w - h1.y)));
+      }
+    }
+  }
+}
+
+template <typename Kernel>
+int64_t resident_grid(Kernel k, int64_t rows) {
+  int b = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k, 256, 0) != cudaSuccess || b < 1) b = 2;
+  return std::min<int64_t>((rows + 7) / 8, (int64_t)num_sms() * b);
+}
+
+template <int kOp, int kNU>
+void launch_act_split_blk(const float* x, const float* a, int64_t rows, int32_t n, uint16_t* rows16, float* row_scale,
+                          cudaStream_t stream) {
+  static const int per_sm = [] {
+    int b = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, act_split_blk_kernel<kOp, kNU>, kActBlk, 0) != cudaSuccess ||
+        b < 1)
+      b = 4;
+    return b;
+  }();
+  const int64_t blocks = std::min<int64_t>(rows, (int64_t)num_sms() * per_sm);
+  act_split_blk_kernel<kOp, kNU><<<(unsigned)blocks, kActBlk, 0, stream>>>((const float4*)x, (const float4*)a, rows,
+                                                                           n / 4, (uint2*)rows16, row_scale);
+}
+
+template <int kOp>
+janus_status act_split_launch(const float* x, const float* a, int64_t rows, int32_t n, uint16_t* rows16,
+                              float* row_scale, cudaStream_t stream) {
+  if (rows == 0) return JANUS_OK;
+  // float4 per thread for the whole row, 128 threads per row
+  switch ((n / 4 + kActBlk - 1) / kActBlk) {
+    case 1: launch_act_split_blk<kOp, 1>(x, a, rows, n, rows16, row_scale, stream); break;
+    case 2: launch_act_split_blk<kOp, 2>(x, a, rows, n, rows16, row_scale, stream); break;
+    case 3: launch_act_split_blk<kOp, 3>(x, a, rows, n, rows16, row_scale, stream); break;
+    case 4: launch_act_split_blk<kOp, 4>(x, a, rows, n, rows16, row_scale, stream); break;
+    case 5: launch_act_split_blk<kOp, 5>(x, a, rows, n, rows16, row_scale, stream); break;
+    case 6: launch_act_split_blk<kOp, 6>(x, a, rows, n, rows16, row_scale, stream); break;
+    case 7: launch_act_split_blk<kOp, 7>(x, a, rows, n, rows16, row_scale, stream); break;
+    case 8: launch_act_split_blk<kOp, 8>(x, a, rows, n, rows16, row_scale, stream); break;
+    default: {
+      // longer rows: two sweeps, the second finding the row in L1 / L2
+      static const int64_t per_sm_probe = resident_grid(act_split_kernel<kOp>, INT64_MAX / 2);
+      const int64_t blocks = std::min<int64_t>((rows + 7) / 8, per_sm_probe);
+      act_split_kernel<kOp><<<(unsigned)blocks, 256, 0, stream>>>((const float4*)x, (const float4*)a, rows, n / 4,
+                                                                   (uint2*)rows16, row_scale);
+    }
+  }
+  return launch_status();
+}
+
 template <int kOp>
 janus_status act_split_f16(const float* x, const float* a, int64_t rows, int32_t n, uint16_t* rows16,
                            float* row_scale, cudaStream_t stream) {
-  if (rows == 0) return JANUS_OK;
-  const int64_t blocks = std::min<int64_t>((rows + 7) / 8, (int64_t)num_sms() * 8);
-  act_split_kernel<kOp><<<(unsigned)blocks, 256, 0, stream>>>((const float4*)x, (const float4*)a, rows, n / 4,
-                                                               (uint2*)rows16, row_scale);
-  return launch_status();
+  TraceScope trace(kOp == kActSilu ? "act_split silu" : "act_split dsilu", stream);
+  return act_split_launch<kOp>(x, a, rows, n, rows16, row_scale, stream);
 }
 
 }  // namespace
 
 janus_status split_weights_f16(const float* w, int32_t E, int32_t Kd, int32_t N, bool transposed, uint16_t* w16,
                                float* winv, cudaStream_t stream) {
+  TraceScope trace(transposed ? "w16_split transposed" : "w16_split rows", stream);
+  if (N % 4 != 0 || Kd % 4 != 0) return JANUS_ERR_MISALIGNED;   // the FFN calls require d, h % 4 == 0
+  if (!transposed) {
+    // x W^T: W [E][N][Kd] is already K-major: the activation split of its E N
+    // rows (one warp per row, the row in registers, 1 / S per row into winv)
+    return act_split_launch<kActPlain>(nullptr, w, (int64_t)E * N, Kd, w16, winv, stream);
+  }
+  // x W: W [E][Kd][N] is transposed on the way
   uint32_t* colmax = reinterpret_cast<uint32_t*>(winv);
   const int64_t n = (int64_t)E * N;
-  if (!transposed) {
-    // x W^T: W [E][N][Kd] is already K-major
-    const int64_t blocks = std::min<int64_t>((n + 7) / 8, (int64_t)num_sms() * 8);
-    w16_rowmax_kernel<<<(unsigned)blocks, 256, 0, stream>>>(w, n, Kd, colmax);
-    const int64_t eb = std::min<int64_t>(n, (int64_t)num_sms() * 16);
-    w16_split_rows_kernel<<<(unsigned)eb, 256, 0, stream>>>(w, n, Kd, colmax, reinterpret_cast<__half*>(w16));
-    w16_inv_scale_kernel<<<(unsigned)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, stream>>>(colmax, n);
-    return launch_status();
-  }
-  JANUS_CUDA_TRY(cudaMemsetAsync(colmax, 0, sizeof(uint32_t) * (size_t)E * N, stream));
+  JANUS_CUDA_TRY(cudaMemsetAsync(colmax, 0, sizeof(uint32_t) * (size_t)n, stream));
   const int k_per = 64;
-  w16_colmax_kernel<<<dim3((N + 255) / 256, (Kd + k_per - 1) / k_per, E), 256, 0, stream>>>(w, Kd, N, k_per,
-                                                                                            colmax);
-  w16_split_kernel<<<dim3((N + 31) / 32, (Kd + 63) / 64, E), 256, 0, stream>>>(w, E, Kd, N, colmax,
-                                                                             reinterpret_cast<__half*>(w16));
+  w16_colmax_kernel<<<dim3((N + 255) / 256, (Kd + k_per - 1) / k_per, E), 256, 0, stream>>>(w, Kd, N, k_per, colmax);
+  const int64_t tiles = (int64_t)E * ((N + 31) / 32) * ((Kd + kColTileK - 1) / kColTileK);
+  const int64_t blocks = std::min<int64_t>(tiles, (int64_t)num_sms() * 8);
+  w16_split_tile_kernel<<<(unsigned)blocks, 256, 0, stream>>>(w, E, Kd, N, colmax, reinterpret_cast<__half*>(w16));
   w16_inv_scale_kernel<<<(unsigned)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, stream>>>(colmax, n);
   return launch_status();
 }

@@ -35,6 +35,7 @@ struct F16Second {
 // The FP16 split of a GEMM's weights for the kind::f16 path: w16 = [hi | mid],
 // each [E][N][Kd] FP16 (2 * E * N * Kd values), winv [E][N] = 1 / S per
 // output feature.  transposed: w is [E][Kd][N] (x W); else [E][N][Kd] (x W^T).
+// One kernel; N % 4 == 0 and Kd % 4 == 0 (JANUS_ERR_MISALIGNED otherwise).
 janus_status split_weights_f16(const float* w, int32_t E, int32_t Kd, int32_t N, bool transposed, uint16_t* w16,
                                float* winv, cudaStream_t stream);
 

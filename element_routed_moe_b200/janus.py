@@ -47,6 +47,7 @@ SYMBOLS = (
     "janus_ep_return", "janus_ep_return_rows",
     "janus_ipc_get_handle", "janus_ipc_open_handle", "janus_ipc_close_handle",
     "janus_debug_build", "janus_debug_check", "janus_debug_inject_launch_failures",
+    "janus_trace_start", "janus_trace_stop", "janus_trace_count", "janus_trace_get", "janus_trace_release",
 )
 
 
@@ -159,6 +160,11 @@ def _declare(L):
         "janus_debug_build": (i32, []),
         "janus_debug_check": (st, [vp]),
         "janus_debug_inject_launch_failures": (None, [i32]),
+        "janus_trace_start": (st, [i32]),
+        "janus_trace_stop": (st, []),
+        "janus_trace_count": (st, [ctypes.POINTER(ctypes.c_int32)]),
+        "janus_trace_get": (st, [i32, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float)]),
+        "janus_trace_release": (st, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -889,3 +895,30 @@ def janus_debug_check(stream=None):
 
 def janus_debug_inject_launch_failures(n_calls: int):
     lib().janus_debug_inject_launch_failures(int(n_calls))
+
+
+def janus_trace_start(capacity: int):
+    """Start recording up to `capacity` traced launches (CUDA events on each
+    launch's stream; the current device)."""
+    _raise(lib().janus_trace_start(int(capacity)), "janus_trace_start")
+
+
+def janus_trace_stop():
+    _raise(lib().janus_trace_stop(), "janus_trace_stop")
+
+
+def janus_trace_records():
+    """[(kernel name, ms)] of the recorded launches, in launch order (waits
+    for each record's end event)."""
+    n = ctypes.c_int32(0)
+    _raise(lib().janus_trace_count(ctypes.byref(n)), "janus_trace_count")
+    out = []
+    name, ms = ctypes.c_char_p(), ctypes.c_float()
+    for i in range(n.value):
+        _raise(lib().janus_trace_get(i, ctypes.byref(name), ctypes.byref(ms)), "janus_trace_get")
+        out.append((name.value.decode(), float(ms.value)))
+    return out
+
+
+def janus_trace_release():
+    _raise(lib().janus_trace_release(), "janus_trace_release")

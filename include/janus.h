@@ -605,6 +605,24 @@ int32_t janus_debug_build(void);
  * build); JANUS_ERR_CUDA if a CUDA call failed. */
 janus_status janus_debug_check(janus_stream_t stream);
 
+/* Launch trace, for measuring the kernels inside a call.  janus_trace_start
+ * creates `capacity` pairs of CUDA events on the current device (1 <= capacity
+ * <= 2^20; any earlier records are dropped) and starts recording: from then on
+ * each traced launch of this library (the expert MLP's tensor-core GEMMs, its
+ * weight and activation splits) is bracketed by two events recorded on the
+ * launch's stream, until janus_trace_stop or until `capacity` launches have
+ * been recorded.  janus_trace_count gives the number of records;
+ * janus_trace_get(i) waits for record i's end event and returns its kernel's
+ * name (a static string owned by the library) and its duration in ms.
+ * janus_trace_release stops recording and destroys the events.  The trace is
+ * process-wide; one device at a time.  JANUS_ERR_CUDA if an event cannot be
+ * created or read; JANUS_ERR_INVALID_ARG for a bad capacity or index. */
+janus_status janus_trace_start(int32_t capacity);
+janus_status janus_trace_stop(void);
+janus_status janus_trace_count(int32_t* n);
+janus_status janus_trace_get(int32_t i, const char** name, float* ms);
+janus_status janus_trace_release(void);
+
 /* Host-side fault injection for tests: the next `n_calls` library calls that
  * would launch work return JANUS_ERR_CUDA before launching anything. */
 void janus_debug_inject_launch_failures(int32_t n_calls);

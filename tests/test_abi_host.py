@@ -172,6 +172,19 @@ def test_empty_inputs_are_no_ops(J):
     assert L.janus_dequant_by_type(None, 0, 8, 2, None, 4, None, None, None, None) == J.JANUS_OK
 
 
+def test_trace_checks_its_arguments(J):
+    # the checks come before any CUDA call: no GPU needed
+    L = J.lib()
+    assert L.janus_trace_start(0) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_trace_start((1 << 20) + 1) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_trace_count(None) == J.JANUS_ERR_INVALID_ARG
+    assert J.janus_trace_records() == []          # nothing recorded
+    name, ms = ctypes.c_char_p(), ctypes.c_float()
+    assert L.janus_trace_get(0, ctypes.byref(name), ctypes.byref(ms)) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_trace_get(0, None, None) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_trace_stop() == J.JANUS_OK and L.janus_trace_release() == J.JANUS_OK
+
+
 def test_release_build_reports_no_debug_faults(J):
     assert J.janus_debug_build() is False
 

@@ -85,6 +85,9 @@ SHAPES = {
     # >= 2048 rows per expert, h % 8 == 0: the forward's second GEMM on the
     # FP16 path too (K = h = 200: three 64-wide blocks and an 8-wide tail)
     "second_f16": ([3000, 0, 3300], 136, 200),
+    # rows of more than 4096 values: the activation and weight-row splits
+    # take their two-sweep kernel
+    "long_rows": ([2100], 16, 4104),
 }
 
 
