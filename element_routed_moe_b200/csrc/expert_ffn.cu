@@ -97,10 +97,15 @@ bool use_f16_second(int64_t R, int32_t E, int32_t h) {
   return h % 8 == 0 && R >= kF16SecondMinRowsPerExpert * E;
 }
 
+// 1 / S of a weight split: per output feature (N) and K chunk of 256.
+size_t winv_bytes(int32_t E, int32_t Kd, int32_t N) {
+  return align_up(sizeof(float) * (size_t)E * (size_t)((Kd + 255) / 256) * (size_t)N, 256);
+}
+
 // Scratch of the FP16 second GEMM (see tc::F16Second), starting at `base`.
 size_t f16_second_bytes(int64_t R, int32_t E, int32_t d, int32_t h) {
   return align_up(2 * sizeof(uint16_t) * (size_t)R * h, 256) + align_up(sizeof(float) * (size_t)R, 256) +
-         align_up(2 * sizeof(uint16_t) * (size_t)E * d * h, 256) + align_up(sizeof(float) * (size_t)E * d, 256);
+         align_up(2 * sizeof(uint16_t) * (size_t)E * d * h, 256) + winv_bytes(E, h, d);
 }
 tc::F16Second f16_second_at(char* base, int64_t R, int32_t E, int32_t d, int32_t h) {
   tc::F16Second f;
@@ -115,11 +120,11 @@ tc::F16Second f16_second_at(char* base, int64_t R, int32_t E, int32_t d, int32_t
 }
 
 // Past the forward's activations: SIMT, the unpacked rows [R,d] FP32;
-// 3xTF32, the FP16 split of W1 (hi and mid, [E][h][d] each), 1 / S [E][h],
+// 3xTF32, the FP16 split of W1 (hi and mid, [E][h][d] each), 1 / S [E][ceil(d/256)][h],
 // and the FP16 second GEMM's scratch when it is used.
 size_t packed_extra(int64_t R, int32_t E, int32_t d, int32_t h, janus_ffn_mode mode) {
   if (mode == JANUS_FFN_FP32_SIMT) return align_up(sizeof(float) * (size_t)R * (size_t)d, 256);
-  return align_up(2 * sizeof(uint16_t) * (size_t)E * d * h, 256) + align_up(sizeof(float) * (size_t)E * h, 256) +
+  return align_up(2 * sizeof(uint16_t) * (size_t)E * d * h, 256) + winv_bytes(E, d, h) +
          (use_f16_second(R, E, h) ? f16_second_bytes(R, E, d, h) : 0);
 }
 
@@ -166,7 +171,7 @@ extern "C" janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, con
     uint16_t* w16 = (uint16_t*)((char*)workspace + L.total);
     const size_t w16_bytes = align_up(2 * sizeof(uint16_t) * (size_t)n_experts * d * h, 256);
     float* winv = (float*)((char*)workspace + L.total + w16_bytes);
-    char* second_base = (char*)workspace + L.total + w16_bytes + align_up(sizeof(float) * (size_t)n_experts * h, 256);
+    char* second_base = (char*)workspace + L.total + w16_bytes + winv_bytes(n_experts, d, h);
     const tc::F16Second second = f16_second_at(second_base, n_rows, n_experts, d, h);
     st = tc::expert_ffn_fwd_packed(payload, row_scale, offsets, n_experts, n_rows, d, h, w1, w2, yd, act, H, w16,
                                    winv, &((WsHeader*)workspace)->error, stream, yd_rows,
@@ -193,7 +198,7 @@ extern "C" janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, con
 // (gd W2^T) on the kind::f16 tensor path; the second on 3xTF32, or on the
 // kind::f16 path at >= 2048 rows per expert with h % 8 == 0.  Workspace:
 // header | H, dH or dA [R,h] | the FP16 split of the first GEMM's weights
-// (hi and mid, [E][h][d] each) | 1 / S [E][h] | the FP16 second GEMM's
+// (hi and mid, [E][h][d] each) | 1 / S [E][ceil(d/256)][h] | the FP16 second GEMM's
 // scratch when it is used.
 // ---------------------------------------------------------------------------
 namespace {
@@ -205,7 +210,7 @@ SplitLayout split_layout(int64_t R, int32_t E, int32_t d, int32_t h) {
   L.off_h = sizeof(WsHeader);
   L.off_w16 = L.off_h + align_up(sizeof(float) * (size_t)R * (size_t)h, 256);
   L.off_winv = L.off_w16 + align_up(2 * sizeof(uint16_t) * (size_t)E * d * h, 256);
-  L.off_second = L.off_winv + align_up(sizeof(float) * (size_t)E * h, 256);
+  L.off_second = L.off_winv + winv_bytes(E, d, h);
   L.total = L.off_second + (use_f16_second(R, E, h) ? f16_second_bytes(R, E, d, h) : 0);
   return L;
 }

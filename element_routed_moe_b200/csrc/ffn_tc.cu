@@ -501,6 +501,15 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
     bool ok = true;
     for (int c0 = 0; c0 < c.nk; c0 += kChunk, ++ch) {
       const uint32_t p = ch & 1, cuse = ch >> 1;
+      // FP16 path: the weights' 1 / S for this lane's feature and this K
+      // chunk (the split scales each feature per chunk of 256), loaded before
+      // the wait; the chunk's sum is scaled by it as it is folded (exact)
+      float wsc = 1.0f;
+      if (f16_path<kBK>()) {
+        const int f = c.m0 + q * 32 + lane;
+        const int nch = (args.Kd + 255) / 256;
+        wsc = f < c.m_end ? __ldg(args.col_scale + ((int64_t)c.e * nch + c0 / kChunk) * N + f) : 0.f;
+      }
       // the warp leaves together (a timeout seen by one lane ends the tile for
       // all 32: the TMEM loads and the row-scale shuffles are warp-wide)
       if (!__all_sync(0xffffffffu, mbar_wait(s, &s->chunk_full[p], cuse & 1, args.err))) { ok = false; break; }
@@ -511,8 +520,12 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
         uint32_t r[16];
         tmem_ld16(taddr + j, r);
 #pragma unroll
-        for (int t = 0; t < 16; ++t)
-          acc[j + t] += __uint_as_float(r[t]);
+        for (int t = 0; t < 16; ++t) {
+          if (f16_path<kBK>())
+            acc[j + t] = fmaf(__uint_as_float(r[t]), wsc, acc[j + t]);
+          else
+            acc[j + t] += __uint_as_float(r[t]);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -549,9 +562,8 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
       const bool f_ok = f < c.m_end;
       if (kShflScale || f_ok) {
         // FP16 path: the product is q (hi + mid) S (kBF16S: q = the row's
-        // two terms); scale column j by its row's s_p and this lane's feature
-        // by 1 / S (powers of two: exact)
-        const float cscale = (f16_path<kBK>() && f_ok) ? __ldg(args.col_scale + (int64_t)c.e * N + f) : 1.0f;
+        // two terms); the sums already carry the weights' 1 / S (folded per
+        // chunk); scale column j by its row's s_p (a power of two: exact)
         // batches of 8 columns; the pre-activations of batch b + 1 are in
         // flight while batch b is finished, so two loads per column overlap
         constexpr int kB = 8;
@@ -574,8 +586,8 @@ __device__ __forceinline__ void epilogue_role(Smem* s, const Args& args, uint32_
             if (f_ok && j0 + jb + j < c.n_valid) {
               const int64_t o = (int64_t)(c.n0 + j0 + jb + j) * N + f;
               float v = acc[jb + j];
-              if (kShflScale) v = v * rs * cscale;
-              else if (f16_path<kBK>()) v = v * __ldg(args.row_scale + c.n0 + j0 + jb + j) * cscale;
+              if (kShflScale) v = v * rs;
+              else if (f16_path<kBK>()) v = v * __ldg(args.row_scale + c.n0 + j0 + jb + j);
               if (kEpi == kEpiStore && args.c_rows) {   // the row's own destination
                 args.c_rows[c.n0 + j0 + jb + j][f] = v;
                 continue;
@@ -1114,14 +1126,15 @@ janus_status launch(const float* A, const float* W, int64_t R, int E, int Kd, in
 // ---- the FP16 split of the weights for the kind::f16 GEMMs ------------------
 // x W (W [E][Kd][N]) or x W^T (W [E][N][Kd]) FP32 -> w16 = [hi | mid], each
 // [E][N][Kd] FP16 (K-major for the kind::f16 MMA: x W's weights are
-// transposed on the way), and winv [E][N] = 1 / S per output feature.
-// S = 2^(141 - b), b = the biased exponent of the column's largest magnitude,
-// so that magnitude times S lies in [2^14, 2^15) (below FP16's 65504); S is
-// clamped to [2^-126, 2^126] and is 1 for an all-zero column.  hi = fp16(w S)
-// and mid = fp16(w S - hi): w S - hi is exact in FP32 and the pair carries
-// 22 bits of w S.  x W: column maxima, the split with the transpose through
-// shared memory, maxima -> 1 / S; x W^T: one pass over each row.  N % 4 == 0
-// and Kd % 4 == 0 (JANUS_ERR_MISALIGNED otherwise).
+// transposed on the way), and winv [E][nch][N] = 1 / S per output feature and
+// K chunk of 256 (nch = ceil(Kd / 256), the GEMM's TMEM chunk, so the
+// epilogue applies each chunk's scale as it folds the chunk).  S = 2^(141 -
+// b), b = the biased exponent of the largest magnitude of the feature's
+// chunk, so that magnitude times S lies in [2^14, 2^15) (below FP16's 65504);
+// S is clamped to [2^-126, 2^126] and is 1 for an all-zero chunk.  hi = fp16(w
+// S) and mid = fp16(w S - hi): w S - hi is exact in FP32 and the pair carries
+// 22 bits of w S.  One kernel, W read once.  N % 4 == 0 and Kd % 4 == 0
+// (JANUS_ERR_MISALIGNED otherwise).
 
 __device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
@@ -1134,56 +1147,61 @@ __device__ __forceinline__ int w16_scale_exp(uint32_t max_bits) {
   return min(max(141 - b, -126), 126);
 }
 
-// x W, three kernels: the column maxima (as ordered bits, into winv), the
-// split, and the maxima turned into 1 / S in place.
-__global__ void __launch_bounds__(256) w16_colmax_kernel(const float* __restrict__ w, int Kd, int N, int k_per,
-                                                         uint32_t* __restrict__ colmax) {
-  const int e = blockIdx.z, f = blockIdx.x * 256 + threadIdx.x, k0 = blockIdx.y * k_per;
-  if (f >= N) return;
-  const float* p = w + (int64_t)e * Kd * N + f;
-  const int k1 = min(k0 + k_per, Kd);
-  uint32_t m = 0;
-  for (int k = k0; k < k1; ++k) m = max(m, __float_as_uint(__ldcs(p + (int64_t)k * N)) & 0x7fffffffu);
-  if (m) atomicMax(colmax + (int64_t)e * N + f, m);
-}
-
-// The split, over tiles of 32 features x 128 k of one expert (grid-stride):
-// each thread loads four float4 (128-byte row segments of W[e], [Kd][N]),
-// scales and splits them, the tile goes through shared memory, and each warp
-// writes four features' 128 k as half2 pairs into the K-major planes.  Many
-// blocks per SM keep enough loads in flight.  N % 4 == 0, Kd % 2 == 0.
-constexpr int kColTileK = 128;
-__global__ void __launch_bounds__(256) w16_split_tile_kernel(const float* __restrict__ w, int E, int Kd, int N,
-                                                             const uint32_t* __restrict__ colmax,
-                                                             __half* __restrict__ w16) {
-  __shared__ __align__(16) __half t_hi[32][kColTileK + 2];
-  __shared__ __align__(16) __half t_mid[32][kColTileK + 2];
+// x W: tiles of one expert's 256 k x 32 features (W[e] is [Kd][N]).  Each
+// thread loads eight float4 (128-byte row segments, all in flight), the 32
+// column maxima of the tile go through shared memory, and the tile is scaled,
+// split and transposed through shared memory into the K-major planes, each
+// warp writing four features' 256 k as half2 pairs: W is read once.
+constexpr int kChunkK = 256;           // the K chunk of the scales (= the GEMM's TMEM chunk)
+__global__ void __launch_bounds__(256) w16_split_cols_kernel(const float* __restrict__ w, int E, int Kd, int N,
+                                                             __half* __restrict__ w16, float* __restrict__ winv) {
+  __shared__ uint32_t red[32][33];
+  __shared__ float s_scale[32];
+  __shared__ __align__(16) __half t_hi[32][kChunkK + 2];
+  __shared__ __align__(16) __half t_mid[32][kChunkK + 2];
   const int tid = threadIdx.x, tx = tid % 8, ty = tid / 8;
   const int warp = tid / 32, lane = tid % 32;
-  const int strips_n = (N + 31) / 32, ktiles = (Kd + kColTileK - 1) / kColTileK;
-  const int64_t n_tiles = (int64_t)E * strips_n * ktiles;
+  const int strips_n = (N + 31) / 32, nch = (Kd + kChunkK - 1) / kChunkK;
+  const int64_t n_tiles = (int64_t)E * nch * strips_n;
   const int64_t plane = (int64_t)E * N * Kd;                 // mid follows hi
   const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-    const int kt = (int)(t % ktiles);
-    const int64_t es = t / ktiles;
-    const int e = (int)(es / strips_n), f0 = (int)(es % strips_n) * 32, k0 = kt * kColTileK;
+    const int st = (int)(t % strips_n);
+    const int64_t ec = t / strips_n;
+    const int e = (int)(ec / nch), ci = (int)(ec % nch), f0 = st * 32, k0 = ci * kChunkK;
     const float* we = w + (int64_t)e * Kd * N;
     const int fc = f0 + 4 * tx;
     const bool col_ok = fc < N;                              // N % 4 == 0: all four columns
-    float sc[4];
+    float4 v[kChunkK / 32];
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      sc[j] = col_ok ? __uint_as_float((uint32_t)(127 + w16_scale_exp(__ldg(colmax + (int64_t)e * N + fc + j))) << 23)
-                     : 0.f;
-    float4 v[kColTileK / 32];
-#pragma unroll
-    for (int u = 0; u < kColTileK / 32; ++u) {
+    for (int u = 0; u < kChunkK / 32; ++u) {
       const int k = k0 + ty + 32 * u;
       v[u] = (col_ok && k < Kd) ? __ldcs(reinterpret_cast<const float4*>(we + (int64_t)k * N + fc)) : zero;
     }
+    uint32_t m[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int u = 0; u < kColTileK / 32; ++u) {
+    for (int u = 0; u < kChunkK / 32; ++u) {
+      m[0] = max(m[0], __float_as_uint(v[u].x) & 0x7fffffffu);
+      m[1] = max(m[1], __float_as_uint(v[u].y) & 0x7fffffffu);
+      m[2] = max(m[2], __float_as_uint(v[u].z) & 0x7fffffffu);
+      m[3] = max(m[3], __float_as_uint(v[u].w) & 0x7fffffffu);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) red[ty][4 * tx + j] = m[j];
+    __syncthreads();
+    if (tid < 32) {
+      uint32_t mm = 0;
+      for (int j = 0; j < 32; ++j) mm = max(mm, red[j][tid]);
+      const int ex = w16_scale_exp(mm);
+      s_scale[tid] = __uint_as_float((uint32_t)(127 + ex) << 23);
+      if (f0 + tid < N) winv[((int64_t)e * nch + ci) * N + f0 + tid] = __uint_as_float((uint32_t)(127 - ex) << 23);
+    }
+    __syncthreads();
+    float sc[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sc[j] = s_scale[4 * tx + j];
+#pragma unroll
+    for (int u = 0; u < kChunkK / 32; ++u) {
       const int kr = ty + 32 * u;
       const float val[4] = {v[u].x * sc[0], v[u].y * sc[1], v[u].z * sc[2], v[u].w * sc[3]};
 #pragma unroll
@@ -1200,7 +1218,7 @@ __global__ void __launch_bounds__(256) w16_split_tile_kernel(const float* __rest
       if (fo >= N) continue;
       const int64_t row = ((int64_t)e * N + fo) * Kd;
 #pragma unroll
-      for (int q = 0; q < kColTileK / 64; ++q) {
+      for (int q = 0; q < kChunkK / 64; ++q) {
         const int kk = 2 * (lane + 32 * q), ko = k0 + kk;
         if (ko + 1 < Kd) {
           __stcs(reinterpret_cast<__half2*>(w16 + row + ko), *reinterpret_cast<const __half2*>(&t_hi[fl][kk]));
@@ -1215,15 +1233,59 @@ __global__ void __launch_bounds__(256) w16_split_tile_kernel(const float* __rest
   }
 }
 
-__global__ void __launch_bounds__(256) w16_inv_scale_kernel(uint32_t* __restrict__ colmax_to_inv, int64_t n) {
-  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (int64_t)gridDim.x * 256)
-    colmax_to_inv[i] = (uint32_t)(127 - w16_scale_exp(colmax_to_inv[i])) << 23;
+// x W^T: W [E][N][Kd] is K-major already: one warp per (row, K chunk of 256),
+// two float4 per lane, the chunk's maximum by shuffles, then hi and mid.
+__global__ void __launch_bounds__(256) w16_split_rows_kernel(const float4* __restrict__ w, int64_t rows, int Kd,
+                                                             int N, uint2* __restrict__ w16,
+                                                             float* __restrict__ winv) {
+  const int lane = threadIdx.x % 32;
+  const int k4 = Kd / 4, nch = (Kd + kChunkK - 1) / kChunkK;
+  const int64_t items = rows * nch;
+  uint2* __restrict__ mid = w16 + rows * k4;
+  const int64_t nw = (int64_t)gridDim.x * 8;
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int64_t it = ((int64_t)blockIdx.x * 256 + threadIdx.x) / 32; it < items; it += nw) {
+    const int64_t r = it / nch;
+    const int ci = (int)(it % nch);
+    const int64_t base = r * k4;
+    float4 v[kChunkK / 128];
+#pragma unroll
+    for (int u = 0; u < kChunkK / 128; ++u) {
+      const int c = ci * (kChunkK / 4) + u * 32 + lane;
+      v[u] = c < k4 ? __ldcs(w + base + c) : zero;
+    }
+    uint32_t m = 0;
+#pragma unroll
+    for (int u = 0; u < kChunkK / 128; ++u)
+      m = max(m, max(max(__float_as_uint(v[u].x) & 0x7fffffffu, __float_as_uint(v[u].y) & 0x7fffffffu),
+                     max(__float_as_uint(v[u].z) & 0x7fffffffu, __float_as_uint(v[u].w) & 0x7fffffffu)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const int ex = w16_scale_exp(m);
+    const float S = __uint_as_float((uint32_t)(127 + ex) << 23);
+    if (lane == 0) {
+      const int64_t e = r / N, n = r % N;
+      winv[(e * nch + ci) * N + n] = __uint_as_float((uint32_t)(127 - ex) << 23);
+    }
+#pragma unroll
+    for (int u = 0; u < kChunkK / 128; ++u) {
+      const int c = ci * (kChunkK / 4) + u * 32 + lane;
+      if (c < k4) {
+        float4 o = v[u];
+        o.x *= S; o.y *= S; o.z *= S; o.w *= S;
+        const uint2 hq = make_uint2(half2_bits(o.x, o.y), half2_bits(o.z, o.w));
+        const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hq.x));
+        const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hq.y));
+        __stcs(w16 + base + c, hq);
+        __stcs(mid + base + c, make_uint2(half2_bits(o.x - h0.x, o.y - h0.y), half2_bits(o.z - h1.x, o.w - h1.y)));
+      }
+    }
+  }
 }
 
 // ---- the FP16 row split of an activation for a kind::f16 GEMM ---------------
 // v = silu(a) (kActSilu) or x silu'(a) (kActDSilu), with the SiLU arithmetic
-// of the GEMM epilogues, or v = a (kActPlain: the rows of a K-major weight
-// matrix, one per output feature), written as hi and mid binary16 planes
+// of the GEMM epilogues, written as hi and mid binary16 planes
 // ([rows][n] each) with one power-of-two scale per row: S_p puts the row's
 // largest |v| in [2^14, 2^15), hi = fp16(v S_p), mid = fp16(v S_p - hi),
 // row_scale[p] = 1 / S_p.  Rows up to 4096 values stay in the registers of a
@@ -1232,13 +1294,12 @@ __global__ void __launch_bounds__(256) w16_inv_scale_kernel(uint32_t* __restrict
 // writing the two terms with loads that find the row in L1 / L2
 // (act_split_kernel).  Either way the inputs are read from DRAM once and the
 // FP32 v is never stored.
-enum ActOp { kActPlain = 0, kActSilu = 1, kActDSilu = 2 };
+enum ActOp { kActSilu = 1, kActDSilu = 2 };
 constexpr int kActU = 4;       // float4 columns per lane in flight per sweep step
 
 template <int kOp, bool kLast>
 __device__ __forceinline__ float4 act_value(const float4* __restrict__ x, const float4* __restrict__ a, int64_t i) {
   const float4 av = kLast ? __ldcs(a + i) : __ldg(a + i);
-  if (kOp == kActPlain) return av;
   if (kOp == kActSilu) return make_float4(silu_f(av.x), silu_f(av.y), silu_f(av.z), silu_f(av.w));
   const float4 xv = kLast ? __ldcs(x + i) : __ldg(x + i);
   float4 v;
@@ -1427,21 +1488,17 @@ janus_status split_weights_f16(const float* w, int32_t E, int32_t Kd, int32_t N,
                                float* winv, cudaStream_t stream) {
   TraceScope trace(transposed ? "w16_split transposed" : "w16_split rows", stream);
   if (N % 4 != 0 || Kd % 4 != 0) return JANUS_ERR_MISALIGNED;   // the FFN calls require d, h % 4 == 0
+  const int64_t nch = (Kd + kChunkK - 1) / kChunkK;
   if (!transposed) {
-    // x W^T: W [E][N][Kd] is already K-major: the activation split of its E N
-    // rows (one warp per row, the row in registers, 1 / S per row into winv)
-    return act_split_launch<kActPlain>(nullptr, w, (int64_t)E * N, Kd, w16, winv, stream);
+    const int64_t items = (int64_t)E * N * nch;
+    const int64_t blocks = std::min<int64_t>((items + 7) / 8, (int64_t)num_sms() * 8);
+    w16_split_rows_kernel<<<(unsigned)blocks, 256, 0, stream>>>((const float4*)w, (int64_t)E * N, Kd, N,
+                                                               (uint2*)w16, winv);
+    return launch_status();
   }
-  // x W: W [E][Kd][N] is transposed on the way
-  uint32_t* colmax = reinterpret_cast<uint32_t*>(winv);
-  const int64_t n = (int64_t)E * N;
-  JANUS_CUDA_TRY(cudaMemsetAsync(colmax, 0, sizeof(uint32_t) * (size_t)n, stream));
-  const int k_per = 64;
-  w16_colmax_kernel<<<dim3((N + 255) / 256, (Kd + k_per - 1) / k_per, E), 256, 0, stream>>>(w, Kd, N, k_per, colmax);
-  const int64_t tiles = (int64_t)E * ((N + 31) / 32) * ((Kd + kColTileK - 1) / kColTileK);
-  const int64_t blocks = std::min<int64_t>(tiles, (int64_t)num_sms() * 8);
-  w16_split_tile_kernel<<<(unsigned)blocks, 256, 0, stream>>>(w, E, Kd, N, colmax, reinterpret_cast<__half*>(w16));
-  w16_inv_scale_kernel<<<(unsigned)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, stream>>>(colmax, n);
+  const int64_t tiles = (int64_t)E * nch * ((N + 31) / 32);
+  const int64_t blocks = std::min<int64_t>(tiles, (int64_t)num_sms() * 4);
+  w16_split_cols_kernel<<<(unsigned)blocks, 256, 0, stream>>>(w, E, Kd, N, reinterpret_cast<__half*>(w16), winv);
   return launch_status();
 }
 

@@ -24,7 +24,7 @@ janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, 
 // Scratch of the MLP's second GEMM on the kind::f16 path (H W2 in the
 // forward, dA W1^T in the VJP, the [R][h] activation split into two FP16
 // terms per row): the activation's planes [2R][h] and row scales [R], the
-// FP16 split of the weights ([2E][d][h]) and its 1 / S [E][d].
+// FP16 split of the weights ([2E][d][h]) and its 1 / S [E][ceil(h/256)][d].
 struct F16Second {
   uint16_t* h16;
   float* hscale;
@@ -33,8 +33,9 @@ struct F16Second {
 };
 
 // The FP16 split of a GEMM's weights for the kind::f16 path: w16 = [hi | mid],
-// each [E][N][Kd] FP16 (2 * E * N * Kd values), winv [E][N] = 1 / S per
-// output feature.  transposed: w is [E][Kd][N] (x W); else [E][N][Kd] (x W^T).
+// each [E][N][Kd] FP16 (2 * E * N * Kd values), winv [E][ceil(Kd/256)][N] =
+// 1 / S per output feature and K chunk of 256.  transposed: w is [E][Kd][N]
+// (x W); else [E][N][Kd] (x W^T).
 // One kernel; N % 4 == 0 and Kd % 4 == 0 (JANUS_ERR_MISALIGNED otherwise).
 janus_status split_weights_f16(const float* w, int32_t E, int32_t Kd, int32_t N, bool transposed, uint16_t* w16,
                                float* winv, cudaStream_t stream);

@@ -74,13 +74,13 @@ class ExpertParallelLayer:
         # this library's kernels per forward + VJP: route 4, layout 1, pack 2,
         # expert MLP 2 + 2, FP32 send 1, combine 1 + 1, the unpack 1 (when not
         # fused), and the return table (fused) or the return copy twice; the
-        # fused 3xTF32 forward adds W1's split (3) and, at >= 2048 receive
+        # fused 3xTF32 forward adds W1's split (1) and, at >= 2048 receive
         # rows per local expert and h % 8 == 0, the FP16 second GEMM's row
-        # split (1) and W2's split (3)
+        # split (1) and W2's split (1)
         self.launches_per_step = 14 + (0 if self.fused_unpack else 1) + (1 if self.fused_return else 2)
         f16_first = self.fused_unpack and mode == J.JANUS_FFN_3XTF32
         self.f16_second = f16_first and h % 8 == 0 and cap >= 2048 * self.El
-        self.launches_per_step += (3 if f16_first else 0) + (4 if self.f16_second else 0)
+        self.launches_per_step += (1 if f16_first else 0) + (2 if self.f16_second else 0)
         self.payload = torch.empty((cap, d), dtype=torch.float16, device=self.dev)
         self.row_scale = torch.empty((cap,), **f32)
         self.recv_rows = torch.empty((cap, d), **f32)       # gradients in, outputs out

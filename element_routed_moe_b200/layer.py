@@ -48,9 +48,9 @@ class MoELayer:
     # this library's kernels per call (see each entry point's launches)
     LAUNCHES = {"edge_aggregate": 1, "quant": 2, "dequant": 1, "row_scales": 1, "route": 4, "dispatch": 1,
                 "ffn_fwd": 2, "combine": 1, "dispatch_w": 1, "ffn_vjp": 2, "combine_vjp": 1}
-    # the FP16 tensor path: row maxima + split dispatch; W1's transposing
-    # split (3 kernels) in front of the two GEMMs
-    LAUNCHES_SPLIT = {"dispatch": 2, "ffn_fwd": 5}
+    # the FP16 tensor path: row maxima + split dispatch; W1's split in front
+    # of the two GEMMs
+    LAUNCHES_SPLIT = {"dispatch": 2, "ffn_fwd": 3}
     SPLIT_MIN_ROWS_PER_EXPERT = 2048
 
     # pinned-host pipeline for edge-message inputs: ring of device buffers
@@ -127,14 +127,14 @@ class MoELayer:
         if self.split:
             launches.update(self.LAUNCHES_SPLIT)
         if self.packed and self.fused_unpack and mode == J.JANUS_FFN_3XTF32:
-            launches["ffn_fwd"] = 5           # W1's split (3) + the two GEMMs
+            launches["ffn_fwd"] = 3           # W1's split + the two GEMMs
         # the library also runs the forward's second GEMM on the FP16 path
         # (with H's row split and W2's split in front) at >= 2048 rows per
         # expert and h % 8 == 0, after either FP16 first GEMM
         fp16_first = self.split or (self.packed and self.fused_unpack and mode == J.JANUS_FFN_3XTF32)
         self.f16_second = fp16_first and h % 8 == 0 and R >= 2048 * E
         if self.f16_second:
-            launches["ffn_fwd"] += 4          # H's row split + W2's transposing split (3)
+            launches["ffn_fwd"] += 2          # H's row split + W2's split
         if self.split_vjp:
             # weighted split dispatch: row maxima + split; VJP: W2 split,
             # gd W2^T, dA's row split, W1 split, dA W1^T
