@@ -227,10 +227,13 @@ class ClockSampler:
 # to full size by its routed rows; valid only for the kernel source it was
 # taken on (else reported as null).
 GEMM_TRAFFIC = {
-    # slice-shaped MoE layer captured at 4,096 and 8,192 atoms, fitted as
-    # 0.41 GB (weights) + b * rows per launch and taken to R = 524,288
-    ("slice", "3xtf32"): {"src": "element_routed_moe_b200/csrc/ffn_tc.cu", "sha256_prefix": "2fbccd613e3b6b18",
-                          "bytes_per_launch": 7.92e9},
+    # the M-shaped MoE layer (the slice's) captured at 12,288 and 16,384 atoms
+    # on the FP16 path, each launch kind fitted as a + b * rows and taken to
+    # the workload's R; mean of the step's four launches
+    ("slice", "3xtf32"): {"src": "element_routed_moe_b200/csrc/ffn_tc.cu", "sha256_prefix": "bbf7aa89a7737e0f",
+                          "bytes_per_launch": 6.678e+09},
+    ("M", "3xtf32"): {"src": "element_routed_moe_b200/csrc/ffn_tc.cu", "sha256_prefix": "bbf7aa89a7737e0f",
+                      "bytes_per_launch": 3.492e+09},
 }
 
 
