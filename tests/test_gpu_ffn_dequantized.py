@@ -205,8 +205,10 @@ def test_fp16_second_gemm_handles_wide_column_ranges_of_w2():
     assert rel_fro(hy, ref_y) <= TOL_FP32
 
 
-def test_packed_forward_into_a_row_table():
-    N, T, E, K, d, h = PACKED["ragged8"]
+@pytest.mark.parametrize("name", ["ragged8", "second_f16"])
+def test_packed_forward_into_a_row_table(name):
+    # second_f16: the FP16 second GEMM stores through the row table
+    N, T, E, K, d, h = PACKED[name]
     types, r, payload, scale = _packed_inputs(N, T, E, K, d, 80)
     w1, w2 = synth.expert_weights(E, d, h, 81, DEV)
     row_scale = J.janus_dispatch_row_scales(types, T, r["perm"], K, scale)

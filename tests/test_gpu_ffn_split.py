@@ -201,6 +201,34 @@ def test_fp16_second_gemms_handle_wide_ranges():
     assert max_row_rel(host(dxd), ref_dx) <= TOL_ROW and max_row_rel(host(yd), ref_y) <= TOL_ROW
 
 
+@pytest.mark.parametrize("name", ["ragged", "second_f16"])
+def test_split_calls_store_through_a_row_table(name):
+    # the same results, row p stored at the address table[p] (the expert-
+    # parallel return); second_f16 stores from the FP16 second GEMMs
+    counts, d, h = SHAPES[name]
+    E = len(counts)
+    offs = _offsets(counts)
+    R = int(offs[-1])
+    w1, w2 = synth.expert_weights(E, d, h, 25, DEV)
+    xd = synth.normal((R, d), 26, DEV)
+    gd = synth.normal((R, d), 27, DEV)
+    o = to_dev(offs)
+    x16, xs = _split_rows(xd)
+    g16, gs = _split_rows(gd)
+    y_ref, act = J.janus_expert_ffn_fwd_split(x16, xs, o, w1, w2, want_act=True)
+    dx_ref = J.janus_expert_ffn_vjp_split(g16, gs, o, w1, w2, act)
+    slot = torch.as_tensor(np.random.default_rng(28).permutation(R + 3)[:R], device=DEV)
+    dest_y = torch.full((R + 3, d), float("nan"), device=DEV)
+    dest_dx = torch.full((R + 3, d), float("nan"), device=DEV)
+    out, _ = J.janus_expert_ffn_fwd_split(x16, xs, o, w1, w2,
+                                          out_rows=dest_y.data_ptr() + 4 * d * slot.to(torch.int64))
+    out2 = J.janus_expert_ffn_vjp_split(g16, gs, o, w1, w2, act,
+                                        out_rows=dest_dx.data_ptr() + 4 * d * slot.to(torch.int64))
+    torch.cuda.synchronize()
+    assert out is None and out2 is None
+    assert torch.equal(dest_y[slot], y_ref) and torch.equal(dest_dx[slot], dx_ref)
+
+
 def test_split_calls_check_their_arguments():
     E, d, h = 3, 12, 8                              # d % 8 != 0
     offs = to_dev(_offsets([10, 0, 6]))
