@@ -306,18 +306,19 @@ janus_status janus_expert_ffn_fwd_ex(const float* xd, const int32_t* offsets, in
  * (exactly one non-NULL) as in janus_expert_ffn_fwd_ex.
  * JANUS_FFN_3XTF32: the first GEMM multiplies the FP16 rows, as they are,
  * on the tcgen05 kind::f16 tensor path against an FP16 split of W1 that the
- * call writes into the workspace first: per expert and output feature f, a
- * power-of-two scale S_f puts the column's largest |w| in [2^14, 2^15), and
- * w S_f = hi + mid (two binary16 terms, 22 bits), so
- *   a[p,f] = row_scale[p] / S_f * sum_k payload[p,k] (hi[f,k] + mid[f,k])
- * with exact FP16 products and FP32 accumulation (chunked as in the 3xTF32
- * GEMM): FP32-accurate, within 1e-5 of the unpacked FP32 forward, at half
- * the tensor-core work of the two-product TF32 form.  The second GEMM (H W2)
- * runs on 3xTF32, or, when n_rows >= 2048 * n_experts and h % 8 == 0, on the
- * same kind::f16 path with three products after H is split into two FP16
- * terms per row in the workspace (as janus_dispatch_split does) and W2 is
- * split like W1.  d must be a multiple of 8 (JANUS_ERR_MISALIGNED
- * otherwise) and the payload 16-byte aligned.
+ * call writes into the workspace first: per expert, output feature f and K
+ * chunk c of 256, a power-of-two scale S_fc puts the chunk's largest |w| in
+ * [2^14, 2^15), and w S_fc = hi + mid (two binary16 terms, 22 bits), so
+ *   a[p,f] = row_scale[p] sum_c (1 / S_fc) sum_{k in c} payload[p,k] (hi + mid)[f,k]
+ * with exact FP16 products and FP32 accumulation per chunk (the chunks of the
+ * 3xTF32 GEMM): FP32-accurate, within 1e-5 of the unpacked FP32 forward, at
+ * half the tensor-core work of the two-product TF32 form.  The second GEMM
+ * (H W2) runs on 3xTF32, or, when n_rows >= 2048 * n_experts and h % 8 == 0,
+ * on the same kind::f16 path with three products: the first GEMM then
+ * stores a only, one pass over each row writes H = silu(a) as two FP16 terms
+ * with a per-row power-of-two scale into the workspace, and W2 is split like
+ * W1.  d must be a multiple of 8 (JANUS_ERR_MISALIGNED otherwise) and the
+ * payload 16-byte aligned.
  * JANUS_FFN_FP32_SIMT: the rows are unpacked into the workspace first; the
  * result is bit-identical to janus_dequant_by_type followed by
  * janus_expert_ffn_fwd.
@@ -342,15 +343,15 @@ janus_status janus_expert_ffn_vjp_rows(const float* xd, const float* gd, const f
  * silu'(a)) runs on the tcgen05 kind::f16 path with three products,
  *   hi_x hi_w + hi_x mid_w + mid_x hi_w,
  * against an FP16 split of the weights written into the workspace first (per
- * output feature a power-of-two scale and two binary16 terms, as in
- * janus_expert_ffn_fwd_packed); products are exact and accumulate in FP32 in
- * chunks of 256, the result is scaled by row_scale[p] and the feature's
- * 1 / S.  The second GEMM (H W2, or dA W1^T) runs on 3xTF32, or, with
+ * output feature and K chunk of 256 a power-of-two scale and two binary16
+ * terms, as in janus_expert_ffn_fwd_packed); products are exact and
+ * accumulate in FP32 per chunk, each chunk's sum is scaled by the feature's
+ * 1 / S for that chunk, and the result by row_scale[p].  The second GEMM (H W2, or dA W1^T) runs on 3xTF32, or, with
  * n_rows >= 2048 * n_experts and h % 8 == 0, on the same kind::f16 path: the
  * first GEMM then stores a (fwd) or dH = gd W2^T (vjp) plainly, and one pass
  * over each row writes H = silu(a), or dA = dH * silu'(a), as two FP16 terms
  * with a per-row power-of-two scale into the workspace, after which the
- * weights of the second GEMM are split per output feature.  FP32-accurate as
+ * weights of the second GEMM are split in the same way.  FP32-accurate as
  * the 3xTF32 forms (within 1e-5), at half their tensor-core work per FP16
  * GEMM.
  * fwd: rows16 = [hi | mid] of xd, act [R,h] nullable, yd or yd_rows (one).
