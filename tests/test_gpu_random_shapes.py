@@ -113,3 +113,38 @@ def test_random_shape_edges(seed):
         dx = synth.normal((N, d), seed + 2, DEV)
         dmsg = J.janus_edge_broadcast(dx, torch.as_tensor(rp, device=DEV))
         assert np.array_equal(host(dmsg), oracle.edge_broadcast(host(dx), rp))
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_random_shape_fp16_second_gemms(seed):
+    # >= 2048 rows per expert with d, h % 8 == 0: both GEMMs of each direction
+    # on the FP16 tensor path (split rows, the FP16 payload for the packed
+    # forward), on ragged segments and random widths with K tails
+    g = np.random.default_rng(2000 + seed)
+    E = int(g.choice([1, 2, 3, 5]))
+    counts = g.integers(0, 2 * 2048, size=E)
+    counts[int(g.integers(0, E))] += 2048 * E            # at least 2048 rows per expert overall
+    R = int(counts.sum())
+    d = int(8 * g.integers(1, 70))
+    h = int(8 * g.integers(1, 70))
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    o = to_dev(offs)
+    w1, w2 = synth.expert_weights(E, d, h, 3000 + seed, DEV)
+    xd = synth.normal((R, d), 3100 + seed, DEV)
+    gd = synth.normal((R, d), 3200 + seed, DEV)
+    ident = torch.arange(R, dtype=torch.int32, device=DEV)
+    x16, xs = J.janus_dispatch_split(xd, ident, 1)
+    g16, gs = J.janus_dispatch_split(gd, ident, 1)
+    ys, a_s = J.janus_expert_ffn_fwd_split(x16, xs, o, w1, w2, want_act=True)
+    dxs = J.janus_expert_ffn_vjp_split(g16, gs, o, w1, w2, a_s)
+    hw1, hw2 = host(w1), host(w2)
+    oyd, oact = oracle.expert_ffn_fwd(host(xd), offs, hw1, hw2, want_act=True)
+    odxd = oracle.expert_ffn_vjp(host(xd), host(gd), offs, hw1, hw2)
+    assert rel_fro(host(a_s), oact) <= TOL_FP32, seed
+    assert rel_fro(host(ys), oyd) <= TOL_FP32 and rel_fro(host(dxs), odxd) <= TOL_FP32, seed
+    # the packed forward: FP16 rows times a power-of-two scale per row
+    payload = synth.normal((R, d), 3300 + seed, DEV).half()
+    rsc = torch.as_tensor(np.ldexp(1.0, g.integers(-20, 20, size=R)).astype(np.float32), device=DEV)
+    yp, _ = J.janus_expert_ffn_fwd_packed(payload, rsc, o, w1, w2, mode=J.JANUS_FFN_3XTF32)
+    xq = host(payload).astype(np.float32) * host(rsc)[:, None]
+    assert rel_fro(host(yp), oracle.expert_ffn_fwd(xq, offs, hw1, hw2)) <= TOL_FP32, seed
