@@ -74,7 +74,7 @@ dispatch_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K,
         if (c < d4) {
           float4 o = v[u];
           if (kWeighted) { o.x *= wk; o.y *= wk; o.z *= wk; o.w *= wk; }
-          __stcs(dst + c, o);   // streaming: scattered rows, written once
+          dst[c] = o;
         }
       }
     }
@@ -221,8 +221,8 @@ dispatch_split_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int
           const uint2 hq = halves(o.x, o.y, o.z, o.w);
           const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hq.x));
           const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hq.y));
-          __stcs(rows16 + p * d4 + c, hq);
-          __stcs(mid_plane + p * d4 + c, halves(o.x - h0.x, o.y - h0.y, o.z - h1.x, o.w - h1.y));
+          rows16[p * d4 + c] = hq;
+          mid_plane[p * d4 + c] = halves(o.x - h0.x, o.y - h0.y, o.z - h1.x, o.w - h1.y);
         }
       }
     }
@@ -281,7 +281,7 @@ quant_pack_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int K,
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
         const int c = c0 + u * 32 + lane;
-        if (c < d4) __stcs(dst + c, q[u]);
+        if (c < d4) dst[c] = q[u];
       }
     }
   }
