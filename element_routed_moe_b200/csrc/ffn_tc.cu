@@ -39,8 +39,7 @@
 //                .kind::tf32 per k-block into one of two 256-column TMEM chunk
 //                buffers, commits signalling both CTAs; the peer's splitters
 //                and epilogues arrive on the leader's barriers;
-//   warps 2,3,12..15  splitters (idle on the kind::f16 path), each owning
-//                every sixth k-block: write the
+//   warps 2,3,12..15  splitters, each owning every sixth k-block: write the
 //                landed tile's residual lo = x - hi into a twin buffer (same
 //                swizzled offsets; the landed FP32 tile is read by the MMA as hi);
 //                when the rows are dequantized FP16 values (exact in TF32,
@@ -140,9 +139,7 @@ enum BKind : int { kBSplit = 0, kBExact = 1, kBF16W = 3, kBF16S = 4 };
 // k-step (a kind::f16 MMA covers twice the K of a TF32 one in the same time).
 // Both operands are K-major FP16 tiles with the 128-byte swizzle: a k-block is
 // 64 wide (128 bytes per row), a stage holds the weights' hi and mid tiles and
-// this CTA's rows (3 x 16 KB), 4 stages.  Both CTAs' loads of a stage complete
-// on the leader CTA's barrier (cta_group::2 TMA), which the MMA issuer waits
-// on directly: there is no splitter hand-off on this path.
+// this CTA's rows (3 x 16 KB), 4 stages.
 constexpr int BK16 = 64;
 constexpr int kStages16 = 4, kStages16S = 3;
 constexpr uint32_t kTile16Bytes = BM * BK16 * 2;          // 16 KB: 128 rows x 128 bytes
@@ -150,6 +147,7 @@ constexpr uint32_t kStage16Bytes = 3 * kTile16Bytes;      // A hi | A mid | B
 constexpr uint32_t kStage16SBytes = 4 * kTile16Bytes;     // A hi | A mid | B hi | B mid
 static_assert(kStages16 * kStage16Bytes <= kStages * kStageBytes, "the FP16 ring fits the same shared memory");
 static_assert(kStages16S * kStage16SBytes <= kStages * kStageBytes, "the FP16 ring fits the same shared memory");
+static_assert(kStages16 <= kNumSplitWarps && kStages16S <= kNumSplitWarps, "one relay warp per FP16 stage");
 template <int kBK> __host__ __device__ constexpr bool f16_path() { return kBK == kBF16W || kBK == kBF16S; }
 template <int kBK> __host__ __device__ constexpr int ring_stages() {
   return kBK == kBF16W ? kStages16 : (kBK == kBF16S ? kStages16S : kStages);
@@ -226,28 +224,6 @@ __device__ __forceinline__ bool mbar_wait(Smem* s, uint64_t* bar, uint32_t parit
     }
   }
 }
-// Loads of either CTA of the pair that signal the leader CTA's barrier
-// (bar_cl: its shared::cluster address), so one barrier tracks both CTAs'
-// tiles of a stage (the kind::f16 path).  No multicast.
-__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_t bar_cl, void* dst, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2 [%0], [%1, {%3, %4}], [%2];"
-      ::"r"(smem_u32(dst)), "l"(map), "r"(bar_cl), "r"(c0), "r"(c1)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_3d_pair(const CUtensorMap* map, uint32_t bar_cl, void* dst, int c0, int c1,
-                                                 int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2 [%0], [%1, {%3, %4, %5}], [%2];"
-      ::"r"(smem_u32(dst)), "l"(map), "r"(bar_cl), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-__device__ __forceinline__ uint32_t leader_addr(const void* p) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(0));
-  return remote;
-}
-
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int c0, int c1) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
@@ -756,18 +732,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
               // the weights' hi and mid tiles (expert e and E + e of the split
               // tensor) and this CTA's rows (kBF16S: their hi and mid planes,
               // rows r and R + r), 64 k wide, 128-byte swizzle
-              // Both CTAs' loads complete on the leader's full[st], which the
-              // MMA issuer waits on: the leader expects the pair's bytes.  (A
-              // peer's bytes may land before the leader's expect: the phase
-              // cannot complete while the leader's arrival is pending.)
               const int row = c.n0 + (int)rank * (c.n_mma / 2);
-              const uint32_t bar = leader_addr(&s->full[st]);
-              if (rank == 0) mbar_arrive_expect_tx(&s->full[st], 2 * kRingBytes);
-              tma_load_3d_pair(&mapA, bar, base, kb * BK16, c.m0, c.e);
-              tma_load_3d_pair(&mapA, bar, base + kTile16Bytes, kb * BK16, c.m0, E + c.e);
-              tma_load_2d_pair(&mapB, bar, base + 2 * kTile16Bytes, kb * BK16, row);
+              mbar_arrive_expect_tx(&s->full[st], kRingBytes);
+              tma_load_3d(&mapA, &s->full[st], base, kb * BK16, c.m0, c.e);
+              tma_load_3d(&mapA, &s->full[st], base + kTile16Bytes, kb * BK16, c.m0, E + c.e);
+              tma_load_2d(&mapB, &s->full[st], base + 2 * kTile16Bytes, kb * BK16, row);
               if (kBK == kBF16S)
-                tma_load_2d_pair(&mapB, bar, base + 3 * kTile16Bytes, kb * BK16, (int)args.rows + row);
+                tma_load_2d(&mapB, &s->full[st], base + 3 * kTile16Bytes, kb * BK16, (int)args.rows + row);
               continue;
             }
             mbar_arrive_expect_tx(&s->full[st], kTxBytes);
@@ -794,10 +765,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
             }
           }
         }
-        // the last issued loads must land before the CTA may exit (FP16 path:
-        // the leader's barriers track both CTAs' loads, and the peer waits for
-        // the leader at the final cluster barrier)
-        const uint32_t n_last = (f16_path<kBK>() && rank != 0) ? 0u : (it < (uint32_t)kRing ? it : (uint32_t)kRing);
+        // the last issued loads must land before the CTA may exit
+        const uint32_t n_last = it < (uint32_t)kRing ? it : (uint32_t)kRing;
         for (uint32_t j = 0; j < n_last; ++j) {
           const uint32_t i2 = it - 1 - j, st = i2 % kRing, use = i2 / kRing;
           const long long t0 = clock64();
@@ -828,12 +797,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
             const int c1 = min(c0 + kChunk, tnk);
             for (int kb = c0; kb < c1; ++kb, ++it) {
               const uint32_t st = it % kRing, use = it / kRing;
-              // the landed stage: split in both CTAs (3xTF32), or both CTAs'
-              // loads complete on this barrier (FP16 path)
-              if (!mbar_wait(s, f16_path<kBK>() ? &s->full[st] : &s->split[st], use & 1, args.err)) {
-                ok = false;
-                break;
-              }
+              if (!mbar_wait(s, &s->split[st], use & 1, args.err)) { ok = false; break; }
               tc_fence_after();
               if (f16_path<kBK>()) {
                 // K-major FP16 tiles, 128-byte swizzle: 8-row groups 1024 B
@@ -919,8 +883,20 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       static_assert(kVec % (32 * kBatch) == 0, "split batches divide the stage");
       uint32_t it = 0;
       bool ok = true;
-      // FP16 path: nothing to split, and the MMA issuer waits on the TMA
-      // barrier itself; these warps are idle
+      if (f16_path<kBK>()) {
+        // nothing to split: warp ci relays stage ci's landing (its own CTA's
+        // TMA) to the leader's MMA issuer, one fixed warp per stage
+        for (int tile = blockIdx.x / 2; tile < total && ok && ci < kRing; tile += n_pairs) {
+          const TileCoord c = decode_tile<kMode>(s, args, n_tiles_n, nk, tile, rank);
+          for (int kb = 0; kb < c.nk; ++kb, ++it) {
+            if ((int)(it % kRing) != ci) continue;
+            const uint32_t st = it % kRing, use = it / kRing;
+            if (!mbar_wait(s, &s->full[st], use & 1, args.err)) { ok = false; break; }
+            __syncwarp();
+            if (lane == 0) mbar_arrive_leader(&s->split[st], rank);
+          }
+        }
+      }
       for (int tile = blockIdx.x / 2; !f16_path<kBK>() && tile < total && ok; tile += n_pairs) {
         const TileCoord c = decode_tile<kMode>(s, args, n_tiles_n, nk, tile, rank);
         for (int kb = 0; kb < c.nk; ++kb, ++it) {
