@@ -226,25 +226,31 @@ class ClockSampler:
 # launches), from ncu captures of a smaller case of the same workload scaled
 # to full size by its routed rows; valid only for the kernel source it was
 # taken on (else reported as null).
+GEMM_SRC_END = "// ---- the FP16 split of the weights for the kind::f16 GEMMs"
 GEMM_TRAFFIC = {
     # the M-shaped MoE layer (the slice's) captured at 12,288 and 16,384 atoms
     # on the FP16 path, each launch kind fitted as a + b * rows and taken to
-    # the workload's R; mean of the step's four launches
-    ("slice", "3xtf32"): {"src": "element_routed_moe_b200/csrc/ffn_tc.cu", "sha256_prefix": "bbf7aa89a7737e0f",
-                          "bytes_per_launch": 6.678e+09},
-    ("M", "3xtf32"): {"src": "element_routed_moe_b200/csrc/ffn_tc.cu", "sha256_prefix": "bbf7aa89a7737e0f",
-                      "bytes_per_launch": 3.492e+09},
+    # the workload's R; mean of the step's four launches.  The hash covers the
+    # GEMM kernel and its launch code: ffn_tc.cu up to the weight-split section.
+    ("slice", "3xtf32"): {"src": "element_routed_moe_b200/csrc/ffn_tc.cu", "upto": GEMM_SRC_END,
+                          "sha256_prefix": "7741159dda9b1309", "bytes_per_launch": 6.678e+09},
+    ("M", "3xtf32"): {"src": "element_routed_moe_b200/csrc/ffn_tc.cu", "upto": GEMM_SRC_END,
+                      "sha256_prefix": "7741159dda9b1309", "bytes_per_launch": 3.492e+09},
 }
 
 
 def measured_traffic(workload: str, mode: str):
+    """The recorded DRAM bytes per GEMM launch, or None once the GEMM's source
+    (the file up to the marker) differs from the one the counters came from."""
     import hashlib
     rec = GEMM_TRAFFIC.get((workload, mode))
     if rec is None:
         return None
     with open(os.path.join(ROOT, rec["src"]), "rb") as f:
-        if hashlib.sha256(f.read()).hexdigest()[:16] != rec["sha256_prefix"]:
-            return None
+        src = f.read()
+    end = src.find(rec["upto"].encode())
+    if end < 0 or hashlib.sha256(src[:end]).hexdigest()[:16] != rec["sha256_prefix"]:
+        return None
     return rec["bytes_per_launch"]
 
 
