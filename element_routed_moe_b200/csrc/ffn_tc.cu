@@ -1234,50 +1234,63 @@ __global__ void __launch_bounds__(256) w16_split_cols_kernel(const float* __rest
 }
 
 // x W^T: W [E][N][Kd] is K-major already: one warp per (row, K chunk of 256),
-// two float4 per lane, the chunk's maximum by shuffles, then hi and mid.
+// two float4 per lane, the chunk's maximum by shuffles, then hi and mid; a
+// warp loads two such items before working on either.
 __global__ void __launch_bounds__(256) w16_split_rows_kernel(const float4* __restrict__ w, int64_t rows, int Kd,
                                                              int N, uint2* __restrict__ w16,
                                                              float* __restrict__ winv) {
+  constexpr int kItems = 2, kU = kChunkK / 128;
   const int lane = threadIdx.x % 32;
   const int k4 = Kd / 4, nch = (Kd + kChunkK - 1) / kChunkK;
   const int64_t items = rows * nch;
   uint2* __restrict__ mid = w16 + rows * k4;
   const int64_t nw = (int64_t)gridDim.x * 8;
   const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int64_t it = ((int64_t)blockIdx.x * 256 + threadIdx.x) / 32; it < items; it += nw) {
-    const int64_t r = it / nch;
-    const int ci = (int)(it % nch);
-    const int64_t base = r * k4;
-    float4 v[kChunkK / 128];
+  for (int64_t it0 = ((int64_t)blockIdx.x * 256 + threadIdx.x) / 32; it0 < items; it0 += kItems * nw) {
+    float4 v[kItems][kU];
 #pragma unroll
-    for (int u = 0; u < kChunkK / 128; ++u) {
-      const int c = ci * (kChunkK / 4) + u * 32 + lane;
-      v[u] = c < k4 ? __ldcs(w + base + c) : zero;
-    }
-    uint32_t m = 0;
+    for (int q = 0; q < kItems; ++q) {
+      const int64_t it = it0 + q * nw;
+      const int64_t base = (it / nch) * k4;
+      const int cb = (int)(it % nch) * (kChunkK / 4);
 #pragma unroll
-    for (int u = 0; u < kChunkK / 128; ++u)
-      m = max(m, max(max(__float_as_uint(v[u].x) & 0x7fffffffu, __float_as_uint(v[u].y) & 0x7fffffffu),
-                     max(__float_as_uint(v[u].z) & 0x7fffffffu, __float_as_uint(v[u].w) & 0x7fffffffu)));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const int ex = w16_scale_exp(m);
-    const float S = __uint_as_float((uint32_t)(127 + ex) << 23);
-    if (lane == 0) {
-      const int64_t e = r / N, n = r % N;
-      winv[(e * nch + ci) * N + n] = __uint_as_float((uint32_t)(127 - ex) << 23);
+      for (int u = 0; u < kU; ++u) {
+        const int c = cb + u * 32 + lane;
+        v[q][u] = (it < items && c < k4) ? __ldcs(w + base + c) : zero;
+      }
     }
 #pragma unroll
-    for (int u = 0; u < kChunkK / 128; ++u) {
-      const int c = ci * (kChunkK / 4) + u * 32 + lane;
-      if (c < k4) {
-        float4 o = v[u];
-        o.x *= S; o.y *= S; o.z *= S; o.w *= S;
-        const uint2 hq = make_uint2(half2_bits(o.x, o.y), half2_bits(o.z, o.w));
-        const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hq.x));
-        const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hq.y));
-        __stcs(w16 + base + c, hq);
-        __stcs(mid + base + c, make_uint2(half2_bits(o.x - h0.x, o.y - h0.y), half2_bits(o.z - h1.x, o.w - h1.y)));
+    for (int q = 0; q < kItems; ++q) {
+      const int64_t it = it0 + q * nw;
+      if (it >= items) break;                       // the same in every lane
+      const int64_t r = it / nch;
+      const int ci = (int)(it % nch);
+      const int64_t base = r * k4;
+      uint32_t m = 0;
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        m = max(m, max(max(__float_as_uint(v[q][u].x) & 0x7fffffffu, __float_as_uint(v[q][u].y) & 0x7fffffffu),
+                       max(__float_as_uint(v[q][u].z) & 0x7fffffffu, __float_as_uint(v[q][u].w) & 0x7fffffffu)));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const int ex = w16_scale_exp(m);
+      const float S = __uint_as_float((uint32_t)(127 + ex) << 23);
+      if (lane == 0) {
+        const int64_t e = r / N, n = r % N;
+        winv[(e * nch + ci) * N + n] = __uint_as_float((uint32_t)(127 - ex) << 23);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = ci * (kChunkK / 4) + u * 32 + lane;
+        if (c < k4) {
+          float4 o = v[q][u];
+          o.x *= S; o.y *= S; o.z *= S; o.w *= S;
+          const uint2 hq = make_uint2(half2_bits(o.x, o.y), half2_bits(o.z, o.w));
+          const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hq.x));
+          const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hq.y));
+          __stcs(w16 + base + c, hq);
+          __stcs(mid + base + c, make_uint2(half2_bits(o.x - h0.x, o.y - h0.y), half2_bits(o.z - h1.x, o.w - h1.y)));
+        }
       }
     }
   }
