@@ -742,8 +742,8 @@ def run_ep(args, world, rank, local):
     r_recv = int(layer.layout[2][rank][-1].item())
     ffn_ms = ph_ms["ffn_fwd"] + ph_ms["ffn_vjp"]
     # the owner's first forward GEMM runs on the received FP16 rows: 2 products
-    kinds = [("f16", 2) if layer.fused_unpack else ("tf32", 2), ("f16", 3) if layer.f16_second else ("tf32", 3),
-             ("tf32", 3), ("tf32", 3)]
+    kinds = [("f16", 2) if layer.fused_unpack else ("tf32", 2), ("f16", 3) if layer.f16_second else ("tf32", 3)]
+    kinds += [("f16", 3)] * 2 if layer.split_vjp else [("tf32", 3)] * 2
     roof = gemm_roofline(J, mode, cfg, kinds, peaks, peak_src, 2.0 * r_recv * d * h, max(ffn_ms, 1e-9), 4)
     roof.update({"kernel": "grouped expert-MLP GEMM (rank 0's experts; ffn phases include the FP16 unpack)",
                  "traffic": None})

@@ -81,6 +81,12 @@ class ExpertParallelLayer:
         f16_first = self.fused_unpack and mode == J.JANUS_FFN_3XTF32
         self.f16_second = f16_first and h % 8 == 0 and cap >= 2048 * self.El
         self.launches_per_step += (1 if f16_first else 0) + (2 if self.f16_second else 0)
+        # the VJP on the FP16 tensor path at the same size: the received
+        # gradient rows split into two FP16 terms (row maxima + split), then
+        # W2's split, dH, dA's split, W1's split, dA W1^T in place of 2 GEMMs
+        self.split_vjp = (mode == J.JANUS_FFN_3XTF32 and d % 8 == 0 and h % 8 == 0
+                          and cap >= 2048 * self.El)
+        self.launches_per_step += 5 if self.split_vjp else 0
         self.payload = torch.empty((cap, d), dtype=torch.float16, device=self.dev)
         self.row_scale = torch.empty((cap,), **f32)
         self.recv_rows = torch.empty((cap, d), **f32)       # gradients in, outputs out
@@ -89,6 +95,14 @@ class ExpertParallelLayer:
         self.yd = torch.empty((cap, d), **f32)
         self.ret = torch.empty((rows, d), **f32)             # this rank's rows coming back
         self.ret_rows = torch.zeros((cap,), dtype=torch.int64, device=self.dev)   # fused-return row table
+        if self.split_vjp:
+            self.gd16 = torch.empty((2 * cap, d), dtype=torch.float16, device=self.dev)
+            self.gd_scale = torch.empty((cap,), **f32)
+            self.ident = torch.arange(cap, dtype=torch.int32, device=self.dev)
+            self.split_ws = torch.empty(J.janus_dispatch_split_workspace_size(cap), dtype=torch.uint8,
+                                        device=self.dev)
+            self.vjp_ws = torch.empty(J.janus_expert_ffn_split_workspace_size(cap, self.El, d, h),
+                                      dtype=torch.uint8, device=self.dev)
         self.counts_all = torch.empty((self.world, n_experts), dtype=torch.int32, device=self.dev)
         # error word of the sends (both directions): rows past the capacity
         self.send_ws = torch.empty(J.janus_quant_by_type_workspace_size(n_types), dtype=torch.uint8,
@@ -226,7 +240,16 @@ class ExpertParallelLayer:
         m(events, "send_vjp", 1)
         recv_off = self.layout[2][self.rank]
         m(events, "ffn_vjp", 0)
-        if self.fused_return:
+        if self.split_vjp:
+            # every receive row is split (the ones past this step's rows are
+            # never read by the GEMMs); the results go through the return
+            # table (fused) or into yd
+            J.janus_dispatch_split(self.recv_rows, self.ident, 1, out=self.gd16, row_scale=self.gd_scale,
+                                   workspace=self.split_ws)
+            out = dict(out_rows=self.ret_rows) if self.fused_return else dict(out=self.yd)
+            J.janus_expert_ffn_vjp_split(self.gd16, self.gd_scale, recv_off, self.w1, self.w2, self.act,
+                                         workspace=self.vjp_ws, **out)
+        elif self.fused_return:
             J.janus_expert_ffn_vjp_rows(self.xd, self.recv_rows, recv_off, self.w1, self.w2, self.ret_rows,
                                         act=self.act, mode=self.mode)
         else:

@@ -310,3 +310,26 @@ def test_ep_capacity_overflow_is_reported_and_stays_in_bounds():
         n = min(int(recv_ref[o, -1]), cap)
         assert torch.equal(pay[o][:n].view(torch.int16), pay_f[o][:n].view(torch.int16)), o
         assert torch.equal(rsc[o][:n], rsc_f[o][:n]), o
+
+
+@pytest.mark.parametrize("fused", [True, False])
+def test_ep_layer_fp16_path_one_rank(fused):
+    # one rank owning every expert, sized so that the owner's expert MLP runs
+    # on the FP16 tensor path in both directions (>= 2048 receive rows per
+    # local expert): the layer's y and dX against its own local chain
+    from element_routed_moe_b200.ep import ExpertParallelLayer
+    N, T, E, K, d, h = 2100, 13, 2, 2, 64, 64
+    gate = to_dev(synth.gate_table(T, E, 41))
+    w1, w2 = synth.expert_weights(E, d, h, 42, DEV)
+    x = synth.normal((N, d), 43, DEV)
+    types = to_dev(synth.types_zipf(N, T, seed=44))
+    g = synth.normal((N, d), 45, DEV)
+    layer = ExpertParallelLayer(N, d, h, T, E, K, w1, w2, mode=J.JANUS_FFN_3XTF32, device=DEV,
+                                fused_return=fused, capacity_factor=1.0)
+    assert layer.f16_second and layer.split_vjp
+    y = layer.forward(x, types, gate)
+    dx = layer.vjp(g)
+    torch.cuda.synchronize()
+    y_ref, dx_ref = _local_chain(x, types, gate, K, w1, w2, J.JANUS_FFN_3XTF32, g)
+    assert rel_fro(host(y), host(y_ref)) <= TOL_FP32 and rel_fro(host(dx), host(dx_ref)) <= TOL_FP32
+    layer.close()
