@@ -231,25 +231,33 @@ GEMM_TRAFFIC = {
     # the M-shaped MoE layer (the slice's) captured at 12,288 and 16,384 atoms
     # on the FP16 path, each launch kind fitted as a + b * rows and taken to
     # the workload's R; mean of the step's four launches.  The hash covers the
-    # GEMM kernel and its launch code: ffn_tc.cu up to the weight-split section.
+    # GEMM kernel and its launch code (ffn_tc.cu up to the weight-split
+    # section) without its comments.
     ("slice", "3xtf32"): {"src": "element_routed_moe_b200/csrc/ffn_tc.cu", "upto": GEMM_SRC_END,
-                          "sha256_prefix": "7741159dda9b1309", "bytes_per_launch": 6.678e+09},
+                          "sha256_prefix": "9a893657e4daa214", "bytes_per_launch": 6.678e+09},
     ("M", "3xtf32"): {"src": "element_routed_moe_b200/csrc/ffn_tc.cu", "upto": GEMM_SRC_END,
-                      "sha256_prefix": "7741159dda9b1309", "bytes_per_launch": 3.492e+09},
+                      "sha256_prefix": "9a893657e4daa214", "bytes_per_launch": 3.492e+09},
 }
 
 
-def measured_traffic(workload: str, mode: str):
-    """The recorded DRAM bytes per GEMM launch, or None once the GEMM's source
-    (the file up to the marker) differs from the one the counters came from."""
+def code_hash(text: str) -> str:
+    """sha256 prefix of source text with its // comments and blank lines removed."""
     import hashlib
+    import re
+    lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+    return hashlib.sha256("\n".join(ln for ln in lines if ln).encode()).hexdigest()[:16]
+
+
+def measured_traffic(workload: str, mode: str):
+    """The recorded DRAM bytes per GEMM launch, or None once the GEMM's code
+    (the file up to the marker) differs from the code the counters came from."""
     rec = GEMM_TRAFFIC.get((workload, mode))
     if rec is None:
         return None
-    with open(os.path.join(ROOT, rec["src"]), "rb") as f:
+    with open(os.path.join(ROOT, rec["src"])) as f:
         src = f.read()
-    end = src.find(rec["upto"].encode())
-    if end < 0 or hashlib.sha256(src[:end]).hexdigest()[:16] != rec["sha256_prefix"]:
+    end = src.find(rec["upto"])
+    if end < 0 or code_hash(src[:end]) != rec["sha256_prefix"]:
         return None
     return rec["bytes_per_launch"]
 

@@ -1,7 +1,8 @@
 // Grouped expert-MLP GEMM on the 5th-generation tensor cores (tcgen05), for
 // JANUS_FFN_3XTF32: the 3xTF32 split on kind::tf32, and (kBF16W / kBF16S
 // below) an FP16 form on kind::f16 for rows that arrive as FP16 values or as
-// two FP16 terms: the FP16-packed dispatch and the split dispatch.
+// two FP16 terms: the FP16-packed dispatch, the split dispatch and the
+// activations' row split (act_split_blk_kernel below).
 //
 // FP32 accuracy from TF32 tensor cores (Ootomo & Yokota 2022, "Recovering
 // single precision accuracy from Tensor Cores while surpassing the FP32
@@ -129,12 +130,13 @@ enum BKind : int { kBSplit = 0, kBExact = 1, kBF16W = 3, kBF16S = 4 };
 
 // kBF16W: FP16 rows x FP16-split weights on tcgen05 kind::f16.
 // A packed row is q * s (q binary16, s a power of two), exact in FP16 up to
-// its scale.  Each weight column f of expert e is scaled by a power of two S
-// that puts its largest magnitude in [2^14, 2^15) and split into two FP16
-// terms, w S = hi + mid + r with |r| <= 2^-22 |w S| (the split the weight
-// pass below writes).  The tensor core multiplies FP16 operands exactly and
-// accumulates in FP32, so
-//   a[p, f] = s_p / S_f * sum_k q[p, k] (hi[f, k] + mid[f, k])
+// its scale.  Each weight column f of expert e is scaled, per K chunk c of
+// 256, by a power of two S_fc that puts the chunk's largest magnitude in
+// [2^14, 2^15) and split into two FP16 terms, w S_fc = hi + mid + r with
+// |r| <= 2^-22 |w S_fc| (the split the weight kernels below write).  The
+// tensor core multiplies FP16 operands exactly and accumulates each chunk in
+// FP32, and the epilogue scales each chunk's sum as it folds it, so
+//   a[p, f] = s_p * sum_c (1 / S_fc) sum_{k in c} q[p, k] (hi[f, k] + mid[f, k])
 // is as accurate as the 3xTF32 product, with two kind::f16 MMAs per 16-wide
 // k-step (a kind::f16 MMA covers twice the K of a TF32 one in the same time).
 // Both operands are K-major FP16 tiles with the 128-byte swizzle: a k-block is
