@@ -198,7 +198,22 @@ dispatch_split_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int c = c0 + u * 32 + lane;
-      if (c < d4) v[u] = __ldcs(x + i * d4 + c);
+      v[u] = c < d4 ? __ldcs(x + i * d4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // unweighted: every destination gets the same two terms, split once
+    uint2 hq0[kU], mq0[kU];
+    const int e0 = split_exp(__float_as_uint(m));
+    if (!kWeighted) {
+      const float S = __uint_as_float((uint32_t)(127 + e0) << 23);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        float4 o = v[u];
+        o.x *= S; o.y *= S; o.z *= S; o.w *= S;
+        hq0[u] = halves(o.x, o.y, o.z, o.w);
+        const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hq0[u].x));
+        const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hq0[u].y));
+        mq0[u] = halves(o.x - h0.x, o.y - h0.y, o.z - h1.x, o.w - h1.y);
+      }
     }
     for (int k = 0; k < K; ++k) {
       int64_t p;
@@ -208,15 +223,20 @@ dispatch_split_kernel(const float4* __restrict__ x, int64_t n_atoms, int d4, int
         if (lane == 0) debug_fault(dbg);
         continue;
       }
-      const int e = split_exp(__float_as_uint(kWeighted ? fabsf(wk) * m : m));
+      const int e = kWeighted ? split_exp(__float_as_uint(fabsf(wk) * m)) : e0;
       const float S = __uint_as_float((uint32_t)(127 + e) << 23);
       if (c0 == 0 && lane == 0) row_scale[p] = __uint_as_float((uint32_t)(127 - e) << 23);
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
         const int c = c0 + u * 32 + lane;
         if (c < d4) {
+          if (!kWeighted) {
+            rows16[p * d4 + c] = hq0[u];
+            mid_plane[p * d4 + c] = mq0[u];
+            continue;
+          }
           float4 o = v[u];
-          if (kWeighted) { o.x *= wk; o.y *= wk; o.z *= wk; o.w *= wk; }
+          o.x *= wk; o.y *= wk; o.z *= wk; o.w *= wk;
           o.x *= S; o.y *= S; o.z *= S; o.w *= S;
           const uint2 hq = halves(o.x, o.y, o.z, o.w);
           const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hq.x));
