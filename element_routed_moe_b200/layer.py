@@ -10,21 +10,22 @@ packing of the dispatch, edge aggregation in front of the MoE block) and
 One pass, all on the current stream:
     [edge_aggregate]  X = segment sums of the edge messages (row_ptr given)
     route             per-type top-K, counts, offsets, permutation
-    dispatch          Xd = X rows in expert order   (or FP16 pack, unpacked by the GEMM)
+    dispatch          Xd = X rows in expert order   (or FP16 pack, fed to the GEMM as it is)
     ffn_fwd           Yd = silu(Xd W1[e]) W2[e]      (a saved)
     combine           Y  = sum_k w * Yd
     dispatch_w        Gd = w * G rows in expert order
     ffn_vjp           dXd = ((Gd W2^T) * silu'(a)) W1^T
     combine_vjp       dX = sum_k dXd
 
-In 3xTF32 mode the forward's first GEMM runs on the FP16 tensor path:
-FP16-packed rows go to janus_expert_ffn_fwd_packed as they are; unpacked rows
-are dispatched as two FP16 terms with a per-row scale (janus_dispatch_split)
-for janus_expert_ffn_fwd_split when the layer has at least SPLIT_MIN_ROWS_PER_EXPERT
-routed rows per expert (below that, re-splitting the weights every call costs
-more than the GEMM saves).  The VJP stays on 3xTF32: its first GEMM is bound
-by the dSiLU epilogue, and the FP16 form (janus_expert_ffn_vjp_split) measured
-no faster.
+In 3xTF32 mode the expert MLP runs on the FP16 tensor path where it pays:
+FP16-packed rows always go to janus_expert_ffn_fwd_packed as they are (its
+first GEMM on kind::f16); with at least SPLIT_MIN_ROWS_PER_EXPERT routed rows
+per expert (and d, h multiples of 8) unpacked rows are dispatched as two FP16
+terms with a per-row scale (janus_dispatch_split) for
+janus_expert_ffn_fwd_split, the gradient's weighted dispatch is split the same
+way for janus_expert_ffn_vjp_split, and the library runs every GEMM of both
+directions on kind::f16.  Below that size, re-splitting the weights every call
+costs more than the FP16 GEMMs save, and the layer stays on 3xTF32.
 
 `run_host` runs the pass from and to pinned host memory with the copies on
 their own streams: the upload of G overlaps the forward, the download of Y
