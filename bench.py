@@ -7,7 +7,7 @@ with the edge aggregation in front where the workload has edges (tiny, L, the
 interaction-block slice) and the per-element-type FP16 packing in place of the
 dispatch where it packs (M, the slice; the payload feeds the first GEMM as it
 is).  --mode 3xtf32 (the default) is the FP32-accurate tensor-core mode: the
-expert GEMMs run on 3xTF32, or, at >= 2048 rows per expert, on the two-term
+expert GEMMs run on 3xTF32, or, from 384 rows per expert, on the two-term
 FP16 path; --mode simt runs them as FP32 FFMA.
 
 Metric: routed atom-expert tokens/s (tokens = N*K routed rows) per layer pass.

@@ -91,8 +91,9 @@ unpack_rows_kernel(const uint2* __restrict__ payload, const float* __restrict__ 
 // The MLP's second GEMM (H W2 in the forward, dA W1^T in the split VJP)
 // runs on the kind::f16 path too when the layer has at least this many
 // routed rows per expert: the activation's row split and the per-call split
-// of the weights then cost less than the GEMM saves.
-constexpr int64_t kF16SecondMinRowsPerExpert = 2048;
+// of the weights then cost less than the GEMMs save (measured break-even near
+// 380 rows per expert; the S-shaped layer, 455, gains 8 %).
+constexpr int64_t kF16SecondMinRowsPerExpert = 384;
 bool use_f16_second(int64_t R, int32_t E, int32_t h) {
   return h % 8 == 0 && R >= kF16SecondMinRowsPerExpert * E;
 }
@@ -132,6 +133,8 @@ size_t packed_extra(int64_t R, int32_t E, int32_t d, int32_t h, janus_ffn_mode m
 }  // namespace janus
 
 using namespace janus;
+
+extern "C" int32_t janus_expert_ffn_f16_min_rows_per_expert(void) { return (int32_t)kF16SecondMinRowsPerExpert; }
 
 extern "C" janus_status janus_expert_ffn_packed_workspace_size(int64_t n_rows, int32_t n_experts, int32_t d,
                                                                int32_t h, janus_ffn_mode mode, size_t* bytes) {

@@ -74,18 +74,19 @@ class ExpertParallelLayer:
         # this library's kernels per forward + VJP: route 4, layout 1, pack 2,
         # expert MLP 2 + 2, FP32 send 1, combine 1 + 1, the unpack 1 (when not
         # fused), and the return table (fused) or the return copy twice; the
-        # fused 3xTF32 forward adds W1's split (1) and, at >= 2048 receive
-        # rows per local expert and h % 8 == 0, the FP16 second GEMM's row
-        # split (1) and W2's split (1)
+        # fused 3xTF32 forward adds W1's split (1) and, from the library's row
+        # threshold per local expert (receive capacity) with h % 8 == 0, the
+        # FP16 second GEMM's row split (1) and W2's split (1)
         self.launches_per_step = 14 + (0 if self.fused_unpack else 1) + (1 if self.fused_return else 2)
         f16_first = self.fused_unpack and mode == J.JANUS_FFN_3XTF32
-        self.f16_second = f16_first and h % 8 == 0 and cap >= 2048 * self.El
+        min_rows = J.janus_expert_ffn_f16_min_rows_per_expert()
+        self.f16_second = f16_first and h % 8 == 0 and cap >= min_rows * self.El
         self.launches_per_step += (1 if f16_first else 0) + (2 if self.f16_second else 0)
         # the VJP on the FP16 tensor path at the same size: the received
         # gradient rows split into two FP16 terms (row maxima + split), then
         # W2's split, dH, dA's split, W1's split, dA W1^T in place of 2 GEMMs
         self.split_vjp = (mode == J.JANUS_FFN_3XTF32 and d % 8 == 0 and h % 8 == 0
-                          and cap >= 2048 * self.El)
+                          and cap >= min_rows * self.El)
         self.launches_per_step += 5 if self.split_vjp else 0
         self.payload = torch.empty((cap, d), dtype=torch.float16, device=self.dev)
         self.row_scale = torch.empty((cap,), **f32)

@@ -38,7 +38,7 @@ SYMBOLS = (
     "janus_dequant_by_type", "janus_dispatch_row_scales",
     "janus_expert_ffn_workspace_size", "janus_expert_ffn_fwd", "janus_expert_ffn_vjp",
     "janus_expert_ffn_fwd_rows", "janus_expert_ffn_vjp_rows", "janus_expert_ffn_fwd_ex",
-    "janus_expert_ffn_packed_workspace_size", "janus_expert_ffn_fwd_packed",
+    "janus_expert_ffn_packed_workspace_size", "janus_expert_ffn_fwd_packed", "janus_expert_ffn_f16_min_rows_per_expert",
     "janus_expert_ffn_split_workspace_size", "janus_expert_ffn_fwd_split", "janus_expert_ffn_vjp_split",
     "janus_expert_ffn_weight_grad_workspace_size", "janus_expert_ffn_weight_grad",
     "janus_expert_ffn_vjp_vjp_workspace_size", "janus_expert_ffn_vjp_vjp",
@@ -132,6 +132,7 @@ def _declare(L):
         "janus_expert_ffn_fwd_ex": (st, [vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, ctypes.c_uint32,
                                          ctypes.c_int, vp, sz, vp]),
         "janus_expert_ffn_packed_workspace_size": (st, [i64, i32, i32, i32, ctypes.c_int, psz]),
+        "janus_expert_ffn_f16_min_rows_per_expert": (i32, []),
         "janus_expert_ffn_fwd_packed": (st, [vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, ctypes.c_int,
                                              vp, sz, vp]),
         "janus_expert_ffn_split_workspace_size": (st, [i64, i32, i32, i32, psz]),
@@ -674,6 +675,12 @@ def janus_expert_ffn_packed_workspace_size(n_rows, n_experts, d, h, mode=JANUS_F
     return b.value
 
 
+def janus_expert_ffn_f16_min_rows_per_expert() -> int:
+    """Rows per expert from which the packed and split MLP calls run both GEMMs
+    of a direction on the FP16 tensor path (the library's rule)."""
+    return int(lib().janus_expert_ffn_f16_min_rows_per_expert())
+
+
 def janus_expert_ffn_fwd_packed(payload, row_scale, offsets, w1, w2, *, out=None, out_rows=None,
                                 mode=JANUS_FFN_FP32_SIMT, want_act=False, act=None, workspace=None, stream=None):
     """The forward on the FP16 payload [R,d] with per-row scales [R] (3xTF32
@@ -712,8 +719,9 @@ def janus_expert_ffn_split_workspace_size(n_rows, n_experts, d, h) -> int:
 def janus_expert_ffn_fwd_split(rows16, row_scale, offsets, w1, w2, *, out=None, out_rows=None, want_act=False,
                                act=None, workspace=None, stream=None):
     """The forward on split rows (janus_dispatch_split): the first GEMM on the
-    FP16 tensor path, the second on 3xTF32, or on the FP16 path too at >= 2048
-    rows per expert with h % 8 == 0.  Returns (out-or-None, act-or-None)."""
+    FP16 tensor path, the second on 3xTF32, or on the FP16 path too from
+    janus_expert_ffn_f16_min_rows_per_expert() rows per expert with h % 8 == 0.
+    Returns (out-or-None, act-or-None)."""
     R2, d = rows16.shape
     R = R2 // 2
     E, _, h = w1.shape
@@ -740,7 +748,8 @@ def janus_expert_ffn_vjp_split(gd16, gd_scale, offsets, w1, w2, act, *, out=None
     """The input VJP on split upstream-gradient rows (janus_dispatch_split,
     weighted) and the forward's pre-activations: dA = (gd W2^T) silu'(a) on
     the FP16 tensor path, dxd = dA W1^T on 3xTF32, or on the FP16 path too at
-    >= 2048 rows per expert with h % 8 == 0.  Returns out-or-None."""
+    janus_expert_ffn_f16_min_rows_per_expert() rows per expert with h % 8 == 0.
+    Returns out-or-None."""
     R2, d = gd16.shape
     R = R2 // 2
     E, _, h = w1.shape

@@ -52,7 +52,7 @@ class MoELayer:
     # the FP16 tensor path: row maxima + split dispatch; W1's split in front
     # of the two GEMMs
     LAUNCHES_SPLIT = {"dispatch": 2, "ffn_fwd": 3}
-    SPLIT_MIN_ROWS_PER_EXPERT = 2048
+    SPLIT_MIN_ROWS_PER_EXPERT = None   # the library's rule (janus_expert_ffn_f16_min_rows_per_expert)
 
     # pinned-host pipeline for edge-message inputs: ring of device buffers
     RING_SLOTS = 8
@@ -92,12 +92,14 @@ class MoELayer:
         # 3xTF32, unpacked rows: the forward's first GEMM on the FP16 tensor
         # path (rows split into two FP16 terms by the dispatch; d % 8 == 0)
         # when the rows per expert amortise the per-call weight split
+        min_rows = (J.janus_expert_ffn_f16_min_rows_per_expert() if self.SPLIT_MIN_ROWS_PER_EXPERT is None
+                    else self.SPLIT_MIN_ROWS_PER_EXPERT)
         self.split = (mode == J.JANUS_FFN_3XTF32 and not packed and d % 8 == 0
-                      and R >= self.SPLIT_MIN_ROWS_PER_EXPERT * E)
+                      and R >= min_rows * E)
         # the input VJP on the FP16 tensor path (both GEMMs; the weighted
         # dispatch writes the gradient rows as two FP16 terms) on the same rule
         self.split_vjp = (mode == J.JANUS_FFN_3XTF32 and d % 8 == 0 and h % 8 == 0
-                          and R >= self.SPLIT_MIN_ROWS_PER_EXPERT * E)
+                          and R >= min_rows * E)
         nb = max(J.janus_expert_ffn_workspace_size(R, d, h, E, False, True, mode),
                  J.janus_expert_ffn_workspace_size(R, d, h, E, True, True, mode),
                  J.janus_expert_ffn_packed_workspace_size(R, E, d, h, mode) if self.fused_unpack else 0,
@@ -130,10 +132,11 @@ class MoELayer:
         if self.packed and self.fused_unpack and mode == J.JANUS_FFN_3XTF32:
             launches["ffn_fwd"] = 3           # W1's split + the two GEMMs
         # the library also runs the forward's second GEMM on the FP16 path
-        # (with H's row split and W2's split in front) at >= 2048 rows per
-        # expert and h % 8 == 0, after either FP16 first GEMM
+        # (with H's row split and W2's split in front) from its row threshold
+        # per expert with h % 8 == 0, after either FP16 first GEMM
         fp16_first = self.split or (self.packed and self.fused_unpack and mode == J.JANUS_FFN_3XTF32)
-        self.f16_second = fp16_first and h % 8 == 0 and R >= 2048 * E
+        self.f16_second = (fp16_first and h % 8 == 0
+                           and R >= J.janus_expert_ffn_f16_min_rows_per_expert() * E)
         if self.f16_second:
             launches["ffn_fwd"] += 2          # H's row split + W2's split
         if self.split_vjp:

@@ -313,7 +313,7 @@ janus_status janus_expert_ffn_fwd_ex(const float* xd, const int32_t* offsets, in
  * with exact FP16 products and FP32 accumulation per chunk (the chunks of the
  * 3xTF32 GEMM): FP32-accurate, within 1e-5 of the unpacked FP32 forward, at
  * half the tensor-core work of the two-product TF32 form.  The second GEMM
- * (H W2) runs on 3xTF32, or, when n_rows >= 2048 * n_experts and h % 8 == 0,
+ * (H W2) runs on 3xTF32, or, when n_rows >= M * n_experts and h % 8 == 0,
  * on the same kind::f16 path with three products: the first GEMM then
  * stores a only, one pass over each row writes H = silu(a) as two FP16 terms
  * with a per-row power-of-two scale into the workspace, and W2 is split like
@@ -326,6 +326,12 @@ janus_status janus_expert_ffn_fwd_ex(const float* xd, const int32_t* offsets, in
  * n_experts through the weight split), 256-byte aligned. */
 janus_status janus_expert_ffn_packed_workspace_size(int64_t n_rows, int32_t n_experts, int32_t d, int32_t h,
                                                     janus_ffn_mode mode, size_t* bytes);
+/* M, the rows per expert (n_rows / n_experts) from which the packed and split
+ * MLP calls run their second GEMM on the kind::f16 path too (384): below it
+ * the per-call splits of the weights and the activation cost more than the
+ * FP16 GEMMs save.  Callers choosing between the 3xTF32 and the split entry
+ * points can use the same rule. */
+int32_t janus_expert_ffn_f16_min_rows_per_expert(void);
 janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, const float* row_scale, const int32_t* offsets,
                                          int32_t n_experts, int64_t n_rows, int32_t d, int32_t h, const float* w1,
                                          const float* w2, float* yd, float* const* yd_rows, float* act,
@@ -347,7 +353,7 @@ janus_status janus_expert_ffn_vjp_rows(const float* xd, const float* gd, const f
  * terms, as in janus_expert_ffn_fwd_packed); products are exact and
  * accumulate in FP32 per chunk, each chunk's sum is scaled by the feature's
  * 1 / S for that chunk, and the result by row_scale[p].  The second GEMM (H W2, or dA W1^T) runs on 3xTF32, or, with
- * n_rows >= 2048 * n_experts and h % 8 == 0, on the same kind::f16 path: the
+ * n_rows >= M * n_experts and h % 8 == 0, on the same kind::f16 path: the
  * first GEMM then stores a (fwd) or dH = gd W2^T (vjp) plainly, and one pass
  * over each row writes H = silu(a), or dA = dH * silu'(a), as two FP16 terms
  * with a per-row power-of-two scale into the workspace, after which the

@@ -315,8 +315,9 @@ def test_ep_capacity_overflow_is_reported_and_stays_in_bounds():
 @pytest.mark.parametrize("fused", [True, False])
 def test_ep_layer_fp16_path_one_rank(fused):
     # one rank owning every expert, sized so that the owner's expert MLP runs
-    # on the FP16 tensor path in both directions (>= 2048 receive rows per
-    # local expert): the layer's y and dX against its own local chain
+    # on the FP16 tensor path in both directions (receive rows per local
+    # expert above the library's threshold): the layer's y and dX against its
+    # own local chain
     from element_routed_moe_b200.ep import ExpertParallelLayer
     N, T, E, K, d, h = 2100, 13, 2, 2, 64, 64
     gate = to_dev(synth.gate_table(T, E, 41))

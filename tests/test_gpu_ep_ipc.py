@@ -54,6 +54,7 @@ def _worker(rank, world, port, mode, fused, q):
                                     w2[rank * El:(rank + 1) * El].contiguous(), mode=mode, device=dev,
                                     fused_return=fused)
         errs = []
+        fp16 = bool(layer.f16_second or layer.split_vjp)
         for _ in range(2):                                  # buffers reused across passes
             y = layer.forward(x, types, gate)
             dx = layer.vjp(g)
@@ -71,7 +72,7 @@ def _worker(rank, world, port, mode, fused, q):
                          rel_fro(dx.cpu().numpy(), dx_ref.cpu().numpy())))
         layer.close()
         dist.destroy_process_group()
-        q.put((rank, "ok", errs))
+        q.put((rank, "ok", (fp16, errs)))
     except Exception as e:  # report, do not hang the parent
         q.put((rank, "error", repr(e)))
 
@@ -90,6 +91,12 @@ def test_ep_layer_two_processes_through_ipc(mode, fused):
         p.join(timeout=60)
     for rank, status, payload in results:
         assert status == "ok", (rank, payload)
-        for ey, edx in payload:
-            assert ey <= 1e-6 and edx <= 1e-6, (rank, ey, edx)
+        fp16, errs = payload
+        # same arithmetic as the local chain: 1e-6 (summation order only); a
+        # receive capacity above the FP16 tensor path's row threshold puts the
+        # owner's MLP on FP16 products while the chain (fewer rows per expert)
+        # stays on 3xTF32, both within 1e-5 of the FP32 result
+        tol = 1e-5 if fp16 else 1e-6
+        for ey, edx in errs:
+            assert ey <= tol and edx <= tol, (rank, fp16, ey, edx)
     assert all(p.exitcode == 0 for p in procs)

@@ -102,7 +102,7 @@ PACKED = {
     "M_like": (4096, 89, 40, 8, 512, 384),
     "tails": (257, 5, 9, 2, 8, 4),
     "wide_k": (300, 7, 3, 2, 1544, 200),       # 24 full 64-wide k-blocks + an 8-wide tail
-    # >= 2048 rows per expert and h % 8 == 0: the second GEMM (H W2) runs on
+    # above the library's rows-per-expert threshold, h % 8 == 0: the second GEMM (H W2) runs on
     # the FP16 path too, over a 200-wide K (three 64-wide blocks + an 8 tail)
     "second_f16": (3200, 9, 3, 2, 136, 200),
 }

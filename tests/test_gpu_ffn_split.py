@@ -4,7 +4,7 @@ janus_dispatch_split writes each dispatch row as two binary16 terms with a
 per-row power-of-two scale; janus_expert_ffn_fwd_split / _vjp_split run the
 first GEMM of each direction on the tcgen05 kind::f16 path (three products
 against a two-term FP16 split of the weights) and the second on 3xTF32, or,
-in the forward at >= 2048 rows per expert, on the same FP16 path
+in the forward above the library's rows-per-expert threshold, on the same FP16 path
 (paper review 'Breaking the Training Barrier of Billion-Parameter Universal
 Machine Learning Interatomic Potentials', section 3.1 Table II and section 3.3:
 the expert MLP and its input gradient, FP32-accurate).
@@ -82,7 +82,7 @@ SHAPES = {
     "multi_tile": ([700, 900, 400], 512, 384),
     "k_tail": ([300, 257], 1544, 200),
     "narrow": ([5, 3, 260], 8, 4),
-    # >= 2048 rows per expert, h % 8 == 0: the forward's second GEMM on the
+    # above the rows-per-expert threshold, h % 8 == 0: the forward's second GEMM on the
     # FP16 path too (K = h = 200: three 64-wide blocks and an 8-wide tail)
     "second_f16": ([3000, 0, 3300], 136, 200),
     # rows of more than 4096 values: the activation and weight-row splits
@@ -161,7 +161,7 @@ def test_split_forward_full_size_sampled_rows():
 
 
 def test_fp16_second_gemms_handle_wide_ranges():
-    # at >= 2048 rows per expert both second GEMMs run on FP16: H W2 with W2
+    # above the rows-per-expert threshold both second GEMMs run on FP16: H W2 with W2
     # split per output feature d, dA W1^T with W1 split per output feature d
     # (a row of W1[e]).  Output features whose weights are 10^6 or 10^-30
     # times the rest, or all zero, stay within the FP32 tolerance column by

@@ -117,7 +117,7 @@ def test_random_shape_edges(seed):
 
 @pytest.mark.parametrize("seed", range(8))
 def test_random_shape_fp16_second_gemms(seed):
-    # >= 2048 rows per expert with d, h % 8 == 0: both GEMMs of each direction
+    # >= 2048 rows per expert (above the library's threshold) with d, h % 8 == 0: both GEMMs of each direction
     # on the FP16 tensor path (split rows, the FP16 payload for the packed
     # forward), on ragged segments and random widths with K tails
     g = np.random.default_rng(2000 + seed)
