@@ -465,13 +465,16 @@ def split_bytes(cfg, layer):
     """Algorithmic bytes of one launch of each traced split kind: the
     activation split reads a (and dH for dSiLU) once and writes the two FP16
     planes and a scale per row; the weight split reads one expert matrix and
-    writes its two FP16 planes and a scale per output feature."""
+    writes its two FP16 planes and a scale per output feature; the split of
+    both orientations reads it once and writes four planes and both scale
+    tables."""
     R, d, h, E = cfg.n_rows, cfg.d, cfg.h, cfg.n_experts
     return {
         "act_split silu": 4 * R * h + 4 * R * h + 4 * R,
         "act_split dsilu": 8 * R * h + 4 * R * h + 4 * R,
         "w16_split transposed": 4 * E * d * h + 4 * E * d * h + 4 * E * max(d, h),
         "w16_split rows": 4 * E * d * h + 4 * E * d * h + 4 * E * max(d, h),
+        "w16_split both": 4 * E * d * h + 8 * E * d * h + 8 * E * max(d, h),
     }
 
 

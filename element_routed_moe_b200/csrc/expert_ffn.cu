@@ -129,12 +129,94 @@ size_t packed_extra(int64_t R, int32_t E, int32_t d, int32_t h, janus_ffn_mode m
          (use_f16_second(R, E, h) ? f16_second_bytes(R, E, d, h) : 0);
 }
 
+// The weight splits of a layer written ahead of its MLP calls
+// (janus_expert_weights_f16): four parts, each the planes [2][E][N][Kd]
+// FP16 then 1 / S [E][ceil(Kd/256)][N]:
+//   0  W1 for x W1     (Kd = d, N = h)   forward, first GEMM
+//   1  W2 for H W2     (Kd = h, N = d)   forward, second GEMM
+//   2  W2 for gd W2^T  (Kd = d, N = h)   input VJP, first GEMM
+//   3  W1 for dA W1^T  (Kd = h, N = d)   input VJP, second GEMM
+struct W16Set {
+  size_t off_w16[4], off_winv[4], total;
+};
+W16Set w16_set_layout(int32_t E, int32_t d, int32_t h) {
+  W16Set S;
+  const int32_t kd[4] = {d, h, d, h}, nn[4] = {h, d, h, d};
+  size_t off = 0;
+  for (int i = 0; i < 4; ++i) {
+    S.off_w16[i] = off;
+    off += align_up(2 * sizeof(uint16_t) * (size_t)E * d * h, 256);
+    S.off_winv[i] = off;
+    off += winv_bytes(E, kd[i], nn[i]);
+  }
+  S.total = off;
+  return S;
+}
+// The pointers of part `i` (first GEMM) and `i + 1` (second GEMM).
+void w16_set_parts(const void* set, int32_t E, int32_t d, int32_t h, int i, uint16_t** w16, float** winv,
+                   tc::F16Second* second) {
+  const W16Set S = w16_set_layout(E, d, h);
+  char* b = (char*)set;
+  *w16 = (uint16_t*)(b + S.off_w16[i]);
+  *winv = (float*)(b + S.off_winv[i]);
+  second->w16 = (uint16_t*)(b + S.off_w16[i + 1]);
+  second->winv = (float*)(b + S.off_winv[i + 1]);
+}
+janus_status check_w16_set(const void* set, size_t bytes, int32_t E, int32_t d, int32_t h) {
+  if (!set) return JANUS_OK;
+  JANUS_CHECK_ALIGN(aligned(set, 256));
+  JANUS_CHECK_ARG(bytes >= w16_set_layout(E, d, h).total);
+  return JANUS_OK;
+}
+
 }  // namespace
 }  // namespace janus
 
 using namespace janus;
 
 extern "C" int32_t janus_expert_ffn_f16_min_rows_per_expert(void) { return (int32_t)kF16SecondMinRowsPerExpert; }
+
+extern "C" janus_status janus_expert_weights_f16_size(int32_t n_experts, int32_t d, int32_t h, size_t* bytes) {
+  JANUS_CHECK_ARG(bytes && n_experts >= 1 && n_experts <= kMaxExperts);
+  JANUS_CHECK_ARG(d >= 1 && d <= kMaxDim && h >= 1 && h <= kMaxDim);
+  *bytes = w16_set_layout(n_experts, d, h).total;
+  return JANUS_OK;
+}
+
+extern "C" janus_status janus_expert_weights_f16(const float* w1, const float* w2, int32_t n_experts, int32_t d,
+                                                 int32_t h, uint32_t which, void* out, size_t out_bytes,
+                                                 janus_stream_t stream_) {
+  cudaStream_t stream = (cudaStream_t)stream_;
+  JANUS_CHECK_ARG(n_experts >= 1 && n_experts <= kMaxExperts);
+  JANUS_CHECK_ARG(d >= 1 && d <= kMaxDim && h >= 1 && h <= kMaxDim);
+  JANUS_CHECK_ARG(which >= 1 && which <= (JANUS_W16_FWD | JANUS_W16_VJP));
+  JANUS_CHECK_ALIGN(d % 8 == 0 && h % 4 == 0);
+  JANUS_CHECK_ARG(w1 && w2 && out);
+  JANUS_CHECK_ALIGN(aligned(w1, 16) && aligned(w2, 16) && aligned(out, 256));
+  const W16Set S = w16_set_layout(n_experts, d, h);
+  JANUS_CHECK_ARG(out_bytes >= S.total);
+  if (consume_injected_failure()) return JANUS_ERR_CUDA;
+  char* b = (char*)out;
+  auto w16 = [&](int i) { return (uint16_t*)(b + S.off_w16[i]); };
+  auto winv = [&](int i) { return (float*)(b + S.off_winv[i]); };
+  janus_status st = JANUS_OK;
+  if (which == (JANUS_W16_FWD | JANUS_W16_VJP)) {
+    // W1 [E][d][h]: x W1's split (part 0) and dA W1^T's (part 3); W2 [E][h][d]:
+    // H W2's (part 1) and gd W2^T's (part 2), each weight read once
+    st = tc::split_weights_f16_both(w1, n_experts, d, h, w16(0), winv(0), w16(3), winv(3), stream);
+    if (st == JANUS_OK)
+      st = tc::split_weights_f16_both(w2, n_experts, h, d, w16(1), winv(1), w16(2), winv(2), stream);
+    return st != JANUS_OK ? st : launch_status();
+  }
+  if (which & JANUS_W16_FWD) {
+    st = tc::split_weights_f16(w1, n_experts, d, h, true, w16(0), winv(0), stream);
+    if (st == JANUS_OK) st = tc::split_weights_f16(w2, n_experts, h, d, true, w16(1), winv(1), stream);
+  } else {
+    st = tc::split_weights_f16(w2, n_experts, d, h, false, w16(2), winv(2), stream);
+    if (st == JANUS_OK) st = tc::split_weights_f16(w1, n_experts, h, d, false, w16(3), winv(3), stream);
+  }
+  return st != JANUS_OK ? st : launch_status();
+}
 
 extern "C" janus_status janus_expert_ffn_packed_workspace_size(int64_t n_rows, int32_t n_experts, int32_t d,
                                                                int32_t h, janus_ffn_mode mode, size_t* bytes) {
@@ -148,6 +230,7 @@ extern "C" janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, con
                                                     const int32_t* offsets, int32_t n_experts, int64_t n_rows,
                                                     int32_t d, int32_t h, const float* w1, const float* w2,
                                                     float* yd, float* const* yd_rows, float* act,
+                                                    const void* weights16, size_t weights16_bytes,
                                                     janus_ffn_mode mode, void* workspace, size_t workspace_bytes,
                                                     janus_stream_t stream_) {
   cudaStream_t stream = (cudaStream_t)stream_;
@@ -160,6 +243,9 @@ extern "C" janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, con
   JANUS_CHECK_ARG(n_rows == 0 || row_scale);
   JANUS_CHECK_ALIGN(mode != JANUS_FFN_3XTF32 || d % 8 == 0);   // FP16 rows: 16-byte TMA strides
   JANUS_CHECK_ALIGN(act == nullptr || aligned(act, 16));
+  JANUS_CHECK_ARG(weights16 == nullptr || mode == JANUS_FFN_3XTF32);
+  st = check_w16_set(weights16, weights16_bytes, n_experts, d, h);
+  if (st != JANUS_OK) return st;
   const FfnLayout L = ffn_layout(n_rows, h, false, true);
   const size_t extra = packed_extra(n_rows, n_experts, d, h, mode);
   JANUS_CHECK_ARG(workspace && workspace_bytes >= L.total + extra);
@@ -175,10 +261,11 @@ extern "C" janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, con
     const size_t w16_bytes = align_up(2 * sizeof(uint16_t) * (size_t)n_experts * d * h, 256);
     float* winv = (float*)((char*)workspace + L.total + w16_bytes);
     char* second_base = (char*)workspace + L.total + w16_bytes + winv_bytes(n_experts, d, h);
-    const tc::F16Second second = f16_second_at(second_base, n_rows, n_experts, d, h);
+    tc::F16Second second = f16_second_at(second_base, n_rows, n_experts, d, h);
+    if (weights16) w16_set_parts(weights16, n_experts, d, h, 0, &w16, &winv, &second);
     st = tc::expert_ffn_fwd_packed(payload, row_scale, offsets, n_experts, n_rows, d, h, w1, w2, yd, act, H, w16,
                                    winv, &((WsHeader*)workspace)->error, stream, yd_rows,
-                                   use_f16_second(n_rows, n_experts, h) ? &second : nullptr);
+                                   use_f16_second(n_rows, n_experts, h) ? &second : nullptr, weights16 != nullptr);
     if (st != JANUS_OK) return st;
     return launch_status();
   }
@@ -199,7 +286,7 @@ extern "C" janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, con
 // The expert MLP on rows given as two FP16 terms with a per-row scale
 // (janus_dispatch_split): the first GEMM of the forward (x W1) or of the VJP
 // (gd W2^T) on the kind::f16 tensor path; the second on 3xTF32, or on the
-// kind::f16 path at >= 2048 rows per expert with h % 8 == 0.  Workspace:
+// kind::f16 path from kF16SecondMinRowsPerExpert rows per expert with h % 8 == 0.  Workspace:
 // header | H, dH or dA [R,h] | the FP16 split of the first GEMM's weights
 // (hi and mid, [E][h][d] each) | 1 / S [E][ceil(d/256)][h] | the FP16 second GEMM's
 // scratch when it is used.
@@ -245,7 +332,8 @@ extern "C" janus_status janus_expert_ffn_split_workspace_size(int64_t n_rows, in
 extern "C" janus_status janus_expert_ffn_fwd_split(const uint16_t* rows16, const float* row_scale,
                                                    const int32_t* offsets, int32_t n_experts, int64_t n_rows,
                                                    int32_t d, int32_t h, const float* w1, const float* w2,
-                                                   float* yd, float* const* yd_rows, float* act, void* workspace,
+                                                   float* yd, float* const* yd_rows, float* act,
+                                                   const void* weights16, size_t weights16_bytes, void* workspace,
                                                    size_t workspace_bytes, janus_stream_t stream_) {
   cudaStream_t stream = (cudaStream_t)stream_;
   JANUS_CHECK_ARG((yd == nullptr) != (yd_rows == nullptr) || n_rows == 0);
@@ -254,16 +342,20 @@ extern "C" janus_status janus_expert_ffn_fwd_split(const uint16_t* rows16, const
                                 workspace_bytes);
   if (st != JANUS_OK) return st;
   JANUS_CHECK_ALIGN(act == nullptr || aligned(act, 16));
+  st = check_w16_set(weights16, weights16_bytes, n_experts, d, h);
+  if (st != JANUS_OK) return st;
   if (n_rows == 0) return JANUS_OK;
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
   const SplitLayout L = split_layout(n_rows, n_experts, d, h);
   char* w = (char*)workspace;
   JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
-  const tc::F16Second second = f16_second_at(w + L.off_second, n_rows, n_experts, d, h);
+  tc::F16Second second = f16_second_at(w + L.off_second, n_rows, n_experts, d, h);
+  uint16_t* w16 = (uint16_t*)(w + L.off_w16);
+  float* winv = (float*)(w + L.off_winv);
+  if (weights16) w16_set_parts(weights16, n_experts, d, h, 0, &w16, &winv, &second);
   st = tc::expert_ffn_fwd_split(rows16, row_scale, offsets, n_experts, n_rows, d, h, w1, w2, yd, act,
-                                (float*)(w + L.off_h), (uint16_t*)(w + L.off_w16), (float*)(w + L.off_winv),
-                                &((WsHeader*)workspace)->error, stream, yd_rows,
-                                use_f16_second(n_rows, n_experts, h) ? &second : nullptr);
+                                (float*)(w + L.off_h), w16, winv, &((WsHeader*)workspace)->error, stream, yd_rows,
+                                use_f16_second(n_rows, n_experts, h) ? &second : nullptr, weights16 != nullptr);
   if (st != JANUS_OK) return st;
   return launch_status();
 }
@@ -271,7 +363,8 @@ extern "C" janus_status janus_expert_ffn_fwd_split(const uint16_t* rows16, const
 extern "C" janus_status janus_expert_ffn_vjp_split(const uint16_t* gd16, const float* gd_scale, const float* act,
                                                    const int32_t* offsets, int32_t n_experts, int64_t n_rows,
                                                    int32_t d, int32_t h, const float* w1, const float* w2,
-                                                   float* dxd, float* const* dxd_rows, void* workspace,
+                                                   float* dxd, float* const* dxd_rows, const void* weights16,
+                                                   size_t weights16_bytes, void* workspace,
                                                    size_t workspace_bytes, janus_stream_t stream_) {
   cudaStream_t stream = (cudaStream_t)stream_;
   JANUS_CHECK_ARG((dxd == nullptr) != (dxd_rows == nullptr) || n_rows == 0);
@@ -281,16 +374,20 @@ extern "C" janus_status janus_expert_ffn_vjp_split(const uint16_t* gd16, const f
   if (st != JANUS_OK) return st;
   JANUS_CHECK_ARG(n_rows == 0 || act);
   JANUS_CHECK_ALIGN(act == nullptr || aligned(act, 16));
+  st = check_w16_set(weights16, weights16_bytes, n_experts, d, h);
+  if (st != JANUS_OK) return st;
   if (n_rows == 0) return JANUS_OK;
   if (consume_injected_failure()) return JANUS_ERR_CUDA;
   const SplitLayout L = split_layout(n_rows, n_experts, d, h);
   char* w = (char*)workspace;
   JANUS_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(WsHeader), stream));
-  const tc::F16Second second = f16_second_at(w + L.off_second, n_rows, n_experts, d, h);
+  tc::F16Second second = f16_second_at(w + L.off_second, n_rows, n_experts, d, h);
+  uint16_t* w16 = (uint16_t*)(w + L.off_w16);
+  float* winv = (float*)(w + L.off_winv);
+  if (weights16) w16_set_parts(weights16, n_experts, d, h, 2, &w16, &winv, &second);
   st = tc::expert_ffn_vjp_split(gd16, gd_scale, act, offsets, n_experts, n_rows, d, h, w1, w2, dxd,
-                                (float*)(w + L.off_h), (uint16_t*)(w + L.off_w16), (float*)(w + L.off_winv),
-                                &((WsHeader*)workspace)->error, stream, dxd_rows,
-                                use_f16_second(n_rows, n_experts, h) ? &second : nullptr);
+                                (float*)(w + L.off_h), w16, winv, &((WsHeader*)workspace)->error, stream, dxd_rows,
+                                use_f16_second(n_rows, n_experts, h) ? &second : nullptr, weights16 != nullptr);
   if (st != JANUS_OK) return st;
   return launch_status();
 }

@@ -1298,6 +1298,166 @@ __global__ void __launch_bounds__(256) w16_split_rows_kernel(const float4* __res
   }
 }
 
+// Both orientations of one weight tensor W [E][A][B] from one DRAM read of W,
+// for a layer whose forward and input VJP use the same weights:
+//   T, the split for x W  (Kd = A, N = B): planes [E][B][A], winvT [E][ceil(A/256)][B];
+//   R, the split for x W^T (N = A, Kd = B): planes [E][A][B], winvR [E][ceil(B/256)][A];
+// bit for bit what w16_split_cols_kernel and w16_split_rows_kernel write.  A
+// CTA takes 256 x 256 blocks of one expert.  The first sweep reads the block
+// for its 256 row maxima (R's scales, chunk = the block's columns) and 256
+// column maxima (T's scales, chunk = its rows) and writes nothing; the second
+// reads it again, from L2 (two CTAs per SM: about 76 MB of blocks are live),
+// in 256-row x 32-column strips, the next strip's loads in flight while the
+// current one is written: R's terms go out from the registers and T's through
+// a shared-memory transpose, as in the transposing kernel.  Two CTAs per SM
+// let one CTA's loads overlap the other's stores.  DRAM traffic: W once, the
+// four planes once.
+constexpr int kBothThreads = 256, kBothWarps = kBothThreads / 32;
+__global__ void __launch_bounds__(kBothThreads, 2) w16_split_both_kernel(const float* __restrict__ w, int E, int A,
+                                                                         int B, __half* __restrict__ w16t,
+                                                                         float* __restrict__ winvt,
+                                                                         __half* __restrict__ w16r,
+                                                                         float* __restrict__ winvr) {
+  __shared__ uint32_t s_cmax[kChunkK];                     // column maxima (|w| bits)
+  __shared__ float s_rs[kChunkK], s_cs[kChunkK];
+  __shared__ __align__(16) __half t_hi[32][kChunkK + 2];
+  __shared__ __align__(16) __half t_mid[32][kChunkK + 2];
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int tx = tid % 8, ty = tid / 8;                   // sweep 2: 4 columns, rows ty + 32 u
+  const int nca = (A + kChunkK - 1) / kChunkK, ncb = (B + kChunkK - 1) / kChunkK, b4 = B / 4;
+  const int64_t n_blocks = (int64_t)E * nca * ncb;
+  const int64_t plane = (int64_t)E * A * B;
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  constexpr int kRowsPerWarp = kChunkK / kBothWarps, kStripRows = kChunkK / 32;
+  if (tid < kChunkK) s_cmax[tid] = 0u;                      // reset again as each block reads it
+  __syncthreads();
+  for (int64_t t = blockIdx.x; t < n_blocks; t += gridDim.x) {
+    const int cb = (int)(t % ncb);
+    const int64_t t1 = t / ncb;
+    const int ca = (int)(t1 % nca), e = (int)(t1 / nca);
+    const int a0 = ca * kChunkK, b0 = cb * kChunkK;
+    const float* we = w + (int64_t)e * A * B;
+    const int n_strips = min(kChunkK, B - b0 + 31) / 32;   // strips with a column in range
+    // sweep 1: warp w takes the block's rows w + 8 i (i < 32), four at a
+    // time; lane l holds the float4 columns l and l + 32 of the block's 64
+    uint32_t cm[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
+#pragma unroll 1
+    for (int i0 = 0; i0 < kRowsPerWarp; i0 += 4) {
+      float4 v[4][2];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int a = a0 + warp + kBothWarps * (i0 + q);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int c = b0 / 4 + lane + 32 * u;
+          v[q][u] = (a < A && c < b4) ? __ldcg(reinterpret_cast<const float4*>(we + (int64_t)a * B) + c) : zero;
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const uint32_t x = __float_as_uint(v[q][u].x) & 0x7fffffffu, y = __float_as_uint(v[q][u].y) & 0x7fffffffu;
+          const uint32_t z = __float_as_uint(v[q][u].z) & 0x7fffffffu, ww = __float_as_uint(v[q][u].w) & 0x7fffffffu;
+          cm[u][0] = max(cm[u][0], x); cm[u][1] = max(cm[u][1], y);
+          cm[u][2] = max(cm[u][2], z); cm[u][3] = max(cm[u][3], ww);
+          m = max(m, max(max(x, y), max(z, ww)));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) {
+          const int ar = warp + kBothWarps * (i0 + q), ex = w16_scale_exp(m);
+          s_rs[ar] = __uint_as_float((uint32_t)(127 + ex) << 23);
+          if (a0 + ar < A) winvr[((int64_t)e * ncb + cb) * A + a0 + ar] = __uint_as_float((uint32_t)(127 - ex) << 23);
+        }
+      }
+    }
+    // the first strip's loads go out before the column maxima meet
+    float4 v[kStripRows];
+    auto load_strip = [&](int sp, float4* dst) {
+      const int bc = b0 + 32 * sp + 4 * tx;
+      const bool col_ok = bc < B;                          // B % 4 == 0: all four columns
+#pragma unroll
+      for (int u = 0; u < kStripRows; ++u) {
+        const int a = a0 + ty + 32 * u;
+        dst[u] = (col_ok && a < A) ? __ldcs(reinterpret_cast<const float4*>(we + (int64_t)a * B + bc)) : zero;
+      }
+    };
+    load_strip(0, v);
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (cm[u][j]) atomicMax(&s_cmax[4 * (lane + 32 * u) + j], cm[u][j]);
+    __syncthreads();
+    if (tid < kChunkK) {
+      const uint32_t mm = s_cmax[tid];
+      s_cmax[tid] = 0u;
+      const int ex = w16_scale_exp(mm);
+      s_cs[tid] = __uint_as_float((uint32_t)(127 + ex) << 23);
+      if (b0 + tid < B) winvt[((int64_t)e * nca + ca) * B + b0 + tid] = __uint_as_float((uint32_t)(127 - ex) << 23);
+    }
+    __syncthreads();
+    // sweep 2: strip sp's values in v, strip sp + 1's loads in flight
+#pragma unroll 1
+    for (int sp = 0; sp < n_strips; ++sp) {
+      const int bs = b0 + 32 * sp, bc = bs + 4 * tx;
+      const bool col_ok = bc < B;
+      float4 vn[kStripRows];
+      if (sp + 1 < n_strips) load_strip(sp + 1, vn);
+      float cs[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) cs[j] = s_cs[32 * sp + 4 * tx + j];
+#pragma unroll
+      for (int u = 0; u < kStripRows; ++u) {
+        const int ar = ty + 32 * u, a = a0 + ar;
+        // R: the row's scale, both terms stored from the registers
+        const float S = s_rs[ar];
+        float4 o = v[u];
+        o.x *= S; o.y *= S; o.z *= S; o.w *= S;
+        const uint2 hq = make_uint2(half2_bits(o.x, o.y), half2_bits(o.z, o.w));
+        const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hq.x));
+        const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hq.y));
+        if (col_ok && a < A) {
+          const int64_t at = ((int64_t)e * A + a) * B + bc;
+          __stcs(reinterpret_cast<uint2*>(w16r + at), hq);
+          __stcs(reinterpret_cast<uint2*>(w16r + plane + at),
+                 make_uint2(half2_bits(o.x - h0.x, o.y - h0.y), half2_bits(o.z - h1.x, o.w - h1.y)));
+        }
+        // T: the column scales, transposed through shared memory
+        const float val[4] = {v[u].x * cs[0], v[u].y * cs[1], v[u].z * cs[2], v[u].w * cs[3]};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half hi = __float2half_rn(val[j]);
+          t_hi[4 * tx + j][ar] = hi;
+          t_mid[4 * tx + j][ar] = __float2half_rn(val[j] - __half2float(hi));
+        }
+      }
+      __syncthreads();
+      // each warp writes four features' 256 values of a as half2 pairs
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int fl = warp * 4 + j, fo = bs + fl;
+        if (fo >= B) continue;
+        const int64_t row = ((int64_t)e * B + fo) * A;
+#pragma unroll
+        for (int q = 0; q < kChunkK / 64; ++q) {
+          const int kk = 2 * (lane + 32 * q), ao = a0 + kk;
+          if (ao < A) {                                       // A % 4 == 0: ao + 1 < A too
+            __stcs(reinterpret_cast<__half2*>(w16t + row + ao), *reinterpret_cast<const __half2*>(&t_hi[fl][kk]));
+            __stcs(reinterpret_cast<__half2*>(w16t + plane + row + ao),
+                   *reinterpret_cast<const __half2*>(&t_mid[fl][kk]));
+          }
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < kStripRows; ++u) v[u] = vn[u];
+    }
+  }
+}
+
 // ---- the FP16 row split of an activation for a kind::f16 GEMM ---------------
 // v = silu(a) (kActSilu) or x silu'(a) (kActDSilu), with the SiLU arithmetic
 // of the GEMM epilogues, written as hi and mid binary16 planes
@@ -1517,6 +1677,17 @@ janus_status split_weights_f16(const float* w, int32_t E, int32_t Kd, int32_t N,
   return launch_status();
 }
 
+janus_status split_weights_f16_both(const float* w, int32_t E, int32_t A, int32_t B, uint16_t* w16t, float* winvt,
+                                    uint16_t* w16r, float* winvr, cudaStream_t stream) {
+  TraceScope trace("w16_split both", stream);
+  if (A % 4 != 0 || B % 4 != 0) return JANUS_ERR_MISALIGNED;
+  const int64_t n_blocks = (int64_t)E * ((A + kChunkK - 1) / kChunkK) * ((B + kChunkK - 1) / kChunkK);
+  const int64_t blocks = std::min<int64_t>(n_blocks, (int64_t)num_sms() * 2);   // two CTAs per SM
+  w16_split_both_kernel<<<(unsigned)blocks, kBothThreads, 0, stream>>>(
+      w, E, A, B, reinterpret_cast<__half*>(w16t), winvt, reinterpret_cast<__half*>(w16r), winvr);
+  return launch_status();
+}
+
 size_t workspace_extra() { return 0; }
 
 janus_status expert_ffn_fwd(const float* xd, const int32_t* offsets, int32_t E, int64_t R, int32_t d,
@@ -1543,8 +1714,8 @@ template <int kBK>
 janus_status fwd_f16(const uint16_t* rows, const float* row_scale, const int32_t* offsets, int32_t E, int64_t R,
                      int32_t d, int32_t h, const float* w1, const float* w2, float* yd, float* act, float* H,
                      uint16_t* w16, float* winv, int32_t* err, cudaStream_t stream, float* const* yd_rows,
-                     const F16Second* second) {
-  janus_status st = split_weights_f16(w1, E, d, h, true, w16, winv, stream);
+                     const F16Second* second, bool presplit) {
+  janus_status st = presplit ? JANUS_OK : split_weights_f16(w1, E, d, h, true, w16, winv, stream);
   if (st != JANUS_OK) return st;
   const float* xq = reinterpret_cast<const float*>(rows);
   const float* wq = reinterpret_cast<const float*>(w16);
@@ -1561,7 +1732,7 @@ janus_status fwd_f16(const uint16_t* rows, const float* row_scale, const int32_t
   if (st != JANUS_OK) return st;
   st = act_split_f16<kActSilu>(nullptr, A, R, h, second->h16, second->hscale, stream);
   if (st != JANUS_OK) return st;
-  st = split_weights_f16(w2, E, h, d, true, second->w16, second->winv, stream);
+  if (!presplit) st = split_weights_f16(w2, E, h, d, true, second->w16, second->winv, stream);
   if (st != JANUS_OK) return st;
   return launch<kModeNN, kEpiStore, kBF16S>(reinterpret_cast<const float*>(second->h16),
                                             reinterpret_cast<const float*>(second->w16), R, E, h, d, yd, nullptr,
@@ -1573,26 +1744,28 @@ janus_status fwd_f16(const uint16_t* rows, const float* row_scale, const int32_t
 janus_status expert_ffn_fwd_packed(const uint16_t* payload, const float* row_scale, const int32_t* offsets,
                                    int32_t E, int64_t R, int32_t d, int32_t h, const float* w1, const float* w2,
                                    float* yd, float* act, float* H, uint16_t* w16, float* winv, int32_t* err,
-                                   cudaStream_t stream, float* const* yd_rows, const F16Second* second) {
+                                   cudaStream_t stream, float* const* yd_rows, const F16Second* second,
+                                   bool weights_presplit) {
   return fwd_f16<kBF16W>(payload, row_scale, offsets, E, R, d, h, w1, w2, yd, act, H, w16, winv, err, stream,
-                         yd_rows, second);
+                         yd_rows, second, weights_presplit);
 }
 
 janus_status expert_ffn_fwd_split(const uint16_t* rows16, const float* row_scale, const int32_t* offsets, int32_t E,
                                   int64_t R, int32_t d, int32_t h, const float* w1, const float* w2, float* yd,
                                   float* act, float* H, uint16_t* w16, float* winv, int32_t* err,
-                                  cudaStream_t stream, float* const* yd_rows, const F16Second* second) {
+                                  cudaStream_t stream, float* const* yd_rows, const F16Second* second,
+                                  bool weights_presplit) {
   return fwd_f16<kBF16S>(rows16, row_scale, offsets, E, R, d, h, w1, w2, yd, act, H, w16, winv, err, stream,
-                         yd_rows, second);
+                         yd_rows, second, weights_presplit);
 }
 
 janus_status expert_ffn_vjp_split(const uint16_t* gd16, const float* gd_scale, const float* act,
                                   const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
                                   const float* w1, const float* w2, float* dxd, float* dA, uint16_t* w16,
                                   float* winv, int32_t* err, cudaStream_t stream, float* const* dxd_rows,
-                                  const F16Second* second) {
+                                  const F16Second* second, bool weights_presplit) {
   // gd W2^T: W2 [E][h][d] is K-major for this product as it stands
-  janus_status st = split_weights_f16(w2, E, d, h, false, w16, winv, stream);
+  janus_status st = weights_presplit ? JANUS_OK : split_weights_f16(w2, E, d, h, false, w16, winv, stream);
   if (st != JANUS_OK) return st;
   const float* gq = reinterpret_cast<const float*>(gd16);
   const float* wq = reinterpret_cast<const float*>(w16);
@@ -1611,7 +1784,7 @@ janus_status expert_ffn_vjp_split(const uint16_t* gd16, const float* gd_scale, c
   if (st != JANUS_OK) return st;
   st = act_split_f16<kActDSilu>(dA, act, R, h, second->h16, second->hscale, stream);
   if (st != JANUS_OK) return st;
-  st = split_weights_f16(w1, E, h, d, false, second->w16, second->winv, stream);
+  if (!weights_presplit) st = split_weights_f16(w1, E, h, d, false, second->w16, second->winv, stream);
   if (st != JANUS_OK) return st;
   return launch<kModeNN, kEpiStore, kBF16S>(reinterpret_cast<const float*>(second->h16),
                                             reinterpret_cast<const float*>(second->w16), R, E, h, d, dxd, nullptr,

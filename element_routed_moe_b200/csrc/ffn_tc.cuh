@@ -39,6 +39,11 @@ struct F16Second {
 // One kernel; N % 4 == 0 and Kd % 4 == 0 (JANUS_ERR_MISALIGNED otherwise).
 janus_status split_weights_f16(const float* w, int32_t E, int32_t Kd, int32_t N, bool transposed, uint16_t* w16,
                                float* winv, cudaStream_t stream);
+// Both splits of W [E][A][B] from one read: (w16t, winvt) = the transposed
+// split (Kd = A, N = B) and (w16r, winvr) = the row split (N = A, Kd = B),
+// the same bits as the two split_weights_f16 calls.  A % 4 == 0, B % 4 == 0.
+janus_status split_weights_f16_both(const float* w, int32_t E, int32_t A, int32_t B, uint16_t* w16t, float* winvt,
+                                    uint16_t* w16r, float* winvr, cudaStream_t stream);
 
 // Forward / input VJP on rows given as two FP16 terms (hi plane [R][d] then
 // mid plane [R][d]) with a per-row scale (janus_dispatch_split): the first
@@ -48,27 +53,30 @@ janus_status split_weights_f16(const float* w, int32_t E, int32_t Kd, int32_t N,
 // dA), or, with `second`, on the kind::f16 path after one pass splits the
 // activation (H = silu(a), or dA = dH silu'(a) with dH stored into dA's
 // buffer) into two FP16 terms per row.  d % 8 == 0; h % 8 == 0 with second.
+// weights_presplit: w16 / winv (and second's w16 / winv) already hold the
+// weights' splits, and no split of the weights is launched.
 janus_status expert_ffn_fwd_split(const uint16_t* rows16, const float* row_scale, const int32_t* offsets, int32_t E,
                                   int64_t R, int32_t d, int32_t h, const float* w1, const float* w2, float* yd,
                                   float* act, float* H, uint16_t* w16, float* winv, int32_t* err,
                                   cudaStream_t stream, float* const* yd_rows = nullptr,
-                                  const F16Second* second = nullptr);
+                                  const F16Second* second = nullptr, bool weights_presplit = false);
 janus_status expert_ffn_vjp_split(const uint16_t* gd16, const float* gd_scale, const float* act,
                                   const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
                                   const float* w1, const float* w2, float* dxd, float* dA, uint16_t* w16,
                                   float* winv, int32_t* err, cudaStream_t stream, float* const* dxd_rows = nullptr,
-                                  const F16Second* second = nullptr);
+                                  const F16Second* second = nullptr, bool weights_presplit = false);
 
 // The forward on the FP16 payload itself: row p of xd is f32(payload[p]) *
 // row_scale[p].  The first GEMM runs on the kind::f16 tensor path against the
 // FP16 split of W1 (written into w16 / winv first); d % 8 == 0, payload
 // 16-byte aligned.
 // second (nullable): run the second GEMM (H W2) on the kind::f16 path too.
+// weights_presplit as in expert_ffn_fwd_split.
 janus_status expert_ffn_fwd_packed(const uint16_t* payload, const float* row_scale, const int32_t* offsets,
                                    int32_t E, int64_t R, int32_t d, int32_t h, const float* w1, const float* w2,
                                    float* yd, float* act, float* H, uint16_t* w16, float* winv, int32_t* err,
                                    cudaStream_t stream, float* const* yd_rows = nullptr,
-                                   const F16Second* second = nullptr);
+                                   const F16Second* second = nullptr, bool weights_presplit = false);
 janus_status expert_ffn_vjp(const float* xd, const float* gd, const float* act_in, float* A,
                             const int32_t* offsets, int32_t E, int64_t R, int32_t d, int32_t h,
                             const float* w1, const float* w2, float* dxd, float* dA, int32_t* err,

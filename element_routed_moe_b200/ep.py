@@ -88,6 +88,14 @@ class ExpertParallelLayer:
         self.split_vjp = (mode == J.JANUS_FFN_3XTF32 and d % 8 == 0 and h % 8 == 0
                           and cap >= min_rows * self.El)
         self.launches_per_step += 5 if self.split_vjp else 0
+        # both directions on the FP16 path: the forward writes the weights'
+        # splits for both (janus_expert_weights_f16, 2 launches in place of
+        # the forward's two splits) and the VJP launches none of its own
+        self.w16set = None
+        if self.f16_second and self.split_vjp:
+            self.w16set = torch.empty(J.janus_expert_weights_f16_size(self.El, d, h), dtype=torch.uint8,
+                                      device=self.dev)
+            self.launches_per_step -= 2
         self.payload = torch.empty((cap, d), dtype=torch.float16, device=self.dev)
         self.row_scale = torch.empty((cap,), **f32)
         self.recv_rows = torch.empty((cap, d), **f32)       # gradients in, outputs out
@@ -211,8 +219,10 @@ class ExpertParallelLayer:
             J.janus_ep_return_rows(self.layout, self.rank, self.peer_ret, self.cap, self.d, out=self.ret_rows)
             out = dict(out_rows=self.ret_rows)
         if self.fused_unpack:
+            if self.w16set is not None:
+                J.janus_expert_weights_f16(self.w1, self.w2, J.JANUS_W16_FWD | J.JANUS_W16_VJP, out=self.w16set)
             J.janus_expert_ffn_fwd_packed(self.payload, self.row_scale, recv_off, self.w1, self.w2, act=self.act,
-                                          mode=self.mode, **out)
+                                          mode=self.mode, weights16=self.w16set, **out)
         else:
             # the unpacked FP16 rows are exact in TF32: the first GEMM skips their residual
             J.janus_ep_dequant_rows(self.payload, self.row_scale, self.layout, self.rank, out=self.xd)
@@ -249,7 +259,7 @@ class ExpertParallelLayer:
                                    workspace=self.split_ws)
             out = dict(out_rows=self.ret_rows) if self.fused_return else dict(out=self.yd)
             J.janus_expert_ffn_vjp_split(self.gd16, self.gd_scale, recv_off, self.w1, self.w2, self.act,
-                                         workspace=self.vjp_ws, **out)
+                                         weights16=self.w16set, workspace=self.vjp_ws, **out)
         elif self.fused_return:
             J.janus_expert_ffn_vjp_rows(self.xd, self.recv_rows, recv_off, self.w1, self.w2, self.ret_rows,
                                         act=self.act, mode=self.mode)

@@ -39,6 +39,7 @@ SYMBOLS = (
     "janus_expert_ffn_workspace_size", "janus_expert_ffn_fwd", "janus_expert_ffn_vjp",
     "janus_expert_ffn_fwd_rows", "janus_expert_ffn_vjp_rows", "janus_expert_ffn_fwd_ex",
     "janus_expert_ffn_packed_workspace_size", "janus_expert_ffn_fwd_packed", "janus_expert_ffn_f16_min_rows_per_expert",
+    "janus_expert_weights_f16_size", "janus_expert_weights_f16",
     "janus_expert_ffn_split_workspace_size", "janus_expert_ffn_fwd_split", "janus_expert_ffn_vjp_split",
     "janus_expert_ffn_weight_grad_workspace_size", "janus_expert_ffn_weight_grad",
     "janus_expert_ffn_vjp_vjp_workspace_size", "janus_expert_ffn_vjp_vjp",
@@ -133,11 +134,15 @@ def _declare(L):
                                          ctypes.c_int, vp, sz, vp]),
         "janus_expert_ffn_packed_workspace_size": (st, [i64, i32, i32, i32, ctypes.c_int, psz]),
         "janus_expert_ffn_f16_min_rows_per_expert": (i32, []),
-        "janus_expert_ffn_fwd_packed": (st, [vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, ctypes.c_int,
-                                             vp, sz, vp]),
+        "janus_expert_weights_f16_size": (st, [i32, i32, i32, psz]),
+        "janus_expert_weights_f16": (st, [vp, vp, i32, i32, i32, ctypes.c_uint32, vp, sz, vp]),
+        "janus_expert_ffn_fwd_packed": (st, [vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, vp, sz,
+                                             ctypes.c_int, vp, sz, vp]),
         "janus_expert_ffn_split_workspace_size": (st, [i64, i32, i32, i32, psz]),
-        "janus_expert_ffn_fwd_split": (st, [vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
-        "janus_expert_ffn_vjp_split": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp]),
+        "janus_expert_ffn_fwd_split": (st, [vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp, sz,
+                                            vp]),
+        "janus_expert_ffn_vjp_split": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp, sz,
+                                            vp]),
         "janus_expert_ffn_weight_grad_workspace_size": (st, [i64, i32, i32, psz]),
         "janus_expert_ffn_weight_grad": (st, [vp, vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, vp,
                                               ctypes.c_int, vp, sz, vp]),
@@ -681,11 +686,43 @@ def janus_expert_ffn_f16_min_rows_per_expert() -> int:
     return int(lib().janus_expert_ffn_f16_min_rows_per_expert())
 
 
+JANUS_W16_FWD = 1
+JANUS_W16_VJP = 2
+
+
+def janus_expert_weights_f16_size(n_experts, d, h) -> int:
+    b = ctypes.c_size_t(0)
+    _raise(lib().janus_expert_weights_f16_size(int(n_experts), int(d), int(h), ctypes.byref(b)),
+           "janus_expert_weights_f16_size")
+    return b.value
+
+
+def janus_expert_weights_f16(w1, w2, which=JANUS_W16_FWD | JANUS_W16_VJP, *, out=None, stream=None):
+    """The FP16 splits of w1 [E,d,h] and w2 [E,h,d] for the FP16 MLP calls
+    (their `weights16`): the forward's parts, the input VJP's, or both from
+    one read of each weight tensor.  Returns the set (uint8 device tensor)."""
+    E, d, h = w1.shape
+    nb = janus_expert_weights_f16_size(E, d, h)
+    out = _workspace(nb, w1.device, out)
+    _raise(lib().janus_expert_weights_f16(_p(w1, torch.float32, "w1"), _p(w2, torch.float32, "w2"), E, d, h,
+                                          int(which), _p(out), out.numel() * out.element_size(), _stream(stream)),
+           "janus_expert_weights_f16")
+    return out
+
+
+def _w16(weights16):
+    if weights16 is None:
+        return None, 0
+    return _p(weights16, torch.uint8, "weights16"), weights16.numel()
+
+
 def janus_expert_ffn_fwd_packed(payload, row_scale, offsets, w1, w2, *, out=None, out_rows=None,
-                                mode=JANUS_FFN_FP32_SIMT, want_act=False, act=None, workspace=None, stream=None):
+                                mode=JANUS_FFN_FP32_SIMT, want_act=False, act=None, weights16=None, workspace=None,
+                                stream=None):
     """The forward on the FP16 payload [R,d] with per-row scales [R] (3xTF32
     mode: the first GEMM on the FP16 tensor path against an FP16 split of
-    w1); output as in janus_expert_ffn_fwd_ex.  Returns (out-or-None,
+    w1, the call's own or weights16's, a set from janus_expert_weights_f16);
+    output as in janus_expert_ffn_fwd_ex.  Returns (out-or-None,
     act-or-None)."""
     R, d = payload.shape
     E, _, h = w1.shape
@@ -704,7 +741,8 @@ def janus_expert_ffn_fwd_packed(payload, row_scale, offsets, w1, w2, *, out=None
                                              _p(w1, torch.float32, "w1"), _p(w2, torch.float32, "w2"),
                                              _p(out, torch.float32, "yd"),
                                              None if out_rows is None else _row_table(out_rows, R),
-                                             _p(act, torch.float32, "act"), int(mode), _p(ws), nb, _stream(stream)),
+                                             _p(act, torch.float32, "act"), *_w16(weights16), int(mode), _p(ws), nb,
+                                             _stream(stream)),
            "janus_expert_ffn_fwd_packed")
     return out, act
 
@@ -717,11 +755,12 @@ def janus_expert_ffn_split_workspace_size(n_rows, n_experts, d, h) -> int:
 
 
 def janus_expert_ffn_fwd_split(rows16, row_scale, offsets, w1, w2, *, out=None, out_rows=None, want_act=False,
-                               act=None, workspace=None, stream=None):
+                               act=None, weights16=None, workspace=None, stream=None):
     """The forward on split rows (janus_dispatch_split): the first GEMM on the
     FP16 tensor path, the second on 3xTF32, or on the FP16 path too from
     janus_expert_ffn_f16_min_rows_per_expert() rows per expert with h % 8 == 0.
-    Returns (out-or-None, act-or-None)."""
+    weights16: a set from janus_expert_weights_f16 (forward parts), else the
+    call splits the weights itself.  Returns (out-or-None, act-or-None)."""
     R2, d = rows16.shape
     R = R2 // 2
     E, _, h = w1.shape
@@ -738,18 +777,20 @@ def janus_expert_ffn_fwd_split(rows16, row_scale, offsets, w1, w2, *, out=None, 
                                             _p(w1, torch.float32, "w1"), _p(w2, torch.float32, "w2"),
                                             _p(out, torch.float32, "yd"),
                                             None if out_rows is None else _row_table(out_rows, R),
-                                            _p(act, torch.float32, "act"), _p(ws), nb, _stream(stream)),
+                                            _p(act, torch.float32, "act"), *_w16(weights16), _p(ws), nb,
+                                            _stream(stream)),
            "janus_expert_ffn_fwd_split")
     return out, act
 
 
-def janus_expert_ffn_vjp_split(gd16, gd_scale, offsets, w1, w2, act, *, out=None, out_rows=None, workspace=None,
-                               stream=None):
+def janus_expert_ffn_vjp_split(gd16, gd_scale, offsets, w1, w2, act, *, out=None, out_rows=None, weights16=None,
+                               workspace=None, stream=None):
     """The input VJP on split upstream-gradient rows (janus_dispatch_split,
     weighted) and the forward's pre-activations: dA = (gd W2^T) silu'(a) on
     the FP16 tensor path, dxd = dA W1^T on 3xTF32, or on the FP16 path too at
     janus_expert_ffn_f16_min_rows_per_expert() rows per expert with h % 8 == 0.
-    Returns out-or-None."""
+    weights16: a set from janus_expert_weights_f16 (VJP parts), else the call
+    splits the weights itself.  Returns out-or-None."""
     R2, d = gd16.shape
     R = R2 // 2
     E, _, h = w1.shape
@@ -763,8 +804,9 @@ def janus_expert_ffn_vjp_split(gd16, gd_scale, offsets, w1, w2, act, *, out=None
                                             _p(act, torch.float32, "act"), _p(offsets, torch.int32, "offsets"), E, R,
                                             d, h, _p(w1, torch.float32, "w1"), _p(w2, torch.float32, "w2"),
                                             _p(out, torch.float32, "dxd"),
-                                            None if out_rows is None else _row_table(out_rows, R), _p(ws), nb,
-                                            _stream(stream)), "janus_expert_ffn_vjp_split")
+                                            None if out_rows is None else _row_table(out_rows, R),
+                                            *_w16(weights16), _p(ws), nb, _stream(stream)),
+           "janus_expert_ffn_vjp_split")
     return out
 
 

@@ -24,8 +24,10 @@ per expert (and d, h multiples of 8) unpacked rows are dispatched as two FP16
 terms with a per-row scale (janus_dispatch_split) for
 janus_expert_ffn_fwd_split, the gradient's weighted dispatch is split the same
 way for janus_expert_ffn_vjp_split, and the library runs every GEMM of both
-directions on kind::f16.  Below that size, re-splitting the weights every call
-costs more than the FP16 GEMMs save, and the layer stays on 3xTF32.
+directions on kind::f16; the weights' FP16 splits for both directions are
+written once per pass, in front of the forward (janus_expert_weights_f16, one
+read of each weight tensor).  Below that size, re-splitting the weights every
+call costs more than the FP16 GEMMs save, and the layer stays on 3xTF32.
 
 `run_host` runs the pass from and to pinned host memory with the copies on
 their own streams: the upload of G overlaps the forward, the download of Y
@@ -144,6 +146,14 @@ class MoELayer:
             # gd W2^T, dA's row split, W1 split, dA W1^T
             launches["dispatch_w"] = 2
             launches["ffn_vjp"] = 5
+        # both directions on the FP16 path: the forward writes the splits of
+        # both weight tensors for both directions (janus_expert_weights_f16,
+        # one read of each tensor, 2 launches in place of the forward's two
+        # splits) and the VJP launches none of its own
+        self.w16set = None
+        if self.f16_second and self.split_vjp:
+            self.w16set = torch.empty(J.janus_expert_weights_f16_size(E, d, h), dtype=torch.uint8, device=dev)
+            launches["ffn_vjp"] = 3
         self.launches_per_call = sum(launches[o] for o in self.ops)
         self._host = None
 
@@ -193,13 +203,16 @@ class MoELayer:
             J.janus_dispatch(x, r["slot_of"], K, out=self.xd)
             mark("dispatch", 1)
         mark("ffn_fwd", 0)
+        if self.w16set is not None:
+            J.janus_expert_weights_f16(self.w1, self.w2, J.JANUS_W16_FWD | J.JANUS_W16_VJP, out=self.w16set)
         if self.split:
             J.janus_expert_ffn_fwd_split(self.xd16, self.xd_scale, r["offsets"], self.w1, self.w2, out=self.yd,
-                                         act=self.act, workspace=self.ffn_ws)
+                                         act=self.act, weights16=self.w16set, workspace=self.ffn_ws)
         elif self.fused_unpack:
             # the FP16 rows go straight into the first GEMM (xd is not written)
             J.janus_expert_ffn_fwd_packed(self.payload, self.row_scale, r["offsets"], self.w1, self.w2, out=self.yd,
-                                          act=self.act, mode=self.mode, workspace=self.ffn_ws)
+                                          act=self.act, mode=self.mode, weights16=self.w16set,
+                                          workspace=self.ffn_ws)
         else:
             # unpacked FP16 rows are exact in TF32: the first GEMM skips their residual
             J.janus_expert_ffn_fwd_ex(self.xd, r["offsets"], self.w1, self.w2, out=self.yd, act=self.act,
@@ -221,7 +234,7 @@ class MoELayer:
         mark("ffn_vjp", 0)
         if self.split_vjp:
             J.janus_expert_ffn_vjp_split(self.gd16, self.gd_scale, r["offsets"], self.w1, self.w2, self.act,
-                                         out=self.dxd, workspace=self.ffn_ws)
+                                         out=self.dxd, weights16=self.w16set, workspace=self.ffn_ws)
         else:
             # (xd is read only when the pre-activations are not saved; here they are)
             J.janus_expert_ffn_vjp(self.xd, self.gd, r["offsets"], self.w1, self.w2, act=self.act,

@@ -332,11 +332,36 @@ janus_status janus_expert_ffn_packed_workspace_size(int64_t n_rows, int32_t n_ex
  * FP16 GEMMs save.  Callers choosing between the 3xTF32 and the split entry
  * points can use the same rule. */
 int32_t janus_expert_ffn_f16_min_rows_per_expert(void);
+
+/* The FP16 splits of a layer's expert weights, written once ahead of the MLP
+ * calls that use them (weights16 of janus_expert_ffn_fwd_packed,
+ * janus_expert_ffn_fwd_split and janus_expert_ffn_vjp_split), so that a
+ * forward followed by its input VJP splits each weight tensor in one pass
+ * instead of two.  Each part is what those calls otherwise write into their
+ * workspace for the same GEMM (power-of-two scale per output feature and K
+ * chunk of 256, two binary16 terms; the same bits):
+ *   JANUS_W16_FWD: W1 for x W1 and W2 for H W2 (the forward's GEMMs);
+ *   JANUS_W16_VJP: W2 for gd W2^T and W1 for dA W1^T (the input VJP's).
+ * Both flags: one kernel per weight tensor reads it from DRAM once and writes
+ * both of its splits.  A set stays valid while w1 and w2 are unchanged.
+ * w1 [E,d,h], w2 [E,h,d] float32, 16-byte aligned; d % 8 == 0, h % 4 == 0
+ * (JANUS_ERR_MISALIGNED otherwise).  out: janus_expert_weights_f16_size
+ * bytes, 256-byte aligned, owned by the caller (parts not named in `which`
+ * are left as they were).  Launches 2 kernels. */
+#define JANUS_W16_FWD 1u
+#define JANUS_W16_VJP 2u
+janus_status janus_expert_weights_f16_size(int32_t n_experts, int32_t d, int32_t h, size_t* bytes);
+janus_status janus_expert_weights_f16(const float* w1, const float* w2, int32_t n_experts, int32_t d, int32_t h,
+                                      uint32_t which, void* out, size_t out_bytes, janus_stream_t stream);
+
+/* weights16 (nullable; JANUS_FFN_3XTF32 only), weights16_bytes: a set from
+ * janus_expert_weights_f16 for these w1, w2 holding the JANUS_W16_FWD parts;
+ * the call then launches no split of the weights and reads the set's. */
 janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, const float* row_scale, const int32_t* offsets,
                                          int32_t n_experts, int64_t n_rows, int32_t d, int32_t h, const float* w1,
                                          const float* w2, float* yd, float* const* yd_rows, float* act,
-                                         janus_ffn_mode mode, void* workspace, size_t workspace_bytes,
-                                         janus_stream_t stream);
+                                         const void* weights16, size_t weights16_bytes, janus_ffn_mode mode,
+                                         void* workspace, size_t workspace_bytes, janus_stream_t stream);
 janus_status janus_expert_ffn_vjp_rows(const float* xd, const float* gd, const float* act,
                                        const int32_t* offsets, int32_t n_experts, int64_t n_rows,
                                        int32_t d, int32_t h, const float* w1, const float* w2,
@@ -364,6 +389,9 @@ janus_status janus_expert_ffn_vjp_rows(const float* xd, const float* gd, const f
  * vjp: gd16 = [hi | mid] of the gate-weighted upstream gradient rows, act
  *      = the forward's pre-activations (required), dxd or dxd_rows (one).
  * d % 8 == 0, h % 4 == 0 (JANUS_ERR_MISALIGNED otherwise); N*K < 2^30.
+ * weights16 (nullable), weights16_bytes: a set from janus_expert_weights_f16
+ * for these w1, w2 holding the JANUS_W16_FWD parts (fwd) or the
+ * JANUS_W16_VJP parts (vjp); the call then launches no split of the weights.
  * workspace: janus_expert_ffn_split_workspace_size bytes, 256-byte aligned;
  * its error word reports as in janus_expert_ffn_fwd. */
 janus_status janus_expert_ffn_split_workspace_size(int64_t n_rows, int32_t n_experts, int32_t d, int32_t h,
@@ -371,12 +399,13 @@ janus_status janus_expert_ffn_split_workspace_size(int64_t n_rows, int32_t n_exp
 janus_status janus_expert_ffn_fwd_split(const uint16_t* rows16, const float* row_scale, const int32_t* offsets,
                                         int32_t n_experts, int64_t n_rows, int32_t d, int32_t h, const float* w1,
                                         const float* w2, float* yd, float* const* yd_rows, float* act,
-                                        void* workspace, size_t workspace_bytes, janus_stream_t stream);
+                                        const void* weights16, size_t weights16_bytes, void* workspace,
+                                        size_t workspace_bytes, janus_stream_t stream);
 janus_status janus_expert_ffn_vjp_split(const uint16_t* gd16, const float* gd_scale, const float* act,
                                         const int32_t* offsets, int32_t n_experts, int64_t n_rows, int32_t d,
                                         int32_t h, const float* w1, const float* w2, float* dxd,
-                                        float* const* dxd_rows, void* workspace, size_t workspace_bytes,
-                                        janus_stream_t stream);
+                                        float* const* dxd_rows, const void* weights16, size_t weights16_bytes,
+                                        void* workspace, size_t workspace_bytes, janus_stream_t stream);
 
 /* Expert weight gradients, the parameter side of the same backward pass
  * (force training differentiates the energy w.r.t. inputs and weights,

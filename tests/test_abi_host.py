@@ -123,12 +123,30 @@ def test_argument_validation_before_launch(J):
     assert L.janus_expert_ffn_fwd_ex(FAKE, FAKE, 4, 100, 64, 64, FAKE, FAKE, FAKE, null, null, 6, 1, FAKE,
                                      1 << 30, null) == J.JANUS_ERR_INVALID_ARG
     # packed forward: d % 8 on the tensor cores, workspace too small, no row scales
-    assert L.janus_expert_ffn_fwd_packed(FAKE, FAKE, FAKE, 4, 100, 12, 64, FAKE, FAKE, FAKE, null, null, 1, FAKE,
-                                         1 << 30, null) == J.JANUS_ERR_MISALIGNED
-    assert L.janus_expert_ffn_fwd_packed(FAKE, FAKE, FAKE, 4, 100, 64, 64, FAKE, FAKE, FAKE, null, null, 0, FAKE,
-                                         1024, null) == J.JANUS_ERR_INVALID_ARG
-    assert L.janus_expert_ffn_fwd_packed(FAKE, null, FAKE, 4, 100, 64, 64, FAKE, FAKE, FAKE, null, null, 1, FAKE,
-                                         1 << 30, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_expert_ffn_fwd_packed(FAKE, FAKE, FAKE, 4, 100, 12, 64, FAKE, FAKE, FAKE, null, null, null, 0,
+                                         1, FAKE, 1 << 30, null) == J.JANUS_ERR_MISALIGNED
+    assert L.janus_expert_ffn_fwd_packed(FAKE, FAKE, FAKE, 4, 100, 64, 64, FAKE, FAKE, FAKE, null, null, null, 0,
+                                         0, FAKE, 1024, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_expert_ffn_fwd_packed(FAKE, null, FAKE, 4, 100, 64, 64, FAKE, FAKE, FAKE, null, null, null, 0,
+                                         1, FAKE, 1 << 30, null) == J.JANUS_ERR_INVALID_ARG
+    # a weight-split set: only on the tensor-core path, large enough, 256-byte aligned
+    assert L.janus_expert_ffn_fwd_packed(FAKE, FAKE, FAKE, 4, 100, 64, 64, FAKE, FAKE, FAKE, null, null, FAKE,
+                                         1 << 30, 0, FAKE, 1 << 30, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_expert_ffn_fwd_packed(FAKE, FAKE, FAKE, 4, 100, 64, 64, FAKE, FAKE, FAKE, null, null, FAKE,
+                                         1024, 1, FAKE, 1 << 30, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_expert_ffn_fwd_split(FAKE, FAKE, FAKE, 4, 100, 64, 64, FAKE, FAKE, FAKE, null, null, FAKE + 16,
+                                        1 << 30, FAKE, 1 << 30, null) == J.JANUS_ERR_MISALIGNED
+    assert L.janus_expert_ffn_vjp_split(FAKE, FAKE, FAKE, FAKE, 4, 100, 64, 64, FAKE, FAKE, FAKE, null, FAKE,
+                                        1024, FAKE, 1 << 30, null) == J.JANUS_ERR_INVALID_ARG
+    # the set's own call: flags, d % 8, size, alignment
+    nb = ctypes.c_size_t(0)
+    assert L.janus_expert_weights_f16_size(4, 64, 96, ctypes.byref(nb)) == J.JANUS_OK
+    assert L.janus_expert_weights_f16(FAKE, FAKE, 4, 64, 96, 0, FAKE, nb.value, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_expert_weights_f16(FAKE, FAKE, 4, 64, 96, 4, FAKE, nb.value, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_expert_weights_f16(FAKE, FAKE, 4, 60, 96, 3, FAKE, 1 << 30, null) == J.JANUS_ERR_MISALIGNED
+    assert L.janus_expert_weights_f16(FAKE, FAKE, 4, 64, 96, 3, FAKE, nb.value - 1, null) == J.JANUS_ERR_INVALID_ARG
+    assert L.janus_expert_weights_f16(FAKE, FAKE, 4, 64, 96, 3, FAKE + 64, nb.value, null) == J.JANUS_ERR_MISALIGNED
+    assert L.janus_expert_weights_f16(null, FAKE, 4, 64, 96, 3, FAKE, nb.value, null) == J.JANUS_ERR_INVALID_ARG
     assert L.janus_dispatch_row_scales(10, 2, FAKE, 0, FAKE, FAKE, FAKE, null) == J.JANUS_ERR_INVALID_ARG
     # EP return table: E not a multiple of P, missing peer buffer, d % 4, misaligned table
     two = (ctypes.c_void_p * 2)(FAKE, FAKE)
