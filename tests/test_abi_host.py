@@ -141,6 +141,11 @@ def test_argument_validation_before_launch(J):
     # the set's own call: flags, d % 8, size, alignment
     nb = ctypes.c_size_t(0)
     assert L.janus_expert_weights_f16_size(4, 64, 96, ctypes.byref(nb)) == J.JANUS_OK
+    # four parts as documented: two f16 planes [E][N][K] and 1/S [E][ceil(K/256)][N] each, 256-byte aligned
+    for E, d, h in ((4, 64, 96), (72, 2560, 2560), (3, 264, 776)):
+        up = lambda b: -(-b // 256) * 256
+        want = sum(up(2 * 2 * E * d * h) + up(4 * E * (-(-kd // 256)) * n) for kd, n in ((d, h), (h, d), (d, h), (h, d)))
+        assert J.janus_expert_weights_f16_size(E, d, h) == want
     assert L.janus_expert_weights_f16(FAKE, FAKE, 4, 64, 96, 0, FAKE, nb.value, null) == J.JANUS_ERR_INVALID_ARG
     assert L.janus_expert_weights_f16(FAKE, FAKE, 4, 64, 96, 4, FAKE, nb.value, null) == J.JANUS_ERR_INVALID_ARG
     assert L.janus_expert_weights_f16(FAKE, FAKE, 4, 60, 96, 3, FAKE, 1 << 30, null) == J.JANUS_ERR_MISALIGNED
