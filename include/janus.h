@@ -333,8 +333,10 @@ janus_status janus_expert_ffn_packed_workspace_size(int64_t n_rows, int32_t n_ex
  * points can use the same rule. */
 int32_t janus_expert_ffn_f16_min_rows_per_expert(void);
 
-/* The FP16 splits of a layer's expert weights, written once ahead of the MLP
- * calls that use them (weights16 of janus_expert_ffn_fwd_packed,
+/* The FP16 splits of a layer's expert weights (the expert MLP of [Review]
+ * section 3.1 and its input VJP, section 3.3, kept FP32-accurate on the FP16
+ * tensor cores; the split is this library's arithmetic, the pages have none),
+ * written once ahead of the MLP calls that use them (weights16 of janus_expert_ffn_fwd_packed,
  * janus_expert_ffn_fwd_split and janus_expert_ffn_vjp_split), so that a
  * forward followed by its input VJP splits each weight tensor in one pass
  * instead of two.  Each part is what those calls otherwise write into their
