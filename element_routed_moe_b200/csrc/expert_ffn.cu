@@ -122,7 +122,8 @@ tc::F16Second f16_second_at(char* base, int64_t R, int32_t E, int32_t d, int32_t
 
 // Past the forward's activations: SIMT, the unpacked rows [R,d] FP32;
 // 3xTF32, the FP16 split of W1 (hi and mid, [E][h][d] each), 1 / S [E][ceil(d/256)][h],
-// and the FP16 second GEMM's scratch when it is used.
+// and the FP16 second GEMM's scratch when it is used (the weight splits in
+// it stay unused when the call is given a weight-split set).
 size_t packed_extra(int64_t R, int32_t E, int32_t d, int32_t h, janus_ffn_mode mode) {
   if (mode == JANUS_FFN_FP32_SIMT) return align_up(sizeof(float) * (size_t)R * (size_t)d, 256);
   return align_up(2 * sizeof(uint16_t) * (size_t)E * d * h, 256) + winv_bytes(E, d, h) +
@@ -289,7 +290,8 @@ extern "C" janus_status janus_expert_ffn_fwd_packed(const uint16_t* payload, con
 // kind::f16 path from kF16SecondMinRowsPerExpert rows per expert with h % 8 == 0.  Workspace:
 // header | H, dH or dA [R,h] | the FP16 split of the first GEMM's weights
 // (hi and mid, [E][h][d] each) | 1 / S [E][ceil(d/256)][h] | the FP16 second GEMM's
-// scratch when it is used.
+// scratch when it is used.  With a weight-split set the weight parts of this
+// layout are not written; the GEMMs read the set's.
 // ---------------------------------------------------------------------------
 namespace {
 struct SplitLayout {
