@@ -61,6 +61,8 @@ def test_split_bytes_count_one_read_and_one_write(bench):
     assert b["act_split silu"] == 1000 * 32 * 4 * 2 + 1000 * 4
     assert b["act_split dsilu"] == 1000 * 32 * 4 * 3 + 1000 * 4
     assert b["w16_split rows"] == b["w16_split transposed"] == 3 * 64 * 32 * 4 * 2 + 3 * 64 * 4
+    # both orientations from one read: W once, four FP16 planes, two scale tables
+    assert b["w16_split both"] == 3 * 64 * 32 * 4 + 2 * (3 * 64 * 32 * 4) + 2 * 3 * 64 * 4
 
 
 def test_code_hash_ignores_comments_and_blank_lines(bench):
